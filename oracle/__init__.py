@@ -1,0 +1,251 @@
+"""CPU oracle for the expert-parallel MoE layer hot path (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+and reference legs may import this package.  The product path never does.
+
+The arithmetic lives in ``moe_oracle.c`` (plain single-threaded C, fp64 for the
+FFN and combine, IEEE fp32 with explicit fma for the routing weights).  This
+module only compiles it with gcc and marshals numpy arrays through ctypes.
+bf16 tensors travel as uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liborc.so")
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+ORC_OK, ORC_ERR_ARG, ORC_ERR_NONFINITE = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/liborc.so`` (atomic rename)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    fd, tmp = tempfile.mkstemp(suffix=".so", dir=_BUILD)
+    os.close(fd)
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L.orc_exp_det.argtypes = [ctypes.c_float]
+        L.orc_exp_det.restype = ctypes.c_float
+        L.orc_route_topk.argtypes = [i, i, i, P, P, P, P, P]
+        L.orc_route_topk.restype = i
+        L.orc_capacity_clip.argtypes = [i, i, i, i, P, P, P, P]
+        L.orc_capacity_clip.restype = i
+        L.orc_dispatch_layout.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P]
+        L.orc_dispatch_layout.restype = i
+        L.orc_permute.argtypes = [i, i, i, P, P, P]
+        L.orc_permute.restype = None
+        L.orc_ffn_row.argtypes = [i, i, i, P, P, P, i, P, P, P]
+        L.orc_ffn_row.restype = None
+        L.orc_combine.argtypes = [i, i, i, i, i, P, P, P, P]
+        L.orc_combine.restype = None
+        L.orc_combine_exact.argtypes = [i, i, i, i, i, P, P, P, P]
+        L.orc_combine_exact.restype = None
+        L.orc_bf16_from_double.argtypes = [ctypes.c_double]
+        L.orc_bf16_from_double.restype = ctypes.c_uint16
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return 0
+    if a.dtype == np.uint16:
+        return 1
+    raise TypeError(f"storage arrays are float32 or uint16 (bf16 bits), got {a.dtype}")
+
+
+# --------------------------------------------------------------------------- steps
+
+def exp_det(r: float) -> float:
+    return float(lib().orc_exp_det(ctypes.c_float(float(r))))
+
+
+def route_topk(logits: np.ndarray, bias: np.ndarray | None, k: int):
+    """Returns (topk_idx int32 [T,k], topk_w float32 [T,k], counts int32 [E], status)."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.float32)
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    counts = np.zeros(E, np.int32)
+    st = lib().orc_route_topk(T, E, k, _p(logits), _p(bias), _p(idx), _p(w), _p(counts))
+    return idx, w, counts, st
+
+
+def capacity_clip(topk_idx: np.ndarray, topk_w: np.ndarray, E: int, capacity: int):
+    """Returns (keep uint8 [T,k], kept_counts int32 [E]).  capacity < 0: no cap."""
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    T, k = topk_idx.shape
+    keep = np.zeros((T, k), np.uint8)
+    kept = np.zeros(E, np.int32)
+    st = lib().orc_capacity_clip(T, E, k, int(capacity), _p(topk_idx), _p(topk_w), _p(keep), _p(kept))
+    if st != ORC_OK:
+        raise ValueError(f"orc_capacity_clip status {st}")
+    return keep, kept
+
+
+def dispatch_layout(topk_idx: np.ndarray, keep: np.ndarray, E: int, ep: int,
+                    tok_begin: int = 0, tok_count: int | None = None) -> dict:
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    T, k = topk_idx.shape
+    if tok_count is None:
+        tok_count = T - tok_begin
+    nmax = tok_count * k
+    out = dict(
+        expert_offsets=np.zeros(E + 1, np.int32),
+        rank_offsets=np.zeros(ep + 1, np.int32),
+        recv_token=np.full(max(nmax, 1), -1, np.int32),
+        recv_slot=np.full(max(nmax, 1), -1, np.int32),
+        pos=np.zeros((tok_count, k), np.int32),
+        send_splits=np.zeros((ep, ep), np.int32),
+    )
+    n = lib().orc_dispatch_layout(T, E, k, ep, tok_begin, tok_count, _p(topk_idx), _p(keep),
+                                  _p(out["expert_offsets"]), _p(out["rank_offsets"]),
+                                  _p(out["recv_token"]), _p(out["recv_slot"]), _p(out["pos"]),
+                                  _p(out["send_splits"]))
+    if n < 0:
+        raise ValueError("orc_dispatch_layout rejected its arguments")
+    out["N"] = n
+    out["recv_token"] = out["recv_token"][:n].copy()
+    out["recv_slot"] = out["recv_slot"][:n].copy()
+    return out
+
+
+def permute(x: np.ndarray, recv_token: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    recv_token = np.ascontiguousarray(recv_token, dtype=np.int32)
+    T, H = x.shape
+    N = recv_token.shape[0]
+    xr = np.zeros((N, H), x.dtype)
+    lib().orc_permute(H, x.dtype.itemsize, N, _p(x), _p(recv_token), _p(xr))
+    return xr
+
+
+def ffn_row(x_row: np.ndarray, w13_e: np.ndarray, w2_e: np.ndarray, round_h: bool = True):
+    """One expert's SwiGLU FFN on one row.  Returns (h_store, y_store, y_exact)."""
+    x_row = np.ascontiguousarray(x_row)
+    w13_e = np.ascontiguousarray(w13_e)
+    w2_e = np.ascontiguousarray(w2_e)
+    dt = _dtype_code(x_row)
+    assert _dtype_code(w13_e) == dt and _dtype_code(w2_e) == dt
+    H = x_row.shape[0]
+    I = w13_e.shape[0] // 2
+    assert w13_e.shape == (2 * I, H) and w2_e.shape == (H, I)
+    h = np.zeros(I, x_row.dtype)
+    y = np.zeros(H, x_row.dtype)
+    ye = np.zeros(H, np.float64)
+    lib().orc_ffn_row(H, I, dt, _p(x_row), _p(w13_e), _p(w2_e), int(bool(round_h)), _p(h), _p(y), _p(ye))
+    return h, y, ye
+
+
+def ffn(xr: np.ndarray, expert_offsets: np.ndarray, w13: np.ndarray, w2: np.ndarray,
+        round_h: bool = True):
+    """FFN over a whole expert-contiguous buffer.  Returns (h, y, y_exact)."""
+    N, H = xr.shape
+    E = w13.shape[0]
+    I = w13.shape[1] // 2
+    h = np.zeros((N, I), xr.dtype)
+    y = np.zeros((N, H), xr.dtype)
+    ye = np.zeros((N, H), np.float64)
+    for e in range(E):
+        for p in range(int(expert_offsets[e]), int(expert_offsets[e + 1])):
+            h[p], y[p], ye[p] = ffn_row(xr[p], w13[e], w2[e], round_h)
+    return h, y, ye
+
+
+def combine(y: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: int,
+            tok_begin: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+    y = np.ascontiguousarray(y)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    dt = _dtype_code(y)
+    H = y.shape[1]
+    tok_count, k = pos.shape
+    if out is None:
+        out = np.zeros((T, H), y.dtype)
+    lib().orc_combine(H, k, dt, tok_begin, tok_count, _p(y), _p(pos), _p(topk_w), _p(out))
+    return out
+
+
+def combine_exact(y_exact: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: int,
+                  out_dtype, tok_begin: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+    y_exact = np.ascontiguousarray(y_exact, dtype=np.float64)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    H = y_exact.shape[1]
+    tok_count, k = pos.shape
+    if out is None:
+        out = np.zeros((T, H), out_dtype)
+    dt = _dtype_code(out)
+    lib().orc_combine_exact(H, k, dt, tok_begin, tok_count, _p(y_exact), _p(pos), _p(topk_w), _p(out))
+    return out
+
+
+def bf16_bits_from_double(v: float) -> int:
+    return int(lib().orc_bf16_from_double(float(v)))
+
+
+# --------------------------------------------------------------------------- whole layer
+
+def moe_layer(logits, bias, x, w13, w2, k: int, ep: int, capacity: int = -1,
+              n_chunks: int = 1, reduce_dense: bool = False) -> dict:
+    """All six steps in the order the pages give them, chunk by chunk.
+
+    Route and clip run once over all T tokens (the capacity is per forward);
+    layout, permute, FFN and combine run per contiguous token chunk (axolotl
+    expert_parallel_dispatch_chunks).  Returns every intermediate.
+    """
+    T, E = logits.shape
+    idx, w, counts, st = route_topk(logits, bias, k)
+    if st != ORC_OK:
+        raise ValueError(f"route_topk status {st}")
+    keep, kept = capacity_clip(idx, w, E, capacity)
+    out = np.zeros((T, x.shape[1]), x.dtype)
+    chunks = []
+    tc = T // n_chunks
+    for c in range(n_chunks):
+        tb = c * tc
+        lay = dispatch_layout(idx, keep, E, ep, tb, tc)
+        xr = permute(x, lay["recv_token"])
+        h, y, ye = ffn(xr, lay["expert_offsets"], w13, w2)
+        if reduce_dense:
+            combine_exact(ye, lay["pos"], w, T, x.dtype, tb, out)
+        else:
+            combine(y, lay["pos"], w, T, tb, out)
+        chunks.append(dict(layout=lay, xr=xr, h=h, y=y, y_exact=ye))
+    return dict(topk_idx=idx, topk_w=w, counts=counts, keep=keep, kept_counts=kept,
+                chunks=chunks, out=out)

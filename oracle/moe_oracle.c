@@ -1,0 +1,377 @@
+/*
+ * Plain CPU oracle for the expert-parallel MoE layer hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline / reference arm may load this.  It shares no code,
+ * header, table or constant with the CUDA library: every constant below is
+ * derived here from its mathematical definition.
+ *
+ * Single-threaded, slow, and written to be read against its sources:
+ *
+ *  - axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
+ *      expert_parallel_backend (torch: all_to_all_single over the EP group),
+ *      expert_parallel_dispatch_chunks, expert_parallel_size,
+ *      expert_parallel_token_capacity ("lowest-weight excess (token,expert)
+ *      assignments are dropped").
+ *  - LightLLM PR 1687 review page: _select_experts (top-k over the logical
+ *      experts, norm_topk_prob renormalisation), the expert prefix-sum
+ *      ("psum") contiguous layout for the grouped GEMM, SwiGLU
+ *      (silu_and_mul) between the two grouped GEMMs, decode reducing expert
+ *      outputs straight into a dense output.
+ *
+ * Readings of points the pages leave open are marked "Reading:".
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC -lm.
+ * -ffp-contract=off matters: the routing weights must come out of exactly the
+ * IEEE operations written here, one rounding each.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_NONFINITE 2
+
+/* ------------------------------------------------------------------------- */
+/* Deterministic exponential for r <= 0 (Cody & Waite argument reduction,    */
+/* "Software Manual for the Elementary Functions", 1980, then a Taylor        */
+/* polynomial).  Reading: the pages only say "softmax"; a bit-reproducible    */
+/* exp is needed because the capacity clip compares weights across tokens.    */
+/* ------------------------------------------------------------------------- */
+
+/* 1/ln 2 rounded to fp32. */
+static float orc_log2e(void) { return (float)(1.0 / 0.69314718055994530941723212145818); }
+/* ln 2 truncated to 16 significant bits: 45426 / 2^16.  n * LN2_HI is exact for
+ * |n| <= 127 and r - n*LN2_HI is exact for |r| < 88, so the reduction loses
+ * nothing in its first step. */
+static float orc_ln2_hi(void) { return 45426.0f / 65536.0f; }
+/* the rest of ln 2, rounded to fp32 */
+static float orc_ln2_lo(void) { return (float)(0.69314718055994530941723212145818 - 45426.0 / 65536.0); }
+
+float orc_exp_det(float r)
+{
+    if (r < -87.0f) return 0.0f;
+    float t = r * orc_log2e();              /* one fp32 multiply */
+    float n = rintf(t);                     /* round half to even */
+    float f = fmaf(-n, orc_ln2_hi(), r);    /* exact */
+    f = fmaf(-n, orc_ln2_lo(), f);          /* one rounding */
+    /* Taylor coefficients 1/j!, j = 7..0, each rounded to fp32 once. */
+    double fact = 1.0;
+    float c[8];
+    for (int j = 0; j < 8; ++j) { if (j > 0) fact *= (double)j; c[j] = (float)(1.0 / fact); }
+    float p = c[7];
+    for (int j = 6; j >= 0; --j) p = fmaf(p, f, c[j]);
+    /* 2^n by assembling the exponent field; n is in [-126, 0] here. */
+    int ni = (int)n;
+    uint32_t bits = (uint32_t)(ni + 127) << 23;
+    float two_n;
+    memcpy(&two_n, &bits, sizeof two_n);
+    return p * two_n;                       /* one fp32 multiply (may round to subnormal) */
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 1: router top-k with renormalised softmax weights.                    */
+/* LightLLM PR 1687, "_select_experts" (top-k over logical experts, weights    */
+/* renormalised with norm_topk_prob); axolotl: "routing topk ... always saved".*/
+/* ------------------------------------------------------------------------- */
+
+/* Returns 1 if (va, a) ranks before (vb, b): larger value first, lower expert
+ * index first among equal values (IEEE ==, so -0 == +0). */
+static int orc_before(float va, int a, float vb, int b)
+{
+    if (va > vb) return 1;
+    if (va < vb) return 0;
+    return a < b;
+}
+
+/*
+ * logits fp32 [T, E]; bias fp32 [E] or NULL.
+ * topk_idx int32 [T, k], topk_w fp32 [T, k] in rank order; counts int32 [E]
+ * (assignments per expert before any clip).
+ *
+ * Weights: with l'_j the selected biased logits in slot order and m = l'_0,
+ *   w_j = exp(l'_j - m) / sum_{i<k} exp(l'_i - m),
+ * which equals the full softmax restricted to the top k and renormalised (the
+ * softmax denominator cancels).  Reading: the bias (skewed-router workload)
+ * enters both the selection and the weights; the sum runs in slot order.
+ */
+int orc_route_topk(int T, int E, int k, const float *logits, const float *bias,
+                   int32_t *topk_idx, float *topk_w, int32_t *counts)
+{
+    if (T < 0 || E <= 0 || k <= 0 || k > E) return ORC_ERR_ARG;
+    float *l = (float *)malloc(sizeof(float) * (size_t)E);
+    unsigned char *taken = (unsigned char *)malloc((size_t)E);
+    float *ev = (float *)malloc(sizeof(float) * (size_t)k);
+    int status = ORC_OK;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            float b = bias ? bias[e] : 0.0f;
+            l[e] = logits[(size_t)t * E + e] + b;   /* -0 + +0 = +0: canonicalises -0 */
+            if (!isfinite(l[e])) status = ORC_ERR_NONFINITE;
+            taken[e] = 0;
+        }
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || orc_before(l[e], e, l[best], best)) best = e;
+            }
+            taken[best] = 1;
+            topk_idx[(size_t)t * k + j] = best;
+            counts[best] += 1;
+        }
+        float m = l[topk_idx[(size_t)t * k]];
+        float S = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            ev[j] = orc_exp_det(l[topk_idx[(size_t)t * k + j]] - m);
+            S = S + ev[j];
+        }
+        for (int j = 0; j < k; ++j) topk_w[(size_t)t * k + j] = ev[j] / S;
+    }
+    free(l); free(taken); free(ev);
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 2: per-expert token capacity (axolotl ExpertParallelArgs,              */
+/* expert_parallel_token_capacity): at most C assignments per expert per       */
+/* forward; the lowest-weight excess (token, expert) pairs are dropped.        */
+/* Tie rule: among equal weights the higher token index is dropped first.      */
+/* Reading: the weight compared is the renormalised top-k weight (the combine  */
+/* weight); survivors are not re-renormalised.  C < 0 means no cap; C = 0    */
+/* drops every assignment.                                                     */
+/* ------------------------------------------------------------------------- */
+
+typedef struct { float w; int t; int j; } orc_assign;
+
+static int orc_cmp_keep_first(const void *pa, const void *pb)
+{
+    const orc_assign *a = (const orc_assign *)pa, *b = (const orc_assign *)pb;
+    if (a->w > b->w) return -1;
+    if (a->w < b->w) return 1;
+    return (a->t < b->t) ? -1 : (a->t > b->t);
+}
+
+int orc_capacity_clip(int T, int E, int k, int C, const int32_t *topk_idx,
+                      const float *topk_w, uint8_t *keep, int32_t *kept_counts)
+{
+    if (T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+    for (size_t i = 0; i < (size_t)T * k; ++i) keep[i] = 1;
+    orc_assign *seg = (orc_assign *)malloc(sizeof(orc_assign) * ((size_t)T + 1));
+    for (int e = 0; e < E; ++e) {
+        int n = 0;
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j)
+                if (topk_idx[(size_t)t * k + j] == e) {
+                    seg[n].w = topk_w[(size_t)t * k + j]; seg[n].t = t; seg[n].j = j; ++n;
+                }
+        if (C >= 0 && n > C) {
+            qsort(seg, (size_t)n, sizeof(orc_assign), orc_cmp_keep_first);
+            for (int i = C; i < n; ++i) keep[(size_t)seg[i].t * k + seg[i].j] = 0;
+            kept_counts[e] = C;
+        } else {
+            kept_counts[e] = n;
+        }
+    }
+    free(seg);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 3: dispatch layout.  The torch backend sends rows with                 */
+/* all_to_all_single over the EP group (axolotl, expert_parallel_backend) and  */
+/* the receiver runs its experts on the expert-contiguous prefix-sum layout    */
+/* (LightLLM PR 1687, "use_psum_layout").  Readings:                           */
+/*  - source rank of token t in a chunk [b, b+n): s = (t - b) / (n / EP)       */
+/*    (contiguous equal token blocks, as in a data-parallel split);            */
+/*  - destination rank of expert e: d = e / (E / EP);                          */
+/*  - receive order: by destination rank, then expert, then token; with the    */
+/*    two readings above this is simply the stable order by (e, t).            */
+/* Outputs: expert_offsets [E+1], rank_offsets [EP+1], recv_token [N]          */
+/* (absolute token index), recv_slot [N], pos [n, k] (chunk-relative rows; -1  */
+/* where dropped), send_splits [EP, EP] (row s = source, column d = dest).     */
+/* Returns N (>= 0) or -ORC_ERR_ARG.                                           */
+/* ------------------------------------------------------------------------- */
+
+int orc_dispatch_layout(int T, int E, int k, int EP, int tok_begin, int tok_count,
+                        const int32_t *topk_idx, const uint8_t *keep,
+                        int32_t *expert_offsets, int32_t *rank_offsets,
+                        int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                        int32_t *send_splits)
+{
+    if (EP <= 0 || E % EP != 0 || tok_count < 0 || tok_begin < 0 ||
+        tok_begin + tok_count > T || tok_count % EP != 0)
+        return -ORC_ERR_ARG;
+    int tpr = tok_count / EP;          /* tokens per source rank */
+    int epr = E / EP;                  /* experts per destination rank */
+    for (size_t i = 0; i < (size_t)tok_count * k; ++i) pos[i] = -1;
+    for (int i = 0; i < EP * EP; ++i) send_splits[i] = 0;
+    int n = 0;
+    for (int e = 0; e < E; ++e) {
+        expert_offsets[e] = n;
+        for (int t = tok_begin; t < tok_begin + tok_count; ++t)
+            for (int j = 0; j < k; ++j) {
+                size_t a = (size_t)t * k + j;
+                if (topk_idx[a] == e && keep[a]) {
+                    recv_token[n] = t;
+                    recv_slot[n] = j;
+                    pos[(size_t)(t - tok_begin) * k + j] = n;
+                    int s = (t - tok_begin) / tpr;
+                    int d = e / epr;
+                    send_splits[s * EP + d] += 1;
+                    ++n;
+                }
+            }
+    }
+    expert_offsets[E] = n;
+    for (int d = 0; d <= EP; ++d) rank_offsets[d] = expert_offsets[d * epr];
+    return n;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 4: permute.  xr[p, :] = x[recv_token[p], :] (bytewise copy).            */
+/* ------------------------------------------------------------------------- */
+void orc_permute(int H, int elem_bytes, int N, const void *x, const int32_t *recv_token,
+                 void *xr)
+{
+    size_t row = (size_t)H * elem_bytes;
+    for (int p = 0; p < N; ++p)
+        memcpy((char *)xr + (size_t)p * row, (const char *)x + (size_t)recv_token[p] * row, row);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Storage types.  dtype 0 = fp32, 1 = bf16 (stored as uint16 bit patterns).  */
+/* ------------------------------------------------------------------------- */
+static double orc_load(const void *base, size_t i, int dtype)
+{
+    if (dtype == 0) return (double)((const float *)base)[i];
+    uint32_t u = (uint32_t)((const uint16_t *)base)[i] << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 (ties to even) in one step and return its
+ * bit pattern.  Normal range only matters here; tiny values flush through the
+ * fp32 path, overflow gives +-inf. */
+uint16_t orc_bf16_from_double(double v)
+{
+    if (v != v) return 0x7FC0;
+    if (v == 0.0) return signbit(v) ? 0x8000 : 0x0000;
+    double a = fabs(v);
+    float out;
+    if (a < 1.1754943508222875e-38) {
+        out = (float)v;                                     /* subnormal region */
+        uint32_t u; memcpy(&u, &out, 4);
+        uint32_t r = u + 0x7FFFu + ((u >> 16) & 1u);
+        return (uint16_t)(r >> 16);
+    }
+    int ex;
+    double m = frexp(a, &ex);                 /* a = m * 2^ex, m in [0.5, 1) */
+    double q = nearbyint(ldexp(m, 8));        /* 8 significant bits, ties to even */
+    double r = ldexp(q, ex - 8);
+    if (r > 3.3895313892515355e38) {          /* above the largest finite bf16 */
+        return signbit(v) ? 0xFF80 : 0x7F80;
+    }
+    out = (float)(signbit(v) ? -r : r);       /* exact: r has 8 significant bits */
+    uint32_t u; memcpy(&u, &out, 4);
+    return (uint16_t)(u >> 16);
+}
+
+static void orc_store(void *base, size_t i, int dtype, double v)
+{
+    if (dtype == 0) ((float *)base)[i] = (float)v;
+    else ((uint16_t *)base)[i] = orc_bf16_from_double(v);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 5: one expert's SwiGLU FFN on one row (LightLLM PR 1687: grouped GEMM  */
+/* on the psum layout, then silu_and_mul, then the second grouped GEMM).       */
+/*   g_i = sum_c W13[i, c] x[c],  u_i = sum_c W13[I + i, c] x[c]   (i < I)     */
+/*   h_i = silu(g_i) * u_i,  silu(a) = a / (1 + exp(-a))                       */
+/*   y_o = sum_i W2[o, i] h_i                                                  */
+/* Dot products in double.  h is rounded to the storage type before the        */
+/* second GEMM when round_h (the CUDA path stores h); y_store (optional) gets  */
+/* y rounded to the storage type, y_exact (optional) the unrounded y.          */
+/* w13 is one expert's [2I, H], w2 one expert's [H, I].                        */
+/* ------------------------------------------------------------------------- */
+void orc_ffn_row(int H, int I, int dtype, const void *x_row, const void *w13_e,
+                 const void *w2_e, int round_h, void *h_store, void *y_store,
+                 double *y_exact)
+{
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int c = 0; c < H; ++c) {
+            double xv = orc_load(x_row, (size_t)c, dtype);
+            g += orc_load(w13_e, (size_t)i * H + c, dtype) * xv;
+            u += orc_load(w13_e, (size_t)(I + i) * H + c, dtype) * xv;
+        }
+        double hv = g / (1.0 + exp(-g)) * u;
+        if (h_store) orc_store(h_store, (size_t)i, dtype, hv);
+        if (round_h) {
+            if (dtype == 0) hv = (double)(float)hv;
+            else {
+                uint32_t bits = (uint32_t)orc_bf16_from_double(hv) << 16;
+                float f; memcpy(&f, &bits, 4); hv = (double)f;
+            }
+        }
+        h[i] = hv;
+    }
+    for (int o = 0; o < H; ++o) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i) acc += orc_load(w2_e, (size_t)o * I + i, dtype) * h[i];
+        if (y_exact) y_exact[o] = acc;
+        if (y_store) orc_store(y_store, (size_t)o, dtype, acc);
+    }
+    free(h);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 6: weighted combine back to token order.                               */
+/*   out[t, :] = sum over kept slots j (in slot order) of w[t, j] * y[pos[t,j]] */
+/* accumulated in double, rounded once to the storage type; a token with every */
+/* slot dropped gets zeros.  pos is chunk-relative [n, k], -1 where dropped.   */
+/* ------------------------------------------------------------------------- */
+void orc_combine(int H, int k, int dtype, int tok_begin, int tok_count, const void *y,
+                 const int32_t *pos, const float *topk_w, void *out)
+{
+    double *acc = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int i = 0; i < tok_count; ++i) {
+        int t = tok_begin + i;
+        for (int c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int p = pos[(size_t)i * k + j];
+            if (p < 0) continue;
+            double w = (double)topk_w[(size_t)t * k + j];
+            for (int c = 0; c < H; ++c) acc[c] += w * orc_load(y, (size_t)p * H + c, dtype);
+        }
+        for (int c = 0; c < H; ++c) orc_store(out, (size_t)t * H + c, dtype, acc[c]);
+    }
+    free(acc);
+}
+
+/* Decode form of step 6 (LightLLM PR 1687: decode reduces expert outputs into
+ * a dense output): the same sum, but over unrounded expert outputs, because
+ * the reduce consumes y before it is ever stored.  y_exact is [N, H] double. */
+void orc_combine_exact(int H, int k, int dtype, int tok_begin, int tok_count,
+                       const double *y_exact, const int32_t *pos, const float *topk_w,
+                       void *out)
+{
+    double *acc = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int i = 0; i < tok_count; ++i) {
+        int t = tok_begin + i;
+        for (int c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int p = pos[(size_t)i * k + j];
+            if (p < 0) continue;
+            double w = (double)topk_w[(size_t)t * k + j];
+            for (int c = 0; c < H; ++c) acc[c] += w * y_exact[(size_t)p * H + c];
+        }
+        for (int c = 0; c < H; ++c) orc_store(out, (size_t)t * H + c, dtype, acc[c]);
+    }
+    free(acc);
+}
