@@ -1,0 +1,454 @@
+// C ABI of the MoE hot path: argument and topology checks, workspace carving,
+// launches, and the two-stream chunked forward.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "moe_common.cuh"
+
+namespace moe {
+cudaError_t launch_route_topk(const moe_config &c, const float *logits, const float *bias,
+                              int32_t *topk_idx, float *topk_w, int32_t *counts,
+                              uint32_t *status, cudaStream_t s, int num_sms);
+cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
+                                 const float *topk_w, const int32_t *counts, uint8_t *keep,
+                                 int32_t *kept_counts, uint64_t *thr, uint32_t *status,
+                                 cudaStream_t s, int num_sms);
+cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
+                                   const int32_t *topk_idx, const uint8_t *keep,
+                                   int32_t *expert_offsets, int32_t *rank_offsets,
+                                   int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                                   int32_t *send_splits, int32_t *splits_host, void *ws,
+                                   int64_t n_rows_max, cudaStream_t s, int num_sms);
+size_t layout_scatter_smem(const moe_config &c);
+cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                           int tc, void *xr, cudaStream_t s);
+cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,
+                           const float *topk_w, int tb, int tc, void *out, cudaStream_t s);
+cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb, int tc,
+                                   void *out, cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *xr,
+                               const int32_t *expert_offsets, const void *w13, const void *w2,
+                               void *h, void *y, const int32_t *recv_token,
+                               const int32_t *recv_slot, const float *topk_w, float *out_reduce,
+                               uint32_t *status, cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
+                            const int32_t *expert_offsets, const void *w13, const void *w2,
+                            void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
+                            const float *topk_w, float *out_reduce, cudaStream_t s);
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+moe_status fail(moe_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+moe_status cuda_fail(cudaError_t err, const char *where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(err));
+}
+
+int current_num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t max_rows(const moe_config &c, int32_t tc) {
+    int64_t n = (int64_t)tc * c.k;
+    if (c.capacity >= 0) {
+        const int64_t cap = (int64_t)c.E * c.capacity;
+        if (cap < n) n = cap;
+    }
+    return n;
+}
+
+moe_status check_ws(void *ws) {
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if (!aligned(ws, 256)) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    return MOE_OK;
+}
+
+moe_status check_range(const moe_config &c, int32_t tb, int32_t tc, bool need_ep) {
+    if (tb < 0 || tc < 0 || (int64_t)tb + tc > c.T)
+        return fail(MOE_ERR_INVALID_ARG, "token range [%d, %d+%d) outside [0, %d)", tb, tb, tc, c.T);
+    if (need_ep && tc % c.ep != 0)
+        return fail(MOE_ERR_INVALID_ARG, "tok_count %d not divisible by ep %d", tc, c.ep);
+    return MOE_OK;
+}
+
+// Forward workspace: scratch first, then saved counts, two chunk slots, and
+// the dense fp32 reduce buffer (decode form).
+struct Slot {
+    size_t eoff, roff, recv_token, recv_slot, pos, splits, xr, h, y;
+};
+struct ForwardLayout {
+    size_t counts, kept_counts;
+    Slot slot[2];
+    size_t out_reduce, total;
+    int64_t nmax;
+    int tc;
+};
+
+ForwardLayout forward_layout(const moe_config &c) {
+    ForwardLayout F{};
+    const ScratchLayout L = scratch_layout(c);
+    size_t off = L.total;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+    F.tc = c.T / c.n_chunks;
+    F.nmax = max_rows(c, F.tc);
+    const size_t eb = c.dtype == MOE_F32 ? 4 : 2;
+    F.counts = take(sizeof(int32_t) * c.E);
+    F.kept_counts = take(sizeof(int32_t) * c.E);
+    const int nslots = c.n_chunks > 1 ? 2 : 1;
+    for (int s = 0; s < 2; ++s) {
+        if (s >= nslots) { F.slot[s] = F.slot[0]; continue; }
+        Slot &S = F.slot[s];
+        S.eoff = take(sizeof(int32_t) * (c.E + 1));
+        S.roff = take(sizeof(int32_t) * (c.ep + 1));
+        S.recv_token = take(sizeof(int32_t) * (size_t)(F.nmax > 0 ? F.nmax : 1));
+        S.recv_slot = take(sizeof(int32_t) * (size_t)(F.nmax > 0 ? F.nmax : 1));
+        S.pos = take(sizeof(int32_t) * (size_t)F.tc * c.k);
+        S.splits = take(sizeof(int32_t) * (size_t)c.ep * c.ep);
+        S.xr = take(eb * (size_t)F.nmax * c.H);
+        S.h = take(eb * (size_t)F.nmax * c.I);
+        S.y = c.reduce_dense ? 0 : take(eb * (size_t)F.nmax * c.H);
+    }
+    F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
+    F.total = off;
+    return F;
+}
+
+// Per-thread, per-device pool of timing-free events for the chunked forward.
+struct EventPool {
+    int device = -1;
+    std::vector<cudaEvent_t> ev;
+};
+thread_local EventPool g_events[16];
+
+cudaError_t get_events(int n, cudaEvent_t **out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    EventPool &P = g_events[dev & 15];
+    if (P.device != dev) { P.ev.clear(); P.device = dev; }
+    while ((int)P.ev.size() < n) {
+        cudaEvent_t e;
+        if ((err = cudaEventCreateWithFlags(&e, cudaEventDisableTiming)) != cudaSuccess) return err;
+        P.ev.push_back(e);
+    }
+    *out = P.ev.data();
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_config_check(const moe_config *cfg) {
+    if (!cfg) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+    const moe_config &c = *cfg;
+    if (c.T < 0 || c.H < 1 || c.E < 1 || c.k < 1 || c.I < 1 || c.ep < 1 || c.n_chunks < 1)
+        return fail(MOE_ERR_INVALID_ARG, "sizes must be positive (T >= 0)");
+    if (c.dtype != MOE_F32 && c.dtype != MOE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "unknown dtype %d", c.dtype);
+    if (c.reduce_dense != 0 && c.reduce_dense != 1)
+        return fail(MOE_ERR_INVALID_ARG, "reduce_dense must be 0 or 1");
+    if (c.k > c.E) return fail(MOE_ERR_INVALID_ARG, "k=%d > E=%d", c.k, c.E);
+    if (c.E % c.ep != 0) return fail(MOE_ERR_INVALID_ARG, "E=%d not divisible by ep=%d", c.E, c.ep);
+    if (c.T % c.n_chunks != 0)
+        return fail(MOE_ERR_INVALID_ARG, "T=%d not divisible by n_chunks=%d", c.T, c.n_chunks);
+    if ((c.T / c.n_chunks) % c.ep != 0)
+        return fail(MOE_ERR_INVALID_ARG, "chunk of %d tokens not divisible by ep=%d",
+                    c.T / c.n_chunks, c.ep);
+    if (c.k > kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k=%d > %d", c.k, kMaxTopK);
+    if (c.E > kMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "E=%d > %d", c.E, kMaxExperts);
+    if ((int64_t)c.T * c.k >= (int64_t)1 << 30) return fail(MOE_ERR_UNSUPPORTED, "T*k >= 2^30");
+    if (c.dtype == MOE_BF16 && (c.H % 64 != 0 || c.I % 64 != 0))
+        return fail(MOE_ERR_UNSUPPORTED, "bf16 needs H and I multiples of 64 (H=%d, I=%d)", c.H, c.I);
+    if (c.dtype == MOE_F32 && (c.H % 4 != 0 || c.I % 4 != 0))
+        return fail(MOE_ERR_UNSUPPORTED, "fp32 needs H and I multiples of 4 (H=%d, I=%d)", c.H, c.I);
+    return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_config *cfg) {
+    if (moe_config_check(cfg) != MOE_OK) return 0;
+    return scratch_layout(*cfg).total;
+}
+
+size_t moe_forward_workspace_bytes(const moe_config *cfg) {
+    if (moe_config_check(cfg) != MOE_OK) return 0;
+    return forward_layout(*cfg).total;
+}
+
+int64_t moe_max_recv_rows(const moe_config *cfg, int32_t tok_count) {
+    if (moe_config_check(cfg) != MOE_OK || tok_count < 0) return -1;
+    return max_rows(*cfg, tok_count);
+}
+
+moe_status moe_route_topk(const moe_config *cfg, const float *logits, const float *bias,
+                          int32_t *topk_idx, float *topk_w, int32_t *counts, void *ws,
+                          cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((c.T > 0 && (!logits || !topk_idx || !topk_w)) || !counts)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_route_topk(c, logits, bias, topk_idx, topk_w, counts,
+                                        ws_at<uint32_t>(ws, L.status), stream, current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route_topk");
+}
+
+moe_status moe_capacity_clip(const moe_config *cfg, const int32_t *topk_idx,
+                             const float *topk_w, const int32_t *counts, uint8_t *keep,
+                             int32_t *kept_counts, void *ws, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((c.T > 0 && (!topk_idx || !topk_w || !keep)) || !counts || !kept_counts)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_capacity_clip(c, topk_idx, topk_w, counts, keep, kept_counts,
+                                           ws_at<uint64_t>(ws, L.clip_thr),
+                                           ws_at<uint32_t>(ws, L.status), stream,
+                                           current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_capacity_clip");
+}
+
+moe_status moe_dispatch_layout(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
+                               const int32_t *topk_idx, const uint8_t *keep,
+                               int32_t *expert_offsets, int32_t *rank_offsets,
+                               int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                               int32_t *send_splits, int32_t *splits_host, void *ws,
+                               cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((st = check_range(c, tok_begin, tok_count, true)) != MOE_OK) return st;
+    if (!expert_offsets || !rank_offsets || !send_splits ||
+        (tok_count > 0 && (!topk_idx || !keep || !recv_token || !recv_slot || !pos)))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    cudaError_t err = launch_dispatch_layout(c, tok_begin, tok_count, topk_idx, keep,
+                                             expert_offsets, rank_offsets, recv_token, recv_slot,
+                                             pos, send_splits, splits_host, ws,
+                                             max_rows(c, tok_count), stream, current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_dispatch_layout");
+}
+
+moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *pos,
+                       int32_t tok_begin, int32_t tok_count, void *xr, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!x || !pos || !xr)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(xr, 16)) return fail(MOE_ERR_INVALID_ARG, "x / xr not 16-byte aligned");
+    cudaError_t err = launch_permute(c, x, pos, tok_begin, tok_count, xr, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute");
+}
+
+moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const void *xr,
+                                  const int32_t *expert_offsets, const void *w13,
+                                  const void *w2, void *h, void *y, const int32_t *recv_token,
+                                  const int32_t *recv_slot, const float *topk_w,
+                                  float *out_reduce, void *ws, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (n_rows == 0) return MOE_OK;
+    if (!xr || !expert_offsets || !w13 || !w2 || !h)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.reduce_dense) {
+        if (!recv_token || !recv_slot || !topk_w || !out_reduce)
+            return fail(MOE_ERR_INVALID_ARG, "decode form needs recv_token, recv_slot, topk_w, out_reduce");
+    } else if (!y) {
+        return fail(MOE_ERR_INVALID_ARG, "y is NULL");
+    }
+    const void *ptrs[5] = {xr, w13, w2, h, y};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    const ScratchLayout L = scratch_layout(c);
+    uint32_t *status = ws_at<uint32_t>(ws, L.status);
+    cudaError_t err;
+    if (c.dtype == MOE_BF16) {
+        int dev = 0, major = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (major != 10)
+            return fail(MOE_ERR_UNSUPPORTED, "the bf16 FFN uses tcgen05 and needs sm_100 (got major %d)", major);
+        err = launch_ffn_tcgen05(c, n_rows, xr, expert_offsets, w13, w2, h, y, recv_token,
+                                 recv_slot, topk_w, out_reduce, status, stream, current_num_sms());
+        if (err == cudaErrorNotSupported)
+            return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+    } else {
+        err = launch_ffn_simt(c, n_rows, xr, expert_offsets, w13, w2, h, y, recv_token,
+                              recv_slot, topk_w, out_reduce, stream);
+    }
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn");
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y, const int32_t *pos,
+                       const float *topk_w, int32_t tok_begin, int32_t tok_count, void *out,
+                       cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!y || !pos || !topk_w || !out))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(y, 16) || !aligned(out, 16)) return fail(MOE_ERR_INVALID_ARG, "y / out not 16-byte aligned");
+    cudaError_t err = launch_combine(c, y, pos, topk_w, tok_begin, tok_count, out, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
+}
+
+moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
+                               int32_t tok_begin, int32_t tok_count, void *out,
+                               cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!out_reduce || !out)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(out_reduce, 16) || !aligned(out, 16))
+        return fail(MOE_ERR_INVALID_ARG, "out_reduce / out not 16-byte aligned");
+    cudaError_t err = launch_reduce_finalize(c, out_reduce, tok_begin, tok_count, out, stream,
+                                             current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_reduce_finalize");
+}
+
+moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
+                               const void *x, const void *w13, const void *w2, void *out,
+                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                               int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
+                               cudaStream_t s_compute) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.T > 0 && (!logits || !x || !w13 || !w2 || !out || !topk_idx || !topk_w || !keep))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.T == 0) return MOE_OK;
+    const ForwardLayout F = forward_layout(c);
+    const ScratchLayout L = scratch_layout(c);
+    uint32_t *status = ws_at<uint32_t>(ws, L.status);
+    int32_t *counts = ws_at<int32_t>(ws, F.counts);
+    int32_t *kept_counts = ws_at<int32_t>(ws, F.kept_counts);
+    float *out_reduce = c.reduce_dense ? ws_at<float>(ws, F.out_reduce) : nullptr;
+    const int nsm = current_num_sms();
+    const int nch = c.n_chunks;
+
+    cudaEvent_t *ev = nullptr;
+    cudaError_t err = get_events(2 * nch + 2, &ev);
+    if (err != cudaSuccess) return cuda_fail(err, "event pool");
+    cudaEvent_t ev_start = ev[0], ev_end = ev[1];
+    cudaEvent_t *ev_disp = ev + 2, *ev_done = ev + 2 + nch;
+
+#define MOE_TRY(expr, where)                                   \
+    do {                                                       \
+        cudaError_t e_ = (expr);                               \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where);    \
+    } while (0)
+
+    // the compute stream's earlier work on this workspace precedes the new dispatch
+    MOE_TRY(cudaEventRecord(ev_start, s_compute), "record start");
+    MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_start, 0), "wait start");
+    MOE_TRY(launch_route_topk(c, logits, bias, topk_idx, topk_w, counts, status, s_dispatch, nsm),
+            "route_topk");
+    MOE_TRY(launch_capacity_clip(c, topk_idx, topk_w, counts, keep, kept_counts,
+                                 ws_at<uint64_t>(ws, L.clip_thr), status, s_dispatch, nsm),
+            "capacity_clip");
+    if (c.reduce_dense)
+        MOE_TRY(cudaMemsetAsync(out_reduce, 0, sizeof(float) * (size_t)c.T * c.H, s_dispatch),
+                "clear reduce buffer");
+
+    const int tc = F.tc;
+    const int split_stride = c.E + 1 + c.ep * c.ep;
+    for (int ch = 0; ch < nch; ++ch) {
+        const Slot &S = F.slot[ch & 1];
+        const int tb = ch * tc;
+        if (ch >= 2) MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_done[ch - 2], 0), "wait slot");
+        int32_t *eoff = ws_at<int32_t>(ws, S.eoff);
+        int32_t *recv_token = ws_at<int32_t>(ws, S.recv_token);
+        int32_t *recv_slot = ws_at<int32_t>(ws, S.recv_slot);
+        int32_t *pos = ws_at<int32_t>(ws, S.pos);
+        void *xr = ws_at<void>(ws, S.xr);
+        void *h = ws_at<void>(ws, S.h);
+        void *y = c.reduce_dense ? nullptr : ws_at<void>(ws, S.y);
+        MOE_TRY(launch_dispatch_layout(c, tb, tc, topk_idx, keep, eoff, ws_at<int32_t>(ws, S.roff),
+                                       recv_token, recv_slot, pos, ws_at<int32_t>(ws, S.splits),
+                                       splits_host ? splits_host + (size_t)ch * split_stride : nullptr,
+                                       ws, F.nmax, s_dispatch, nsm),
+                "dispatch_layout");
+        MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, s_dispatch), "permute");
+        MOE_TRY(cudaEventRecord(ev_disp[ch], s_dispatch), "record dispatch");
+        MOE_TRY(cudaStreamWaitEvent(s_compute, ev_disp[ch], 0), "wait dispatch");
+        if (F.nmax > 0) {
+            if (c.dtype == MOE_BF16) {
+                err = launch_ffn_tcgen05(c, F.nmax, xr, eoff, w13, w2, h, y, recv_token, recv_slot,
+                                         topk_w, out_reduce, status, s_compute, nsm);
+                if (err == cudaErrorNotSupported)
+                    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+            } else {
+                err = launch_ffn_simt(c, F.nmax, xr, eoff, w13, w2, h, y, recv_token, recv_slot,
+                                      topk_w, out_reduce, s_compute);
+            }
+            MOE_TRY(err, "grouped_swiglu_ffn");
+        }
+        if (c.reduce_dense)
+            MOE_TRY(launch_reduce_finalize(c, out_reduce, tb, tc, out, s_compute, nsm), "reduce_finalize");
+        else
+            MOE_TRY(launch_combine(c, y, pos, topk_w, tb, tc, out, s_compute), "combine");
+        MOE_TRY(cudaEventRecord(ev_done[ch], s_compute), "record done");
+    }
+    MOE_TRY(cudaEventRecord(ev_end, s_compute), "record end");
+    MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_end, 0), "wait end");
+#undef MOE_TRY
+    return MOE_OK;
+}
+
+moe_status moe_device_status(void *ws, uint32_t *flags, cudaStream_t stream) {
+    if (!ws || !flags) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    uint32_t v = 0;
+    cudaError_t err = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, stream);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(stream);
+    if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, sizeof v, stream);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(stream);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_device_status");
+    *flags = v;
+    if (v) return fail(MOE_ERR_DEVICE, "device status bits 0x%x", v);
+    return MOE_OK;
+}
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_WORKSPACE: return "bad workspace";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE: return "device-detected error";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_error_detail(void) { return g_detail; }
+
+}  // extern "C"

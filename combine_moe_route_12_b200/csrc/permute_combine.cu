@@ -1,0 +1,166 @@
+// Steps 4 and 6: the row permutation into the receive layout and the weighted
+// combine back to token order (axolotl ExpertParallelArgs: dispatch / combine
+// all_to_all_single outputs; LightLLM PR 1687: decode reduce into a dense
+// output).  Both are HBM-bound row copies: one CTA per token, 16-byte vector
+// loads and stores, each source row read once.
+//
+//   permute:  x[t] is read once and written to each of its kept receive rows.
+//   combine:  out[t] = sum_j w[t, j] * y[pos[t, j]] in fp32, slot order,
+//             rounded once to the storage type.
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kRowThreads = 128;
+
+__global__ void __launch_bounds__(kRowThreads) permute_rows_kernel(
+    int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
+    uint4 *__restrict__ xr) {
+    __shared__ int32_t s_pos[kMaxTopK];
+    const int i = blockIdx.x;
+    if (threadIdx.x < k) s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
+    __syncthreads();
+    const uint4 *src = x + (size_t)(tb + i) * row_vecs;
+    for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
+        const uint4 d = __ldg(src + v);
+        for (int j = 0; j < k; ++j) {
+            const int p = s_pos[j];
+            if (p >= 0) xr[(size_t)p * row_vecs + v] = d;
+        }
+    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        f[2 * q] = __uint_as_float(w[q] << 16);
+        f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat16 l = __float2bfloat16_rn(lo), h = __float2bfloat16_rn(hi);
+    return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
+}
+
+// bf16 storage: one uint4 = 8 elements.
+__global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
+    int tb, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
+    const float *__restrict__ topk_w, uint4 *__restrict__ out) {
+    __shared__ int32_t s_pos[kMaxTopK];
+    __shared__ float s_w[kMaxTopK];
+    const int i = blockIdx.x;
+    const int t = tb + i;
+    if (threadIdx.x < k) {
+        s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
+        s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j) {
+            const int p = s_pos[j];
+            if (p < 0) continue;
+            float f[8];
+            unpack8(__ldg(y + (size_t)p * row_vecs + v), f);
+            const float w = s_w[j];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(w, f[q], acc[q]);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        out[(size_t)t * row_vecs + v] = o;
+    }
+}
+
+// fp32 storage: one float4 = 4 elements.
+__global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
+    int tb, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
+    const float *__restrict__ topk_w, float4 *__restrict__ out) {
+    __shared__ int32_t s_pos[kMaxTopK];
+    __shared__ float s_w[kMaxTopK];
+    const int i = blockIdx.x;
+    const int t = tb + i;
+    if (threadIdx.x < k) {
+        s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
+        s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const int p = s_pos[j];
+            if (p < 0) continue;
+            const float4 f = __ldg(y + (size_t)p * row_vecs + v);
+            const float w = s_w[j];
+            acc.x = __fmaf_rn(w, f.x, acc.x);
+            acc.y = __fmaf_rn(w, f.y, acc.y);
+            acc.z = __fmaf_rn(w, f.z, acc.z);
+            acc.w = __fmaf_rn(w, f.w, acc.w);
+        }
+        out[(size_t)t * row_vecs + v] = acc;
+    }
+}
+
+// Decode form: out[t] = round(out_reduce[t]) for the chunk's tokens.
+__global__ void reduce_finalize_kernel(int tb, int tc, int H, int dtype,
+                                       const float4 *__restrict__ red, void *__restrict__ out) {
+    const size_t n4 = (size_t)tc * H / 4;
+    const size_t base4 = (size_t)tb * H / 4;
+    for (size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
+         q += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = red[base4 + q];
+        if (dtype == MOE_F32) {
+            reinterpret_cast<float4 *>(out)[base4 + q] = v;
+        } else {
+            uint2 o;
+            o.x = pack_bf16x2(v.x, v.y);
+            o.y = pack_bf16x2(v.z, v.w);
+            reinterpret_cast<uint2 *>(out)[base4 + q] = o;
+        }
+    }
+}
+
+cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                           int tc, void *xr, cudaStream_t s) {
+    if (tc == 0) return cudaSuccess;
+    const int row_vecs = (int)((size_t)c.H * (c.dtype == MOE_F32 ? 4 : 2) / 16);
+    permute_rows_kernel<<<tc, kRowThreads, 0, s>>>(tb, c.k, row_vecs,
+                                                   static_cast<const uint4 *>(x), pos,
+                                                   static_cast<uint4 *>(xr));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,
+                           const float *topk_w, int tb, int tc, void *out, cudaStream_t s) {
+    if (tc == 0) return cudaSuccess;
+    if (c.dtype == MOE_F32) {
+        const int row_vecs = c.H / 4;
+        combine_rows_f32_kernel<<<tc, kRowThreads, 0, s>>>(
+            tb, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
+            static_cast<float4 *>(out));
+    } else {
+        const int row_vecs = c.H / 8;
+        combine_rows_bf16_kernel<<<tc, kRowThreads, 0, s>>>(
+            tb, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
+            static_cast<uint4 *>(out));
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb, int tc,
+                                   void *out, cudaStream_t s, int num_sms) {
+    if (tc == 0) return cudaSuccess;
+    const size_t n4 = (size_t)tc * c.H / 4;
+    int blocks = (int)((n4 + 255) / 256);
+    if (blocks > num_sms * 8) blocks = num_sms * 8;
+    reduce_finalize_kernel<<<blocks, 256, 0, s>>>(tb, tc, c.H, c.dtype,
+                                                  reinterpret_cast<const float4 *>(red), out);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

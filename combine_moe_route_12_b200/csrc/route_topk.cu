@@ -1,0 +1,145 @@
+// Step 1: router top-k with renormalised softmax weights (LightLLM PR 1687,
+// _select_experts with norm_topk_prob; axolotl ExpertParallelArgs: the routing
+// top-k is saved state).
+//
+// One warp per token.  Lane l holds the biased logits of experts l, l+32, ...
+// k rounds of a butterfly arg-max (value descending, lower expert index first
+// among equal values) pick the experts in rank order; lane j keeps slot j.
+// The weights w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) use a fixed fp32
+// exponential (Cody & Waite reduction, degree-7 Taylor polynomial, every step
+// one IEEE-rounded operation) and a slot-ordered sum, so they are bit-exact
+// against any implementation that performs the same operations.
+#include "moe_common.cuh"
+
+namespace moe {
+
+// e^r for r <= 0 in fp32.  Derivation:
+//   n = rint(r * log2(e)),  f = r - n ln2 (ln2 = hi + lo, hi = 45426 / 2^16 has
+//   16 significant bits so n*hi and r - n*hi are exact for |n| <= 127),
+//   e^f by Horner on the Taylor series to degree 7 (|f| <= ln2/2 leaves a
+//   truncation error near 5e-9), then scaled by 2^n through the exponent field.
+__device__ __forceinline__ float det_exp_nonpos(float r) {
+    constexpr double kLn2 = 0.69314718055994530941723212145818;
+    constexpr float kLog2e = (float)(1.0 / kLn2);
+    constexpr float kLn2Hi = 45426.0f / 65536.0f;
+    constexpr float kLn2Lo = (float)(kLn2 - 45426.0 / 65536.0);
+    constexpr float kC7 = (float)(1.0 / 5040.0), kC6 = (float)(1.0 / 720.0),
+                    kC5 = (float)(1.0 / 120.0), kC4 = (float)(1.0 / 24.0),
+                    kC3 = (float)(1.0 / 6.0), kC2 = 0.5f, kC1 = 1.0f, kC0 = 1.0f;
+    if (r < -87.0f) return 0.0f;
+    const float n = rintf(__fmul_rn(r, kLog2e));
+    float f = __fmaf_rn(-n, kLn2Hi, r);
+    f = __fmaf_rn(-n, kLn2Lo, f);
+    float p = kC7;
+    p = __fmaf_rn(p, f, kC6);
+    p = __fmaf_rn(p, f, kC5);
+    p = __fmaf_rn(p, f, kC4);
+    p = __fmaf_rn(p, f, kC3);
+    p = __fmaf_rn(p, f, kC2);
+    p = __fmaf_rn(p, f, kC1);
+    p = __fmaf_rn(p, f, kC0);
+    const float two_n = __int_as_float(((int)n + 127) << 23);
+    return __fmul_rn(p, two_n);
+}
+
+// (va, a) ranks before (vb, b)?  Larger value first, lower index among equals.
+__device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b) {
+    return (va > vb) || (va == vb && a < b);
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_topk_kernel(
+    int T, int E, int k, const float *__restrict__ logits, const float *__restrict__ bias,
+    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int32_t *__restrict__ counts,
+    uint32_t *__restrict__ status) {
+    extern __shared__ int32_t s_hist[];  // [E]
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    bool nonfinite = false;
+
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+        const float *row = logits + (size_t)t * E;
+        float v[VPL];
+        uint32_t taken = 0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) {
+                float l = __fadd_rn(__ldg(row + e), bias ? __ldg(bias + e) : 0.0f);
+                if (!isfinite(l)) {
+                    nonfinite = true;
+                    if (isnan(l)) l = -INFINITY;  // keep the ranking a total order
+                }
+                v[i] = l;
+            } else {
+                v[i] = -INFINITY;
+                taken |= 1u << i;  // padding never wins
+            }
+        }
+        float my_v = 0.0f;  // slot `lane`'s biased logit
+        int my_e = 0;
+        for (int j = 0; j < k; ++j) {
+            bool has = false;
+            float bv = 0.0f;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int e = lane + 32 * i;
+                if (!((taken >> i) & 1u) && (!has || ranks_before(v[i], e, bv, be))) {
+                    has = true; bv = v[i]; be = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                const bool oh = __shfl_xor_sync(0xffffffffu, (int)has, off) != 0;
+                if (oh && (!has || ranks_before(ov, oe, bv, be))) { has = true; bv = ov; be = oe; }
+            }
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            if (lane == j) { my_v = bv; my_e = be; }
+        }
+        const float m = __shfl_sync(0xffffffffu, my_v, 0);
+        const float ex = (lane < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
+        float S = 0.0f;
+        for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ex, j));
+        if (lane < k) {
+            topk_idx[(size_t)t * k + lane] = my_e;
+            topk_w[(size_t)t * k + lane] = __fdiv_rn(ex, S);
+            atomicAdd(&s_hist[my_e], 1);
+        }
+    }
+    if (nonfinite) raise_status(status, MOE_DEV_NONFINITE_LOGIT);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        if (s_hist[e]) atomicAdd(&counts[e], s_hist[e]);
+}
+
+cudaError_t launch_route_topk(const moe_config &c, const float *logits, const float *bias,
+                              int32_t *topk_idx, float *topk_w, int32_t *counts,
+                              uint32_t *status, cudaStream_t s, int num_sms) {
+    cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)c.E, s);
+    if (err != cudaSuccess || c.T == 0) return err;
+    const int warps_per_block = 8;
+    int blocks = (c.T + warps_per_block - 1) / warps_per_block;
+    const int cap = num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    const size_t smem = sizeof(int32_t) * (size_t)c.E;
+    const int vpl = (c.E + 31) / 32;
+#define MOE_ROUTE_CASE(V)                                                                   \
+    route_topk_kernel<V><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, topk_idx, \
+                                                   topk_w, counts, status)
+    if (vpl <= 1) MOE_ROUTE_CASE(1);
+    else if (vpl <= 2) MOE_ROUTE_CASE(2);
+    else if (vpl <= 4) MOE_ROUTE_CASE(4);
+    else if (vpl <= 8) MOE_ROUTE_CASE(8);
+    else if (vpl <= 16) MOE_ROUTE_CASE(16);
+    else MOE_ROUTE_CASE(32);
+#undef MOE_ROUTE_CASE
+    return cudaGetLastError();
+}
+
+}  // namespace moe

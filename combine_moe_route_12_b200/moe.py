@@ -1,0 +1,237 @@
+"""ctypes binding over libmoe_b200.so (include/moe_b200.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (device pointers are taken with
+``data_ptr()``); ``stream`` defaults to torch's current stream.  Importing
+this module raises if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from .build import LIB, ROOT
+
+if not os.path.exists(LIB):
+    raise ImportError(f"{LIB} is missing: build it with `python -m combine_moe_route_12_b200.build`")
+
+_lib = ctypes.CDLL(LIB)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_DEV_NONFINITE_LOGIT = 0x1
+MOE_DEV_WAIT_TIMEOUT = 0x2
+MOE_DEV_BAD_INDEX = 0x4
+
+
+class MoEConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T", "H", "E", "k", "I", "ep", "capacity", "dtype", "n_chunks", "reduce_dense")]
+
+    def __repr__(self):
+        return "MoEConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{status_string(status)} ({status}): {detail}")
+        self.status = status
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_CFG = ctypes.POINTER(MoEConfig)
+
+
+def _decl(name, restype, *argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = list(argtypes)
+    return f
+
+
+_decl("moe_config_check", _I32, _CFG)
+_decl("moe_workspace_bytes", ctypes.c_size_t, _CFG)
+_decl("moe_forward_workspace_bytes", ctypes.c_size_t, _CFG)
+_decl("moe_max_recv_rows", ctypes.c_int64, _CFG, _I32)
+_decl("moe_route_topk", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_capacity_clip", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_dispatch_layout", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_permute", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
+_decl("moe_grouped_swiglu_ffn", _I32, _CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P)
+_decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P)
+_decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
+_decl("moe_status_string", ctypes.c_char_p, _I32)
+_decl("moe_last_error_detail", ctypes.c_char_p)
+
+
+def header_symbols() -> list[str]:
+    """Entry points declared in include/moe_b200.h."""
+    text = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def last_error_detail() -> str:
+    return _lib.moe_last_error_detail().decode()
+
+
+def _check(status: int) -> None:
+    if status != MOE_OK:
+        raise MoEError(status, last_error_detail())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_config(T, H, E, k, I, ep, capacity=-1, dtype=MOE_BF16, n_chunks=1,
+                reduce_dense=False) -> MoEConfig:
+    if isinstance(dtype, str):
+        dtype = MOE_F32 if dtype == "f32" else MOE_BF16
+    return MoEConfig(T, H, E, k, I, ep, -1 if capacity is None else capacity, dtype, n_chunks,
+                     int(bool(reduce_dense)))
+
+
+def config_from_workload(wl) -> MoEConfig:
+    return make_config(wl.T, wl.H, wl.E, wl.k, wl.I, wl.ep, wl.capacity, wl.dtype, wl.n_chunks,
+                       wl.reduce_dense)
+
+
+# ------------------------------------------------------------------ sizes
+
+def config_check(cfg: MoEConfig) -> None:
+    _check(_lib.moe_config_check(ctypes.byref(cfg)))
+
+
+def workspace_bytes(cfg: MoEConfig) -> int:
+    return int(_lib.moe_workspace_bytes(ctypes.byref(cfg)))
+
+
+def forward_workspace_bytes(cfg: MoEConfig) -> int:
+    return int(_lib.moe_forward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def max_recv_rows(cfg: MoEConfig, tok_count: int) -> int:
+    return int(_lib.moe_max_recv_rows(ctypes.byref(cfg), tok_count))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace (torch allocations are 256-byte aligned)."""
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ the six steps
+
+def moe_route_topk(cfg, logits, bias, topk_idx, topk_w, counts, ws, stream=None):
+    _check(_lib.moe_route_topk(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(topk_idx),
+                               _ptr(topk_w), _ptr(counts), _ptr(ws), _stream(stream)))
+
+
+def moe_capacity_clip(cfg, topk_idx, topk_w, counts, keep, kept_counts, ws, stream=None):
+    _check(_lib.moe_capacity_clip(ctypes.byref(cfg), _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
+                                  _ptr(keep), _ptr(kept_counts), _ptr(ws), _stream(stream)))
+
+
+def moe_dispatch_layout(cfg, tok_begin, tok_count, topk_idx, keep, expert_offsets, rank_offsets,
+                        recv_token, recv_slot, pos, send_splits, splits_host, ws, stream=None):
+    _check(_lib.moe_dispatch_layout(ctypes.byref(cfg), tok_begin, tok_count, _ptr(topk_idx),
+                                    _ptr(keep), _ptr(expert_offsets), _ptr(rank_offsets),
+                                    _ptr(recv_token), _ptr(recv_slot), _ptr(pos),
+                                    _ptr(send_splits), _ptr(splits_host), _ptr(ws),
+                                    _stream(stream)))
+
+
+def moe_permute(cfg, x, pos, tok_begin, tok_count, xr, stream=None):
+    _check(_lib.moe_permute(ctypes.byref(cfg), _ptr(x), _ptr(pos), tok_begin, tok_count, _ptr(xr),
+                            _stream(stream)))
+
+
+def moe_grouped_swiglu_ffn(cfg, n_rows, xr, expert_offsets, w13, w2, h, y, recv_token,
+                           recv_slot, topk_w, out_reduce, ws, stream=None):
+    _check(_lib.moe_grouped_swiglu_ffn(ctypes.byref(cfg), n_rows, _ptr(xr), _ptr(expert_offsets),
+                                       _ptr(w13), _ptr(w2), _ptr(h), _ptr(y), _ptr(recv_token),
+                                       _ptr(recv_slot), _ptr(topk_w), _ptr(out_reduce), _ptr(ws),
+                                       _stream(stream)))
+
+
+def moe_combine(cfg, y, pos, topk_w, tok_begin, tok_count, out, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(cfg), _ptr(y), _ptr(pos), _ptr(topk_w), tok_begin,
+                            tok_count, _ptr(out), _stream(stream)))
+
+
+def moe_reduce_finalize(cfg, out_reduce, tok_begin, tok_count, out, stream=None):
+    _check(_lib.moe_reduce_finalize(ctypes.byref(cfg), _ptr(out_reduce), tok_begin, tok_count,
+                                    _ptr(out), _stream(stream)))
+
+
+def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, keep, splits_host,
+                        ws, s_dispatch=None, s_compute=None):
+    _check(_lib.moe_forward_chunked(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(x),
+                                    _ptr(w13), _ptr(w2), _ptr(out), _ptr(topk_idx), _ptr(topk_w),
+                                    _ptr(keep), _ptr(splits_host), _ptr(ws),
+                                    _stream(s_dispatch), _stream(s_compute)))
+
+
+def moe_device_status(ws, stream=None) -> int:
+    """Synchronises the stream; returns and clears the device status bits."""
+    flags = ctypes.c_uint32(0)
+    st = _lib.moe_device_status(_ptr(ws), ctypes.byref(flags), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        _check(st)
+    return int(flags.value)
+
+
+# ------------------------------------------------------------------ convenience
+
+class MoELayer:
+    """Owns the buffers of one layer shape and runs ``moe_forward_chunked``.
+
+    Weights are the caller's ([E, 2I, H] and [E, H, I] in the layer dtype).
+    Allocation goes through torch; the library allocates nothing.
+    """
+
+    def __init__(self, cfg: MoEConfig, device="cuda", host_splits: bool = True):
+        config_check(cfg)
+        self.cfg = cfg
+        dev = torch.device(device)
+        T, k = cfg.T, cfg.k
+        self.ws = alloc_workspace(forward_workspace_bytes(cfg), dev)
+        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.keep = torch.empty(T, k, dtype=torch.uint8, device=dev)
+        n = cfg.n_chunks * (cfg.E + 1 + cfg.ep * cfg.ep)
+        self.splits_host = torch.zeros(n, dtype=torch.int32, pin_memory=True) if host_splits else None
+        self.s_dispatch = torch.cuda.Stream(device=dev)
+
+    def forward(self, logits, bias, x, w13, w2, out, s_compute=None):
+        s_compute = s_compute or torch.cuda.current_stream()
+        moe_forward_chunked(self.cfg, logits, bias, x, w13, w2, out, self.topk_idx, self.topk_w,
+                            self.keep, self.splits_host, self.ws, self.s_dispatch, s_compute)
+        return out
+
+    def splits(self, chunk: int):
+        """Host copy of chunk `chunk`'s (expert_offsets, send_splits); valid after a sync."""
+        c = self.cfg
+        stride = c.E + 1 + c.ep * c.ep
+        v = self.splits_host[chunk * stride:(chunk + 1) * stride]
+        return v[:c.E + 1], v[c.E + 1:].view(c.ep, c.ep)

@@ -1,0 +1,275 @@
+/*
+ * moe_b200.h - C ABI of the B200 (sm_100a) expert-parallel MoE layer hot path.
+ *
+ * The layer, in the order the calls run:
+ *
+ *   1. moe_route_topk          router top-k with renormalised softmax weights
+ *   2. moe_capacity_clip       per-expert token capacity, lowest-weight excess dropped
+ *   3. moe_dispatch_layout     expert-contiguous, EP-rank-grouped receive layout,
+ *                              the all_to_all_single split counts, optional host copy
+ *   4. moe_permute             token rows -> receive rows
+ *   5. moe_grouped_swiglu_ffn  per-expert gate/up GEMM, silu(g)*u, down GEMM
+ *   6. moe_combine             weighted sum of each token's expert rows
+ *
+ * plus moe_forward_chunked, which runs 1-2 once and pipelines 3-6 over token
+ * chunks on two streams (dispatch of chunk c+1 overlaps the FFN of chunk c).
+ *
+ * Sources (restated, not copied):
+ *   [AX]  axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
+ *         expert_parallel_backend (torch = all_to_all_single over the EP group),
+ *         expert_parallel_dispatch_chunks, expert_parallel_save_dispatch
+ *         ("routing topk and host-side split counts are always saved"),
+ *         expert_parallel_size, expert_parallel_token_capacity, and
+ *         validate_expert_parallel_topology.
+ *   [LL]  LightLLM PR 1687 review page: _select_experts / norm_topk_prob,
+ *         the expert prefix-sum ("psum") contiguous layout of the grouped GEMM,
+ *         silu_and_mul between the grouped GEMMs, decode reducing expert
+ *         outputs straight into a dense output, comm-stream / compute-stream
+ *         ownership with record_stream, and dispatch capacity sized from the
+ *         padded worst case.
+ *
+ * Conventions that hold for every call:
+ *   - All pointers are DEVICE pointers unless the parameter name ends in
+ *     _host.  The caller allocates and owns every buffer, including the
+ *     workspace; the library never allocates or frees device memory and never
+ *     synchronises the device.  Every call is asynchronous on its stream(s).
+ *   - Layouts are row-major and dense.  x, xr, h, y, out, w13 and w2 hold
+ *     cfg->dtype elements (MOE_F32: float, MOE_BF16: bfloat16 bit patterns).
+ *   - Host-side argument errors return immediately and launch nothing.
+ *     Launch failures return MOE_ERR_CUDA.  Conditions only the device can see
+ *     (a non-finite logit, a bounded wait that ran out) set bits in the status
+ *     word inside the workspace; read them with moe_device_status.  No kernel
+ *     traps.
+ *   - moe_last_error_detail() describes the last non-OK status of the calling
+ *     thread.
+ *   - Workspace: a caller-owned device buffer of moe_workspace_bytes(cfg)
+ *     bytes (moe_forward_workspace_bytes(cfg) for moe_forward_chunked),
+ *     256-byte aligned, zero-filled ONCE before its first use.  A workspace
+ *     serves one stream (or one moe_forward_chunked stream pair) at a time.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* bad pointer, size or topology; nothing launched */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits (below)   */
+    MOE_ERR_WORKSPACE = 3,    /* workspace pointer misaligned                    */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed            */
+    MOE_ERR_DEVICE = 5        /* the device status word has bits set             */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Device status bits (moe_device_status). */
+#define MOE_DEV_NONFINITE_LOGIT 0x1u  /* a logit (+bias) was NaN or +-Inf          */
+#define MOE_DEV_WAIT_TIMEOUT    0x2u  /* a bounded spin (lookback scan, mbarrier)  */
+                                      /* gave up; outputs of that call are invalid */
+#define MOE_DEV_BAD_INDEX       0x4u  /* an expert id outside [0, E) was read      */
+
+/*
+ * Layer shape.  T tokens, hidden size H, E experts, top-k k, FFN intermediate
+ * size I, ep logical EP ranks ([AX] expert_parallel_size; rank d owns the
+ * contiguous experts [d*E/ep, (d+1)*E/ep)), capacity per expert per forward
+ * ([AX] expert_parallel_token_capacity; < 0 = no cap), n_chunks dispatch
+ * chunks ([AX] expert_parallel_dispatch_chunks), reduce_dense = 1 for the
+ * decode form in which the FFN reduces w*y straight into a dense fp32 [T, H]
+ * buffer ([LL] decode reduce) instead of storing y.
+ *
+ * Topology checks ([AX] validate_expert_parallel_topology, restated):
+ * T >= 0, H, E, k, I, ep, n_chunks >= 1, k <= E, E % ep == 0,
+ * T % n_chunks == 0, (T / n_chunks) % ep == 0 (each chunk splits into equal
+ * contiguous source-rank blocks).
+ * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30;
+ * MOE_BF16 needs H % 64 == 0 and I % 64 == 0 (tensor-core tiles);
+ * MOE_F32 needs H % 4 == 0 and I % 4 == 0.
+ */
+typedef struct {
+    int32_t T, H, E, k, I, ep;
+    int32_t capacity;
+    int32_t dtype;          /* moe_dtype */
+    int32_t n_chunks;
+    int32_t reduce_dense;
+} moe_config;
+
+/* Validates cfg (topology and limits).  MOE_OK or the reason it is rejected. */
+moe_status moe_config_check(const moe_config *cfg);
+
+/* Scratch bytes the step calls need (status word, scan state, thresholds,
+ * tile scheduler).  0 if cfg is invalid. */
+size_t moe_workspace_bytes(const moe_config *cfg);
+
+/* Bytes moe_forward_chunked needs: the scratch above plus two chunk slots of
+ * layout arrays, xr, h and y, and the dense fp32 reduce buffer in decode form.
+ * 0 if cfg is invalid. */
+size_t moe_forward_workspace_bytes(const moe_config *cfg);
+
+/* Worst-case receive rows of one call over tok_count tokens:
+ * min(tok_count * k, E * capacity) (capacity >= 0), else tok_count * k.
+ * Receive buffers (recv_token, recv_slot, xr, h, y) need this many rows; it is
+ * the padded worst case, not the count of the current batch ([LL] decode
+ * dispatch capacity).  -1 if cfg is invalid. */
+int64_t moe_max_recv_rows(const moe_config *cfg, int32_t tok_count);
+
+/*
+ * Step 1 - router top-k ([LL] _select_experts with norm_topk_prob; [AX] the
+ * routing top-k is saved state, so it is a caller-owned output).
+ *   logits   fp32 [T, E]; bias fp32 [E] or NULL (added to the logits before
+ *            selection and weighting).
+ *   topk_idx int32 [T, k]: experts by (logit+bias) descending, the lower expert
+ *            index first among equal values; slot j = rank j.
+ *   topk_w   fp32 [T, k]: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0), i.e.
+ *            the softmax restricted to the top k and renormalised.  The
+ *            exponential is a fixed Cody-Waite + degree-7 Taylor evaluation in
+ *            fp32 and the sum runs in slot order, so the weights are
+ *            bit-reproducible.
+ *   counts   int32 [E]: assignments per expert (before the clip).
+ * A non-finite logit sets MOE_DEV_NONFINITE_LOGIT; that token's outputs are
+ * then unspecified.
+ */
+moe_status moe_route_topk(const moe_config *cfg, const float *logits, const float *bias,
+                          int32_t *topk_idx, float *topk_w, int32_t *counts,
+                          void *ws, cudaStream_t stream);
+
+/*
+ * Step 2 - per-expert capacity ([AX] expert_parallel_token_capacity): an
+ * expert that received more than C = cfg->capacity assignments keeps the C
+ * with the largest topk_w and drops the rest; among equal weights the higher
+ * token index is dropped first.  Kept weights are not renormalised.
+ *   topk_idx, topk_w, counts: outputs of step 1 over all T tokens.
+ *   keep        uint8 [T, k]: 1 kept, 0 dropped.
+ *   kept_counts int32 [E].
+ * With capacity < 0 every assignment is kept.  The clip always runs over the
+ * whole forward (all T tokens), before any chunking.
+ */
+moe_status moe_capacity_clip(const moe_config *cfg, const int32_t *topk_idx,
+                             const float *topk_w, const int32_t *counts, uint8_t *keep,
+                             int32_t *kept_counts, void *ws, cudaStream_t stream);
+
+/*
+ * Step 3 - dispatch layout of the tokens [tok_begin, tok_begin + tok_count)
+ * ([AX] torch backend: all_to_all_single over the EP group; [LL] psum layout).
+ * The ep ranks are logical: source rank s holds the chunk's tokens
+ * [tok_begin + s*tok_count/ep, tok_begin + (s+1)*tok_count/ep) and destination
+ * rank d owns experts [d*E/ep, (d+1)*E/ep).  Receive rows are ordered by
+ * (destination rank, expert, token), which is the all_to_all_single arrival
+ * order regrouped by expert, and equals the stable order by (expert, token).
+ *   expert_offsets int32 [E+1]: rows of expert e are [expert_offsets[e],
+ *                  expert_offsets[e+1]); expert_offsets[E] = N.
+ *   rank_offsets   int32 [ep+1]: rank_offsets[d] = expert_offsets[d*E/ep].
+ *   recv_token     int32 [N_max]: absolute token index of each row.
+ *   recv_slot      int32 [N_max]: top-k slot of each row.
+ *   pos            int32 [tok_count, k]: row of (tok_begin+i, j), -1 if dropped.
+ *   send_splits    int32 [ep, ep]: rows source s sends to destination d
+ *                  (the receive splits are its transpose).
+ *   splits_host    pinned host int32 [E+1 + ep*ep] or NULL: receives
+ *                  expert_offsets then send_splits by an async copy on
+ *                  `stream` ([AX]: the host-side split counts); valid once
+ *                  the stream (or an event recorded after this call) completes.
+ * N_max = moe_max_recv_rows(cfg, tok_count).
+ */
+moe_status moe_dispatch_layout(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
+                               const int32_t *topk_idx, const uint8_t *keep,
+                               int32_t *expert_offsets, int32_t *rank_offsets,
+                               int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                               int32_t *send_splits, int32_t *splits_host,
+                               void *ws, cudaStream_t stream);
+
+/*
+ * Step 4 - permute: xr[pos[i, j], :] = x[tok_begin + i, :] for every kept
+ * (i, j).  x is [T, H]; xr is [N_max, H]; rows >= N are left untouched.
+ */
+moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *pos,
+                       int32_t tok_begin, int32_t tok_count, void *xr, cudaStream_t stream);
+
+/*
+ * Step 5 - grouped SwiGLU FFN over the expert-contiguous rows ([LL] grouped
+ * GEMM on the psum layout, silu_and_mul, grouped GEMM).  For each expert e and
+ * row p in [expert_offsets[e], expert_offsets[e+1]):
+ *   g = W13[e, 0:I, :] . xr[p],  u = W13[e, I:2I, :] . xr[p],
+ *   h[p] = silu(g) * u           (stored in cfg->dtype),
+ *   y[p] = W2[e] . h[p]          (stored in cfg->dtype).
+ *   w13 [E, 2I, H] and w2 [E, H, I]: row-major, K contiguous, used as given.
+ *   n_rows: allocated rows of xr, h and y (>= N; normally N_max).
+ *   xr [n_rows, H], h [n_rows, I], y [n_rows, H] (y may be NULL in decode form).
+ * Decode form (cfg->reduce_dense = 1): y is not stored; instead
+ *   out_reduce[recv_token[p], :] += topk_w[recv_token[p], recv_slot[p]] * y[p]
+ * in fp32 (out_reduce: fp32 [T, H], zero-filled by the caller; the order of
+ * the additions is unspecified).  recv_token, recv_slot and topk_w are only
+ * read in decode form.
+ * MOE_BF16 runs on tcgen05 tensor cores (bf16 x bf16 -> fp32 in TMEM);
+ * MOE_F32 runs fp32 FMA on the CUDA cores.
+ */
+moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const void *xr,
+                                  const int32_t *expert_offsets, const void *w13,
+                                  const void *w2, void *h, void *y,
+                                  const int32_t *recv_token, const int32_t *recv_slot,
+                                  const float *topk_w, float *out_reduce,
+                                  void *ws, cudaStream_t stream);
+
+/*
+ * Step 6 - combine back to token order ([AX] combine all-to-all then the
+ * weighted sum): for t in [tok_begin, tok_begin + tok_count)
+ *   out[t, :] = sum over j = 0..k-1 with pos[t - tok_begin, j] >= 0 of
+ *               topk_w[t, j] * y[pos[t - tok_begin, j], :]
+ * accumulated in fp32 in slot order and rounded once to cfg->dtype; a token
+ * whose every slot was dropped gets zeros.
+ */
+moe_status moe_combine(const moe_config *cfg, const void *y, const int32_t *pos,
+                       const float *topk_w, int32_t tok_begin, int32_t tok_count,
+                       void *out, cudaStream_t stream);
+
+/* Decode form of step 6: out[t, :] = round(out_reduce[t, :]) for the tokens
+ * [tok_begin, tok_begin + tok_count). */
+moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
+                               int32_t tok_begin, int32_t tok_count, void *out,
+                               cudaStream_t stream);
+
+/*
+ * The whole layer, chunked ([AX] expert_parallel_dispatch_chunks; [LL]
+ * chunked prefill with comm / compute streams).  Steps 1-2 run once over all
+ * T tokens on s_dispatch (the capacity is per forward).  Then for each
+ * contiguous chunk c of T/n_chunks tokens, steps 3-4 run on s_dispatch and
+ * steps 5-6 on s_compute, so chunk c+1's dispatch overlaps chunk c's FFN.
+ * Intermediates live in two chunk slots of the workspace; slot c%2 is reused
+ * only after chunk c-2's combine finished.  n_chunks = 1 gives the unchunked
+ * layer.  The result equals the unchunked one bit for bit.
+ *   logits, bias, x, w13, w2 as in steps 1-5; out [T, H] cfg->dtype.
+ *   topk_idx [T,k], topk_w [T,k], keep [T,k]: caller-owned saved state
+ *            ([AX] the routing top-k is always saved).
+ *   splits_host: pinned host int32 [n_chunks * (E+1 + ep*ep)] or NULL; chunk c
+ *            writes expert_offsets then send_splits at offset c*(E+1+ep*ep).
+ *   ws: moe_forward_workspace_bytes(cfg) bytes.
+ *   s_dispatch, s_compute: may be the same stream.  On return both streams
+ *            are ordered after all the layer's work ([LL] record_stream: the
+ *            caller's buffers are touched by both streams, so a caching
+ *            allocator must see them used on both).
+ */
+moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
+                               const void *x, const void *w13, const void *w2, void *out,
+                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                               int32_t *splits_host, void *ws,
+                               cudaStream_t s_dispatch, cudaStream_t s_compute);
+
+/* Synchronises `stream`, copies the device status word of ws to *flags and
+ * clears it.  Returns MOE_ERR_DEVICE if any bit was set. */
+moe_status moe_device_status(void *ws, uint32_t *flags, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *moe_status_string(moe_status status);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char *moe_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,83 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every
+entry point the header declares, and its argument / topology checks
+(axolotl ExpertParallelArgs, validate_expert_parallel_topology) reject what
+they should.  No call here touches a device."""
+import ctypes
+
+import pytest
+
+from combine_moe_route_12_b200 import build
+
+build.build()
+from combine_moe_route_12_b200 import moe  # noqa: E402
+from combine_moe_route_12_b200.workload import WORKLOADS  # noqa: E402
+
+
+def test_library_exports_every_header_symbol():
+    lib = ctypes.CDLL(build.LIB)
+    names = moe.header_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    for required in ("moe_route_topk", "moe_capacity_clip", "moe_dispatch_layout",
+                     "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine",
+                     "moe_forward_chunked"):
+        assert required in names
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workloads_pass_topology_checks(name):
+    cfg = moe.config_from_workload(WORKLOADS[name])
+    moe.config_check(cfg)
+    assert moe.workspace_bytes(cfg) > 0
+    assert moe.forward_workspace_bytes(cfg) >= moe.workspace_bytes(cfg)
+
+
+def test_max_recv_rows_is_padded_worst_case():
+    c = moe.make_config(256, 7168, 256, 8, 2048, 64, capacity=1024)
+    assert moe.max_recv_rows(c, 256) == 256 * 8           # cap never binds
+    c = moe.make_config(16384, 2048, 128, 8, 768, 4, capacity=1024)
+    assert moe.max_recv_rows(c, 16384) == 128 * 1024      # cap binds
+    c = moe.make_config(64, 128, 8, 2, 128, 2, capacity=0)
+    assert moe.max_recv_rows(c, 64) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(E=10, ep=4), moe.MOE_ERR_INVALID_ARG),           # E % ep
+    (dict(T=100, ep=8), moe.MOE_ERR_INVALID_ARG),          # tokens per source rank
+    (dict(T=96, n_chunks=5), moe.MOE_ERR_INVALID_ARG),     # T % n_chunks
+    (dict(k=9, E=8, ep=1), moe.MOE_ERR_INVALID_ARG),       # k > E
+    (dict(k=33, E=64), moe.MOE_ERR_UNSUPPORTED),
+    (dict(E=2048, ep=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=96), moe.MOE_ERR_UNSUPPORTED),                 # bf16 tiles need H % 64
+    (dict(I=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(dtype=7), moe.MOE_ERR_INVALID_ARG),
+    (dict(n_chunks=0), moe.MOE_ERR_INVALID_ARG),
+])
+def test_config_rejections(kw, status):
+    base = dict(T=64, H=128, E=8, k=2, I=128, ep=2, capacity=-1, dtype=moe.MOE_BF16,
+                n_chunks=1, reduce_dense=False)
+    base.update(kw)
+    cfg = moe.make_config(**base)
+    with pytest.raises(moe.MoEError) as ei:
+        moe.config_check(cfg)
+    assert ei.value.status == status
+    assert moe.last_error_detail()
+    assert moe.workspace_bytes(cfg) == 0
+
+
+def test_null_workspace_rejected_before_any_launch():
+    cfg = moe.make_config(64, 128, 8, 2, 128, 2)
+    st = moe._lib.moe_route_topk(ctypes.byref(cfg), None, None, None, None, None, None, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    st = moe._lib.moe_dispatch_layout(ctypes.byref(cfg), 0, 60, None, None, None, None, None,
+                                      None, None, None, None, ctypes.c_void_p(256), None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+    st = moe._lib.moe_dispatch_layout(ctypes.byref(cfg), 0, 63, None, None, None, None, None,
+                                      None, None, None, None, ctypes.c_void_p(256), None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "divisible" in moe.last_error_detail()
+
+
+def test_status_strings():
+    for s in range(6):
+        assert moe.status_string(s)
