@@ -1,0 +1,546 @@
+#!/usr/bin/env python
+"""Benchmark of the expert-parallel MoE layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole layer (router top-k, capacity clip, dispatch
+layout, permute, grouped SwiGLU FFN, combine) over one batch of seeded
+synthetic inputs that are resident in HBM.  The default workload is the
+Qwen3-30B-A3B-shaped layer (T=4096, H=2048, E=128, k=8, I=768, bf16, EP=2).
+
+Prints one JSON line (rank 0).  Besides the contract keys it reports a
+per-stage breakdown, dispatch+combine HBM GB/s, FFN TFLOP/s, the roofline of
+the dominant kernel (the grouped FFN), an end-to-end number through the
+public API with host buffers, and the CPU oracle timed on a bounded sample.
+
+With --gpus N > 1 (launched by torchrun) every rank runs an independent
+replica of the workload (the layer's EP ranks are logical, inside one GPU),
+so there is no data-path collective; the time is the max over ranks and the
+value counts the tokens of all ranks (weak scaling).
+
+--impl reference times the CPU oracle (plain C, one core) on a bounded sample
+of the same workload, each step a sample, and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec at 1 B200; dispatch+combine HBM GB/s; FFN tensor-pipe %"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of the grouped FFN (both GEMM launches) per layer pass, from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); see
+# profiles/ffn_tcgen05_qwen3_30b_a3b.md.  Keyed by workload; ``src`` is the
+# sha256 prefix of the kernel source the counters were taken on - a changed
+# kernel reports null until it is captured again.
+FFN_TRAFFIC = {}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="qwen3_30b_a3b")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    p.add_argument("--seed", type=int, default=None)
+    return p.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_src_hash():
+    p = os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", "ffn_tcgen05.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML (reads
+    only) on a background thread while the GPU is busy."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((sm, pw, rs, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "no NVML samples"}
+        busy = [s for s in self.samples if s[3] > 0] or self.samples
+        reasons = set()
+        for s in busy:
+            for name, bit in self.REASONS.items():
+                if s[2] & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(busy),
+                "power_w_max": max(s[1] for s in busy)}
+
+
+# --------------------------------------------------------------------------- workload
+
+def kernels_per_step(wl) -> int:
+    # route 1, clip 2 (select, mark); per chunk: layout 3 (hist, scatter, splits),
+    # permute 1, FFN 2 (two GEMM launches), combine or finalize 1
+    return 3 + wl.n_chunks * 7
+
+
+def algorithmic(wl, n_kept_chunks):
+    """Bytes / flops the method must move or compute (nothing for dropped rows)."""
+    b = wl.elem_bytes
+    N = sum(n_kept_chunks)
+    tok_bytes = wl.T * wl.H * b
+    row_bytes = N * wl.H * b
+    return {
+        "permute_bytes": tok_bytes + row_bytes,
+        "combine_bytes": (0 if wl.reduce_dense else row_bytes) + tok_bytes,
+        "ffn_flops": 6.0 * wl.H * wl.I * N,
+        "N": N,
+    }
+
+
+class StepBuffers:
+    """Every buffer the six ABI calls of one unchunked step touch."""
+
+    def __init__(self, moe, wl, cfg, dev):
+        import torch
+        T, E, k, H, I, ep = wl.T, wl.E, wl.k, wl.H, wl.I, wl.ep
+        self.ws = moe.alloc_workspace(moe.workspace_bytes(cfg), dev)
+        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.keep = torch.empty(T, k, dtype=torch.uint8, device=dev)
+        self.kept = torch.empty(E, dtype=torch.int32, device=dev)
+        tc = T // wl.n_chunks
+        self.tc = tc
+        self.nmax = moe.max_recv_rows(cfg, tc)
+        n = max(self.nmax, 1)
+        self.eoff = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.roff = torch.empty(ep + 1, dtype=torch.int32, device=dev)
+        self.rt = torch.empty(n, dtype=torch.int32, device=dev)
+        self.rs = torch.empty(n, dtype=torch.int32, device=dev)
+        self.pos = torch.empty(tc, k, dtype=torch.int32, device=dev)
+        self.spl = torch.empty(ep, ep, dtype=torch.int32, device=dev)
+        self.xr = torch.empty(n, H, dtype=wl.torch_dtype, device=dev)
+        self.h = torch.empty(n, I, dtype=wl.torch_dtype, device=dev)
+        self.y = None if wl.reduce_dense else torch.empty(n, H, dtype=wl.torch_dtype, device=dev)
+        self.red = torch.zeros(T, H, dtype=torch.float32, device=dev) if wl.reduce_dense else None
+        self.out = torch.empty(T, H, dtype=wl.torch_dtype, device=dev)
+
+
+def n_marks(wl) -> int:
+    return 3 + 4 * wl.n_chunks
+
+
+def run_steps(moe, wl, cfg, inp, B, ev=None):
+    """One layer pass through the step ABI on the current stream.  ev: list of
+    n_marks(wl) events recorded between the stages, or None."""
+    rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+    rec(0)
+    moe.moe_route_topk(cfg, inp.logits, inp.bias, B.topk_idx, B.topk_w, B.counts, B.ws)
+    rec(1)
+    moe.moe_capacity_clip(cfg, B.topk_idx, B.topk_w, B.counts, B.keep, B.kept, B.ws)
+    if wl.reduce_dense:
+        B.red.zero_()
+    rec(2)
+    for c in range(wl.n_chunks):
+        tb = c * B.tc
+        base = 3 + 4 * c
+        moe.moe_dispatch_layout(cfg, tb, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
+                                B.pos, B.spl, None, B.ws)
+        rec(base)
+        moe.moe_permute(cfg, inp.x, B.pos, tb, B.tc, B.xr)
+        rec(base + 1)
+        moe.moe_grouped_swiglu_ffn(cfg, B.nmax, B.xr, B.eoff, inp.w13, inp.w2, B.h, B.y, B.rt,
+                                   B.rs, B.topk_w, B.red, B.ws)
+        rec(base + 2)
+        if wl.reduce_dense:
+            moe.moe_reduce_finalize(cfg, B.red, tb, B.tc, B.out)
+        else:
+            moe.moe_combine(cfg, B.y, B.pos, B.topk_w, tb, B.tc, B.out)
+        rec(base + 3)
+
+
+def stage_times(wl, ev):
+    """Per-stage milliseconds of one step recorded by run_steps."""
+    t = {"route_topk": ev[0].elapsed_time(ev[1]), "capacity_clip": ev[1].elapsed_time(ev[2]),
+         "dispatch_layout": 0.0, "permute": 0.0, "grouped_ffn": 0.0, "combine": 0.0}
+    for c in range(wl.n_chunks):
+        b = 3 + 4 * c
+        t["dispatch_layout"] += ev[b - 1].elapsed_time(ev[b])
+        t["permute"] += ev[b].elapsed_time(ev[b + 1])
+        t["grouped_ffn"] += ev[b + 1].elapsed_time(ev[b + 2])
+        t["combine"] += ev[b + 2].elapsed_time(ev[b + 3])
+    return t
+
+
+STAGES = ["route_topk", "capacity_clip", "dispatch_layout", "permute", "grouped_ffn", "combine"]
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens):
+    """Times the oracle, as it stands, on a bounded sample: route + clip +
+    layout + permute over all T tokens, then FFN + combine for the rows of the
+    first `sample_tokens` tokens.  Returns (tokens/s extrapolated to the whole
+    layer, seconds of CPU work, description)."""
+    import numpy as np
+    import oracle
+    t0 = time.perf_counter()
+    idx, w, _, st = oracle.route_topk(logits, bias, wl.k)
+    keep, _ = oracle.capacity_clip(idx, w, wl.E, wl.capacity)
+    tc = wl.T // wl.n_chunks
+    lays = [oracle.dispatch_layout(idx, keep, wl.E, wl.ep, c * tc, tc) for c in range(wl.n_chunks)]
+    xrs = [oracle.permute(x_np, lay["recv_token"]) for lay in lays]
+    t_index = time.perf_counter() - t0
+    # rows of the sampled tokens (they sit in chunk 0)
+    lay = lays[0]
+    rows = [(p, e) for e in range(wl.E) for p in range(int(lay["expert_offsets"][e]), int(lay["expert_offsets"][e + 1]))
+            if lay["recv_token"][p] < sample_tokens]
+    weights = {e: fetch_expert(e) for e in sorted({e for _, e in rows})}   # host copies, untimed
+    N = lay["N"]
+    y = np.zeros((max(N, 1), wl.H), x_np.dtype)
+    ye = np.zeros((max(N, 1), wl.H), np.float64)
+    t1 = time.perf_counter()
+    for p, e in rows:
+        _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
+    sub_pos = lay["pos"][:sample_tokens]
+    if wl.reduce_dense:
+        oracle.combine_exact(ye, sub_pos, w, wl.T, x_np.dtype)
+    else:
+        oracle.combine(y, sub_pos, w, wl.T)
+    t_ffn = time.perf_counter() - t1
+    layer_s = t_index + t_ffn * (wl.T / sample_tokens)
+    desc = (f"oracle route+clip+layout+permute over all {wl.T} tokens ({t_index:.2f} s), FFN+combine "
+            f"for the {len(rows)} rows of the first {sample_tokens} tokens ({t_ffn:.2f} s), "
+            f"extrapolated linearly to {wl.T} tokens")
+    return wl.T / layer_s, t_index + t_ffn, desc
+
+
+def sample_tokens_for(wl, seconds):
+    row_s = 7.7e-3 * (wl.H * wl.I) / (2048 * 768)      # measured oracle cost of one FFN row
+    s = int(seconds / (wl.k * row_s))
+    return max(1, min(wl.T // wl.n_chunks, s))
+
+
+# --------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    from combine_moe_route_12_b200.workload import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.config]
+    # inputs drawn on the CPU generator (no GPU needed for this arm)
+    torch.manual_seed(0)
+    inp = make_inputs(wl, "cpu", seed=args.seed, weights=False)
+    g = torch.Generator().manual_seed(wl.seed + 1)
+    std = 1.0 / math.sqrt(wl.H)
+    cache = {}
+
+    def fetch(e):
+        if e not in cache:
+            a = (torch.randn(2 * wl.I, wl.H, generator=g) * std).to(wl.torch_dtype)
+            b = (torch.randn(wl.H, wl.I, generator=g) * std).to(wl.torch_dtype)
+            conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
+                else (lambda t: t.numpy().copy())
+            cache[e] = (conv(a), conv(b))
+        return cache[e]
+
+    conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
+        else (lambda t: t.numpy().copy())
+    logits = inp.logits.numpy()
+    bias = None if inp.bias is None else inp.bias.numpy()
+    x_np = conv(inp.x)
+    s_tok = sample_tokens_for(wl, 1.0)
+    vals = []
+    t_all = 0.0
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        v, secs, desc = oracle_sample(wl, logits, bias, x_np, fetch, s_tok)
+        if i >= args.warmup:
+            vals.append(v)
+            t_all += secs
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.T / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64" if wl.dtype == "bf16" else "f64", "data": "synthetic",
+        "config": workload_config(wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, n):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+            "ep_logical": wl.ep, "capacity": wl.capacity, "dispatch_chunks": wl.n_chunks,
+            "decode_reduce": wl.reduce_dense, "global_batch_tokens": wl.T * n,
+            "parallelism": "replicas" if n > 1 else "single",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    from combine_moe_route_12_b200 import moe
+    from combine_moe_route_12_b200.workload import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.config]
+    cfg = moe.config_from_workload(wl)
+    peaks, peak_src = load_peaks()
+    inp = make_inputs(wl, dev, seed=args.seed)
+    torch.cuda.synchronize()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+
+    # ---------------- timed region: K layer passes
+    steps_mode = wl.n_chunks == 1
+    B = StepBuffers(moe, wl, cfg, dev)
+    layer = moe.MoELayer(cfg, dev, host_splits=False)
+    out_fw = torch.empty(wl.T, wl.H, dtype=wl.torch_dtype, device=dev)
+
+    def one_step(ev):
+        if steps_mode:
+            run_steps(moe, wl, cfg, inp, B, ev)
+        else:
+            ev[0].record()
+            layer.forward(inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out_fw)
+            ev[-1].record()
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(n_marks(wl))]
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        one_step(mk())
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [mk() for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(1)
+        one_step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if moe.moe_device_status(B.ws if steps_mode else layer.ws) != 0:
+        raise RuntimeError("device status bits set during the timed region")
+
+    # ---------------- per-stage breakdown (same kernels, one stream)
+    stage_ms = {s: 0.0 for s in STAGES}
+    if steps_mode:
+        bd = evs
+    else:
+        bd = [mk() for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(1)
+            run_steps(moe, wl, cfg, inp, B, bd[i])
+        torch.cuda.synchronize()
+    for e in bd:
+        for s, v in stage_times(wl, e).items():
+            stage_ms[s] += v / len(bd)
+    n_kept = []
+    for c in range(wl.n_chunks):
+        moe.moe_dispatch_layout(cfg, c * B.tc, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
+                                B.pos, B.spl, None, B.ws)
+        n_kept.append(int(B.eoff[wl.E].item()))
+    alg = algorithmic(wl, n_kept)
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_logits = inp.logits.cpu().pin_memory()
+        h_x = inp.x.cpu().pin_memory()
+        h_bias = None if inp.bias is None else inp.bias.cpu().pin_memory()
+        h_out = torch.empty(wl.T, wl.H, dtype=wl.torch_dtype).pin_memory()
+        d_logits = torch.empty_like(inp.logits)
+        d_x = torch.empty_like(inp.x)
+        d_bias = None if inp.bias is None else torch.empty_like(inp.bias)
+        e2e_ms = 0.0
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            d_logits.copy_(h_logits, non_blocking=True)
+            d_x.copy_(h_x, non_blocking=True)
+            if d_bias is not None:
+                d_bias.copy_(h_bias, non_blocking=True)
+            layer.forward(d_logits, d_bias, d_x, inp.w13, inp.w2, out_fw)
+            h_out.copy_(out_fw, non_blocking=True)
+            b.record()
+            b.synchronize()
+            if i >= args.warmup:
+                e2e_ms += a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = h_logits.numel() * 4 + h_x.numel() * h_x.element_size() + (0 if h_bias is None else h_bias.numel() * 4)
+        d2h = h_out.numel() * h_out.element_size()
+        e2e = {"value": world * wl.T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    sampler.stop()
+    clocks = sampler.summary()
+
+    # ---------------- CPU oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        conv = (lambda t: t.detach().cpu().view(torch.int16).numpy().view(np.uint16).copy()) \
+            if wl.dtype == "bf16" else (lambda t: t.detach().cpu().numpy().copy())
+        fetch = lambda e: (conv(inp.w13[e]), conv(inp.w2[e]))
+        s_tok = sample_tokens_for(wl, 15.0)
+        v, secs, desc = oracle_sample(wl, inp.logits.cpu().numpy(),
+                                      None if inp.bias is None else inp.bias.cpu().numpy(),
+                                      conv(inp.x), fetch, s_tok)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+               "cpu_seconds": round(secs, 2)}
+
+    if rank == 0:
+        ms_per_step = total_ms / args.steps
+        value = world * wl.T * args.steps / (total_ms / 1e3)
+        ffn_s = stage_ms["grouped_ffn"] / 1e3
+        dc_s = (stage_ms["permute"] + stage_ms["combine"]) / 1e3
+        ffn_tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
+        dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
+        src = kernel_src_hash()
+        tr = FFN_TRAFFIC.get(wl.name)
+        traffic = tr["bytes"] if tr and tr.get("src") == src else None
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, world),
+            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2)",
+                         "bound": "tensor", "achieved": ffn_tflops,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": ffn_tflops / peaks["bf16_tflops"] if ffn_tflops else None,
+                         "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "algorithmic_per_launch": f"6*H*I*N = {alg['ffn_flops']:.4g} flop over N={alg['N']} kept rows"},
+            "dispatch_combine": {"achieved_gbs": dc_gbs, "peak_gbs": peaks["hbm_gbs"],
+                                 "frac": dc_gbs / peaks["hbm_gbs"] if dc_gbs else None,
+                                 "bytes_per_step": alg["permute_bytes"] + alg["combine_bytes"],
+                                 "peak_source": f"{peak_src} hbm_gbs"},
+            "ffn_tflops": ffn_tflops,
+            "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "kept_rows": alg["N"],
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": kernels_per_step(wl) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

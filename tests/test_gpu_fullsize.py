@@ -1,0 +1,116 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times.
+
+Routing, drop sets, layouts and split counts are compared whole against the
+oracle (bit-exact).  Permuted rows are checked whole by the defining property
+xr[p] = x[recv_token[p]] (bitwise).  The FFN and the combined output are
+compared on sampled rows and tokens that the oracle computes one by one:
+experts at both ends of the expert range, the most loaded expert and a random
+one, each with its first, last and random rows; and tokens spread over the
+batch.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_moe_route_12_b200 import moe
+from combine_moe_route_12_b200.workload import WORKLOADS, MoEInputs, make_inputs
+
+from moe_testlib import (assert_float_close, assert_routing_equal, oracle_routing,
+                         run_gpu_steps, storage_np)
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode"]
+
+
+def _host_expert(inp, e, cache):
+    if e not in cache:
+        cache[e] = (storage_np(inp.w13[e]), storage_np(inp.w2[e]))
+    return cache[e]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_fullsize_against_oracle(name):
+    wl = WORKLOADS[name]
+    torch.cuda.empty_cache()
+    inp = make_inputs(wl, "cuda")
+    g = run_gpu_steps(wl, inp, keep_rows=False)
+    assert g["status"] == 0
+    cpu_inp = MoEInputs(logits=inp.logits.cpu(), bias=None if inp.bias is None else inp.bias.cpu(),
+                        x=inp.x.cpu(), w13=inp.w13, w2=inp.w2)
+    orc = oracle_routing(wl, cpu_inp)
+    assert_routing_equal(g, orc, wl)
+    if wl.capacity >= 0:
+        assert (orc["kept_counts"] <= wl.capacity).all()
+
+    x_np = storage_np(inp.x)
+    rng = np.random.default_rng(0)
+    cache = {}
+    for c, (gc, lay) in enumerate(zip(g["chunks"], orc["layouts"])):
+        n = lay["N"]
+        rt = torch.from_numpy(lay["recv_token"]).long().cuda()
+        assert torch.equal(gc["xr_dev"][:n], inp.x[rt]), "permute must copy rows bitwise"
+        eoff = lay["expert_offsets"]
+        sizes = np.diff(eoff)
+        nonempty = np.nonzero(sizes)[0]
+        experts = {int(nonempty[0]), int(nonempty[-1]), int(np.argmax(sizes)),
+                   int(rng.choice(nonempty))}
+        for e in sorted(experts):
+            lo, hi = int(eoff[e]), int(eoff[e + 1])
+            rows = sorted({lo, hi - 1, *rng.integers(lo, hi, 2).tolist()})
+            w13e, w2e = _host_expert(inp, e, cache)
+            for p in rows:
+                h_ref, y_ref, ye_ref = oracle.ffn_row(x_np[lay["recv_token"][p]], w13e, w2e)
+                assert_float_close(storage_np(gc["h_dev"][p]), h_ref, wl.dtype, f"h[{p}] expert {e}")
+                if gc["y_dev"] is not None:
+                    assert_float_close(storage_np(gc["y_dev"][p]), y_ref, wl.dtype, f"y[{p}] expert {e}")
+
+    out = storage_np(g["out"])
+    tokens = sorted({0, wl.T - 1, *rng.integers(0, wl.T, 2).tolist()})
+    for t in tokens:
+        ys, yes, pos = [], [], []
+        for j in range(wl.k):
+            if not orc["keep"][t, j]:
+                pos.append(-1)
+                continue
+            w13e, w2e = _host_expert(inp, int(orc["topk_idx"][t, j]), cache)
+            _, y_ref, ye_ref = oracle.ffn_row(x_np[t], w13e, w2e)
+            pos.append(len(ys))
+            ys.append(y_ref)
+            yes.append(ye_ref)
+        posa = np.array([pos], np.int32)
+        w_t = orc["topk_w"][t:t + 1]
+        if not ys:
+            ref = np.zeros((1, wl.H), x_np.dtype)
+        elif wl.reduce_dense:
+            ref = oracle.combine_exact(np.stack(yes), posa, w_t, 1, x_np.dtype)
+        else:
+            ref = oracle.combine(np.stack(ys), posa, w_t, 1)
+        assert_float_close(out[t:t + 1], ref, wl.dtype, f"out[{t}]")
+    del g, inp
+    torch.cuda.empty_cache()
+
+
+def test_dsv3_prefill_chunked_forward_equals_steps():
+    """Two-stream chunked forward at the full DeepSeek-V3 prefill shape gives
+    the same bits as the step-by-step path, and as the unchunked forward."""
+    wl = WORKLOADS["dsv3_prefill"]
+    torch.cuda.empty_cache()
+    inp = make_inputs(wl, "cuda", seed=3)
+    g = run_gpu_steps(wl, inp, keep_rows=False)
+    ref = g["out"]
+    del g
+    outs = []
+    for n_chunks in (2, 1):
+        w = wl.with_(n_chunks=n_chunks)
+        layer = moe.MoELayer(moe.config_from_workload(w))
+        out = torch.empty(wl.T, wl.H, dtype=wl.torch_dtype, device="cuda")
+        layer.forward(inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out)
+        torch.cuda.synchronize()
+        assert moe.moe_device_status(layer.ws) == 0
+        outs.append(out)
+        del layer
+    assert torch.equal(outs[0], ref)
+    assert torch.equal(outs[1], ref)
