@@ -133,9 +133,14 @@ cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
     int smem_keys = c.T < kClipMaxSmemKeys ? c.T : kClipMaxSmemKeys;
     if (smem_keys < 1) smem_keys = 1;
     const size_t smem = sizeof(uint64_t) * (size_t)smem_keys;
-    cudaError_t err = cudaFuncSetAttribute(clip_select_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
+    static size_t configured = 48 * 1024;
+    if (smem > configured) {
+        err = cudaFuncSetAttribute(clip_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem);
+        if (err != cudaSuccess) return err;
+        configured = smem;
+    }
     clip_select_kernel<<<c.E, kClipThreads, smem, s>>>(c.T, c.E, c.k, c.capacity, smem_keys,
                                                        topk_idx, topk_w, counts, kept_counts, thr);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;

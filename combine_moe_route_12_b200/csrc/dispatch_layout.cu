@@ -18,8 +18,9 @@
 //                   look-back (Merrill & Garland 2016), one expert per thread.
 //                   The row of (t, j) is expert_offsets[e] + (rows of e in
 //                   earlier tiles) + (rank of t among this tile's rows of e).
-//   layout_splits   one CTA per destination rank counts its rows by source
-//                   rank, giving the EP x EP all_to_all_single split matrix.
+//                   While scattering, each tile also counts its rows by
+//                   (source rank, destination rank): the EP x EP
+//                   all_to_all_single split matrix.
 //
 // The look-back waits are bounded: on a timeout the tile raises
 // MOE_DEV_WAIT_TIMEOUT, publishes what it has so that later tiles finish,
@@ -36,10 +37,13 @@ constexpr uint32_t kFlagInclusive = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1;
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(
-    int tb, int tc, int k, int E, const int32_t *__restrict__ topk_idx,
-    const uint8_t *__restrict__ keep, int32_t *__restrict__ chunk_counts) {
+    int tb, int tc, int k, int E, int ep, const int32_t *__restrict__ topk_idx,
+    const uint8_t *__restrict__ keep, int32_t *__restrict__ chunk_counts,
+    int32_t *__restrict__ send_splits) {
     extern __shared__ int32_t s_hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    if (blockIdx.x == 0)   // the scatter kernel accumulates the split matrix into zeros
+        for (int i = threadIdx.x; i < ep * ep; i += blockDim.x) send_splits[i] = 0;
     __syncthreads();
     const size_t a0 = (size_t)tb * k, a1 = (size_t)(tb + tc) * k;
     for (size_t a = a0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; a < a1;
@@ -92,24 +96,72 @@ __device__ int block_exclusive_scan(int32_t *s, int n, int32_t *s_warp_tot) {
     return total;
 }
 
+// The split matrix is accumulated in shared memory when it fits.
+constexpr int kSplitSmemMax = 4096;
+constexpr int kLookbackWindow = 8;
+
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Exclusive prefix of expert e over the tiles before `tile`, by decoupled
+// look-back: descriptors pack a 2-bit flag (aggregate / inclusive prefix) and a
+// 30-bit count in one word, so relaxed loads of the word are enough.  Loads run
+// kLookbackWindow predecessors at a time.  Returns false if a predecessor never
+// published within the wait limit.
+__device__ __forceinline__ bool lookback_prefix(const uint32_t *tile_state, int tile, int E, int e,
+                                                uint32_t &excl) {
+    excl = 0;
+    int p = tile - 1;
+    while (p >= 0) {
+        const int n = min(kLookbackWindow, p + 1);
+        uint32_t v[kLookbackWindow];
+#pragma unroll
+        for (int i = 0; i < kLookbackWindow; ++i)
+            if (i < n) v[i] = ld_relaxed_u32(tile_state + (size_t)(p - i) * E + e);
+#pragma unroll
+        for (int i = 0; i < kLookbackWindow; ++i) {
+            if (i >= n) break;
+            uint32_t w = v[i];
+            if ((w >> 30) == 0) {
+                const uint32_t *q = tile_state + (size_t)(p - i) * E + e;
+                const uint64_t t0 = global_timer_ns();
+                while (((w = ld_relaxed_u32(q)) >> 30) == 0)
+                    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+            }
+            excl += w & kValueMask;
+            if ((w & ~kValueMask) == kFlagInclusive) return true;
+        }
+        p -= n;
+    }
+    return true;
+}
+
 __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     int tb, int tc, int k, int E, int ep, int64_t n_rows_max,
     const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ keep,
     const int32_t *__restrict__ chunk_counts, uint32_t *__restrict__ ticket,
     uint32_t *__restrict__ tile_state, int32_t *__restrict__ expert_offsets,
     int32_t *__restrict__ rank_offsets, int32_t *__restrict__ recv_token,
-    int32_t *__restrict__ recv_slot, int32_t *__restrict__ pos, uint32_t *__restrict__ status) {
+    int32_t *__restrict__ recv_slot, int32_t *__restrict__ pos, int32_t *__restrict__ send_splits,
+    uint32_t *__restrict__ status) {
     extern __shared__ int32_t s_dyn[];
     int32_t *s_eoff = s_dyn;                                 // [E + 1]
     int32_t *s_base = s_eoff + (E + 1);                      // [E]
     int32_t *s_cnt = s_base + E;                             // [kLayoutWarps][E]
     int32_t *s_rank = s_cnt + kLayoutWarps * E;              // [kLayoutTileTokens * k]
+    int32_t *s_split = s_rank + kLayoutTileTokens * k;       // [ep * ep] when it fits
     __shared__ int32_t s_warp_tot[33];
     __shared__ uint32_t s_tile;
+    const bool split_in_smem = ep * ep <= kSplitSmemMax;
 
     if (threadIdx.x == 0) s_tile = atomicAdd(ticket, 1u);
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_eoff[e] = chunk_counts[e];
     for (int i = threadIdx.x; i < kLayoutWarps * E; i += blockDim.x) s_cnt[i] = 0;
+    if (split_in_smem)
+        for (int i = threadIdx.x; i < ep * ep; i += blockDim.x) s_split[i] = 0;
     __syncthreads();
     const int tile = (int)s_tile;
     const int total = block_exclusive_scan(s_eoff, E, s_warp_tot);
@@ -164,21 +216,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
             st_release_u32(my, kFlagInclusive | agg);
         } else {
             st_release_u32(my, kFlagAggregate | agg);
-            for (int p = tile - 1; p >= 0; --p) {
-                const uint32_t *q = tile_state + (size_t)p * E + e;
-                uint32_t v = ld_acquire_u32(q);
-                if ((v >> 30) == 0) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (((v = ld_acquire_u32(q)) >> 30) == 0)
-                        if (global_timer_ns() - t0 > kWaitLimitNs) break;
-                }
-                if ((v >> 30) == 0) {                 // gave up: predecessor never published
-                    raise_status(status, MOE_DEV_WAIT_TIMEOUT);
-                    excl = 0x3FFFFFFFu;               // forces every write of this expert out of range
-                    break;
-                }
-                excl += v & kValueMask;
-                if ((v & ~kValueMask) == kFlagInclusive) break;
+            if (!lookback_prefix(tile_state, tile, E, e, excl)) {
+                raise_status(status, MOE_DEV_WAIT_TIMEOUT);
+                excl = 0x3FFFFFFFu;  // forces every write of this expert out of range
             }
             st_release_u32(my, kFlagInclusive | ((excl + agg) & kValueMask));
         }
@@ -186,13 +226,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     }
     __syncthreads();
 
-    // 3) scatter rows: recv_token / recv_slot / pos
+    // 3) scatter rows (recv_token / recv_slot / pos) and count the split matrix
     const int nt = min(kLayoutTileTokens, tb + tc - t_tile0);
+    const int tpr = tc / ep, epr = E / ep;
     for (int i = threadIdx.x; i < nt * k; i += blockDim.x) {
         const int ti = i / k, j = i % k;
         const int t = t_tile0 + ti;
         const size_t a = (size_t)t * k + j;
         int p = -1;
+        int key = -1;
         if (keep[a]) {
             const int e = topk_idx[a];
             if (e >= 0 && e < E) {
@@ -202,38 +244,32 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
                     p = (int)row;
                     recv_token[p] = t;
                     recv_slot[p] = j;
+                    key = ((t - tb) / tpr) * ep + e / epr;
                 } else {
                     bad = true;
                 }
             }
         }
         pos[(size_t)(t - tb) * k + j] = p;
+        const unsigned active = __activemask();
+        const unsigned peers = __match_any_sync(active, key);
+        if (key >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) {
+            if (split_in_smem) atomicAdd(&s_split[key], __popc(peers));
+            else atomicAdd(&send_splits[key], __popc(peers));
+        }
+    }
+    if (split_in_smem) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < ep * ep; i += blockDim.x)
+            if (s_split[i]) atomicAdd(&send_splits[i], s_split[i]);
     }
     if (bad) raise_status(status, MOE_DEV_BAD_INDEX);
 }
 
-__global__ void __launch_bounds__(kLayoutThreads) layout_splits_kernel(
-    int tb, int tc, int ep, const int32_t *__restrict__ rank_offsets,
-    const int32_t *__restrict__ recv_token, int32_t *__restrict__ send_splits) {
-    extern __shared__ int32_t s_src[];  // [ep]
-    const int d = blockIdx.x;
-    for (int s = threadIdx.x; s < ep; s += blockDim.x) s_src[s] = 0;
-    __syncthreads();
-    const int tpr = tc / ep;
-    const int p0 = rank_offsets[d], p1 = rank_offsets[d + 1];
-    for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
-        const int s = (recv_token[p] - tb) / tpr;
-        const unsigned active = __activemask();
-        const unsigned peers = __match_any_sync(active, s);
-        if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_src[s], __popc(peers));
-    }
-    __syncthreads();
-    for (int s = threadIdx.x; s < ep; s += blockDim.x) send_splits[(size_t)s * ep + d] = s_src[s];
-}
-
 size_t layout_scatter_smem(const moe_config &c) {
+    const size_t split = (size_t)c.ep * c.ep <= (size_t)kSplitSmemMax ? (size_t)c.ep * c.ep : 0;
     return sizeof(int32_t) * ((size_t)(c.E + 1) + c.E + (size_t)kLayoutWarps * c.E +
-                              (size_t)kLayoutTileTokens * c.k);
+                              (size_t)kLayoutTileTokens * c.k + split);
 }
 
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
@@ -258,20 +294,21 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
         if (err == cudaSuccess) err = cudaMemsetAsync(send_splits, 0, sizeof(int32_t) * (size_t)c.ep * c.ep, s);
     } else {
         int hb = (int)(((size_t)tc * c.k + kLayoutThreads - 1) / kLayoutThreads);
-        if (hb > num_sms * 4) hb = num_sms * 4;
+        if (hb > num_sms * 2) hb = num_sms * 2;
         layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, s>>>(
-            tb, tc, c.k, c.E, topk_idx, keep, chunk_counts);
+            tb, tc, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         const size_t smem = layout_scatter_smem(c);
-        err = cudaFuncSetAttribute(layout_scatter_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
+        static size_t configured = 48 * 1024;
+        if (smem > configured) {
+            err = cudaFuncSetAttribute(layout_scatter_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return err;
+            configured = smem;
+        }
         layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, s>>>(
             tb, tc, c.k, c.E, c.ep, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
-            expert_offsets, rank_offsets, recv_token, recv_slot, pos, status);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
-        layout_splits_kernel<<<c.ep, kLayoutThreads, sizeof(int32_t) * c.ep, s>>>(
-            tb, tc, c.ep, rank_offsets, recv_token, send_splits);
+            expert_offsets, rank_offsets, recv_token, recv_slot, pos, send_splits, status);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     if (err != cudaSuccess) return err;

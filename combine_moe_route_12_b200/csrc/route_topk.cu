@@ -125,7 +125,7 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     if (err != cudaSuccess || c.T == 0) return err;
     const int warps_per_block = 8;
     int blocks = (c.T + warps_per_block - 1) / warps_per_block;
-    const int cap = num_sms * 8;
+    const int cap = num_sms * 2;   // few CTAs: one global atomic per CTA and expert
     if (blocks > cap) blocks = cap;
     const size_t smem = sizeof(int32_t) * (size_t)c.E;
     const int vpl = (c.E + 31) / 32;
