@@ -2,47 +2,57 @@
 // rows (LightLLM PR 1687: contiguous "psum" grouped GEMM, silu_and_mul, second
 // grouped GEMM; decode reduces w*y straight into a dense output).
 //
-// Two launches of one persistent, warp-specialised tcgen05 kernel:
+// Two launches of one persistent, warp-specialised tcgen05 kernel that runs on
+// CTA pairs (clusters of 2, cta_group::2 MMA with M = 256):
 //   GEMM1  gate|up = W13[e] . xr^T, epilogue h = silu(gate) * up (bf16)
 //   GEMM2  y = W2[e] . h^T (bf16), or in decode form
 //          out_reduce[t] += w * y in fp32.
 //
 // Operands are swapped relative to the row-major product: the weights are the
-// 128-row MMA operand (A) and the expert's tokens are the N operand (B), so a
-// tile is (expert, 128 output features, up to 128 / 256 tokens) and the
-// token count is only rounded up to the MMA's N granularity of 16.  A ragged
-// expert segment of M_e rows wastes < 16 rows instead of up to 127.  In
-// GEMM1 the gate rows and the up rows of the same 128 features are two MMAs
-// into two TMEM accumulators, so TMEM lane i holds gate_i and up_i of every
-// token and the SwiGLU is lane-local.
+// M operand and the expert's tokens are the N operand, so a pair tile is
+// (expert, 256 weight rows, up to 256 tokens) and the token count is only
+// rounded up to the MMA's N granularity of 16: a ragged expert segment wastes
+// < 16 rows instead of up to 127, and each weight tile meets all (up to 256)
+// tokens of its expert while it sits in shared memory.  The pair's MMA keeps
+// 128 weight rows and half the tokens in each CTA's shared memory, which
+// halves the operand bytes each SM's shared memory must deliver per MMA;
+// with one CTA per MMA the shared memory (tile fills plus operand reads), not
+// the tensor pipe, bounds the main loop.
 //
-// CTA = 6 warps.  Warp 4 (one lane) streams weight and token tiles with TMA
-// into a 4-stage ring of 128B-swizzled shared-memory buffers; warp 5 (one
-// lane) issues tcgen05.mma (M=128, N=16..256, K=16, bf16 -> fp32) into one of
-// two TMEM accumulator buffers, so the epilogue of tile i overlaps the main
-// loop of tile i+1; warps 0-3 drain TMEM (warp q owns features 32q..32q+31 of
-// the tile) and write h / y one token row at a time (each warp store covers
-// 32 consecutive features).  Tiles run expert by expert, feature block by
-// feature block, token block innermost, so the CTAs that share a weight slice
-// run together and read it from DRAM once.
+// In GEMM1 a CTA's 128 weight rows are the gate rows of 64 features followed
+// by the up rows of the same 64 features, so TMEM lanes i and 64+i hold gate_i
+// and up_i; the two epilogue warps that own them swap half their columns
+// through shared memory and each finishes h for half the tokens.
+//
+// CTA = 6 warps.  Warp 4 (one lane) of each CTA streams its weight and token
+// tiles with TMA into a 6-stage ring of 128B-swizzled buffers, counting the
+// bytes on the leader CTA's mbarrier; warp 5 (one lane) of the leader issues
+// the pair's tcgen05.mma (bf16 -> fp32) into one of two TMEM accumulator
+// buffers and commits to both CTAs' barriers, so the epilogue of tile i
+// overlaps the main loop of tile i+1; warps 0-3 of each CTA drain its TMEM
+// (warp q owns lanes 32q..32q+31) and write h / y one token row at a time.
+// Tiles run expert by expert, weight block by weight block, token block
+// innermost.
 //
 // Every mbarrier wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT,
 // stops the other roles, lets in-flight copies and MMAs land, frees TMEM and
-// returns.
+// returns.  No TMA load uses cluster multicast.
 #include <cudaTypedefs.h>
 
 #include "moe_common.cuh"
 
 namespace moe {
 
-constexpr int kBK = 64, kStages = 4;
-constexpr int kFeat = 128;                           // weight rows (output features) per tile
+constexpr int kBK = 64, kStages = 6;
+constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
 constexpr int kTokRows = 32;                         // rows per token TMA box
+constexpr int kTokBlock = 256;                       // tokens per pair tile (MMA N <= 256)
 constexpr int kFfnThreads = 192;
-constexpr uint32_t kWBytes = kFeat * kBK * 2;        // 16 KiB: one 128-row weight box
+constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;  // 16 KiB of weights per stage and CTA
 constexpr uint32_t kTokBoxBytes = kTokRows * kBK * 2;  // 4 KiB
-constexpr uint32_t kStageBytes = 48 * 1024;
+constexpr uint32_t kStageBytes = kWBytes + (kTokBlock / 2) * kBK * 2;  // 32 KiB per CTA
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
+constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (2 pairs x 2 buffers x 2 ways)
 
 enum EpiMode : int { kEpiSwiGLU = 0, kEpiStore = 1, kEpiReduce = 2 };
 
@@ -50,10 +60,11 @@ struct FfnGemmParams {
     const int32_t *expert_offsets;
     int E;
     int K;                 // reduction length (H for GEMM1, I for GEMM2)
-    int n_fblocks;         // 128-feature blocks per expert (I/128 or H/128, rounded up)
+    int n_fblocks;         // pair feature blocks per expert: I/128 (GEMM1) or H/256 (GEMM2), rounded up
+    int feat_per_cta;      // output features per CTA of a pair tile: 64 (GEMM1) or 128 (GEMM2)
     int w_rows_per_expert; // 2I for GEMM1, H for GEMM2
     int up_offset;         // GEMM1: rows from a gate row to its up row (I)
-    int tok_block;         // tokens per tile: 128 (GEMM1) or 256 (GEMM2)
+    int tok_block;         // tokens per tile (256)
     int out_cols;          // row length of the output (I for h, H for y / out_reduce)
     void *out;             // h or y
     float *out_reduce;
@@ -71,6 +82,7 @@ struct FfnSmem {
     uint64_t tmem_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
+    int go_flag[2];        // GEMM1: per warp pair, did the gate warp's accumulator wait succeed
     int abort_flag;
     int total_tiles;
 };
@@ -102,23 +114,28 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int32_t *s_tpre,
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const FfnGemmParams P) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
-    // weight boxes at the start of a stage (gate + up for GEMM1), token rows after
-    constexpr uint32_t kTokOff = kSwiGLU ? 2 * kWBytes : kWBytes;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    // 1024-byte alignment for the swizzled tiles
+    // 1024-byte alignment for the swizzled tiles (same offsets in both CTAs of the pair)
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *tiles = base;
-    FfnSmem *S = reinterpret_cast<FfnSmem *>(base + kStages * kStageBytes);
+    unsigned char *tiles = base;                              // [kStages][weights | tokens]
+    float *xchg = reinterpret_cast<float *>(base + kStages * kStageBytes);   // GEMM1 only
+    FfnSmem *S = reinterpret_cast<FfnSmem *>(base + kStages * kStageBytes + (kSwiGLU ? kXchgBytes : 0));
     int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);   // [E + 1] tile prefix
     int32_t *s_tb = s_tpre + (P.E + 1);                       // [E] token blocks per expert
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();                  // 0: leader (issues the MMA)
+    const int pair = (int)cluster_id_x(), npairs = (int)ncluster_x();
 
     // --- tile table (every CTA builds the same one from the expert offsets)
     if (warp == 0) {
@@ -145,15 +162,15 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&S->full[s], 1); mbar_init(&S->empty[s], 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(&S->tmem_full[a], 1); mbar_init(&S->tmem_empty[a], 4); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&S->tmem_full[a], 1); mbar_init(&S->tmem_empty[a], 8); }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 4 && lane == 0) { tma_prefetch_desc(&tmap_w); tma_prefetch_desc(&tmap_x); }
-    if (warp == 5) { tmem_alloc(&S->tmem_base, kTmemCols); tmem_relinquish(); }
+    if (warp == 5) { tmem_alloc_pair(&S->tmem_base, kTmemCols); tmem_relinquish_pair(); }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();      // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
 
     const int total = S->total_tiles;
@@ -162,27 +179,37 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     volatile int *abort_flag = &S->abort_flag;
 
     if (warp == 4) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < total && ok; tile += npairs) {
                 const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
-                const int w_row = ti.e * P.w_rows_per_expert + ti.f_blk * kFeat;
-                const int n_box = (ti.n_mma + kTokRows - 1) / kTokRows;
-                const uint32_t bytes = (kSwiGLU ? 2 : 1) * kWBytes + n_box * kTokBoxBytes;
+                // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows, GEMM2 128 rows
+                const int w_row = ti.e * P.w_rows_per_expert +
+                                  (ti.f_blk * 2 + (int)rank) * P.feat_per_cta;
+                // this CTA's half of the token rows
+                const int half = ti.n_mma / 2;
+                const int tok_row = ti.p0 + (int)rank * half;
+                const int n_box = (half + kTokRows - 1) / kTokRows;
+                const uint32_t bytes = kWBytes + n_box * kTokBoxBytes;
                 for (int kb = 0; kb < num_k; ++kb) {
                     if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     unsigned char *st = tiles + stage * kStageBytes;
+                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
                     const int kx = kb * kBK;
-                    mbar_arrive_expect_tx(&S->full[stage], bytes);
-                    tma_load_2d(st, &tmap_w, &S->full[stage], kx, w_row);
-                    if (kSwiGLU) tma_load_2d(st + kWBytes, &tmap_w, &S->full[stage], kx, w_row + P.up_offset);
+                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * bytes);
+                    if (kSwiGLU) {
+                        tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
+                        tma_load_2d_pair(st + kWBytes / 2, &tmap_w, full_leader, kx, w_row + P.up_offset);
+                    } else {
+                        tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
+                    }
                     for (int b = 0; b < n_box; ++b)
-                        tma_load_2d(st + kTokOff + b * kTokBoxBytes, &tmap_x, &S->full[stage], kx,
-                                    ti.p0 + b * kTokRows);
+                        tma_load_2d_pair(st + kWBytes + b * kTokBoxBytes, &tmap_x, full_leader, kx,
+                                         tok_row + b * kTokRows);
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -191,94 +218,124 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
                 raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
             }
-            // let the last copies land before the CTA can exit
-            volatile int never = 0;
-            const long long last = issued < kStages ? issued : kStages;
-            int st = stage;
-            uint32_t ph = phase;
-            for (long long i = 0; i < last; ++i) {
-                if (--st < 0) { st = kStages - 1; ph ^= 1u; }
-                mbar_wait_bounded(&S->full[st], ph, &never);
+            // the leader's full barriers count both CTAs' bytes: let the last copies land
+            if (rank == 0) {
+                volatile int never = 0;
+                const long long last = issued < kStages ? issued : kStages;
+                int st = stage;
+                uint32_t ph = phase;
+                for (long long i = 0; i < last; ++i) {
+                    if (--st < 0) { st = kStages - 1; ph ^= 1u; }
+                    mbar_wait_bounded(&S->full[st], ph, &never);
+                }
             }
         }
     } else if (warp == 5) {
-        // ------------------------------------------------ MMA issuer
+        // ------------------------------------------------ MMA issuer (leader CTA)
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
-                const uint32_t idesc = make_idesc_bf16_f32(kFeat, ti.n_mma);
-                if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d0 = tmem_base + (uint32_t)(acc * 256);
-                for (int kb = 0; kb < num_k; ++kb) {
-                    if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+            if (rank == 0) {
+                int stage = 0;
+                uint32_t phase = 0;
+                int acc = 0;
+                uint32_t acc_phase = 0;
+                bool ok = true;
+                for (int tile = pair; tile < total && ok; tile += npairs) {
+                    const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
+                    const uint32_t idesc = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
+                    if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t st = smem_u32(tiles + stage * kStageBytes);
+                    const uint32_t d0 = tmem_base + (uint32_t)(acc * kTokBlock);
+                    for (int kb = 0; kb < num_k; ++kb) {
+                        if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t st = smem_u32(tiles + stage * kStageBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint32_t acc_in = (kb > 0 || kk > 0) ? 1u : 0u;
-                        const uint64_t xdesc = make_sw128_desc(st + kTokOff + kk * 32);
-                        tc_mma_f16(d0, make_sw128_desc(st + kk * 32), xdesc, idesc, acc_in);
-                        if (kSwiGLU)
-                            tc_mma_f16(d0 + 128, make_sw128_desc(st + kWBytes + kk * 32), xdesc, idesc, acc_in);
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            tc_mma_f16_pair(d0, make_sw128_desc(st + kk * 32),
+                                            make_sw128_desc(st + kWBytes + kk * 32), idesc,
+                                            (kb > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     }
-                    tc_commit(&S->empty[stage]);   // frees the stage once these MMAs finish
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (!ok) break;
+                    tc_commit_pair_mc(&S->tmem_full[acc], 0x3);    // accumulators ready in both CTAs
+                    if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
                 }
-                if (!ok) break;
-                tc_commit(&S->tmem_full[acc]);     // accumulator ready for the epilogue
-                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-            }
-            if (!ok) {
-                raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
-                *abort_flag = 1;
+                if (!ok) {
+                    raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                tc_commit_pair_mc(&S->mma_done, 0x3);
             }
             // every MMA issued so far must finish before TMEM is released
             volatile int never = 0;
-            tc_commit(&S->mma_done);
             mbar_wait_bounded(&S->mma_done, 0, &never);
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 0-3)
-        const int q = warp;  // TMEM lanes 32q .. 32q+31 = features 32q .. 32q+31 of the tile
+        // ------------------------------------------------ epilogue (warps 0-3 of both CTAs)
+        const int q = warp;  // TMEM lanes 32q .. 32q+31
+        // GEMM1: warp q < 2 holds gate, warp q + 2 the up rows of the same 32 features;
+        // GEMM2: warp q holds output features 32q .. 32q+31 of this CTA's 128
+        const int feat_lane = kSwiGLU ? (q & 1) * 32 + lane : q * 32 + lane;
+        const bool is_gate = q < 2;
+        const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
+                                          mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            if (!mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag)) {
+        int xbuf = 0;
+        for (int tile = pair; tile < total; tile += npairs) {
+            bool go;
+            if (kSwiGLU) {
+                // the gate warp waits (bounded) and tells its up partner; both then
+                // pass the same exchange barriers or both leave
+                if (is_gate) {
+                    go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
+                    if (lane == 0) S->go_flag[q & 1] = go ? 1 : 0;
+                }
+                named_barrier_sync(1 + (q & 1), 64);
+                if (!is_gate) go = S->go_flag[q & 1] != 0;
+            } else {
+                go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
+            }
+            if (!go) {
                 if (lane == 0) { raise_status(P.status, MOE_DEV_WAIT_TIMEOUT); *abort_flag = 1; }
                 break;
             }
             tc_fence_after();
             const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
-            const int f = ti.f_blk * kFeat + q * 32 + lane;       // this thread's output feature
+            const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
             const bool f_ok = f < P.out_cols;
-            const uint32_t tbase = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
+            const uint32_t tbase = tmem_base + (uint32_t)(acc * kTokBlock) + ((uint32_t)(q * 32) << 16);
 
             for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
+                tc_wait_ld();
                 if (kSwiGLU) {
-                    uint32_t u[32];
-                    tmem_ld_32x32b_x32(tbase + 128 + c0, u);
-                    tc_wait_ld();
-                    __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
-                    const int nc = min(32, ti.n_valid - c0);
+                    // exchange: gate warps hand over tokens 16..31, up warps tokens 0..15
+                    float *mine = xchg + (((q & 1) * 2 + xbuf) * 2 + (is_gate ? 0 : 1)) * 512;
+                    float *theirs = xchg + (((q & 1) * 2 + xbuf) * 2 + (is_gate ? 1 : 0)) * 512;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]);
+                    named_barrier_sync(1 + (q & 1), 64);
+                    const int cbase = c0 + (is_gate ? 0 : 16);
+                    const int nc = min(16, ti.n_valid - cbase);
+                    __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) +
+                                       (size_t)(ti.p0 + cbase) * P.out_cols + f;
                     if (f_ok) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
+                        for (int j = 0; j < 16; ++j) {
                             if (j < nc) {
-                                const float hv = silu_f(__uint_as_float(r[j])) * __uint_as_float(u[j]);
-                                h[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(hv);
+                                const float own = __uint_as_float(r[is_gate ? j : 16 + j]);
+                                const float other = theirs[j * 32 + lane];
+                                const float g = is_gate ? own : other, u = is_gate ? other : own;
+                                h[(size_t)j * P.out_cols] = __float2bfloat16_rn(silu_f(g) * u);
                             }
                         }
                     }
+                    xbuf ^= 1;
                 } else if (MODE == kEpiStore) {
-                    tc_wait_ld();
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
                     const int nc = min(32, ti.n_valid - c0);
                     if (f_ok) {
@@ -287,7 +344,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
                             if (j < nc) y[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(__uint_as_float(r[j]));
                     }
                 } else {  // kEpiReduce: out_reduce[t] += w * y, one token column at a time
-                    tc_wait_ld();
                     int my_t = 0;
                     float my_w = 0.0f;
                     const int nc = min(32, ti.n_valid - c0);
@@ -307,16 +363,16 @@ __global__ void __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S->tmem_empty[acc]);
+            if (lane == 0) mbar_arrive_cluster(empty_leader[acc]);   // release the pair's accumulator
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();      // both CTAs done: no MMA, copy or remote arrive in flight
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
@@ -351,14 +407,15 @@ static bool make_tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t rows, uint6
     return r == CUDA_SUCCESS;
 }
 
-size_t ffn_tcgen05_smem(int E) {
-    return 1024 + (size_t)kStages * kStageBytes + sizeof(FfnSmem) + sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
+size_t ffn_tcgen05_smem(int E, bool swiglu) {
+    return 1024 + (size_t)kStages * kStageBytes + (swiglu ? kXchgBytes : 0) + sizeof(FfnSmem) +
+           sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
 template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
                                const FfnGemmParams &P, int grid, cudaStream_t s) {
-    const size_t smem = ffn_tcgen05_smem(P.E);
+    const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
     if (smem > configured) {
         cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE>,
@@ -378,9 +435,9 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
                                uint32_t *status, cudaStream_t s, int num_sms) {
     if (n_rows <= 0) return cudaSuccess;
     CUtensorMap tw1, tx1, tw2, tx2;
-    if (!make_tmap_bf16(&tw1, w13, (uint64_t)c.E * 2 * c.I, (uint64_t)c.H, kFeat) ||
+    if (!make_tmap_bf16(&tw1, w13, (uint64_t)c.E * 2 * c.I, (uint64_t)c.H, kRowsPerCta / 2) ||
         !make_tmap_bf16(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTokRows) ||
-        !make_tmap_bf16(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kFeat) ||
+        !make_tmap_bf16(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
         !make_tmap_bf16(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTokRows))
         return cudaErrorNotSupported;
 
@@ -388,26 +445,29 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P1.expert_offsets = expert_offsets;
     P1.E = c.E;
     P1.K = c.H;
-    P1.n_fblocks = (c.I + kFeat - 1) / kFeat;
+    P1.feat_per_cta = kRowsPerCta / 2;
+    P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
     P1.w_rows_per_expert = 2 * c.I;
     P1.up_offset = c.I;
-    P1.tok_block = 128;
+    P1.tok_block = kTokBlock;
     P1.out_cols = c.I;
     P1.out = h;
     P1.k = c.k;
     P1.status = status;
-    // an upper bound on the tiles: sum_e ceil(M_e / tok) <= n_rows / tok + E
+    // CTA pairs: an upper bound on the pair tiles is (n_rows / tok + E) * n_fblocks
+    const long long max_pairs = num_sms / 2;
     long long g1 = (n_rows / P1.tok_block + c.E) * (long long)P1.n_fblocks;
-    int grid1 = (int)(g1 < num_sms ? g1 : num_sms);
+    int grid1 = 2 * (int)(g1 < max_pairs ? g1 : max_pairs);
     cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, P1, grid1, s);
     if (err != cudaSuccess) return err;
 
     FfnGemmParams P2 = P1;
     P2.K = c.I;
-    P2.n_fblocks = (c.H + kFeat - 1) / kFeat;
+    P2.feat_per_cta = kRowsPerCta;
+    P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
     P2.w_rows_per_expert = c.H;
     P2.up_offset = 0;
-    P2.tok_block = 256;
+    P2.tok_block = kTokBlock;
     P2.out_cols = c.H;
     P2.out = y;
     P2.out_reduce = out_reduce;
@@ -415,7 +475,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P2.recv_slot = recv_slot;
     P2.topk_w = topk_w;
     long long g2 = (n_rows / P2.tok_block + c.E) * (long long)P2.n_fblocks;
-    int grid2 = (int)(g2 < num_sms ? g2 : num_sms);
+    int grid2 = 2 * (int)(g2 < max_pairs ? g2 : max_pairs);
     if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, P2, grid2, s);
     return launch_gemm<kEpiStore>(tw2, tx2, P2, grid2, s);
 }
