@@ -71,6 +71,20 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one).
+    NCCL needs a CUDA tensor; gloo (used by the CPU tests) a CPU one."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -433,11 +447,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     if moe.moe_device_status(layer.ws) != 0:
         raise RuntimeError("device status bits set during the timed region")
 
@@ -490,10 +500,7 @@ def run_ours(args):
             b.synchronize()
             if i >= args.warmup:
                 e2e_ms += a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
         h2d = h_logits.numel() * 4 + h_x.numel() * h_x.element_size() + (0 if h_bias is None else h_bias.numel() * 4)
         d2h = h_out.numel() * h_out.element_size()
         e2e = {"value": world * wl.T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
