@@ -25,6 +25,8 @@
 // The look-back waits are bounded: on a timeout the tile raises
 // MOE_DEV_WAIT_TIMEOUT, publishes what it has so that later tiles finish,
 // and skips every write that would leave the receive buffers.
+#include <mutex>
+
 #include "moe_common.cuh"
 
 namespace moe {
@@ -323,3 +325,123 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of moe_dispatch_layout.
+//
+// Some callers cannot call cudaMalloc or hand the library a workspace: code
+// that runs while another framework is capturing the stream into a CUDA graph
+// (an allocation there would break or be left out of the capture), code whose
+// device memory all belongs to an allocator it does not control (a
+// pre-reserved pool it may not grow), and latency-critical loops that must not
+// hit the implicit device synchronisation of cudaMalloc / cudaFree.  For them
+// this entry point keeps the dispatch layout's scratch (the tile ticket, the
+// chunk's per-expert counts and the look-back descriptors) in one fixed
+// device array inside the library instead of a caller workspace.
+//
+// Limits: at most kNoAllocMaxTiles * 256 tokens per call and E <= 1024.  The
+// array (about 261 KiB) exists on every device that loads the library, until
+// the process exits.  Every call shares it: calls that may overlap on the GPU
+// (different streams without ordering, or several host threads) race and
+// corrupt each other's layouts; order them.  The first call on a device looks
+// up the array's device address (cudaGetSymbolAddress) with that device
+// current; make that first call before any stream capture.
+namespace {
+
+constexpr int kNoAllocMaxTiles = 64;   // 16384 tokens per call
+constexpr size_t kNoAllocTicket = 0;
+constexpr size_t kNoAllocStatus = 256;
+constexpr size_t kNoAllocCounts = 512;
+constexpr size_t kNoAllocTiles = kNoAllocCounts + sizeof(int32_t) * moe::kMaxExperts;
+constexpr size_t kNoAllocBytes = kNoAllocTiles + sizeof(uint32_t) * (size_t)kNoAllocMaxTiles * moe::kMaxExperts;
+
+static __device__ __align__(256) unsigned char g_noalloc_layout_scratch[kNoAllocBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_base[kNoAllocMaxDevices] = {};
+
+// Device address of the array for the current device (looked up once per device).
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_base[dev]) {
+        void *p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_noalloc_layout_scratch);
+        if (err != cudaSuccess) return err;
+        g_noalloc_base[dev] = p;
+    }
+    *out = g_noalloc_base[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+namespace moe {
+moe_status report_error(moe_status st, const char *msg);
+int64_t max_recv_rows_of(const moe_config &c, int32_t tok_count);
+}
+
+extern "C" moe_status moe_dispatch_layout_noalloc(
+    const moe_config *cfg, int32_t tok_begin, int32_t tok_count, const int32_t *topk_idx,
+    const uint8_t *keep, int32_t *expert_offsets, int32_t *rank_offsets, int32_t *recv_token,
+    int32_t *recv_slot, int32_t *pos, int32_t *send_splits, int32_t *splits_host,
+    uint32_t *status, cudaStream_t stream) {
+    using namespace moe;
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (tok_begin < 0 || tok_count < 0 || (int64_t)tok_begin + tok_count > c.T || tok_count % c.ep != 0)
+        return report_error(MOE_ERR_INVALID_ARG, "token range outside [0, T) or not divisible by ep");
+    const int n_tiles = (tok_count + kLayoutTileTokens - 1) / kLayoutTileTokens;
+    if (n_tiles > kNoAllocMaxTiles)
+        return report_error(MOE_ERR_UNSUPPORTED,
+                            "moe_dispatch_layout_noalloc handles at most 16384 tokens per call");
+    if (!expert_offsets || !rank_offsets || !send_splits ||
+        (tok_count > 0 && (!topk_idx || !keep || !recv_token || !recv_slot || !pos)))
+        return report_error(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    void *base = nullptr;
+    cudaError_t err = noalloc_scratch(&base);
+    if (err != cudaSuccess) return report_error(MOE_ERR_CUDA, cudaGetErrorString(err));
+    unsigned char *b = static_cast<unsigned char *>(base);
+    uint32_t *ticket = reinterpret_cast<uint32_t *>(b + kNoAllocTicket);
+    uint32_t *st_word = status ? status : reinterpret_cast<uint32_t *>(b + kNoAllocStatus);
+    int32_t *chunk_counts = reinterpret_cast<int32_t *>(b + kNoAllocCounts);
+    uint32_t *tile_state = reinterpret_cast<uint32_t *>(b + kNoAllocTiles);
+    const int num_sms = [] { int d = 0, n = 148; cudaGetDevice(&d); cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d); return n; }();
+    // the previous call's ticket, counts and look-back descriptors start again at zero
+    err = cudaMemsetAsync(b, 0, kNoAllocTiles + sizeof(uint32_t) * (size_t)n_tiles * c.E, stream);
+    if (err == cudaSuccess && tok_count == 0) {
+        err = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (size_t)(c.E + 1), stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(rank_offsets, 0, sizeof(int32_t) * (size_t)(c.ep + 1), stream);
+        if (err == cudaSuccess) err = cudaMemsetAsync(send_splits, 0, sizeof(int32_t) * (size_t)c.ep * c.ep, stream);
+    } else if (err == cudaSuccess) {
+        int hb = (int)(((size_t)tok_count * c.k + kLayoutThreads - 1) / kLayoutThreads);
+        if (hb > num_sms * 2) hb = num_sms * 2;
+        layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, stream>>>(
+            tok_begin, tok_count, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
+        err = cudaGetLastError();
+        const size_t smem = layout_scatter_smem(c);
+        if (err == cudaSuccess && smem > 48 * 1024)
+            err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err == cudaSuccess) {
+            layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, stream>>>(
+                tok_begin, tok_count, c.k, c.E, c.ep, max_recv_rows_of(c, tok_count), topk_idx, keep,
+                chunk_counts, ticket, tile_state, expert_offsets, rank_offsets, recv_token, recv_slot,
+                pos, send_splits, st_word);
+            err = cudaGetLastError();
+        }
+    }
+    if (err == cudaSuccess && splits_host) {
+        err = cudaMemcpyAsync(splits_host, expert_offsets, sizeof(int32_t) * (size_t)(c.E + 1),
+                              cudaMemcpyDeviceToHost, stream);
+        if (err == cudaSuccess)
+            err = cudaMemcpyAsync(splits_host + c.E + 1, send_splits,
+                                  sizeof(int32_t) * (size_t)c.ep * c.ep, cudaMemcpyDeviceToHost, stream);
+    }
+    if (err != cudaSuccess) return report_error(MOE_ERR_CUDA, cudaGetErrorString(err));
+    return MOE_OK;
+}

@@ -155,6 +155,12 @@ cudaError_t get_events(int n, cudaEvent_t **out) {
 
 }  // namespace
 
+namespace moe {
+// Used by entry points defined in other translation units.
+moe_status report_error(moe_status st, const char *msg) { return fail(st, "%s", msg); }
+int64_t max_recv_rows_of(const moe_config &c, int32_t tok_count) { return max_rows(c, tok_count); }
+}  // namespace moe
+
 extern "C" {
 
 moe_status moe_config_check(const moe_config *cfg) {

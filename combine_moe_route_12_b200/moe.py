@@ -60,6 +60,7 @@ _decl("moe_max_recv_rows", ctypes.c_int64, _CFG, _I32)
 _decl("moe_route_topk", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_capacity_clip", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_dispatch_layout", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_dispatch_layout_noalloc", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
 _decl("moe_grouped_swiglu_ffn", _I32, _CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P)
@@ -159,6 +160,19 @@ def moe_dispatch_layout(cfg, tok_begin, tok_count, topk_idx, keep, expert_offset
                                     _ptr(recv_token), _ptr(recv_slot), _ptr(pos),
                                     _ptr(send_splits), _ptr(splits_host), _ptr(ws),
                                     _stream(stream)))
+
+
+def moe_dispatch_layout_noalloc(cfg, tok_begin, tok_count, topk_idx, keep, expert_offsets,
+                                rank_offsets, recv_token, recv_slot, pos, send_splits, splits_host,
+                                status=None, stream=None):
+    """moe_dispatch_layout without a workspace: for callers that cannot
+    allocate device memory (see include/moe_b200.h).  Its scratch is one
+    library-owned device array shared by every call, so calls must not overlap."""
+    _check(_lib.moe_dispatch_layout_noalloc(ctypes.byref(cfg), tok_begin, tok_count, _ptr(topk_idx),
+                                            _ptr(keep), _ptr(expert_offsets), _ptr(rank_offsets),
+                                            _ptr(recv_token), _ptr(recv_slot), _ptr(pos),
+                                            _ptr(send_splits), _ptr(splits_host), _ptr(status),
+                                            _stream(stream)))
 
 
 def moe_permute(cfg, x, pos, tok_begin, tok_count, xr, stream=None):

@@ -184,6 +184,30 @@ moe_status moe_dispatch_layout(const moe_config *cfg, int32_t tok_begin, int32_t
                                void *ws, cudaStream_t stream);
 
 /*
+ * Allocation-free form of moe_dispatch_layout, for callers that cannot call
+ * cudaMalloc or pass a workspace: code running while another framework
+ * captures the stream into a CUDA graph, code whose device memory belongs to
+ * an allocator it cannot grow, and latency-critical loops that must avoid the
+ * implicit synchronisation of cudaMalloc / cudaFree.  The pages describe no
+ * such variant: the paper has no counterpart of this entry point.
+ *   Arguments and outputs are those of moe_dispatch_layout, without ws.
+ *   status: device uint32 that receives the MOE_DEV_* bits (OR-ed in), or
+ *           NULL to drop them.
+ * The layout's scratch lives in one fixed device array inside the library
+ * (about 261 KiB per device, held until the process exits).  Limits:
+ * tok_count <= 16384 (MOE_ERR_UNSUPPORTED beyond).  All calls share the
+ * array: calls that may overlap on the GPU race and must be ordered.  The
+ * first call on a device looks up the array's address with that device
+ * current; make it before any stream capture.  Allocates nothing.
+ */
+moe_status moe_dispatch_layout_noalloc(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
+                                       const int32_t *topk_idx, const uint8_t *keep,
+                                       int32_t *expert_offsets, int32_t *rank_offsets,
+                                       int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                                       int32_t *send_splits, int32_t *splits_host,
+                                       uint32_t *status, cudaStream_t stream);
+
+/*
  * Step 4 - permute: xr[pos[i, j], :] = x[tok_begin + i, :] for every kept
  * (i, j).  x is [T, H]; xr is [N_max, H]; rows >= N are left untouched.
  */
