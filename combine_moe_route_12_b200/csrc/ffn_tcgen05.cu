@@ -24,12 +24,13 @@
 // and up_i; the two epilogue warps that own them swap half their columns
 // through shared memory and each finishes h for half the tokens.
 //
-// CTA = 6 warps.  Warp 4 (one lane) of each CTA streams its weight and token
+// CTA = 10 warps.  Warp 4 (one lane) of each CTA streams its weight and token
 // tiles with TMA into a 6-stage ring of 128B-swizzled buffers, counting the
 // bytes on the leader CTA's mbarrier; warp 5 (one lane) of the leader issues
 // the pair's tcgen05.mma (bf16 -> fp32) into one of two TMEM accumulator
 // buffers and commits to both CTAs' barriers, so the epilogue of tile i
-// overlaps the main loop of tile i+1; warps 0-3 of each CTA drain its TMEM
+// overlaps the main loop of tile i+1 (a tile with 257..512 tokens takes both
+// buffers: one pass over its weights feeds two MMAs); warps 0-3 of each CTA drain its TMEM
 // (warp q owns lanes 32q..32q+31) and write h / y one token row at a time.
 // Tiles run expert by expert, weight block by weight block, token block
 // innermost.
@@ -43,16 +44,28 @@
 
 namespace moe {
 
-constexpr int kBK = 64, kStages = 6;
+constexpr int kBK = 64;
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
 constexpr int kTokRows = 32;                         // rows per token TMA box
-constexpr int kTokBlock = 256;                       // tokens per pair tile (MMA N <= 256)
-constexpr int kFfnThreads = 192;
+constexpr int kSlotTok = 256;                        // tokens per accumulator slot (MMA N <= 256)
+constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
+constexpr int kProdWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
 constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;  // 16 KiB of weights per stage and CTA
 constexpr uint32_t kTokBoxBytes = kTokRows * kBK * 2;  // 4 KiB
-constexpr uint32_t kStageBytes = kWBytes + (kTokBlock / 2) * kBK * 2;  // 32 KiB per CTA
+constexpr uint32_t kSlotBytes = (kSlotTok / 2) * kBK * 2;  // 16 KiB of one slot's tokens per CTA
+constexpr uint32_t kRingBytes = 192 * 1024;
+// A tile meets up to kMaxSlots * 256 tokens of its expert in one pass over its
+// weights (one MMA per 256-token slot, each into its own TMEM buffer).  Two
+// slots keep an expert with 257..512 rows to a single weight pass; launches
+// whose chunks cannot exceed 256 rows per expert use one slot and a deeper ring.
+template <int kMaxSlots>
+struct RingCfg {
+    static constexpr uint32_t kStageBytes = kWBytes + kMaxSlots * kSlotBytes;  // 32 / 48 KiB
+    static constexpr int kStages = kRingBytes / kStageBytes;                   // 6 / 4
+};
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
-constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (2 pairs x 2 buffers x 2 ways)
+constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (4 warp pairs x 2 ways x 2 KiB)
 
 enum EpiMode : int { kEpiSwiGLU = 0, kEpiStore = 1, kEpiReduce = 2 };
 
@@ -76,19 +89,21 @@ struct FfnGemmParams {
 };
 
 struct FfnSmem {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[6];
+    uint64_t empty[6];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
-    int go_flag[2];        // GEMM1: per warp pair, did the gate warp's accumulator wait succeed
+    int go_flag[4];        // GEMM1: per warp pair, did the gate warp's accumulator wait succeed
     int abort_flag;
     int total_tiles;
 };
 
 struct TileInfo {
-    int e, f_blk, p0, n_valid, n_mma;
+    int e, f_blk, p0, n_valid, n_mma;   // n_valid <= tok_block tokens; n_mma: slot 0's N
+    int n_slots;                         // accumulator slots the tile uses (1 or 2)
+    int n_mma1;                          // slot 1's N (tokens 256..n_valid-1, rounded to 16)
 };
 
 __device__ __forceinline__ TileInfo decode_tile(int tile, const int32_t *s_tpre, const int32_t *s_tb,
@@ -108,7 +123,9 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int32_t *s_tpre,
     const int m_e = P.expert_offsets[lo + 1] - off;
     t.p0 = off + t_blk * P.tok_block;
     t.n_valid = min(P.tok_block, m_e - t_blk * P.tok_block);
-    t.n_mma = (t.n_valid + 15) & ~15;
+    t.n_mma = (min(t.n_valid, kSlotTok) + 15) & ~15;
+    t.n_slots = t.n_valid > kSlotTok ? 2 : 1;
+    t.n_mma1 = t.n_slots == 2 ? ((t.n_valid - kSlotTok + 15) & ~15) : 0;
     return t;
 }
 
@@ -118,18 +135,20 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int MODE>
+template <int MODE, int kMaxSlots>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const FfnGemmParams P) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
+    constexpr int kStages = RingCfg<kMaxSlots>::kStages;
+    constexpr uint32_t kStageBytes = RingCfg<kMaxSlots>::kStageBytes;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles (same offsets in both CTAs of the pair)
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char *tiles = base;                              // [kStages][weights | tokens]
-    float *xchg = reinterpret_cast<float *>(base + kStages * kStageBytes);   // GEMM1 only
-    FfnSmem *S = reinterpret_cast<FfnSmem *>(base + kStages * kStageBytes + (kSwiGLU ? kXchgBytes : 0));
+    float *xchg = reinterpret_cast<float *>(base + kRingBytes);   // GEMM1 only
+    FfnSmem *S = reinterpret_cast<FfnSmem *>(base + kRingBytes + (kSwiGLU ? kXchgBytes : 0));
     int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);   // [E + 1] tile prefix
     int32_t *s_tb = s_tpre + (P.E + 1);                       // [E] token blocks per expert
 
@@ -162,13 +181,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&S->full[s], 1); mbar_init(&S->empty[s], 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(&S->tmem_full[a], 1); mbar_init(&S->tmem_empty[a], 8); }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S->tmem_full[a], 1);
+            mbar_init(&S->tmem_empty[a], 2 * kEpiWarps);   // every epilogue warp of both CTAs
+        }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) { tma_prefetch_desc(&tmap_w); tma_prefetch_desc(&tmap_x); }
-    if (warp == 5) { tmem_alloc_pair(&S->tmem_base, kTmemCols); tmem_relinquish_pair(); }
+    if (warp == kProdWarp && lane == 0) { tma_prefetch_desc(&tmap_w); tma_prefetch_desc(&tmap_x); }
+    if (warp == kMmaWarp) { tmem_alloc_pair(&S->tmem_base, kTmemCols); tmem_relinquish_pair(); }
     tc_fence_before();
     cluster_sync_all();      // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
@@ -178,7 +200,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
     const int num_k = (P.K + kBK - 1) / kBK;
     volatile int *abort_flag = &S->abort_flag;
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             int stage = 0;
@@ -190,11 +212,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows, GEMM2 128 rows
                 const int w_row = ti.e * P.w_rows_per_expert +
                                   (ti.f_blk * 2 + (int)rank) * P.feat_per_cta;
-                // this CTA's half of the token rows
-                const int half = ti.n_mma / 2;
-                const int tok_row = ti.p0 + (int)rank * half;
-                const int n_box = (half + kTokRows - 1) / kTokRows;
-                const uint32_t bytes = kWBytes + n_box * kTokBoxBytes;
+                // this CTA's half of each slot's token rows
+                const int half0 = ti.n_mma / 2, half1 = ti.n_mma1 / 2;
+                const int tok_row0 = ti.p0 + (int)rank * half0;
+                const int tok_row1 = ti.p0 + kSlotTok + (int)rank * half1;
+                const int n_box0 = (half0 + kTokRows - 1) / kTokRows;
+                const int n_box1 = (half1 + kTokRows - 1) / kTokRows;
+                const uint32_t bytes = kWBytes + (n_box0 + n_box1) * kTokBoxBytes;
                 for (int kb = 0; kb < num_k; ++kb) {
                     if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     unsigned char *st = tiles + stage * kStageBytes;
@@ -207,9 +231,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     } else {
                         tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
                     }
-                    for (int b = 0; b < n_box; ++b)
+                    for (int b = 0; b < n_box0; ++b)
                         tma_load_2d_pair(st + kWBytes + b * kTokBoxBytes, &tmap_x, full_leader, kx,
-                                         tok_row + b * kTokRows);
+                                         tok_row0 + b * kTokRows);
+                    for (int b = 0; b < n_box1; ++b)
+                        tma_load_2d_pair(st + kWBytes + kSlotBytes + b * kTokBoxBytes, &tmap_x,
+                                         full_leader, kx, tok_row1 + b * kTokRows);
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -230,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer (leader CTA)
         if (lane == 0) {
             if (rank == 0) {
@@ -242,24 +269,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 for (int tile = pair; tile < total && ok; tile += npairs) {
                     const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
                     const uint32_t idesc = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
+                    const uint32_t idesc1 = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma1 > 0 ? ti.n_mma1 : 16);
+                    // slot 0 takes buffer `acc`, slot 1 (if any) the next buffer in the ring
+                    const int acc1 = acc ^ 1;
+                    const uint32_t acc1_phase = acc == 1 ? acc_phase ^ 1u : acc_phase;
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+                    if (ti.n_slots == 2 &&
+                        !mbar_wait_bounded(&S->tmem_empty[acc1], acc1_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d0 = tmem_base + (uint32_t)(acc * kTokBlock);
+                    const uint32_t d0 = tmem_base + (uint32_t)(acc * kSlotTok);
+                    const uint32_t d1 = tmem_base + (uint32_t)(acc1 * kSlotTok);
                     for (int kb = 0; kb < num_k; ++kb) {
                         if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t st = smem_u32(tiles + stage * kStageBytes);
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            tc_mma_f16_pair(d0, make_sw128_desc(st + kk * 32),
-                                            make_sw128_desc(st + kWBytes + kk * 32), idesc,
-                                            (kb > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t wdesc = make_sw128_desc(st + kk * 32);
+                            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                            tc_mma_f16_pair(d0, wdesc, make_sw128_desc(st + kWBytes + kk * 32), idesc, accum);
+                            if (kMaxSlots == 2 && ti.n_slots == 2)
+                                tc_mma_f16_pair(d1, wdesc, make_sw128_desc(st + kWBytes + kSlotBytes + kk * 32),
+                                                idesc1, accum);
+                        }
                         tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
                         if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     }
                     if (!ok) break;
-                    tc_commit_pair_mc(&S->tmem_full[acc], 0x3);    // accumulators ready in both CTAs
-                    if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+                    // accumulators ready in both CTAs, slot by slot
+                    for (int sl = 0; sl < ti.n_slots; ++sl) {
+                        tc_commit_pair_mc(&S->tmem_full[acc], 0x3);
+                        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+                    }
                 }
                 if (!ok) {
                     raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
@@ -272,53 +313,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             mbar_wait_bounded(&S->mma_done, 0, &never);
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 0-3 of both CTAs)
-        const int q = warp;  // TMEM lanes 32q .. 32q+31
-        // GEMM1: warp q < 2 holds gate, warp q + 2 the up rows of the same 32 features;
-        // GEMM2: warp q holds output features 32q .. 32q+31 of this CTA's 128
+        // ------------------------------------------------ epilogue (warps 0-7 of both CTAs)
+        // warp w drains TMEM lanes 32q .. 32q+31 (q = w % 4) for the 32-token
+        // chunks of parity w / 4, so two warps share each lane quadrant
+        const int q = warp & 3, half = warp >> 2;
+        // GEMM1: quadrants 0-1 hold gate, quadrants 2-3 the up rows of the same features;
+        // GEMM2: quadrant q holds output features 32q .. 32q+31 of this CTA's 128
         const int feat_lane = kSwiGLU ? (q & 1) * 32 + lane : q * 32 + lane;
         const bool is_gate = q < 2;
+        const int xpair = half * 2 + (q & 1);                 // gate/up warp pair (GEMM1)
         const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
                                           mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
         int acc = 0;
         uint32_t acc_phase = 0;
-        int xbuf = 0;
-        for (int tile = pair; tile < total; tile += npairs) {
+        bool run_on = true;
+        for (int tile = pair; tile < total && run_on; tile += npairs) {
+          const TileInfo tinfo = decode_tile(tile, s_tpre, s_tb, P);
+          for (int sl = 0; sl < tinfo.n_slots; ++sl) {
             bool go;
             if (kSwiGLU) {
                 // the gate warp waits (bounded) and tells its up partner; both then
                 // pass the same exchange barriers or both leave
                 if (is_gate) {
                     go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
-                    if (lane == 0) S->go_flag[q & 1] = go ? 1 : 0;
+                    if (lane == 0) S->go_flag[xpair] = go ? 1 : 0;
                 }
-                named_barrier_sync(1 + (q & 1), 64);
-                if (!is_gate) go = S->go_flag[q & 1] != 0;
+                named_barrier_sync(1 + xpair, 64);
+                if (!is_gate) go = S->go_flag[xpair] != 0;
             } else {
                 go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
             }
             if (!go) {
                 if (lane == 0) { raise_status(P.status, MOE_DEV_WAIT_TIMEOUT); *abort_flag = 1; }
+                run_on = false;
                 break;
             }
             tc_fence_after();
-            const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
+            // this slot's tokens: [sl * 256, sl * 256 + 256) of the tile
+            TileInfo ti = tinfo;
+            ti.p0 += sl * kSlotTok;
+            ti.n_valid = min(kSlotTok, tinfo.n_valid - sl * kSlotTok);
+            ti.n_mma = sl == 0 ? tinfo.n_mma : tinfo.n_mma1;
             const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
             const bool f_ok = f < P.out_cols;
-            const uint32_t tbase = tmem_base + (uint32_t)(acc * kTokBlock) + ((uint32_t)(q * 32) << 16);
+            const uint32_t tbase = tmem_base + (uint32_t)(acc * kSlotTok) + ((uint32_t)(q * 32) << 16);
 
-            for (int c0 = 0; c0 < ti.n_mma; c0 += 32) {
+            for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
                 tc_wait_ld();
                 if (kSwiGLU) {
                     // exchange: gate warps hand over tokens 16..31, up warps tokens 0..15
-                    float *mine = xchg + (((q & 1) * 2 + xbuf) * 2 + (is_gate ? 0 : 1)) * 512;
-                    float *theirs = xchg + (((q & 1) * 2 + xbuf) * 2 + (is_gate ? 1 : 0)) * 512;
+                    float *mine = xchg + (xpair * 2 + (is_gate ? 0 : 1)) * 512;
+                    float *theirs = xchg + (xpair * 2 + (is_gate ? 1 : 0)) * 512;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]);
-                    named_barrier_sync(1 + (q & 1), 64);
+                    named_barrier_sync(1 + xpair, 64);
                     const int cbase = c0 + (is_gate ? 0 : 16);
                     const int nc = min(16, ti.n_valid - cbase);
                     __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) +
@@ -334,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                             }
                         }
                     }
-                    xbuf ^= 1;
+                    named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
                 } else if (MODE == kEpiStore) {
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
                     const int nc = min(32, ti.n_valid - c0);
@@ -365,12 +416,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_leader[acc]);   // release the pair's accumulator
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+          }
         }
     }
 
     tc_fence_before();
     cluster_sync_all();      // both CTAs done: no MMA, copy or remote arrive in flight
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, kTmemCols);
     }
@@ -408,23 +460,39 @@ static bool make_tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t rows, uint6
 }
 
 size_t ffn_tcgen05_smem(int E, bool swiglu) {
-    return 1024 + (size_t)kStages * kStageBytes + (swiglu ? kXchgBytes : 0) + sizeof(FfnSmem) +
+    return 1024 + (size_t)kRingBytes + (swiglu ? kXchgBytes : 0) + sizeof(FfnSmem) +
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
+}
+
+template <int MODE, int kMaxSlots>
+static cudaError_t launch_gemm_slots(const CUtensorMap &tw, const CUtensorMap &tx,
+                                     const FfnGemmParams &P, int grid, cudaStream_t s) {
+    const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
+    static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
+    if (smem > configured) {
+        cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE, kMaxSlots>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        configured = smem;
+    }
+    ffn_gemm_tcgen05_kernel<MODE, kMaxSlots><<<grid, kFfnThreads, smem, s>>>(tw, tx, P);
+    return cudaGetLastError();
 }
 
 template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
                                const FfnGemmParams &P, int grid, cudaStream_t s) {
-    const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
-    static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
-    if (smem > configured) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        configured = smem;
-    }
-    ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, P);
-    return cudaGetLastError();
+    if (P.tok_block > kSlotTok) return launch_gemm_slots<MODE, 2>(tw, tx, P, grid, s);
+    return launch_gemm_slots<MODE, 1>(tw, tx, P, grid, s);
+}
+
+// Rows one expert can receive in a launch over n_rows receive rows: a token
+// picks an expert at most once, so at most the chunk's tokens (n_rows / k when
+// nothing is clipped) and at most the capacity.
+static int64_t tok_count_of_launch(const moe_config &c, int64_t n_rows) {
+    int64_t m = (n_rows + c.k - 1) / c.k;
+    if (c.capacity >= 0 && c.capacity < m) m = c.capacity;
+    return m;
 }
 
 // Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
@@ -449,7 +517,13 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
     P1.w_rows_per_expert = 2 * c.I;
     P1.up_offset = c.I;
-    P1.tok_block = kTokBlock;
+    // Two accumulator slots (up to 512 tokens per weight pass) save a second
+    // pass over a slice's weights for experts with 257..512 rows, but a 2-slot
+    // tile holds both TMEM buffers, so its epilogue no longer overlaps the next
+    // main loop.  That pays off when the main loop is long (K >= 4096) and some
+    // expert of the launch can hold more than 256 rows.
+    const bool many_rows = tok_count_of_launch(c, n_rows) > kSlotTok;
+    P1.tok_block = (many_rows && c.H >= 4096) ? 2 * kSlotTok : kSlotTok;
     P1.out_cols = c.I;
     P1.out = h;
     P1.k = c.k;
@@ -467,7 +541,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
     P2.w_rows_per_expert = c.H;
     P2.up_offset = 0;
-    P2.tok_block = kTokBlock;
+    P2.tok_block = (many_rows && c.I >= 4096) ? 2 * kSlotTok : kSlotTok;
     P2.out_cols = c.H;
     P2.out = y;
     P2.out_reduce = out_reduce;
