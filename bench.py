@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/ffn_tcgen05_qwen3_30b_a3b.md.  Keyed by workload; ``src`` is the
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
-FFN_TRAFFIC = {"qwen3_30b_a3b": {"bytes": 2015.3e6, "src": "a00e6fdb8f46c53a"}}
+FFN_TRAFFIC = {}
 
 
 def parse_args(argv=None):

@@ -30,7 +30,9 @@
 // the pair's tcgen05.mma (bf16 -> fp32) into one of two TMEM accumulator
 // buffers and commits to both CTAs' barriers, so the epilogue of tile i
 // overlaps the main loop of tile i+1 (a tile with 257..512 tokens takes both
-// buffers: one pass over its weights feeds two MMAs); warps 0-3 of each CTA drain its TMEM
+// buffers: one pass over its weights feeds two MMAs).  The leader's producer
+// takes tiles from a global counter and publishes them to both CTAs through a
+// small mbarrier queue; warps 0-3 of each CTA drain its TMEM
 // (warp q owns lanes 32q..32q+31) and write h / y one token row at a time.
 // Tiles run expert by expert, weight block by weight block, token block
 // innermost.
@@ -88,16 +90,22 @@ struct FfnGemmParams {
     uint32_t *status;
 };
 
+constexpr int kQueue = 8;                            // slices published ahead of the slowest consumer
+
 struct FfnSmem {
     uint64_t full[6];
     uint64_t empty[6];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
+    uint64_t q_full[kQueue];   // slice queue: published (count 1), per CTA
+    uint64_t q_empty[kQueue];  // slice queue: read by every consumer (leader CTA only)
+    int q_slice[kQueue];
     uint32_t tmem_base;
+    int pair_slice[4];     // GEMM1: slice the gate warp of a warp pair read for its partner
     int go_flag[4];        // GEMM1: per warp pair, did the gate warp's accumulator wait succeed
     int abort_flag;
-    int total_tiles;
+    int total_slices;      // tiles (the name is kept for the queue's work units)
 };
 
 struct TileInfo {
@@ -106,21 +114,29 @@ struct TileInfo {
     int n_mma1;                          // slot 1's N (tokens 256..n_valid-1, rounded to 16)
 };
 
-__device__ __forceinline__ TileInfo decode_tile(int tile, const int32_t *s_tpre, const int32_t *s_tb,
-                                                const FfnGemmParams &P) {
-    int lo = 0, hi = P.E - 1;  // last e with s_tpre[e] <= tile (it owns >= 1 tile)
+// Work is dealt out tile by tile from a global counter, so a pair that finishes
+// early takes more.  Tiles are numbered expert by expert, weight slice (expert,
+// pair feature block) by weight slice, token block innermost: the tiles of one
+// slice are taken back to back and stream the same weights at the same time.
+__device__ __forceinline__ void decode_tile(int tile, const int32_t *s_tpre, const int32_t *s_tb,
+                                            int E, int &e, int &f_blk, int &t_blk) {
+    int lo = 0, hi = E - 1;  // last e with s_tpre[e] <= tile (it owns >= 1 tile)
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (s_tpre[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    TileInfo t;
-    t.e = lo;
+    e = lo;
     const int local = tile - s_tpre[lo];
-    const int tb = s_tb[lo];
-    t.f_blk = local / tb;
-    const int t_blk = local - t.f_blk * tb;
-    const int off = P.expert_offsets[lo];
-    const int m_e = P.expert_offsets[lo + 1] - off;
+    f_blk = local / s_tb[lo];
+    t_blk = local - f_blk * s_tb[lo];
+}
+
+__device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const FfnGemmParams &P) {
+    TileInfo t;
+    t.e = e;
+    t.f_blk = f_blk;
+    const int off = P.expert_offsets[e];
+    const int m_e = P.expert_offsets[e + 1] - off;
     t.p0 = off + t_blk * P.tok_block;
     t.n_valid = min(P.tok_block, m_e - t_blk * P.tok_block);
     t.n_mma = (min(t.n_valid, kSlotTok) + 15) & ~15;
@@ -135,13 +151,32 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// One consumer's position in the slice queue.  next() waits (bounded) for the
+// next published slice, reads it and releases the entry on the leader's
+// q_empty; it returns false on a timeout.  A slice of -1 ends the work.
+struct SliceReader {
+    int qi = 0;
+    uint32_t qph = 0;
+    __device__ __forceinline__ bool next(FfnSmem *S, volatile int *abort_flag, bool release,
+                                         int &slice) {
+        if (!mbar_wait_cluster_bounded(&S->q_full[qi], qph, abort_flag)) return false;
+        slice = *reinterpret_cast<volatile int *>(&S->q_slice[qi]);
+        if (release) mbar_arrive_cluster(mapa_shared(smem_u32(&S->q_empty[qi]), 0));
+        if (++qi == kQueue) { qi = 0; qph ^= 1u; }
+        return true;
+    }
+};
+
 template <int MODE, int kMaxSlots>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-    const FfnGemmParams P) {
+    const FfnGemmParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
     constexpr int kStages = RingCfg<kMaxSlots>::kStages;
     constexpr uint32_t kStageBytes = RingCfg<kMaxSlots>::kStageBytes;
+    // queue consumers per entry: the MMA thread, the follower's producer, and
+    // every epilogue warp of both CTAs (GEMM1: the gate warp of each pair only)
+    constexpr uint32_t kQueueConsumers = 2 + 2 * (kSwiGLU ? kEpiWarps / 2 : kEpiWarps);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles (same offsets in both CTAs of the pair)
     unsigned char *base = reinterpret_cast<unsigned char *>(
@@ -154,9 +189,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();                  // 0: leader (issues the MMA)
-    const int pair = (int)cluster_id_x(), npairs = (int)ncluster_x();
 
-    // --- tile table (every CTA builds the same one from the expert offsets)
+    // --- slice table (every CTA builds the same one from the expert offsets)
     if (warp == 0) {
         int run = 0;
         for (int e0 = 0; e0 < P.E; e0 += 32) {
@@ -177,7 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             if (e < P.E) s_tpre[e] = run + incl - t;
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) { s_tpre[P.E] = run; S->total_tiles = run; }
+        if (lane == 0) { s_tpre[P.E] = run; S->total_slices = run; }
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) { mbar_init(&S->full[s], 1); mbar_init(&S->empty[s], 1); }
@@ -185,6 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             mbar_init(&S->tmem_full[a], 1);
             mbar_init(&S->tmem_empty[a], 2 * kEpiWarps);   // every epilogue warp of both CTAs
         }
+        for (int i = 0; i < kQueue; ++i) { mbar_init(&S->q_full[i], 1); mbar_init(&S->q_empty[i], kQueueConsumers); }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
         fence_mbar_init();
@@ -195,7 +230,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
     cluster_sync_all();      // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
 
-    const int total = S->total_tiles;
+    const int total = S->total_slices;
     const uint32_t tmem_base = S->tmem_base;
     const int num_k = (P.K + kBK - 1) / kBK;
     volatile int *abort_flag = &S->abort_flag;
@@ -207,38 +242,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int tile = pair; tile < total && ok; tile += npairs) {
-                const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
+            // leader: takes slices from the global counter and publishes them to
+            // every consumer of both CTAs; follower: reads them like a consumer
+            int qi = 0;
+            uint32_t qph = 0;
+            SliceReader reader;
+            auto next_slice = [&](int &slice) -> bool {
+                if (rank != 0) return reader.next(S, abort_flag, true, slice);
+                if (!mbar_wait_bounded(&S->q_empty[qi], qph ^ 1u, abort_flag)) return false;
+                const int got = (int)atomicAdd(work_counter, 1u);
+                slice = got < total ? got : -1;
+                S->q_slice[qi] = slice;
+                st_cluster_u32(mapa_shared(smem_u32(&S->q_slice[qi]), 1), (uint32_t)slice);
+                mbar_arrive(&S->q_full[qi]);
+                mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->q_full[qi]), 1));
+                if (++qi == kQueue) { qi = 0; qph ^= 1u; }
+                return true;
+            };
+            int slice;
+            while (ok) {
+                if (!next_slice(slice)) { ok = false; break; }
+                if (slice < 0) break;
+                int se, sf, t_blk;
+                decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
                 // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows, GEMM2 128 rows
-                const int w_row = ti.e * P.w_rows_per_expert +
-                                  (ti.f_blk * 2 + (int)rank) * P.feat_per_cta;
-                // this CTA's half of each slot's token rows
-                const int half0 = ti.n_mma / 2, half1 = ti.n_mma1 / 2;
-                const int tok_row0 = ti.p0 + (int)rank * half0;
-                const int tok_row1 = ti.p0 + kSlotTok + (int)rank * half1;
-                const int n_box0 = (half0 + kTokRows - 1) / kTokRows;
-                const int n_box1 = (half1 + kTokRows - 1) / kTokRows;
-                const uint32_t bytes = kWBytes + (n_box0 + n_box1) * kTokBoxBytes;
-                for (int kb = 0; kb < num_k; ++kb) {
-                    if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-                    unsigned char *st = tiles + stage * kStageBytes;
-                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
-                    const int kx = kb * kBK;
-                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * bytes);
-                    if (kSwiGLU) {
-                        tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
-                        tma_load_2d_pair(st + kWBytes / 2, &tmap_w, full_leader, kx, w_row + P.up_offset);
-                    } else {
-                        tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
+                const int w_row = se * P.w_rows_per_expert + (sf * 2 + (int)rank) * P.feat_per_cta;
+                {
+                    const TileInfo ti = tile_info(se, sf, t_blk, P);
+                    // this CTA's half of each slot's token rows
+                    const int half0 = ti.n_mma / 2, half1 = ti.n_mma1 / 2;
+                    const int tok_row0 = ti.p0 + (int)rank * half0;
+                    const int tok_row1 = ti.p0 + kSlotTok + (int)rank * half1;
+                    const int n_box0 = (half0 + kTokRows - 1) / kTokRows;
+                    const int n_box1 = (half1 + kTokRows - 1) / kTokRows;
+                    const uint32_t bytes = kWBytes + (n_box0 + n_box1) * kTokBoxBytes;
+                    for (int kb = 0; kb < num_k; ++kb) {
+                        if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                        unsigned char *st = tiles + stage * kStageBytes;
+                        const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
+                        const int kx = kb * kBK;
+                        if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * bytes);
+                        if (kSwiGLU) {
+                            tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
+                            tma_load_2d_pair(st + kWBytes / 2, &tmap_w, full_leader, kx, w_row + P.up_offset);
+                        } else {
+                            tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
+                        }
+                        for (int b = 0; b < n_box0; ++b)
+                            tma_load_2d_pair(st + kWBytes + b * kTokBoxBytes, &tmap_x, full_leader, kx,
+                                             tok_row0 + b * kTokRows);
+                        for (int b = 0; b < n_box1; ++b)
+                            tma_load_2d_pair(st + kWBytes + kSlotBytes + b * kTokBoxBytes, &tmap_x,
+                                             full_leader, kx, tok_row1 + b * kTokRows);
+                        ++issued;
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     }
-                    for (int b = 0; b < n_box0; ++b)
-                        tma_load_2d_pair(st + kWBytes + b * kTokBoxBytes, &tmap_x, full_leader, kx,
-                                         tok_row0 + b * kTokRows);
-                    for (int b = 0; b < n_box1; ++b)
-                        tma_load_2d_pair(st + kWBytes + kSlotBytes + b * kTokBoxBytes, &tmap_x,
-                                         full_leader, kx, tok_row1 + b * kTokRows);
-                    ++issued;
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
             }
             if (!ok) {
@@ -266,8 +324,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 int acc = 0;
                 uint32_t acc_phase = 0;
                 bool ok = true;
-                for (int tile = pair; tile < total && ok; tile += npairs) {
-                    const TileInfo ti = decode_tile(tile, s_tpre, s_tb, P);
+                SliceReader reader;
+                int slice;
+                while (ok) {
+                  if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
+                  if (slice < 0) break;
+                  int se, sf, t_blk;
+                  decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
+                  {
+                    const TileInfo ti = tile_info(se, sf, t_blk, P);
                     const uint32_t idesc = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
                     const uint32_t idesc1 = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma1 > 0 ? ti.n_mma1 : 16);
                     // slot 0 takes buffer `acc`, slot 1 (if any) the next buffer in the ring
@@ -301,6 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                         tc_commit_pair_mc(&S->tmem_full[acc], 0x3);
                         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
                     }
+                  }
                 }
                 if (!ok) {
                     raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
@@ -326,14 +392,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                                           mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
         int acc = 0;
         uint32_t acc_phase = 0;
+        SliceReader reader;
         bool run_on = true;
-        for (int tile = pair; tile < total && run_on; tile += npairs) {
-          const TileInfo tinfo = decode_tile(tile, s_tpre, s_tb, P);
-          for (int sl = 0; sl < tinfo.n_slots; ++sl) {
+        while (run_on) {
+          int slice = -1;
+          if (kSwiGLU) {
+              // the gate warp reads the queue and hands the slice to its up partner;
+              // both then pass the same exchange barriers or both leave
+              if (is_gate) {
+                  if (!reader.next(S, abort_flag, lane == 0, slice)) slice = -2;
+                  if (lane == 0) S->pair_slice[xpair] = slice;
+              }
+              named_barrier_sync(1 + xpair, 64);
+              if (!is_gate) slice = *reinterpret_cast<volatile int *>(&S->pair_slice[xpair]);
+          } else {
+              if (!reader.next(S, abort_flag, lane == 0, slice)) slice = -2;
+          }
+          if (slice == -2) {
+              if (lane == 0) { raise_status(P.status, MOE_DEV_WAIT_TIMEOUT); *abort_flag = 1; }
+              break;
+          }
+          if (slice < 0) break;
+          int se, sf, t_blk;
+          decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
+          {
+           const TileInfo tinfo = tile_info(se, sf, t_blk, P);
+           for (int sl = 0; sl < tinfo.n_slots; ++sl) {
             bool go;
             if (kSwiGLU) {
-                // the gate warp waits (bounded) and tells its up partner; both then
-                // pass the same exchange barriers or both leave
+                // same hand-over for the accumulator wait
                 if (is_gate) {
                     go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
                     if (lane == 0) S->go_flag[xpair] = go ? 1 : 0;
@@ -416,6 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_leader[acc]);   // release the pair's accumulator
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+           }
           }
         }
     }
@@ -466,7 +554,8 @@ size_t ffn_tcgen05_smem(int E, bool swiglu) {
 
 template <int MODE, int kMaxSlots>
 static cudaError_t launch_gemm_slots(const CUtensorMap &tw, const CUtensorMap &tx,
-                                     const FfnGemmParams &P, int grid, cudaStream_t s) {
+                                     const FfnGemmParams &P, int grid, uint32_t *counter,
+                                     cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
     if (smem > configured) {
@@ -475,15 +564,15 @@ static cudaError_t launch_gemm_slots(const CUtensorMap &tw, const CUtensorMap &t
         if (err != cudaSuccess) return err;
         configured = smem;
     }
-    ffn_gemm_tcgen05_kernel<MODE, kMaxSlots><<<grid, kFfnThreads, smem, s>>>(tw, tx, P);
+    ffn_gemm_tcgen05_kernel<MODE, kMaxSlots><<<grid, kFfnThreads, smem, s>>>(tw, tx, P, counter);
     return cudaGetLastError();
 }
 
 template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
-                               const FfnGemmParams &P, int grid, cudaStream_t s) {
-    if (P.tok_block > kSlotTok) return launch_gemm_slots<MODE, 2>(tw, tx, P, grid, s);
-    return launch_gemm_slots<MODE, 1>(tw, tx, P, grid, s);
+                               const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
+    if (P.tok_block > kSlotTok) return launch_gemm_slots<MODE, 2>(tw, tx, P, grid, counter, s);
+    return launch_gemm_slots<MODE, 1>(tw, tx, P, grid, counter, s);
 }
 
 // Rows one expert can receive in a launch over n_rows receive rows: a token
@@ -500,8 +589,11 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
                                const int32_t *expert_offsets, const void *w13, const void *w2,
                                void *h, void *y, const int32_t *recv_token,
                                const int32_t *recv_slot, const float *topk_w, float *out_reduce,
-                               uint32_t *status, cudaStream_t s, int num_sms) {
+                               uint32_t *status, uint32_t *counters, cudaStream_t s, int num_sms) {
     if (n_rows <= 0) return cudaSuccess;
+    // the two launches' work counters start at zero
+    cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
+    if (cerr != cudaSuccess) return cerr;
     CUtensorMap tw1, tx1, tw2, tx2;
     if (!make_tmap_bf16(&tw1, w13, (uint64_t)c.E * 2 * c.I, (uint64_t)c.H, kRowsPerCta / 2) ||
         !make_tmap_bf16(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTokRows) ||
@@ -532,7 +624,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     const long long max_pairs = num_sms / 2;
     long long g1 = (n_rows / P1.tok_block + c.E) * (long long)P1.n_fblocks;
     int grid1 = 2 * (int)(g1 < max_pairs ? g1 : max_pairs);
-    cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, P1, grid1, s);
+    cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, P1, grid1, counters, s);
     if (err != cudaSuccess) return err;
 
     FfnGemmParams P2 = P1;
@@ -550,8 +642,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P2.topk_w = topk_w;
     long long g2 = (n_rows / P2.tok_block + c.E) * (long long)P2.n_fblocks;
     int grid2 = 2 * (int)(g2 < max_pairs ? g2 : max_pairs);
-    if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, P2, grid2, s);
-    return launch_gemm<kEpiStore>(tw2, tx2, P2, grid2, s);
+    if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, P2, grid2, counters + 1, s);
+    return launch_gemm<kEpiStore>(tw2, tx2, P2, grid2, counters + 1, s);
 }
 
 }  // namespace moe

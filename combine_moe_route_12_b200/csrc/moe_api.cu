@@ -32,7 +32,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
                                const int32_t *expert_offsets, const void *w13, const void *w2,
                                void *h, void *y, const int32_t *recv_token,
                                const int32_t *recv_slot, const float *topk_w, float *out_reduce,
-                               uint32_t *status, cudaStream_t s, int num_sms);
+                               uint32_t *status, uint32_t *counters, cudaStream_t s, int num_sms);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -301,7 +301,8 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
         if (major != 10)
             return fail(MOE_ERR_UNSUPPORTED, "the bf16 FFN uses tcgen05 and needs sm_100 (got major %d)", major);
         err = launch_ffn_tcgen05(c, n_rows, xr, expert_offsets, w13, w2, h, y, recv_token,
-                                 recv_slot, topk_w, out_reduce, status, stream, current_num_sms());
+                                 recv_slot, topk_w, out_reduce, status,
+                                 ws_at<uint32_t>(ws, L.ffn_ctr), stream, current_num_sms());
         if (err == cudaErrorNotSupported)
             return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
     } else {
@@ -409,7 +410,8 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
         if (F.nmax > 0) {
             if (c.dtype == MOE_BF16) {
                 err = launch_ffn_tcgen05(c, F.nmax, xr, eoff, w13, w2, h, y, recv_token, recv_slot,
-                                         topk_w, out_reduce, status, s_compute, nsm);
+                                         topk_w, out_reduce, status, ws_at<uint32_t>(ws, L.ffn_ctr),
+                                         s_compute, nsm);
                 if (err == cudaErrorNotSupported)
                     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
             } else {

@@ -23,8 +23,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up aft
 //   layout ticket   uint32, then chunk_counts int32[E]
 //   tile_state      uint32[max_tiles * E] (decoupled-lookback descriptors)
 //   clip threshold  uint64[E]
+//   ffn counters    uint32[2] (dynamic work distribution of the FFN GEMMs)
 struct ScratchLayout {
-    size_t status, ticket, chunk_counts, tile_state, clip_thr, total;
+    size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr, total;
     int max_tiles;
 };
 
@@ -40,6 +41,7 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     if (L.max_tiles < 1) L.max_tiles = 1;
     L.tile_state = off;           off = align_up(off + sizeof(uint32_t) * (size_t)L.max_tiles * c.E, 256);
     L.clip_thr = off;             off = align_up(off + sizeof(uint64_t) * (size_t)c.E, 256);
+    L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
     L.total = off;
     return L;
 }
@@ -194,6 +196,35 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Arrive on a (possibly remote) mbarrier with cluster-scope release: orders this
+// thread's earlier shared::cluster stores before the arrival.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// try_wait with cluster-scope acquire (pairs with mbar_arrive_cluster_release)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity,
+                                                          volatile int *abort_flag) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((i & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
 }
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
