@@ -175,9 +175,11 @@ class ClockSampler:
 # --------------------------------------------------------------------------- workload
 
 def kernels_per_step(wl) -> int:
-    # route 1, clip 2 (select, mark); per chunk: layout 3 (hist, scatter, splits),
-    # permute 1, FFN 2 (two GEMM launches), combine or finalize 1
-    return 3 + wl.n_chunks * 7
+    # route 1; clip 2 (prep, mark) or 4 with a binding capacity (+ gather, select);
+    # per chunk: layout 2 (hist, scatter), permute 1, FFN 2 (two GEMM launches),
+    # combine or finalize 1
+    clip = 4 if wl.capacity > 0 else 2
+    return 1 + clip + wl.n_chunks * 6
 
 
 def algorithmic(wl, n_kept_chunks):
@@ -451,23 +453,46 @@ def run_ours(args):
     if moe.moe_device_status(layer.ws) != 0:
         raise RuntimeError("device status bits set during the timed region")
 
-    # ---------------- per-stage breakdown: the same kernels through the step
-    # ABI on one stream, events between the stages (eager launches)
+    # ---------------- per-stage breakdown: the same kernels through the step ABI
+    # on one stream with events between the stages, captured into a CUDA graph
+    # with the events (no host launch gaps); eager launches if capture fails
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(n_marks(wl))]
     for _ in range(2):
         run_steps(moe, wl, cfg, inp, B, None)
-    bd = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    stage_ms = {s: 0.0 for s in STAGES}
+    step_sum = 0.0
+    bd_ev = mk()
+    bd_graph = None
+    if use_graph:
+        try:
+            # external events stay timing events inside a captured graph
+            gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks(wl))]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_steps(moe, wl, cfg, inp, B, gev)
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            stage_times(wl, gev)          # raises if the events cannot be timed
+            bd_graph, bd_ev = g, gev
+        except Exception:
+            bd_graph = None
+            torch.cuda.synchronize()
     for i in range(args.steps):
         flush.fill_(1)
-        run_steps(moe, wl, cfg, inp, B, bd[i])
-    torch.cuda.synchronize()
+        if bd_graph is not None:
+            bd_graph.replay()
+        else:
+            run_steps(moe, wl, cfg, inp, B, bd_ev)
+        torch.cuda.synchronize()
+        for s_, v in stage_times(wl, bd_ev).items():
+            stage_ms[s_] += v / args.steps
+        step_sum += bd_ev[0].elapsed_time(bd_ev[-1]) / args.steps
     if moe.moe_device_status(B.ws) != 0:
         raise RuntimeError("device status bits set during the breakdown pass")
-    stage_ms = {s: 0.0 for s in STAGES}
-    for e in bd:
-        for s_, v in stage_times(wl, e).items():
-            stage_ms[s_] += v / len(bd)
-    eager_step_ms = sum(e[0].elapsed_time(e[-1]) for e in bd) / len(bd)
+    eager_step_ms = step_sum
+    breakdown_mode = "graph" if bd_graph is not None else "eager"
     n_kept = []
     for c in range(wl.n_chunks):
         moe.moe_dispatch_layout(cfg, c * B.tc, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
@@ -548,7 +573,8 @@ def run_ours(args):
                                  "peak_source": f"{peak_src} hbm_gbs"},
             "ffn_tflops": ffn_tflops,
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "eager_step_ms": round(eager_step_ms, 4),
+            "breakdown_step_ms": round(eager_step_ms, 4),
+            "breakdown_mode": breakdown_mode,
             "kept_rows": alg["N"],
             "e2e": e2e,
             "cpu_baseline": cpu,

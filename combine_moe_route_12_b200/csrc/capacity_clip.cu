@@ -7,10 +7,16 @@
 //     (bits(w[t, j]) << 32) | (2^32 - 1 - t),
 // which orders by weight descending then token ascending (weights are >= 0,
 // so their bit patterns order like their values; keys of one expert are
-// distinct because a token picks an expert at most once).  For each
-// over-capacity expert one CTA finds the C-th largest key by an MSB-first
-// radix select (8 passes of 8-bit digits); an assignment is kept iff its key
-// is >= that threshold, which keeps exactly C.
+// distinct because a token picks an expert at most once).
+//
+//   clip_prep    one CTA: which experts are over capacity, their key segment
+//                offsets (prefix sum of their counts); thresholds of the rest
+//   clip_gather  one pass over all assignments: the keys of over-capacity
+//                experts go to their segments (per-CTA ranges reserved with one
+//                atomic per CTA and expert)
+//   clip_select  one CTA per over-capacity expert: the C-th largest key of its
+//                segment by an MSB-first radix select (8 passes of 8-bit digits)
+//   clip_mark    keep[t, j] = key >= threshold of its expert, which keeps exactly C
 #include "moe_common.cuh"
 
 namespace moe {
@@ -24,11 +30,13 @@ __device__ __forceinline__ uint64_t clip_key(float w, int t) {
 
 // Radix select of the rank-`want` (1-based, descending) key among the keys that
 // `visit` produces.  visit(f) calls f(key) for every key of the segment; it is
-// called once per pass by every thread of the CTA.
+// called once per pass by every thread of the CTA.  The digit holding the
+// target rank is found by warp 0 with a suffix-sum over the 256 bins.
 template <typename Visit>
 __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hist,
                                       uint32_t *s_sel) {
     uint64_t prefix = 0, mask = 0;
+    const int lane = threadIdx.x & 31;
     for (int pass = 0; pass < 8; ++pass) {
         const int shift = 56 - 8 * pass;
         for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0;
@@ -43,14 +51,27 @@ __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hi
                 atomicAdd(&s_hist[d], (uint32_t)__popc(peers));
         });
         __syncthreads();
-        if (threadIdx.x == 0) {
-            uint32_t cum = 0, sel = 0;
-            for (int d = 255; d >= 0; --d) {
-                if (cum + s_hist[d] >= want) { sel = (uint32_t)d; break; }
-                cum += s_hist[d];
+        if (threadIdx.x < 32) {
+            // lane l owns bins 255-8l .. 248-8l (high digits first)
+            uint32_t c[8], tot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c[i] = s_hist[255 - 8 * lane - i]; tot += c[i]; }
+            uint32_t incl = tot;   // inclusive prefix over lanes = counts of digits >= this lane's
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
             }
-            s_sel[0] = sel;
-            s_sel[1] = want - cum;
+            const uint32_t before = incl - tot;
+            const bool mine = before < want && want <= incl;
+            if (mine) {
+                uint32_t cum = before;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (cum + c[i] >= want) { s_sel[0] = 255 - 8 * lane - i; s_sel[1] = want - cum; break; }
+                    cum += c[i];
+                }
+            }
         }
         __syncthreads();
         prefix |= (uint64_t)s_sel[0] << shift;
@@ -61,52 +82,121 @@ __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hi
     return prefix;
 }
 
-__global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
-    int T, int E, int k, int C, int smem_keys, const int32_t *__restrict__ topk_idx,
+constexpr int kGatherThreads = 256;
+constexpr int kGatherPerThread = 8;
+
+__global__ void __launch_bounds__(1024) clip_prep_kernel(int E, int C, const int32_t *__restrict__ counts,
+                                                         int32_t *__restrict__ seg,  // [2][E+1]: offsets, cursors
+                                                         int32_t *__restrict__ kept_counts,
+                                                         uint64_t *__restrict__ thr) {
+    __shared__ int32_t s_v[1025];
+    __shared__ int32_t s_w[33];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int n = counts[e];
+        const bool over = C >= 0 && n > C;
+        s_v[e] = over ? n : 0;
+        if (!over) { kept_counts[e] = n; thr[e] = 0; }
+        else { kept_counts[e] = C; if (C == 0) thr[e] = ~0ull; }
+    }
+    __syncthreads();
+    // exclusive scan of s_v (E <= 1024) by one warp, 32 entries per lane
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int sum = 0;
+        for (int i = 0; i < 32; ++i) { const int e = lane * 32 + i; if (e < E) sum += s_v[e]; }
+        int incl = sum;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < 32; ++i) {
+            const int e = lane * 32 + i;
+            if (e < E) { const int v = s_v[e]; s_v[e] = run; run += v; }
+        }
+        if (lane == 31) s_w[0] = incl;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) { seg[e] = s_v[e]; seg[E + 1 + e] = 0; }
+    if (threadIdx.x == 0) seg[E] = s_w[0];
+}
+
+__global__ void __launch_bounds__(kGatherThreads) clip_gather_kernel(
+    int T, int E, int k, int C, const int32_t *__restrict__ topk_idx,
     const float *__restrict__ topk_w, const int32_t *__restrict__ counts,
-    int32_t *__restrict__ kept_counts, uint64_t *__restrict__ thr) {
+    int32_t *__restrict__ seg, uint64_t *__restrict__ keys) {
+    extern __shared__ int32_t s_cnt[];   // [E] this CTA's keys per expert, then its base
+    const size_t total = (size_t)T * k;
+    const size_t a0 = (size_t)blockIdx.x * kGatherThreads * kGatherPerThread;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    int ex[kGatherPerThread], slot[kGatherPerThread];
+#pragma unroll
+    for (int i = 0; i < kGatherPerThread; ++i) {
+        const size_t a = a0 + (size_t)i * kGatherThreads + threadIdx.x;
+        int e = -1;
+        if (a < total) {
+            const int ev = __ldg(topk_idx + a);
+            if (ev >= 0 && ev < E && C >= 0 && __ldg(counts + ev) > C && C > 0) e = ev;
+        }
+        ex[i] = e;
+        slot[i] = -1;
+        const unsigned active = __activemask();
+        const unsigned peers = __match_any_sync(active, e);
+        if (e >= 0) {
+            const int leader = __ffs(peers) - 1;
+            int base = 0;
+            if ((int)(threadIdx.x & 31) == leader) base = atomicAdd(&s_cnt[e], __popc(peers));
+            base = __shfl_sync(peers, base, leader);
+            slot[i] = base + __popc(peers & ((1u << (threadIdx.x & 31)) - 1u));
+        }
+    }
+    __syncthreads();
+    // reserve this CTA's range in each touched expert's segment
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int n = s_cnt[e];
+        s_cnt[e] = n > 0 ? seg[e] + atomicAdd(&seg[E + 1 + e], n) : 0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kGatherPerThread; ++i) {
+        if (ex[i] < 0) continue;
+        const size_t a = a0 + (size_t)i * kGatherThreads + threadIdx.x;
+        const size_t dst = (size_t)s_cnt[ex[i]] + slot[i];
+        if (dst < total)   // counts inconsistent with topk_idx cannot write out of range
+            keys[dst] = clip_key(__ldg(topk_w + a), (int)(a / (size_t)k));
+    }
+}
+
+__global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
+    int E, int C, int smem_keys, long long total_keys, const int32_t *__restrict__ counts,
+    const int32_t *__restrict__ seg, const uint64_t *__restrict__ keys, uint64_t *__restrict__ thr) {
     extern __shared__ __align__(16) unsigned char s_raw[];
     __shared__ uint32_t s_hist[256];
     __shared__ uint32_t s_sel[2];
-    __shared__ uint32_t s_n;
     const int e = blockIdx.x;
-    const int n = counts[e];
-    if (C < 0 || n <= C) {
-        if (threadIdx.x == 0) { kept_counts[e] = n; thr[e] = 0; }
-        return;
-    }
-    if (C == 0) {
-        if (threadIdx.x == 0) { kept_counts[e] = 0; thr[e] = ~0ull; }
-        return;
-    }
-    const size_t total = (size_t)T * k;
+    int n = counts[e];
+    if (C <= 0 || n <= C) return;    // thresholds of these experts come from clip_prep
+    const uint64_t *mine = keys + seg[e];
+    if ((long long)seg[e] + n > total_keys) n = (int)(total_keys - seg[e]);   // inconsistent counts
     uint64_t key;
     if (n <= smem_keys) {
         uint64_t *s_keys = reinterpret_cast<uint64_t *>(s_raw);
-        if (threadIdx.x == 0) s_n = 0;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) s_keys[i] = __ldcg(mine + i);
         __syncthreads();
-        for (size_t a = threadIdx.x; a < total; a += blockDim.x) {
-            if (__ldg(topk_idx + a) == e) {
-                const uint32_t slot = atomicAdd(&s_n, 1u);
-                if (slot < (uint32_t)smem_keys) s_keys[slot] = clip_key(__ldg(topk_w + a), (int)(a / k));
-            }
-        }
-        __syncthreads();
-        const uint32_t m = min(s_n, (uint32_t)smem_keys);
         key = radix_select_desc(
             [&](auto f) {
-                for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) f(s_keys[i]);
+                for (int i = threadIdx.x; i < n; i += blockDim.x) f(s_keys[i]);
             },
             (uint32_t)C, s_hist, s_sel);
     } else {
         key = radix_select_desc(
             [&](auto f) {
-                for (size_t a = threadIdx.x; a < total; a += blockDim.x)
-                    if (__ldg(topk_idx + a) == e) f(clip_key(__ldg(topk_w + a), (int)(a / k)));
+                for (int i = threadIdx.x; i < n; i += blockDim.x) f(__ldcg(mine + i));
             },
             (uint32_t)C, s_hist, s_sel);
     }
-    if (threadIdx.x == 0) { kept_counts[e] = C; thr[e] = key; }
+    if (threadIdx.x == 0) thr[e] = key;
 }
 
 __global__ void clip_mark_kernel(int T, int E, int k, const int32_t *__restrict__ topk_idx,
@@ -128,24 +218,33 @@ __global__ void clip_mark_kernel(int T, int E, int k, const int32_t *__restrict_
 
 cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
                                  const float *topk_w, const int32_t *counts, uint8_t *keep,
-                                 int32_t *kept_counts, uint64_t *thr, uint32_t *status,
-                                 cudaStream_t s, int num_sms) {
-    int smem_keys = c.T < kClipMaxSmemKeys ? c.T : kClipMaxSmemKeys;
-    if (smem_keys < 1) smem_keys = 1;
-    const size_t smem = sizeof(uint64_t) * (size_t)smem_keys;
-    cudaError_t err;
-    static size_t configured = 48 * 1024;
-    if (smem > configured) {
-        err = cudaFuncSetAttribute(clip_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem);
-        if (err != cudaSuccess) return err;
-        configured = smem;
-    }
-    clip_select_kernel<<<c.E, kClipThreads, smem, s>>>(c.T, c.E, c.k, c.capacity, smem_keys,
-                                                       topk_idx, topk_w, counts, kept_counts, thr);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+                                 int32_t *kept_counts, uint64_t *thr, int32_t *seg, uint64_t *keys,
+                                 uint32_t *status, cudaStream_t s, int num_sms) {
+    clip_prep_kernel<<<1, 1024, 0, s>>>(c.E, c.capacity, counts, seg, kept_counts, thr);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
     const size_t total = (size_t)c.T * c.k;
     if (total == 0) return cudaSuccess;
+    if (c.capacity > 0) {
+        const int per_block = kGatherThreads * kGatherPerThread;
+        const int gblocks = (int)((total + per_block - 1) / per_block);
+        clip_gather_kernel<<<gblocks, kGatherThreads, sizeof(int32_t) * c.E, s>>>(
+            c.T, c.E, c.k, c.capacity, topk_idx, topk_w, counts, seg, keys);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        int smem_keys = c.T < kClipMaxSmemKeys ? c.T : kClipMaxSmemKeys;
+        if (smem_keys < 1) smem_keys = 1;
+        const size_t smem = sizeof(uint64_t) * (size_t)smem_keys;
+        static size_t configured = 48 * 1024;
+        if (smem > configured) {
+            err = cudaFuncSetAttribute(clip_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+            if (err != cudaSuccess) return err;
+            configured = smem;
+        }
+        clip_select_kernel<<<c.E, kClipThreads, smem, s>>>(c.E, c.capacity, smem_keys, (long long)total,
+                                                           counts, seg, keys, thr);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
     int blocks = (int)((total + 255) / 256);
     if (blocks > num_sms * 16) blocks = num_sms * 16;
     clip_mark_kernel<<<blocks, 256, 0, s>>>(c.T, c.E, c.k, topk_idx, topk_w, thr, keep, status);

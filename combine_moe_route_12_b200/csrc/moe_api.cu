@@ -13,8 +13,8 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
                               uint32_t *status, cudaStream_t s, int num_sms);
 cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
                                  const float *topk_w, const int32_t *counts, uint8_t *keep,
-                                 int32_t *kept_counts, uint64_t *thr, uint32_t *status,
-                                 cudaStream_t s, int num_sms);
+                                 int32_t *kept_counts, uint64_t *thr, int32_t *seg, uint64_t *keys,
+                                 uint32_t *status, cudaStream_t s, int num_sms);
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
                                    const int32_t *topk_idx, const uint8_t *keep,
                                    int32_t *expert_offsets, int32_t *rank_offsets,
@@ -230,7 +230,8 @@ moe_status moe_capacity_clip(const moe_config *cfg, const int32_t *topk_idx,
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
     const ScratchLayout L = scratch_layout(c);
     cudaError_t err = launch_capacity_clip(c, topk_idx, topk_w, counts, keep, kept_counts,
-                                           ws_at<uint64_t>(ws, L.clip_thr),
+                                           ws_at<uint64_t>(ws, L.clip_thr), ws_at<int32_t>(ws, L.clip_seg),
+                                           ws_at<uint64_t>(ws, L.clip_keys),
                                            ws_at<uint32_t>(ws, L.status), stream,
                                            current_num_sms());
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_capacity_clip");
@@ -380,7 +381,8 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     MOE_TRY(launch_route_topk(c, logits, bias, topk_idx, topk_w, counts, status, s_dispatch, nsm),
             "route_topk");
     MOE_TRY(launch_capacity_clip(c, topk_idx, topk_w, counts, keep, kept_counts,
-                                 ws_at<uint64_t>(ws, L.clip_thr), status, s_dispatch, nsm),
+                                 ws_at<uint64_t>(ws, L.clip_thr), ws_at<int32_t>(ws, L.clip_seg),
+                                 ws_at<uint64_t>(ws, L.clip_keys), status, s_dispatch, nsm),
             "capacity_clip");
     if (c.reduce_dense)
         MOE_TRY(cudaMemsetAsync(out_reduce, 0, sizeof(float) * (size_t)c.T * c.H, s_dispatch),

@@ -24,8 +24,10 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up aft
 //   tile_state      uint32[max_tiles * E] (decoupled-lookback descriptors)
 //   clip threshold  uint64[E]
 //   ffn counters    uint32[2] (dynamic work distribution of the FFN GEMMs)
+//   clip segments   int32[2 * (E + 1)] offsets / cursors, keys uint64[T * k]
 struct ScratchLayout {
-    size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr, total;
+    size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr;
+    size_t clip_seg, clip_keys, total;
     int max_tiles;
 };
 
@@ -42,6 +44,8 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     L.tile_state = off;           off = align_up(off + sizeof(uint32_t) * (size_t)L.max_tiles * c.E, 256);
     L.clip_thr = off;             off = align_up(off + sizeof(uint64_t) * (size_t)c.E, 256);
     L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
+    L.clip_seg = off;             off = align_up(off + sizeof(int32_t) * 2 * ((size_t)c.E + 1), 256);
+    L.clip_keys = off;            off = align_up(off + sizeof(uint64_t) * (size_t)c.T * c.k, 256);
     L.total = off;
     return L;
 }

@@ -2,9 +2,12 @@
 // _select_experts with norm_topk_prob; axolotl ExpertParallelArgs: the routing
 // top-k is saved state).
 //
-// One warp per token.  Lane l holds the biased logits of experts l, l+32, ...
-// k rounds of a butterfly arg-max (value descending, lower expert index first
-// among equal values) pick the experts in rank order; lane j keeps slot j.
+// A group of LPT lanes (8, 16 or 32) per token, 32/LPT tokens per warp at a
+// time.  Lane l of a group holds the biased logits of experts l, l+LPT, ...
+// k rounds of a butterfly arg-max inside the group (value descending, lower
+// expert index first among equal values) pick the experts in rank order; lane
+// j of the group keeps slot j.  Narrow groups keep each round's shuffle chain
+// short and several tokens in flight per warp.
 // The weights w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) use a fixed fp32
 // exponential (Cody & Waite reduction, degree-7 Taylor polynomial, every step
 // one IEEE-rounded operation) and a slot-ordered sum, so they are bit-exact
@@ -47,7 +50,7 @@ __device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b) {
     return (va > vb) || (va == vb && a < b);
 }
 
-template <int VPL>
+template <int LPT, int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(
     int T, int E, int k, const float *__restrict__ logits, const float *__restrict__ bias,
     int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int32_t *__restrict__ counts,
@@ -56,18 +59,24 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
     __syncthreads();
 
+    constexpr int kGroups = 32 / LPT;
     const int lane = threadIdx.x & 31;
-    const int warps_total = gridDim.x * (blockDim.x >> 5);
+    const int gl = lane % LPT, g = lane / LPT;
+    const int glane0 = g * LPT;
+    const long long warps_total = (long long)gridDim.x * (blockDim.x >> 5);
     bool nonfinite = false;
 
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
-        const float *row = logits + (size_t)t * E;
+    for (long long t0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kGroups;
+         t0 < T; t0 += warps_total * kGroups) {
+        const long long t = t0 + g;
+        const bool valid = t < T;
+        const float *row = logits + (size_t)(valid ? t : 0) * E;
         float v[VPL];
         uint32_t taken = 0;
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E) {
+            const int e = gl + LPT * i;
+            if (valid && e < E) {
                 float l = __fadd_rn(__ldg(row + e), bias ? __ldg(bias + e) : 0.0f);
                 if (!isfinite(l)) {
                     nonfinite = true;
@@ -79,7 +88,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
                 taken |= 1u << i;  // padding never wins
             }
         }
-        float my_v = 0.0f;  // slot `lane`'s biased logit
+        float my_v = 0.0f;  // slot `gl`'s biased logit
         int my_e = 0;
         for (int j = 0; j < k; ++j) {
             bool has = false;
@@ -87,28 +96,28 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
             int be = 0x7fffffff;
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
-                const int e = lane + 32 * i;
+                const int e = gl + LPT * i;
                 if (!((taken >> i) & 1u) && (!has || ranks_before(v[i], e, bv, be))) {
                     has = true; bv = v[i]; be = e;
                 }
             }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
+            for (int off = LPT / 2; off > 0; off >>= 1) {
                 const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
                 const int oe = __shfl_xor_sync(0xffffffffu, be, off);
                 const bool oh = __shfl_xor_sync(0xffffffffu, (int)has, off) != 0;
                 if (oh && (!has || ranks_before(ov, oe, bv, be))) { has = true; bv = ov; be = oe; }
             }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == j) { my_v = bv; my_e = be; }
+            if (has && (be % LPT) == gl) taken |= 1u << (be / LPT);
+            if (gl == j) { my_v = bv; my_e = be; }
         }
-        const float m = __shfl_sync(0xffffffffu, my_v, 0);
-        const float ex = (lane < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
+        const float m = __shfl_sync(0xffffffffu, my_v, glane0);
+        const float ex = (gl < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
         float S = 0.0f;
-        for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ex, j));
-        if (lane < k) {
-            topk_idx[(size_t)t * k + lane] = my_e;
-            topk_w[(size_t)t * k + lane] = __fdiv_rn(ex, S);
+        for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ex, glane0 + j));
+        if (valid && gl < k) {
+            topk_idx[(size_t)t * k + gl] = my_e;
+            topk_w[(size_t)t * k + gl] = __fdiv_rn(ex, S);
             atomicAdd(&s_hist[my_e], 1);
         }
     }
@@ -125,19 +134,40 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     if (err != cudaSuccess || c.T == 0) return err;
     const int warps_per_block = 8;
     int blocks = (c.T + warps_per_block - 1) / warps_per_block;
-    const int cap = num_sms * 2;   // few CTAs: one global atomic per CTA and expert
+    const int cap = num_sms * 4;   // one global atomic per CTA and expert
     if (blocks > cap) blocks = cap;
     const size_t smem = sizeof(int32_t) * (size_t)c.E;
-    const int vpl = (c.E + 31) / 32;
-#define MOE_ROUTE_CASE(V)                                                                   \
-    route_topk_kernel<V><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, topk_idx, \
-                                                   topk_w, counts, status)
-    if (vpl <= 1) MOE_ROUTE_CASE(1);
-    else if (vpl <= 2) MOE_ROUTE_CASE(2);
-    else if (vpl <= 4) MOE_ROUTE_CASE(4);
-    else if (vpl <= 8) MOE_ROUTE_CASE(8);
-    else if (vpl <= 16) MOE_ROUTE_CASE(16);
-    else MOE_ROUTE_CASE(32);
+    // lanes per token: at least k (slot j lives in group lane j), at most 32,
+    // aiming at 16 values per lane
+    int lpt = 8;
+    while (lpt < 32 && (lpt < c.k || (c.E + lpt - 1) / lpt > 16)) lpt *= 2;
+    const int vpl = (c.E + lpt - 1) / lpt;
+    blocks = (int)(((long long)c.T * lpt / 32 + warps_per_block - 1) / warps_per_block);
+    if (blocks < 1) blocks = 1;
+    if (blocks > cap) blocks = cap;
+#define MOE_ROUTE_CASE(L, V)                                                                    \
+    route_topk_kernel<L, V><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, topk_idx, \
+                                                      topk_w, counts, status)
+    if (lpt == 8) {
+        if (vpl <= 1) MOE_ROUTE_CASE(8, 1);
+        else if (vpl <= 2) MOE_ROUTE_CASE(8, 2);
+        else if (vpl <= 4) MOE_ROUTE_CASE(8, 4);
+        else if (vpl <= 8) MOE_ROUTE_CASE(8, 8);
+        else MOE_ROUTE_CASE(8, 16);
+    } else if (lpt == 16) {
+        if (vpl <= 1) MOE_ROUTE_CASE(16, 1);
+        else if (vpl <= 2) MOE_ROUTE_CASE(16, 2);
+        else if (vpl <= 4) MOE_ROUTE_CASE(16, 4);
+        else if (vpl <= 8) MOE_ROUTE_CASE(16, 8);
+        else MOE_ROUTE_CASE(16, 16);
+    } else {
+        if (vpl <= 1) MOE_ROUTE_CASE(32, 1);
+        else if (vpl <= 2) MOE_ROUTE_CASE(32, 2);
+        else if (vpl <= 4) MOE_ROUTE_CASE(32, 4);
+        else if (vpl <= 8) MOE_ROUTE_CASE(32, 8);
+        else if (vpl <= 16) MOE_ROUTE_CASE(32, 16);
+        else MOE_ROUTE_CASE(32, 32);
+    }
 #undef MOE_ROUTE_CASE
     return cudaGetLastError();
 }
