@@ -48,7 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/ffn_tcgen05_qwen3_30b_a3b.md.  Keyed by workload; ``src`` is the
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
-FFN_TRAFFIC = {}
+FFN_TRAFFIC = {
+    "qwen3_30b_a3b": {"bytes": 1559.61728e6, "src": "9690687f49587448"},
+}
 
 
 def parse_args(argv=None):

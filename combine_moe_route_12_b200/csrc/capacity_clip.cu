@@ -15,7 +15,8 @@
 //                experts go to their segments (per-CTA ranges reserved with one
 //                atomic per CTA and expert)
 //   clip_select  one CTA per over-capacity expert: the C-th largest key of its
-//                segment by an MSB-first radix select (8 passes of 8-bit digits)
+//                segment by an MSB-first radix select (up to 8 passes of 8-bit
+//                digits, ending early once one key is left under the prefix)
 //   clip_mark    keep[t, j] = key >= threshold of its expert, which keeps exactly C
 #include "moe_common.cuh"
 
@@ -31,10 +32,13 @@ __device__ __forceinline__ uint64_t clip_key(float w, int t) {
 // Radix select of the rank-`want` (1-based, descending) key among the keys that
 // `visit` produces.  visit(f) calls f(key) for every key of the segment; it is
 // called once per pass by every thread of the CTA.  The digit holding the
-// target rank is found by warp 0 with a suffix-sum over the 256 bins.
+// target rank is found by warp 0 with a suffix-sum over the 256 bins.  Once the
+// chosen bin holds a single key, that key is the answer: one more visit picks
+// it up instead of the remaining digit passes (distinct fp32 weights are
+// usually told apart by the first two or three digits).
 template <typename Visit>
 __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hist,
-                                      uint32_t *s_sel) {
+                                      uint32_t *s_sel, uint64_t *s_found) {
     uint64_t prefix = 0, mask = 0;
     const int lane = threadIdx.x & 31;
     for (int pass = 0; pass < 8; ++pass) {
@@ -68,7 +72,10 @@ __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hi
                 uint32_t cum = before;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    if (cum + c[i] >= want) { s_sel[0] = 255 - 8 * lane - i; s_sel[1] = want - cum; break; }
+                    if (cum + c[i] >= want) {
+                        s_sel[0] = 255 - 8 * lane - i; s_sel[1] = want - cum; s_sel[2] = c[i];
+                        break;
+                    }
                     cum += c[i];
                 }
             }
@@ -77,7 +84,16 @@ __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hi
         prefix |= (uint64_t)s_sel[0] << shift;
         mask |= (uint64_t)255u << shift;
         want = s_sel[1];
+        const uint32_t left = s_sel[2];
         __syncthreads();
+        if (left == 1 && pass < 7) {
+            // the only key under this prefix (keys are distinct)
+            visit([&](uint64_t key) {
+                if ((key & mask) == prefix) *s_found = key;
+            });
+            __syncthreads();
+            return *s_found;
+        }
     }
     return prefix;
 }
@@ -173,7 +189,8 @@ __global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
     const int32_t *__restrict__ seg, const uint64_t *__restrict__ keys, uint64_t *__restrict__ thr) {
     extern __shared__ __align__(16) unsigned char s_raw[];
     __shared__ uint32_t s_hist[256];
-    __shared__ uint32_t s_sel[2];
+    __shared__ uint32_t s_sel[3];
+    __shared__ uint64_t s_found;
     const int e = blockIdx.x;
     int n = counts[e];
     if (C <= 0 || n <= C) return;    // thresholds of these experts come from clip_prep
@@ -188,13 +205,13 @@ __global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
             [&](auto f) {
                 for (int i = threadIdx.x; i < n; i += blockDim.x) f(s_keys[i]);
             },
-            (uint32_t)C, s_hist, s_sel);
+            (uint32_t)C, s_hist, s_sel, &s_found);
     } else {
         key = radix_select_desc(
             [&](auto f) {
                 for (int i = threadIdx.x; i < n; i += blockDim.x) f(__ldcg(mine + i));
             },
-            (uint32_t)C, s_hist, s_sel);
+            (uint32_t)C, s_hist, s_sel, &s_found);
     }
     if (threadIdx.x == 0) thr[e] = key;
 }

@@ -247,16 +247,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             int qi = 0;
             uint32_t qph = 0;
             SliceReader reader;
+            // the leader holds one ticket ahead: the counter's round trip for the
+            // next tile overlaps the loads of the current one
+            int ticket = rank == 0 ? (int)atomicAdd(work_counter, 1u) : 0;
             auto next_slice = [&](int &slice) -> bool {
                 if (rank != 0) return reader.next(S, abort_flag, true, slice);
                 if (!mbar_wait_bounded(&S->q_empty[qi], qph ^ 1u, abort_flag)) return false;
-                const int got = (int)atomicAdd(work_counter, 1u);
-                slice = got < total ? got : -1;
+                slice = ticket < total ? ticket : -1;
                 S->q_slice[qi] = slice;
                 st_cluster_u32(mapa_shared(smem_u32(&S->q_slice[qi]), 1), (uint32_t)slice);
                 mbar_arrive(&S->q_full[qi]);
                 mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->q_full[qi]), 1));
                 if (++qi == kQueue) { qi = 0; qph ^= 1u; }
+                if (slice >= 0) ticket = (int)atomicAdd(work_counter, 1u);
                 return true;
             };
             int slice;
@@ -448,7 +451,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
-                tc_wait_ld();
+                tc_wait_ld_regs(r);
                 if (kSwiGLU) {
                     // exchange: gate warps hand over tokens 16..31, up warps tokens 0..15
                     float *mine = xchg + (xpair * 2 + (is_gate ? 0 : 1)) * 512;
