@@ -24,18 +24,23 @@
 // and up_i; the two epilogue warps that own them swap half their columns
 // through shared memory and each finishes h for half the tokens.
 //
-// CTA = 10 warps.  Warp 4 (one lane) of each CTA streams its weight and token
-// tiles with TMA into a 6-stage ring of 128B-swizzled buffers, counting the
-// bytes on the leader CTA's mbarrier; warp 5 (one lane) of the leader issues
-// the pair's tcgen05.mma (bf16 -> fp32) into one of two TMEM accumulator
-// buffers and commits to both CTAs' barriers, so the epilogue of tile i
-// overlaps the main loop of tile i+1 (a tile with 257..512 tokens takes both
-// buffers: one pass over its weights feeds two MMAs).  The leader's producer
-// takes tiles from a global counter and publishes them to both CTAs through a
-// small mbarrier queue; warps 0-3 of each CTA drain its TMEM
-// (warp q owns lanes 32q..32q+31) and write h / y one token row at a time.
-// Tiles run expert by expert, weight block by weight block, token block
-// innermost.
+// CTA = 10 warps.  Warp 8 (one lane) of each CTA streams its weight and token
+// tiles with TMA into a ring of 128B-swizzled stages (6 stages of 32 KiB, or 4
+// of 48 KiB when a tile may carry two token slots), counting the bytes on the
+// leader CTA's mbarrier.  A stage takes one weight box (GEMM1: a 3-D box of 64
+// gate rows and the 64 matching up rows) and one 128-row token box per slot:
+// each TMA issue costs the producer on the order of a hundred cycles whatever
+// its size, so few large boxes keep it ahead of the tensor pipe (rows of a box
+// past the tile's tokens are loaded but never read by the MMA).  Warp 9 (one
+// lane) of the leader issues the pair's tcgen05.mma (bf16 -> fp32) into one of
+// two TMEM accumulator buffers and commits to both CTAs' barriers, so the
+// epilogue of tile i overlaps the main loop of tile i+1 (a tile with 257..512
+// tokens takes both buffers: one pass over its weights feeds two MMAs).  The
+// leader's producer takes tiles from a global counter, one ticket ahead, and
+// publishes them to both CTAs through a small mbarrier queue; warps 0-7 of
+// each CTA drain its TMEM (warps q and q+4 own lanes 32q..32q+31 and take
+// alternate 32-token chunks) and write h / y one token row at a time.  Tiles
+// run expert by expert, weight block by weight block, token block innermost.
 //
 // Every mbarrier wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT,
 // stops the other roles, lets in-flight copies and MMAs land, frees TMEM and
@@ -48,13 +53,13 @@ namespace moe {
 
 constexpr int kBK = 64;
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
-constexpr int kTokRows = 32;                         // rows per token TMA box
+constexpr int kTokRows = 128;                        // rows per token TMA box (one box per slot and CTA)
 constexpr int kSlotTok = 256;                        // tokens per accumulator slot (MMA N <= 256)
 constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
 constexpr int kProdWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
 constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;  // 16 KiB of weights per stage and CTA
-constexpr uint32_t kTokBoxBytes = kTokRows * kBK * 2;  // 4 KiB
+constexpr uint32_t kTokBoxBytes = kTokRows * kBK * 2;  // 16 KiB
 constexpr uint32_t kSlotBytes = (kSlotTok / 2) * kBK * 2;  // 16 KiB of one slot's tokens per CTA
 constexpr uint32_t kRingBytes = 192 * 1024;
 // A tile meets up to kMaxSlots * 256 tokens of its expert in one pass over its
@@ -286,8 +291,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                         const int kx = kb * kBK;
                         if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * bytes);
                         if (kSwiGLU) {
-                            tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
-                            tma_load_2d_pair(st + kWBytes / 2, &tmap_w, full_leader, kx, w_row + P.up_offset);
+                            // gate rows then the matching up rows, one 3-D box
+                            tma_load_3d_pair(st, &tmap_w, full_leader, kx, (sf * 2 + (int)rank) * P.feat_per_cta,
+                                             2 * se);
                         } else {
                             tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
                         }
@@ -535,6 +541,23 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix, box 64 cols x box_rows,
 // 128-byte swizzle, zero fill outside the matrix.
+// W13 [E][2][I][H] seen as the 3-D tensor (H, I, 2E): one box of 64 columns x
+// 64 feature rows x {gate, up} fills a CTA's 128 weight rows of a stage.
+static bool make_tmap_w13_bf16(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I, uint64_t H,
+                               uint32_t box_rows) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {H, I, 2 * E};
+    cuuint64_t strides[2] = {H * 2, I * H * 2};
+    cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 2u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 static bool make_tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
                            uint32_t box_rows) {
     auto enc = get_encode_fn();
@@ -598,7 +621,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
     if (cerr != cudaSuccess) return cerr;
     CUtensorMap tw1, tx1, tw2, tx2;
-    if (!make_tmap_bf16(&tw1, w13, (uint64_t)c.E * 2 * c.I, (uint64_t)c.H, kRowsPerCta / 2) ||
+    if (!make_tmap_w13_bf16(&tw1, w13, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H, kRowsPerCta / 2) ||
         !make_tmap_bf16(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTokRows) ||
         !make_tmap_bf16(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
         !make_tmap_bf16(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTokRows))
