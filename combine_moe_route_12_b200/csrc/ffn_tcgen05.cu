@@ -25,22 +25,23 @@
 // through shared memory and each finishes h for half the tokens.
 //
 // CTA = 10 warps.  Warp 8 (one lane) of each CTA streams its weight and token
-// tiles with TMA into a ring of 128B-swizzled stages (6 stages of 32 KiB, or 4
-// of 48 KiB when a tile may carry two token slots), counting the bytes on the
-// leader CTA's mbarrier.  A stage takes one weight box (GEMM1: a 3-D box of 64
-// gate rows and the 64 matching up rows) and one 128-row token box per slot:
-// each TMA issue costs the producer on the order of a hundred cycles whatever
-// its size, so few large boxes keep it ahead of the tensor pipe (rows of a box
-// past the tile's tokens are loaded but never read by the MMA).  Warp 9 (one
-// lane) of the leader issues the pair's tcgen05.mma (bf16 -> fp32) into one of
-// two TMEM accumulator buffers and commits to both CTAs' barriers, so the
-// epilogue of tile i overlaps the main loop of tile i+1 (a tile with 257..512
-// tokens takes both buffers: one pass over its weights feeds two MMAs).  The
-// leader's producer takes tiles from a global counter, one ticket ahead, and
-// publishes them to both CTAs through a small mbarrier queue; warps 0-7 of
-// each CTA drain its TMEM (warps q and q+4 own lanes 32q..32q+31 and take
-// alternate 32-token chunks) and write h / y one token row at a time.  Tiles
-// run expert by expert, weight block by weight block, token block innermost.
+// tiles with TMA into a ring of three 64 KiB stages of 128B-swizzled buffers,
+// counting the bytes on the leader CTA's mbarrier.  A stage holds two 64-column
+// k-chunks and takes two TMA boxes: the weights (GEMM1: one 4-D box of 64 gate
+// rows and the 64 matching up rows) and 128 token rows.  Each TMA issue costs
+// the producer on the order of a hundred cycles whatever its size, so few large
+// boxes keep it ahead of the tensor pipe (token rows of a box past the tile's N
+// are loaded but never read by the MMA).  Warp 9 (one lane) of the leader
+// issues the pair's tcgen05.mma (bf16 -> fp32) into one of two 256-column TMEM
+// accumulator buffers and commits to both CTAs' barriers, so the epilogue of
+// tile i overlaps the main loop of tile i+1.  An expert with more than 256 rows
+// takes one tile per 256-token block; the tiles of one weight slice are dealt
+// back to back, so the later ones read the slice from L2.  The leader's
+// producer takes tiles from a global counter, one ticket ahead, and publishes
+// them to both CTAs through a small mbarrier queue; warps 0-7 of each CTA
+// drain its TMEM (warps q and q+4 own lanes 32q..32q+31 and take alternate
+// 32-token chunks) and write h / y one token row at a time.  Tiles run expert
+// by expert, weight block by weight block, token block innermost.
 //
 // Every mbarrier wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT,
 // stops the other roles, lets in-flight copies and MMAs land, frees TMEM and
@@ -51,26 +52,18 @@
 
 namespace moe {
 
-constexpr int kBK = 64;
+constexpr int kBK = 64;                              // columns of one 128-byte swizzled k-chunk
+constexpr int kKS = 2;                               // k-chunks per ring stage (one TMA box each)
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
-constexpr int kTokRows = 128;                        // rows per token TMA box (one box per slot and CTA)
-constexpr int kSlotTok = 256;                        // tokens per accumulator slot (MMA N <= 256)
+constexpr int kTileTok = 256;                        // tokens per tile (MMA N <= 256)
 constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
 constexpr int kProdWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
-constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;  // 16 KiB of weights per stage and CTA
-constexpr uint32_t kTokBoxBytes = kTokRows * kBK * 2;  // 16 KiB
-constexpr uint32_t kSlotBytes = (kSlotTok / 2) * kBK * 2;  // 16 KiB of one slot's tokens per CTA
-constexpr uint32_t kRingBytes = 192 * 1024;
-// A tile meets up to kMaxSlots * 256 tokens of its expert in one pass over its
-// weights (one MMA per 256-token slot, each into its own TMEM buffer).  Two
-// slots keep an expert with 257..512 rows to a single weight pass; launches
-// whose chunks cannot exceed 256 rows per expert use one slot and a deeper ring.
-template <int kMaxSlots>
-struct RingCfg {
-    static constexpr uint32_t kStageBytes = kWBytes + kMaxSlots * kSlotBytes;  // 32 / 48 KiB
-    static constexpr int kStages = kRingBytes / kStageBytes;                   // 6 / 4
-};
+constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;         // 16 KiB: a CTA's weight rows of one k-chunk
+constexpr uint32_t kTokBytes = (kTileTok / 2) * kBK * 2;    // 16 KiB: a CTA's 128 token rows of one k-chunk
+constexpr uint32_t kStageBytes = kKS * (kWBytes + kTokBytes);  // 64 KiB
+constexpr int kStages = 3;
+constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 192 KiB
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
 constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (4 warp pairs x 2 ways x 2 KiB)
 
@@ -83,8 +76,6 @@ struct FfnGemmParams {
     int n_fblocks;         // pair feature blocks per expert: I/128 (GEMM1) or H/256 (GEMM2), rounded up
     int feat_per_cta;      // output features per CTA of a pair tile: 64 (GEMM1) or 128 (GEMM2)
     int w_rows_per_expert; // 2I for GEMM1, H for GEMM2
-    int up_offset;         // GEMM1: rows from a gate row to its up row (I)
-    int tok_block;         // tokens per tile (256)
     int out_cols;          // row length of the output (I for h, H for y / out_reduce)
     void *out;             // h or y
     float *out_reduce;
@@ -98,8 +89,8 @@ struct FfnGemmParams {
 constexpr int kQueue = 8;                            // slices published ahead of the slowest consumer
 
 struct FfnSmem {
-    uint64_t full[6];
-    uint64_t empty[6];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
@@ -114,9 +105,7 @@ struct FfnSmem {
 };
 
 struct TileInfo {
-    int e, f_blk, p0, n_valid, n_mma;   // n_valid <= tok_block tokens; n_mma: slot 0's N
-    int n_slots;                         // accumulator slots the tile uses (1 or 2)
-    int n_mma1;                          // slot 1's N (tokens 256..n_valid-1, rounded to 16)
+    int e, f_blk, p0, n_valid, n_mma;   // n_valid <= 256 tokens; n_mma: the MMA's N (rounded to 16)
 };
 
 // Work is dealt out tile by tile from a global counter, so a pair that finishes
@@ -142,11 +131,9 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
     t.f_blk = f_blk;
     const int off = P.expert_offsets[e];
     const int m_e = P.expert_offsets[e + 1] - off;
-    t.p0 = off + t_blk * P.tok_block;
-    t.n_valid = min(P.tok_block, m_e - t_blk * P.tok_block);
-    t.n_mma = (min(t.n_valid, kSlotTok) + 15) & ~15;
-    t.n_slots = t.n_valid > kSlotTok ? 2 : 1;
-    t.n_mma1 = t.n_slots == 2 ? ((t.n_valid - kSlotTok + 15) & ~15) : 0;
+    t.p0 = off + t_blk * kTileTok;
+    t.n_valid = min(kTileTok, m_e - t_blk * kTileTok);
+    t.n_mma = (t.n_valid + 15) & ~15;
     return t;
 }
 
@@ -172,13 +159,11 @@ struct SliceReader {
     }
 };
 
-template <int MODE, int kMaxSlots>
+template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const FfnGemmParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
-    constexpr int kStages = RingCfg<kMaxSlots>::kStages;
-    constexpr uint32_t kStageBytes = RingCfg<kMaxSlots>::kStageBytes;
     // queue consumers per entry: the MMA thread, the follower's producer, and
     // every epilogue warp of both CTAs (GEMM1: the gate warp of each pair only)
     constexpr uint32_t kQueueConsumers = 2 + 2 * (kSwiGLU ? kEpiWarps / 2 : kEpiWarps);
@@ -203,7 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             int tb = 0;
             if (e < P.E) {
                 const int m = P.expert_offsets[e + 1] - P.expert_offsets[e];
-                tb = (m + P.tok_block - 1) / P.tok_block;
+                tb = (m + kTileTok - 1) / kTileTok;
                 s_tb[e] = tb;
             }
             const int t = tb * P.n_fblocks;
@@ -237,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 
     const int total = S->total_slices;
     const uint32_t tmem_base = S->tmem_base;
-    const int num_k = (P.K + kBK - 1) / kBK;
+    const int num_k = (P.K + kBK * kKS - 1) / (kBK * kKS);   // ring stages per tile
     volatile int *abort_flag = &S->abort_flag;
 
     if (warp == kProdWarp) {
@@ -273,39 +258,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 if (slice < 0) break;
                 int se, sf, t_blk;
                 decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
-                // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows, GEMM2 128 rows
-                const int w_row = se * P.w_rows_per_expert + (sf * 2 + (int)rank) * P.feat_per_cta;
-                {
-                    const TileInfo ti = tile_info(se, sf, t_blk, P);
-                    // this CTA's half of each slot's token rows
-                    const int half0 = ti.n_mma / 2, half1 = ti.n_mma1 / 2;
-                    const int tok_row0 = ti.p0 + (int)rank * half0;
-                    const int tok_row1 = ti.p0 + kSlotTok + (int)rank * half1;
-                    const int n_box0 = (half0 + kTokRows - 1) / kTokRows;
-                    const int n_box1 = (half1 + kTokRows - 1) / kTokRows;
-                    const uint32_t bytes = kWBytes + (n_box0 + n_box1) * kTokBoxBytes;
-                    for (int kb = 0; kb < num_k; ++kb) {
-                        if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-                        unsigned char *st = tiles + stage * kStageBytes;
-                        const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
-                        const int kx = kb * kBK;
-                        if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * bytes);
-                        if (kSwiGLU) {
-                            // gate rows then the matching up rows, one 3-D box
-                            tma_load_3d_pair(st, &tmap_w, full_leader, kx, (sf * 2 + (int)rank) * P.feat_per_cta,
-                                             2 * se);
-                        } else {
-                            tma_load_2d_pair(st, &tmap_w, full_leader, kx, w_row);
-                        }
-                        for (int b = 0; b < n_box0; ++b)
-                            tma_load_2d_pair(st + kWBytes + b * kTokBoxBytes, &tmap_x, full_leader, kx,
-                                             tok_row0 + b * kTokRows);
-                        for (int b = 0; b < n_box1; ++b)
-                            tma_load_2d_pair(st + kWBytes + kSlotBytes + b * kTokBoxBytes, &tmap_x,
-                                             full_leader, kx, tok_row1 + b * kTokRows);
-                        ++issued;
-                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                    }
+                // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows
+                // (one 4-D box), GEMM2 128 rows; its token rows: half of the tile's N
+                const int f_row = (sf * 2 + (int)rank) * P.feat_per_cta;
+                const int w_row = se * P.w_rows_per_expert + f_row;
+                const TileInfo ti = tile_info(se, sf, t_blk, P);
+                const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
+                for (int kb = 0; kb < num_k; ++kb) {
+                    if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                    unsigned char *st = tiles + stage * kStageBytes;
+                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
+                    const int ch = kb * kKS;   // first k-chunk of the stage
+                    // full boxes land in both CTAs (rows or chunks past the tensor are zero-filled)
+                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
+                    if (kSwiGLU)
+                        tma_load_4d_pair(st, &tmap_w, full_leader, 0, f_row, 2 * se, ch);
+                    else
+                        tma_load_3d_pair(st, &tmap_w, full_leader, 0, w_row, ch);
+                    tma_load_3d_pair(st + kKS * kWBytes, &tmap_x, full_leader, 0, tok_row, ch);
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
             }
             if (!ok) {
@@ -343,38 +315,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                   {
                     const TileInfo ti = tile_info(se, sf, t_blk, P);
                     const uint32_t idesc = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
-                    const uint32_t idesc1 = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma1 > 0 ? ti.n_mma1 : 16);
-                    // slot 0 takes buffer `acc`, slot 1 (if any) the next buffer in the ring
-                    const int acc1 = acc ^ 1;
-                    const uint32_t acc1_phase = acc == 1 ? acc_phase ^ 1u : acc_phase;
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-                    if (ti.n_slots == 2 &&
-                        !mbar_wait_bounded(&S->tmem_empty[acc1], acc1_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d0 = tmem_base + (uint32_t)(acc * kSlotTok);
-                    const uint32_t d1 = tmem_base + (uint32_t)(acc1 * kSlotTok);
+                    const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
                     for (int kb = 0; kb < num_k; ++kb) {
                         if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t st = smem_u32(tiles + stage * kStageBytes);
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk) {
-                            const uint64_t wdesc = make_sw128_desc(st + kk * 32);
-                            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-                            tc_mma_f16_pair(d0, wdesc, make_sw128_desc(st + kWBytes + kk * 32), idesc, accum);
-                            if (kMaxSlots == 2 && ti.n_slots == 2)
-                                tc_mma_f16_pair(d1, wdesc, make_sw128_desc(st + kWBytes + kSlotBytes + kk * 32),
-                                                idesc1, accum);
+                        for (int c = 0; c < kKS; ++c) {
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk) {
+                                const uint64_t wdesc = make_sw128_desc(st + c * kWBytes + kk * 32);
+                                const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * kTokBytes + kk * 32);
+                                tc_mma_f16_pair(d, wdesc, tdesc, idesc, (kb > 0 || c > 0 || kk > 0) ? 1u : 0u);
+                            }
                         }
                         tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
                         if (++stage == kStages) { stage = 0; phase ^= 1u; }
                     }
                     if (!ok) break;
-                    // accumulators ready in both CTAs, slot by slot
-                    for (int sl = 0; sl < ti.n_slots; ++sl) {
-                        tc_commit_pair_mc(&S->tmem_full[acc], 0x3);
-                        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-                    }
+                    tc_commit_pair_mc(&S->tmem_full[acc], 0x3);    // accumulator ready in both CTAs
+                    if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
                   }
                 }
                 if (!ok) {
@@ -425,8 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
           int se, sf, t_blk;
           decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
           {
-           const TileInfo tinfo = tile_info(se, sf, t_blk, P);
-           for (int sl = 0; sl < tinfo.n_slots; ++sl) {
+           const TileInfo ti = tile_info(se, sf, t_blk, P);
+           do {   // one pass; `break` leaves it on a failed wait
             bool go;
             if (kSwiGLU) {
                 // same hand-over for the accumulator wait
@@ -445,14 +407,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 break;
             }
             tc_fence_after();
-            // this slot's tokens: [sl * 256, sl * 256 + 256) of the tile
-            TileInfo ti = tinfo;
-            ti.p0 += sl * kSlotTok;
-            ti.n_valid = min(kSlotTok, tinfo.n_valid - sl * kSlotTok);
-            ti.n_mma = sl == 0 ? tinfo.n_mma : tinfo.n_mma1;
             const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
             const bool f_ok = f < P.out_cols;
-            const uint32_t tbase = tmem_base + (uint32_t)(acc * kSlotTok) + ((uint32_t)(q * 32) << 16);
+            const uint32_t tbase = tmem_base + (uint32_t)(acc * kTileTok) + ((uint32_t)(q * 32) << 16);
 
             for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64) {
                 uint32_t r[32];
@@ -512,7 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_leader[acc]);   // release the pair's accumulator
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-           }
+           } while (0);
           }
         }
     }
@@ -541,36 +498,37 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix, box 64 cols x box_rows,
 // 128-byte swizzle, zero fill outside the matrix.
-// W13 [E][2][I][H] seen as the 3-D tensor (H, I, 2E): one box of 64 columns x
-// 64 feature rows x {gate, up} fills a CTA's 128 weight rows of a stage.
-static bool make_tmap_w13_bf16(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I, uint64_t H,
-                               uint32_t box_rows) {
+// A bf16 tensor map with 128-byte swizzled boxes whose innermost extent is one
+// 64-column k-chunk; the k-chunk index is the outermost dimension, so one box
+// brings kKS consecutive k-chunks of its rows.
+static bool make_tmap_kchunks(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims,
+                              const cuuint64_t *strides, const cuuint32_t *box) {
     auto enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {H, I, 2 * E};
-    cuuint64_t strides[2] = {H * 2, I * H * 2};
-    cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 2u};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+    cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-static bool make_tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
+// Rows [rows][K] (row stride K * 2 bytes) as (64, rows, K / 64).
+static bool make_tmap_rows(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t K,
                            uint32_t box_rows) {
-    auto enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
-    cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    const cuuint64_t dims[3] = {(cuuint64_t)kBK, rows, K / kBK};
+    const cuuint64_t strides[2] = {K * 2, (cuuint64_t)kBK * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, (cuuint32_t)kKS};
+    return make_tmap_kchunks(m, ptr, 3, dims, strides, box);
+}
+
+// W13 [E][2][I][H] as (64, I, 2E, H / 64): one box holds 64 gate rows of a
+// feature block followed by the 64 matching up rows, kKS k-chunks deep.
+static bool make_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I, uint64_t H) {
+    const cuuint64_t dims[4] = {(cuuint64_t)kBK, I, 2 * E, H / kBK};
+    const cuuint64_t strides[3] = {H * 2, I * H * 2, (cuuint64_t)kBK * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)kBK, (cuuint32_t)kRowsPerCta / 2, 2u, (cuuint32_t)kKS};
+    return make_tmap_kchunks(m, ptr, 4, dims, strides, box);
 }
 
 size_t ffn_tcgen05_smem(int E, bool swiglu) {
@@ -578,36 +536,19 @@ size_t ffn_tcgen05_smem(int E, bool swiglu) {
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
-template <int MODE, int kMaxSlots>
-static cudaError_t launch_gemm_slots(const CUtensorMap &tw, const CUtensorMap &tx,
-                                     const FfnGemmParams &P, int grid, uint32_t *counter,
-                                     cudaStream_t s) {
+template <int MODE>
+static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
+                               const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
     if (smem > configured) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE, kMaxSlots>,
+        cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
         configured = smem;
     }
-    ffn_gemm_tcgen05_kernel<MODE, kMaxSlots><<<grid, kFfnThreads, smem, s>>>(tw, tx, P, counter);
+    ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, P, counter);
     return cudaGetLastError();
-}
-
-template <int MODE>
-static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
-                               const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
-    if (P.tok_block > kSlotTok) return launch_gemm_slots<MODE, 2>(tw, tx, P, grid, counter, s);
-    return launch_gemm_slots<MODE, 1>(tw, tx, P, grid, counter, s);
-}
-
-// Rows one expert can receive in a launch over n_rows receive rows: a token
-// picks an expert at most once, so at most the chunk's tokens (n_rows / k when
-// nothing is clipped) and at most the capacity.
-static int64_t tok_count_of_launch(const moe_config &c, int64_t n_rows) {
-    int64_t m = (n_rows + c.k - 1) / c.k;
-    if (c.capacity >= 0 && c.capacity < m) m = c.capacity;
-    return m;
 }
 
 // Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
@@ -621,10 +562,10 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
     if (cerr != cudaSuccess) return cerr;
     CUtensorMap tw1, tx1, tw2, tx2;
-    if (!make_tmap_w13_bf16(&tw1, w13, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H, kRowsPerCta / 2) ||
-        !make_tmap_bf16(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTokRows) ||
-        !make_tmap_bf16(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
-        !make_tmap_bf16(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTokRows))
+    if (!make_tmap_w13(&tw1, w13, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H) ||
+        !make_tmap_rows(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTileTok / 2) ||
+        !make_tmap_rows(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
+        !make_tmap_rows(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTileTok / 2))
         return cudaErrorNotSupported;
 
     FfnGemmParams P1{};
@@ -634,21 +575,13 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P1.feat_per_cta = kRowsPerCta / 2;
     P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
     P1.w_rows_per_expert = 2 * c.I;
-    P1.up_offset = c.I;
-    // Two accumulator slots (up to 512 tokens per weight pass) save a second
-    // pass over a slice's weights for experts with 257..512 rows, but a 2-slot
-    // tile holds both TMEM buffers, so its epilogue no longer overlaps the next
-    // main loop.  That pays off when the main loop is long (K >= 4096) and some
-    // expert of the launch can hold more than 256 rows.
-    const bool many_rows = tok_count_of_launch(c, n_rows) > kSlotTok;
-    P1.tok_block = (many_rows && c.H >= 4096) ? 2 * kSlotTok : kSlotTok;
     P1.out_cols = c.I;
     P1.out = h;
     P1.k = c.k;
     P1.status = status;
-    // CTA pairs: an upper bound on the pair tiles is (n_rows / tok + E) * n_fblocks
+    // CTA pairs: an upper bound on the pair tiles is (n_rows / 256 + E) * n_fblocks
     const long long max_pairs = num_sms / 2;
-    long long g1 = (n_rows / P1.tok_block + c.E) * (long long)P1.n_fblocks;
+    long long g1 = (n_rows / kTileTok + c.E) * (long long)P1.n_fblocks;
     int grid1 = 2 * (int)(g1 < max_pairs ? g1 : max_pairs);
     cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, P1, grid1, counters, s);
     if (err != cudaSuccess) return err;
@@ -658,15 +591,13 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P2.feat_per_cta = kRowsPerCta;
     P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
     P2.w_rows_per_expert = c.H;
-    P2.up_offset = 0;
-    P2.tok_block = (many_rows && c.I >= 4096) ? 2 * kSlotTok : kSlotTok;
     P2.out_cols = c.H;
     P2.out = y;
     P2.out_reduce = out_reduce;
     P2.recv_token = recv_token;
     P2.recv_slot = recv_slot;
     P2.topk_w = topk_w;
-    long long g2 = (n_rows / P2.tok_block + c.E) * (long long)P2.n_fblocks;
+    long long g2 = (n_rows / kTileTok + c.E) * (long long)P2.n_fblocks;
     int grid2 = 2 * (int)(g2 < max_pairs ? g2 : max_pairs);
     if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, P2, grid2, counters + 1, s);
     return launch_gemm<kEpiStore>(tw2, tx2, P2, grid2, counters + 1, s);
