@@ -137,7 +137,10 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
     return t;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu in the bf16 epilogue: the fast exponential and reciprocal-based divide
+// (a few ulp in fp32) are far inside the bf16 rounding of h, and the IEEE divide
+// made the epilogue instruction-bound.  For g -> -inf the quotient is -0.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -427,18 +430,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     const int nc = min(16, ti.n_valid - cbase);
                     __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) +
                                        (size_t)(ti.p0 + cbase) * P.out_cols + f;
+                    // all 16 partner values into registers before the first store:
+                    // h and the exchange buffer are both generic pointers, so a load
+                    // after a store could not be moved ahead of it and every token
+                    // would wait for the previous one's whole chain
+                    float other[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) other[j] = theirs[j * 32 + lane];
+                    named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
                     if (f_ok) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             if (j < nc) {
                                 const float own = __uint_as_float(r[is_gate ? j : 16 + j]);
-                                const float other = theirs[j * 32 + lane];
-                                const float g = is_gate ? own : other, u = is_gate ? other : own;
+                                const float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
                                 h[(size_t)j * P.out_cols] = __float2bfloat16_rn(silu_f(g) * u);
                             }
                         }
                     }
-                    named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
                 } else if (MODE == kEpiStore) {
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
                     const int nc = min(32, ti.n_valid - c0);
