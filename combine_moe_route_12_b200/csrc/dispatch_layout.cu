@@ -34,6 +34,7 @@ namespace moe {
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kTokensPerWarp = kLayoutTileTokens / kLayoutWarps;
+constexpr int kLoadBatch = 8;              // warp steps whose loads are issued together
 constexpr uint32_t kFlagAggregate = 1u << 30;
 constexpr uint32_t kFlagInclusive = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1;
@@ -154,7 +155,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     int32_t *s_base = s_eoff + (E + 1);                      // [E]
     int32_t *s_cnt = s_base + E;                             // [kLayoutWarps][E]
     int32_t *s_rank = s_cnt + kLayoutWarps * E;              // [kLayoutTileTokens * k]
-    int32_t *s_split = s_rank + kLayoutTileTokens * k;       // [ep * ep] when it fits
+    int32_t *s_exp = s_rank + kLayoutTileTokens * k;         // [kLayoutTileTokens * k] expert or -1
+    int32_t *s_split = s_exp + kLayoutTileTokens * k;        // [ep * ep] when it fits
     __shared__ int32_t s_warp_tot[33];
     __shared__ uint32_t s_tile;
     const bool split_in_smem = ep * ep <= kSplitSmemMax;
@@ -176,30 +178,52 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
         for (int d = threadIdx.x; d <= ep; d += blockDim.x) rank_offsets[d] = s_eoff[d * epr];
     }
 
-    // 1) rank every kept assignment of this tile among the warp's rows of its expert
+    // 1) rank every kept assignment of this tile among the warp's rows of its expert.
+    // Warp w walks its kTokensPerWarp tokens G = 32 / k at a time (lane -> token
+    // b + lane / k, slot lane % k).  The experts of up to kLoadBatch steps are
+    // loaded before the first is ranked, so a walk costs a memory round trip per
+    // batch instead of per step; step 3 reads them back from shared memory.
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int t_tile0 = tb + tile * kLayoutTileTokens;
     const int G = 32 / k;                      // tokens per warp step
+    const int n_steps = (kTokensPerWarp + G - 1) / G;
     const unsigned lt_mask = (1u << lane) - 1u;
+    const int jl = lane % k;
     bool bad = false;
-    for (int b = 0; b < kTokensPerWarp; b += G) {
-        const int ti = wid * kTokensPerWarp + b + lane / k;  // token within the tile
-        const int j = lane % k;
-        const int t = t_tile0 + ti;
-        int e = -1 - lane;                     // unique sentinel: matches nobody
-        if (lane < G * k && b + lane / k < kTokensPerWarp && t < tb + tc) {
-            const size_t a = (size_t)t * k + j;
-            if (keep[a]) {
-                const int ev = topk_idx[a];
-                if (ev >= 0 && ev < E) e = ev;
-                else bad = true;
+    for (int s0 = 0; s0 < n_steps; s0 += kLoadBatch) {
+        uint8_t kv[kLoadBatch];
+        int ix[kLoadBatch];
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i) {
+            kv[i] = 0;
+            ix[i] = -1;
+            const int b = (s0 + i) * G;
+            const int t = t_tile0 + wid * kTokensPerWarp + b + lane / k;
+            if (s0 + i < n_steps && lane < G * k && b + lane / k < kTokensPerWarp && t < tb + tc) {
+                const size_t a = (size_t)t * k + jl;
+                kv[i] = __ldg(keep + a);
+                ix[i] = __ldg(topk_idx + a);
             }
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        if (e >= 0) s_rank[ti * k + j] = s_cnt[wid * E + e] + __popc(peers & lt_mask);
-        __syncwarp();
-        if (e >= 0 && (31 - __clz(peers)) == lane) s_cnt[wid * E + e] += __popc(peers);
-        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i) {
+            if (s0 + i >= n_steps) break;
+            const int b = (s0 + i) * G;
+            const int ti = wid * kTokensPerWarp + b + lane / k;   // token within the tile
+            const bool mine = lane < G * k && b + lane / k < kTokensPerWarp;
+            int e = -1;
+            if (kv[i]) {
+                if (ix[i] >= 0 && ix[i] < E) e = ix[i];
+                else bad = true;
+            }
+            if (mine) s_exp[ti * k + jl] = e;
+            const int me = e >= 0 ? e : -1 - lane;                 // unique sentinel: matches nobody
+            const unsigned peers = __match_any_sync(0xffffffffu, me);
+            if (e >= 0) s_rank[ti * k + jl] = s_cnt[wid * E + e] + __popc(peers & lt_mask);
+            __syncwarp();
+            if (e >= 0 && (31 - __clz(peers)) == lane) s_cnt[wid * E + e] += __popc(peers);
+            __syncwarp();
+        }
     }
     __syncthreads();
 
@@ -228,34 +252,31 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     }
     __syncthreads();
 
-    // 3) scatter rows (recv_token / recv_slot / pos) and count the split matrix
-    const int nt = min(kLayoutTileTokens, tb + tc - t_tile0);
+    // 3) scatter rows (recv_token / recv_slot / pos) and count the split matrix,
+    // with the same lane -> assignment map as step 1
     const int tpr = tc / ep, epr = E / ep;
-    for (int i = threadIdx.x; i < nt * k; i += blockDim.x) {
-        const int ti = i / k, j = i % k;
+    for (int st = 0; st < n_steps; ++st) {
+        const int b = st * G;
+        const int ti = wid * kTokensPerWarp + b + lane / k;
         const int t = t_tile0 + ti;
-        const size_t a = (size_t)t * k + j;
+        const bool mine = lane < G * k && b + lane / k < kTokensPerWarp && t < tb + tc;
         int p = -1;
         int key = -1;
-        if (keep[a]) {
-            const int e = topk_idx[a];
-            if (e >= 0 && e < E) {
-                const int w = ti / kTokensPerWarp;
-                const long long row = (long long)s_base[e] + s_cnt[w * E + e] + s_rank[ti * k + j];
-                if (row >= 0 && row < n_rows_max) {
-                    p = (int)row;
-                    recv_token[p] = t;
-                    recv_slot[p] = j;
-                    key = ((t - tb) / tpr) * ep + e / epr;
-                } else {
-                    bad = true;
-                }
+        const int e = mine ? s_exp[ti * k + jl] : -1;
+        if (mine && e >= 0) {
+            const long long row = (long long)s_base[e] + s_cnt[wid * E + e] + s_rank[ti * k + jl];
+            if (row >= 0 && row < n_rows_max) {
+                p = (int)row;
+                recv_token[p] = t;
+                recv_slot[p] = jl;
+                key = ((t - tb) / tpr) * ep + e / epr;
+            } else {
+                bad = true;
             }
         }
-        pos[(size_t)(t - tb) * k + j] = p;
-        const unsigned active = __activemask();
-        const unsigned peers = __match_any_sync(active, key);
-        if (key >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) {
+        if (mine) pos[(size_t)(t - tb) * k + jl] = p;
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) {
             if (split_in_smem) atomicAdd(&s_split[key], __popc(peers));
             else atomicAdd(&send_splits[key], __popc(peers));
         }
@@ -271,7 +292,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
 size_t layout_scatter_smem(const moe_config &c) {
     const size_t split = (size_t)c.ep * c.ep <= (size_t)kSplitSmemMax ? (size_t)c.ep * c.ep : 0;
     return sizeof(int32_t) * ((size_t)(c.E + 1) + c.E + (size_t)kLayoutWarps * c.E +
-                              (size_t)kLayoutTileTokens * c.k + split);
+                              2 * (size_t)kLayoutTileTokens * c.k + split);
 }
 
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,

@@ -62,6 +62,7 @@ constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
 constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;         // 16 KiB: a CTA's weight rows of one k-chunk
 constexpr uint32_t kTokBytes = (kTileTok / 2) * kBK * 2;    // 16 KiB: a CTA's 128 token rows of one k-chunk
 constexpr uint32_t kStageBytes = kKS * (kWBytes + kTokBytes);  // 64 KiB
+constexpr int kSmallBoxRows = 32;                            // token box of tiles with N <= 64
 constexpr int kStages = 3;
 constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 192 KiB
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
@@ -165,6 +166,7 @@ struct SliceReader {
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+    const __grid_constant__ CUtensorMap tmap_xs,
     const FfnGemmParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
     // queue consumers per entry: the MMA thread, the follower's producer, and
@@ -217,7 +219,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
         S->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kProdWarp && lane == 0) { tma_prefetch_desc(&tmap_w); tma_prefetch_desc(&tmap_x); }
+    if (warp == kProdWarp && lane == 0) {
+        tma_prefetch_desc(&tmap_w);
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_xs);
+    }
     if (warp == kMmaWarp) { tmem_alloc_pair(&S->tmem_base, kTmemCols); tmem_relinquish_pair(); }
     tc_fence_before();
     cluster_sync_all();      // barriers of both CTAs initialised, TMEM allocated
@@ -267,18 +273,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 const int w_row = se * P.w_rows_per_expert + f_row;
                 const TileInfo ti = tile_info(se, sf, t_blk, P);
                 const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
+                // a tile of an expert's short last token block takes a 32-row token box:
+                // fewer bytes through L2 for the same stage slot
+                const bool small_box = ti.n_mma / 2 <= kSmallBoxRows;
+                const uint32_t stage_bytes = small_box ? kKS * (kWBytes + kSmallBoxRows * kBK * 2) : kStageBytes;
                 for (int kb = 0; kb < num_k; ++kb) {
                     if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     unsigned char *st = tiles + stage * kStageBytes;
                     const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
                     const int ch = kb * kKS;   // first k-chunk of the stage
                     // full boxes land in both CTAs (rows or chunks past the tensor are zero-filled)
-                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
+                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * stage_bytes);
                     if (kSwiGLU)
                         tma_load_4d_pair(st, &tmap_w, full_leader, 0, f_row, 2 * se, ch);
                     else
                         tma_load_3d_pair(st, &tmap_w, full_leader, 0, w_row, ch);
-                    tma_load_3d_pair(st + kKS * kWBytes, &tmap_x, full_leader, 0, tok_row, ch);
+                    tma_load_3d_pair(st + kKS * kWBytes, small_box ? &tmap_xs : &tmap_x, full_leader, 0, tok_row, ch);
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -321,6 +331,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
+                    // k-chunk stride inside the stage's token box (32 or 128 rows)
+                    const uint32_t tchunk = ti.n_mma / 2 <= kSmallBoxRows ? kSmallBoxRows * kBK * 2 : kTokBytes;
                     for (int kb = 0; kb < num_k; ++kb) {
                         if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -330,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 #pragma unroll
                             for (int kk = 0; kk < kBK / 16; ++kk) {
                                 const uint64_t wdesc = make_sw128_desc(st + c * kWBytes + kk * 32);
-                                const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * kTokBytes + kk * 32);
+                                const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * tchunk + kk * 32);
                                 tc_mma_f16_pair(d, wdesc, tdesc, idesc, (kb > 0 || c > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
@@ -546,7 +558,7 @@ size_t ffn_tcgen05_smem(int E, bool swiglu) {
 }
 
 template <int MODE>
-static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
+static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx, const CUtensorMap &txs,
                                const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
@@ -556,7 +568,7 @@ static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx,
         if (err != cudaSuccess) return err;
         configured = smem;
     }
-    ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, P, counter);
+    ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
     return cudaGetLastError();
 }
 
@@ -570,7 +582,10 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     // the two launches' work counters start at zero
     cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
     if (cerr != cudaSuccess) return cerr;
-    CUtensorMap tw1, tx1, tw2, tx2;
+    CUtensorMap tw1, tx1, tw2, tx2, tx1s, tx2s;
+    if (!make_tmap_rows(&tx1s, xr, (uint64_t)n_rows, (uint64_t)c.H, kSmallBoxRows) ||
+        !make_tmap_rows(&tx2s, h, (uint64_t)n_rows, (uint64_t)c.I, kSmallBoxRows))
+        return cudaErrorNotSupported;
     if (!make_tmap_w13(&tw1, w13, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H) ||
         !make_tmap_rows(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTileTok / 2) ||
         !make_tmap_rows(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
@@ -592,7 +607,7 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     const long long max_pairs = num_sms / 2;
     long long g1 = (n_rows / kTileTok + c.E) * (long long)P1.n_fblocks;
     int grid1 = 2 * (int)(g1 < max_pairs ? g1 : max_pairs);
-    cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, P1, grid1, counters, s);
+    cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, tx1s, P1, grid1, counters, s);
     if (err != cudaSuccess) return err;
 
     FfnGemmParams P2 = P1;
@@ -608,8 +623,8 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     P2.topk_w = topk_w;
     long long g2 = (n_rows / kTileTok + c.E) * (long long)P2.n_fblocks;
     int grid2 = 2 * (int)(g2 < max_pairs ? g2 : max_pairs);
-    if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, P2, grid2, counters + 1, s);
-    return launch_gemm<kEpiStore>(tw2, tx2, P2, grid2, counters + 1, s);
+    if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+    return launch_gemm<kEpiStore>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
 }
 
 }  // namespace moe

@@ -3,11 +3,12 @@
 // top-k is saved state).
 //
 // A group of LPT lanes (8, 16 or 32) per token, 32/LPT tokens per warp at a
-// time.  Lane l of a group holds the biased logits of experts l, l+LPT, ...
-// k rounds of a butterfly arg-max inside the group (value descending, lower
-// expert index first among equal values) pick the experts in rank order; lane
-// j of the group keeps slot j.  Narrow groups keep each round's shuffle chain
-// short and several tokens in flight per warp.
+// time.  Lane l of a group holds the biased logits of experts l, l+LPT, ... as
+// 64-bit rank keys (value descending, lower expert index first among equal
+// values).  k rounds of a butterfly max over the lanes' best remaining keys pick
+// the experts in rank order; lane j of the group keeps slot j, and only the lane
+// whose key won rescans its values.  Narrow groups keep each round's shuffle
+// chain short and several tokens in flight per warp.
 // The weights w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) use a fixed fp32
 // exponential (Cody & Waite reduction, degree-7 Taylor polynomial, every step
 // one IEEE-rounded operation) and a slot-ordered sum, so they are bit-exact
@@ -45,10 +46,24 @@ __device__ __forceinline__ float det_exp_nonpos(float r) {
     return __fmul_rn(p, two_n);
 }
 
-// (va, a) ranks before (vb, b)?  Larger value first, lower index among equals.
-__device__ __forceinline__ bool ranks_before(float va, int a, float vb, int b) {
-    return (va > vb) || (va == vb && a < b);
+
+// Rank key of (biased logit l, expert e): larger l first, lower e among equal
+// l.  The fp32 bits are mapped to an unsigned order (negatives flipped) in the
+// high word and the complemented expert index fills the low word, so one 64-bit
+// comparison ranks two candidates; 0 is below every real key (empty slot).
+__device__ __forceinline__ uint64_t rank_key(float l, int e) {
+    const uint32_t u = __float_as_uint(l);
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((uint64_t)ord << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
 }
+__device__ __forceinline__ float key_value(uint64_t key) {
+    const uint32_t ord = (uint32_t)(key >> 32);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+}
+__device__ __forceinline__ int key_expert(uint64_t key) {
+    return (int)(0xFFFFFFFFu - (uint32_t)key);
+}
+__device__ __forceinline__ uint64_t max_u64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 
 template <int LPT, int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(
@@ -71,46 +86,44 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
         const long long t = t0 + g;
         const bool valid = t < T;
         const float *row = logits + (size_t)(valid ? t : 0) * E;
-        float v[VPL];
-        uint32_t taken = 0;
+        uint64_t key[VPL];
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
             const int e = gl + LPT * i;
+            key[i] = 0;
             if (valid && e < E) {
+                // the add also turns -0 into +0, so the key order matches IEEE ==
                 float l = __fadd_rn(__ldg(row + e), bias ? __ldg(bias + e) : 0.0f);
                 if (!isfinite(l)) {
                     nonfinite = true;
                     if (isnan(l)) l = -INFINITY;  // keep the ranking a total order
                 }
-                v[i] = l;
-            } else {
-                v[i] = -INFINITY;
-                taken |= 1u << i;  // padding never wins
+                key[i] = rank_key(l, e);
             }
         }
-        float my_v = 0.0f;  // slot `gl`'s biased logit
-        int my_e = 0;
-        for (int j = 0; j < k; ++j) {
-            bool has = false;
-            float bv = 0.0f;
-            int be = 0x7fffffff;
+        // each lane keeps its best remaining key; a round takes the group's best
+        // and only the lane that held it looks for its next one
+        uint64_t best = 0;
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int e = gl + LPT * i;
-                if (!((taken >> i) & 1u) && (!has || ranks_before(v[i], e, bv, be))) {
-                    has = true; bv = v[i]; be = e;
+        for (int i = 0; i < VPL; ++i) best = max_u64(best, key[i]);
+        uint64_t my_key = 0;  // slot `gl`'s key
+        for (int j = 0; j < k; ++j) {
+            uint64_t top = best;
+#pragma unroll
+            for (int off = LPT / 2; off > 0; off >>= 1)
+                top = max_u64(top, __shfl_xor_sync(0xffffffffu, top, off));
+            if (gl == j) my_key = top;
+            if (best == top && top != 0) {
+                best = 0;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    if (key[i] == top) key[i] = 0;
+                    best = max_u64(best, key[i]);
                 }
             }
-#pragma unroll
-            for (int off = LPT / 2; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                const bool oh = __shfl_xor_sync(0xffffffffu, (int)has, off) != 0;
-                if (oh && (!has || ranks_before(ov, oe, bv, be))) { has = true; bv = ov; be = oe; }
-            }
-            if (has && (be % LPT) == gl) taken |= 1u << (be / LPT);
-            if (gl == j) { my_v = bv; my_e = be; }
         }
+        const float my_v = key_value(my_key);
+        const int my_e = key_expert(my_key);
         const float m = __shfl_sync(0xffffffffu, my_v, glane0);
         const float ex = (gl < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
         float S = 0.0f;
