@@ -147,14 +147,21 @@ __global__ void __launch_bounds__(kGatherThreads) clip_gather_kernel(
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
     __syncthreads();
     int ex[kGatherPerThread], slot[kGatherPerThread];
+    // all of the thread's expert ids, then all their counts, are loaded before the
+    // first warp-collective step, so the loads overlap instead of queueing
 #pragma unroll
     for (int i = 0; i < kGatherPerThread; ++i) {
         const size_t a = a0 + (size_t)i * kGatherThreads + threadIdx.x;
-        int e = -1;
-        if (a < total) {
-            const int ev = __ldg(topk_idx + a);
-            if (ev >= 0 && ev < E && C >= 0 && __ldg(counts + ev) > C && C > 0) e = ev;
-        }
+        ex[i] = a < total ? __ldg(topk_idx + a) : -1;
+    }
+    int cnt[kGatherPerThread];
+#pragma unroll
+    for (int i = 0; i < kGatherPerThread; ++i)
+        cnt[i] = (ex[i] >= 0 && ex[i] < E) ? __ldg(counts + ex[i]) : 0;
+#pragma unroll
+    for (int i = 0; i < kGatherPerThread; ++i) {
+        const int ev = ex[i];
+        const int e = (ev >= 0 && ev < E && C > 0 && cnt[i] > C) ? ev : -1;
         ex[i] = e;
         slot[i] = -1;
         const unsigned active = __activemask();
@@ -199,7 +206,20 @@ __global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
     uint64_t key;
     if (n <= smem_keys) {
         uint64_t *s_keys = reinterpret_cast<uint64_t *>(s_raw);
-        for (int i = threadIdx.x; i < n; i += blockDim.x) s_keys[i] = __ldcg(mine + i);
+        // eight loads in flight per thread before the stores to shared memory
+        for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+            uint64_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * (int)blockDim.x;
+                v[u] = i < n ? __ldcg(mine + i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * (int)blockDim.x;
+                if (i < n) s_keys[i] = v[u];
+            }
+        }
         __syncthreads();
         key = radix_select_desc(
             [&](auto f) {

@@ -44,6 +44,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
 }
 
+constexpr int kCombineBatch = 4;   // expert rows of a token loaded together
+
 // bf16 storage: one uint4 = 8 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
     int tb, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
@@ -59,14 +61,24 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
     __syncthreads();
     for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < k; ++j) {
-            const int p = s_pos[j];
-            if (p < 0) continue;
-            float f[8];
-            unpack8(__ldg(y + (size_t)p * row_vecs + v), f);
-            const float w = s_w[j];
+        for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
+            // the batch's rows are loaded before the first is added, so one
+            // thread has up to kCombineBatch loads in flight; the adds keep slot order
+            uint4 u[kCombineBatch];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(w, f[q], acc[q]);
+            for (int jj = 0; jj < kCombineBatch; ++jj) {
+                const int p = j0 + jj < k ? s_pos[j0 + jj] : -1;
+                u[jj] = p >= 0 ? __ldg(y + (size_t)p * row_vecs + v) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int jj = 0; jj < kCombineBatch; ++jj) {
+                if (j0 + jj >= k || s_pos[j0 + jj] < 0) continue;
+                float f[8];
+                unpack8(u[jj], f);
+                const float w = s_w[j0 + jj];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(w, f[q], acc[q]);
+            }
         }
         uint4 o;
         o.x = pack_bf16x2(acc[0], acc[1]);
