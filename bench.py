@@ -49,7 +49,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": 1558.385664e6, "src": "ff2c956c69a2ac4b"},
+    "qwen3_30b_a3b": {"bytes": 1558.534912e6, "src": "81a9932ff07c390d"},
 }
 
 
