@@ -184,16 +184,24 @@ def kernels_per_step(wl) -> int:
     return 1 + clip + wl.n_chunks * 6
 
 
-def algorithmic(wl, n_kept_chunks):
-    """Bytes / flops the method must move or compute (nothing for dropped rows)."""
+def algorithmic(wl, n_kept_chunks, active_chunks):
+    """Bytes / flops the method must move or compute (nothing for dropped rows).
+
+    ffn_bytes: per layer pass, the weights of every expert with a row in each
+    chunk (each chunk streams them once), the receive rows read by GEMM1, h
+    written and read back, and y written (decode form: the dense fp32 buffer
+    read and written once instead)."""
     b = wl.elem_bytes
     N = sum(n_kept_chunks)
     tok_bytes = wl.T * wl.H * b
     row_bytes = N * wl.H * b
+    w_bytes = sum(active_chunks) * 3 * wl.H * wl.I * b
+    out_bytes = 2 * wl.T * wl.H * 4 if wl.reduce_dense else row_bytes
     return {
         "permute_bytes": tok_bytes + row_bytes,
         "combine_bytes": (0 if wl.reduce_dense else row_bytes) + tok_bytes,
         "ffn_flops": 6.0 * wl.H * wl.I * N,
+        "ffn_bytes": w_bytes + row_bytes + 2 * N * wl.I * b + out_bytes,
         "N": N,
     }
 
@@ -495,12 +503,13 @@ def run_ours(args):
         raise RuntimeError("device status bits set during the breakdown pass")
     eager_step_ms = step_sum
     breakdown_mode = "graph" if bd_graph is not None else "eager"
-    n_kept = []
+    n_kept, n_active = [], []
     for c in range(wl.n_chunks):
         moe.moe_dispatch_layout(cfg, c * B.tc, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
                                 B.pos, B.spl, None, B.ws)
         n_kept.append(int(B.eoff[wl.E].item()))
-    alg = algorithmic(wl, n_kept)
+        n_active.append(int(((B.eoff[1:] - B.eoff[:-1]) > 0).sum().item()))
+    alg = algorithmic(wl, n_kept, n_active)
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -554,6 +563,11 @@ def run_ours(args):
         ffn_s = stage_ms["grouped_ffn"] / 1e3
         dc_s = (stage_ms["permute"] + stage_ms["combine"]) / 1e3
         ffn_tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
+        ffn_gbs = alg["ffn_bytes"] / ffn_s / 1e9 if ffn_s > 0 else None
+        # the binding roof: HBM when the pass's flop per byte is below the ridge
+        t_flop = alg["ffn_flops"] / (peaks["bf16_tflops"] * 1e12)
+        t_byte = alg["ffn_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        hbm_bound = t_byte > t_flop
         dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
         src = kernel_src_hash()
         tr = FFN_TRAFFIC.get(wl.name)
@@ -563,17 +577,25 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
             "config": workload_config(wl, world, use_graph),
-            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2)",
-                         "bound": "tensor", "achieved": ffn_tflops,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": ffn_tflops / peaks["bf16_tflops"] if ffn_tflops else None,
-                         "traffic": traffic, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "algorithmic_per_launch": f"6*H*I*N = {alg['ffn_flops']:.4g} flop over N={alg['N']} kept rows"},
+            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass)",
+                         "bound": "hbm" if hbm_bound else "tensor",
+                         "achieved": ffn_gbs if hbm_bound else ffn_tflops,
+                         "peak": peaks["hbm_gbs"] if hbm_bound else peaks["bf16_tflops"],
+                         "unit": "GB/s" if hbm_bound else "TFLOP/s",
+                         "frac": (ffn_gbs / peaks["hbm_gbs"] if hbm_bound else ffn_tflops / peaks["bf16_tflops"])
+                         if ffn_s > 0 else None,
+                         "traffic": traffic,
+                         "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else "bf16_tflops (burst)"),
+                         "algorithmic_per_launch": f"{alg['ffn_bytes']:.4g} B and 6*H*I*N = {alg['ffn_flops']:.4g} flop "
+                                                   f"over N={alg['N']} kept rows",
+                         "tensor_frac": ffn_tflops / peaks["bf16_tflops"] if ffn_tflops else None,
+                         "hbm_frac": ffn_gbs / peaks["hbm_gbs"] if ffn_gbs else None},
             "dispatch_combine": {"achieved_gbs": dc_gbs, "peak_gbs": peaks["hbm_gbs"],
                                  "frac": dc_gbs / peaks["hbm_gbs"] if dc_gbs else None,
                                  "bytes_per_step": alg["permute_bytes"] + alg["combine_bytes"],
                                  "peak_source": f"{peak_src} hbm_gbs"},
             "ffn_tflops": ffn_tflops,
+            "ffn_gbs": ffn_gbs,
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "breakdown_step_ms": round(eager_step_ms, 4),
             "breakdown_mode": breakdown_mode,
