@@ -53,12 +53,20 @@ FFN_TRAFFIC = {
 }
 
 
+def workload_of(args):
+    from combine_moe_route_12_b200.workload import WORKLOADS
+    wl = WORKLOADS[args.config]
+    return wl if args.chunks is None else wl.with_(n_chunks=args.chunks)
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--config", default="qwen3_30b_a3b")
+    p.add_argument("--chunks", type=int, default=None,
+                   help="override the workload's dispatch chunk count (e.g. 1 for the unchunked DSV3 prefill FFN)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
@@ -339,7 +347,7 @@ def run_reference(args):
     import numpy as np
     import torch
     from combine_moe_route_12_b200.workload import WORKLOADS, make_inputs
-    wl = WORKLOADS[args.config]
+    wl = workload_of(args)
     # inputs drawn on the CPU generator (no GPU needed for this arm)
     torch.manual_seed(0)
     inp = make_inputs(wl, "cpu", seed=args.seed, weights=False)
@@ -407,7 +415,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
     from combine_moe_route_12_b200 import moe
     from combine_moe_route_12_b200.workload import WORKLOADS, make_inputs
-    wl = WORKLOADS[args.config]
+    wl = workload_of(args)
     cfg = moe.config_from_workload(wl)
     peaks, peak_src = load_peaks()
     inp = make_inputs(wl, dev, seed=args.seed)
@@ -571,7 +579,7 @@ def run_ours(args):
         dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
         src = kernel_src_hash()
         tr = FFN_TRAFFIC.get(wl.name)
-        traffic = tr["bytes"] if tr and tr.get("src") == src else None
+        traffic = tr["bytes"] if tr and tr.get("src") == src and tr.get("chunks", 1) == wl.n_chunks else None
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

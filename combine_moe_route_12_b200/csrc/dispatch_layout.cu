@@ -10,7 +10,8 @@
 //
 //   layout_hist     per-expert kept counts of the chunk (shared-memory
 //                   histogram, one global atomic per CTA and expert);
-//   layout_scatter  one CTA per 256-token tile, tiles taken in launch order
+//   layout_scatter  one CTA per tile of 64, 128 or 256 tokens (the smallest that
+//                   keeps the launch within max(64, tokens / 256) tiles), taken in launch order
 //                   from an atomic ticket.  Each tile ranks its assignments
 //                   per expert in token order (warps walk their tokens with
 //                   __match_any_sync), publishes its per-expert counts, and
@@ -33,7 +34,6 @@ namespace moe {
 
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
-constexpr int kTokensPerWarp = kLayoutTileTokens / kLayoutWarps;
 constexpr int kLoadBatch = 8;              // warp steps whose loads are issued together
 constexpr uint32_t kFlagAggregate = 1u << 30;
 constexpr uint32_t kFlagInclusive = 2u << 30;
@@ -143,7 +143,7 @@ __device__ __forceinline__ bool lookback_prefix(const uint32_t *tile_state, int 
 }
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
-    int tb, int tc, int k, int E, int ep, int64_t n_rows_max,
+    int tb, int tc, int k, int E, int ep, int tile_tokens, int64_t n_rows_max,
     const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ keep,
     const int32_t *__restrict__ chunk_counts, uint32_t *__restrict__ ticket,
     uint32_t *__restrict__ tile_state, int32_t *__restrict__ expert_offsets,
@@ -154,9 +154,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     int32_t *s_eoff = s_dyn;                                 // [E + 1]
     int32_t *s_base = s_eoff + (E + 1);                      // [E]
     int32_t *s_cnt = s_base + E;                             // [kLayoutWarps][E]
-    int32_t *s_rank = s_cnt + kLayoutWarps * E;              // [kLayoutTileTokens * k]
-    int32_t *s_exp = s_rank + kLayoutTileTokens * k;         // [kLayoutTileTokens * k] expert or -1
-    int32_t *s_split = s_exp + kLayoutTileTokens * k;        // [ep * ep] when it fits
+    int32_t *s_rank = s_cnt + kLayoutWarps * E;              // [tile_tokens * k]
+    int32_t *s_exp = s_rank + tile_tokens * k;               // [tile_tokens * k] expert or -1
+    int32_t *s_split = s_exp + tile_tokens * k;              // [ep * ep] when it fits
     __shared__ int32_t s_warp_tot[33];
     __shared__ uint32_t s_tile;
     const bool split_in_smem = ep * ep <= kSplitSmemMax;
@@ -179,14 +179,15 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     }
 
     // 1) rank every kept assignment of this tile among the warp's rows of its expert.
-    // Warp w walks its kTokensPerWarp tokens G = 32 / k at a time (lane -> token
+    // Warp w walks its tokens_per_warp tokens G = 32 / k at a time (lane -> token
     // b + lane / k, slot lane % k).  The experts of up to kLoadBatch steps are
     // loaded before the first is ranked, so a walk costs a memory round trip per
     // batch instead of per step; step 3 reads them back from shared memory.
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int t_tile0 = tb + tile * kLayoutTileTokens;
+    const int t_tile0 = tb + tile * tile_tokens;
+    const int tokens_per_warp = tile_tokens / kLayoutWarps;   // 8, 16 or 32
     const int G = 32 / k;                      // tokens per warp step
-    const int n_steps = (kTokensPerWarp + G - 1) / G;
+    const int n_steps = (tokens_per_warp + G - 1) / G;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int jl = lane % k;
     bool bad = false;
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
             kv[i] = 0;
             ix[i] = -1;
             const int b = (s0 + i) * G;
-            const int t = t_tile0 + wid * kTokensPerWarp + b + lane / k;
-            if (s0 + i < n_steps && lane < G * k && b + lane / k < kTokensPerWarp && t < tb + tc) {
+            const int t = t_tile0 + wid * tokens_per_warp + b + lane / k;
+            if (s0 + i < n_steps && lane < G * k && b + lane / k < tokens_per_warp && t < tb + tc) {
                 const size_t a = (size_t)t * k + jl;
                 kv[i] = __ldg(keep + a);
                 ix[i] = __ldg(topk_idx + a);
@@ -209,8 +210,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
         for (int i = 0; i < kLoadBatch; ++i) {
             if (s0 + i >= n_steps) break;
             const int b = (s0 + i) * G;
-            const int ti = wid * kTokensPerWarp + b + lane / k;   // token within the tile
-            const bool mine = lane < G * k && b + lane / k < kTokensPerWarp;
+            const int ti = wid * tokens_per_warp + b + lane / k;   // token within the tile
+            const bool mine = lane < G * k && b + lane / k < tokens_per_warp;
             int e = -1;
             if (kv[i]) {
                 if (ix[i] >= 0 && ix[i] < E) e = ix[i];
@@ -257,9 +258,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     const int tpr = tc / ep, epr = E / ep;
     for (int st = 0; st < n_steps; ++st) {
         const int b = st * G;
-        const int ti = wid * kTokensPerWarp + b + lane / k;
+        const int ti = wid * tokens_per_warp + b + lane / k;
         const int t = t_tile0 + ti;
-        const bool mine = lane < G * k && b + lane / k < kTokensPerWarp && t < tb + tc;
+        const bool mine = lane < G * k && b + lane / k < tokens_per_warp && t < tb + tc;
         int p = -1;
         int key = -1;
         const int e = mine ? s_exp[ti * k + jl] : -1;
@@ -289,10 +290,10 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     if (bad) raise_status(status, MOE_DEV_BAD_INDEX);
 }
 
-size_t layout_scatter_smem(const moe_config &c) {
+size_t layout_scatter_smem(const moe_config &c, int tile_tokens) {
     const size_t split = (size_t)c.ep * c.ep <= (size_t)kSplitSmemMax ? (size_t)c.ep * c.ep : 0;
     return sizeof(int32_t) * ((size_t)(c.E + 1) + c.E + (size_t)kLayoutWarps * c.E +
-                              2 * (size_t)kLayoutTileTokens * c.k + split);
+                              2 * (size_t)tile_tokens * c.k + split);
 }
 
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
@@ -306,7 +307,8 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
     uint32_t *ticket = ws_at<uint32_t>(ws, L.ticket);
     int32_t *chunk_counts = ws_at<int32_t>(ws, L.chunk_counts);
     uint32_t *tile_state = ws_at<uint32_t>(ws, L.tile_state);
-    const int n_tiles = (tc + kLayoutTileTokens - 1) / kLayoutTileTokens;
+    const int tile_tokens = layout_tile_tokens(tc);
+    const int n_tiles = (tc + tile_tokens - 1) / tile_tokens;
     // ticket, chunk counts and the tiles' look-back descriptors start at zero
     const size_t clear_bytes = L.tile_state - L.ticket + sizeof(uint32_t) * (size_t)n_tiles * c.E;
     cudaError_t err = cudaMemsetAsync(ws_at<char>(ws, L.ticket), 0, clear_bytes, s);
@@ -321,7 +323,7 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
         layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, s>>>(
             tb, tc, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
-        const size_t smem = layout_scatter_smem(c);
+        const size_t smem = layout_scatter_smem(c, tile_tokens);
         static size_t configured = 48 * 1024;
         if (smem > configured) {
             err = cudaFuncSetAttribute(layout_scatter_kernel,
@@ -330,7 +332,7 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
             configured = smem;
         }
         layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, s>>>(
-            tb, tc, c.k, c.E, c.ep, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
+            tb, tc, c.k, c.E, c.ep, tile_tokens, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
             expert_offsets, rank_offsets, recv_token, recv_slot, pos, send_splits, status);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
@@ -417,7 +419,8 @@ extern "C" moe_status moe_dispatch_layout_noalloc(
     const moe_config &c = *cfg;
     if (tok_begin < 0 || tok_count < 0 || (int64_t)tok_begin + tok_count > c.T || tok_count % c.ep != 0)
         return report_error(MOE_ERR_INVALID_ARG, "token range outside [0, T) or not divisible by ep");
-    const int n_tiles = (tok_count + kLayoutTileTokens - 1) / kLayoutTileTokens;
+    const int tile_tokens = layout_tile_tokens(tok_count);
+    const int n_tiles = (tok_count + tile_tokens - 1) / tile_tokens;
     if (n_tiles > kNoAllocMaxTiles)
         return report_error(MOE_ERR_UNSUPPORTED,
                             "moe_dispatch_layout_noalloc handles at most 16384 tokens per call");
@@ -445,12 +448,12 @@ extern "C" moe_status moe_dispatch_layout_noalloc(
         layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, stream>>>(
             tok_begin, tok_count, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         err = cudaGetLastError();
-        const size_t smem = layout_scatter_smem(c);
+        const size_t smem = layout_scatter_smem(c, tile_tokens);
         if (err == cudaSuccess && smem > 48 * 1024)
             err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err == cudaSuccess) {
             layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, stream>>>(
-                tok_begin, tok_count, c.k, c.E, c.ep, max_recv_rows_of(c, tok_count), topk_idx, keep,
+                tok_begin, tok_count, c.k, c.E, c.ep, tile_tokens, max_recv_rows_of(c, tok_count), topk_idx, keep,
                 chunk_counts, ticket, tile_state, expert_offsets, rank_offsets, recv_token, recv_slot,
                 pos, send_splits, st_word);
             err = cudaGetLastError();

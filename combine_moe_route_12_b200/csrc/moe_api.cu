@@ -21,7 +21,6 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
                                    int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
                                    int32_t *send_splits, int32_t *splits_host, void *ws,
                                    int64_t n_rows_max, cudaStream_t s, int num_sms);
-size_t layout_scatter_smem(const moe_config &c);
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
                            int tc, void *xr, cudaStream_t s);
 cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,

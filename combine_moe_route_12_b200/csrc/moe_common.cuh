@@ -14,7 +14,23 @@ namespace moe {
 // ---------------------------------------------------------------- constants
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
-constexpr int kLayoutTileTokens = 256;      // tokens per dispatch-layout tile
+constexpr int kLayoutTileTokens = 256;      // largest dispatch-layout tile (tokens)
+constexpr int kLayoutMinTiles = 64;         // tiles shrink while there are at most this many
+
+// A dispatch-layout launch over tc tokens uses tiles of 64, 128 or 256 tokens:
+// the smallest that keeps the tile count within max(64, ceil(tc / 256)), so a
+// chunk of a few thousand tokens still spreads over dozens of CTAs.
+inline int layout_tile_tokens(int64_t tc) {
+    const int64_t cap = (tc + kLayoutTileTokens - 1) / kLayoutTileTokens;
+    const int64_t max_tiles = cap > kLayoutMinTiles ? cap : kLayoutMinTiles;
+    for (int t = kLayoutTileTokens / 4; t < kLayoutTileTokens; t *= 2)
+        if ((tc + t - 1) / t <= max_tiles) return t;
+    return kLayoutTileTokens;
+}
+inline int64_t layout_max_tiles(int64_t tc) {
+    const int64_t cap = (tc + kLayoutTileTokens - 1) / kLayoutTileTokens;
+    return cap > kLayoutMinTiles ? cap : kLayoutMinTiles;
+}
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up after 2 s
 
 // ---------------------------------------------------------------- workspace
@@ -39,8 +55,7 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     L.status = off;               off += 256;
     L.ticket = off;               off += 256;
     L.chunk_counts = off;         off = align_up(off + sizeof(int32_t) * (size_t)c.E, 256);
-    L.max_tiles = (c.T + kLayoutTileTokens - 1) / kLayoutTileTokens;
-    if (L.max_tiles < 1) L.max_tiles = 1;
+    L.max_tiles = (int)layout_max_tiles(c.T);
     L.tile_state = off;           off = align_up(off + sizeof(uint32_t) * (size_t)L.max_tiles * c.E, 256);
     L.clip_thr = off;             off = align_up(off + sizeof(uint64_t) * (size_t)c.E, 256);
     L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
