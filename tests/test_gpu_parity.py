@@ -42,6 +42,10 @@ CASES = {
     "bf16_k1": W("bf16_k1", T=128, H=128, E=4, k=1, I=64, dtype="bf16", ep=1),
     "bf16_k_all": W("bf16_k_all", T=64, H=64, E=32, k=32, I=64, dtype="bf16", ep=2, capacity=40),
     "bf16_cap0": W("bf16_cap0", T=64, H=128, E=8, k=2, I=128, dtype="bf16", ep=2, capacity=0),
+    # a chunk of 6144 tokens: the dispatch layout takes 128-token tiles (48 of them)
+    "bf16_layout_128": W("bf16_layout_128", T=6144, H=64, E=16, k=2, I=64, dtype="bf16", ep=2),
+    # 512 experts: the router's 32-lane groups with 16 values per lane
+    "bf16_512_experts": W("bf16_512_experts", T=128, H=64, E=512, k=4, I=64, dtype="bf16", ep=4),
 }
 
 
