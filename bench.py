@@ -302,7 +302,8 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens):
     import numpy as np
     import oracle
     t0 = time.perf_counter()
-    idx, w, _, st = oracle.route_topk(logits, bias, wl.k)
+    idx, w, _, st = oracle.route_topk(logits, bias, wl.k, wl.n_group, wl.topk_group,
+                                      wl.group_score, wl.bias_select_only)
     keep, _ = oracle.capacity_clip(idx, w, wl.E, wl.capacity)
     tc = wl.T // wl.n_chunks
     lays = [oracle.dispatch_layout(idx, keep, wl.E, wl.ep, c * tc, tc) for c in range(wl.n_chunks)]

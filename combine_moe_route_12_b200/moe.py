@@ -29,7 +29,8 @@ MOE_DEV_BAD_INDEX = 0x4
 
 class MoEConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("T", "H", "E", "k", "I", "ep", "capacity", "dtype", "n_chunks", "reduce_dense")]
+                ("T", "H", "E", "k", "I", "ep", "capacity", "dtype", "n_chunks", "reduce_dense",
+                 "n_group", "topk_group", "group_score", "bias_select_only")]
 
     def __repr__(self):
         return "MoEConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -106,16 +107,19 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 def make_config(T, H, E, k, I, ep, capacity=-1, dtype=MOE_BF16, n_chunks=1,
-                reduce_dense=False) -> MoEConfig:
+                reduce_dense=False, n_group=0, topk_group=0, group_score=0,
+                bias_select_only=False) -> MoEConfig:
     if isinstance(dtype, str):
         dtype = MOE_F32 if dtype == "f32" else MOE_BF16
     return MoEConfig(T, H, E, k, I, ep, -1 if capacity is None else capacity, dtype, n_chunks,
-                     int(bool(reduce_dense)))
+                     int(bool(reduce_dense)), n_group, topk_group, group_score,
+                     int(bool(bias_select_only)))
 
 
 def config_from_workload(wl) -> MoEConfig:
     return make_config(wl.T, wl.H, wl.E, wl.k, wl.I, wl.ep, wl.capacity, wl.dtype, wl.n_chunks,
-                       wl.reduce_dense)
+                       wl.reduce_dense, wl.n_group, wl.topk_group, wl.group_score,
+                       wl.bias_select_only)
 
 
 # ------------------------------------------------------------------ sizes

@@ -35,6 +35,10 @@ Input recipe (the pages fix none of it; every choice is a stated reading):
   part of the hot path.
 * the skewed workload adds bias[e] = 3 * ln(p_{rank(e)}), p_r proportional to
   r^-1.2 for r = 1..128 and normalised, with rank(e) a seeded permutation.
+* ``dsv3_grouped`` (routing variants, DSV3 prefill shape in one chunk): grouped
+  top-k with 8 groups of 32 experts and 4 kept per token (group score: the sum
+  of a group's two best biased logits), and a load-balancing-like bias
+  bias[e] ~ N(0, 0.5^2) (seeded) that steers the selection only.
 """
 from __future__ import annotations
 
@@ -59,6 +63,12 @@ class MoEWorkload:
     reduce_dense: bool = False   # decode mode: y is reduced straight into out
     skew_bias: bool = False
     seed: int = 0
+    # routing variants (grouped top-k, bias in the selection only)
+    n_group: int = 0
+    topk_group: int = 0
+    group_score: int = 0          # 0: best logit of the group; 1: sum of its two best
+    bias_select_only: bool = False
+    balance_bias: bool = False    # a small per-expert bias ~ N(0, 0.5^2), the load-balancing kind
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -82,6 +92,12 @@ WORKLOADS = {
                                 dtype="bf16", ep=8, n_chunks=2),
     "dsv3_decode": MoEWorkload("dsv3_decode", T=256, H=7168, E=256, k=8, I=2048,
                                dtype="bf16", ep=64, capacity=1024, reduce_dense=True),
+    # routing variants on the DSV3 prefill shape (one chunk): 8 groups of 32
+    # experts, 4 kept per token by the sum of their two best biased logits, the
+    # bias used for the selection only
+    "dsv3_grouped": MoEWorkload("dsv3_grouped", T=8192, H=7168, E=256, k=8, I=2048,
+                                dtype="bf16", ep=8, n_group=8, topk_group=4, group_score=1,
+                                bias_select_only=True, balance_bias=True),
 }
 
 
@@ -133,6 +149,10 @@ def make_inputs(wl: MoEWorkload, device: str | torch.device = "cpu",
         gb = torch.Generator(device="cpu")
         gb.manual_seed(seed + 7919)
         bias = zipf_bias(wl.E, 1.2, gb).to(device)
+    elif wl.balance_bias:
+        gb = torch.Generator(device="cpu")
+        gb.manual_seed(seed + 104729)
+        bias = (0.5 * torch.randn(wl.E, generator=gb)).to(device)
 
     if weights:
         w13 = torch.empty(wl.E, 2 * wl.I, wl.H, dtype=dt, device=device)

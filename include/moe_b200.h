@@ -88,7 +88,11 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * T >= 0, H, E, k, I, ep, n_chunks >= 1, k <= E, E % ep == 0,
  * T % n_chunks == 0, (T / n_chunks) % ep == 0 (each chunk splits into equal
  * contiguous source-rank blocks).
- * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30;
+ * Routing-variant checks (MOE_ERR_INVALID_ARG): n_group >= 0, E % n_group == 0,
+ * topk_group and k as stated at the fields, group_score in {0, 1},
+ * bias_select_only in {0, 1}.
+ * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30,
+ * n_group <= 32;
  * MOE_BF16 needs H % 64 == 0 and I % 64 == 0 (tensor-core tiles);
  * MOE_F32 needs H % 4 == 0 and I % 4 == 0.
  */
@@ -98,6 +102,25 @@ typedef struct {
     int32_t dtype;          /* moe_dtype */
     int32_t n_chunks;
     int32_t reduce_dense;
+    /* Routing variants (LightLLM PR 1687: the experts() path keeps "grouped
+     * top-k" for DeepSeek-V2, GLM-4-MoE-Lite and Qwen3-MoE).  All zero gives
+     * plain top-k with the bias in both selection and weights.
+     *   n_group      experts form n_group contiguous groups of E / n_group
+     *                (<= 1: no grouping); a token first keeps the topk_group
+     *                groups with the best group score, then takes its top-k
+     *                among their experts.
+     *   topk_group   groups kept per token (1 <= topk_group <= n_group,
+     *                k <= topk_group * E / n_group).
+     *   group_score  0: a group's score is its best biased logit; 1: the sum of
+     *                its two best (E / n_group >= 2).  Groups rank by score,
+     *                lower group index first among equal scores.
+     *   bias_select_only  1: the bias steers the selection (experts and groups)
+     *                only; the weights are the softmax of the unbiased logits of
+     *                the chosen experts. */
+    int32_t n_group;
+    int32_t topk_group;
+    int32_t group_score;
+    int32_t bias_select_only;
 } moe_config;
 
 /* Validates cfg (topology and limits).  MOE_OK or the reason it is rejected. */

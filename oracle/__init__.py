@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
         L.orc_exp_det.restype = ctypes.c_float
         L.orc_route_topk.argtypes = [i, i, i, P, P, P, P, P]
         L.orc_route_topk.restype = i
+        L.orc_route_topk_ex.argtypes = [i, i, i, P, P, i, i, i, i, P, P, P]
+        L.orc_route_topk_ex.restype = i
         L.orc_capacity_clip.argtypes = [i, i, i, i, P, P, P, P]
         L.orc_capacity_clip.restype = i
         L.orc_dispatch_layout.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P]
@@ -91,8 +93,13 @@ def exp_det(r: float) -> float:
     return float(lib().orc_exp_det(ctypes.c_float(float(r))))
 
 
-def route_topk(logits: np.ndarray, bias: np.ndarray | None, k: int):
-    """Returns (topk_idx int32 [T,k], topk_w float32 [T,k], counts int32 [E], status)."""
+def route_topk(logits: np.ndarray, bias: np.ndarray | None, k: int, n_group: int = 0,
+               topk_group: int = 0, group_score: int = 0, bias_select_only: bool = False):
+    """Returns (topk_idx int32 [T,k], topk_w float32 [T,k], counts int32 [E], status).
+
+    n_group > 1 selects grouped top-k (topk_group groups kept per token by the
+    best biased logit of a group, group_score 0, or the sum of its two best, 1);
+    bias_select_only makes the bias steer the selection only."""
     logits = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = logits.shape
     if bias is not None:
@@ -100,7 +107,9 @@ def route_topk(logits: np.ndarray, bias: np.ndarray | None, k: int):
     idx = np.zeros((T, k), np.int32)
     w = np.zeros((T, k), np.float32)
     counts = np.zeros(E, np.int32)
-    st = lib().orc_route_topk(T, E, k, _p(logits), _p(bias), _p(idx), _p(w), _p(counts))
+    st = lib().orc_route_topk_ex(T, E, k, _p(logits), _p(bias), int(n_group), int(topk_group),
+                                 int(group_score), int(bool(bias_select_only)),
+                                 _p(idx), _p(w), _p(counts))
     return idx, w, counts, st
 
 
@@ -222,7 +231,8 @@ def bf16_bits_from_double(v: float) -> int:
 # --------------------------------------------------------------------------- whole layer
 
 def moe_layer(logits, bias, x, w13, w2, k: int, ep: int, capacity: int = -1,
-              n_chunks: int = 1, reduce_dense: bool = False) -> dict:
+              n_chunks: int = 1, reduce_dense: bool = False, n_group: int = 0,
+              topk_group: int = 0, group_score: int = 0, bias_select_only: bool = False) -> dict:
     """All six steps in the order the pages give them, chunk by chunk.
 
     Route and clip run once over all T tokens (the capacity is per forward);
@@ -230,7 +240,7 @@ def moe_layer(logits, bias, x, w13, w2, k: int, ep: int, capacity: int = -1,
     expert_parallel_dispatch_chunks).  Returns every intermediate.
     """
     T, E = logits.shape
-    idx, w, counts, st = route_topk(logits, bias, k)
+    idx, w, counts, st = route_topk(logits, bias, k, n_group, topk_group, group_score, bias_select_only)
     if st != ORC_OK:
         raise ValueError(f"route_topk status {st}")
     keep, kept = capacity_clip(idx, w, E, capacity)

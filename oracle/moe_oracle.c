@@ -91,19 +91,43 @@ static int orc_before(float va, int a, float vb, int b)
  * topk_idx int32 [T, k], topk_w fp32 [T, k] in rank order; counts int32 [E]
  * (assignments per expert before any clip).
  *
- * Weights: with l'_j the selected biased logits in slot order and m = l'_0,
- *   w_j = exp(l'_j - m) / sum_{i<k} exp(l'_i - m),
+ * Weights: with v_j the logits of the selected experts in slot order and
+ * m = max_j v_j,
+ *   w_j = exp(v_j - m) / sum_{i<k} exp(v_i - m),
  * which equals the full softmax restricted to the top k and renormalised (the
  * softmax denominator cancels).  Reading: the bias (skewed-router workload)
- * enters both the selection and the weights; the sum runs in slot order.
+ * enters both the selection and the weights (v_j = l'_j, so m = l'_0); the sum
+ * runs in slot order.
+ *
+ * Routing variants (LightLLM PR 1687: "grouped top-k" kept inside experts()
+ * for DeepSeek-V2, GLM-4-MoE-Lite and Qwen3-MoE).  The page names them only;
+ * the plainest readings, stated:
+ *  - grouped top-k (n_group > 1): experts form n_group contiguous groups of
+ *    E / n_group.  A group's score is its best biased logit (group_score 0) or
+ *    the fp32 sum of its two best (group_score 1).  The topk_group groups with
+ *    the best scores are kept (larger score first, lower group index among
+ *    equal scores); the top-k is then taken among their experts only.
+ *  - bias_select_only: the bias steers the choice of experts (and of groups)
+ *    but the weights use the unbiased logits, v_j = logit_j (+0 for -0).
  */
-int orc_route_topk(int T, int E, int k, const float *logits, const float *bias,
-                   int32_t *topk_idx, float *topk_w, int32_t *counts)
+int orc_route_topk_ex(int T, int E, int k, const float *logits, const float *bias,
+                      int n_group, int topk_group, int group_score, int bias_select_only,
+                      int32_t *topk_idx, float *topk_w, int32_t *counts)
 {
     if (T < 0 || E <= 0 || k <= 0 || k > E) return ORC_ERR_ARG;
+    const int grouped = n_group > 1;
+    if (grouped) {
+        if (E % n_group != 0 || topk_group < 1 || topk_group > n_group ||
+            k > topk_group * (E / n_group) || (group_score != 0 && group_score != 1) ||
+            (group_score == 1 && E / n_group < 2))
+            return ORC_ERR_ARG;
+    }
+    const int gs = grouped ? E / n_group : E;
     float *l = (float *)malloc(sizeof(float) * (size_t)E);
     unsigned char *taken = (unsigned char *)malloc((size_t)E);
     float *ev = (float *)malloc(sizeof(float) * (size_t)k);
+    float *gscore = (float *)malloc(sizeof(float) * (size_t)(grouped ? n_group : 1));
+    unsigned char *gkeep = (unsigned char *)malloc((size_t)(grouped ? n_group : 1));
     int status = ORC_OK;
     for (int e = 0; e < E; ++e) counts[e] = 0;
     for (int t = 0; t < T; ++t) {
@@ -112,6 +136,29 @@ int orc_route_topk(int T, int E, int k, const float *logits, const float *bias,
             l[e] = logits[(size_t)t * E + e] + b;   /* -0 + +0 = +0: canonicalises -0 */
             if (!isfinite(l[e])) status = ORC_ERR_NONFINITE;
             taken[e] = 0;
+        }
+        if (grouped) {
+            /* group scores, then keep the best topk_group groups by repeated selection */
+            for (int g = 0; g < n_group; ++g) {
+                int b1 = -1, b2 = -1;       /* the group's best and second-best experts */
+                for (int e = g * gs; e < (g + 1) * gs; ++e) {
+                    if (b1 < 0 || l[e] > l[b1]) { b2 = b1; b1 = e; }
+                    else if (b2 < 0 || l[e] > l[b2]) b2 = e;
+                }
+                gscore[g] = group_score == 0 ? l[b1] : l[b1] + l[b2];
+                gkeep[g] = 0;
+            }
+            for (int j = 0; j < topk_group; ++j) {
+                int best = -1;
+                for (int g = 0; g < n_group; ++g) {
+                    if (gkeep[g]) continue;
+                    if (best < 0 || orc_before(gscore[g], g, gscore[best], best)) best = g;
+                }
+                gkeep[best] = 1;
+            }
+            /* experts of the dropped groups cannot be chosen */
+            for (int e = 0; e < E; ++e)
+                if (!gkeep[e / gs]) taken[e] = 1;
         }
         for (int j = 0; j < k; ++j) {
             int best = -1;
@@ -123,16 +170,29 @@ int orc_route_topk(int T, int E, int k, const float *logits, const float *bias,
             topk_idx[(size_t)t * k + j] = best;
             counts[best] += 1;
         }
-        float m = l[topk_idx[(size_t)t * k]];
+        /* the weights' logits: biased, or unbiased when the bias only selects */
+        float m = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(size_t)t * k + j];
+            const float v = bias_select_only ? logits[(size_t)t * E + e] + 0.0f : l[e];
+            ev[j] = v;
+            if (j == 0 || v > m) m = v;
+        }
         float S = 0.0f;
         for (int j = 0; j < k; ++j) {
-            ev[j] = orc_exp_det(l[topk_idx[(size_t)t * k + j]] - m);
+            ev[j] = orc_exp_det(ev[j] - m);
             S = S + ev[j];
         }
         for (int j = 0; j < k; ++j) topk_w[(size_t)t * k + j] = ev[j] / S;
     }
-    free(l); free(taken); free(ev);
+    free(l); free(taken); free(ev); free(gscore); free(gkeep);
     return status;
+}
+
+int orc_route_topk(int T, int E, int k, const float *logits, const float *bias,
+                   int32_t *topk_idx, float *topk_w, int32_t *counts)
+{
+    return orc_route_topk_ex(T, E, k, logits, bias, 0, 0, 0, 0, topk_idx, topk_w, counts);
 }
 
 /* ------------------------------------------------------------------------- */

@@ -108,7 +108,8 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
 def oracle_routing(wl: MoEWorkload, inp: MoEInputs) -> dict:
     logits = inp.logits.detach().cpu().numpy()
     bias = None if inp.bias is None else inp.bias.detach().cpu().numpy()
-    idx, w, counts, st = oracle.route_topk(logits, bias, wl.k)
+    idx, w, counts, st = oracle.route_topk(logits, bias, wl.k, wl.n_group, wl.topk_group,
+                                           wl.group_score, wl.bias_select_only)
     assert st == oracle.ORC_OK
     keep, kept = oracle.capacity_clip(idx, w, wl.E, wl.capacity)
     tc = wl.T // wl.n_chunks

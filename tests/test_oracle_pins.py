@@ -164,6 +164,120 @@ def test_topk_rejects_nonfinite():
     assert st == oracle.ORC_ERR_NONFINITE
 
 
+# ----------------------------------------------------------------- routing variants
+
+def _ranks_before(va, a, vb, b):
+    return va > vb or (va == vb and a < b)
+
+
+def _group_scores_f32(l, n_group, mode):
+    """A group's best value, or the fp32 sum of its two best (mode 1)."""
+    gs = l.shape[0] // n_group
+    out = []
+    for g in range(n_group):
+        v = sorted((float(x) for x in l[g * gs:(g + 1) * gs]), reverse=True)
+        out.append(np.float32(v[0]) if mode == 0 else np.float32(np.float32(v[0]) + np.float32(v[1])))
+    return out
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_grouped_topk_reduces_to_plain(mode):
+    rng = np.random.default_rng(21)
+    logits = rng.standard_normal((40, 12)).astype(np.float32)
+    ref_idx, ref_w, ref_c, _ = oracle.route_topk(logits, None, 3)
+    for n_group, topk_group in ((1, 1), (4, 4), (6, 6)):
+        idx, w, c, st = oracle.route_topk(logits, None, 3, n_group=n_group, topk_group=topk_group,
+                                          group_score=mode)
+        assert st == oracle.ORC_OK
+        np.testing.assert_array_equal(idx, ref_idx)
+        np.testing.assert_array_equal(w.view(np.uint32), ref_w.view(np.uint32))
+        np.testing.assert_array_equal(c, ref_c)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_grouped_topk_brute_force_with_ties(mode):
+    """Characterisation on tiny inputs with many ties: every kept group outranks
+    every dropped one (score desc, lower group first), every chosen expert lies in
+    a kept group and outranks every unchosen expert of the kept groups, and the
+    slots are in rank order."""
+    rng = np.random.default_rng(5 + mode)
+    E, n_group = 8, 4
+    gs = E // n_group
+    for trial in range(60):
+        logits = rng.integers(-3, 4, size=(6, E)).astype(np.float32) * np.float32(0.5)
+        topk_group = 1 + trial % 3
+        k = 1 + trial % (topk_group * gs)
+        idx, w, counts, st = oracle.route_topk(logits, None, k, n_group=n_group,
+                                               topk_group=topk_group, group_score=mode)
+        assert st == oracle.ORC_OK
+        for t in range(logits.shape[0]):
+            l = logits[t]
+            sc = _group_scores_f32(l, n_group, mode)
+            # the kept groups: the topk_group best by (score desc, index asc), by exhaustion
+            best_set = None
+            for G in itertools.combinations(range(n_group), topk_group):
+                ok = all(_ranks_before(sc[g], g, sc[h], h)
+                         for g in G for h in range(n_group) if h not in G)
+                if ok:
+                    assert best_set is None
+                    best_set = set(G)
+            allowed = [e for e in range(E) if e // gs in best_set]
+            chosen = [int(e) for e in idx[t]]
+            assert len(set(chosen)) == k and all(e in allowed for e in chosen)
+            for e in chosen:
+                for f in allowed:
+                    if f not in chosen:
+                        assert _ranks_before(l[e], e, l[f], f)
+            for a, b in zip(chosen, chosen[1:]):
+                assert _ranks_before(l[a], a, l[b], b)
+            # weights: renormalised softmax over the chosen biased logits
+            ref = np.exp(np.array([float(l[e]) for e in chosen]) - float(l[chosen[0]]))
+            np.testing.assert_allclose(w[t], ref / ref.sum(), rtol=1e-6)
+        assert int(counts.sum()) == k * logits.shape[0]
+
+
+def test_grouped_topk_rejects_bad_arguments():
+    logits = np.zeros((2, 8), np.float32)
+    for kw in (dict(n_group=3, topk_group=1),            # E not divisible
+               dict(n_group=4, topk_group=0),            # no group kept
+               dict(n_group=4, topk_group=5),            # more than there are
+               dict(n_group=8, topk_group=1, group_score=1)):   # one-expert groups, sum of two
+        *_, st = oracle.route_topk(logits, None, 1, **kw)
+        assert st == oracle.ORC_ERR_ARG
+    *_, st = oracle.route_topk(logits, None, 3, n_group=4, topk_group=1)   # k > 1 group of 2
+    assert st == oracle.ORC_ERR_ARG
+
+
+def test_bias_select_only():
+    rng = np.random.default_rng(8)
+    logits = rng.standard_normal((50, 16)).astype(np.float32)
+    bias = (2.0 * rng.standard_normal(16)).astype(np.float32)
+    # zero bias: the same as plain routing, bit for bit
+    z = np.zeros(16, np.float32)
+    a = oracle.route_topk(logits, z, 4, bias_select_only=True)
+    b = oracle.route_topk(logits, None, 4)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+    # with a bias: the experts are the biased choice, the weights the softmax of
+    # the unbiased logits of those experts (closed form in double)
+    idx, w, _, st = oracle.route_topk(logits, bias, 4, bias_select_only=True)
+    assert st == oracle.ORC_OK
+    ref_idx, ref_w_biased, _, _ = oracle.route_topk(logits, bias, 4)
+    np.testing.assert_array_equal(idx, ref_idx)
+    for t in range(logits.shape[0]):
+        v = np.array([float(logits[t, e]) for e in idx[t]])
+        ref = np.exp(v - v.max())
+        np.testing.assert_allclose(w[t], ref / ref.sum(), rtol=1e-6)
+        assert abs(float(w[t].sum()) - 1.0) <= 4 * 2.0 ** -23
+    assert not np.array_equal(w, ref_w_biased)   # the bias does change the weights otherwise
+    # combined with grouping: the chosen experts are those of grouped routing on the
+    # biased logits
+    g = oracle.route_topk(logits, bias, 4, n_group=4, topk_group=2, group_score=1,
+                          bias_select_only=True)
+    g_ref = oracle.route_topk(logits, bias, 4, n_group=4, topk_group=2, group_score=1)
+    np.testing.assert_array_equal(g[0], g_ref[0])
+
+
 # ----------------------------------------------------------------- capacity clip
 
 def _brute_force_keep(assigns, C):
