@@ -172,6 +172,23 @@ moe_status moe_config_check(const moe_config *cfg) {
     if (c.reduce_dense != 0 && c.reduce_dense != 1)
         return fail(MOE_ERR_INVALID_ARG, "reduce_dense must be 0 or 1");
     if (c.k > c.E) return fail(MOE_ERR_INVALID_ARG, "k=%d > E=%d", c.k, c.E);
+    if (c.n_group < 0) return fail(MOE_ERR_INVALID_ARG, "n_group=%d < 0", c.n_group);
+    if (c.bias_select_only != 0 && c.bias_select_only != 1)
+        return fail(MOE_ERR_INVALID_ARG, "bias_select_only must be 0 or 1");
+    if (c.n_group > 1) {
+        if (c.n_group > kMaxGroups) return fail(MOE_ERR_UNSUPPORTED, "n_group=%d > %d", c.n_group, kMaxGroups);
+        if (c.E % c.n_group != 0)
+            return fail(MOE_ERR_INVALID_ARG, "E=%d not divisible by n_group=%d", c.E, c.n_group);
+        if (c.topk_group < 1 || c.topk_group > c.n_group)
+            return fail(MOE_ERR_INVALID_ARG, "topk_group=%d outside [1, n_group=%d]", c.topk_group, c.n_group);
+        if (c.k > c.topk_group * (c.E / c.n_group))
+            return fail(MOE_ERR_INVALID_ARG, "k=%d > topk_group * E / n_group = %d", c.k,
+                        c.topk_group * (c.E / c.n_group));
+        if (c.group_score != 0 && c.group_score != 1)
+            return fail(MOE_ERR_INVALID_ARG, "group_score must be 0 or 1");
+        if (c.group_score == 1 && c.E / c.n_group < 2)
+            return fail(MOE_ERR_INVALID_ARG, "group_score 1 needs groups of at least two experts");
+    }
     if (c.E % c.ep != 0) return fail(MOE_ERR_INVALID_ARG, "E=%d not divisible by ep=%d", c.E, c.ep);
     if (c.T % c.n_chunks != 0)
         return fail(MOE_ERR_INVALID_ARG, "T=%d not divisible by n_chunks=%d", c.T, c.n_chunks);

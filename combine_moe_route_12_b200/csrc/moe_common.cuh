@@ -14,6 +14,7 @@ namespace moe {
 // ---------------------------------------------------------------- constants
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
+constexpr int kMaxGroups = 32;              // grouped top-k: groups per token
 constexpr int kLayoutTileTokens = 256;      // largest dispatch-layout tile (tokens)
 constexpr int kLayoutMinTiles = 64;         // tiles shrink while there are at most this many
 

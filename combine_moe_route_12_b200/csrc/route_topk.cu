@@ -1,6 +1,7 @@
 // Step 1: router top-k with renormalised softmax weights (LightLLM PR 1687,
 // _select_experts with norm_topk_prob; axolotl ExpertParallelArgs: the routing
-// top-k is saved state).
+// top-k is saved state), and its variants: grouped top-k (the experts() path of
+// the same page) and a bias that steers the selection only.
 //
 // A group of LPT lanes (8, 16 or 32) per token, 32/LPT tokens per warp at a
 // time.  Lane l of a group holds the biased logits of experts l, l+LPT, ... as
@@ -65,9 +66,28 @@ __device__ __forceinline__ int key_expert(uint64_t key) {
 }
 __device__ __forceinline__ uint64_t max_u64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 
-template <int LPT, int VPL>
+// Routing variants: grouped top-k and a bias that steers the selection only.
+struct RouteVariant {
+    int n_group;          // <= 1: no grouping
+    int topk_group;
+    int group_score;      // 0: best biased logit of the group; 1: sum of its two best
+    int bias_select_only;
+};
+
+// Top two keys of the union of (a1 >= a2) and (b1 >= b2); keys are distinct or 0.
+__device__ __forceinline__ void merge_top2(uint64_t &a1, uint64_t &a2, uint64_t b1, uint64_t b2) {
+    if (a1 > b1) {
+        a2 = max_u64(a2, b1);
+    } else {
+        a2 = max_u64(a1, b2);
+        a1 = b1;
+    }
+}
+
+template <int LPT, int VPL, bool kGrouped>
 __global__ void __launch_bounds__(256) route_topk_kernel(
     int T, int E, int k, const float *__restrict__ logits, const float *__restrict__ bias,
+    RouteVariant rv,
     int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int32_t *__restrict__ counts,
     uint32_t *__restrict__ status) {
     extern __shared__ int32_t s_hist[];  // [E]
@@ -101,6 +121,66 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
                 key[i] = rank_key(l, e);
             }
         }
+        if (kGrouped) {
+            // grouped top-k: the score of every expert group (in-group butterfly per
+            // group), kept as rank keys (score, group) spread over the lanes like the
+            // experts (lane l holds groups l, l + LPT, ...); the topk_group best groups
+            // are taken with the same rounds as the experts, and the experts of the
+            // other groups drop out
+            const int gsz = E / rv.n_group;
+            constexpr int kGPL = (kMaxGroups + LPT - 1) / LPT;   // group keys per lane
+            int eg[VPL];                                          // group of each held expert
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) eg[i] = (gl + LPT * i) / gsz;
+            uint64_t gkey[kGPL];
+#pragma unroll
+            for (int i = 0; i < kGPL; ++i) gkey[i] = 0;
+            for (int grp = 0; grp < rv.n_group; ++grp) {
+                uint64_t b1 = 0, b2 = 0;   // this lane's two best keys in the group
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    if (key[i] != 0 && eg[i] == grp) {
+                        if (key[i] > b1) { b2 = b1; b1 = key[i]; }
+                        else b2 = max_u64(b2, key[i]);
+                    }
+                }
+#pragma unroll
+                for (int off = LPT / 2; off > 0; off >>= 1) {
+                    const uint64_t o1 = __shfl_xor_sync(0xffffffffu, b1, off);
+                    const uint64_t o2 = __shfl_xor_sync(0xffffffffu, b2, off);
+                    merge_top2(b1, b2, o1, o2);
+                }
+                const float score = rv.group_score == 0 ? key_value(b1)
+                                                        : __fadd_rn(key_value(b1), key_value(b2));
+                if (grp % LPT == gl) {
+#pragma unroll
+                    for (int i = 0; i < kGPL; ++i)
+                        if (i == grp / LPT) gkey[i] = rank_key(score, grp);
+                }
+            }
+            uint64_t gbest = 0;
+#pragma unroll
+            for (int i = 0; i < kGPL; ++i) gbest = max_u64(gbest, gkey[i]);
+            uint32_t kept = 0;   // bit g: group g kept
+            for (int j = 0; j < rv.topk_group; ++j) {
+                uint64_t top = gbest;
+#pragma unroll
+                for (int off = LPT / 2; off > 0; off >>= 1)
+                    top = max_u64(top, __shfl_xor_sync(0xffffffffu, top, off));
+                kept |= 1u << key_expert(top);
+                if (gbest == top && top != 0) {
+                    gbest = 0;
+#pragma unroll
+                    for (int i = 0; i < kGPL; ++i) {
+                        if (gkey[i] == top) gkey[i] = 0;
+                        gbest = max_u64(gbest, gkey[i]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+                if (key[i] != 0 && !((kept >> eg[i]) & 1u)) key[i] = 0;
+        }
         // each lane keeps its best remaining key; a round takes the group's best
         // and only the lane that held it looks for its next one
         uint64_t best = 0;
@@ -122,9 +202,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
                 }
             }
         }
-        const float my_v = key_value(my_key);
         const int my_e = key_expert(my_key);
-        const float m = __shfl_sync(0xffffffffu, my_v, glane0);
+        // the weights' logit: biased, or the unbiased logit when the bias only selects
+        float my_v = key_value(my_key);
+        if (rv.bias_select_only && valid && gl < k) my_v = __fadd_rn(__ldg(row + my_e), 0.0f);
+        float m = gl < k ? my_v : -INFINITY;   // the largest of the k (slot 0's when biased)
+#pragma unroll
+        for (int off = LPT / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         const float ex = (gl < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
         float S = 0.0f;
         for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ex, glane0 + j));
@@ -150,6 +234,7 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     const int cap = num_sms * 4;   // one global atomic per CTA and expert
     if (blocks > cap) blocks = cap;
     const size_t smem = sizeof(int32_t) * (size_t)c.E;
+    const RouteVariant rv{c.n_group, c.topk_group, c.group_score, c.bias_select_only};
     // lanes per token: at least k (slot j lives in group lane j), at most 32,
     // aiming at 16 values per lane
     int lpt = 8;
@@ -158,9 +243,14 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     blocks = (int)(((long long)c.T * lpt / 32 + warps_per_block - 1) / warps_per_block);
     if (blocks < 1) blocks = 1;
     if (blocks > cap) blocks = cap;
-#define MOE_ROUTE_CASE(L, V)                                                                    \
-    route_topk_kernel<L, V><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, topk_idx, \
-                                                      topk_w, counts, status)
+#define MOE_ROUTE_LAUNCH(L, V, G)                                                               \
+    route_topk_kernel<L, V, G><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, rv, topk_idx, \
+                                                         topk_w, counts, status)
+#define MOE_ROUTE_CASE(L, V)                      \
+    do {                                          \
+        if (rv.n_group > 1) MOE_ROUTE_LAUNCH(L, V, true); \
+        else MOE_ROUTE_LAUNCH(L, V, false);       \
+    } while (0)
     if (lpt == 8) {
         if (vpl <= 1) MOE_ROUTE_CASE(8, 1);
         else if (vpl <= 2) MOE_ROUTE_CASE(8, 2);
@@ -181,6 +271,7 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
         else if (vpl <= 16) MOE_ROUTE_CASE(32, 16);
         else MOE_ROUTE_CASE(32, 32);
     }
+#undef MOE_ROUTE_LAUNCH
 #undef MOE_ROUTE_CASE
     return cudaGetLastError();
 }

@@ -22,7 +22,7 @@ from moe_testlib import (assert_float_close, assert_routing_equal, oracle_routin
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode"]
+FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode", "dsv3_grouped"]
 
 
 def _host_expert(inp, e, cache):

@@ -46,6 +46,19 @@ CASES = {
     "bf16_layout_128": W("bf16_layout_128", T=6144, H=64, E=16, k=2, I=64, dtype="bf16", ep=2),
     # 512 experts: the router's 32-lane groups with 16 values per lane
     "bf16_512_experts": W("bf16_512_experts", T=128, H=64, E=512, k=4, I=64, dtype="bf16", ep=4),
+    # routing variants: grouped top-k by the best logit of a group
+    "bf16_grouped": W("bf16_grouped", T=256, H=128, E=64, k=6, I=64, dtype="bf16", ep=4,
+                      n_group=8, topk_group=3, group_score=0),
+    # DSV3-like: 8 groups of 32, 4 kept by the sum of their two best, bias in the selection only
+    "bf16_grouped_top2_selbias": W("bf16_grouped_top2_selbias", T=256, H=128, E=256, k=8, I=64,
+                                   dtype="bf16", ep=8, n_group=8, topk_group=4, group_score=1,
+                                   bias_select_only=True, balance_bias=True),
+    # grouped with k > 16 (32-lane token groups) and a binding capacity
+    "bf16_grouped_k20": W("bf16_grouped_k20", T=128, H=64, E=64, k=20, I=64, dtype="bf16", ep=2,
+                          n_group=4, topk_group=2, group_score=1, capacity=40),
+    # fp32, skewed bias in the selection only
+    "f32_selbias_skew": W("f32_selbias_skew", T=256, H=128, E=8, k=2, I=128, dtype="f32", ep=2,
+                          skew_bias=True, bias_select_only=True),
 }
 
 
