@@ -62,9 +62,9 @@ def lib() -> ctypes.CDLL:
         L.orc_permute.restype = None
         L.orc_ffn_row.argtypes = [i, i, i, P, P, P, i, P, P, P]
         L.orc_ffn_row.restype = None
-        L.orc_combine.argtypes = [i, i, i, i, i, P, P, P, P]
+        L.orc_combine.argtypes = [i, i, i, i, i, P, P, P, P, P]
         L.orc_combine.restype = None
-        L.orc_combine_exact.argtypes = [i, i, i, i, i, P, P, P, P]
+        L.orc_combine_exact.argtypes = [i, i, i, i, i, P, P, P, P, P]
         L.orc_combine_exact.restype = None
         L.orc_bf16_from_double.argtypes = [ctypes.c_double]
         L.orc_bf16_from_double.restype = ctypes.c_uint16
@@ -197,7 +197,10 @@ def ffn(xr: np.ndarray, expert_offsets: np.ndarray, w13: np.ndarray, w2: np.ndar
 
 
 def combine(y: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: int,
-            tok_begin: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+            tok_begin: int = 0, out: np.ndarray | None = None,
+            y_shared: np.ndarray | None = None) -> np.ndarray:
+    """y_shared: the chunk's [tok_count, H] rows of the shared expert's output
+    (same dtype as y), added into the sum before its rounding, or None."""
     y = np.ascontiguousarray(y)
     pos = np.ascontiguousarray(pos, dtype=np.int32)
     topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
@@ -206,12 +209,15 @@ def combine(y: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: int,
     tok_count, k = pos.shape
     if out is None:
         out = np.zeros((T, H), y.dtype)
-    lib().orc_combine(H, k, dt, tok_begin, tok_count, _p(y), _p(pos), _p(topk_w), _p(out))
+    if y_shared is not None:
+        y_shared = np.ascontiguousarray(y_shared, dtype=y.dtype)
+    lib().orc_combine(H, k, dt, tok_begin, tok_count, _p(y), _p(pos), _p(topk_w), _p(y_shared), _p(out))
     return out
 
 
 def combine_exact(y_exact: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: int,
-                  out_dtype, tok_begin: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+                  out_dtype, tok_begin: int = 0, out: np.ndarray | None = None,
+                  y_shared: np.ndarray | None = None) -> np.ndarray:
     y_exact = np.ascontiguousarray(y_exact, dtype=np.float64)
     pos = np.ascontiguousarray(pos, dtype=np.int32)
     topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
@@ -220,7 +226,10 @@ def combine_exact(y_exact: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: i
     if out is None:
         out = np.zeros((T, H), out_dtype)
     dt = _dtype_code(out)
-    lib().orc_combine_exact(H, k, dt, tok_begin, tok_count, _p(y_exact), _p(pos), _p(topk_w), _p(out))
+    if y_shared is not None:
+        y_shared = np.ascontiguousarray(y_shared, dtype=out.dtype)
+    lib().orc_combine_exact(H, k, dt, tok_begin, tok_count, _p(y_exact), _p(pos), _p(topk_w),
+                            _p(y_shared), _p(out))
     return out
 
 
@@ -230,9 +239,17 @@ def bf16_bits_from_double(v: float) -> int:
 
 # --------------------------------------------------------------------------- whole layer
 
+def shared_expert(x: np.ndarray, w13s: np.ndarray, w2s: np.ndarray):
+    """The shared expert over the rows of x: one expert's FFN (w13s [2I_s, H],
+    w2s [H, I_s]) applied to every row.  Returns (h, y, y_exact) like ffn()."""
+    T = x.shape[0]
+    return ffn(x, np.array([0, T], np.int32), w13s[None], w2s[None])
+
+
 def moe_layer(logits, bias, x, w13, w2, k: int, ep: int, capacity: int = -1,
               n_chunks: int = 1, reduce_dense: bool = False, n_group: int = 0,
-              topk_group: int = 0, group_score: int = 0, bias_select_only: bool = False) -> dict:
+              topk_group: int = 0, group_score: int = 0, bias_select_only: bool = False,
+              w13_shared=None, w2_shared=None) -> dict:
     """All six steps in the order the pages give them, chunk by chunk.
 
     Route and clip run once over all T tokens (the capacity is per forward);
@@ -252,10 +269,13 @@ def moe_layer(logits, bias, x, w13, w2, k: int, ep: int, capacity: int = -1,
         lay = dispatch_layout(idx, keep, E, ep, tb, tc)
         xr = permute(x, lay["recv_token"])
         h, y, ye = ffn(xr, lay["expert_offsets"], w13, w2)
+        ys = None
+        if w13_shared is not None:
+            _, ys, _ = shared_expert(x[tb:tb + tc], w13_shared, w2_shared)
         if reduce_dense:
-            combine_exact(ye, lay["pos"], w, T, x.dtype, tb, out)
+            combine_exact(ye, lay["pos"], w, T, x.dtype, tb, out, y_shared=ys)
         else:
-            combine(y, lay["pos"], w, T, tb, out)
-        chunks.append(dict(layout=lay, xr=xr, h=h, y=y, y_exact=ye))
+            combine(y, lay["pos"], w, T, tb, out, y_shared=ys)
+        chunks.append(dict(layout=lay, xr=xr, h=h, y=y, y_exact=ye, y_shared=ys))
     return dict(topk_idx=idx, topk_w=w, counts=counts, keep=keep, kept_counts=kept,
                 chunks=chunks, out=out)

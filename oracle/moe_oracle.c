@@ -395,14 +395,19 @@ void orc_ffn_row(int H, int I, int dtype, const void *x_row, const void *w13_e,
 /*   out[t, :] = sum over kept slots j (in slot order) of w[t, j] * y[pos[t,j]] */
 /* accumulated in double, rounded once to the storage type; a token with every */
 /* slot dropped gets zeros.  pos is chunk-relative [n, k], -1 where dropped.   */
+/* Shared expert (LightLLM PR 1687: the shared expert's output is added in the */
+/* combine, which overlaps it): y_shared [n, H], the chunk's rows of the       */
+/* shared expert's stored output, or NULL; reading: it enters the same sum     */
+/* before the one rounding.                                                    */
 /* ------------------------------------------------------------------------- */
 void orc_combine(int H, int k, int dtype, int tok_begin, int tok_count, const void *y,
-                 const int32_t *pos, const float *topk_w, void *out)
+                 const int32_t *pos, const float *topk_w, const void *y_shared, void *out)
 {
     double *acc = (double *)malloc(sizeof(double) * (size_t)H);
     for (int i = 0; i < tok_count; ++i) {
         int t = tok_begin + i;
-        for (int c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int c = 0; c < H; ++c)
+            acc[c] = y_shared ? orc_load(y_shared, (size_t)i * H + c, dtype) : 0.0;
         for (int j = 0; j < k; ++j) {
             int p = pos[(size_t)i * k + j];
             if (p < 0) continue;
@@ -419,12 +424,13 @@ void orc_combine(int H, int k, int dtype, int tok_begin, int tok_count, const vo
  * the reduce consumes y before it is ever stored.  y_exact is [N, H] double. */
 void orc_combine_exact(int H, int k, int dtype, int tok_begin, int tok_count,
                        const double *y_exact, const int32_t *pos, const float *topk_w,
-                       void *out)
+                       const void *y_shared, void *out)
 {
     double *acc = (double *)malloc(sizeof(double) * (size_t)H);
     for (int i = 0; i < tok_count; ++i) {
         int t = tok_begin + i;
-        for (int c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int c = 0; c < H; ++c)
+            acc[c] = y_shared ? orc_load(y_shared, (size_t)i * H + c, dtype) : 0.0;
         for (int j = 0; j < k; ++j) {
             int p = pos[(size_t)i * k + j];
             if (p < 0) continue;

@@ -551,6 +551,52 @@ def test_chunking_changes_nothing():
     np.testing.assert_array_equal(a, b)
 
 
+# ----------------------------------------------------------------- shared expert
+
+def _shared_case(rng, T=24, H=16, E=6, k=2, I=12, Is=10):
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w13 = (rng.standard_normal((E, 2 * I, H)) / 4).astype(np.float32)
+    w2 = (rng.standard_normal((E, H, I)) / 4).astype(np.float32)
+    w13s = (rng.standard_normal((2 * Is, H)) / 4).astype(np.float32)
+    w2s = (rng.standard_normal((H, Is)) / 4).astype(np.float32)
+    return logits, x, w13, w2, w13s, w2s
+
+
+@pytest.mark.parametrize("reduce_dense", [False, True])
+def test_shared_expert_zero_weights_change_nothing(reduce_dense):
+    logits, x, w13, w2, w13s, w2s = _shared_case(np.random.default_rng(31))
+    a = oracle.moe_layer(logits, None, x, w13, w2, 2, 2, reduce_dense=reduce_dense)["out"]
+    b = oracle.moe_layer(logits, None, x, w13, w2, 2, 2, reduce_dense=reduce_dense,
+                         w13_shared=np.zeros_like(w13s), w2_shared=np.zeros_like(w2s))["out"]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_shared_expert_alone_when_every_assignment_is_dropped():
+    logits, x, w13, w2, w13s, w2s = _shared_case(np.random.default_rng(32))
+    res = oracle.moe_layer(logits, None, x, w13, w2, 2, 2, capacity=0,
+                           w13_shared=w13s, w2_shared=w2s, n_chunks=2)
+    ys = np.concatenate([c["y_shared"] for c in res["chunks"]])
+    np.testing.assert_array_equal(res["out"], ys)
+    # and ys is the dense SwiGLU of every row (closed form in double)
+    Is = w2s.shape[1]
+    g = x.astype(np.float64) @ w13s[:Is].T.astype(np.float64)
+    u = x.astype(np.float64) @ w13s[Is:].T.astype(np.float64)
+    ref = ((g / (1 + np.exp(-g))) * u).astype(np.float32).astype(np.float64) @ w2s.T.astype(np.float64)
+    np.testing.assert_allclose(ys, ref, rtol=1e-5, atol=1e-6)
+
+
+def test_shared_expert_equal_to_the_routed_one_doubles_it():
+    # all-equal logits and k = 1 route every token to expert 0 with w = 1; with the
+    # shared expert's weights equal to expert 0's, out = round(y + y) = 2 y exactly
+    logits, x, w13, w2, _, _ = _shared_case(np.random.default_rng(33))
+    logits[:] = 0.5
+    res = oracle.moe_layer(logits, None, x, w13, w2, 1, 2, w13_shared=w13[0], w2_shared=w2[0])
+    assert (res["topk_idx"] == 0).all() and (res["topk_w"] == 1.0).all()
+    ys = res["chunks"][0]["y_shared"]
+    np.testing.assert_array_equal(res["out"], 2 * ys)
+
+
 def test_worked_example_by_hand():
     """T=4, E=4, k=2, EP=2, C=2, derived by hand from the definitions.
 
