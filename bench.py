@@ -188,8 +188,9 @@ def kernels_per_step(wl) -> int:
     # route 1; clip 2 (prep, mark) or 4 with a binding capacity (+ gather, select);
     # per chunk: layout 2 (hist, scatter), permute 1, FFN 2 (two GEMM launches),
     # combine or finalize 1
+    # with a shared expert, per chunk 3 more (its offsets and two GEMM launches)
     clip = 4 if wl.capacity > 0 else 2
-    return 1 + clip + wl.n_chunks * 6
+    return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0))
 
 
 def algorithmic(wl, n_kept_chunks, active_chunks):
@@ -241,10 +242,14 @@ class StepBuffers:
         self.y = None if wl.reduce_dense else torch.empty(n, H, dtype=wl.torch_dtype, device=dev)
         self.red = torch.zeros(T, H, dtype=torch.float32, device=dev) if wl.reduce_dense else None
         self.out = torch.empty(T, H, dtype=wl.torch_dtype, device=dev)
+        self.hs = self.ys = None
+        if wl.shared_I > 0:
+            self.hs = torch.empty(tc, wl.shared_I, dtype=wl.torch_dtype, device=dev)
+            self.ys = torch.empty(tc, H, dtype=wl.torch_dtype, device=dev)
 
 
 def n_marks(wl) -> int:
-    return 3 + 4 * wl.n_chunks
+    return 3 + 5 * wl.n_chunks
 
 
 def run_steps(moe, wl, cfg, inp, B, ev=None):
@@ -260,7 +265,7 @@ def run_steps(moe, wl, cfg, inp, B, ev=None):
     rec(2)
     for c in range(wl.n_chunks):
         tb = c * B.tc
-        base = 3 + 4 * c
+        base = 3 + 5 * c
         moe.moe_dispatch_layout(cfg, tb, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
                                 B.pos, B.spl, None, B.ws)
         rec(base)
@@ -269,36 +274,44 @@ def run_steps(moe, wl, cfg, inp, B, ev=None):
         moe.moe_grouped_swiglu_ffn(cfg, B.nmax, B.xr, B.eoff, inp.w13, inp.w2, B.h, B.y, B.rt,
                                    B.rs, B.topk_w, B.red, B.ws)
         rec(base + 2)
-        if wl.reduce_dense:
-            moe.moe_reduce_finalize(cfg, B.red, tb, B.tc, B.out)
-        else:
-            moe.moe_combine(cfg, B.y, B.pos, B.topk_w, tb, B.tc, B.out)
+        if wl.shared_I > 0:
+            moe.moe_shared_expert_ffn(cfg, tb, B.tc, inp.x, inp.w13s, inp.w2s, B.hs, B.ys, B.ws)
         rec(base + 3)
+        if wl.reduce_dense:
+            moe.moe_reduce_finalize(cfg, B.red, tb, B.tc, B.out, y_shared=B.ys)
+        else:
+            moe.moe_combine(cfg, B.y, B.pos, B.topk_w, tb, B.tc, B.out, y_shared=B.ys)
+        rec(base + 4)
 
 
 def stage_times(wl, ev):
     """Per-stage milliseconds of one step recorded by run_steps."""
     t = {"route_topk": ev[0].elapsed_time(ev[1]), "capacity_clip": ev[1].elapsed_time(ev[2]),
-         "dispatch_layout": 0.0, "permute": 0.0, "grouped_ffn": 0.0, "combine": 0.0}
+         "dispatch_layout": 0.0, "permute": 0.0, "grouped_ffn": 0.0, "shared_expert": 0.0,
+         "combine": 0.0}
     for c in range(wl.n_chunks):
-        b = 3 + 4 * c
-        t["dispatch_layout"] += ev[b - 1].elapsed_time(ev[b])
+        b = 3 + 5 * c
+        prev = ev[2] if c == 0 else ev[b - 1]
+        t["dispatch_layout"] += prev.elapsed_time(ev[b])
         t["permute"] += ev[b].elapsed_time(ev[b + 1])
         t["grouped_ffn"] += ev[b + 1].elapsed_time(ev[b + 2])
-        t["combine"] += ev[b + 2].elapsed_time(ev[b + 3])
+        t["shared_expert"] += ev[b + 2].elapsed_time(ev[b + 3])
+        t["combine"] += ev[b + 3].elapsed_time(ev[b + 4])
     return t
 
 
-STAGES = ["route_topk", "capacity_clip", "dispatch_layout", "permute", "grouped_ffn", "combine"]
+STAGES = ["route_topk", "capacity_clip", "dispatch_layout", "permute", "grouped_ffn",
+          "shared_expert", "combine"]
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
 
-def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens):
+def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=None):
     """Times the oracle, as it stands, on a bounded sample: route + clip +
-    layout + permute over all T tokens, then FFN + combine for the rows of the
-    first `sample_tokens` tokens.  Returns (tokens/s extrapolated to the whole
-    layer, seconds of CPU work, description)."""
+    layout + permute over all T tokens, then FFN + combine (+ the shared expert,
+    `shared` = its host weights) for the rows of the first `sample_tokens`
+    tokens.  Returns (tokens/s extrapolated to the whole layer, seconds of CPU
+    work, description)."""
     import numpy as np
     import oracle
     t0 = time.perf_counter()
@@ -321,10 +334,13 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens):
     for p, e in rows:
         _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
     sub_pos = lay["pos"][:sample_tokens]
+    ys = None
+    if shared is not None:
+        _, ys, _ = oracle.shared_expert(x_np[:sample_tokens], shared[0], shared[1])
     if wl.reduce_dense:
-        oracle.combine_exact(ye, sub_pos, w, wl.T, x_np.dtype)
+        oracle.combine_exact(ye, sub_pos, w, wl.T, x_np.dtype, y_shared=ys)
     else:
-        oracle.combine(y, sub_pos, w, wl.T)
+        oracle.combine(y, sub_pos, w, wl.T, y_shared=ys)
     t_ffn = time.perf_counter() - t1
     layer_s = t_index + t_ffn * (wl.T / sample_tokens)
     desc = (f"oracle route+clip+layout+permute over all {wl.T} tokens ({t_index:.2f} s), FFN+combine "
@@ -370,12 +386,13 @@ def run_reference(args):
     logits = inp.logits.numpy()
     bias = None if inp.bias is None else inp.bias.numpy()
     x_np = conv(inp.x)
+    shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
     s_tok = sample_tokens_for(wl, 1.0)
     vals = []
     t_all = 0.0
     desc = ""
     for i in range(args.warmup + args.steps):
-        v, secs, desc = oracle_sample(wl, logits, bias, x_np, fetch, s_tok)
+        v, secs, desc = oracle_sample(wl, logits, bias, x_np, fetch, s_tok, shared)
         if i >= args.warmup:
             vals.append(v)
             t_all += secs
@@ -437,7 +454,8 @@ def run_ours(args):
     use_graph = not args.no_graph
 
     def layer_pass():
-        layer.forward(inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out_fw)
+        layer.forward(inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out_fw,
+                      w13_shared=inp.w13s, w2_shared=inp.w2s)
 
     for _ in range(max(args.warmup, 1)):
         flush.fill_(1)
@@ -539,7 +557,8 @@ def run_ours(args):
             d_x.copy_(h_x, non_blocking=True)
             if d_bias is not None:
                 d_bias.copy_(h_bias, non_blocking=True)
-            layer.forward(d_logits, d_bias, d_x, inp.w13, inp.w2, out_fw)
+            layer.forward(d_logits, d_bias, d_x, inp.w13, inp.w2, out_fw,
+                          w13_shared=inp.w13s, w2_shared=inp.w2s)
             h_out.copy_(out_fw, non_blocking=True)
             b.record()
             b.synchronize()
@@ -560,9 +579,10 @@ def run_ours(args):
             if wl.dtype == "bf16" else (lambda t: t.detach().cpu().numpy().copy())
         fetch = lambda e: (conv(inp.w13[e]), conv(inp.w2[e]))
         s_tok = sample_tokens_for(wl, 15.0)
+        shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
         v, secs, desc = oracle_sample(wl, inp.logits.cpu().numpy(),
                                       None if inp.bias is None else inp.bias.cpu().numpy(),
-                                      conv(inp.x), fetch, s_tok)
+                                      conv(inp.x), fetch, s_tok, shared)
         cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                "cpu_seconds": round(secs, 2)}
 

@@ -24,9 +24,11 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
                            int tc, void *xr, cudaStream_t s);
 cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,
-                           const float *topk_w, int tb, int tc, void *out, cudaStream_t s);
+                           const float *topk_w, int tb, int tc, const void *y_shared, void *out,
+                           cudaStream_t s);
 cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb, int tc,
-                                   void *out, cudaStream_t s, int num_sms);
+                                   const void *y_shared, void *out, cudaStream_t s, int num_sms);
+cudaError_t launch_shared_offsets(int32_t *off, int rows, cudaStream_t s);
 cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *xr,
                                const int32_t *expert_offsets, const void *w13, const void *w2,
                                void *h, void *y, const int32_t *recv_token,
@@ -92,6 +94,7 @@ moe_status check_range(const moe_config &c, int32_t tb, int32_t tc, bool need_ep
 // the dense fp32 reduce buffer (decode form).
 struct Slot {
     size_t eoff, roff, recv_token, recv_slot, pos, splits, xr, h, y;
+    size_t hs, ys;   // the shared expert's h and y for the chunk's rows (shared_I > 0)
 };
 struct ForwardLayout {
     size_t counts, kept_counts;
@@ -124,6 +127,8 @@ ForwardLayout forward_layout(const moe_config &c) {
         S.xr = take(eb * (size_t)F.nmax * c.H);
         S.h = take(eb * (size_t)F.nmax * c.I);
         S.y = c.reduce_dense ? 0 : take(eb * (size_t)F.nmax * c.H);
+        S.hs = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.shared_I) : 0;
+        S.ys = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.H) : 0;
     }
     F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
     F.total = off;
@@ -175,6 +180,11 @@ moe_status moe_config_check(const moe_config *cfg) {
     if (c.n_group < 0) return fail(MOE_ERR_INVALID_ARG, "n_group=%d < 0", c.n_group);
     if (c.bias_select_only != 0 && c.bias_select_only != 1)
         return fail(MOE_ERR_INVALID_ARG, "bias_select_only must be 0 or 1");
+    if (c.shared_I < 0) return fail(MOE_ERR_INVALID_ARG, "shared_I=%d < 0", c.shared_I);
+    if (c.shared_I > 0 && c.dtype == MOE_BF16 && c.shared_I % 64 != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "bf16 needs shared_I a multiple of 64 (got %d)", c.shared_I);
+    if (c.shared_I > 0 && c.dtype == MOE_F32 && c.shared_I % 4 != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "fp32 needs shared_I a multiple of 4 (got %d)", c.shared_I);
     if (c.n_group > 1) {
         if (c.n_group > kMaxGroups) return fail(MOE_ERR_UNSUPPORTED, "n_group=%d > %d", c.n_group, kMaxGroups);
         if (c.E % c.n_group != 0)
@@ -329,37 +339,92 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn");
 }
 
+// The shared expert over rows [tb, tb + tc) of x: the step-5 kernel as one
+// expert whose offsets {0, tc} live in the workspace, with its own counters.
+static cudaError_t launch_shared_ffn(const moe_config &c, int tb, int tc, const void *x,
+                                     const void *w13s, const void *w2s, void *hs, void *ys,
+                                     void *ws, cudaStream_t s, int nsm) {
+    if (tc == 0) return cudaSuccess;
+    const ScratchLayout L = scratch_layout(c);
+    int32_t *off = ws_at<int32_t>(ws, L.shared_off);
+    cudaError_t err = launch_shared_offsets(off, tc, s);
+    if (err != cudaSuccess) return err;
+    moe_config cs = c;
+    cs.E = 1;
+    cs.I = c.shared_I;
+    cs.reduce_dense = 0;
+    cs.capacity = -1;
+    const size_t eb = c.dtype == MOE_F32 ? 4 : 2;
+    const void *xs = static_cast<const unsigned char *>(x) + eb * (size_t)tb * c.H;
+    uint32_t *status = ws_at<uint32_t>(ws, L.status);
+    if (c.dtype == MOE_BF16)
+        return launch_ffn_tcgen05(cs, tc, xs, off, w13s, w2s, hs, ys, nullptr, nullptr, nullptr,
+                                  nullptr, status, ws_at<uint32_t>(ws, L.shared_ctr), s, nsm);
+    return launch_ffn_simt(cs, tc, xs, off, w13s, w2s, hs, ys, nullptr, nullptr, nullptr, nullptr, s);
+}
+
+moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
+                                 const void *x, const void *w13_shared, const void *w2_shared,
+                                 void *h_shared, void *y_shared, void *ws, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.shared_I <= 0) return fail(MOE_ERR_INVALID_ARG, "cfg has no shared expert (shared_I = 0)");
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count == 0) return MOE_OK;
+    if (!x || !w13_shared || !w2_shared || !h_shared || !y_shared)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const void *ptrs[5] = {x, w13_shared, w2_shared, h_shared, y_shared};
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    if (c.dtype == MOE_BF16) {
+        int dev = 0, major = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (major != 10)
+            return fail(MOE_ERR_UNSUPPORTED, "the bf16 FFN uses tcgen05 and needs sm_100 (got major %d)", major);
+    }
+    cudaError_t err = launch_shared_ffn(c, tok_begin, tok_count, x, w13_shared, w2_shared, h_shared,
+                                        y_shared, ws, stream, current_num_sms());
+    if (err == cudaErrorNotSupported)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_shared_expert_ffn");
+}
+
 moe_status moe_combine(const moe_config *cfg, const void *y, const int32_t *pos,
-                       const float *topk_w, int32_t tok_begin, int32_t tok_count, void *out,
-                       cudaStream_t stream) {
+                       const float *topk_w, int32_t tok_begin, int32_t tok_count,
+                       const void *y_shared, void *out, cudaStream_t stream) {
     moe_status st = moe_config_check(cfg);
     if (st != MOE_OK) return st;
     const moe_config &c = *cfg;
     if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
     if (tok_count > 0 && (!y || !pos || !topk_w || !out))
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
-    if (!aligned(y, 16) || !aligned(out, 16)) return fail(MOE_ERR_INVALID_ARG, "y / out not 16-byte aligned");
-    cudaError_t err = launch_combine(c, y, pos, topk_w, tok_begin, tok_count, out, stream);
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(y_shared, 16))
+        return fail(MOE_ERR_INVALID_ARG, "y / y_shared / out not 16-byte aligned");
+    cudaError_t err = launch_combine(c, y, pos, topk_w, tok_begin, tok_count, y_shared, out, stream);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
 }
 
 moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
-                               int32_t tok_begin, int32_t tok_count, void *out,
-                               cudaStream_t stream) {
+                               int32_t tok_begin, int32_t tok_count, const void *y_shared,
+                               void *out, cudaStream_t stream) {
     moe_status st = moe_config_check(cfg);
     if (st != MOE_OK) return st;
     const moe_config &c = *cfg;
     if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
     if (tok_count > 0 && (!out_reduce || !out)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
-    if (!aligned(out_reduce, 16) || !aligned(out, 16))
-        return fail(MOE_ERR_INVALID_ARG, "out_reduce / out not 16-byte aligned");
-    cudaError_t err = launch_reduce_finalize(c, out_reduce, tok_begin, tok_count, out, stream,
-                                             current_num_sms());
+    if (!aligned(out_reduce, 16) || !aligned(out, 16) || !aligned(y_shared, 16))
+        return fail(MOE_ERR_INVALID_ARG, "out_reduce / y_shared / out not 16-byte aligned");
+    cudaError_t err = launch_reduce_finalize(c, out_reduce, tok_begin, tok_count, y_shared, out,
+                                             stream, current_num_sms());
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_reduce_finalize");
 }
 
 moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
-                               const void *x, const void *w13, const void *w2, void *out,
+                               const void *x, const void *w13, const void *w2,
+                               const void *w13_shared, const void *w2_shared, void *out,
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
                                cudaStream_t s_compute) {
@@ -369,6 +434,8 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     const moe_config &c = *cfg;
     if (c.T > 0 && (!logits || !x || !w13 || !w2 || !out || !topk_idx || !topk_w || !keep))
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
+        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
     if (c.T == 0) return MOE_OK;
     const ForwardLayout F = forward_layout(c);
     const ScratchLayout L = scratch_layout(c);
@@ -379,11 +446,12 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     const int nsm = current_num_sms();
     const int nch = c.n_chunks;
 
+    const bool shared = c.shared_I > 0;
     cudaEvent_t *ev = nullptr;
-    cudaError_t err = get_events(2 * nch + 2, &ev);
+    cudaError_t err = get_events(3 * nch + 2, &ev);
     if (err != cudaSuccess) return cuda_fail(err, "event pool");
     cudaEvent_t ev_start = ev[0], ev_end = ev[1];
-    cudaEvent_t *ev_disp = ev + 2, *ev_done = ev + 2 + nch;
+    cudaEvent_t *ev_disp = ev + 2, *ev_done = ev + 2 + nch, *ev_shared = ev + 2 + 2 * nch;
 
 #define MOE_TRY(expr, where)                                   \
     do {                                                       \
@@ -424,6 +492,16 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
                 "dispatch_layout");
         MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, s_dispatch), "permute");
         MOE_TRY(cudaEventRecord(ev_disp[ch], s_dispatch), "record dispatch");
+        void *ys = shared ? ws_at<void>(ws, S.ys) : nullptr;
+        if (shared) {
+            // the shared expert of the chunk beside its routed FFN; the combine waits for it
+            err = launch_shared_ffn(c, tb, tc, x, w13_shared, w2_shared, ws_at<void>(ws, S.hs), ys,
+                                    ws, s_dispatch, nsm);
+            if (err == cudaErrorNotSupported)
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+            MOE_TRY(err, "shared_expert_ffn");
+            MOE_TRY(cudaEventRecord(ev_shared[ch], s_dispatch), "record shared");
+        }
         MOE_TRY(cudaStreamWaitEvent(s_compute, ev_disp[ch], 0), "wait dispatch");
         if (F.nmax > 0) {
             if (c.dtype == MOE_BF16) {
@@ -438,10 +516,11 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
             }
             MOE_TRY(err, "grouped_swiglu_ffn");
         }
+        if (shared) MOE_TRY(cudaStreamWaitEvent(s_compute, ev_shared[ch], 0), "wait shared");
         if (c.reduce_dense)
-            MOE_TRY(launch_reduce_finalize(c, out_reduce, tb, tc, out, s_compute, nsm), "reduce_finalize");
+            MOE_TRY(launch_reduce_finalize(c, out_reduce, tb, tc, ys, out, s_compute, nsm), "reduce_finalize");
         else
-            MOE_TRY(launch_combine(c, y, pos, topk_w, tb, tc, out, s_compute), "combine");
+            MOE_TRY(launch_combine(c, y, pos, topk_w, tb, tc, ys, out, s_compute), "combine");
         MOE_TRY(cudaEventRecord(ev_done[ch], s_compute), "record done");
     }
     MOE_TRY(cudaEventRecord(ev_end, s_compute), "record end");

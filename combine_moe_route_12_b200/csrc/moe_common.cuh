@@ -41,9 +41,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up aft
 //   tile_state      uint32[max_tiles * E] (decoupled-lookback descriptors)
 //   clip threshold  uint64[E]
 //   ffn counters    uint32[2] (dynamic work distribution of the FFN GEMMs)
+//   shared expert   uint32[2] counters, int32[2] expert offsets
 //   clip segments   int32[2 * (E + 1)] offsets / cursors, keys uint64[T * k]
 struct ScratchLayout {
     size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr;
+    size_t shared_ctr, shared_off;
     size_t clip_seg, clip_keys, total;
     int max_tiles;
 };
@@ -60,6 +62,8 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     L.tile_state = off;           off = align_up(off + sizeof(uint32_t) * (size_t)L.max_tiles * c.E, 256);
     L.clip_thr = off;             off = align_up(off + sizeof(uint64_t) * (size_t)c.E, 256);
     L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
+    L.shared_ctr = off;           off += 256;   // the shared expert's own two counters
+    L.shared_off = off;           off += 256;   // its expert offsets {0, rows}
     L.clip_seg = off;             off = align_up(off + sizeof(int32_t) * 2 * ((size_t)c.E + 1), 256);
     L.clip_keys = off;            off = align_up(off + sizeof(uint64_t) * (size_t)c.T * c.k, 256);
     L.total = off;

@@ -49,7 +49,7 @@ constexpr int kCombineBatch = 4;   // expert rows of a token loaded together
 // bf16 storage: one uint4 = 8 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
     int tb, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
-    const float *__restrict__ topk_w, uint4 *__restrict__ out) {
+    const float *__restrict__ topk_w, const uint4 *__restrict__ y_shared, uint4 *__restrict__ out) {
     __shared__ int32_t s_pos[kMaxTopK];
     __shared__ float s_w[kMaxTopK];
     const int i = blockIdx.x;
@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
     __syncthreads();
     for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (y_shared) unpack8(__ldg(y_shared + (size_t)i * row_vecs + v), acc);   // the shared expert's row
         for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
             // the batch's rows are loaded before the first is added, so one
             // thread has up to kCombineBatch loads in flight; the adds keep slot order
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
 // fp32 storage: one float4 = 4 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
     int tb, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
-    const float *__restrict__ topk_w, float4 *__restrict__ out) {
+    const float *__restrict__ topk_w, const float4 *__restrict__ y_shared, float4 *__restrict__ out) {
     __shared__ int32_t s_pos[kMaxTopK];
     __shared__ float s_w[kMaxTopK];
     const int i = blockIdx.x;
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
     }
     __syncthreads();
     for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = y_shared ? __ldg(y_shared + (size_t)i * row_vecs + v) : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
             const int p = s_pos[j];
             if (p < 0) continue;
@@ -120,12 +121,26 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
 
 // Decode form: out[t] = round(out_reduce[t]) for the chunk's tokens.
 __global__ void reduce_finalize_kernel(int tb, int tc, int H, int dtype,
-                                       const float4 *__restrict__ red, void *__restrict__ out) {
+                                       const float4 *__restrict__ red, const void *__restrict__ y_shared,
+                                       void *__restrict__ out) {
     const size_t n4 = (size_t)tc * H / 4;
     const size_t base4 = (size_t)tb * H / 4;
     for (size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
          q += (size_t)gridDim.x * blockDim.x) {
-        const float4 v = red[base4 + q];
+        float4 v = red[base4 + q];
+        if (y_shared) {   // the shared expert's row (chunk-relative), added before the rounding
+            float s[4];
+            if (dtype == MOE_F32) {
+                const float4 f = reinterpret_cast<const float4 *>(y_shared)[q];
+                s[0] = f.x; s[1] = f.y; s[2] = f.z; s[3] = f.w;
+            } else {
+                const uint2 u = reinterpret_cast<const uint2 *>(y_shared)[q];
+                s[0] = __uint_as_float(u.x << 16); s[1] = __uint_as_float(u.x & 0xFFFF0000u);
+                s[2] = __uint_as_float(u.y << 16); s[3] = __uint_as_float(u.y & 0xFFFF0000u);
+            }
+            v.x = __fadd_rn(s[0], v.x); v.y = __fadd_rn(s[1], v.y);
+            v.z = __fadd_rn(s[2], v.z); v.w = __fadd_rn(s[3], v.w);
+        }
         if (dtype == MOE_F32) {
             reinterpret_cast<float4 *>(out)[base4 + q] = v;
         } else {
@@ -148,30 +163,41 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *po
 }
 
 cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,
-                           const float *topk_w, int tb, int tc, void *out, cudaStream_t s) {
+                           const float *topk_w, int tb, int tc, const void *y_shared, void *out,
+                           cudaStream_t s) {
     if (tc == 0) return cudaSuccess;
     if (c.dtype == MOE_F32) {
         const int row_vecs = c.H / 4;
         combine_rows_f32_kernel<<<tc, kRowThreads, 0, s>>>(
             tb, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
-            static_cast<float4 *>(out));
+            static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
     } else {
         const int row_vecs = c.H / 8;
         combine_rows_bf16_kernel<<<tc, kRowThreads, 0, s>>>(
             tb, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
-            static_cast<uint4 *>(out));
+            static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb, int tc,
-                                   void *out, cudaStream_t s, int num_sms) {
+                                   const void *y_shared, void *out, cudaStream_t s, int num_sms) {
     if (tc == 0) return cudaSuccess;
     const size_t n4 = (size_t)tc * c.H / 4;
     int blocks = (int)((n4 + 255) / 256);
     if (blocks > num_sms * 8) blocks = num_sms * 8;
     reduce_finalize_kernel<<<blocks, 256, 0, s>>>(tb, tc, c.H, c.dtype,
-                                                  reinterpret_cast<const float4 *>(red), out);
+                                                  reinterpret_cast<const float4 *>(red), y_shared, out);
+    return cudaGetLastError();
+}
+
+// Expert offsets {0, rows} of the shared expert's one-expert FFN launch.
+__global__ void shared_offsets_kernel(int32_t *off, int rows) {
+    off[0] = 0;
+    off[1] = rows;
+}
+cudaError_t launch_shared_offsets(int32_t *off, int rows, cudaStream_t s) {
+    shared_offsets_kernel<<<1, 1, 0, s>>>(off, rows);
     return cudaGetLastError();
 }
 

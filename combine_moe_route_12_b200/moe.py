@@ -30,7 +30,7 @@ MOE_DEV_BAD_INDEX = 0x4
 class MoEConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "H", "E", "k", "I", "ep", "capacity", "dtype", "n_chunks", "reduce_dense",
-                 "n_group", "topk_group", "group_score", "bias_select_only")]
+                 "n_group", "topk_group", "group_score", "bias_select_only", "shared_I")]
 
     def __repr__(self):
         return "MoEConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -64,9 +64,10 @@ _decl("moe_dispatch_layout", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P,
 _decl("moe_dispatch_layout_noalloc", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
 _decl("moe_grouped_swiglu_ffn", _I32, _CFG, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
-_decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P)
-_decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P)
-_decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_shared_expert_ffn", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_last_error_detail", ctypes.c_char_p)
@@ -108,18 +109,18 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def make_config(T, H, E, k, I, ep, capacity=-1, dtype=MOE_BF16, n_chunks=1,
                 reduce_dense=False, n_group=0, topk_group=0, group_score=0,
-                bias_select_only=False) -> MoEConfig:
+                bias_select_only=False, shared_I=0) -> MoEConfig:
     if isinstance(dtype, str):
         dtype = MOE_F32 if dtype == "f32" else MOE_BF16
     return MoEConfig(T, H, E, k, I, ep, -1 if capacity is None else capacity, dtype, n_chunks,
                      int(bool(reduce_dense)), n_group, topk_group, group_score,
-                     int(bool(bias_select_only)))
+                     int(bool(bias_select_only)), shared_I)
 
 
 def config_from_workload(wl) -> MoEConfig:
     return make_config(wl.T, wl.H, wl.E, wl.k, wl.I, wl.ep, wl.capacity, wl.dtype, wl.n_chunks,
                        wl.reduce_dense, wl.n_group, wl.topk_group, wl.group_score,
-                       wl.bias_select_only)
+                       wl.bias_select_only, wl.shared_I)
 
 
 # ------------------------------------------------------------------ sizes
@@ -192,20 +193,28 @@ def moe_grouped_swiglu_ffn(cfg, n_rows, xr, expert_offsets, w13, w2, h, y, recv_
                                        _stream(stream)))
 
 
-def moe_combine(cfg, y, pos, topk_w, tok_begin, tok_count, out, stream=None):
+def moe_combine(cfg, y, pos, topk_w, tok_begin, tok_count, out, stream=None, y_shared=None):
     _check(_lib.moe_combine(ctypes.byref(cfg), _ptr(y), _ptr(pos), _ptr(topk_w), tok_begin,
-                            tok_count, _ptr(out), _stream(stream)))
+                            tok_count, _ptr(y_shared), _ptr(out), _stream(stream)))
 
 
-def moe_reduce_finalize(cfg, out_reduce, tok_begin, tok_count, out, stream=None):
+def moe_reduce_finalize(cfg, out_reduce, tok_begin, tok_count, out, stream=None, y_shared=None):
     _check(_lib.moe_reduce_finalize(ctypes.byref(cfg), _ptr(out_reduce), tok_begin, tok_count,
-                                    _ptr(out), _stream(stream)))
+                                    _ptr(y_shared), _ptr(out), _stream(stream)))
+
+
+def moe_shared_expert_ffn(cfg, tok_begin, tok_count, x, w13_shared, w2_shared, h_shared, y_shared,
+                          ws, stream=None):
+    _check(_lib.moe_shared_expert_ffn(ctypes.byref(cfg), tok_begin, tok_count, _ptr(x),
+                                      _ptr(w13_shared), _ptr(w2_shared), _ptr(h_shared),
+                                      _ptr(y_shared), _ptr(ws), _stream(stream)))
 
 
 def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, keep, splits_host,
-                        ws, s_dispatch=None, s_compute=None):
+                        ws, s_dispatch=None, s_compute=None, w13_shared=None, w2_shared=None):
     _check(_lib.moe_forward_chunked(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(x),
-                                    _ptr(w13), _ptr(w2), _ptr(out), _ptr(topk_idx), _ptr(topk_w),
+                                    _ptr(w13), _ptr(w2), _ptr(w13_shared), _ptr(w2_shared),
+                                    _ptr(out), _ptr(topk_idx), _ptr(topk_w),
                                     _ptr(keep), _ptr(splits_host), _ptr(ws),
                                     _stream(s_dispatch), _stream(s_compute)))
 
@@ -241,10 +250,12 @@ class MoELayer:
         self.splits_host = torch.zeros(n, dtype=torch.int32, pin_memory=True) if host_splits else None
         self.s_dispatch = torch.cuda.Stream(device=dev)
 
-    def forward(self, logits, bias, x, w13, w2, out, s_compute=None):
+    def forward(self, logits, bias, x, w13, w2, out, s_compute=None, w13_shared=None,
+                w2_shared=None):
         s_compute = s_compute or torch.cuda.current_stream()
         moe_forward_chunked(self.cfg, logits, bias, x, w13, w2, out, self.topk_idx, self.topk_w,
-                            self.keep, self.splits_host, self.ws, self.s_dispatch, s_compute)
+                            self.keep, self.splits_host, self.ws, self.s_dispatch, s_compute,
+                            w13_shared, w2_shared)
         return out
 
     def splits(self, chunk: int):

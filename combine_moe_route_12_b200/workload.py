@@ -35,6 +35,8 @@ Input recipe (the pages fix none of it; every choice is a stated reading):
   part of the hot path.
 * the skewed workload adds bias[e] = 3 * ln(p_{rank(e)}), p_r proportional to
   r^-1.2 for r = 1..128 and normalised, with rank(e) a seeded permutation.
+* a workload with ``shared_I`` > 0 also draws a shared expert, w13s [2 I_s, H]
+  and w2s [H, I_s] ~ N(0, 1/H), from its own seeded generator.
 * ``dsv3_grouped`` (routing variants, DSV3 prefill shape in one chunk): grouped
   top-k with 8 groups of 32 experts and 4 kept per token (group score: the sum
   of a group's two best biased logits), and a load-balancing-like bias
@@ -69,6 +71,7 @@ class MoEWorkload:
     group_score: int = 0          # 0: best logit of the group; 1: sum of its two best
     bias_select_only: bool = False
     balance_bias: bool = False    # a small per-expert bias ~ N(0, 0.5^2), the load-balancing kind
+    shared_I: int = 0             # a shared expert of this intermediate size (0: none)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -94,10 +97,10 @@ WORKLOADS = {
                                dtype="bf16", ep=64, capacity=1024, reduce_dense=True),
     # routing variants on the DSV3 prefill shape (one chunk): 8 groups of 32
     # experts, 4 kept per token by the sum of their two best biased logits, the
-    # bias used for the selection only
+    # bias used for the selection only, and one shared expert of I = 2048
     "dsv3_grouped": MoEWorkload("dsv3_grouped", T=8192, H=7168, E=256, k=8, I=2048,
                                 dtype="bf16", ep=8, n_group=8, topk_group=4, group_score=1,
-                                bias_select_only=True, balance_bias=True),
+                                bias_select_only=True, balance_bias=True, shared_I=2048),
 }
 
 
@@ -110,6 +113,8 @@ class MoEInputs:
     x: torch.Tensor           # [T, H]
     w13: torch.Tensor         # [E, 2I, H]
     w2: torch.Tensor          # [E, H, I]
+    w13s: torch.Tensor | None = None   # shared expert [2 I_s, H]
+    w2s: torch.Tensor | None = None    # shared expert [H, I_s]
 
 
 def zipf_bias(E: int, s: float, gen: torch.Generator) -> torch.Tensor:
@@ -163,5 +168,12 @@ def make_inputs(wl: MoEWorkload, device: str | torch.device = "cpu",
     else:
         w13 = torch.empty(0, dtype=dt, device=device)
         w2 = torch.empty(0, dtype=dt, device=device)
+    w13s = w2s = None
+    if wl.shared_I > 0:
+        # the shared expert draws from its own seeded stream, after the routed ones
+        gs = torch.Generator(device=device)
+        gs.manual_seed(seed + 15485863)
+        w13s = (torch.randn(2 * wl.shared_I, wl.H, generator=gs, device=device) * std).to(dt)
+        w2s = (torch.randn(wl.H, wl.shared_I, generator=gs, device=device) * std).to(dt)
     return MoEInputs(logits=logits.contiguous(), bias=bias, x=x.contiguous(),
-                     w13=w13, w2=w2)
+                     w13=w13, w2=w2, w13s=w13s, w2s=w2s)

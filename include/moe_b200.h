@@ -90,7 +90,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * contiguous source-rank blocks).
  * Routing-variant checks (MOE_ERR_INVALID_ARG): n_group >= 0, E % n_group == 0,
  * topk_group and k as stated at the fields, group_score in {0, 1},
- * bias_select_only in {0, 1}.
+ * bias_select_only in {0, 1}, shared_I >= 0 (a multiple of 64 for MOE_BF16, of
+ * 4 for MOE_F32).
  * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30,
  * n_group <= 32;
  * MOE_BF16 needs H % 64 == 0 and I % 64 == 0 (tensor-core tiles);
@@ -121,6 +122,11 @@ typedef struct {
     int32_t topk_group;
     int32_t group_score;
     int32_t bias_select_only;
+    /* Shared expert ([LL]: shared expert overlap kept in the combine): its
+     * intermediate size (0: none).  One dense SwiGLU expert with weights
+     * w13_shared [2*shared_I, H] and w2_shared [H, shared_I] applied to every
+     * token; its output is added into the combine's sum. */
+    int32_t shared_I;
 } moe_config;
 
 /* Validates cfg (topology and limits).  MOE_OK or the reason it is rejected. */
@@ -272,13 +278,32 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
  */
 moe_status moe_combine(const moe_config *cfg, const void *y, const int32_t *pos,
                        const float *topk_w, int32_t tok_begin, int32_t tok_count,
-                       void *out, cudaStream_t stream);
+                       const void *y_shared, void *out, cudaStream_t stream);
 
 /* Decode form of step 6: out[t, :] = round(out_reduce[t, :]) for the tokens
- * [tok_begin, tok_begin + tok_count). */
+ * [tok_begin, tok_begin + tok_count).
+ * In both, y_shared is NULL or the chunk's [tok_count, H] rows of the shared
+ * expert's output (moe_shared_expert_ffn, cfg->dtype), added into the fp32 sum
+ * before its one rounding. */
 moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
-                               int32_t tok_begin, int32_t tok_count, void *out,
-                               cudaStream_t stream);
+                               int32_t tok_begin, int32_t tok_count, const void *y_shared,
+                               void *out, cudaStream_t stream);
+
+/*
+ * The shared expert ([LL]: DeepSeek-style shared expert, its work overlapped
+ * with the routed path and its output added in the combine): for the rows
+ * t in [tok_begin, tok_begin + tok_count) of x [T, H]
+ *   h_shared[t - tok_begin] = silu(Wg x_t) * (Wu x_t)    [tok_count, shared_I]
+ *   y_shared[t - tok_begin] = W2s h_shared[t - tok_begin] [tok_count, H]
+ * with w13_shared [2*shared_I, H] (gate rows then up rows) and w2_shared
+ * [H, shared_I], both cfg->dtype, row-major.  The same kernel as step 5, run
+ * as one expert over the chunk's rows (no permutation).  Needs shared_I > 0;
+ * ws: moe_workspace_bytes(cfg) (its work counters are not those of step 5, so
+ * the two may run on different streams at once).
+ */
+moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
+                                 const void *x, const void *w13_shared, const void *w2_shared,
+                                 void *h_shared, void *y_shared, void *ws, cudaStream_t stream);
 
 /*
  * The whole layer, chunked ([AX] expert_parallel_dispatch_chunks; [LL]
@@ -290,6 +315,10 @@ moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
  * only after chunk c-2's combine finished.  n_chunks = 1 gives the unchunked
  * layer.  The result equals the unchunked one bit for bit.
  *   logits, bias, x, w13, w2 as in steps 1-5; out [T, H] cfg->dtype.
+ *   w13_shared, w2_shared: the shared expert's weights when cfg->shared_I > 0
+ *            (else ignored, may be NULL).  Chunk c's shared expert runs on
+ *            s_dispatch after its dispatch, beside chunk c's routed FFN on
+ *            s_compute, and its rows are added in chunk c's combine.
  *   topk_idx [T,k], topk_w [T,k], keep [T,k]: caller-owned saved state
  *            ([AX] the routing top-k is always saved).
  *   splits_host: pinned host int32 [n_chunks * (E+1 + ep*ep)] or NULL; chunk c
@@ -301,7 +330,8 @@ moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
  *            allocator must see them used on both).
  */
 moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
-                               const void *x, const void *w13, const void *w2, void *out,
+                               const void *x, const void *w13, const void *w2,
+                               const void *w13_shared, const void *w2_shared, void *out,
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws,
                                cudaStream_t s_dispatch, cudaStream_t s_compute);

@@ -50,6 +50,12 @@ def assert_float_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str) 
     return rel
 
 
+def to_device(inp: MoEInputs, device="cuda") -> MoEInputs:
+    mv = lambda t: None if t is None else t.to(device)
+    return MoEInputs(logits=mv(inp.logits), bias=mv(inp.bias), x=mv(inp.x), w13=mv(inp.w13),
+                     w2=mv(inp.w2), w13s=mv(inp.w13s), w2s=mv(inp.w2s))
+
+
 def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> dict:
     """Runs the six ABI steps chunk by chunk on the current CUDA stream."""
     cfg = moe.config_from_workload(wl)
@@ -83,10 +89,15 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
         h = torch.empty((max(nmax, 1), I), dtype=wl.torch_dtype, device=dev)
         y = None if wl.reduce_dense else torch.empty((max(nmax, 1), H), dtype=wl.torch_dtype, device=dev)
         moe.moe_grouped_swiglu_ffn(cfg, nmax, xr, eoff, inp.w13, inp.w2, h, y, rt, rs, topk_w, red, ws)
+        ys = None
+        if wl.shared_I > 0:
+            hs = torch.empty((tc, wl.shared_I), dtype=wl.torch_dtype, device=dev)
+            ys = torch.empty((tc, H), dtype=wl.torch_dtype, device=dev)
+            moe.moe_shared_expert_ffn(cfg, tb, tc, inp.x, inp.w13s, inp.w2s, hs, ys, ws)
         if wl.reduce_dense:
-            moe.moe_reduce_finalize(cfg, red, tb, tc, out)
+            moe.moe_reduce_finalize(cfg, red, tb, tc, out, y_shared=ys)
         else:
-            moe.moe_combine(cfg, y, pos, topk_w, tb, tc, out)
+            moe.moe_combine(cfg, y, pos, topk_w, tb, tc, out, y_shared=ys)
         torch.cuda.synchronize()
         n = int(eoff[E].item())
         ch = dict(N=n, expert_offsets=eoff.cpu().numpy(), rank_offsets=roff.cpu().numpy(),
@@ -94,9 +105,10 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
                   pos=pos.cpu().numpy(), send_splits=spl.cpu().numpy(), host=host.numpy().copy())
         if keep_rows:
             ch.update(xr=storage_np(xr[:n]), h=storage_np(h[:n]),
-                      y=None if y is None else storage_np(y[:n]))
+                      y=None if y is None else storage_np(y[:n]),
+                      ys=None if ys is None else storage_np(ys))
         else:
-            ch.update(xr_dev=xr, h_dev=h, y_dev=y)
+            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys)
         chunks.append(ch)
     status = moe.moe_device_status(ws)
     torch.cuda.synchronize()

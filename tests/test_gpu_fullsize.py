@@ -69,7 +69,17 @@ def test_fullsize_against_oracle(name):
 
     out = storage_np(g["out"])
     tokens = sorted({0, wl.T - 1, *rng.integers(0, wl.T, 2).tolist()})
+    shared = None
+    if wl.shared_I > 0:
+        shared = (storage_np(inp.w13s), storage_np(inp.w2s))
+    tc = wl.T // wl.n_chunks
     for t in tokens:
+        ysh = None
+        if shared is not None:
+            # the shared expert's row of token t, checked against the GPU's and used below
+            _, ysh, _ = oracle.shared_expert(x_np[t:t + 1], *shared)
+            gys = storage_np(g["chunks"][t // tc]["ys_dev"][t % tc:t % tc + 1])
+            assert_float_close(gys, ysh, wl.dtype, f"y_shared[{t}]")
         ys, yes, pos = [], [], []
         for j in range(wl.k):
             if not orc["keep"][t, j]:
@@ -83,11 +93,11 @@ def test_fullsize_against_oracle(name):
         posa = np.array([pos], np.int32)
         w_t = orc["topk_w"][t:t + 1]
         if not ys:
-            ref = np.zeros((1, wl.H), x_np.dtype)
+            ref = np.zeros((1, wl.H), x_np.dtype) if ysh is None else ysh
         elif wl.reduce_dense:
-            ref = oracle.combine_exact(np.stack(yes), posa, w_t, 1, x_np.dtype)
+            ref = oracle.combine_exact(np.stack(yes), posa, w_t, 1, x_np.dtype, y_shared=ysh)
         else:
-            ref = oracle.combine(np.stack(ys), posa, w_t, 1)
+            ref = oracle.combine(np.stack(ys), posa, w_t, 1, y_shared=ysh)
         assert_float_close(out[t:t + 1], ref, wl.dtype, f"out[{t}]")
     del g, inp
     torch.cuda.empty_cache()

@@ -15,7 +15,7 @@ import oracle
 from combine_moe_route_12_b200.workload import MoEWorkload, make_inputs
 
 from moe_testlib import (assert_float_close, assert_routing_equal, oracle_routing,
-                         run_gpu_steps, storage_np)
+                         run_gpu_steps, storage_np, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +59,12 @@ CASES = {
     # fp32, skewed bias in the selection only
     "f32_selbias_skew": W("f32_selbias_skew", T=256, H=128, E=8, k=2, I=128, dtype="f32", ep=2,
                           skew_bias=True, bias_select_only=True),
+    # a shared expert beside the routed ones (two chunks, and in the decode form)
+    "bf16_shared": W("bf16_shared", T=256, H=128, E=16, k=4, I=64, dtype="bf16", ep=2,
+                     shared_I=128, n_chunks=2),
+    "bf16_shared_decode": W("bf16_shared_decode", T=64, H=256, E=32, k=8, I=128, dtype="bf16",
+                            ep=8, capacity=32, reduce_dense=True, shared_I=192),
+    "f32_shared": W("f32_shared", T=128, H=128, E=8, k=2, I=128, dtype="f32", ep=2, shared_I=64),
 }
 
 
@@ -72,11 +78,15 @@ def _oracle_ffn_and_out(wl, inp, orc):
     for c, lay in enumerate(orc["layouts"]):
         xr = oracle.permute(x, lay["recv_token"])
         h, y, ye = oracle.ffn(xr, lay["expert_offsets"], w13, w2)
+        ys = None
+        if wl.shared_I > 0:
+            _, ys, _ = oracle.shared_expert(x[c * tc:(c + 1) * tc], storage_np(inp.w13s),
+                                            storage_np(inp.w2s))
         if wl.reduce_dense:
-            oracle.combine_exact(ye, lay["pos"], orc["topk_w"], wl.T, x.dtype, c * tc, out)
+            oracle.combine_exact(ye, lay["pos"], orc["topk_w"], wl.T, x.dtype, c * tc, out, y_shared=ys)
         else:
-            oracle.combine(y, lay["pos"], orc["topk_w"], wl.T, c * tc, out)
-        res.append(dict(xr=xr, h=h, y=y))
+            oracle.combine(y, lay["pos"], orc["topk_w"], wl.T, c * tc, out, y_shared=ys)
+        res.append(dict(xr=xr, h=h, y=y, ys=ys))
     return res, out
 
 
@@ -84,8 +94,7 @@ def _oracle_ffn_and_out(wl, inp, orc):
 def test_layer_steps_match_oracle(name):
     wl = CASES[name]
     inp = make_inputs(wl, "cpu", seed=1)
-    dinp = type(inp)(logits=inp.logits.cuda(), bias=None if inp.bias is None else inp.bias.cuda(),
-                     x=inp.x.cuda(), w13=inp.w13.cuda(), w2=inp.w2.cuda())
+    dinp = to_device(inp)
     g = run_gpu_steps(wl, dinp)
     assert g["status"] == 0
     orc = oracle_routing(wl, inp)
@@ -96,6 +105,8 @@ def test_layer_steps_match_oracle(name):
         assert_float_close(gc["h"], oc["h"], wl.dtype, "h")
         if not wl.reduce_dense:
             assert_float_close(gc["y"], oc["y"], wl.dtype, "y")
+        if oc["ys"] is not None:
+            assert_float_close(gc["ys"], oc["ys"], wl.dtype, "y_shared")
     assert_float_close(storage_np(g["out"]), out, wl.dtype, "out")
     if wl.capacity == 0:
         assert (storage_np(g["out"]) == 0).all()
@@ -110,21 +121,22 @@ def _forward(wl, dinp, n_chunks, same_stream=False):
     if same_stream:
         moe.moe_forward_chunked(layer.cfg, dinp.logits, dinp.bias, dinp.x, dinp.w13, dinp.w2, out,
                                 layer.topk_idx, layer.topk_w, layer.keep, layer.splits_host,
-                                layer.ws, s, s)
+                                layer.ws, s, s, dinp.w13s, dinp.w2s)
     else:
-        layer.forward(dinp.logits, dinp.bias, dinp.x, dinp.w13, dinp.w2, out)
+        layer.forward(dinp.logits, dinp.bias, dinp.x, dinp.w13, dinp.w2, out,
+                      w13_shared=dinp.w13s, w2_shared=dinp.w2s)
     torch.cuda.synchronize()
     assert moe.moe_device_status(layer.ws) == 0
     return out, layer
 
 
 @pytest.mark.parametrize("name", ["bf16_ragged_m", "bf16_capacity", "bf16_chunked", "tiny_f32",
-                                  "bf16_decode"])
+                                  "bf16_decode", "bf16_shared", "bf16_shared_decode",
+                                  "bf16_grouped_top2_selbias"])
 def test_forward_chunked_matches_steps_and_oracle(name):
     wl = CASES[name]
     inp = make_inputs(wl, "cpu", seed=2)
-    dinp = type(inp)(logits=inp.logits.cuda(), bias=None if inp.bias is None else inp.bias.cuda(),
-                     x=inp.x.cuda(), w13=inp.w13.cuda(), w2=inp.w2.cuda())
+    dinp = to_device(inp)
     out_c, layer = _forward(wl, dinp, wl.n_chunks)
     orc = oracle_routing(wl, inp)
     np.testing.assert_array_equal(layer.topk_idx.cpu().numpy(), orc["topk_idx"])
