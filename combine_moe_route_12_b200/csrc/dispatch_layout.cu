@@ -128,12 +128,9 @@ __device__ __forceinline__ bool lookback_prefix(const uint32_t *tile_state, int 
         for (int i = 0; i < kLookbackWindow; ++i) {
             if (i >= n) break;
             uint32_t w = v[i];
-            if ((w >> 30) == 0) {
-                const uint32_t *q = tile_state + (size_t)(p - i) * E + e;
-                const uint64_t t0 = global_timer_ns();
-                while (((w = ld_relaxed_u32(q)) >> 30) == 0)
-                    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-            }
+            if ((w >> 30) == 0 &&
+                !wait_flag_word_bounded(tile_state + (size_t)(p - i) * E + e, w))
+                return false;
             excl += w & kValueMask;
             if ((w & ~kValueMask) == kFlagInclusive) return true;
         }

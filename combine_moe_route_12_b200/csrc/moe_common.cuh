@@ -45,7 +45,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up aft
 //   clip segments   int32[2 * (E + 1)] offsets / cursors, keys uint64[T * k]
 struct ScratchLayout {
     size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr;
-    size_t shared_ctr, shared_off;
+    size_t shared_ctr, shared_off, watchdog;
     size_t clip_seg, clip_keys, total;
     int max_tiles;
 };
@@ -64,6 +64,7 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
     L.shared_ctr = off;           off += 256;   // the shared expert's own two counters
     L.shared_off = off;           off += 256;   // its expert offsets {0, rows}
+    L.watchdog = off;             off += 256;   // a word nothing ever sets (watchdog self-test)
     L.clip_seg = off;             off = align_up(off + sizeof(int32_t) * 2 * ((size_t)c.E + 1), 256);
     L.clip_keys = off;            off = align_up(off + sizeof(uint64_t) * (size_t)c.T * c.k, 256);
     L.total = off;
@@ -119,15 +120,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // kWaitLimitNs or as soon as another role of the CTA set *abort_flag;
 // returns false then.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort_flag) {
+                                                  volatile int *abort_flag,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
         }
+    }
+}
+
+// Spins (relaxed loads) until the 2-bit flag field (bits 30-31) of *q is set,
+// as the dispatch layout's look-back waits for a predecessor's descriptor.
+// Returns false after limit_ns; w receives the last value read.
+__device__ __forceinline__ bool wait_flag_word_bounded(const uint32_t *q, uint32_t &w,
+                                                       uint64_t limit_ns = kWaitLimitNs) {
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w) : "l"(q) : "memory");
+        if ((w >> 30) != 0) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 

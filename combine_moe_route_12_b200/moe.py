@@ -68,6 +68,7 @@ _decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_shared_expert_ffn", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_last_error_detail", ctypes.c_char_p)
@@ -217,6 +218,12 @@ def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, ke
                                     _ptr(out), _ptr(topk_idx), _ptr(topk_w),
                                     _ptr(keep), _ptr(splits_host), _ptr(ws),
                                     _stream(s_dispatch), _stream(s_compute)))
+
+
+def moe_watchdog_selftest(cfg, which: int, limit_us: int, ws, stream=None):
+    """Runs one of the library's bounded waits on something that never completes
+    (0: the look-back spin, 1: an mbarrier wait); it sets MOE_DEV_WAIT_TIMEOUT."""
+    _check(_lib.moe_watchdog_selftest(ctypes.byref(cfg), which, limit_us, _ptr(ws), _stream(stream)))
 
 
 def moe_device_status(ws, stream=None) -> int:

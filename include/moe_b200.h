@@ -336,6 +336,21 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
                                int32_t *splits_host, void *ws,
                                cudaStream_t s_dispatch, cudaStream_t s_compute);
 
+/*
+ * Watchdog self-test (failure detection; no counterpart on the pages): runs the
+ * library's own bounded-wait code on something that never completes, with a
+ * short limit, so a caller can check that a wait that runs out is reported and
+ * that the context stays usable.
+ *   which 0: the dispatch layout's look-back spin on a descriptor word nothing
+ *            publishes (a zero word of ws);
+ *   which 1: the FFN's mbarrier wait on a barrier nothing arrives at.
+ *   limit_us in [1, 2000000].
+ * One thread waits about limit_us, sets MOE_DEV_WAIT_TIMEOUT in ws's status word
+ * and returns; read it with moe_device_status.  ws: moe_workspace_bytes(cfg).
+ */
+moe_status moe_watchdog_selftest(const moe_config *cfg, int32_t which, int32_t limit_us,
+                                 void *ws, cudaStream_t stream);
+
 /* Synchronises `stream`, copies the device status word of ws to *flags and
  * clears it.  Returns MOE_ERR_DEVICE if any bit was set. */
 moe_status moe_device_status(void *ws, uint32_t *flags, cudaStream_t stream);
