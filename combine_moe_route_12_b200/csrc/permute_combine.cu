@@ -59,34 +59,53 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
         s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
     }
     __syncthreads();
-    for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (y_shared) unpack8(__ldg(y_shared + (size_t)i * row_vecs + v), acc);   // the shared expert's row
+    // two 16-byte columns per pass, all their row loads issued before any add or
+    // store: a token with one or two kept rows still has several loads in flight
+    for (int v0 = threadIdx.x; v0 < row_vecs; v0 += 2 * kRowThreads) {
+        const int v1 = v0 + kRowThreads;
+        const bool has1 = v1 < row_vecs;
+        float acc0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (y_shared) {   // the shared expert's row
+            unpack8(__ldg(y_shared + (size_t)i * row_vecs + v0), acc0);
+            if (has1) unpack8(__ldg(y_shared + (size_t)i * row_vecs + v1), acc1);
+        }
         for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
-            // the batch's rows are loaded before the first is added, so one
-            // thread has up to kCombineBatch loads in flight; the adds keep slot order
-            uint4 u[kCombineBatch];
+            // the adds keep slot order
+            uint4 u0[kCombineBatch], u1[kCombineBatch];
 #pragma unroll
             for (int jj = 0; jj < kCombineBatch; ++jj) {
                 const int p = j0 + jj < k ? s_pos[j0 + jj] : -1;
-                u[jj] = p >= 0 ? __ldg(y + (size_t)p * row_vecs + v) : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 *row = y + (size_t)(p >= 0 ? p : 0) * row_vecs;
+                u0[jj] = p >= 0 ? __ldg(row + v0) : make_uint4(0u, 0u, 0u, 0u);
+                u1[jj] = (p >= 0 && has1) ? __ldg(row + v1) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int jj = 0; jj < kCombineBatch; ++jj) {
                 if (j0 + jj >= k || s_pos[j0 + jj] < 0) continue;
-                float f[8];
-                unpack8(u[jj], f);
                 const float w = s_w[j0 + jj];
+                float f[8];
+                unpack8(u0[jj], f);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(w, f[q], acc[q]);
+                for (int q = 0; q < 8; ++q) acc0[q] = __fmaf_rn(w, f[q], acc0[q]);
+                unpack8(u1[jj], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc1[q] = __fmaf_rn(w, f[q], acc1[q]);
             }
         }
         uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        out[(size_t)t * row_vecs + v] = o;
+        o.x = pack_bf16x2(acc0[0], acc0[1]);
+        o.y = pack_bf16x2(acc0[2], acc0[3]);
+        o.z = pack_bf16x2(acc0[4], acc0[5]);
+        o.w = pack_bf16x2(acc0[6], acc0[7]);
+        out[(size_t)t * row_vecs + v0] = o;
+        if (has1) {
+            o.x = pack_bf16x2(acc1[0], acc1[1]);
+            o.y = pack_bf16x2(acc1[2], acc1[3]);
+            o.z = pack_bf16x2(acc1[4], acc1[5]);
+            o.w = pack_bf16x2(acc1[6], acc1[7]);
+            out[(size_t)t * row_vecs + v1] = o;
+        }
     }
 }
 
