@@ -31,7 +31,9 @@ __device__ __forceinline__ uint64_t clip_key(float w, int t) {
 
 // Radix select of the rank-`want` (1-based, descending) key among the keys that
 // `visit` produces.  visit(f) calls f(key) for every key of the segment; it is
-// called once per pass by every thread of the CTA.  The digit holding the
+// called once per pass by every thread of the CTA (whole warps enter f
+// together, the last iteration of a strided loop possibly with fewer lanes).
+// The digit holding the
 // target rank is found by warp 0 with a suffix-sum over the 256 bins.  Once the
 // chosen bin holds a single key, that key is the answer: one more visit picks
 // it up instead of the remaining digit passes (distinct fp32 weights are
@@ -46,13 +48,20 @@ __device__ uint64_t radix_select_desc(Visit visit, uint32_t want, uint32_t *s_hi
         for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0;
         __syncthreads();
         visit([&](uint64_t key) {
-            // warp-aggregated: keys of one expert share their leading digits, so
-            // plain per-key shared atomics would serialise on one bin
+            // keys of one expert share their leading digits: when a whole warp
+            // holds one digit (the common case in the first passes) one lane adds
+            // the warp's count, otherwise each key adds itself (the bins are then
+            // mostly distinct)
             const unsigned active = __activemask();
             const int d = ((key & mask) == prefix) ? (int)((key >> shift) & 255u) : -1;
-            const unsigned peers = __match_any_sync(active, d);
-            if (d >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1)
-                atomicAdd(&s_hist[d], (uint32_t)__popc(peers));
+            const int first = __ffs(active) - 1;
+            const int d0 = __shfl_sync(active, d, first);
+            if (__all_sync(active, d == d0)) {
+                if (d0 >= 0 && (int)(threadIdx.x & 31) == first)
+                    atomicAdd(&s_hist[d0], (uint32_t)__popc(active));
+            } else if (d >= 0) {
+                atomicAdd(&s_hist[d], 1u);
+            }
         });
         __syncthreads();
         if (threadIdx.x < 32) {
