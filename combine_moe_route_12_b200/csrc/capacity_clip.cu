@@ -13,7 +13,7 @@
 //                offsets (prefix sum of their counts); thresholds of the rest
 //   clip_gather  one pass over all assignments: the keys of over-capacity
 //                experts go to their segments (per-CTA ranges reserved with one
-//                atomic per CTA and expert)
+//                atomic per CTA and expert; slots inside a range by shared atomics)
 //   clip_select  one CTA per over-capacity expert: the C-th largest key of its
 //                segment by an MSB-first radix select (up to 8 passes of 8-bit
 //                digits, ending early once one key is left under the prefix)
@@ -173,14 +173,22 @@ __global__ void __launch_bounds__(kGatherThreads) clip_gather_kernel(
         const int e = (ev >= 0 && ev < E && C > 0 && cnt[i] > C) ? ev : -1;
         ex[i] = e;
         slot[i] = -1;
+        // a slot in this CTA's range of expert e (the order inside a segment does
+        // not matter: the select finds a threshold): one reservation when the whole
+        // warp holds one expert, otherwise one shared atomic per key
         const unsigned active = __activemask();
-        const unsigned peers = __match_any_sync(active, e);
-        if (e >= 0) {
-            const int leader = __ffs(peers) - 1;
-            int base = 0;
-            if ((int)(threadIdx.x & 31) == leader) base = atomicAdd(&s_cnt[e], __popc(peers));
-            base = __shfl_sync(peers, base, leader);
-            slot[i] = base + __popc(peers & ((1u << (threadIdx.x & 31)) - 1u));
+        const int lane = threadIdx.x & 31;
+        const int first = __ffs(active) - 1;
+        const int e0 = __shfl_sync(active, e, first);
+        if (__all_sync(active, e == e0)) {
+            if (e0 >= 0) {
+                int base = 0;
+                if (lane == first) base = atomicAdd(&s_cnt[e0], __popc(active));
+                base = __shfl_sync(active, base, first);
+                slot[i] = base + __popc(active & ((1u << lane) - 1u));
+            }
+        } else if (e >= 0) {
+            slot[i] = atomicAdd(&s_cnt[e], 1);
         }
     }
     __syncthreads();
