@@ -14,6 +14,12 @@
  * plus moe_forward_chunked, which runs 1-2 once and pipelines 3-6 over token
  * chunks on two streams (dispatch of chunk c+1 overlaps the FFN of chunk c).
  *
+ * Also: routing variants through moe_config (grouped top-k, a bias that steers
+ * the selection only); moe_shared_expert_ffn, a dense shared expert whose rows
+ * the combine adds; moe_dispatch_layout_noalloc, step 3 with its scratch in a
+ * fixed library array; moe_watchdog_selftest, which makes a bounded wait run
+ * out on purpose; moe_device_status, the device-side error bits.
+ *
  * Sources (restated, not copied):
  *   [AX]  axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
  *         expert_parallel_backend (torch = all_to_all_single over the EP group),
@@ -22,11 +28,12 @@
  *         expert_parallel_size, expert_parallel_token_capacity, and
  *         validate_expert_parallel_topology.
  *   [LL]  LightLLM PR 1687 review page: _select_experts / norm_topk_prob,
- *         the expert prefix-sum ("psum") contiguous layout of the grouped GEMM,
- *         silu_and_mul between the grouped GEMMs, decode reducing expert
- *         outputs straight into a dense output, comm-stream / compute-stream
- *         ownership with record_stream, and dispatch capacity sized from the
- *         padded worst case.
+ *         grouped top-k in experts(), the expert prefix-sum ("psum") contiguous
+ *         layout of the grouped GEMM, silu_and_mul between the grouped GEMMs,
+ *         decode reducing expert outputs straight into a dense output, the
+ *         shared expert overlapped with and added in the combine, comm-stream /
+ *         compute-stream ownership with record_stream, and dispatch capacity
+ *         sized from the padded worst case.
  *
  * Conventions that hold for every call:
  *   - All pointers are DEVICE pointers unless the parameter name ends in
