@@ -288,13 +288,8 @@ cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
         int smem_keys = c.T < kClipMaxSmemKeys ? c.T : kClipMaxSmemKeys;
         if (smem_keys < 1) smem_keys = 1;
         const size_t smem = sizeof(uint64_t) * (size_t)smem_keys;
-        static size_t configured = 48 * 1024;
-        if (smem > configured) {
-            err = cudaFuncSetAttribute(clip_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-            if (err != cudaSuccess) return err;
-            configured = smem;
-        }
+        static SmemOptIn opt_in;
+        if ((err = opt_in.ensure(clip_select_kernel, smem)) != cudaSuccess) return err;
         clip_select_kernel<<<c.E, kClipThreads, smem, s>>>(c.E, c.capacity, smem_keys, (long long)total,
                                                            counts, seg, keys, thr);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;

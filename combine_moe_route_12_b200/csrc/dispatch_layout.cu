@@ -321,13 +321,8 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
             tb, tc, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         const size_t smem = layout_scatter_smem(c, tile_tokens);
-        static size_t configured = 48 * 1024;
-        if (smem > configured) {
-            err = cudaFuncSetAttribute(layout_scatter_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (err != cudaSuccess) return err;
-            configured = smem;
-        }
+        static SmemOptIn opt_in;
+        if ((err = opt_in.ensure(layout_scatter_kernel, smem)) != cudaSuccess) return err;
         layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, s>>>(
             tb, tc, c.k, c.E, c.ep, tile_tokens, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
             expert_offsets, rank_offsets, recv_token, recv_slot, pos, send_splits, status);

@@ -561,13 +561,9 @@ template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx, const CUtensorMap &txs,
                                const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
-    static size_t configured = 0;   // largest dynamic smem this kernel was opened up to
-    if (smem > configured) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_gemm_tcgen05_kernel<MODE>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        configured = smem;
-    }
+    static SmemOptIn opt_in;   // one per kernel instantiation
+    cudaError_t err = opt_in.ensure(ffn_gemm_tcgen05_kernel<MODE>, smem);
+    if (err != cudaSuccess) return err;
     ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
     return cudaGetLastError();
 }

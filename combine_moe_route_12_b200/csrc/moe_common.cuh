@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <mutex>
 
 #include "../../include/moe_b200.h"
 
@@ -33,6 +34,33 @@ inline int64_t layout_max_tiles(int64_t tc) {
     return cap > kLayoutMinTiles ? cap : kLayoutMinTiles;
 }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up after 2 s
+
+// Opens a kernel's dynamic shared memory beyond the default 48 KiB.  The
+// attribute belongs to the current device, so the largest size already set is
+// remembered per device.
+class SmemOptIn {
+  public:
+    template <typename Kernel>
+    cudaError_t ensure(Kernel *kernel, size_t bytes) {
+        if (bytes <= kDefault) return cudaSuccess;
+        int dev = 0;
+        cudaError_t err = cudaGetDevice(&dev);
+        if (err != cudaSuccess) return err;
+        if (dev < 0 || dev >= kDevices)
+            return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        std::lock_guard<std::mutex> lock(m_);
+        if (bytes <= set_[dev]) return cudaSuccess;
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (err == cudaSuccess) set_[dev] = bytes;
+        return err;
+    }
+
+  private:
+    static constexpr size_t kDefault = 48 * 1024;
+    static constexpr int kDevices = 64;
+    std::mutex m_;
+    size_t set_[kDevices] = {};
+};
 
 // ---------------------------------------------------------------- workspace
 // Scratch layout (all offsets 256-byte aligned):
