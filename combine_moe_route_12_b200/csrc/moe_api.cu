@@ -99,12 +99,15 @@ struct Slot {
 struct ForwardLayout {
     size_t counts, kept_counts;
     Slot slot[2];
-    size_t out_reduce, total;
+    size_t out_reduce;
+    // device staging of the host-buffer entry point's activations (host_io only)
+    size_t stage_logits, stage_bias, stage_x, stage_out;
+    size_t total;
     int64_t nmax;
     int tc;
 };
 
-ForwardLayout forward_layout(const moe_config &c) {
+ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
     ForwardLayout F{};
     const ScratchLayout L = scratch_layout(c);
     size_t off = L.total;
@@ -131,6 +134,12 @@ ForwardLayout forward_layout(const moe_config &c) {
         S.ys = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.H) : 0;
     }
     F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
+    if (host_io) {
+        F.stage_logits = take(sizeof(float) * (size_t)c.T * c.E);
+        F.stage_bias = take(sizeof(float) * (size_t)c.E);
+        F.stage_x = take(eb * (size_t)c.T * c.H);
+        F.stage_out = take(eb * (size_t)c.T * c.H);
+    }
     F.total = off;
     return F;
 }
@@ -422,22 +431,24 @@ moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_reduce_finalize");
 }
 
-moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
-                               const void *x, const void *w13, const void *w2,
-                               const void *w13_shared, const void *w2_shared, void *out,
-                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
-                               int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
-                               cudaStream_t s_compute) {
-    moe_status st = moe_config_check(cfg);
-    if (st != MOE_OK) return st;
-    if ((st = check_ws(ws)) != MOE_OK) return st;
-    const moe_config &c = *cfg;
-    if (c.T > 0 && (!logits || !x || !w13 || !w2 || !out || !topk_idx || !topk_w || !keep))
-        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
-    if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
-        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
-    if (c.T == 0) return MOE_OK;
-    const ForwardLayout F = forward_layout(c);
+// Host side of moe_forward_host: pinned activations in, the layer's output out.
+struct HostIO {
+    const float *logits, *bias;
+    const void *x;
+    void *out;
+};
+
+// The two-stream chunked layer.  With io set, logits, bias, x and out are the
+// workspace's staging buffers: the copies in are enqueued first (logits and
+// bias on s_dispatch ahead of routing, each chunk's x on s_compute so that it
+// overlaps routing), and chunk c's output goes back on s_dispatch behind chunk
+// c+1's dispatch, overlapping chunk c+1's FFN.
+static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const float *logits,
+                              const float *bias, const void *x, const void *w13, const void *w2,
+                              const void *w13_shared, const void *w2_shared, void *out,
+                              int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                              int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
+                              cudaStream_t s_compute, const HostIO *io) {
     const ScratchLayout L = scratch_layout(c);
     uint32_t *status = ws_at<uint32_t>(ws, L.status);
     int32_t *counts = ws_at<int32_t>(ws, F.counts);
@@ -445,13 +456,17 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     float *out_reduce = c.reduce_dense ? ws_at<float>(ws, F.out_reduce) : nullptr;
     const int nsm = current_num_sms();
     const int nch = c.n_chunks;
+    const int tc = F.tc;
+    const size_t eb = c.dtype == MOE_F32 ? 4 : 2;
+    const size_t chunk_bytes = eb * (size_t)tc * c.H;
 
     const bool shared = c.shared_I > 0;
     cudaEvent_t *ev = nullptr;
-    cudaError_t err = get_events(3 * nch + 2, &ev);
+    cudaError_t err = get_events(4 * nch + 3, &ev);
     if (err != cudaSuccess) return cuda_fail(err, "event pool");
-    cudaEvent_t ev_start = ev[0], ev_end = ev[1];
-    cudaEvent_t *ev_disp = ev + 2, *ev_done = ev + 2 + nch, *ev_shared = ev + 2 + 2 * nch;
+    cudaEvent_t ev_start = ev[0], ev_end = ev[1], ev_tail = ev[2];
+    cudaEvent_t *ev_disp = ev + 3, *ev_done = ev + 3 + nch, *ev_shared = ev + 3 + 2 * nch;
+    cudaEvent_t *ev_x = ev + 3 + 3 * nch;
 
 #define MOE_TRY(expr, where)                                   \
     do {                                                       \
@@ -462,6 +477,19 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     // the compute stream's earlier work on this workspace precedes the new dispatch
     MOE_TRY(cudaEventRecord(ev_start, s_compute), "record start");
     MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_start, 0), "wait start");
+    if (io) {
+        MOE_TRY(cudaMemcpyAsync((void *)logits, io->logits, sizeof(float) * (size_t)c.T * c.E,
+                                cudaMemcpyHostToDevice, s_dispatch), "copy logits in");
+        if (bias)
+            MOE_TRY(cudaMemcpyAsync((void *)bias, io->bias, sizeof(float) * (size_t)c.E,
+                                    cudaMemcpyHostToDevice, s_dispatch), "copy bias in");
+        for (int ch = 0; ch < nch; ++ch) {
+            MOE_TRY(cudaMemcpyAsync((char *)x + (size_t)ch * chunk_bytes,
+                                    (const char *)io->x + (size_t)ch * chunk_bytes, chunk_bytes,
+                                    cudaMemcpyHostToDevice, s_compute), "copy x in");
+            MOE_TRY(cudaEventRecord(ev_x[ch], s_compute), "record x");
+        }
+    }
     MOE_TRY(launch_route_topk(c, logits, bias, topk_idx, topk_w, counts, status, s_dispatch, nsm),
             "route_topk");
     MOE_TRY(launch_capacity_clip(c, topk_idx, topk_w, counts, keep, kept_counts,
@@ -472,7 +500,14 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
         MOE_TRY(cudaMemsetAsync(out_reduce, 0, sizeof(float) * (size_t)c.T * c.H, s_dispatch),
                 "clear reduce buffer");
 
-    const int tc = F.tc;
+    // chunk ch's output back to the host, on s_dispatch once its combine is done
+    auto copy_out = [&](int ch) -> cudaError_t {
+        cudaError_t e = cudaStreamWaitEvent(s_dispatch, ev_done[ch], 0);
+        if (e != cudaSuccess) return e;
+        return cudaMemcpyAsync((char *)io->out + (size_t)ch * chunk_bytes,
+                               (const char *)out + (size_t)ch * chunk_bytes, chunk_bytes,
+                               cudaMemcpyDeviceToHost, s_dispatch);
+    };
     const int split_stride = c.E + 1 + c.ep * c.ep;
     for (int ch = 0; ch < nch; ++ch) {
         const Slot &S = F.slot[ch & 1];
@@ -490,6 +525,7 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
                                        splits_host ? splits_host + (size_t)ch * split_stride : nullptr,
                                        ws, F.nmax, s_dispatch, nsm),
                 "dispatch_layout");
+        if (io) MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_x[ch], 0), "wait x");
         MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, s_dispatch), "permute");
         MOE_TRY(cudaEventRecord(ev_disp[ch], s_dispatch), "record dispatch");
         void *ys = shared ? ws_at<void>(ws, S.ys) : nullptr;
@@ -502,6 +538,7 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
             MOE_TRY(err, "shared_expert_ffn");
             MOE_TRY(cudaEventRecord(ev_shared[ch], s_dispatch), "record shared");
         }
+        if (io && ch >= 1) MOE_TRY(copy_out(ch - 1), "copy out");
         MOE_TRY(cudaStreamWaitEvent(s_compute, ev_disp[ch], 0), "wait dispatch");
         if (F.nmax > 0) {
             if (c.dtype == MOE_BF16) {
@@ -525,8 +562,62 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     }
     MOE_TRY(cudaEventRecord(ev_end, s_compute), "record end");
     MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_end, 0), "wait end");
+    if (io) {
+        MOE_TRY(copy_out(nch - 1), "copy out");
+        MOE_TRY(cudaEventRecord(ev_tail, s_dispatch), "record tail");
+        MOE_TRY(cudaStreamWaitEvent(s_compute, ev_tail, 0), "wait tail");
+    }
 #undef MOE_TRY
     return MOE_OK;
+}
+
+moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
+                               const void *x, const void *w13, const void *w2,
+                               const void *w13_shared, const void *w2_shared, void *out,
+                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                               int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
+                               cudaStream_t s_compute) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.T > 0 && (!logits || !x || !w13 || !w2 || !out || !topk_idx || !topk_w || !keep))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
+        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
+    if (c.T == 0) return MOE_OK;
+    return forward_run(c, forward_layout(c), logits, bias, x, w13, w2, w13_shared, w2_shared, out,
+                       topk_idx, topk_w, keep, splits_host, ws, s_dispatch, s_compute, nullptr);
+}
+
+size_t moe_forward_host_workspace_bytes(const moe_config *cfg) {
+    if (moe_config_check(cfg) != MOE_OK) return 0;
+    return forward_layout(*cfg, true).total;
+}
+
+moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
+                            const float *bias_host, const void *x_host, const void *w13,
+                            const void *w2, const void *w13_shared, const void *w2_shared,
+                            void *out_host, int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                            int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
+                            cudaStream_t s_compute) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.T > 0 && (!logits_host || !x_host || !w13 || !w2 || !out_host || !topk_idx || !topk_w ||
+                    !keep))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
+        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
+    if (c.T == 0) return MOE_OK;
+    const ForwardLayout F = forward_layout(c, true);
+    const HostIO io{logits_host, bias_host, x_host, out_host};
+    return forward_run(c, F, ws_at<float>(ws, F.stage_logits),
+                       bias_host ? ws_at<float>(ws, F.stage_bias) : nullptr,
+                       ws_at<void>(ws, F.stage_x), w13, w2, w13_shared, w2_shared,
+                       ws_at<void>(ws, F.stage_out), topk_idx, topk_w, keep, splits_host, ws,
+                       s_dispatch, s_compute, &io);
 }
 
 // One thread waits on something that never completes, through the same bounded

@@ -68,6 +68,8 @@ _decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_shared_expert_ffn", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_forward_host_workspace_bytes", ctypes.c_size_t, _CFG)
+_decl("moe_forward_host", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
@@ -136,6 +138,10 @@ def workspace_bytes(cfg: MoEConfig) -> int:
 
 def forward_workspace_bytes(cfg: MoEConfig) -> int:
     return int(_lib.moe_forward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def forward_host_workspace_bytes(cfg: MoEConfig) -> int:
+    return int(_lib.moe_forward_host_workspace_bytes(ctypes.byref(cfg)))
 
 
 def max_recv_rows(cfg: MoEConfig, tok_count: int) -> int:
@@ -220,6 +226,20 @@ def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, ke
                                     _stream(s_dispatch), _stream(s_compute)))
 
 
+def moe_forward_host(cfg, logits_host, bias_host, x_host, w13, w2, out_host, topk_idx, topk_w,
+                     keep, splits_host, ws, s_dispatch=None, s_compute=None, w13_shared=None,
+                     w2_shared=None):
+    """The chunked layer with logits, bias, x and out in (pinned) host memory."""
+    for t in (logits_host, bias_host, x_host, out_host):
+        if t is not None and t.is_cuda:
+            raise ValueError("moe_forward_host takes host tensors for logits, bias, x and out")
+    _check(_lib.moe_forward_host(ctypes.byref(cfg), _ptr(logits_host), _ptr(bias_host),
+                                 _ptr(x_host), _ptr(w13), _ptr(w2), _ptr(w13_shared),
+                                 _ptr(w2_shared), _ptr(out_host), _ptr(topk_idx), _ptr(topk_w),
+                                 _ptr(keep), _ptr(splits_host), _ptr(ws), _stream(s_dispatch),
+                                 _stream(s_compute)))
+
+
 def moe_watchdog_selftest(cfg, which: int, limit_us: int, ws, stream=None):
     """Runs one of the library's bounded waits on something that never completes
     (0: the look-back spin, 1: an mbarrier wait); it sets MOE_DEV_WAIT_TIMEOUT."""
@@ -244,12 +264,16 @@ class MoELayer:
     Allocation goes through torch; the library allocates nothing.
     """
 
-    def __init__(self, cfg: MoEConfig, device="cuda", host_splits: bool = True):
+    def __init__(self, cfg: MoEConfig, device="cuda", host_splits: bool = True,
+                 host_io: bool = False):
         config_check(cfg)
         self.cfg = cfg
         dev = torch.device(device)
         T, k = cfg.T, cfg.k
-        self.ws = alloc_workspace(forward_workspace_bytes(cfg), dev)
+        # host_io: room to stage host activations, for forward_host
+        nbytes = forward_host_workspace_bytes(cfg) if host_io else forward_workspace_bytes(cfg)
+        self.host_io = host_io
+        self.ws = alloc_workspace(nbytes, dev)
         self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
         self.topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
         self.keep = torch.empty(T, k, dtype=torch.uint8, device=dev)
@@ -264,6 +288,18 @@ class MoELayer:
                             self.keep, self.splits_host, self.ws, self.s_dispatch, s_compute,
                             w13_shared, w2_shared)
         return out
+
+    def forward_host(self, logits_host, bias_host, x_host, w13, w2, out_host, s_compute=None,
+                     w13_shared=None, w2_shared=None):
+        """forward() with logits, bias, x and out in pinned host memory; out_host
+        is valid once s_compute (or the dispatch stream) has been synchronised."""
+        if not self.host_io:
+            raise ValueError("MoELayer(host_io=True) is needed for forward_host")
+        s_compute = s_compute or torch.cuda.current_stream()
+        moe_forward_host(self.cfg, logits_host, bias_host, x_host, w13, w2, out_host,
+                         self.topk_idx, self.topk_w, self.keep, self.splits_host, self.ws,
+                         self.s_dispatch, s_compute, w13_shared, w2_shared)
+        return out_host
 
     def splits(self, chunk: int):
         """Host copy of chunk `chunk`'s (expert_offsets, send_splits); valid after a sync."""

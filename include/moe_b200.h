@@ -12,7 +12,8 @@
  *   6. moe_combine             weighted sum of each token's expert rows
  *
  * plus moe_forward_chunked, which runs 1-2 once and pipelines 3-6 over token
- * chunks on two streams (dispatch of chunk c+1 overlaps the FFN of chunk c).
+ * chunks on two streams (dispatch of chunk c+1 overlaps the FFN of chunk c),
+ * and moe_forward_host, the same layer with its activations in host memory.
  *
  * Also: routing variants through moe_config (grouped top-k, a bias that steers
  * the selection only); moe_shared_expert_ffn, a dense shared expert whose rows
@@ -50,7 +51,8 @@
  *   - moe_last_error_detail() describes the last non-OK status of the calling
  *     thread.
  *   - Workspace: a caller-owned device buffer of moe_workspace_bytes(cfg)
- *     bytes (moe_forward_workspace_bytes(cfg) for moe_forward_chunked),
+ *     bytes (moe_forward_workspace_bytes(cfg) for moe_forward_chunked,
+ *     moe_forward_host_workspace_bytes(cfg) for moe_forward_host),
  *     256-byte aligned, zero-filled ONCE before its first use.  A workspace
  *     serves one stream (or one moe_forward_chunked stream pair) at a time.
  */
@@ -342,6 +344,34 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws,
                                cudaStream_t s_dispatch, cudaStream_t s_compute);
+
+/*
+ * moe_forward_chunked with the activations in HOST memory: what a caller whose
+ * tokens arrive from the host calls.  The weights stay device-resident.
+ *   logits_host [T, E] float, bias_host [E] float or NULL, x_host [T, H]
+ *            cfg->dtype: read by host-to-device copies into the workspace.
+ *   out_host [T, H] cfg->dtype: written by device-to-host copies, chunk by
+ *            chunk as each chunk's combine finishes.
+ *   w13, w2, w13_shared, w2_shared, topk_idx, topk_w, keep, splits_host: as
+ *            in moe_forward_chunked (device pointers but for splits_host).
+ *   ws: moe_forward_host_workspace_bytes(cfg) bytes (the forward workspace
+ *            plus staging for logits, bias, x and out).
+ * Ordering: logits and bias are copied on s_dispatch ahead of routing; chunk
+ * c's rows of x on s_compute, overlapping routing; chunk c's output on
+ * s_dispatch behind chunk c+1's dispatch, overlapping chunk c+1's FFN.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for
+ * the copies to be asynchronous; pageable ones work but the copies then block
+ * the host.  The caller must leave the inputs unchanged and must not read
+ * out_host until both streams have passed the call (e.g. synchronise
+ * s_dispatch).  The device result equals moe_forward_chunked's bit for bit.
+ */
+size_t moe_forward_host_workspace_bytes(const moe_config *cfg);
+moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
+                            const float *bias_host, const void *x_host, const void *w13,
+                            const void *w2, const void *w13_shared, const void *w2_shared,
+                            void *out_host, int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                            int32_t *splits_host, void *ws,
+                            cudaStream_t s_dispatch, cudaStream_t s_compute);
 
 /*
  * Watchdog self-test (failure detection; no counterpart on the pages): runs the

@@ -159,6 +159,46 @@ def test_forward_chunked_matches_steps_and_oracle(name):
         np.testing.assert_array_equal(storage_np(out_c), storage_np(out_s))
 
 
+@pytest.mark.parametrize("name", ["bf16_chunked", "tiny_f32", "bf16_decode", "bf16_shared",
+                                  "bf16_grouped_top2_selbias", "f32_shared"])
+def test_forward_host_equals_device_forward(name):
+    """The host-buffer entry point stages the activations in its workspace and
+    copies the output back chunk by chunk; its result is the device forward's,
+    bit for bit, also for two calls enqueued back to back on one workspace."""
+    from combine_moe_route_12_b200 import moe
+    wl = CASES[name]
+    inps = [make_inputs(wl, "cpu", seed=s) for s in (2, 5)]
+    layer = moe.MoELayer(moe.config_from_workload(wl), host_io=True)
+    pin = lambda t: None if t is None else t.pin_memory()
+    dinp = to_device(inps[0])
+    outs = []
+    for inp in inps:
+        out_h = torch.full((wl.T, wl.H), float("nan"), dtype=wl.torch_dtype).pin_memory()
+        layer.forward_host(pin(inp.logits), pin(inp.bias), pin(inp.x), dinp.w13, dinp.w2, out_h,
+                           w13_shared=dinp.w13s, w2_shared=dinp.w2s)
+        outs.append(out_h)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status(layer.ws) == 0
+    for inp, out_h in zip(inps, outs):
+        ref, ref_layer = _forward(wl, to_device(inp), wl.n_chunks)
+        np.testing.assert_array_equal(storage_np(out_h), storage_np(ref))
+    # the saved routing state is the second call's
+    np.testing.assert_array_equal(layer.topk_idx.cpu().numpy(), ref_layer.topk_idx.cpu().numpy())
+    np.testing.assert_array_equal(layer.keep.cpu().numpy(), ref_layer.keep.cpu().numpy())
+
+
+def test_forward_host_rejects_device_activations():
+    from combine_moe_route_12_b200 import moe
+    wl = CASES["bf16_chunked"]
+    dinp = to_device(make_inputs(wl, "cpu", seed=2))
+    layer = moe.MoELayer(moe.config_from_workload(wl), host_io=True)
+    out = torch.empty(wl.T, wl.H, dtype=wl.torch_dtype, device="cuda")
+    with pytest.raises(ValueError):
+        layer.forward_host(dinp.logits, dinp.bias, dinp.x, dinp.w13, dinp.w2, out)
+    with pytest.raises(ValueError):
+        moe.MoELayer(moe.config_from_workload(wl)).forward_host(None, None, None, None, None, None)
+
+
 def test_nonfinite_logit_sets_status_bit():
     from combine_moe_route_12_b200 import moe
     wl = CASES["bf16_ragged_m"]
