@@ -363,7 +363,9 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
  * the copies to be asynchronous; pageable ones work but the copies then block
  * the host.  The caller must leave the inputs unchanged and must not read
  * out_host until both streams have passed the call (e.g. synchronise
- * s_dispatch).  The device result equals moe_forward_chunked's bit for bit.
+ * s_dispatch).  The result equals moe_forward_chunked's bit for bit (with
+ * reduce_dense = 1 up to the order of the fp32 atomic additions, which varies
+ * from run to run in both).
  */
 size_t moe_forward_host_workspace_bytes(const moe_config *cfg);
 moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
