@@ -68,6 +68,16 @@ def lib() -> ctypes.CDLL:
         L.orc_combine_exact.restype = None
         L.orc_bf16_from_double.argtypes = [ctypes.c_double]
         L.orc_bf16_from_double.restype = ctypes.c_uint16
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_ue8m0_scale.argtypes = [ctypes.c_double]
+        L.orc_ue8m0_scale.restype = ctypes.c_uint8
+        L.orc_quantize_rows.argtypes = [ctypes.c_int64, i, i, P, P, P]
+        L.orc_quantize_rows.restype = None
+        L.orc_ffn_row_fp8.argtypes = [i, i, P, ctypes.c_uint8, P, P, P, P, P, P, P, P, P]
+        L.orc_ffn_row_fp8.restype = None
         _lib = L
     return _lib
 
@@ -235,6 +245,65 @@ def combine_exact(y_exact: np.ndarray, pos: np.ndarray, topk_w: np.ndarray, T: i
 
 def bf16_bits_from_double(v: float) -> int:
     return int(lib().orc_bf16_from_double(float(v)))
+
+
+# --------------------------------------------------------------------------- FP8 FFN
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> their values (float64; NaN for the NaN codes)."""
+    c = np.asarray(codes, np.uint8)
+    f = lib().orc_e4m3_decode
+    return np.array([f(int(v)) for v in c.ravel()], np.float64).reshape(c.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """Nearest E4M3 code, ties to even, saturating at +-448."""
+    v = np.asarray(values, np.float64)
+    f = lib().orc_e4m3_encode
+    return np.array([f(float(a)) for a in v.ravel()], np.uint8).reshape(v.shape)
+
+
+def ue8m0_scale(amax: float) -> int:
+    """Biased exponent byte of the smallest 2^e with amax <= 448 * 2^e."""
+    return int(lib().orc_ue8m0_scale(float(amax)))
+
+
+def quantize_rows(a: np.ndarray):
+    """Row-wise FP8 quantisation of a float32 or bf16-bits [rows, cols] array.
+    Returns (codes uint8 [rows, cols], scales uint8 [rows])."""
+    a = np.ascontiguousarray(a)
+    dt = _dtype_code(a)
+    rows, cols = a.shape
+    codes = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros(rows, np.uint8)
+    lib().orc_quantize_rows(rows, cols, dt, _p(a), _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    return e4m3_decode(codes) * np.ldexp(1.0, scales.astype(np.int32) - 127)[:, None]
+
+
+def ffn_row_fp8(x_codes, x_scale, w13_codes, w13_scales, w2_codes, w2_scales):
+    """One expert's FP8 SwiGLU FFN on one row.  Returns
+    (h bf16 bits [I], hq codes [I], h scale byte, y bf16 bits [H], y_exact [H])."""
+    x_codes = np.ascontiguousarray(x_codes, np.uint8)
+    w13_codes = np.ascontiguousarray(w13_codes, np.uint8)
+    w13_scales = np.ascontiguousarray(w13_scales, np.uint8)
+    w2_codes = np.ascontiguousarray(w2_codes, np.uint8)
+    w2_scales = np.ascontiguousarray(w2_scales, np.uint8)
+    H = x_codes.shape[0]
+    I = w13_codes.shape[0] // 2
+    assert w13_codes.shape == (2 * I, H) and w2_codes.shape == (H, I)
+    assert w13_scales.shape == (2 * I,) and w2_scales.shape == (H,)
+    h = np.zeros(I, np.uint16)
+    hq = np.zeros(I, np.uint8)
+    sh = ctypes.c_uint8(0)
+    y = np.zeros(H, np.uint16)
+    ye = np.zeros(H, np.float64)
+    lib().orc_ffn_row_fp8(H, I, _p(x_codes), int(x_scale), _p(w13_codes), _p(w13_scales),
+                          _p(w2_codes), _p(w2_scales), _p(h), _p(hq), ctypes.byref(sh), _p(y), _p(ye))
+    return h, hq, int(sh.value), y, ye
 
 
 # --------------------------------------------------------------------------- whole layer

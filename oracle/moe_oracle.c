@@ -17,7 +17,8 @@
  *      experts, norm_topk_prob renormalisation), the expert prefix-sum
  *      ("psum") contiguous layout for the grouped GEMM, SwiGLU
  *      (silu_and_mul) between the two grouped GEMMs, decode reducing expert
- *      outputs straight into a dense output.
+ *      outputs straight into a dense output, the FP8 grouped GEMM with UE8M0
+ *      (power-of-two) scales and the quantisation of h after silu_and_mul.
  *
  * Readings of points the pages leave open are marked "Reading:".
  *
@@ -440,4 +441,125 @@ void orc_combine_exact(int H, int k, int dtype, int tok_begin, int tok_count,
         for (int c = 0; c < H; ++c) orc_store(out, (size_t)t * H + c, dtype, acc[c]);
     }
     free(acc);
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP8 expert FFN (LightLLM PR 1687: the DeepGEMM FP8 grouped GEMM over the    */
+/* psum layout, UE8M0 quantisation, silu_and_mul followed by quantisation of  */
+/* h before the second grouped GEMM).                                          */
+/*                                                                             */
+/* E4M3 (the variant without infinities): 1 sign bit, 4 exponent bits with     */
+/* bias 7, 3 fraction bits; exponent field 15 with fraction 7 is NaN, so the   */
+/* largest finite magnitude is 1.75 * 2^8 = 448; normals reach down to 2^-6,   */
+/* subnormals are j * 2^-9 for j = 1..7.                                       */
+/* UE8M0: an unsigned 8-bit biased exponent (bias 127) with no mantissa, i.e.  */
+/* a power-of-two scale.                                                       */
+/* Reading: the pages fix power-of-two (UE8M0) scales but not their            */
+/* granularity; here one scale per row: per token for activations, per output  */
+/* channel (weight row) for weights.                                           */
+/* ------------------------------------------------------------------------- */
+double orc_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, f = c & 7;
+    if (e == 15 && f == 7) return NAN;
+    double v = e == 0 ? ldexp((double)f, -9) : ldexp(8.0 + f, e - 10);
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 value, ties to the even fraction; magnitudes beyond 448 give
+ * +-448 ("satfinite"); NaN gives 0x7F. */
+uint8_t orc_e4m3_encode(double v)
+{
+    if (v != v) return 0x7F;
+    uint8_t s = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return s | 0x7E;
+    if (a == 0.0) return s;
+    int ex;
+    frexp(a, &ex);                         /* a in [2^(ex-1), 2^ex) */
+    int e = ex - 1;
+    if (e < -6) e = -6;                    /* the subnormal quantum is 2^-9 */
+    double n = nearbyint(ldexp(a, 3 - e)); /* a in quanta of 2^(e-3), ties to even */
+    double r = ldexp(n, e - 3);            /* <= 448: the largest a below 448 rounds to it */
+    if (r == 0.0) return s;
+    frexp(r, &ex);
+    e = ex - 1;
+    if (e < -6) return s | (uint8_t)ldexp(r, 9);            /* subnormal: j * 2^-9 */
+    int f = (int)ldexp(r, 3 - e) - 8;                        /* r = (8 + f) 2^(e-3) */
+    return s | (uint8_t)((e + 7) << 3) | (uint8_t)f;
+}
+
+/* UE8M0 scale of a row with largest magnitude amax: the smallest power of two
+ * 2^e with amax <= 448 * 2^e, so that every scaled value fits E4M3 and the
+ * largest uses its top binade; e clamped to [-126, 127]; a zero row takes
+ * e = 0.  Returns the biased byte e + 127. */
+uint8_t orc_ue8m0_scale(double amax)
+{
+    if (!(amax > 0.0)) return 127;
+    int e = (int)ceil(log2(amax / 448.0));
+    while (ldexp(448.0, e) < amax) ++e;          /* exact comparisons fix any */
+    while (ldexp(448.0, e - 1) >= amax) --e;     /* rounding of the logarithm */
+    if (e < -126) e = -126;
+    if (e > 127) e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/* Row-wise quantisation: scales[r] = UE8M0 scale of row r, codes[r, c] =
+ * E4M3(in[r, c] / 2^e) (the division by a power of two is exact). */
+void orc_quantize_rows(int64_t rows, int cols, int dtype, const void *in, uint8_t *codes,
+                       uint8_t *scales)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double amax = 0.0;
+        for (int c = 0; c < cols; ++c) {
+            double a = fabs(orc_load(in, (size_t)r * cols + c, dtype));
+            if (a > amax) amax = a;
+        }
+        uint8_t b = orc_ue8m0_scale(amax);
+        scales[r] = b;
+        for (int c = 0; c < cols; ++c)
+            codes[(size_t)r * cols + c] =
+                orc_e4m3_encode(ldexp(orc_load(in, (size_t)r * cols + c, dtype), 127 - (int)b));
+    }
+}
+
+static double orc_dq(uint8_t code, uint8_t scale) { return ldexp(orc_e4m3_decode(code), (int)scale - 127); }
+
+/* One expert's SwiGLU FFN on one receive row in FP8: the steps of
+ * orc_ffn_row on dequantised operands (value = E4M3(code) * 2^(scale - 127)).
+ *   x [H] codes with scale sx; w13 [2I, H] codes with row scales w13_s [2I];
+ *   w2 [H, I] codes with row scales w2_s [H].
+ *   g_i, u_i: dot products in double; h_i = silu(g_i) u_i rounded to bf16
+ *   (h_store, bf16 bits: the CUDA path stores h); h then quantised as one row
+ *   (hq_store [I] codes, *sh_store its scale); y_o = sum_i dq(W2[o,i]) dq(hq_i)
+ *   in double (y_exact, optional) and rounded to bf16 (y_store, optional). */
+void orc_ffn_row_fp8(int H, int I, const uint8_t *x, uint8_t sx, const uint8_t *w13,
+                     const uint8_t *w13_s, const uint8_t *w2, const uint8_t *w2_s,
+                     uint16_t *h_store, uint8_t *hq_store, uint8_t *sh_store, uint16_t *y_store,
+                     double *y_exact)
+{
+    uint16_t *h = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
+    uint8_t *hq = (uint8_t *)malloc((size_t)I);
+    uint8_t sh;
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int c = 0; c < H; ++c) {
+            double xv = orc_dq(x[c], sx);
+            g += orc_dq(w13[(size_t)i * H + c], w13_s[i]) * xv;
+            u += orc_dq(w13[(size_t)(I + i) * H + c], w13_s[I + i]) * xv;
+        }
+        h[i] = orc_bf16_from_double(g / (1.0 + exp(-g)) * u);
+    }
+    orc_quantize_rows(1, I, 1, h, hq, &sh);
+    for (int o = 0; o < H; ++o) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i) acc += orc_dq(w2[(size_t)o * I + i], w2_s[o]) * orc_dq(hq[i], sh);
+        if (y_exact) y_exact[o] = acc;
+        if (y_store) y_store[o] = orc_bf16_from_double(acc);
+    }
+    if (h_store) memcpy(h_store, h, sizeof(uint16_t) * (size_t)I);
+    if (hq_store) memcpy(hq_store, hq, (size_t)I);
+    if (sh_store) *sh_store = sh;
+    free(h);
+    free(hq);
 }
