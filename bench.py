@@ -188,9 +188,10 @@ def kernels_per_step(wl) -> int:
     # route 1; clip 2 (prep, mark) or 4 with a binding capacity (+ gather, select);
     # per chunk: layout 2 (hist, scatter), permute 1, FFN 2 (two GEMM launches),
     # combine or finalize 1
-    # with a shared expert, per chunk 3 more (its offsets and two GEMM launches)
+    # with a shared expert, per chunk 3 more (its offsets and two GEMM launches);
+    # with the FP8 FFN, per chunk 2 more (x's and h's row quantisation)
     clip = 4 if wl.capacity > 0 else 2
-    return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0))
+    return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + (2 if wl.ffn_fp8 else 0))
 
 
 def algorithmic(wl, n_kept_chunks, active_chunks):
@@ -199,18 +200,32 @@ def algorithmic(wl, n_kept_chunks, active_chunks):
     ffn_bytes: per layer pass, the weights of every expert with a row in each
     chunk (each chunk streams them once), the receive rows read by GEMM1, h
     written and read back, and y written (decode form: the dense fp32 buffer
-    read and written once instead)."""
+    read and written once instead).
+
+    FP8 FFN: weights and receive rows are one-byte codes (plus one scale byte
+    per weight row); h is written in bf16, read by its quantisation, whose
+    codes are written and read by GEMM2; the permute stage also quantises x
+    (reads it in bf16, writes its codes) before permuting the codes."""
     b = wl.elem_bytes
     N = sum(n_kept_chunks)
     tok_bytes = wl.T * wl.H * b
-    row_bytes = N * wl.H * b
-    w_bytes = sum(active_chunks) * 3 * wl.H * wl.I * b
-    out_bytes = 2 * wl.T * wl.H * 4 if wl.reduce_dense else row_bytes
+    y_bytes = N * wl.H * b
+    out_bytes = 2 * wl.T * wl.H * 4 if wl.reduce_dense else y_bytes
+    if wl.ffn_fp8:
+        row_bytes = N * wl.H
+        w_bytes = sum(active_chunks) * (3 * wl.H * wl.I + 2 * wl.I + wl.H)
+        permute_bytes = tok_bytes + 2 * wl.T * wl.H + row_bytes
+        h_bytes = N * wl.I * (2 * b + 2)
+    else:
+        row_bytes = y_bytes
+        w_bytes = sum(active_chunks) * 3 * wl.H * wl.I * b
+        permute_bytes = tok_bytes + row_bytes
+        h_bytes = 2 * N * wl.I * b
     return {
-        "permute_bytes": tok_bytes + row_bytes,
-        "combine_bytes": (0 if wl.reduce_dense else row_bytes) + tok_bytes,
+        "permute_bytes": permute_bytes,
+        "combine_bytes": (0 if wl.reduce_dense else y_bytes) + tok_bytes,
         "ffn_flops": 6.0 * wl.H * wl.I * N,
-        "ffn_bytes": w_bytes + row_bytes + 2 * N * wl.I * b + out_bytes,
+        "ffn_bytes": w_bytes + row_bytes + h_bytes + out_bytes,
         "N": N,
     }
 
@@ -237,7 +252,12 @@ class StepBuffers:
         self.rs = torch.empty(n, dtype=torch.int32, device=dev)
         self.pos = torch.empty(tc, k, dtype=torch.int32, device=dev)
         self.spl = torch.empty(ep, ep, dtype=torch.int32, device=dev)
-        self.xr = torch.empty(n, H, dtype=wl.torch_dtype, device=dev)
+        self.xr = torch.empty(n, H, dtype=torch.uint8 if wl.ffn_fp8 else wl.torch_dtype, device=dev)
+        if wl.ffn_fp8:
+            self.xq = torch.empty(T, H, dtype=torch.uint8, device=dev)
+            self.xsc = torch.empty(T, dtype=torch.uint8, device=dev)
+            self.hq = torch.empty(n, I, dtype=torch.uint8, device=dev)
+            self.hsc = torch.empty(n, dtype=torch.uint8, device=dev)
         self.h = torch.empty(n, I, dtype=wl.torch_dtype, device=dev)
         self.y = None if wl.reduce_dense else torch.empty(n, H, dtype=wl.torch_dtype, device=dev)
         self.red = torch.zeros(T, H, dtype=torch.float32, device=dev) if wl.reduce_dense else None
@@ -252,9 +272,11 @@ def n_marks(wl) -> int:
     return 3 + 5 * wl.n_chunks
 
 
-def run_steps(moe, wl, cfg, inp, B, ev=None):
+def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
     """One layer pass through the step ABI on the current stream.  ev: list of
-    n_marks(wl) events recorded between the stages, or None."""
+    n_marks(wl) events recorded between the stages, or None.  fp8: the device
+    (w13 codes, w13 scales, w2 codes, w2 scales) of an FP8 workload; its
+    permute stage quantises the chunk's x rows first."""
     rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
     rec(0)
     moe.moe_route_topk(cfg, inp.logits, inp.bias, B.topk_idx, B.topk_w, B.counts, B.ws)
@@ -269,10 +291,19 @@ def run_steps(moe, wl, cfg, inp, B, ev=None):
         moe.moe_dispatch_layout(cfg, tb, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
                                 B.pos, B.spl, None, B.ws)
         rec(base)
-        moe.moe_permute(cfg, inp.x, B.pos, tb, B.tc, B.xr)
+        if wl.ffn_fp8:
+            moe.moe_quantize_fp8_rows(inp.x[tb:tb + B.tc], B.xq[tb:tb + B.tc], B.xsc[tb:tb + B.tc])
+            moe.moe_permute(cfg, B.xq, B.pos, tb, B.tc, B.xr)
+        else:
+            moe.moe_permute(cfg, inp.x, B.pos, tb, B.tc, B.xr)
         rec(base + 1)
-        moe.moe_grouped_swiglu_ffn(cfg, B.nmax, B.xr, B.eoff, inp.w13, inp.w2, B.h, B.y, B.rt,
-                                   B.rs, B.topk_w, B.red, B.ws)
+        if wl.ffn_fp8:
+            w13q, w13s, w2q, w2s = fp8
+            moe.moe_grouped_swiglu_ffn_fp8(cfg, B.nmax, B.xr, B.xsc, B.eoff, w13q, w13s, w2q, w2s,
+                                           B.h, B.hq, B.hsc, B.y, B.rt, B.rs, B.topk_w, B.red, B.ws)
+        else:
+            moe.moe_grouped_swiglu_ffn(cfg, B.nmax, B.xr, B.eoff, inp.w13, inp.w2, B.h, B.y, B.rt,
+                                       B.rs, B.topk_w, B.red, B.ws)
         rec(base + 2)
         if wl.shared_I > 0:
             moe.moe_shared_expert_ffn(cfg, tb, B.tc, inp.x, inp.w13s, inp.w2s, B.hs, B.ys, B.ws)
@@ -320,7 +351,11 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     keep, _ = oracle.capacity_clip(idx, w, wl.E, wl.capacity)
     tc = wl.T // wl.n_chunks
     lays = [oracle.dispatch_layout(idx, keep, wl.E, wl.ep, c * tc, tc) for c in range(wl.n_chunks)]
-    xrs = [oracle.permute(x_np, lay["recv_token"]) for lay in lays]
+    if wl.ffn_fp8:
+        xq, xs = oracle.quantize_rows(x_np)
+        xrs = [oracle.permute(xq, lay["recv_token"]) for lay in lays]
+    else:
+        xrs = [oracle.permute(x_np, lay["recv_token"]) for lay in lays]
     t_index = time.perf_counter() - t0
     # rows of the sampled tokens (they sit in chunk 0)
     lay = lays[0]
@@ -332,7 +367,10 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     ye = np.zeros((max(N, 1), wl.H), np.float64)
     t1 = time.perf_counter()
     for p, e in rows:
-        _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
+        if wl.ffn_fp8:
+            _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xrs[0][p], xs[lay["recv_token"][p]], *weights[e])
+        else:
+            _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
     sub_pos = lay["pos"][:sample_tokens]
     ys = None
     if shared is not None:
@@ -349,8 +387,18 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     return wl.T / layer_s, t_index + t_ffn, desc
 
 
+def fp8_expert(w13_e, w2_e):
+    """The oracle's codes and row scales of one expert's bf16 weights (host
+    uint16 bits): (w13 codes, w13 scales, w2 codes, w2 scales)."""
+    import oracle
+    a, sa = oracle.quantize_rows(w13_e)
+    b, sb = oracle.quantize_rows(w2_e)
+    return a, sa, b, sb
+
+
 def sample_tokens_for(wl, seconds):
-    row_s = 7.7e-3 * (wl.H * wl.I) / (2048 * 768)      # measured oracle cost of one FFN row
+    # measured oracle cost of one FFN row at H = 2048, I = 768 (bf16 / FP8)
+    row_s = (3.0e-3 if wl.ffn_fp8 else 7.7e-3) * (wl.H * wl.I) / (2048 * 768)
     s = int(seconds / (wl.k * row_s))
     return max(1, min(wl.T // wl.n_chunks, s))
 
@@ -378,7 +426,7 @@ def run_reference(args):
             b = (torch.randn(wl.H, wl.I, generator=g) * std).to(wl.torch_dtype)
             conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
                 else (lambda t: t.numpy().copy())
-            cache[e] = (conv(a), conv(b))
+            cache[e] = fp8_expert(conv(a), conv(b)) if wl.ffn_fp8 else (conv(a), conv(b))
         return cache[e]
 
     conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
@@ -414,7 +462,7 @@ def run_reference(args):
 def workload_config(wl, n, graph=None):
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
             "ep_logical": wl.ep, "capacity": wl.capacity, "dispatch_chunks": wl.n_chunks,
-            "decode_reduce": wl.reduce_dense, "global_batch_tokens": wl.T * n,
+            "decode_reduce": wl.reduce_dense, "ffn_fp8": wl.ffn_fp8, "global_batch_tokens": wl.T * n,
             "parallelism": "replicas" if n > 1 else "single",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
             "timed": ("CPU oracle" if graph is None else
@@ -452,10 +500,18 @@ def run_ours(args):
     layer = moe.MoELayer(cfg, dev, host_splits=False)
     out_fw = torch.empty(wl.T, wl.H, dtype=wl.torch_dtype, device=dev)
     use_graph = not args.no_graph
+    # FP8 FFN: the weights are quantised once, before any timing
+    fp8 = None
+    w13_l, w2_l, w13_sc, w2_sc = inp.w13, inp.w2, None, None
+    if wl.ffn_fp8:
+        w13_l, w13_sc = moe.quantize_fp8(inp.w13)
+        w2_l, w2_sc = moe.quantize_fp8(inp.w2)
+        fp8 = (w13_l, w13_sc, w2_l, w2_sc)
+        torch.cuda.synchronize()
 
     def layer_pass():
-        layer.forward(inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out_fw,
-                      w13_shared=inp.w13s, w2_shared=inp.w2s)
+        layer.forward(inp.logits, inp.bias, inp.x, w13_l, w2_l, out_fw,
+                      w13_shared=inp.w13s, w2_shared=inp.w2s, w13_scale=w13_sc, w2_scale=w2_sc)
 
     for _ in range(max(args.warmup, 1)):
         flush.fill_(1)
@@ -495,7 +551,7 @@ def run_ours(args):
     # with the events (no host launch gaps); eager launches if capture fails
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(n_marks(wl))]
     for _ in range(2):
-        run_steps(moe, wl, cfg, inp, B, None)
+        run_steps(moe, wl, cfg, inp, B, None, fp8)
     torch.cuda.synchronize()
     stage_ms = {s: 0.0 for s in STAGES}
     step_sum = 0.0
@@ -507,7 +563,7 @@ def run_ours(args):
             gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks(wl))]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                run_steps(moe, wl, cfg, inp, B, gev)
+                run_steps(moe, wl, cfg, inp, B, gev, fp8)
             torch.cuda.synchronize()
             g.replay()
             torch.cuda.synchronize()
@@ -521,7 +577,7 @@ def run_ours(args):
         if bd_graph is not None:
             bd_graph.replay()
         else:
-            run_steps(moe, wl, cfg, inp, B, bd_ev)
+            run_steps(moe, wl, cfg, inp, B, bd_ev, fp8)
         torch.cuda.synchronize()
         for s_, v in stage_times(wl, bd_ev).items():
             stage_ms[s_] += v / args.steps
@@ -552,8 +608,9 @@ def run_ours(args):
             flush.fill_(1)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            layer_h.forward_host(h_logits, h_bias, h_x, inp.w13, inp.w2, h_out,
-                                 w13_shared=inp.w13s, w2_shared=inp.w2s)
+            layer_h.forward_host(h_logits, h_bias, h_x, w13_l, w2_l, h_out,
+                                 w13_shared=inp.w13s, w2_shared=inp.w2s, w13_scale=w13_sc,
+                                 w2_scale=w2_sc)
             b.record()
             b.synchronize()
             if i >= args.warmup:
@@ -575,7 +632,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         conv = (lambda t: t.detach().cpu().view(torch.int16).numpy().view(np.uint16).copy()) \
             if wl.dtype == "bf16" else (lambda t: t.detach().cpu().numpy().copy())
-        fetch = lambda e: (conv(inp.w13[e]), conv(inp.w2[e]))
+        fetch = (lambda e: fp8_expert(conv(inp.w13[e]), conv(inp.w2[e]))) if wl.ffn_fp8 else \
+            (lambda e: (conv(inp.w13[e]), conv(inp.w2[e])))
         s_tok = sample_tokens_for(wl, 15.0)
         shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
         v, secs, desc = oracle_sample(wl, inp.logits.cpu().numpy(),
@@ -591,8 +649,12 @@ def run_ours(args):
         dc_s = (stage_ms["permute"] + stage_ms["combine"]) / 1e3
         ffn_tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
         ffn_gbs = alg["ffn_bytes"] / ffn_s / 1e9 if ffn_s > 0 else None
+        # the tensor peak of the FFN's operand type: the measured bf16 figure, times
+        # the nominal dense FP8 / bf16 ratio (4.5 / 2.25) for E4M3 operands
+        t_peak = peaks["bf16_tflops"] * (2.0 if wl.ffn_fp8 else 1.0)
+        t_peak_src = "bf16_tflops (burst) x 2 (nominal e4m3 / bf16)" if wl.ffn_fp8 else "bf16_tflops (burst)"
         # the binding roof: HBM when the pass's flop per byte is below the ridge
-        t_flop = alg["ffn_flops"] / (peaks["bf16_tflops"] * 1e12)
+        t_flop = alg["ffn_flops"] / (t_peak * 1e12)
         t_byte = alg["ffn_bytes"] / (peaks["hbm_gbs"] * 1e9)
         hbm_bound = t_byte > t_flop
         dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
@@ -602,20 +664,22 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 (expert FFN) / bf16" if wl.ffn_fp8 else wl.dtype, "data": "synthetic",
             "config": workload_config(wl, world, use_graph),
-            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass)",
+            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass"
+                                   + (", E4M3 operands, h quantised between them)" if wl.ffn_fp8 else ")"),
                          "bound": "hbm" if hbm_bound else "tensor",
                          "achieved": ffn_gbs if hbm_bound else ffn_tflops,
-                         "peak": peaks["hbm_gbs"] if hbm_bound else peaks["bf16_tflops"],
+                         "peak": peaks["hbm_gbs"] if hbm_bound else t_peak,
                          "unit": "GB/s" if hbm_bound else "TFLOP/s",
-                         "frac": (ffn_gbs / peaks["hbm_gbs"] if hbm_bound else ffn_tflops / peaks["bf16_tflops"])
+                         "frac": (ffn_gbs / peaks["hbm_gbs"] if hbm_bound else ffn_tflops / t_peak)
                          if ffn_s > 0 else None,
                          "traffic": traffic,
-                         "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else "bf16_tflops (burst)"),
+                         "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else t_peak_src),
                          "algorithmic_per_launch": f"{alg['ffn_bytes']:.4g} B and 6*H*I*N = {alg['ffn_flops']:.4g} flop "
                                                    f"over N={alg['N']} kept rows",
-                         "tensor_frac": ffn_tflops / peaks["bf16_tflops"] if ffn_tflops else None,
+                         "tensor_frac": ffn_tflops / t_peak if ffn_tflops else None,
                          "hbm_frac": ffn_gbs / peaks["hbm_gbs"] if ffn_gbs else None},
             "dispatch_combine": {"achieved_gbs": dc_gbs, "peak_gbs": peaks["hbm_gbs"],
                                  "frac": dc_gbs / peaks["hbm_gbs"] if dc_gbs else None,

@@ -52,7 +52,8 @@
 
 namespace moe {
 
-constexpr int kBK = 64;                              // columns of one 128-byte swizzled k-chunk
+constexpr int kBK = 64;                              // bf16 columns of one 128-byte swizzled k-chunk
+constexpr int kBK8 = 128;                            // E4M3 columns of one 128-byte k-chunk
 constexpr int kKS = 2;                               // k-chunks per ring stage (one TMA box each)
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
 constexpr int kTileTok = 256;                        // tokens per tile (MMA N <= 256)
@@ -85,6 +86,12 @@ struct FfnGemmParams {
     const float *topk_w;
     int k;
     uint32_t *status;
+    // FP8 operands: UE8M0 scale bytes of the weight rows (index e *
+    // w_rows_per_expert + row within the expert) and of the token rows
+    // (t_scale[recv_token[p]] when t_scale_by_token, else t_scale[p])
+    const uint8_t *w_scale;
+    const uint8_t *t_scale;
+    int t_scale_by_token;
 };
 
 constexpr int kQueue = 8;                            // slices published ahead of the slowest consumer
@@ -143,6 +150,11 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
 // made the epilogue instruction-bound.  For g -> -inf the quotient is -0.
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
+// A UE8M0 scale byte as a float: 2^(b - 127) (b = 0 gives the subnormal 2^-127).
+__device__ __forceinline__ float ue8m0_value(uint32_t b) {
+    return b == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -163,7 +175,9 @@ struct SliceReader {
     }
 };
 
-template <int MODE>
+// F8: E4M3 operands (tcgen05 kind::f8f6f4, 128 columns per k-chunk) with the
+// row scales applied to the fp32 accumulators in the epilogue; else bf16.
+template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const __grid_constant__ CUtensorMap tmap_xs,
@@ -231,7 +245,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 
     const int total = S->total_slices;
     const uint32_t tmem_base = S->tmem_base;
-    const int num_k = (P.K + kBK * kKS - 1) / (kBK * kKS);   // ring stages per tile
+    constexpr int kChunkCols = F8 ? kBK8 : kBK;             // columns of a 128-byte k-chunk
+    const int num_k = (P.K + kChunkCols * kKS - 1) / (kChunkCols * kKS);   // ring stages per tile
     volatile int *abort_flag = &S->abort_flag;
 
     if (warp == kProdWarp) {
@@ -327,7 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                   decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
                   {
                     const TileInfo ti = tile_info(se, sf, t_blk, P);
-                    const uint32_t idesc = make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
+                    const uint32_t idesc = F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_mma)
+                                              : make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
@@ -340,10 +356,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 #pragma unroll
                         for (int c = 0; c < kKS; ++c) {
 #pragma unroll
-                            for (int kk = 0; kk < kBK / 16; ++kk) {
+                            for (int kk = 0; kk < 4; ++kk) {   // 32-byte k-steps: 16 bf16 or 32 E4M3
                                 const uint64_t wdesc = make_sw128_desc(st + c * kWBytes + kk * 32);
                                 const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * tchunk + kk * 32);
-                                tc_mma_f16_pair(d, wdesc, tdesc, idesc, (kb > 0 || c > 0 || kk > 0) ? 1u : 0u);
+                                const uint32_t accum = (kb > 0 || c > 0 || kk > 0) ? 1u : 0u;
+                                if (F8) tc_mma_f8_pair(d, wdesc, tdesc, idesc, accum);
+                                else tc_mma_f16_pair(d, wdesc, tdesc, idesc, accum);
                             }
                         }
                         tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
@@ -403,6 +421,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
           decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
           {
            const TileInfo ti = tile_info(se, sf, t_blk, P);
+           const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
+           const bool f_ok = f < P.out_cols;
+           // FP8: this lane's weight-row scale, and the token scales of the warp's
+           // 32-token chunks (token half*32 + 64i + lane in chunk i), loaded before
+           // the accumulator wait so that their latency hides behind it
+           float wsc = 1.0f, tsc0 = 1.0f, tsc1 = 1.0f, tsc2 = 1.0f, tsc3 = 1.0f;
+           if (F8) {
+               if (f_ok)
+                   wsc = ue8m0_value(P.w_scale[(size_t)ti.e * P.w_rows_per_expert +
+                                               (kSwiGLU && !is_gate ? P.out_cols : 0) + f]);
+               float t4[4];
+#pragma unroll
+               for (int i = 0; i < 4; ++i) {
+                   const int c = half * 32 + 64 * i + lane;
+                   t4[i] = 1.0f;
+                   if (c < ti.n_valid) {
+                       const int p = ti.p0 + c;
+                       t4[i] = ue8m0_value(P.t_scale[P.t_scale_by_token ? P.recv_token[p] : p]);
+                   }
+               }
+               tsc0 = t4[0]; tsc1 = t4[1]; tsc2 = t4[2]; tsc3 = t4[3];
+           }
            do {   // one pass; `break` leaves it on a failed wait
             bool go;
             if (kSwiGLU) {
@@ -422,21 +462,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 break;
             }
             tc_fence_after();
-            const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
-            const bool f_ok = f < P.out_cols;
             const uint32_t tbase = tmem_base + (uint32_t)(acc * kTileTok) + ((uint32_t)(q * 32) << 16);
 
-            for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64) {
+            int ci = 0;
+            for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64, ++ci) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
                 tc_wait_ld_regs(r);
+                // FP8: the scale of token c0 + lane
+                const float ts_lane = ci == 0 ? tsc0 : ci == 1 ? tsc1 : ci == 2 ? tsc2 : tsc3;
                 if (kSwiGLU) {
                     // exchange: gate warps hand over tokens 16..31, up warps tokens 0..15
                     float *mine = xchg + (xpair * 2 + (is_gate ? 0 : 1)) * 512;
                     float *theirs = xchg + (xpair * 2 + (is_gate ? 1 : 0)) * 512;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]);
+                        mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]) * (F8 ? wsc : 1.0f);
                     named_barrier_sync(1 + xpair, 64);
                     const int cbase = c0 + (is_gate ? 0 : 16);
                     const int nc = min(16, ti.n_valid - cbase);
@@ -450,12 +491,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 #pragma unroll
                     for (int j = 0; j < 16; ++j) other[j] = theirs[j * 32 + lane];
                     named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
+                    float tj[16];                          // FP8: scales of this warp's 16 tokens
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        tj[j] = F8 ? __shfl_sync(0xffffffffu, ts_lane, (is_gate ? 0 : 16) + j) : 1.0f;
                     if (f_ok) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             if (j < nc) {
-                                const float own = __uint_as_float(r[is_gate ? j : 16 + j]);
-                                const float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
+                                const float own = __uint_as_float(r[is_gate ? j : 16 + j]) * (F8 ? wsc : 1.0f);
+                                float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
+                                if (F8) { g *= tj[j]; u *= tj[j]; }
                                 h[(size_t)j * P.out_cols] = __float2bfloat16_rn(silu_f(g) * u);
                             }
                         }
@@ -463,10 +509,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 } else if (MODE == kEpiStore) {
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
                     const int nc = min(32, ti.n_valid - c0);
-                    if (f_ok) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (j < nc) y[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                    for (int j = 0; j < 32; ++j) {
+                        float v = __uint_as_float(r[j]);
+                        if (F8) v *= __shfl_sync(0xffffffffu, ts_lane, j) * wsc;
+                        if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(v);
                     }
                 } else {  // kEpiReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
@@ -476,13 +523,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                         const int p = ti.p0 + c0 + lane;
                         my_t = P.recv_token[p];
                         my_w = P.topk_w[(size_t)my_t * P.k + P.recv_slot[p]];
+                        if (F8) my_w *= ts_lane;
                     }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int t = __shfl_sync(0xffffffffu, my_t, j);
                         const float w = __shfl_sync(0xffffffffu, my_w, j);
                         if (j < nc && f_ok)
-                            atomicAdd(P.out_reduce + (size_t)t * P.out_cols + f, w * __uint_as_float(r[j]));
+                            atomicAdd(P.out_reduce + (size_t)t * P.out_cols + f,
+                                      w * (__uint_as_float(r[j]) * (F8 ? wsc : 1.0f)));
                     }
                 }
             }
@@ -517,39 +566,42 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box 64 cols x box_rows,
-// 128-byte swizzle, zero fill outside the matrix.
-// A bf16 tensor map with 128-byte swizzled boxes whose innermost extent is one
-// 64-column k-chunk; the k-chunk index is the outermost dimension, so one box
-// brings kKS consecutive k-chunks of its rows.
-static bool make_tmap_kchunks(CUtensorMap *m, const void *ptr, int rank, const cuuint64_t *dims,
-                              const cuuint64_t *strides, const cuuint32_t *box) {
+// A tensor map with 128-byte swizzled boxes whose innermost extent is one
+// 128-byte k-chunk (64 bf16 or 128 E4M3 columns); the k-chunk index is the
+// outermost dimension, so one box brings kKS consecutive k-chunks of its rows.
+static bool make_tmap_kchunks(CUtensorMap *m, const void *ptr, bool f8, int rank,
+                              const cuuint64_t *dims, const cuuint64_t *strides,
+                              const cuuint32_t *box) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                     const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-// Rows [rows][K] (row stride K * 2 bytes) as (64, rows, K / 64).
+// Rows [rows][K] (row stride K elements) as (cc, rows, K / cc), cc the columns
+// of a 128-byte k-chunk.
 static bool make_tmap_rows(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t K,
-                           uint32_t box_rows) {
-    const cuuint64_t dims[3] = {(cuuint64_t)kBK, rows, K / kBK};
-    const cuuint64_t strides[2] = {K * 2, (cuuint64_t)kBK * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, (cuuint32_t)kKS};
-    return make_tmap_kchunks(m, ptr, 3, dims, strides, box);
+                           uint32_t box_rows, bool f8 = false) {
+    const uint64_t cc = f8 ? kBK8 : kBK, es = f8 ? 1 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)cc, rows, K / cc};
+    const cuuint64_t strides[2] = {K * es, (cuuint64_t)cc * es};
+    const cuuint32_t box[3] = {(cuuint32_t)cc, box_rows, (cuuint32_t)kKS};
+    return make_tmap_kchunks(m, ptr, f8, 3, dims, strides, box);
 }
 
-// W13 [E][2][I][H] as (64, I, 2E, H / 64): one box holds 64 gate rows of a
+// W13 [E][2][I][H] as (cc, I, 2E, H / cc): one box holds 64 gate rows of a
 // feature block followed by the 64 matching up rows, kKS k-chunks deep.
-static bool make_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I, uint64_t H) {
-    const cuuint64_t dims[4] = {(cuuint64_t)kBK, I, 2 * E, H / kBK};
-    const cuuint64_t strides[3] = {H * 2, I * H * 2, (cuuint64_t)kBK * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)kBK, (cuuint32_t)kRowsPerCta / 2, 2u, (cuuint32_t)kKS};
-    return make_tmap_kchunks(m, ptr, 4, dims, strides, box);
+static bool make_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I, uint64_t H,
+                          bool f8 = false) {
+    const uint64_t cc = f8 ? kBK8 : kBK, es = f8 ? 1 : 2;
+    const cuuint64_t dims[4] = {(cuuint64_t)cc, I, 2 * E, H / cc};
+    const cuuint64_t strides[3] = {H * es, I * H * es, (cuuint64_t)cc * es};
+    const cuuint32_t box[4] = {(cuuint32_t)cc, (cuuint32_t)kRowsPerCta / 2, 2u, (cuuint32_t)kKS};
+    return make_tmap_kchunks(m, ptr, f8, 4, dims, strides, box);
 }
 
 size_t ffn_tcgen05_smem(int E, bool swiglu) {
@@ -557,15 +609,50 @@ size_t ffn_tcgen05_smem(int E, bool swiglu) {
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx, const CUtensorMap &txs,
                                const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static SmemOptIn opt_in;   // one per kernel instantiation
-    cudaError_t err = opt_in.ensure(ffn_gemm_tcgen05_kernel<MODE>, smem);
+    cudaError_t err = opt_in.ensure(ffn_gemm_tcgen05_kernel<MODE, F8>, smem);
     if (err != cudaSuccess) return err;
-    ffn_gemm_tcgen05_kernel<MODE><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
+    ffn_gemm_tcgen05_kernel<MODE, F8><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
     return cudaGetLastError();
+}
+
+// The two launches' parameters (GEMM1 then GEMM2) of one grouped FFN.
+static void ffn_params(const moe_config &c, const int32_t *expert_offsets, void *h, void *y,
+                       const int32_t *recv_token, const int32_t *recv_slot, const float *topk_w,
+                       float *out_reduce, uint32_t *status, FfnGemmParams &P1, FfnGemmParams &P2) {
+    P1 = FfnGemmParams{};
+    P1.expert_offsets = expert_offsets;
+    P1.E = c.E;
+    P1.K = c.H;
+    P1.feat_per_cta = kRowsPerCta / 2;
+    P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
+    P1.w_rows_per_expert = 2 * c.I;
+    P1.out_cols = c.I;
+    P1.out = h;
+    P1.k = c.k;
+    P1.status = status;
+    P1.recv_token = recv_token;
+    P2 = P1;
+    P2.K = c.I;
+    P2.feat_per_cta = kRowsPerCta;
+    P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
+    P2.w_rows_per_expert = c.H;
+    P2.out_cols = c.H;
+    P2.out = y;
+    P2.out_reduce = out_reduce;
+    P2.recv_slot = recv_slot;
+    P2.topk_w = topk_w;
+}
+
+// CTA pairs: an upper bound on the pair tiles is (n_rows / 256 + E) * n_fblocks
+static int ffn_grid(const moe_config &c, int64_t n_rows, const FfnGemmParams &P, int num_sms) {
+    const long long max_pairs = num_sms / 2;
+    const long long g = (n_rows / kTileTok + c.E) * (long long)P.n_fblocks;
+    return 2 * (int)(g < max_pairs ? g : max_pairs);
 }
 
 // Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
@@ -588,39 +675,58 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
         !make_tmap_rows(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTileTok / 2))
         return cudaErrorNotSupported;
 
-    FfnGemmParams P1{};
-    P1.expert_offsets = expert_offsets;
-    P1.E = c.E;
-    P1.K = c.H;
-    P1.feat_per_cta = kRowsPerCta / 2;
-    P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
-    P1.w_rows_per_expert = 2 * c.I;
-    P1.out_cols = c.I;
-    P1.out = h;
-    P1.k = c.k;
-    P1.status = status;
-    // CTA pairs: an upper bound on the pair tiles is (n_rows / 256 + E) * n_fblocks
-    const long long max_pairs = num_sms / 2;
-    long long g1 = (n_rows / kTileTok + c.E) * (long long)P1.n_fblocks;
-    int grid1 = 2 * (int)(g1 < max_pairs ? g1 : max_pairs);
-    cudaError_t err = launch_gemm<kEpiSwiGLU>(tw1, tx1, tx1s, P1, grid1, counters, s);
+    FfnGemmParams P1, P2;
+    ffn_params(c, expert_offsets, h, y, recv_token, recv_slot, topk_w, out_reduce, status, P1, P2);
+    cudaError_t err = launch_gemm<kEpiSwiGLU, false>(tw1, tx1, tx1s, P1, ffn_grid(c, n_rows, P1, num_sms),
+                                                     counters, s);
     if (err != cudaSuccess) return err;
+    const int grid2 = ffn_grid(c, n_rows, P2, num_sms);
+    if (c.reduce_dense) return launch_gemm<kEpiReduce, false>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+    return launch_gemm<kEpiStore, false>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+}
 
-    FfnGemmParams P2 = P1;
-    P2.K = c.I;
-    P2.feat_per_cta = kRowsPerCta;
-    P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
-    P2.w_rows_per_expert = c.H;
-    P2.out_cols = c.H;
-    P2.out = y;
-    P2.out_reduce = out_reduce;
-    P2.recv_token = recv_token;
-    P2.recv_slot = recv_slot;
-    P2.topk_w = topk_w;
-    long long g2 = (n_rows / kTileTok + c.E) * (long long)P2.n_fblocks;
-    int grid2 = 2 * (int)(g2 < max_pairs ? g2 : max_pairs);
-    if (c.reduce_dense) return launch_gemm<kEpiReduce>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
-    return launch_gemm<kEpiStore>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
+                              uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms);
+
+// The FP8 form: GEMM1 on E4M3 codes of xr and W13, h stored in bf16, h
+// quantised by rows (its first expert_offsets[E] rows), GEMM2 on the codes of
+// h and W2.  Returns cudaErrorNotSupported when the tensor-map encoder is
+// unavailable.
+cudaError_t launch_ffn_tcgen05_fp8(const moe_config &c, int64_t n_rows, const uint8_t *xr_q,
+                                   const uint8_t *x_scale, const int32_t *expert_offsets,
+                                   const uint8_t *w13_q, const uint8_t *w13_scale,
+                                   const uint8_t *w2_q, const uint8_t *w2_scale, void *h,
+                                   uint8_t *h_q, uint8_t *h_scale, void *y,
+                                   const int32_t *recv_token, const int32_t *recv_slot,
+                                   const float *topk_w, float *out_reduce, uint32_t *status,
+                                   uint32_t *counters, cudaStream_t s, int num_sms) {
+    if (n_rows <= 0) return cudaSuccess;
+    cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
+    if (cerr != cudaSuccess) return cerr;
+    CUtensorMap tw1, tx1, tw2, tx2, tx1s, tx2s;
+    if (!make_tmap_rows(&tx1s, xr_q, (uint64_t)n_rows, (uint64_t)c.H, kSmallBoxRows, true) ||
+        !make_tmap_rows(&tx2s, h_q, (uint64_t)n_rows, (uint64_t)c.I, kSmallBoxRows, true) ||
+        !make_tmap_w13(&tw1, w13_q, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H, true) ||
+        !make_tmap_rows(&tx1, xr_q, (uint64_t)n_rows, (uint64_t)c.H, kTileTok / 2, true) ||
+        !make_tmap_rows(&tw2, w2_q, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta, true) ||
+        !make_tmap_rows(&tx2, h_q, (uint64_t)n_rows, (uint64_t)c.I, kTileTok / 2, true))
+        return cudaErrorNotSupported;
+    FfnGemmParams P1, P2;
+    ffn_params(c, expert_offsets, h, y, recv_token, recv_slot, topk_w, out_reduce, status, P1, P2);
+    P1.w_scale = w13_scale;
+    P1.t_scale = x_scale;
+    P1.t_scale_by_token = 1;
+    P2.w_scale = w2_scale;
+    P2.t_scale = h_scale;
+    P2.t_scale_by_token = 0;
+    cudaError_t err = launch_gemm<kEpiSwiGLU, true>(tw1, tx1, tx1s, P1, ffn_grid(c, n_rows, P1, num_sms),
+                                                    counters, s);
+    if (err != cudaSuccess) return err;
+    err = launch_quant_rows(n_rows, c.I, true, h, h_q, h_scale, expert_offsets + c.E, s, num_sms);
+    if (err != cudaSuccess) return err;
+    const int grid2 = ffn_grid(c, n_rows, P2, num_sms);
+    if (c.reduce_dense) return launch_gemm<kEpiReduce, true>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+    return launch_gemm<kEpiStore, true>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
 }
 
 }  // namespace moe

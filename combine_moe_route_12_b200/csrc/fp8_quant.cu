@@ -1,0 +1,108 @@
+// FP8 quantisation by rows (LightLLM PR 1687: UE8M0 FP8 quantisation of the
+// dispatch input and of h after silu_and_mul): E4M3 codes and one UE8M0
+// (power-of-two) scale per row.  Used on x per chunk, on h between the two
+// grouped GEMMs, and once on the expert weights.
+//
+// One warp per row, 16-byte loads: a first pass takes the row's largest
+// magnitude, a second (from L1) writes the codes.  HBM-bound: rows * cols *
+// (element + 1) bytes.
+#include <cfloat>
+#include <cuda_fp8.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kQuantWarps = 8;
+
+// The scale exponent: the smallest e with amax <= 448 * 2^e.  With amax =
+// m * 2^x, m in [0.5, 1), and 448 = 0.875 * 2^9, that is e = x - 9 when
+// m <= 0.875 and x - 8 otherwise; clamped to the UE8M0 range used here.
+__device__ __forceinline__ int ue8m0_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    if (amax > FLT_MAX) return 127;
+    int x;
+    const float m = frexpf(amax, &x);
+    const int e = m <= 0.875f ? x - 9 : x - 8;
+    return min(127, max(-126, e));
+}
+
+// 2^-e for e in [-126, 127] (2^-127 is an fp32 subnormal).
+__device__ __forceinline__ float pow2_neg(int e) {
+    return e == 127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - e) << 23);
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    // the first value lands in the low byte (memory order)
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// rows: allocated rows; n_dev (optional): the device-side row count, rows
+// past it are left untouched.
+template <bool BF16>
+__global__ void __launch_bounds__(32 * kQuantWarps) quant_rows_kernel(
+    int64_t rows, int cols, const void *__restrict__ in, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ scales, const int32_t *__restrict__ n_dev) {
+    int64_t n = rows;
+    if (n_dev) n = min(n, (int64_t)max(*n_dev, 0));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kVecElems = BF16 ? 8 : 4;
+    const int nv = cols / kVecElems;
+    for (int64_t r = (int64_t)blockIdx.x * kQuantWarps + warp; r < n;
+         r += (int64_t)gridDim.x * kQuantWarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            static_cast<const char *>(in) + (size_t)r * cols * (BF16 ? 2 : 4));
+        float amax = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            const uint4 q = src[v];
+            if (BF16) {
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(q.x)), fabsf(bf16_hi(q.x))),
+                                         fmaxf(fabsf(bf16_lo(q.y)), fabsf(bf16_hi(q.y)))));
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(q.z)), fabsf(bf16_hi(q.z))),
+                                         fmaxf(fabsf(bf16_lo(q.w)), fabsf(bf16_hi(q.w)))));
+            } else {
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(__uint_as_float(q.x)), fabsf(__uint_as_float(q.y))),
+                                         fmaxf(fabsf(__uint_as_float(q.z)), fabsf(__uint_as_float(q.w)))));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const int e = ue8m0_exponent(amax);
+        const float inv = pow2_neg(e);      // exact: the scaled values are x / 2^e
+        if (lane == 0) scales[r] = (uint8_t)(e + 127);
+        uint8_t *dst = codes + (size_t)r * cols;
+        for (int v = lane; v < nv; v += 32) {
+            const uint4 q = src[v];
+            if (BF16) {
+                uint2 o;
+                o.x = e4m3x2(bf16_lo(q.x) * inv, bf16_hi(q.x) * inv) |
+                      e4m3x2(bf16_lo(q.y) * inv, bf16_hi(q.y) * inv) << 16;
+                o.y = e4m3x2(bf16_lo(q.z) * inv, bf16_hi(q.z) * inv) |
+                      e4m3x2(bf16_lo(q.w) * inv, bf16_hi(q.w) * inv) << 16;
+                reinterpret_cast<uint2 *>(dst)[v] = o;
+            } else {
+                const uint32_t o = e4m3x2(__uint_as_float(q.x) * inv, __uint_as_float(q.y) * inv) |
+                                   e4m3x2(__uint_as_float(q.z) * inv, __uint_as_float(q.w) * inv) << 16;
+                reinterpret_cast<uint32_t *>(dst)[v] = o;
+            }
+        }
+    }
+}
+
+cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
+                              uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms) {
+    if (rows <= 0) return cudaSuccess;
+    long long blocks = (rows + kQuantWarps - 1) / kQuantWarps;
+    const long long cap = (long long)num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    if (bf16)
+        quant_rows_kernel<true><<<(int)blocks, 32 * kQuantWarps, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+    else
+        quant_rows_kernel<false><<<(int)blocks, 32 * kQuantWarps, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

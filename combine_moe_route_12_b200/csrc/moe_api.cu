@@ -34,6 +34,16 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
                                void *h, void *y, const int32_t *recv_token,
                                const int32_t *recv_slot, const float *topk_w, float *out_reduce,
                                uint32_t *status, uint32_t *counters, cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_tcgen05_fp8(const moe_config &c, int64_t n_rows, const uint8_t *xr_q,
+                                   const uint8_t *x_scale, const int32_t *expert_offsets,
+                                   const uint8_t *w13_q, const uint8_t *w13_scale,
+                                   const uint8_t *w2_q, const uint8_t *w2_scale, void *h,
+                                   uint8_t *h_q, uint8_t *h_scale, void *y,
+                                   const int32_t *recv_token, const int32_t *recv_slot,
+                                   const float *topk_w, float *out_reduce, uint32_t *status,
+                                   uint32_t *counters, cudaStream_t s, int num_sms);
+cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
+                              uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -95,9 +105,11 @@ moe_status check_range(const moe_config &c, int32_t tb, int32_t tc, bool need_ep
 struct Slot {
     size_t eoff, roff, recv_token, recv_slot, pos, splits, xr, h, y;
     size_t hs, ys;   // the shared expert's h and y for the chunk's rows (shared_I > 0)
+    size_t hq, hsc;  // ffn_fp8: h's E4M3 codes and row scales
 };
 struct ForwardLayout {
     size_t counts, kept_counts;
+    size_t xq, xsc;  // ffn_fp8: x's E4M3 codes [T, H] and row scales [T]
     Slot slot[2];
     size_t out_reduce;
     // device staging of the host-buffer entry point's activations (host_io only)
@@ -127,12 +139,16 @@ ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
         S.recv_slot = take(sizeof(int32_t) * (size_t)(F.nmax > 0 ? F.nmax : 1));
         S.pos = take(sizeof(int32_t) * (size_t)F.tc * c.k);
         S.splits = take(sizeof(int32_t) * (size_t)c.ep * c.ep);
-        S.xr = take(eb * (size_t)F.nmax * c.H);
+        S.xr = take((c.ffn_fp8 ? 1 : eb) * (size_t)F.nmax * c.H);   // codes when ffn_fp8
         S.h = take(eb * (size_t)F.nmax * c.I);
         S.y = c.reduce_dense ? 0 : take(eb * (size_t)F.nmax * c.H);
         S.hs = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.shared_I) : 0;
         S.ys = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.H) : 0;
+        S.hq = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1) * c.I) : 0;
+        S.hsc = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1)) : 0;
     }
+    F.xq = c.ffn_fp8 ? take((size_t)c.T * c.H) : 0;
+    F.xsc = c.ffn_fp8 ? take((size_t)c.T) : 0;
     F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
     if (host_io) {
         F.stage_logits = take(sizeof(float) * (size_t)c.T * c.E);
@@ -190,6 +206,13 @@ moe_status moe_config_check(const moe_config *cfg) {
     if (c.bias_select_only != 0 && c.bias_select_only != 1)
         return fail(MOE_ERR_INVALID_ARG, "bias_select_only must be 0 or 1");
     if (c.shared_I < 0) return fail(MOE_ERR_INVALID_ARG, "shared_I=%d < 0", c.shared_I);
+    if (c.ffn_fp8 != 0 && c.ffn_fp8 != 1) return fail(MOE_ERR_INVALID_ARG, "ffn_fp8 must be 0 or 1");
+    if (c.ffn_fp8) {
+        if (c.dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 needs dtype MOE_BF16");
+        if (c.H % 128 != 0 || c.I % 128 != 0)
+            return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 needs H and I multiples of 128 (H=%d, I=%d)", c.H, c.I);
+        if (c.shared_I != 0) return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 with a shared expert");
+    }
     if (c.shared_I > 0 && c.dtype == MOE_BF16 && c.shared_I % 64 != 0)
         return fail(MOE_ERR_UNSUPPORTED, "bf16 needs shared_I a multiple of 64 (got %d)", c.shared_I);
     if (c.shared_I > 0 && c.dtype == MOE_F32 && c.shared_I % 4 != 0)
@@ -315,6 +338,7 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
     if ((st = check_ws(ws)) != MOE_OK) return st;
     const moe_config &c = *cfg;
     if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 1: use moe_grouped_swiglu_ffn_fp8");
     if (n_rows == 0) return MOE_OK;
     if (!xr || !expert_offsets || !w13 || !w2 || !h)
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
@@ -346,6 +370,67 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
                               recv_slot, topk_w, out_reduce, stream);
     }
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn");
+}
+
+moe_status moe_quantize_fp8_rows(int64_t rows, int32_t cols, int32_t in_dtype, const void *in,
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t stream) {
+    if (rows < 0 || cols < 1) return fail(MOE_ERR_INVALID_ARG, "rows < 0 or cols < 1");
+    if (in_dtype != MOE_BF16 && in_dtype != MOE_F32)
+        return fail(MOE_ERR_INVALID_ARG, "in_dtype must be MOE_BF16 or MOE_F32");
+    const bool bf16 = in_dtype == MOE_BF16;
+    if (cols % (bf16 ? 8 : 4) != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "cols %% %d != 0 (cols=%d)", bf16 ? 8 : 4, cols);
+    if (rows == 0) return MOE_OK;
+    if (!in || !codes || !scales) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(in, 16) || !aligned(codes, bf16 ? 8 : 4))
+        return fail(MOE_ERR_INVALID_ARG, "in not 16-byte or codes not %d-byte aligned", bf16 ? 8 : 4);
+    cudaError_t err = launch_quant_rows(rows, cols, bf16, in, codes, scales, nullptr, stream,
+                                        current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_fp8_rows");
+}
+
+moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, const uint8_t *xr_q,
+                                      const uint8_t *x_scale, const int32_t *expert_offsets,
+                                      const uint8_t *w13_q, const uint8_t *w13_scale,
+                                      const uint8_t *w2_q, const uint8_t *w2_scale, void *h,
+                                      uint8_t *h_q, uint8_t *h_scale, void *y,
+                                      const int32_t *recv_token, const int32_t *recv_slot,
+                                      const float *topk_w, float *out_reduce, void *ws,
+                                      cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (!c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 0: use moe_grouped_swiglu_ffn");
+    if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (n_rows == 0) return MOE_OK;
+    if (!xr_q || !x_scale || !expert_offsets || !w13_q || !w13_scale || !w2_q || !w2_scale || !h ||
+        !h_q || !h_scale || !recv_token)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.reduce_dense) {
+        if (!recv_slot || !topk_w || !out_reduce)
+            return fail(MOE_ERR_INVALID_ARG, "decode form needs recv_slot, topk_w, out_reduce");
+    } else if (!y) {
+        return fail(MOE_ERR_INVALID_ARG, "y is NULL");
+    }
+    const void *ptrs[6] = {xr_q, w13_q, w2_q, h, h_q, y};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    int dev = 0, major = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10)
+        return fail(MOE_ERR_UNSUPPORTED, "the FP8 FFN uses tcgen05 and needs sm_100 (got major %d)", major);
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_ffn_tcgen05_fp8(c, n_rows, xr_q, x_scale, expert_offsets, w13_q,
+                                             w13_scale, w2_q, w2_scale, h, h_q, h_scale, y,
+                                             recv_token, recv_slot, topk_w, out_reduce,
+                                             ws_at<uint32_t>(ws, L.status),
+                                             ws_at<uint32_t>(ws, L.ffn_ctr), stream,
+                                             current_num_sms());
+    if (err == cudaErrorNotSupported)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn_fp8");
 }
 
 // The shared expert over rows [tb, tb + tc) of x: the step-5 kernel as one
@@ -445,7 +530,8 @@ struct HostIO {
 // c+1's dispatch, overlapping chunk c+1's FFN.
 static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const float *logits,
                               const float *bias, const void *x, const void *w13, const void *w2,
-                              const void *w13_shared, const void *w2_shared, void *out,
+                              const void *w13_shared, const void *w2_shared,
+                              const uint8_t *w13_scale, const uint8_t *w2_scale, void *out,
                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
                               int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
                               cudaStream_t s_compute, const HostIO *io) {
@@ -526,7 +612,16 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
                                        ws, F.nmax, s_dispatch, nsm),
                 "dispatch_layout");
         if (io) MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_x[ch], 0), "wait x");
-        MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, s_dispatch), "permute");
+        if (c.ffn_fp8) {
+            // the chunk's token rows to E4M3 codes, then the codes are permuted
+            uint8_t *xq = ws_at<uint8_t>(ws, F.xq);
+            MOE_TRY(launch_quant_rows(tc, c.H, true, static_cast<const char *>(x) + eb * (size_t)tb * c.H,
+                                      xq + (size_t)tb * c.H, ws_at<uint8_t>(ws, F.xsc) + tb, nullptr,
+                                      s_dispatch, nsm), "quantize x");
+            MOE_TRY(launch_permute(c, xq, pos, tb, tc, xr, s_dispatch), "permute");
+        } else {
+            MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, s_dispatch), "permute");
+        }
         MOE_TRY(cudaEventRecord(ev_disp[ch], s_dispatch), "record dispatch");
         void *ys = shared ? ws_at<void>(ws, S.ys) : nullptr;
         if (shared) {
@@ -541,7 +636,17 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
         if (io && ch >= 1) MOE_TRY(copy_out(ch - 1), "copy out");
         MOE_TRY(cudaStreamWaitEvent(s_compute, ev_disp[ch], 0), "wait dispatch");
         if (F.nmax > 0) {
-            if (c.dtype == MOE_BF16) {
+            if (c.ffn_fp8) {
+                err = launch_ffn_tcgen05_fp8(c, F.nmax, static_cast<const uint8_t *>(xr),
+                                             ws_at<uint8_t>(ws, F.xsc), eoff,
+                                             static_cast<const uint8_t *>(w13), w13_scale,
+                                             static_cast<const uint8_t *>(w2), w2_scale, h,
+                                             ws_at<uint8_t>(ws, S.hq), ws_at<uint8_t>(ws, S.hsc), y,
+                                             recv_token, recv_slot, topk_w, out_reduce, status,
+                                             ws_at<uint32_t>(ws, L.ffn_ctr), s_compute, nsm);
+                if (err == cudaErrorNotSupported)
+                    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+            } else if (c.dtype == MOE_BF16) {
                 err = launch_ffn_tcgen05(c, F.nmax, xr, eoff, w13, w2, h, y, recv_token, recv_slot,
                                          topk_w, out_reduce, status, ws_at<uint32_t>(ws, L.ffn_ctr),
                                          s_compute, nsm);
@@ -573,7 +678,8 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
 
 moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
                                const void *x, const void *w13, const void *w2,
-                               const void *w13_shared, const void *w2_shared, void *out,
+                               const void *w13_shared, const void *w2_shared,
+                               const uint8_t *w13_scale, const uint8_t *w2_scale, void *out,
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
                                cudaStream_t s_compute) {
@@ -585,9 +691,12 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
     if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
         return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
+    if (c.T > 0 && c.ffn_fp8 && (!w13_scale || !w2_scale))
+        return fail(MOE_ERR_INVALID_ARG, "ffn_fp8 needs w13_scale and w2_scale");
     if (c.T == 0) return MOE_OK;
-    return forward_run(c, forward_layout(c), logits, bias, x, w13, w2, w13_shared, w2_shared, out,
-                       topk_idx, topk_w, keep, splits_host, ws, s_dispatch, s_compute, nullptr);
+    return forward_run(c, forward_layout(c), logits, bias, x, w13, w2, w13_shared, w2_shared,
+                       w13_scale, w2_scale, out, topk_idx, topk_w, keep, splits_host, ws,
+                       s_dispatch, s_compute, nullptr);
 }
 
 size_t moe_forward_host_workspace_bytes(const moe_config *cfg) {
@@ -598,6 +707,7 @@ size_t moe_forward_host_workspace_bytes(const moe_config *cfg) {
 moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
                             const float *bias_host, const void *x_host, const void *w13,
                             const void *w2, const void *w13_shared, const void *w2_shared,
+                            const uint8_t *w13_scale, const uint8_t *w2_scale,
                             void *out_host, int32_t *topk_idx, float *topk_w, uint8_t *keep,
                             int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
                             cudaStream_t s_compute) {
@@ -610,13 +720,15 @@ moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
     if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
         return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
+    if (c.T > 0 && c.ffn_fp8 && (!w13_scale || !w2_scale))
+        return fail(MOE_ERR_INVALID_ARG, "ffn_fp8 needs w13_scale and w2_scale");
     if (c.T == 0) return MOE_OK;
     const ForwardLayout F = forward_layout(c, true);
     const HostIO io{logits_host, bias_host, x_host, out_host};
     return forward_run(c, F, ws_at<float>(ws, F.stage_logits),
                        bias_host ? ws_at<float>(ws, F.stage_bias) : nullptr,
-                       ws_at<void>(ws, F.stage_x), w13, w2, w13_shared, w2_shared,
-                       ws_at<void>(ws, F.stage_out), topk_idx, topk_w, keep, splits_host, ws,
+                       ws_at<void>(ws, F.stage_x), w13, w2, w13_shared, w2_shared, w13_scale,
+                       w2_scale, ws_at<void>(ws, F.stage_out), topk_idx, topk_w, keep, splits_host, ws,
                        s_dispatch, s_compute, &io);
 }
 

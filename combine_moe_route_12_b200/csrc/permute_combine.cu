@@ -174,7 +174,8 @@ __global__ void reduce_finalize_kernel(int tb, int tc, int H, int dtype,
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
                            int tc, void *xr, cudaStream_t s) {
     if (tc == 0) return cudaSuccess;
-    const int row_vecs = (int)((size_t)c.H * (c.dtype == MOE_F32 ? 4 : 2) / 16);
+    // row bytes: E4M3 codes when the FFN runs in FP8, else the layer dtype
+    const int row_vecs = (int)((size_t)c.H * (c.ffn_fp8 ? 1 : c.dtype == MOE_F32 ? 4 : 2) / 16);
     permute_rows_kernel<<<tc, kRowThreads, 0, s>>>(tb, c.k, row_vecs,
                                                    static_cast<const uint4 *>(x), pos,
                                                    static_cast<uint4 *>(xr));

@@ -30,7 +30,8 @@ MOE_DEV_BAD_INDEX = 0x4
 class MoEConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "H", "E", "k", "I", "ep", "capacity", "dtype", "n_chunks", "reduce_dense",
-                 "n_group", "topk_group", "group_score", "bias_select_only", "shared_I")]
+                 "n_group", "topk_group", "group_score", "bias_select_only", "shared_I",
+                 "ffn_fp8")]
 
     def __repr__(self):
         return "MoEConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -67,9 +68,11 @@ _decl("moe_grouped_swiglu_ffn", _I32, _CFG, ctypes.c_int64, _P, _P, _P, _P, _P, 
 _decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_shared_expert_ffn", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P)
-_decl("moe_forward_chunked", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_forward_chunked", _I32, _CFG, *([_P] * 17))
 _decl("moe_forward_host_workspace_bytes", ctypes.c_size_t, _CFG)
-_decl("moe_forward_host", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
+_decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
+_decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
 _decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
@@ -112,18 +115,18 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def make_config(T, H, E, k, I, ep, capacity=-1, dtype=MOE_BF16, n_chunks=1,
                 reduce_dense=False, n_group=0, topk_group=0, group_score=0,
-                bias_select_only=False, shared_I=0) -> MoEConfig:
+                bias_select_only=False, shared_I=0, ffn_fp8=False) -> MoEConfig:
     if isinstance(dtype, str):
         dtype = MOE_F32 if dtype == "f32" else MOE_BF16
     return MoEConfig(T, H, E, k, I, ep, -1 if capacity is None else capacity, dtype, n_chunks,
                      int(bool(reduce_dense)), n_group, topk_group, group_score,
-                     int(bool(bias_select_only)), shared_I)
+                     int(bool(bias_select_only)), shared_I, int(bool(ffn_fp8)))
 
 
 def config_from_workload(wl) -> MoEConfig:
     return make_config(wl.T, wl.H, wl.E, wl.k, wl.I, wl.ep, wl.capacity, wl.dtype, wl.n_chunks,
                        wl.reduce_dense, wl.n_group, wl.topk_group, wl.group_score,
-                       wl.bias_select_only, wl.shared_I)
+                       wl.bias_select_only, wl.shared_I, wl.ffn_fp8)
 
 
 # ------------------------------------------------------------------ sizes
@@ -200,6 +203,35 @@ def moe_grouped_swiglu_ffn(cfg, n_rows, xr, expert_offsets, w13, w2, h, y, recv_
                                        _stream(stream)))
 
 
+def moe_quantize_fp8_rows(inp, codes, scales, stream=None):
+    """Row-wise E4M3 codes and UE8M0 scale bytes of a bf16 or fp32 [rows, cols] tensor."""
+    rows, cols = inp.shape
+    in_dtype = MOE_BF16 if inp.dtype == torch.bfloat16 else MOE_F32
+    assert codes.dtype == torch.uint8 and scales.dtype == torch.uint8
+    assert tuple(codes.shape) == (rows, cols) and scales.numel() >= rows
+    _check(_lib.moe_quantize_fp8_rows(rows, cols, in_dtype, _ptr(inp), _ptr(codes), _ptr(scales),
+                                      _stream(stream)))
+
+
+def quantize_fp8(inp, stream=None):
+    """(codes, scales) of moe_quantize_fp8_rows over the last dimension of inp."""
+    flat = inp.reshape(-1, inp.shape[-1])
+    codes = torch.empty(flat.shape, dtype=torch.uint8, device=inp.device)
+    scales = torch.empty(flat.shape[0], dtype=torch.uint8, device=inp.device)
+    moe_quantize_fp8_rows(flat, codes, scales, stream)
+    return codes.view(inp.shape), scales.view(inp.shape[:-1])
+
+
+def moe_grouped_swiglu_ffn_fp8(cfg, n_rows, xr_q, x_scale, expert_offsets, w13_q, w13_scale, w2_q,
+                               w2_scale, h, h_q, h_scale, y, recv_token, recv_slot, topk_w,
+                               out_reduce, ws, stream=None):
+    _check(_lib.moe_grouped_swiglu_ffn_fp8(
+        ctypes.byref(cfg), n_rows, _ptr(xr_q), _ptr(x_scale), _ptr(expert_offsets), _ptr(w13_q),
+        _ptr(w13_scale), _ptr(w2_q), _ptr(w2_scale), _ptr(h), _ptr(h_q), _ptr(h_scale), _ptr(y),
+        _ptr(recv_token), _ptr(recv_slot), _ptr(topk_w), _ptr(out_reduce), _ptr(ws),
+        _stream(stream)))
+
+
 def moe_combine(cfg, y, pos, topk_w, tok_begin, tok_count, out, stream=None, y_shared=None):
     _check(_lib.moe_combine(ctypes.byref(cfg), _ptr(y), _ptr(pos), _ptr(topk_w), tok_begin,
                             tok_count, _ptr(y_shared), _ptr(out), _stream(stream)))
@@ -218,9 +250,11 @@ def moe_shared_expert_ffn(cfg, tok_begin, tok_count, x, w13_shared, w2_shared, h
 
 
 def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, keep, splits_host,
-                        ws, s_dispatch=None, s_compute=None, w13_shared=None, w2_shared=None):
+                        ws, s_dispatch=None, s_compute=None, w13_shared=None, w2_shared=None,
+                        w13_scale=None, w2_scale=None):
     _check(_lib.moe_forward_chunked(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(x),
                                     _ptr(w13), _ptr(w2), _ptr(w13_shared), _ptr(w2_shared),
+                                    _ptr(w13_scale), _ptr(w2_scale),
                                     _ptr(out), _ptr(topk_idx), _ptr(topk_w),
                                     _ptr(keep), _ptr(splits_host), _ptr(ws),
                                     _stream(s_dispatch), _stream(s_compute)))
@@ -228,14 +262,14 @@ def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, ke
 
 def moe_forward_host(cfg, logits_host, bias_host, x_host, w13, w2, out_host, topk_idx, topk_w,
                      keep, splits_host, ws, s_dispatch=None, s_compute=None, w13_shared=None,
-                     w2_shared=None):
+                     w2_shared=None, w13_scale=None, w2_scale=None):
     """The chunked layer with logits, bias, x and out in (pinned) host memory."""
     for t in (logits_host, bias_host, x_host, out_host):
         if t is not None and t.is_cuda:
             raise ValueError("moe_forward_host takes host tensors for logits, bias, x and out")
     _check(_lib.moe_forward_host(ctypes.byref(cfg), _ptr(logits_host), _ptr(bias_host),
                                  _ptr(x_host), _ptr(w13), _ptr(w2), _ptr(w13_shared),
-                                 _ptr(w2_shared), _ptr(out_host), _ptr(topk_idx), _ptr(topk_w),
+                                 _ptr(w2_shared), _ptr(w13_scale), _ptr(w2_scale), _ptr(out_host), _ptr(topk_idx), _ptr(topk_w),
                                  _ptr(keep), _ptr(splits_host), _ptr(ws), _stream(s_dispatch),
                                  _stream(s_compute)))
 
@@ -282,15 +316,17 @@ class MoELayer:
         self.s_dispatch = torch.cuda.Stream(device=dev)
 
     def forward(self, logits, bias, x, w13, w2, out, s_compute=None, w13_shared=None,
-                w2_shared=None):
+                w2_shared=None, w13_scale=None, w2_scale=None):
+        """w13_scale, w2_scale: with cfg.ffn_fp8, w13 and w2 are E4M3 codes and
+        these their UE8M0 row scales (quantize_fp8)."""
         s_compute = s_compute or torch.cuda.current_stream()
         moe_forward_chunked(self.cfg, logits, bias, x, w13, w2, out, self.topk_idx, self.topk_w,
                             self.keep, self.splits_host, self.ws, self.s_dispatch, s_compute,
-                            w13_shared, w2_shared)
+                            w13_shared, w2_shared, w13_scale, w2_scale)
         return out
 
     def forward_host(self, logits_host, bias_host, x_host, w13, w2, out_host, s_compute=None,
-                     w13_shared=None, w2_shared=None):
+                     w13_shared=None, w2_shared=None, w13_scale=None, w2_scale=None):
         """forward() with logits, bias, x and out in pinned host memory; out_host
         is valid once s_compute (or the dispatch stream) has been synchronised."""
         if not self.host_io:
@@ -298,7 +334,7 @@ class MoELayer:
         s_compute = s_compute or torch.cuda.current_stream()
         moe_forward_host(self.cfg, logits_host, bias_host, x_host, w13, w2, out_host,
                          self.topk_idx, self.topk_w, self.keep, self.splits_host, self.ws,
-                         self.s_dispatch, s_compute, w13_shared, w2_shared)
+                         self.s_dispatch, s_compute, w13_shared, w2_shared, w13_scale, w2_scale)
         return out_host
 
     def splits(self, chunk: int):

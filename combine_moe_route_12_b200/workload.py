@@ -41,6 +41,11 @@ Input recipe (the pages fix none of it; every choice is a stated reading):
   top-k with 8 groups of 32 experts and 4 kept per token (group score: the sum
   of a group's two best biased logits), and a load-balancing-like bias
   bias[e] ~ N(0, 0.5^2) (seeded) that steers the selection only.
+* ``qwen3_30b_a3b_fp8`` and ``dsv3_prefill_fp8``: the Qwen3 and DSV3 prefill
+  shapes with the expert FFN in FP8 (LightLLM PR 1687: FP8 grouped GEMM with
+  UE8M0 scales).  Inputs are drawn exactly as for the bf16 workloads; the
+  weights are quantised row by row to E4M3 codes with UE8M0 scales once, before
+  the layer runs, and x per call inside it.
 """
 from __future__ import annotations
 
@@ -72,6 +77,7 @@ class MoEWorkload:
     bias_select_only: bool = False
     balance_bias: bool = False    # a small per-expert bias ~ N(0, 0.5^2), the load-balancing kind
     shared_I: int = 0             # a shared expert of this intermediate size (0: none)
+    ffn_fp8: bool = False         # the expert FFN on E4M3 codes with UE8M0 row scales
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -101,6 +107,11 @@ WORKLOADS = {
     "dsv3_grouped": MoEWorkload("dsv3_grouped", T=8192, H=7168, E=256, k=8, I=2048,
                                 dtype="bf16", ep=8, n_group=8, topk_group=4, group_score=1,
                                 bias_select_only=True, balance_bias=True, shared_I=2048),
+    # the expert FFN in FP8 on the same shapes
+    "qwen3_30b_a3b_fp8": MoEWorkload("qwen3_30b_a3b_fp8", T=4096, H=2048, E=128, k=8, I=768,
+                                     dtype="bf16", ep=2, ffn_fp8=True),
+    "dsv3_prefill_fp8": MoEWorkload("dsv3_prefill_fp8", T=8192, H=7168, E=256, k=8, I=2048,
+                                    dtype="bf16", ep=8, n_chunks=2, ffn_fp8=True),
 }
 
 

@@ -18,8 +18,10 @@
  * Also: routing variants through moe_config (grouped top-k, a bias that steers
  * the selection only); moe_shared_expert_ffn, a dense shared expert whose rows
  * the combine adds; moe_dispatch_layout_noalloc, step 3 with its scratch in a
- * fixed library array; moe_watchdog_selftest, which makes a bounded wait run
- * out on purpose; moe_device_status, the device-side error bits.
+ * fixed library array; moe_quantize_fp8_rows and moe_grouped_swiglu_ffn_fp8,
+ * the expert FFN on E4M3 codes with UE8M0 row scales (cfg->ffn_fp8);
+ * moe_watchdog_selftest, which makes a bounded wait run out on purpose;
+ * moe_device_status, the device-side error bits.
  *
  * Sources (restated, not copied):
  *   [AX]  axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
@@ -102,7 +104,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * bias_select_only in {0, 1}, shared_I >= 0 (a multiple of 64 for MOE_BF16, of
  * 4 for MOE_F32).
  * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30,
- * n_group <= 32;
+ * n_group <= 32; ffn_fp8 = 1 only with MOE_BF16, H % 128 == I % 128 == 0 and
+ * shared_I = 0;
  * MOE_BF16 needs H % 64 == 0 and I % 64 == 0 (tensor-core tiles);
  * MOE_F32 needs H % 4 == 0 and I % 4 == 0.
  */
@@ -136,6 +139,12 @@ typedef struct {
      * w13_shared [2*shared_I, H] and w2_shared [H, shared_I] applied to every
      * token; its output is added into the combine's sum. */
     int32_t shared_I;
+    /* FP8 expert FFN ([LL]: the FP8 grouped GEMM with UE8M0 scales over the
+     * psum layout, silu_and_mul followed by quantisation): 1 runs step 5 on
+     * E4M3 codes with one UE8M0 (power-of-two) scale per row, see
+     * moe_quantize_fp8_rows; the permuted rows are then E4M3 codes.  Needs
+     * dtype MOE_BF16, H and I multiples of 128 and shared_I = 0. */
+    int32_t ffn_fp8;
 } moe_config;
 
 /* Validates cfg (topology and limits).  MOE_OK or the reason it is rejected. */
@@ -146,8 +155,9 @@ moe_status moe_config_check(const moe_config *cfg);
 size_t moe_workspace_bytes(const moe_config *cfg);
 
 /* Bytes moe_forward_chunked needs: the scratch above plus two chunk slots of
- * layout arrays, xr, h and y, and the dense fp32 reduce buffer in decode form.
- * 0 if cfg is invalid. */
+ * layout arrays, xr, h and y, and the dense fp32 reduce buffer in decode form
+ * (with ffn_fp8: also x's codes and scales, h's codes and scales).  0 if cfg
+ * is invalid. */
 size_t moe_forward_workspace_bytes(const moe_config *cfg);
 
 /* Worst-case receive rows of one call over tok_count tokens:
@@ -248,6 +258,7 @@ moe_status moe_dispatch_layout_noalloc(const moe_config *cfg, int32_t tok_begin,
 /*
  * Step 4 - permute: xr[pos[i, j], :] = x[tok_begin + i, :] for every kept
  * (i, j).  x is [T, H]; xr is [N_max, H]; rows >= N are left untouched.
+ * Elements are cfg->dtype, or E4M3 codes (one byte) when cfg->ffn_fp8 = 1.
  */
 moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *pos,
                        int32_t tok_begin, int32_t tok_count, void *xr, cudaStream_t stream);
@@ -276,6 +287,52 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
                                   const int32_t *recv_token, const int32_t *recv_slot,
                                   const float *topk_w, float *out_reduce,
                                   void *ws, cudaStream_t stream);
+
+/*
+ * FP8 quantisation by rows ([LL] UE8M0 FP8 quantisation; the E4M3 format has
+ * 1 sign, 4 exponent bits with bias 7 and 3 fraction bits, no infinities,
+ * largest finite 448).  For each row r of in [rows, cols] (in_dtype MOE_BF16
+ * or MOE_F32):
+ *   e = the smallest integer with max_c |in[r, c]| <= 448 * 2^e, clamped to
+ *       [-126, 127] (0 for a zero row);  scales[r] = e + 127 (UE8M0 byte);
+ *   codes[r, c] = E4M3(in[r, c] / 2^e), round to nearest even, magnitudes
+ *       beyond 448 saturate to 448.
+ * Reading: the pages fix power-of-two scales but not their granularity; one
+ * scale per row is taken (per token for activations, per output channel for
+ * weights).  A value is codes -> E4M3 value times 2^(scales - 127).  Read as
+ * int32, four consecutive scale bytes are the packed form (row 4i in the low
+ * byte).  Use it once on W13 ([E*2I, H] rows) and W2 ([E*H, I] rows) for the
+ * FP8 FFN, and per call on x.  cols % 8 == 0 (bf16) or % 4 == 0 (fp32).
+ * Inputs are expected finite; an infinite row takes e = 127 and saturates.
+ */
+moe_status moe_quantize_fp8_rows(int64_t rows, int32_t cols, int32_t in_dtype, const void *in,
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t stream);
+
+/*
+ * Step 5 in FP8 (cfg->ffn_fp8 = 1): the SwiGLU FFN of moe_grouped_swiglu_ffn
+ * on E4M3 operands with UE8M0 row scales (value = code * 2^(scale - 127)):
+ *   xr_q [n_rows, H]: codes of the receive rows (moe_permute of the codes of
+ *        x); x_scale [T]: the scale bytes of x's token rows, read through
+ *        recv_token[p];
+ *   w13_q [E, 2I, H] with w13_scale [E*2I] (one per weight row), w2_q
+ *        [E, H, I] with w2_scale [E*H];
+ *   g, u = the dequantised dot products (tcgen05 kind::f8f6f4, fp32 in TMEM,
+ *        row and token scales applied to the accumulators);
+ *   h [n_rows, I] bf16 = silu(g) * u;  then h_q [n_rows, I], h_scale [n_rows]
+ *        = moe_quantize_fp8_rows of h's first N rows (N = expert_offsets[E]);
+ *   y [n_rows, H] bf16 = the dequantised W2[e] . h_q[p], or in decode form the
+ *        fp32 reduce into out_reduce as in moe_grouped_swiglu_ffn.
+ * recv_token is always read; recv_slot and topk_w in decode form only.
+ * ws: moe_workspace_bytes(cfg).
+ */
+moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, const uint8_t *xr_q,
+                                      const uint8_t *x_scale, const int32_t *expert_offsets,
+                                      const uint8_t *w13_q, const uint8_t *w13_scale,
+                                      const uint8_t *w2_q, const uint8_t *w2_scale, void *h,
+                                      uint8_t *h_q, uint8_t *h_scale, void *y,
+                                      const int32_t *recv_token, const int32_t *recv_slot,
+                                      const float *topk_w, float *out_reduce, void *ws,
+                                      cudaStream_t stream);
 
 /*
  * Step 6 - combine back to token order ([AX] combine all-to-all then the
@@ -328,6 +385,10 @@ moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32
  *            (else ignored, may be NULL).  Chunk c's shared expert runs on
  *            s_dispatch after its dispatch, beside chunk c's routed FFN on
  *            s_compute, and its rows are added in chunk c's combine.
+ *   w13_scale, w2_scale: with cfg->ffn_fp8 = 1, w13 and w2 are E4M3 codes and
+ *            these their row scales (moe_grouped_swiglu_ffn_fp8); x stays
+ *            bf16 and each chunk's rows are quantised (moe_quantize_fp8_rows)
+ *            before their permutation.  Else ignored, may be NULL.
  *   topk_idx [T,k], topk_w [T,k], keep [T,k]: caller-owned saved state
  *            ([AX] the routing top-k is always saved).
  *   splits_host: pinned host int32 [n_chunks * (E+1 + ep*ep)] or NULL; chunk c
@@ -340,7 +401,8 @@ moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32
  */
 moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const float *bias,
                                const void *x, const void *w13, const void *w2,
-                               const void *w13_shared, const void *w2_shared, void *out,
+                               const void *w13_shared, const void *w2_shared,
+                               const uint8_t *w13_scale, const uint8_t *w2_scale, void *out,
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws,
                                cudaStream_t s_dispatch, cudaStream_t s_compute);
@@ -352,8 +414,9 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
  *            cfg->dtype: read by host-to-device copies into the workspace.
  *   out_host [T, H] cfg->dtype: written by device-to-host copies, chunk by
  *            chunk as each chunk's combine finishes.
- *   w13, w2, w13_shared, w2_shared, topk_idx, topk_w, keep, splits_host: as
- *            in moe_forward_chunked (device pointers but for splits_host).
+ *   w13, w2, w13_shared, w2_shared, w13_scale, w2_scale, topk_idx, topk_w,
+ *            keep, splits_host: as in moe_forward_chunked (device pointers but
+ *            for splits_host).
  *   ws: moe_forward_host_workspace_bytes(cfg) bytes (the forward workspace
  *            plus staging for logits, bias, x and out).
  * Ordering: logits and bias are copied on s_dispatch ahead of routing; chunk
@@ -371,6 +434,7 @@ size_t moe_forward_host_workspace_bytes(const moe_config *cfg);
 moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
                             const float *bias_host, const void *x_host, const void *w13,
                             const void *w2, const void *w13_shared, const void *w2_shared,
+                            const uint8_t *w13_scale, const uint8_t *w2_scale,
                             void *out_host, int32_t *topk_idx, float *topk_w, uint8_t *keep,
                             int32_t *splits_host, void *ws,
                             cudaStream_t s_dispatch, cudaStream_t s_compute);

@@ -538,28 +538,40 @@ void orc_ffn_row_fp8(int H, int I, const uint8_t *x, uint8_t sx, const uint8_t *
                      uint16_t *h_store, uint8_t *hq_store, uint8_t *sh_store, uint16_t *y_store,
                      double *y_exact)
 {
+    /* dequantised value = dec[code] * 2^(scale - 127), both factors exact */
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = orc_e4m3_decode((uint8_t)c);
+    double *xv = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int c = 0; c < H; ++c) xv[c] = orc_dq(x[c], sx);
     uint16_t *h = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
     uint8_t *hq = (uint8_t *)malloc((size_t)I);
+    double *hv = (double *)malloc(sizeof(double) * (size_t)I);
     uint8_t sh;
     for (int i = 0; i < I; ++i) {
+        const double sg = ldexp(1.0, (int)w13_s[i] - 127), su = ldexp(1.0, (int)w13_s[I + i] - 127);
+        const uint8_t *wg = w13 + (size_t)i * H, *wu = w13 + (size_t)(I + i) * H;
         double g = 0.0, u = 0.0;
         for (int c = 0; c < H; ++c) {
-            double xv = orc_dq(x[c], sx);
-            g += orc_dq(w13[(size_t)i * H + c], w13_s[i]) * xv;
-            u += orc_dq(w13[(size_t)(I + i) * H + c], w13_s[I + i]) * xv;
+            g += dec[wg[c]] * sg * xv[c];
+            u += dec[wu[c]] * su * xv[c];
         }
         h[i] = orc_bf16_from_double(g / (1.0 + exp(-g)) * u);
     }
     orc_quantize_rows(1, I, 1, h, hq, &sh);
+    for (int i = 0; i < I; ++i) hv[i] = orc_dq(hq[i], sh);
     for (int o = 0; o < H; ++o) {
+        const double so = ldexp(1.0, (int)w2_s[o] - 127);
+        const uint8_t *wo = w2 + (size_t)o * I;
         double acc = 0.0;
-        for (int i = 0; i < I; ++i) acc += orc_dq(w2[(size_t)o * I + i], w2_s[o]) * orc_dq(hq[i], sh);
+        for (int i = 0; i < I; ++i) acc += dec[wo[i]] * so * hv[i];
         if (y_exact) y_exact[o] = acc;
         if (y_store) y_store[o] = orc_bf16_from_double(acc);
     }
     if (h_store) memcpy(h_store, h, sizeof(uint16_t) * (size_t)I);
     if (hq_store) memcpy(hq_store, hq, (size_t)I);
     if (sh_store) *sh_store = sh;
+    free(xv);
     free(h);
     free(hq);
+    free(hv);
 }

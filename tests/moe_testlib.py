@@ -56,8 +56,12 @@ def to_device(inp: MoEInputs, device="cuda") -> MoEInputs:
                      w2=mv(inp.w2), w13s=mv(inp.w13s), w2s=mv(inp.w2s))
 
 
-def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> dict:
-    """Runs the six ABI steps chunk by chunk on the current CUDA stream."""
+def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=None) -> dict:
+    """Runs the six ABI steps chunk by chunk on the current CUDA stream.
+
+    fp8: for a workload with ffn_fp8, the device (w13 codes, w13 scales, w2
+    codes, w2 scales); x is then quantised once, its codes are permuted and
+    step 5 is moe_grouped_swiglu_ffn_fp8."""
     cfg = moe.config_from_workload(wl)
     dev = inp.logits.device
     T, E, k, H, I, ep = wl.T, wl.E, wl.k, wl.H, wl.I, wl.ep
@@ -74,6 +78,9 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
     tc = T // wl.n_chunks
     nmax = moe.max_recv_rows(cfg, tc)
     chunks = []
+    xq = xs = None
+    if wl.ffn_fp8:
+        xq, xs = moe.quantize_fp8(inp.x)
     for c in range(wl.n_chunks):
         tb = c * tc
         eoff = torch.full((E + 1,), -7, dtype=torch.int32, device=dev)
@@ -84,11 +91,21 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
         spl = torch.full((ep, ep), -7, dtype=torch.int32, device=dev)
         host = torch.full((E + 1 + ep * ep,), -7, dtype=torch.int32).pin_memory()
         moe.moe_dispatch_layout(cfg, tb, tc, topk_idx, keep, eoff, roff, rt, rs, pos, spl, host, ws)
-        xr = torch.empty((max(nmax, 1), H), dtype=wl.torch_dtype, device=dev)
-        moe.moe_permute(cfg, inp.x, pos, tb, tc, xr)
+        xr = torch.empty((max(nmax, 1), H), dtype=torch.uint8 if wl.ffn_fp8 else wl.torch_dtype,
+                         device=dev)
+        moe.moe_permute(cfg, xq if wl.ffn_fp8 else inp.x, pos, tb, tc, xr)
         h = torch.empty((max(nmax, 1), I), dtype=wl.torch_dtype, device=dev)
         y = None if wl.reduce_dense else torch.empty((max(nmax, 1), H), dtype=wl.torch_dtype, device=dev)
-        moe.moe_grouped_swiglu_ffn(cfg, nmax, xr, eoff, inp.w13, inp.w2, h, y, rt, rs, topk_w, red, ws)
+        hq = hs = None
+        if wl.ffn_fp8:
+            hq = torch.empty((max(nmax, 1), I), dtype=torch.uint8, device=dev)
+            hs = torch.empty((max(nmax, 1),), dtype=torch.uint8, device=dev)
+            w13q, w13s, w2q, w2s = fp8
+            moe.moe_grouped_swiglu_ffn_fp8(cfg, nmax, xr, xs, eoff, w13q, w13s, w2q, w2s, h, hq, hs,
+                                           y, rt, rs, topk_w, red, ws)
+        else:
+            moe.moe_grouped_swiglu_ffn(cfg, nmax, xr, eoff, inp.w13, inp.w2, h, y, rt, rs, topk_w,
+                                       red, ws)
         ys = None
         if wl.shared_I > 0:
             hs = torch.empty((tc, wl.shared_I), dtype=wl.torch_dtype, device=dev)
@@ -106,15 +123,18 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True) -> di
         if keep_rows:
             ch.update(xr=storage_np(xr[:n]), h=storage_np(h[:n]),
                       y=None if y is None else storage_np(y[:n]),
-                      ys=None if ys is None else storage_np(ys))
+                      ys=None if ys is None else storage_np(ys),
+                      hq=None if hq is None else hq[:n].cpu().numpy(),
+                      hs=None if hs is None else hs[:n].cpu().numpy())
         else:
-            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys)
+            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys, hq_dev=hq, hs_dev=hs)
         chunks.append(ch)
     status = moe.moe_device_status(ws)
     torch.cuda.synchronize()
     return dict(topk_idx=topk_idx.cpu().numpy(), topk_w=topk_w.cpu().numpy(),
                 counts=counts.cpu().numpy(), keep=keep.cpu().numpy(), kept_counts=kept.cpu().numpy(),
-                chunks=chunks, out=out, status=status)
+                chunks=chunks, out=out, status=status,
+                xq=None if xq is None else xq.cpu().numpy(), xs=None if xs is None else xs.cpu().numpy())
 
 
 def oracle_routing(wl: MoEWorkload, inp: MoEInputs) -> dict:
@@ -141,3 +161,70 @@ def assert_routing_equal(g: dict, o: dict, wl: MoEWorkload) -> None:
             np.testing.assert_array_equal(gc[key], oc[key], err_msg=key)
         np.testing.assert_array_equal(gc["host"][:wl.E + 1], oc["expert_offsets"])
         np.testing.assert_array_equal(gc["host"][wl.E + 1:].reshape(wl.ep, wl.ep), oc["send_splits"])
+
+
+def oracle_fp8_weights(inp: MoEInputs, experts=None) -> dict:
+    """The oracle's E4M3 codes and UE8M0 row scales of the expert weights (all
+    experts, or a dict for the listed ones): w13q [E, 2I, H], w13s [E, 2I],
+    w2q [E, H, I], w2s [E, H]."""
+    def q(w):
+        a = storage_np(w)
+        c, s = oracle.quantize_rows(a.reshape(-1, a.shape[-1]))
+        return c.reshape(a.shape), s.reshape(a.shape[:-1])
+    if experts is None:
+        w13q, w13s = q(inp.w13)
+        w2q, w2s = q(inp.w2)
+        return dict(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s)
+    out = {}
+    for e in experts:
+        w13q, w13s = q(inp.w13[e])
+        w2q, w2s = q(inp.w2[e])
+        out[e] = dict(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s)
+    return out
+
+
+def fp8_weights_to_device(wq: dict, device="cuda"):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    return t(wq["w13q"]), t(wq["w13s"]), t(wq["w2q"]), t(wq["w2s"])
+
+
+def oracle_fp8_ffn_and_out(wl: MoEWorkload, inp: MoEInputs, orc: dict, wq: dict):
+    """The oracle's FP8 layer after routing: x quantised by rows, its codes
+    permuted, the FP8 SwiGLU row by row, then the combine (decode form: over
+    the unrounded y)."""
+    x = storage_np(inp.x)
+    xq, xs = oracle.quantize_rows(x)
+    tc = wl.T // wl.n_chunks
+    out = np.zeros((wl.T, wl.H), np.uint16)
+    res = []
+    for c, lay in enumerate(orc["layouts"]):
+        n = lay["N"]
+        xrq = oracle.permute(xq, lay["recv_token"])
+        h = np.zeros((n, wl.I), np.uint16)
+        hq = np.zeros((n, wl.I), np.uint8)
+        hs = np.zeros(n, np.uint8)
+        y = np.zeros((n, wl.H), np.uint16)
+        ye = np.zeros((n, wl.H), np.float64)
+        eoff = lay["expert_offsets"]
+        for e in range(wl.E):
+            for p in range(int(eoff[e]), int(eoff[e + 1])):
+                h[p], hq[p], hs[p], y[p], ye[p] = oracle.ffn_row_fp8(
+                    xrq[p], xs[lay["recv_token"][p]], wq["w13q"][e], wq["w13s"][e],
+                    wq["w2q"][e], wq["w2s"][e])
+        if wl.reduce_dense:
+            oracle.combine_exact(ye, lay["pos"], orc["topk_w"], wl.T, np.uint16, c * tc, out)
+        else:
+            oracle.combine(y, lay["pos"], orc["topk_w"], wl.T, c * tc, out)
+        res.append(dict(xrq=xrq, h=h, hq=hq, hs=hs, y=y))
+    return dict(xq=xq, xs=xs, chunks=res, out=out)
+
+
+def assert_codes_close(got_codes, got_scales, ref_codes, ref_scales, what, min_equal=0.99):
+    """Quantised rows whose inputs differ by float rounding: almost every code
+    and scale equal, and the dequantised values within the bf16 tolerance."""
+    if ref_codes.size == 0:
+        return
+    assert (got_codes == ref_codes).mean() >= min_equal, f"{what}: codes differ too often"
+    assert (got_scales == ref_scales).mean() >= min_equal, f"{what}: scales differ too often"
+    assert_float_close(oracle.dequantize_rows(got_codes, got_scales),
+                       oracle.dequantize_rows(ref_codes, ref_scales), "bf16", what)
