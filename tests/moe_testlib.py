@@ -96,12 +96,12 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
         moe.moe_permute(cfg, xq if wl.ffn_fp8 else inp.x, pos, tb, tc, xr)
         h = torch.empty((max(nmax, 1), I), dtype=wl.torch_dtype, device=dev)
         y = None if wl.reduce_dense else torch.empty((max(nmax, 1), H), dtype=wl.torch_dtype, device=dev)
-        hq = hs = None
+        hq = hsc = None
         if wl.ffn_fp8:
             hq = torch.empty((max(nmax, 1), I), dtype=torch.uint8, device=dev)
-            hs = torch.empty((max(nmax, 1),), dtype=torch.uint8, device=dev)
+            hsc = torch.empty((max(nmax, 1),), dtype=torch.uint8, device=dev)
             w13q, w13s, w2q, w2s = fp8
-            moe.moe_grouped_swiglu_ffn_fp8(cfg, nmax, xr, xs, eoff, w13q, w13s, w2q, w2s, h, hq, hs,
+            moe.moe_grouped_swiglu_ffn_fp8(cfg, nmax, xr, xs, eoff, w13q, w13s, w2q, w2s, h, hq, hsc,
                                            y, rt, rs, topk_w, red, ws)
         else:
             moe.moe_grouped_swiglu_ffn(cfg, nmax, xr, eoff, inp.w13, inp.w2, h, y, rt, rs, topk_w,
@@ -125,9 +125,9 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
                       y=None if y is None else storage_np(y[:n]),
                       ys=None if ys is None else storage_np(ys),
                       hq=None if hq is None else hq[:n].cpu().numpy(),
-                      hs=None if hs is None else hs[:n].cpu().numpy())
+                      hs=None if hsc is None else hsc[:n].cpu().numpy())
         else:
-            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys, hq_dev=hq, hs_dev=hs)
+            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys, hq_dev=hq, hs_dev=hsc)
         chunks.append(ch)
     status = moe.moe_device_status(ws)
     torch.cuda.synchronize()
