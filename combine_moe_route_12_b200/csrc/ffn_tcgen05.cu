@@ -155,6 +155,43 @@ __device__ __forceinline__ float ue8m0_value(uint32_t b) {
     return b == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);   // lo in the low half
+    return *reinterpret_cast<const uint32_t *>(&p);
+}
+
+// The epilogue holds one feature per lane and T tokens per lane; global rows
+// want tokens.  Three butterfly rounds (lane bit 0, 1, 2) swap halves so that,
+// for each group g of 8 tokens, lane L ends up with token 8g + (L & 7) and the
+// 8 consecutive features 8 (L >> 3) .. +7, rounded to bf16 and packed: one
+// 16-byte store per lane and group instead of one 2-byte store per token.
+template <int T>
+__device__ __forceinline__ void warp_tokens_to_rows(const float (&v)[T], uint4 (&out)[T / 8], int lane) {
+    const bool b0 = lane & 1, b1 = (lane >> 1) & 1, b2 = (lane >> 2) & 1;
+    uint32_t p1[T / 2];     // features {L & ~1, L | 1} of token a + (L & 1)
+#pragma unroll
+    for (int a = 0; a < T; a += 2) {
+        const float recv = __shfl_xor_sync(0xffffffffu, b0 ? v[a] : v[a + 1], 1);
+        p1[a / 2] = b0 ? pack_bf16x2(recv, v[a + 1]) : pack_bf16x2(v[a], recv);
+    }
+    uint32_t q[T / 4][2];   // features 4 (L >> 2) .. +3 of token 4k + (L & 3)
+#pragma unroll
+    for (int k = 0; k < T / 4; ++k) {
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, b1 ? p1[2 * k] : p1[2 * k + 1], 2);
+        q[k][0] = b1 ? recv : p1[2 * k];
+        q[k][1] = b1 ? p1[2 * k + 1] : recv;
+    }
+#pragma unroll
+    for (int g = 0; g < T / 8; ++g) {
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, b2 ? q[2 * g][0] : q[2 * g + 1][0], 4);
+        const uint32_t r1 = __shfl_xor_sync(0xffffffffu, b2 ? q[2 * g][1] : q[2 * g + 1][1], 4);
+        out[g].x = b2 ? r0 : q[2 * g][0];
+        out[g].y = b2 ? r1 : q[2 * g][1];
+        out[g].z = b2 ? q[2 * g + 1][0] : r0;
+        out[g].w = b2 ? q[2 * g + 1][1] : r1;
+    }
+}
+
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -481,8 +518,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     named_barrier_sync(1 + xpair, 64);
                     const int cbase = c0 + (is_gate ? 0 : 16);
                     const int nc = min(16, ti.n_valid - cbase);
-                    __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) +
-                                       (size_t)(ti.p0 + cbase) * P.out_cols + f;
                     // all 16 partner values into registers before the first store:
                     // h and the exchange buffer are both generic pointers, so a load
                     // after a store could not be moved ahead of it and every token
@@ -491,22 +526,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 #pragma unroll
                     for (int j = 0; j < 16; ++j) other[j] = theirs[j * 32 + lane];
                     named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
-                    float tj[16];                          // FP8: scales of this warp's 16 tokens
+                    // h of this warp's 16 tokens (every lane, for the shuffles; tokens
+                    // past nc are never stored)
+                    float hv[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        tj[j] = F8 ? __shfl_sync(0xffffffffu, ts_lane, (is_gate ? 0 : 16) + j) : 1.0f;
-                    if (f_ok) {
+                    for (int j = 0; j < 16; ++j) {
+                        const float own = __uint_as_float(r[is_gate ? j : 16 + j]) * (F8 ? wsc : 1.0f);
+                        float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
+                        if (F8) {
+                            const float tj = __shfl_sync(0xffffffffu, ts_lane, (is_gate ? 0 : 16) + j);
+                            g *= tj;
+                            u *= tj;
+                        }
+                        hv[j] = silu_f(g) * u;
+                    }
+                    uint4 o[2];
+                    warp_tokens_to_rows<16>(hv, o, lane);
+                    const int col = f - feat_lane + (q & 1) * 32 + 8 * (lane >> 3);   // this lane's 8 features
+                    if (col + 8 <= P.out_cols) {
+                        __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(P.out) + (size_t)(ti.p0 + cbase) * P.out_cols + col;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (j < nc) {
-                                const float own = __uint_as_float(r[is_gate ? j : 16 + j]) * (F8 ? wsc : 1.0f);
-                                float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
-                                if (F8) { g *= tj[j]; u *= tj[j]; }
-                                h[(size_t)j * P.out_cols] = __float2bfloat16_rn(silu_f(g) * u);
-                            }
+                        for (int g8 = 0; g8 < 2; ++g8) {
+                            const int tok = 8 * g8 + (lane & 7);
+                            if (tok < nc) *reinterpret_cast<uint4 *>(h + (size_t)tok * P.out_cols) = o[g8];
                         }
                     }
                 } else if (MODE == kEpiStore) {
+                    // one 64-byte warp store per token row (the shuffle rearrangement
+                    // of the SwiGLU epilogue measured slower here)
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
                     const int nc = min(32, ti.n_valid - c0);
 #pragma unroll

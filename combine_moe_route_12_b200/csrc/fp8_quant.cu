@@ -3,9 +3,10 @@
 // (power-of-two) scale per row.  Used on x per chunk, on h between the two
 // grouped GEMMs, and once on the expert weights.
 //
-// One warp per row, 16-byte loads: a first pass takes the row's largest
-// magnitude, a second (from L1) writes the codes.  HBM-bound: rows * cols *
-// (element + 1) bytes.
+// One warp per row, 16-byte loads.  Rows of up to 256 vectors (2048 bf16 or
+// 1024 fp32 values) stay in registers between the maximum and the codes;
+// longer rows take a second pass over the row (from L1).  HBM-bound: rows *
+// cols * (element + 1) bytes.
 #include <cfloat>
 #include <cuda_fp8.h>
 
@@ -40,9 +41,38 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// rows: allocated rows; n_dev (optional): the device-side row count, rows
-// past it are left untouched.
 template <bool BF16>
+__device__ __forceinline__ float vec_amax(const uint4 &q) {
+    if (BF16)
+        return fmaxf(fmaxf(fmaxf(fabsf(bf16_lo(q.x)), fabsf(bf16_hi(q.x))),
+                           fmaxf(fabsf(bf16_lo(q.y)), fabsf(bf16_hi(q.y)))),
+                     fmaxf(fmaxf(fabsf(bf16_lo(q.z)), fabsf(bf16_hi(q.z))),
+                           fmaxf(fabsf(bf16_lo(q.w)), fabsf(bf16_hi(q.w)))));
+    return fmaxf(fmaxf(fabsf(__uint_as_float(q.x)), fabsf(__uint_as_float(q.y))),
+                 fmaxf(fabsf(__uint_as_float(q.z)), fabsf(__uint_as_float(q.w))));
+}
+
+// The codes of one 16-byte vector (8 bf16 or 4 fp32 values) at vector v of dst.
+template <bool BF16>
+__device__ __forceinline__ void vec_store_codes(uint8_t *dst, int v, const uint4 &q, float inv) {
+    if (BF16) {
+        uint2 o;
+        o.x = e4m3x2(bf16_lo(q.x) * inv, bf16_hi(q.x) * inv) |
+              e4m3x2(bf16_lo(q.y) * inv, bf16_hi(q.y) * inv) << 16;
+        o.y = e4m3x2(bf16_lo(q.z) * inv, bf16_hi(q.z) * inv) |
+              e4m3x2(bf16_lo(q.w) * inv, bf16_hi(q.w) * inv) << 16;
+        reinterpret_cast<uint2 *>(dst)[v] = o;
+    } else {
+        reinterpret_cast<uint32_t *>(dst)[v] =
+            e4m3x2(__uint_as_float(q.x) * inv, __uint_as_float(q.y) * inv) |
+            e4m3x2(__uint_as_float(q.z) * inv, __uint_as_float(q.w) * inv) << 16;
+    }
+}
+
+// rows: allocated rows; n_dev (optional): the device-side row count, rows
+// past it are left untouched.  kRegVecs > 0: every lane holds its (at most
+// kRegVecs) vectors of the row in registers; 0: two passes over the row.
+template <bool BF16, int kRegVecs>
 __global__ void __launch_bounds__(32 * kQuantWarps) quant_rows_kernel(
     int64_t rows, int cols, const void *__restrict__ in, uint8_t *__restrict__ codes,
     uint8_t *__restrict__ scales, const int32_t *__restrict__ n_dev) {
@@ -55,39 +85,33 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_rows_kernel(
          r += (int64_t)gridDim.x * kQuantWarps) {
         const uint4 *src = reinterpret_cast<const uint4 *>(
             static_cast<const char *>(in) + (size_t)r * cols * (BF16 ? 2 : 4));
+        uint8_t *dst = codes + (size_t)r * cols;
         float amax = 0.0f;
-        for (int v = lane; v < nv; v += 32) {
-            const uint4 q = src[v];
-            if (BF16) {
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(q.x)), fabsf(bf16_hi(q.x))),
-                                         fmaxf(fabsf(bf16_lo(q.y)), fabsf(bf16_hi(q.y)))));
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(q.z)), fabsf(bf16_hi(q.z))),
-                                         fmaxf(fabsf(bf16_lo(q.w)), fabsf(bf16_hi(q.w)))));
-            } else {
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(__uint_as_float(q.x)), fabsf(__uint_as_float(q.y))),
-                                         fmaxf(fabsf(__uint_as_float(q.z)), fabsf(__uint_as_float(q.w)))));
+        uint4 q[kRegVecs > 0 ? kRegVecs : 1];
+        if (kRegVecs > 0) {
+#pragma unroll
+            for (int i = 0; i < kRegVecs; ++i) {
+                const int v = lane + 32 * i;
+                q[i] = v < nv ? src[v] : make_uint4(0u, 0u, 0u, 0u);
             }
+#pragma unroll
+            for (int i = 0; i < kRegVecs; ++i) amax = fmaxf(amax, vec_amax<BF16>(q[i]));
+        } else {
+            for (int v = lane; v < nv; v += 32) amax = fmaxf(amax, vec_amax<BF16>(src[v]));
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
         const int e = ue8m0_exponent(amax);
         const float inv = pow2_neg(e);      // exact: the scaled values are x / 2^e
         if (lane == 0) scales[r] = (uint8_t)(e + 127);
-        uint8_t *dst = codes + (size_t)r * cols;
-        for (int v = lane; v < nv; v += 32) {
-            const uint4 q = src[v];
-            if (BF16) {
-                uint2 o;
-                o.x = e4m3x2(bf16_lo(q.x) * inv, bf16_hi(q.x) * inv) |
-                      e4m3x2(bf16_lo(q.y) * inv, bf16_hi(q.y) * inv) << 16;
-                o.y = e4m3x2(bf16_lo(q.z) * inv, bf16_hi(q.z) * inv) |
-                      e4m3x2(bf16_lo(q.w) * inv, bf16_hi(q.w) * inv) << 16;
-                reinterpret_cast<uint2 *>(dst)[v] = o;
-            } else {
-                const uint32_t o = e4m3x2(__uint_as_float(q.x) * inv, __uint_as_float(q.y) * inv) |
-                                   e4m3x2(__uint_as_float(q.z) * inv, __uint_as_float(q.w) * inv) << 16;
-                reinterpret_cast<uint32_t *>(dst)[v] = o;
+        if (kRegVecs > 0) {
+#pragma unroll
+            for (int i = 0; i < kRegVecs; ++i) {
+                const int v = lane + 32 * i;
+                if (v < nv) vec_store_codes<BF16>(dst, v, q[i], inv);
             }
+        } else {
+            for (int v = lane; v < nv; v += 32) vec_store_codes<BF16>(dst, v, src[v], inv);
         }
     }
 }
@@ -98,10 +122,15 @@ cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in,
     long long blocks = (rows + kQuantWarps - 1) / kQuantWarps;
     const long long cap = (long long)num_sms * 16;
     if (blocks > cap) blocks = cap;
-    if (bf16)
-        quant_rows_kernel<true><<<(int)blocks, 32 * kQuantWarps, 0, s>>>(rows, cols, in, codes, scales, n_dev);
-    else
-        quant_rows_kernel<false><<<(int)blocks, 32 * kQuantWarps, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+    const int nv = cols / (bf16 ? 8 : 4);
+    const dim3 g((unsigned)blocks), b(32 * kQuantWarps);
+    if (bf16) {
+        if (nv <= 32 * 8) quant_rows_kernel<true, 8><<<g, b, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+        else quant_rows_kernel<true, 0><<<g, b, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+    } else {
+        if (nv <= 32 * 8) quant_rows_kernel<false, 8><<<g, b, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+        else quant_rows_kernel<false, 0><<<g, b, 0, s>>>(rows, cols, in, codes, scales, n_dev);
+    }
     return cudaGetLastError();
 }
 
