@@ -49,7 +49,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": 1558.534912e6, "src": "81a9932ff07c390d"},
+    "qwen3_30b_a3b": {"bytes": 1558.986496e6, "src": "1ef986a2c4ae5f1d"},
+    # both GEMM launches and the quantisation of h between them
+    "qwen3_30b_a3b_fp8": {"bytes": 894.446848e6, "src": "1ef986a2c4ae5f1d"},
 }
 
 
@@ -106,9 +108,13 @@ def load_peaks():
 
 
 def kernel_src_hash():
-    p = os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", "ffn_tcgen05.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the FFN's sources (the grouped GEMM kernel and the row quantisation
+    between its launches): recorded traffic holds only for these bytes."""
+    h = hashlib.sha256()
+    for name in ("ffn_tcgen05.cu", "fp8_quant.cu"):
+        with open(os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # --------------------------------------------------------------------------- clocks
