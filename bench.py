@@ -200,8 +200,10 @@ def kernels_per_step(wl) -> int:
     return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + (2 if wl.ffn_fp8 else 0))
 
 
-def algorithmic(wl, n_kept_chunks, active_chunks):
-    """Bytes / flops the method must move or compute (nothing for dropped rows).
+def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
+    """Bytes / flops the method must move or compute (nothing for dropped rows;
+    the permute reads the x rows of the tokens_read tokens that keep at least one
+    slot, all T when not given).
 
     ffn_bytes: per layer pass, the weights of every expert with a row in each
     chunk (each chunk streams them once), the receive rows read by GEMM1, h
@@ -215,17 +217,18 @@ def algorithmic(wl, n_kept_chunks, active_chunks):
     b = wl.elem_bytes
     N = sum(n_kept_chunks)
     tok_bytes = wl.T * wl.H * b
+    read_bytes = (wl.T if tokens_read is None else tokens_read) * wl.H
     y_bytes = N * wl.H * b
     out_bytes = 2 * wl.T * wl.H * 4 if wl.reduce_dense else y_bytes
     if wl.ffn_fp8:
         row_bytes = N * wl.H
         w_bytes = sum(active_chunks) * (3 * wl.H * wl.I + 2 * wl.I + wl.H)
-        permute_bytes = tok_bytes + 2 * wl.T * wl.H + row_bytes
+        permute_bytes = tok_bytes + wl.T * wl.H + read_bytes + row_bytes
         h_bytes = N * wl.I * (2 * b + 2)
     else:
         row_bytes = y_bytes
         w_bytes = sum(active_chunks) * 3 * wl.H * wl.I * b
-        permute_bytes = tok_bytes + row_bytes
+        permute_bytes = read_bytes * b + row_bytes
         h_bytes = 2 * N * wl.I * b
     return {
         "permute_bytes": permute_bytes,
@@ -598,7 +601,8 @@ def run_ours(args):
                                 B.pos, B.spl, None, B.ws)
         n_kept.append(int(B.eoff[wl.E].item()))
         n_active.append(int(((B.eoff[1:] - B.eoff[:-1]) > 0).sum().item()))
-    alg = algorithmic(wl, n_kept, n_active)
+    tokens_read = int((B.keep.view(wl.T, wl.k) != 0).any(dim=1).sum().item())
+    alg = algorithmic(wl, n_kept, n_active, tokens_read)
 
     # ---------------- end to end through the public API with host buffers
     e2e = None

@@ -1,10 +1,14 @@
 // Steps 4 and 6: the row permutation into the receive layout and the weighted
 // combine back to token order (axolotl ExpertParallelArgs: dispatch / combine
 // all_to_all_single outputs; LightLLM PR 1687: decode reduce into a dense
-// output).  Both are HBM-bound row copies: one CTA per token, 16-byte vector
-// loads and stores, each source row read once.
+// output).  Both are HBM-bound row copies with 16-byte vector loads and stores,
+// each source row read once.  A CTA takes kTokPerCta consecutive tokens: their
+// pos (and weights) arrive with one load round and one barrier, and the CTAs
+// are few enough that a token with one kept row or none is not dominated by
+// the CTA's start-up.
 //
-//   permute:  x[t] is read once and written to each of its kept receive rows.
+//   permute:  x[t] is read once and written to each of its kept receive rows;
+//             a token with no kept row is not read at all.
 //   combine:  out[t] = sum_j w[t, j] * y[pos[t, j]] in fp32, slot order,
 //             rounded once to the storage type.
 #include "moe_common.cuh"
@@ -12,20 +16,39 @@
 namespace moe {
 
 constexpr int kRowThreads = 128;
+constexpr int kTokPerCta = 4;                 // kTokPerCta * kMaxTopK <= kRowThreads
+static_assert(kTokPerCta * kMaxTopK <= kRowThreads, "one pos per thread");
+
+// pos (and topk_w) of the CTA's tokens [i0, i0 + n) into shared memory.
+__device__ __forceinline__ void load_slots(int tb, int i0, int n, int k, const int32_t *pos,
+                                           const float *topk_w, int32_t (*s_pos)[kMaxTopK],
+                                           float (*s_w)[kMaxTopK]) {
+    const int a = threadIdx.x / k, j = threadIdx.x - a * k;
+    if (a < n) {
+        s_pos[a][j] = pos[(size_t)(i0 + a) * k + j];
+        if (s_w) s_w[a][j] = topk_w[(size_t)(tb + i0 + a) * k + j];
+    }
+}
 
 __global__ void __launch_bounds__(kRowThreads) permute_rows_kernel(
-    int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
+    int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint4 *__restrict__ xr) {
-    __shared__ int32_t s_pos[kMaxTopK];
-    const int i = blockIdx.x;
-    if (threadIdx.x < k) s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
+    __shared__ int32_t s_pos[kTokPerCta][kMaxTopK];
+    const int i0 = blockIdx.x * kTokPerCta;
+    const int n = min(kTokPerCta, tc - i0);
+    load_slots(tb, i0, n, k, pos, nullptr, s_pos, nullptr);
     __syncthreads();
-    const uint4 *src = x + (size_t)(tb + i) * row_vecs;
-    for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
-        const uint4 d = __ldg(src + v);
-        for (int j = 0; j < k; ++j) {
-            const int p = s_pos[j];
-            if (p >= 0) xr[(size_t)p * row_vecs + v] = d;
+    for (int a = 0; a < n; ++a) {
+        bool any = false;
+        for (int j = 0; j < k; ++j) any |= s_pos[a][j] >= 0;
+        if (!any) continue;                   // every slot dropped: x[t] is not needed
+        const uint4 *src = x + (size_t)(tb + i0 + a) * row_vecs;
+        for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
+            const uint4 d = __ldg(src + v);
+            for (int j = 0; j < k; ++j) {
+                const int p = s_pos[a][j];
+                if (p >= 0) xr[(size_t)p * row_vecs + v] = d;
+            }
         }
     }
 }
@@ -48,17 +71,19 @@ constexpr int kCombineBatch = 4;   // expert rows of a token loaded together
 
 // bf16 storage: one uint4 = 8 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
-    int tb, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
+    int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const uint4 *__restrict__ y_shared, uint4 *__restrict__ out) {
-    __shared__ int32_t s_pos[kMaxTopK];
-    __shared__ float s_w[kMaxTopK];
-    const int i = blockIdx.x;
-    const int t = tb + i;
-    if (threadIdx.x < k) {
-        s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
-        s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
-    }
+    __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
+    __shared__ float s_w_all[kTokPerCta][kMaxTopK];
+    const int i0 = blockIdx.x * kTokPerCta;
+    const int n = min(kTokPerCta, tc - i0);
+    load_slots(tb, i0, n, k, pos, topk_w, s_pos_all, s_w_all);
     __syncthreads();
+    for (int a = 0; a < n; ++a) {
+    const int i = i0 + a;
+    const int t = tb + i;
+    const int32_t *s_pos = s_pos_all[a];
+    const float *s_w = s_w_all[a];
     // two 16-byte columns per pass, all their row loads issued before any add or
     // store: a token with one or two kept rows still has several loads in flight
     for (int v0 = threadIdx.x; v0 < row_vecs; v0 += 2 * kRowThreads) {
@@ -107,21 +132,24 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
             out[(size_t)t * row_vecs + v1] = o;
         }
     }
+    }
 }
 
 // fp32 storage: one float4 = 4 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
-    int tb, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
+    int tb, int tc, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const float4 *__restrict__ y_shared, float4 *__restrict__ out) {
-    __shared__ int32_t s_pos[kMaxTopK];
-    __shared__ float s_w[kMaxTopK];
-    const int i = blockIdx.x;
-    const int t = tb + i;
-    if (threadIdx.x < k) {
-        s_pos[threadIdx.x] = pos[(size_t)i * k + threadIdx.x];
-        s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
-    }
+    __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
+    __shared__ float s_w_all[kTokPerCta][kMaxTopK];
+    const int i0 = blockIdx.x * kTokPerCta;
+    const int n = min(kTokPerCta, tc - i0);
+    load_slots(tb, i0, n, k, pos, topk_w, s_pos_all, s_w_all);
     __syncthreads();
+    for (int a = 0; a < n; ++a) {
+    const int i = i0 + a;
+    const int t = tb + i;
+    const int32_t *s_pos = s_pos_all[a];
+    const float *s_w = s_w_all[a];
     for (int v = threadIdx.x; v < row_vecs; v += kRowThreads) {
         float4 acc = y_shared ? __ldg(y_shared + (size_t)i * row_vecs + v) : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
@@ -135,6 +163,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
             acc.w = __fmaf_rn(w, f.w, acc.w);
         }
         out[(size_t)t * row_vecs + v] = acc;
+    }
     }
 }
 
@@ -176,9 +205,8 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *po
     if (tc == 0) return cudaSuccess;
     // row bytes: E4M3 codes when the FFN runs in FP8, else the layer dtype
     const int row_vecs = (int)((size_t)c.H * (c.ffn_fp8 ? 1 : c.dtype == MOE_F32 ? 4 : 2) / 16);
-    permute_rows_kernel<<<tc, kRowThreads, 0, s>>>(tb, c.k, row_vecs,
-                                                   static_cast<const uint4 *>(x), pos,
-                                                   static_cast<uint4 *>(xr));
+    permute_rows_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
+        tb, tc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
     return cudaGetLastError();
 }
 
@@ -188,13 +216,13 @@ cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *po
     if (tc == 0) return cudaSuccess;
     if (c.dtype == MOE_F32) {
         const int row_vecs = c.H / 4;
-        combine_rows_f32_kernel<<<tc, kRowThreads, 0, s>>>(
-            tb, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
+        combine_rows_f32_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
+            tb, tc, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
             static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
     } else {
         const int row_vecs = c.H / 8;
-        combine_rows_bf16_kernel<<<tc, kRowThreads, 0, s>>>(
-            tb, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
+        combine_rows_bf16_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
+            tb, tc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
             static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
     }
     return cudaGetLastError();
