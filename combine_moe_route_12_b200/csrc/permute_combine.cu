@@ -2,10 +2,11 @@
 // combine back to token order (axolotl ExpertParallelArgs: dispatch / combine
 // all_to_all_single outputs; LightLLM PR 1687: decode reduce into a dense
 // output).  Both are HBM-bound row copies with 16-byte vector loads and stores,
-// each source row read once.  A CTA takes kTokPerCta consecutive tokens: their
-// pos (and weights) arrive with one load round and one barrier, and the CTAs
-// are few enough that a token with one kept row or none is not dominated by
-// the CTA's start-up.
+// each source row read once.  A CTA takes tpc <= kTokPerCta consecutive
+// tokens: their pos (and weights) arrive with one load round and one barrier.
+// Large chunks take several tokens per CTA, so that a token with one kept row
+// or none is not dominated by the CTA's start-up; chunks that would then leave
+// SMs idle take one (tok_per_cta).
 //
 //   permute:  x[t] is read once and written to each of its kept receive rows;
 //             a token with no kept row is not read at all.
@@ -19,6 +20,17 @@ constexpr int kRowThreads = 128;
 constexpr int kTokPerCta = 4;                 // kTokPerCta * kMaxTopK <= kRowThreads
 static_assert(kTokPerCta * kMaxTopK <= kRowThreads, "one pos per thread");
 
+// Tokens per CTA: as many (up to kTokPerCta) as still leave about 27 CTAs per
+// SM (1.7 waves of 16 resident): 16384 tokens take 4 per CTA on 148 SMs, 4096
+// take 1 (measured: 4 per CTA there left SMs idle and slowed the permute).
+static int tok_per_cta(int tc) {
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int t = tc / (nsm * 27);
+    return t < 1 ? 1 : (t > kTokPerCta ? kTokPerCta : t);
+}
+
 // pos (and topk_w) of the CTA's tokens [i0, i0 + n) into shared memory.
 __device__ __forceinline__ void load_slots(int tb, int i0, int n, int k, const int32_t *pos,
                                            const float *topk_w, int32_t (*s_pos)[kMaxTopK],
@@ -31,11 +43,11 @@ __device__ __forceinline__ void load_slots(int tb, int i0, int n, int k, const i
 }
 
 __global__ void __launch_bounds__(kRowThreads) permute_rows_kernel(
-    int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
+    int tb, int tc, int tpc, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint4 *__restrict__ xr) {
     __shared__ int32_t s_pos[kTokPerCta][kMaxTopK];
-    const int i0 = blockIdx.x * kTokPerCta;
-    const int n = min(kTokPerCta, tc - i0);
+    const int i0 = blockIdx.x * tpc;
+    const int n = min(tpc, tc - i0);
     load_slots(tb, i0, n, k, pos, nullptr, s_pos, nullptr);
     __syncthreads();
     for (int a = 0; a < n; ++a) {
@@ -71,12 +83,12 @@ constexpr int kCombineBatch = 4;   // expert rows of a token loaded together
 
 // bf16 storage: one uint4 = 8 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
-    int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
+    int tb, int tc, int tpc, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const uint4 *__restrict__ y_shared, uint4 *__restrict__ out) {
     __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
     __shared__ float s_w_all[kTokPerCta][kMaxTopK];
-    const int i0 = blockIdx.x * kTokPerCta;
-    const int n = min(kTokPerCta, tc - i0);
+    const int i0 = blockIdx.x * tpc;
+    const int n = min(tpc, tc - i0);
     load_slots(tb, i0, n, k, pos, topk_w, s_pos_all, s_w_all);
     __syncthreads();
     for (int a = 0; a < n; ++a) {
@@ -137,12 +149,12 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
 
 // fp32 storage: one float4 = 4 elements.
 __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
-    int tb, int tc, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
+    int tb, int tc, int tpc, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const float4 *__restrict__ y_shared, float4 *__restrict__ out) {
     __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
     __shared__ float s_w_all[kTokPerCta][kMaxTopK];
-    const int i0 = blockIdx.x * kTokPerCta;
-    const int n = min(kTokPerCta, tc - i0);
+    const int i0 = blockIdx.x * tpc;
+    const int n = min(tpc, tc - i0);
     load_slots(tb, i0, n, k, pos, topk_w, s_pos_all, s_w_all);
     __syncthreads();
     for (int a = 0; a < n; ++a) {
@@ -205,8 +217,9 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *po
     if (tc == 0) return cudaSuccess;
     // row bytes: E4M3 codes when the FFN runs in FP8, else the layer dtype
     const int row_vecs = (int)((size_t)c.H * (c.ffn_fp8 ? 1 : c.dtype == MOE_F32 ? 4 : 2) / 16);
-    permute_rows_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
-        tb, tc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
+    const int tpc = tok_per_cta(tc);
+    permute_rows_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
+        tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
     return cudaGetLastError();
 }
 
@@ -214,15 +227,16 @@ cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *po
                            const float *topk_w, int tb, int tc, const void *y_shared, void *out,
                            cudaStream_t s) {
     if (tc == 0) return cudaSuccess;
+    const int tpc = tok_per_cta(tc);
     if (c.dtype == MOE_F32) {
         const int row_vecs = c.H / 4;
-        combine_rows_f32_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
-            tb, tc, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
+        combine_rows_f32_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
+            tb, tc, tpc, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
             static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
     } else {
         const int row_vecs = c.H / 8;
-        combine_rows_bf16_kernel<<<(tc + kTokPerCta - 1) / kTokPerCta, kRowThreads, 0, s>>>(
-            tb, tc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
+        combine_rows_bf16_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
+            tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
             static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
     }
     return cudaGetLastError();
