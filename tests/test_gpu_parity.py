@@ -65,6 +65,10 @@ CASES = {
     "bf16_shared_decode": W("bf16_shared_decode", T=64, H=256, E=32, k=8, I=128, dtype="bf16",
                             ep=8, capacity=32, reduce_dense=True, shared_I=192),
     "f32_shared": W("f32_shared", T=128, H=128, E=8, k=2, I=128, dtype="f32", ep=2, shared_I=64),
+    # a large chunk (8192 tokens) with most slots dropped: the warp-per-token permute
+    # and combine (tokens with no kept row at all among them)
+    "bf16_sparse_chunk": W("bf16_sparse_chunk", T=8192, H=256, E=16, k=2, I=64, dtype="bf16",
+                           ep=2, capacity=256, skew_bias=True),
 }
 
 
@@ -132,7 +136,7 @@ def _forward(wl, dinp, n_chunks, same_stream=False):
 
 @pytest.mark.parametrize("name", ["bf16_ragged_m", "bf16_capacity", "bf16_chunked", "tiny_f32",
                                   "bf16_decode", "bf16_shared", "bf16_shared_decode",
-                                  "bf16_grouped_top2_selbias"])
+                                  "bf16_grouped_top2_selbias", "bf16_sparse_chunk"])
 def test_forward_chunked_matches_steps_and_oracle(name):
     wl = CASES[name]
     inp = make_inputs(wl, "cpu", seed=2)
