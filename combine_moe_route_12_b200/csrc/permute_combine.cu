@@ -212,11 +212,12 @@ __global__ void reduce_finalize_kernel(int tb, int tc, int H, int dtype,
     }
 }
 
-// Warp-per-token forms for large chunks of rows of at most 32 * kWarpVecs
+// Warp-per-token permute for large chunks of rows of at most 32 * kWarpVecs
 // 16-byte vectors (2048 bf16 values): four independent warps per CTA, no
-// barrier; a warp reads its token's pos / weights once (a lane per slot) and
-// then has the whole row in flight, kWarpVecs loads per lane, instead of a
-// chain of dependent rounds per token.
+// barrier; a warp reads its token's pos once (a lane per slot) and then has the
+// whole row in flight, kWarpVecs loads per lane, instead of a chain of
+// dependent rounds per token.  (The same form of the combine measured slower
+// than four tokens per CTA and is not used.)
 constexpr int kWarpVecs = 8;
 
 __global__ void __launch_bounds__(kRowThreads) permute_rows_warp_kernel(
@@ -248,62 +249,6 @@ __global__ void __launch_bounds__(kRowThreads) permute_rows_warp_kernel(
     }
 }
 
-// bf16 combine, warp per token: the kept rows in slot order, each loaded whole
-// (kWarpVecs vectors per lane) before its adds.
-__global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_warp_kernel(
-    int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
-    const float *__restrict__ topk_w, const uint4 *__restrict__ y_shared, uint4 *__restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const int i = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
-    if (i >= tc) return;
-    const int t = tb + i;
-    const int my_p = lane < k ? pos[(size_t)i * k + lane] : -1;
-    const float my_w = lane < k ? topk_w[(size_t)t * k + lane] : 0.0f;
-    uint32_t kept = __ballot_sync(0xffffffffu, my_p >= 0);
-    float acc[kWarpVecs][8];
-#pragma unroll
-    for (int q = 0; q < kWarpVecs; ++q) {
-        const int v = lane + 32 * q;
-        if (y_shared && v < row_vecs) {
-            unpack8(__ldg(y_shared + (size_t)i * row_vecs + v), acc[q]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[q][e] = 0.0f;
-        }
-    }
-    while (kept) {                            // slot order: lowest set bit first
-        const int j = __ffs(kept) - 1;
-        kept &= kept - 1;
-        const int p = __shfl_sync(0xffffffffu, my_p, j);
-        const float w = __shfl_sync(0xffffffffu, my_w, j);
-        const uint4 *row = y + (size_t)p * row_vecs;
-        uint4 u[kWarpVecs];
-#pragma unroll
-        for (int q = 0; q < kWarpVecs; ++q) {
-            const int v = lane + 32 * q;
-            u[q] = v < row_vecs ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int q = 0; q < kWarpVecs; ++q) {
-            float f[8];
-            unpack8(u[q], f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[q][e] = __fmaf_rn(w, f[e], acc[q][e]);
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < kWarpVecs; ++q) {
-        const int v = lane + 32 * q;
-        if (v >= row_vecs) continue;
-        uint4 o;
-        o.x = pack_bf16x2(acc[q][0], acc[q][1]);
-        o.y = pack_bf16x2(acc[q][2], acc[q][3]);
-        o.z = pack_bf16x2(acc[q][4], acc[q][5]);
-        o.w = pack_bf16x2(acc[q][6], acc[q][7]);
-        out[(size_t)t * row_vecs + v] = o;
-    }
-}
-
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *pos, int tb,
                            int tc, void *xr, cudaStream_t s) {
     if (tc == 0) return cudaSuccess;
@@ -332,12 +277,6 @@ cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *po
             static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
     } else {
         const int row_vecs = c.H / 8;
-        if (tpc > 1 && row_vecs <= 32 * kWarpVecs) {
-            combine_rows_bf16_warp_kernel<<<(tc + 3) / 4, kRowThreads, 0, s>>>(
-                tb, tc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
-                static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
-            return cudaGetLastError();
-        }
         combine_rows_bf16_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
             tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
             static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
