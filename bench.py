@@ -195,9 +195,16 @@ def kernels_per_step(wl) -> int:
     # per chunk: layout 2 (hist, scatter), permute 1, FFN 2 (two GEMM launches),
     # combine or finalize 1
     # with a shared expert, per chunk 3 more (its offsets and two GEMM launches);
-    # with the FP8 FFN, per chunk 2 more (x's and h's row quantisation)
+    # with the FP8 FFN, per chunk 1 more (h's row quantisation), 2 when x's
+    # quantisation is not fused into the permute (H > 8192)
     clip = 4 if wl.capacity > 0 else 2
-    return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + (2 if wl.ffn_fp8 else 0))
+    fp8 = (1 if fused_permute_quant(wl) else 2) if wl.ffn_fp8 else 0
+    return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + fp8)
+
+
+def fused_permute_quant(wl) -> bool:
+    """The FP8 path quantises x inside the permute for rows of up to 8192 values."""
+    return wl.ffn_fp8 and wl.H <= 8192
 
 
 def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
@@ -212,8 +219,9 @@ def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
 
     FP8 FFN: weights and receive rows are one-byte codes (plus one scale byte
     per weight row); h is written in bf16, read by its quantisation, whose
-    codes are written and read by GEMM2; the permute stage also quantises x
-    (reads it in bf16, writes its codes) before permuting the codes."""
+    codes are written and read by GEMM2; the permute stage reads the kept
+    tokens' bf16 rows and writes their codes (H <= 8192: one fused pass), or
+    quantises all of x, writes its codes and permutes them (longer rows)."""
     b = wl.elem_bytes
     N = sum(n_kept_chunks)
     tok_bytes = wl.T * wl.H * b
@@ -223,7 +231,10 @@ def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
     if wl.ffn_fp8:
         row_bytes = N * wl.H
         w_bytes = sum(active_chunks) * (3 * wl.H * wl.I + 2 * wl.I + wl.H)
-        permute_bytes = tok_bytes + wl.T * wl.H + read_bytes + row_bytes
+        if fused_permute_quant(wl):
+            permute_bytes = read_bytes * b + row_bytes
+        else:
+            permute_bytes = tok_bytes + wl.T * wl.H + read_bytes + row_bytes
         h_bytes = N * wl.I * (2 * b + 2)
     else:
         row_bytes = y_bytes
@@ -285,7 +296,7 @@ def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
     """One layer pass through the step ABI on the current stream.  ev: list of
     n_marks(wl) events recorded between the stages, or None.  fp8: the device
     (w13 codes, w13 scales, w2 codes, w2 scales) of an FP8 workload; its
-    permute stage quantises the chunk's x rows first."""
+    permute stage quantises the chunk's x rows (inside the permute for H <= 8192)."""
     rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
     rec(0)
     moe.moe_route_topk(cfg, inp.logits, inp.bias, B.topk_idx, B.topk_w, B.counts, B.ws)
@@ -300,7 +311,9 @@ def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
         moe.moe_dispatch_layout(cfg, tb, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
                                 B.pos, B.spl, None, B.ws)
         rec(base)
-        if wl.ffn_fp8:
+        if fused_permute_quant(wl):
+            moe.moe_permute_quantize_fp8(cfg, inp.x, B.pos, tb, B.tc, B.xr, B.xsc)
+        elif wl.ffn_fp8:
             moe.moe_quantize_fp8_rows(inp.x[tb:tb + B.tc], B.xq[tb:tb + B.tc], B.xsc[tb:tb + B.tc])
             moe.moe_permute(cfg, B.xq, B.pos, tb, B.tc, B.xr)
         else:

@@ -52,16 +52,21 @@ __device__ __forceinline__ float vec_amax(const uint4 &q) {
                  fmaxf(fabsf(__uint_as_float(q.z)), fabsf(__uint_as_float(q.w))));
 }
 
+// The 8 codes of one 16-byte vector of 8 bf16 values.
+__device__ __forceinline__ uint2 bf16_vec_codes(const uint4 &q, float inv) {
+    uint2 o;
+    o.x = e4m3x2(bf16_lo(q.x) * inv, bf16_hi(q.x) * inv) |
+          e4m3x2(bf16_lo(q.y) * inv, bf16_hi(q.y) * inv) << 16;
+    o.y = e4m3x2(bf16_lo(q.z) * inv, bf16_hi(q.z) * inv) |
+          e4m3x2(bf16_lo(q.w) * inv, bf16_hi(q.w) * inv) << 16;
+    return o;
+}
+
 // The codes of one 16-byte vector (8 bf16 or 4 fp32 values) at vector v of dst.
 template <bool BF16>
 __device__ __forceinline__ void vec_store_codes(uint8_t *dst, int v, const uint4 &q, float inv) {
     if (BF16) {
-        uint2 o;
-        o.x = e4m3x2(bf16_lo(q.x) * inv, bf16_hi(q.x) * inv) |
-              e4m3x2(bf16_lo(q.y) * inv, bf16_hi(q.y) * inv) << 16;
-        o.y = e4m3x2(bf16_lo(q.z) * inv, bf16_hi(q.z) * inv) |
-              e4m3x2(bf16_lo(q.w) * inv, bf16_hi(q.w) * inv) << 16;
-        reinterpret_cast<uint2 *>(dst)[v] = o;
+        reinterpret_cast<uint2 *>(dst)[v] = bf16_vec_codes(q, inv);
     } else {
         reinterpret_cast<uint32_t *>(dst)[v] =
             e4m3x2(__uint_as_float(q.x) * inv, __uint_as_float(q.y) * inv) |
@@ -114,6 +119,76 @@ __global__ void __launch_bounds__(32 * kQuantWarps) quant_rows_kernel(
             for (int v = lane; v < nv; v += 32) vec_store_codes<BF16>(dst, v, src[v], inv);
         }
     }
+}
+
+// Quantise-and-permute of a chunk's bf16 token rows (the forward's FP8 path):
+// one CTA per token; the row is read once into registers (VPT 16-byte vectors
+// per thread), its scale taken over the CTA, and its codes written straight to
+// each kept receive row; a token with every slot dropped is not read.  The
+// codes equal those of quant_rows_kernel followed by the permute.
+constexpr int kPqThreads = 128;
+
+template <int VPT>
+__global__ void __launch_bounds__(kPqThreads) permute_quant_kernel(
+    int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
+    uint8_t *__restrict__ xr_q, uint8_t *__restrict__ x_scale) {
+    __shared__ int32_t s_pos[kMaxTopK];
+    __shared__ float s_red[kPqThreads / 32];
+    __shared__ int s_any;
+    const int i = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        const int p = lane < k ? pos[(size_t)i * k + lane] : -1;
+        if (lane < k) s_pos[lane] = p;
+        const uint32_t any = __ballot_sync(0xffffffffu, p >= 0);
+        if (lane == 0) s_any = any != 0u;
+    }
+    __syncthreads();
+    if (!s_any) return;                         // every slot dropped: x[t] is not needed
+    const uint4 *src = x + (size_t)(tb + i) * row_vecs;
+    uint4 q[VPT];
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int v = threadIdx.x + kPqThreads * j;
+        q[j] = v < row_vecs ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+        amax = fmaxf(amax, vec_amax<true>(q[j]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) s_red[warp] = amax;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kPqThreads / 32; ++w) amax = fmaxf(amax, s_red[w]);
+    const int e = ue8m0_exponent(amax);
+    const float inv = pow2_neg(e);
+    if (threadIdx.x == 0) x_scale[tb + i] = (uint8_t)(e + 127);
+    const size_t row_bytes = (size_t)row_vecs * 8;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int v = threadIdx.x + kPqThreads * j;
+        if (v >= row_vecs) continue;
+        const uint2 c = bf16_vec_codes(q[j], inv);
+        for (int jj = 0; jj < k; ++jj) {
+            const int p = s_pos[jj];
+            if (p >= 0) reinterpret_cast<uint2 *>(xr_q + (size_t)p * row_bytes)[v] = c;
+        }
+    }
+}
+
+// Returns cudaErrorNotSupported for rows longer than 1024 vectors (8192 values).
+cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                                 int tc, uint8_t *xr_q, uint8_t *x_scale, cudaStream_t s) {
+    if (tc == 0) return cudaSuccess;
+    const int row_vecs = c.H / 8;
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    if (row_vecs <= 2 * kPqThreads)
+        permute_quant_kernel<2><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
+    else if (row_vecs <= 8 * kPqThreads)
+        permute_quant_kernel<8><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
+    else
+        return cudaErrorNotSupported;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,

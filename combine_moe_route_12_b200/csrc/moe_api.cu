@@ -44,6 +44,8 @@ cudaError_t launch_ffn_tcgen05_fp8(const moe_config &c, int64_t n_rows, const ui
                                    uint32_t *counters, cudaStream_t s, int num_sms);
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
                               uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms);
+cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                                 int tc, uint8_t *xr_q, uint8_t *x_scale, cudaStream_t s);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -100,6 +102,10 @@ moe_status check_range(const moe_config &c, int32_t tb, int32_t tc, bool need_ep
     return MOE_OK;
 }
 
+// The forward's FP8 path quantises x inside the permute for rows of up to 8192
+// values; longer rows take a separate quantisation pass through x's codes.
+bool fused_permute_quant(const moe_config &c) { return c.H <= 8192; }
+
 // Forward workspace: scratch first, then saved counts, two chunk slots, and
 // the dense fp32 reduce buffer (decode form).
 struct Slot {
@@ -147,7 +153,7 @@ ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
         S.hq = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1) * c.I) : 0;
         S.hsc = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1)) : 0;
     }
-    F.xq = c.ffn_fp8 ? take((size_t)c.T * c.H) : 0;
+    F.xq = c.ffn_fp8 && !fused_permute_quant(c) ? take((size_t)c.T * c.H) : 0;
     F.xsc = c.ffn_fp8 ? take((size_t)c.T) : 0;
     F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
     if (host_io) {
@@ -389,6 +395,22 @@ moe_status moe_quantize_fp8_rows(int64_t rows, int32_t cols, int32_t in_dtype, c
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_fp8_rows");
 }
 
+moe_status moe_permute_quantize_fp8(const moe_config *cfg, const void *x, const int32_t *pos,
+                                    int32_t tok_begin, int32_t tok_count, uint8_t *xr_q,
+                                    uint8_t *x_scale, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (!c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 0: use moe_permute");
+    if (!fused_permute_quant(c)) return fail(MOE_ERR_UNSUPPORTED, "H=%d > 8192", c.H);
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!x || !pos || !xr_q || !x_scale))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(xr_q, 16)) return fail(MOE_ERR_INVALID_ARG, "x / xr_q not 16-byte aligned");
+    cudaError_t err = launch_permute_quant(c, x, pos, tok_begin, tok_count, xr_q, x_scale, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute_quantize_fp8");
+}
+
 moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, const uint8_t *xr_q,
                                       const uint8_t *x_scale, const int32_t *expert_offsets,
                                       const uint8_t *w13_q, const uint8_t *w13_scale,
@@ -612,8 +634,12 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
                                        ws, F.nmax, s_dispatch, nsm),
                 "dispatch_layout");
         if (io) MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_x[ch], 0), "wait x");
-        if (c.ffn_fp8) {
-            // the chunk's token rows to E4M3 codes, then the codes are permuted
+        if (c.ffn_fp8 && fused_permute_quant(c)) {
+            // each kept token row quantised once and its codes written to its receive rows
+            MOE_TRY(launch_permute_quant(c, x, pos, tb, tc, static_cast<uint8_t *>(xr),
+                                         ws_at<uint8_t>(ws, F.xsc), s_dispatch), "permute + quantize x");
+        } else if (c.ffn_fp8) {
+            // rows too long for the fused kernel: quantise the chunk's rows, then permute the codes
             uint8_t *xq = ws_at<uint8_t>(ws, F.xq);
             MOE_TRY(launch_quant_rows(tc, c.H, true, static_cast<const char *>(x) + eb * (size_t)tb * c.H,
                                       xq + (size_t)tb * c.H, ws_at<uint8_t>(ws, F.xsc) + tb, nullptr,

@@ -73,6 +73,7 @@ _decl("moe_forward_host_workspace_bytes", ctypes.c_size_t, _CFG)
 _decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
 _decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
 _decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
+_decl("moe_permute_quantize_fp8", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
@@ -220,6 +221,12 @@ def quantize_fp8(inp, stream=None):
     scales = torch.empty(flat.shape[0], dtype=torch.uint8, device=inp.device)
     moe_quantize_fp8_rows(flat, codes, scales, stream)
     return codes.view(inp.shape), scales.view(inp.shape[:-1])
+
+
+def moe_permute_quantize_fp8(cfg, x, pos, tok_begin, tok_count, xr_q, x_scale, stream=None):
+    """Kept token rows of x quantised to E4M3 codes and written to their receive rows."""
+    _check(_lib.moe_permute_quantize_fp8(ctypes.byref(cfg), _ptr(x), _ptr(pos), tok_begin,
+                                         tok_count, _ptr(xr_q), _ptr(x_scale), _stream(stream)))
 
 
 def moe_grouped_swiglu_ffn_fp8(cfg, n_rows, xr_q, x_scale, expert_offsets, w13_q, w13_scale, w2_q,

@@ -18,8 +18,9 @@
  * Also: routing variants through moe_config (grouped top-k, a bias that steers
  * the selection only); moe_shared_expert_ffn, a dense shared expert whose rows
  * the combine adds; moe_dispatch_layout_noalloc, step 3 with its scratch in a
- * fixed library array; moe_quantize_fp8_rows and moe_grouped_swiglu_ffn_fp8,
- * the expert FFN on E4M3 codes with UE8M0 row scales (cfg->ffn_fp8);
+ * fixed library array; moe_quantize_fp8_rows, moe_permute_quantize_fp8 and
+ * moe_grouped_swiglu_ffn_fp8, the expert FFN on E4M3 codes with UE8M0 row
+ * scales (cfg->ffn_fp8);
  * moe_watchdog_selftest, which makes a bounded wait run out on purpose;
  * moe_device_status, the device-side error bits.
  *
@@ -309,6 +310,20 @@ moe_status moe_quantize_fp8_rows(int64_t rows, int32_t cols, int32_t in_dtype, c
                                  uint8_t *codes, uint8_t *scales, cudaStream_t stream);
 
 /*
+ * Steps 4 and the quantisation of x fused (cfg->ffn_fp8 = 1, cfg->H <= 8192): for
+ * t in [tok_begin, tok_begin + tok_count) with at least one kept slot, the bf16
+ * row x[t] is quantised as moe_quantize_fp8_rows does (x_scale[t] = its UE8M0
+ * byte) and its E4M3 codes are written to every receive row pos[t - tok_begin,
+ * j] >= 0 of xr_q [N_max, H].  Rows and scales of tokens without a kept slot are
+ * left untouched (x[t] is not read).  The codes and scales equal those of
+ * moe_quantize_fp8_rows followed by moe_permute; moe_forward_chunked and
+ * moe_forward_host use this form.  MOE_ERR_UNSUPPORTED for H > 8192.
+ */
+moe_status moe_permute_quantize_fp8(const moe_config *cfg, const void *x, const int32_t *pos,
+                                    int32_t tok_begin, int32_t tok_count, uint8_t *xr_q,
+                                    uint8_t *x_scale, cudaStream_t stream);
+
+/*
  * Step 5 in FP8 (cfg->ffn_fp8 = 1): the SwiGLU FFN of moe_grouped_swiglu_ffn
  * on E4M3 operands with UE8M0 row scales (value = code * 2^(scale - 127)):
  *   xr_q [n_rows, H]: codes of the receive rows (moe_permute of the codes of
@@ -387,8 +402,9 @@ moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32
  *            s_compute, and its rows are added in chunk c's combine.
  *   w13_scale, w2_scale: with cfg->ffn_fp8 = 1, w13 and w2 are E4M3 codes and
  *            these their row scales (moe_grouped_swiglu_ffn_fp8); x stays
- *            bf16 and each chunk's rows are quantised (moe_quantize_fp8_rows)
- *            before their permutation.  Else ignored, may be NULL.
+ *            bf16 and each chunk's kept rows are quantised inside the permute
+ *            (moe_permute_quantize_fp8; for H > 8192 by moe_quantize_fp8_rows
+ *            then moe_permute).  Else ignored, may be NULL.
  *   topk_idx [T,k], topk_w [T,k], keep [T,k]: caller-owned saved state
  *            ([AX] the routing top-k is always saved).
  *   splits_host: pinned host int32 [n_chunks * (E+1 + ep*ep)] or NULL; chunk c

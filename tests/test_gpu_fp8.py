@@ -149,3 +149,35 @@ def test_fp8_forward_needs_scales_and_rejects_shared_expert():
         moe.config_check(moe.config_from_workload(wl.with_(shared_I=128)))
     with pytest.raises(moe.MoEError):
         moe.config_check(moe.config_from_workload(wl.with_(H=192)))
+
+
+@pytest.mark.parametrize("name", ["fp8_basic", "fp8_capacity", "fp8_many_experts", "fp8_chunked"])
+def test_permute_quantize_equals_quantize_then_permute(name):
+    """The fused form writes the same codes to the same receive rows, and the
+    same scales for every token that keeps a slot, as row quantisation followed
+    by the permute; rows and scales of other tokens stay untouched."""
+    wl, inp, wq = _prepare(name, seed=4)
+    dinp = to_device(inp)
+    g = run_gpu_steps(wl, dinp, fp8=fp8_weights_to_device(wq))
+    cfg = moe.config_from_workload(wl)
+    tc = wl.T // wl.n_chunks
+    nmax = moe.max_recv_rows(cfg, tc)
+    xs = torch.full((wl.T,), 0xEE, dtype=torch.uint8, device="cuda")
+    for c, gc in enumerate(g["chunks"]):
+        pos = torch.from_numpy(gc["pos"]).cuda()
+        xr = torch.full((max(nmax, 1), wl.H), 0xEE, dtype=torch.uint8, device="cuda")
+        moe.moe_permute_quantize_fp8(cfg, dinp.x, pos, c * tc, tc, xr, xs)
+        torch.cuda.synchronize()
+        n = gc["N"]
+        np.testing.assert_array_equal(xr[:n].cpu().numpy(), gc["xr"])
+        assert (xr[n:].cpu().numpy() == 0xEE).all()
+    kept_tok = g["keep"].any(axis=1)
+    np.testing.assert_array_equal(xs.cpu().numpy()[kept_tok], g["xs"][kept_tok])
+    assert (xs.cpu().numpy()[~kept_tok] == 0xEE).all()
+
+
+def test_permute_quantize_rejects_long_rows():
+    cfg = moe.config_from_workload(CASES["fp8_basic"].with_(H=8320))
+    z = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoEError):
+        moe.moe_permute_quantize_fp8(cfg, z, z, 0, 0, z, z)
