@@ -153,12 +153,15 @@ def test_fp8_forward_needs_scales_and_rejects_shared_expert():
 
 @pytest.mark.parametrize("name", ["fp8_basic", "fp8_capacity", "fp8_many_experts", "fp8_chunked"])
 def test_permute_quantize_equals_quantize_then_permute(name):
-    """The fused form writes the same codes to the same receive rows, and the
-    same scales for every token that keeps a slot, as row quantisation followed
-    by the permute; rows and scales of other tokens stay untouched."""
+    """The fused form writes the oracle's codes (its row quantisation followed by
+    its permute) to the receive rows, and the oracle's scales for every token
+    that keeps a slot; rows and scales of other tokens stay untouched."""
     wl, inp, wq = _prepare(name, seed=4)
     dinp = to_device(inp)
     g = run_gpu_steps(wl, dinp, fp8=fp8_weights_to_device(wq))
+    orc = oracle_routing(wl, inp)
+    assert_routing_equal(g, orc, wl)
+    xq_ref, xs_ref = oracle.quantize_rows(storage_np(inp.x))
     cfg = moe.config_from_workload(wl)
     tc = wl.T // wl.n_chunks
     nmax = moe.max_recv_rows(cfg, tc)
@@ -168,11 +171,12 @@ def test_permute_quantize_equals_quantize_then_permute(name):
         xr = torch.full((max(nmax, 1), wl.H), 0xEE, dtype=torch.uint8, device="cuda")
         moe.moe_permute_quantize_fp8(cfg, dinp.x, pos, c * tc, tc, xr, xs)
         torch.cuda.synchronize()
-        n = gc["N"]
-        np.testing.assert_array_equal(xr[:n].cpu().numpy(), gc["xr"])
+        lay = orc["layouts"][c]
+        n = lay["N"]
+        np.testing.assert_array_equal(xr[:n].cpu().numpy(), oracle.permute(xq_ref, lay["recv_token"]))
         assert (xr[n:].cpu().numpy() == 0xEE).all()
-    kept_tok = g["keep"].any(axis=1)
-    np.testing.assert_array_equal(xs.cpu().numpy()[kept_tok], g["xs"][kept_tok])
+    kept_tok = orc["keep"].any(axis=1)
+    np.testing.assert_array_equal(xs.cpu().numpy()[kept_tok], xs_ref[kept_tok])
     assert (xs.cpu().numpy()[~kept_tok] == 0xEE).all()
 
 
