@@ -49,7 +49,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": 1560.882432e6, "src": "ab5f51ea4de56437"},
+    "qwen3_30b_a3b": {"bytes": 1560.882432e6, "src": "24bdbd71939c8d30"},
     # both GEMM launches and the quantisation of h between them
     "qwen3_30b_a3b_fp8": {"bytes": 893.983232e6, "src": "ab5f51ea4de56437"},
 }
@@ -107,11 +107,12 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_src_hash():
-    """Hash of the FFN's sources (the grouped GEMM kernel and the row quantisation
-    between its launches): recorded traffic holds only for these bytes."""
+def kernel_src_hash(fp8: bool = False):
+    """Hash of the FFN's sources: the grouped GEMM kernel, and for the FP8 FFN also
+    the row quantisation between its launches.  Recorded traffic holds only for
+    these bytes."""
     h = hashlib.sha256()
-    for name in ("ffn_tcgen05.cu", "fp8_quant.cu"):
+    for name in ("ffn_tcgen05.cu", "fp8_quant.cu") if fp8 else ("ffn_tcgen05.cu",):
         with open(os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -681,7 +682,7 @@ def run_ours(args):
         t_byte = alg["ffn_bytes"] / (peaks["hbm_gbs"] * 1e9)
         hbm_bound = t_byte > t_flop
         dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
-        src = kernel_src_hash()
+        src = kernel_src_hash(wl.ffn_fp8)
         tr = FFN_TRAFFIC.get(wl.name)
         traffic = tr["bytes"] if tr and tr.get("src") == src and tr.get("chunks", 1) == wl.n_chunks else None
         line = {
