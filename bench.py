@@ -145,7 +145,7 @@ class ClockSampler:
             self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self.ok = True
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - depends on the NVML of the machine
             self.err = str(e)
 
     def _run(self):

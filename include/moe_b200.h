@@ -73,7 +73,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,  /* bad pointer, size or topology; nothing launched */
-    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits (below)   */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid but outside the library's limits (below) */
     MOE_ERR_WORKSPACE = 3,    /* workspace pointer misaligned                    */
     MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed            */
     MOE_ERR_DEVICE = 5        /* the device status word has bits set             */
