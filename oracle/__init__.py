@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
         L.orc_quantize_rows.restype = None
         L.orc_ffn_row_fp8.argtypes = [i, i, P, ctypes.c_uint8, P, P, P, P, P, P, P, P, P]
         L.orc_ffn_row_fp8.restype = None
+        L.orc_ffn_row_bwd.argtypes = [i, i, i, P, P, P, P, P, P, P, P]
+        L.orc_ffn_row_bwd.restype = None
+        L.orc_layer_bwd.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_layer_bwd.restype = None
         _lib = L
     return _lib
 
@@ -94,7 +98,9 @@ def _dtype_code(a: np.ndarray) -> int:
         return 0
     if a.dtype == np.uint16:
         return 1
-    raise TypeError(f"storage arrays are float32 or uint16 (bf16 bits), got {a.dtype}")
+    if a.dtype == np.float64:
+        return 2          # no rounding anywhere: the backward's finite-difference checks
+    raise TypeError(f"storage arrays are float32, uint16 (bf16 bits) or float64, got {a.dtype}")
 
 
 # --------------------------------------------------------------------------- steps
@@ -304,6 +310,89 @@ def ffn_row_fp8(x_codes, x_scale, w13_codes, w13_scales, w2_codes, w2_scales):
     lib().orc_ffn_row_fp8(H, I, _p(x_codes), int(x_scale), _p(w13_codes), _p(w13_scales),
                           _p(w2_codes), _p(w2_scales), _p(h), _p(hq), ctypes.byref(sh), _p(y), _p(ye))
     return h, hq, int(sh.value), y, ye
+
+
+# --------------------------------------------------------------------------- backward
+
+def ffn_row_backward(x_row, w13_e, w2_e, dy):
+    """One expert's SwiGLU FFN backward on one row.  Returns (dx [H], dW13 [2I, H],
+    dW2 [H, I], y [H]) in float64."""
+    x_row = np.ascontiguousarray(x_row)
+    w13_e = np.ascontiguousarray(w13_e)
+    w2_e = np.ascontiguousarray(w2_e)
+    dt = _dtype_code(x_row)
+    H = x_row.shape[0]
+    I = w13_e.shape[0] // 2
+    dy = np.ascontiguousarray(dy, np.float64)
+    dx = np.zeros(H, np.float64)
+    dW13 = np.zeros((2 * I, H), np.float64)
+    dW2 = np.zeros((H, I), np.float64)
+    y = np.zeros(H, np.float64)
+    lib().orc_ffn_row_bwd(H, I, dt, _p(x_row), _p(w13_e), _p(w2_e), _p(dy), _p(dx), _p(dW13),
+                          _p(dW2), _p(y))
+    return dx, dW13, dW2, y
+
+
+def moe_layer_backward(logits, bias, x, w13, w2, k: int, ep: int, dout, capacity: int = -1,
+                       n_chunks: int = 1, n_group: int = 0, topk_group: int = 0,
+                       group_score: int = 0, bias_select_only: bool = False,
+                       w13_shared=None, w2_shared=None, save_dispatch: bool = False) -> dict:
+    """Gradient of L = <dout, out> for the layer of moe_layer (axolotl
+    expert_parallel_save_dispatch): the routing top-k, keep mask and layouts are
+    what the forward saved; with save_dispatch the expert rows are read from the
+    forward's receive buffers (the saved dispatch outputs), otherwise they are
+    recomputed from x (the same values).  Returns float64 dx [T, H], dlogits
+    [T, E], dbias [E] (zero when the bias steers the selection only), dW13,
+    dW2 and, with a shared expert, dW13_shared, dW2_shared; and the saved
+    routing."""
+    T, E = logits.shape
+    H = x.shape[1]
+    I = w13.shape[1] // 2
+    dt = _dtype_code(x)
+    idx, w, _, st = route_topk(logits, bias, k, n_group, topk_group, group_score, bias_select_only)
+    if st != ORC_OK:
+        raise ValueError(f"route_topk status {st}")
+    keep, _ = capacity_clip(idx, w, E, capacity)
+    if save_dispatch:
+        # the forward's receive rows, chunk after chunk, and each slot's row in them
+        tc = T // n_chunks
+        rows, row_of, base = [], np.zeros((T, k), np.int32), 0
+        for c in range(n_chunks):
+            lay = dispatch_layout(idx, keep, E, ep, c * tc, tc)
+            rows.append(permute(x, lay["recv_token"]))
+            pos = lay["pos"]
+            row_of[c * tc:(c + 1) * tc] = np.where(pos >= 0, pos + base, 0)
+            base += lay["N"]
+        x_rows = np.ascontiguousarray(np.concatenate(rows) if base > 0 else x[:1])
+    else:
+        x_rows = x
+        row_of = np.repeat(np.arange(T, dtype=np.int32)[:, None], k, axis=1)
+    dout = np.ascontiguousarray(dout, np.float64)
+    dx = np.zeros((T, H), np.float64)
+    dz = np.zeros((T, k), np.float64)
+    dW13 = np.zeros((E, 2 * I, H), np.float64)
+    dW2 = np.zeros((E, H, I), np.float64)
+    lib().orc_layer_bwd(T, H, E, k, I, dt, _p(idx), _p(w), _p(keep), _p(x_rows),
+                        _p(np.ascontiguousarray(row_of)), _p(np.ascontiguousarray(w13)),
+                        _p(np.ascontiguousarray(w2)), _p(dout), _p(dx), _p(dz), _p(dW13), _p(dW2))
+    dlogits = np.zeros((T, E), np.float64)
+    np.add.at(dlogits, (np.repeat(np.arange(T), k), idx.ravel()), dz.ravel())
+    dbias = np.zeros(E, np.float64) if bias is None or bias_select_only else dlogits.sum(axis=0)
+    res = dict(dx=dx, dlogits=dlogits, dbias=dbias, dW13=dW13, dW2=dW2, topk_idx=idx, topk_w=w,
+               keep=keep)
+    if w13_shared is not None:
+        # the shared expert: every token, weight 1 (one expert, one slot)
+        Is = w13_shared.shape[0] // 2
+        dW13s = np.zeros((1, 2 * Is, H), np.float64)
+        dW2s = np.zeros((1, H, Is), np.float64)
+        ones = np.ones((T, 1), np.float32)
+        lib().orc_layer_bwd(T, H, 1, 1, Is, dt, _p(np.zeros((T, 1), np.int32)), _p(ones),
+                            _p(np.ones((T, 1), np.uint8)), _p(np.ascontiguousarray(x)),
+                            _p(np.arange(T, dtype=np.int32)[:, None].copy()),
+                            _p(np.ascontiguousarray(w13_shared)), _p(np.ascontiguousarray(w2_shared)),
+                            _p(dout), _p(dx), _p(np.zeros((T, 1), np.float64)), _p(dW13s), _p(dW2s))
+        res.update(dW13_shared=dW13s[0], dW2_shared=dW2s[0])
+    return res
 
 
 # --------------------------------------------------------------------------- whole layer

@@ -19,6 +19,8 @@
  *      (silu_and_mul) between the two grouped GEMMs, decode reducing expert
  *      outputs straight into a dense output, the FP8 grouped GEMM with UE8M0
  *      (power-of-two) scales and the quantisation of h after silu_and_mul.
+ *  - the same axolotl page, expert_parallel_save_dispatch: the layer's
+ *      backward with the dispatch outputs saved or recomputed.
  *
  * Readings of points the pages leave open are marked "Reading:".
  *
@@ -304,10 +306,12 @@ void orc_permute(int H, int elem_bytes, int N, const void *x, const int32_t *rec
 }
 
 /* ------------------------------------------------------------------------- */
-/* Storage types.  dtype 0 = fp32, 1 = bf16 (stored as uint16 bit patterns).  */
+/* Storage types.  dtype 0 = fp32, 1 = bf16 (stored as uint16 bit patterns),   */
+/* 2 = fp64 (for the backward's finite-difference checks: no rounding at all). */
 /* ------------------------------------------------------------------------- */
 static double orc_load(const void *base, size_t i, int dtype)
 {
+    if (dtype == 2) return ((const double *)base)[i];
     if (dtype == 0) return (double)((const float *)base)[i];
     uint32_t u = (uint32_t)((const uint16_t *)base)[i] << 16;
     float f;
@@ -344,7 +348,8 @@ uint16_t orc_bf16_from_double(double v)
 
 static void orc_store(void *base, size_t i, int dtype, double v)
 {
-    if (dtype == 0) ((float *)base)[i] = (float)v;
+    if (dtype == 2) ((double *)base)[i] = v;
+    else if (dtype == 0) ((float *)base)[i] = (float)v;
     else ((uint16_t *)base)[i] = orc_bf16_from_double(v);
 }
 
@@ -373,7 +378,7 @@ void orc_ffn_row(int H, int I, int dtype, const void *x_row, const void *w13_e,
         }
         double hv = g / (1.0 + exp(-g)) * u;
         if (h_store) orc_store(h_store, (size_t)i, dtype, hv);
-        if (round_h) {
+        if (round_h && dtype != 2) {
             if (dtype == 0) hv = (double)(float)hv;
             else {
                 uint32_t bits = (uint32_t)orc_bf16_from_double(hv) << 16;
@@ -574,4 +579,114 @@ void orc_ffn_row_fp8(int H, int I, const uint8_t *x, uint8_t sx, const uint8_t *
     free(h);
     free(hq);
     free(hv);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Backward of the layer (axolotl ExpertParallelArgs, expert_parallel_save_   */
+/* dispatch: under activation checkpointing the backward either holds the     */
+/* dispatch / combine all-to-all outputs from the forward or re-issues them;  */
+/* the routing top-k and the split counts are always saved).                  */
+/* Reading: the backward is the gradient of the layer's exact function at the */
+/* stored inputs: fp64 throughout, h and y not rounded; the top-k selection   */
+/* and the capacity clip are piecewise constant (no gradient through them).   */
+/*   out[t] = sum over kept slots j of w[t,j] * FFN_{e_j}(x[t])               */
+/*   w[t,:] = softmax over the k selected (biased, or with bias_select_only   */
+/*            unbiased) logits z[t,:]                                          */
+/* For L = <dout, out>:                                                        */
+/*   dy[t,j] = w[t,j] dout[t];  dw[t,j] = <dout[t], FFN_{e_j}(x[t])> (kept j,   */
+/*   else 0);  dz[t,j] = w[t,j] (dw[t,j] - sum_i w[t,i] dw[t,i]).              */
+/* ------------------------------------------------------------------------- */
+
+/* One expert's SwiGLU FFN backward on one row, for an incoming dy [H]:
+ *   g_i, u_i as in orc_ffn_row (double);  s_i = 1 / (1 + exp(-g_i));
+ *   h_i = g_i s_i u_i;  dh_i = sum_o W2[o,i] dy_o;
+ *   dg_i = dh_i u_i s_i (1 + g_i (1 - s_i))     (d silu(g) / dg)
+ *   du_i = dh_i g_i s_i
+ *   dx_c += sum_i W13[i,c] dg_i + W13[I+i,c] du_i
+ *   dW2[o,i] += dy_o h_i;  dW13[i,c] += dg_i x_c;  dW13[I+i,c] += du_i x_c.
+ * dx, dW13 [2I, H] and dW2 [H, I] accumulate (double); y_exact (optional)
+ * gets the row's forward output. */
+void orc_ffn_row_bwd(int H, int I, int dtype, const void *x_row, const void *w13_e,
+                     const void *w2_e, const double *dy, double *dx, double *dW13,
+                     double *dW2, double *y_exact)
+{
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    for (int i = 0; i < I; ++i) {
+        double gi = 0.0, ui = 0.0;
+        for (int c = 0; c < H; ++c) {
+            double xv = orc_load(x_row, (size_t)c, dtype);
+            gi += orc_load(w13_e, (size_t)i * H + c, dtype) * xv;
+            ui += orc_load(w13_e, (size_t)(I + i) * H + c, dtype) * xv;
+        }
+        g[i] = gi;
+        u[i] = ui;
+        h[i] = gi / (1.0 + exp(-gi)) * ui;
+    }
+    if (y_exact)
+        for (int o = 0; o < H; ++o) {
+            double acc = 0.0;
+            for (int i = 0; i < I; ++i) acc += orc_load(w2_e, (size_t)o * I + i, dtype) * h[i];
+            y_exact[o] = acc;
+        }
+    for (int i = 0; i < I; ++i) {
+        double dh = 0.0;
+        for (int o = 0; o < H; ++o) dh += orc_load(w2_e, (size_t)o * I + i, dtype) * dy[o];
+        const double s = 1.0 / (1.0 + exp(-g[i]));
+        const double dg = dh * u[i] * s * (1.0 + g[i] * (1.0 - s));
+        const double du = dh * g[i] * s;
+        for (int c = 0; c < H; ++c) {
+            const double xv = orc_load(x_row, (size_t)c, dtype);
+            dx[c] += orc_load(w13_e, (size_t)i * H + c, dtype) * dg +
+                     orc_load(w13_e, (size_t)(I + i) * H + c, dtype) * du;
+            dW13[(size_t)i * H + c] += dg * xv;
+            dW13[(size_t)(I + i) * H + c] += du * xv;
+        }
+    }
+    for (int o = 0; o < H; ++o)
+        for (int i = 0; i < I; ++i) dW2[(size_t)o * I + i] += dy[o] * h[i];
+    free(g);
+    free(u);
+    free(h);
+}
+
+/* The routed part of the backward for tokens [0, T): every kept slot (t, j)
+ * of expert e = topk_idx[t, j] takes its row backward with dy = w dout[t]
+ * (x[t] read as x_rows[row_of[t*k + j]]: the saved receive rows, or x itself
+ * with row_of = the token, when they are recomputed) and gives dw[t, j];
+ * then dz[t, :] by the softmax backward over the token's k slots.
+ * dx [T, H], dW13 [E, 2I, H], dW2 [E, H, I] accumulate; dz [T, k] is written. */
+void orc_layer_bwd(int T, int H, int E, int k, int I, int dtype, const int32_t *topk_idx,
+                   const float *topk_w, const uint8_t *keep, const void *x_rows,
+                   const int32_t *row_of, const void *w13, const void *w2, const double *dout,
+                   double *dx, double *dz, double *dW13, double *dW2)
+{
+    const size_t eb = dtype == 2 ? 8 : dtype == 0 ? 4 : 2;
+    double *dy = (double *)malloc(sizeof(double) * (size_t)H);
+    double *y = (double *)malloc(sizeof(double) * (size_t)H);
+    double *dw = (double *)malloc(sizeof(double) * (size_t)k);
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            dw[j] = 0.0;
+            if (!keep[(size_t)t * k + j]) continue;
+            const int e = topk_idx[(size_t)t * k + j];
+            const double w = (double)topk_w[(size_t)t * k + j];
+            for (int c = 0; c < H; ++c) dy[c] = w * dout[(size_t)t * H + c];
+            const void *xr = (const char *)x_rows + (size_t)row_of[(size_t)t * k + j] * H * eb;
+            orc_ffn_row_bwd(H, I, dtype, xr, (const char *)w13 + (size_t)e * 2 * I * H * eb,
+                            (const char *)w2 + (size_t)e * H * I * eb, dy, dx + (size_t)t * H,
+                            dW13 + (size_t)e * 2 * I * H, dW2 + (size_t)e * H * I, y);
+            double acc = 0.0;
+            for (int c = 0; c < H; ++c) acc += dout[(size_t)t * H + c] * y[c];
+            dw[j] = acc;
+        }
+        double sw = 0.0;
+        for (int j = 0; j < k; ++j) sw += (double)topk_w[(size_t)t * k + j] * dw[j];
+        for (int j = 0; j < k; ++j)
+            dz[(size_t)t * k + j] = (double)topk_w[(size_t)t * k + j] * (dw[j] - sw);
+    }
+    free(dy);
+    free(y);
+    free(dw);
 }
