@@ -53,6 +53,10 @@ def test_max_recv_rows_is_padded_worst_case():
     (dict(I=100), moe.MOE_ERR_UNSUPPORTED),
     (dict(dtype=7), moe.MOE_ERR_INVALID_ARG),
     (dict(n_chunks=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(ffn_fp8=True, dtype=moe.MOE_F32), moe.MOE_ERR_UNSUPPORTED),   # FP8 FFN needs bf16
+    (dict(ffn_fp8=True, H=192), moe.MOE_ERR_UNSUPPORTED),               # and H, I % 128
+    (dict(ffn_fp8=True, I=192), moe.MOE_ERR_UNSUPPORTED),
+    (dict(ffn_fp8=True, shared_I=128), moe.MOE_ERR_UNSUPPORTED),        # no FP8 shared expert
 ])
 def test_config_rejections(kw, status):
     base = dict(T=64, H=128, E=8, k=2, I=128, ep=2, capacity=-1, dtype=moe.MOE_BF16,
@@ -81,3 +85,48 @@ def test_null_workspace_rejected_before_any_launch():
 def test_status_strings():
     for s in range(6):
         assert moe.status_string(s)
+
+
+def test_fp8_entry_points_reject_bad_arguments_before_any_launch():
+    ws = ctypes.c_void_p(256)            # aligned, never dereferenced on these paths
+    # the row quantisation: bf16 rows must be a whole number of 8-value vectors
+    st = moe._lib.moe_quantize_fp8_rows(4, 12, moe.MOE_BF16, None, None, None, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    st = moe._lib.moe_quantize_fp8_rows(4, 16, moe.MOE_BF16, None, None, None, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+    st = moe._lib.moe_quantize_fp8_rows(0, 16, moe.MOE_BF16, None, None, None, None)
+    assert st == moe.MOE_OK                                  # nothing to do
+    st = moe._lib.moe_quantize_fp8_rows(4, 16, 5, None, None, None, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    bf = moe.make_config(64, 128, 8, 2, 128, 2)
+    f8 = moe.make_config(64, 128, 8, 2, 128, 2, ffn_fp8=True)
+    # the FFN entry points refuse the other form's config
+    st = moe._lib.moe_grouped_swiglu_ffn(ctypes.byref(f8), 16, *([None] * 10), ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "fp8" in moe.last_error_detail()
+    st = moe._lib.moe_grouped_swiglu_ffn_fp8(ctypes.byref(bf), 16, *([None] * 15), ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "fp8" in moe.last_error_detail()
+    st = moe._lib.moe_grouped_swiglu_ffn_fp8(ctypes.byref(f8), 16, *([None] * 15), ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+    # the fused quantise-and-permute: FP8 configs with H <= 8192 only
+    st = moe._lib.moe_permute_quantize_fp8(ctypes.byref(bf), None, None, 0, 64, None, None, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    big = moe.make_config(64, 8320, 8, 2, 128, 2, ffn_fp8=True)
+    st = moe._lib.moe_permute_quantize_fp8(ctypes.byref(big), None, None, 0, 64, None, None, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    # the forward entries need the weights' scales in FP8
+    for fn in (moe._lib.moe_forward_chunked, moe._lib.moe_forward_host):
+        p = ctypes.c_void_p(512)
+        st = fn(ctypes.byref(f8), p, None, p, p, p, None, None, None, None, p, p, p, p, None, ws,
+                None, None)
+        assert st == moe.MOE_ERR_INVALID_ARG and "scale" in moe.last_error_detail()
+
+
+def test_forward_workspace_sizes():
+    bf = moe.make_config(4096, 2048, 128, 8, 768, 2)
+    f8 = moe.make_config(4096, 2048, 128, 8, 768, 2, ffn_fp8=True)
+    # FP8 receive rows take one byte per value instead of two; h's codes and scales are added
+    assert moe.forward_workspace_bytes(f8) < moe.forward_workspace_bytes(bf)
+    # the host-buffer form adds staging for logits, bias, x and out
+    extra = moe.forward_host_workspace_bytes(bf) - moe.forward_workspace_bytes(bf)
+    assert extra >= 4 * 4096 * 128 + 4 * 128 + 2 * 2 * 4096 * 2048
+    assert extra < 4 * 4096 * 128 + 4 * 128 + 2 * 2 * 4096 * 2048 + 4 * 256
