@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.orc_ffn_row_bwd.restype = None
         L.orc_layer_bwd.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_layer_bwd.restype = None
+        L.orc_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, P]
+        L.orc_combine_bwd.restype = None
+        L.orc_route_bwd.argtypes = [i, i, i, P, P, P, P]
+        L.orc_route_bwd.restype = None
         _lib = L
     return _lib
 
@@ -331,6 +335,36 @@ def ffn_row_backward(x_row, w13_e, w2_e, dy):
     lib().orc_ffn_row_bwd(H, I, dt, _p(x_row), _p(w13_e), _p(w2_e), _p(dy), _p(dx), _p(dW13),
                           _p(dW2), _p(y))
     return dx, dW13, dW2, y
+
+
+def combine_backward(dout, y, pos, topk_w, tok_begin: int = 0):
+    """Backward of the combine for the chunk's tokens: (dy [N, H] in y's storage
+    type, zero on rows no slot points to; dw [T, k] float64, zero outside the chunk
+    and for dropped slots)."""
+    dout = np.ascontiguousarray(dout)
+    y = np.ascontiguousarray(y)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    dt = _dtype_code(y)
+    assert _dtype_code(dout) == dt
+    tok_count, k = pos.shape
+    H = y.shape[1]
+    dy = np.zeros_like(y)
+    dw = np.zeros(topk_w.shape, np.float64)
+    lib().orc_combine_bwd(H, k, dt, tok_begin, tok_count, _p(dout), _p(y), _p(pos), _p(topk_w),
+                          _p(dy), _p(dw))
+    return dy, dw
+
+
+def route_backward(topk_idx, topk_w, dw, E: int):
+    """dlogits [T, E] (float64) from dw [T, k] through the softmax over the selected."""
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    topk_w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    dw = np.ascontiguousarray(dw, dtype=np.float64)
+    T, k = topk_idx.shape
+    dl = np.zeros((T, E), np.float64)
+    lib().orc_route_bwd(T, E, k, _p(topk_idx), _p(topk_w), _p(dw), _p(dl))
+    return dl
 
 
 def moe_layer_backward(logits, bias, x, w13, w2, k: int, ep: int, dout, capacity: int = -1,

@@ -690,3 +690,44 @@ void orc_layer_bwd(int T, int H, int E, int k, int I, int dtype, const int32_t *
     free(y);
     free(dw);
 }
+
+/* Backward of step 6 for tokens [tok_begin, tok_begin + tok_count): for each
+ * kept slot (pos >= 0) dy[p] = w[t,j] dout[t] (rounded once to the storage
+ * type) and dw[t,j] = sum_c dout[t,c] y[p,c] (double, y as stored); dw of a
+ * dropped slot is 0.  dout [T, H], y / dy [N, H], dw [T, k]. */
+void orc_combine_bwd(int H, int k, int dtype, int tok_begin, int tok_count, const void *dout,
+                     const void *y, const int32_t *pos, const float *topk_w, void *dy, double *dw)
+{
+    for (int i = 0; i < tok_count; ++i) {
+        int t = tok_begin + i;
+        for (int j = 0; j < k; ++j) {
+            int p = pos[(size_t)i * k + j];
+            double acc = 0.0;
+            if (p >= 0) {
+                double w = (double)topk_w[(size_t)t * k + j];
+                for (int c = 0; c < H; ++c) {
+                    double d = orc_load(dout, (size_t)t * H + c, dtype);
+                    orc_store(dy, (size_t)p * H + c, dtype, w * d);
+                    acc += d * orc_load(y, (size_t)p * H + c, dtype);
+                }
+            }
+            dw[(size_t)t * k + j] = acc;
+        }
+    }
+}
+
+/* Backward of step 1 (reading: the softmax over the k selected logits):
+ * dz[t,j] = w[t,j] (dw[t,j] - sum_i w[t,i] dw[t,i]); dlogits [T, E] is dz at
+ * the selected experts and 0 elsewhere. */
+void orc_route_bwd(int T, int E, int k, const int32_t *topk_idx, const float *topk_w,
+                   const double *dw, double *dlogits)
+{
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) dlogits[(size_t)t * E + e] = 0.0;
+        double sw = 0.0;
+        for (int j = 0; j < k; ++j) sw += (double)topk_w[(size_t)t * k + j] * dw[(size_t)t * k + j];
+        for (int j = 0; j < k; ++j)
+            dlogits[(size_t)t * E + topk_idx[(size_t)t * k + j]] =
+                (double)topk_w[(size_t)t * k + j] * (dw[(size_t)t * k + j] - sw);
+    }
+}

@@ -149,3 +149,34 @@ def test_backward_save_dispatch_equals_recompute(dtype):
     for key in ("dx", "dlogits", "dW13", "dW2"):
         np.testing.assert_array_equal(a[key], b[key])
     assert not a["keep"].all()
+
+
+def test_backward_steps_compose_to_the_layer_backward():
+    """The combine's and the routing's backward steps, fed the forward's exact
+    expert rows (fp64 storage), give the layer backward's dlogits (pinned above by
+    finite differences); the rows' backward fed the combine's dy, summed per
+    token with unit weights (the permute's backward), gives its dx."""
+    d = _inputs(8, T=8, E=4)
+    k, ep = 2, 2
+    g = _grad(d, k, ep, capacity=3)
+    fw = oracle.moe_layer(d["logits"], None, d["x"], d["w13"], d["w2"], k, ep, 3)
+    lay = fw["chunks"][0]["layout"]
+    y = fw["chunks"][0]["y"]                      # float64 storage: the exact rows
+    dy, dw = oracle.combine_backward(d["dout"], y, lay["pos"], fw["topk_w"])
+    np.testing.assert_allclose(oracle.route_backward(fw["topk_idx"], fw["topk_w"], dw, 4),
+                               g["dlogits"], rtol=1e-12, atol=1e-14)
+    # dy[p] = w dout[t] for each kept slot
+    for t in range(8):
+        for j in range(k):
+            p = lay["pos"][t, j]
+            if p >= 0:
+                np.testing.assert_array_equal(dy[p], np.float64(fw["topk_w"][t, j]) * d["dout"][t])
+    # the rows' backward, then the permute's backward (the combine with unit weights)
+    n = lay["N"]
+    dxr = np.zeros((n, 8))
+    eoff = lay["expert_offsets"]
+    for e in range(4):
+        for p in range(int(eoff[e]), int(eoff[e + 1])):
+            dxr[p] = oracle.ffn_row_backward(d["x"][lay["recv_token"][p]], d["w13"][e], d["w2"][e], dy[p])[0]
+    dx = oracle.combine(dxr, lay["pos"], np.ones((8, k), np.float32), 8)
+    np.testing.assert_allclose(dx, g["dx"], rtol=1e-12, atol=1e-14)
