@@ -46,6 +46,12 @@ cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in,
                               uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms);
 cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32_t *pos, int tb,
                                  int tc, uint8_t *xr_q, uint8_t *x_scale, cudaStream_t s);
+cudaError_t launch_combine_bwd(const moe_config &c, const void *dout, const void *y,
+                               const int32_t *pos, const float *topk_w, int tb, int tc, void *dy,
+                               float *dw, cudaStream_t s);
+cudaError_t launch_route_bwd(const moe_config &c, const int32_t *topk_idx, const float *topk_w,
+                             const float *dw, float *dlogits, float *dbias, uint32_t *status,
+                             cudaStream_t s);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -521,6 +527,51 @@ moe_status moe_combine(const moe_config *cfg, const void *y, const int32_t *pos,
         return fail(MOE_ERR_INVALID_ARG, "y / y_shared / out not 16-byte aligned");
     cudaError_t err = launch_combine(c, y, pos, topk_w, tok_begin, tok_count, y_shared, out, stream);
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine");
+}
+
+moe_status moe_combine_backward(const moe_config *cfg, const void *dout, const void *y,
+                                const int32_t *pos, const float *topk_w, int32_t tok_begin,
+                                int32_t tok_count, void *dy, float *dw, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.reduce_dense)
+        return fail(MOE_ERR_UNSUPPORTED, "decode form: the expert rows y are not stored");
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!dout || !y || !pos || !topk_w || !dy || !dw))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(dout, 16) || !aligned(y, 16) || !aligned(dy, 16))
+        return fail(MOE_ERR_INVALID_ARG, "dout / y / dy not 16-byte aligned");
+    cudaError_t err = launch_combine_bwd(c, dout, y, pos, topk_w, tok_begin, tok_count, dy, dw, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_combine_backward");
+}
+
+moe_status moe_route_backward(const moe_config *cfg, const int32_t *topk_idx, const float *topk_w,
+                              const float *dw, float *dlogits, float *dbias, void *ws,
+                              cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.T > 0 && (!topk_idx || !topk_w || !dw || !dlogits))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_route_bwd(c, topk_idx, topk_w, dw, dlogits, dbias,
+                                       ws_at<uint32_t>(ws, L.status), stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route_backward");
+}
+
+moe_status moe_permute_backward(const moe_config *cfg, const void *dxr, const int32_t *pos,
+                                int32_t tok_begin, int32_t tok_count, void *dx, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!dxr || !pos || !dx)) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(dxr, 16) || !aligned(dx, 16)) return fail(MOE_ERR_INVALID_ARG, "dxr / dx not 16-byte aligned");
+    // the combine with unit weights: dx[t] = sum of the token's kept receive rows
+    cudaError_t err = launch_combine(c, dxr, pos, nullptr, tok_begin, tok_count, nullptr, dx, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute_backward");
 }
 
 moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,

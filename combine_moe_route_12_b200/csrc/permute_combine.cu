@@ -31,14 +31,15 @@ static int tok_per_cta(int tc) {
     return t < 1 ? 1 : (t > kTokPerCta ? kTokPerCta : t);
 }
 
-// pos (and topk_w) of the CTA's tokens [i0, i0 + n) into shared memory.
+// pos (and topk_w; unit weights when it is NULL, the permute's backward) of the
+// CTA's tokens [i0, i0 + n) into shared memory.
 __device__ __forceinline__ void load_slots(int tb, int i0, int n, int k, const int32_t *pos,
                                            const float *topk_w, int32_t (*s_pos)[kMaxTopK],
                                            float (*s_w)[kMaxTopK]) {
     const int a = threadIdx.x / k, j = threadIdx.x - a * k;
     if (a < n) {
         s_pos[a][j] = pos[(size_t)(i0 + a) * k + j];
-        if (s_w) s_w[a][j] = topk_w[(size_t)(tb + i0 + a) * k + j];
+        if (s_w) s_w[a][j] = topk_w ? topk_w[(size_t)(tb + i0 + a) * k + j] : 1.0f;
     }
 }
 

@@ -74,6 +74,9 @@ _decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
 _decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
 _decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
 _decl("moe_permute_quantize_fp8", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_combine_backward", _I32, _CFG, _P, _P, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_route_backward", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
+_decl("moe_permute_backward", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
 _decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
@@ -227,6 +230,25 @@ def moe_permute_quantize_fp8(cfg, x, pos, tok_begin, tok_count, xr_q, x_scale, s
     """Kept token rows of x quantised to E4M3 codes and written to their receive rows."""
     _check(_lib.moe_permute_quantize_fp8(ctypes.byref(cfg), _ptr(x), _ptr(pos), tok_begin,
                                          tok_count, _ptr(xr_q), _ptr(x_scale), _stream(stream)))
+
+
+def moe_combine_backward(cfg, dout, y, pos, topk_w, tok_begin, tok_count, dy, dw, stream=None):
+    """dy[pos] = w * dout and dw = <dout, y[pos]> for the chunk's kept slots."""
+    _check(_lib.moe_combine_backward(ctypes.byref(cfg), _ptr(dout), _ptr(y), _ptr(pos),
+                                     _ptr(topk_w), tok_begin, tok_count, _ptr(dy), _ptr(dw),
+                                     _stream(stream)))
+
+
+def moe_route_backward(cfg, topk_idx, topk_w, dw, dlogits, dbias, ws, stream=None):
+    """dlogits through the softmax over the selected logits; dbias its column sums."""
+    _check(_lib.moe_route_backward(ctypes.byref(cfg), _ptr(topk_idx), _ptr(topk_w), _ptr(dw),
+                                   _ptr(dlogits), _ptr(dbias), _ptr(ws), _stream(stream)))
+
+
+def moe_permute_backward(cfg, dxr, pos, tok_begin, tok_count, dx, stream=None):
+    """dx[t] = the sum of the token's kept receive rows of dxr."""
+    _check(_lib.moe_permute_backward(ctypes.byref(cfg), _ptr(dxr), _ptr(pos), tok_begin,
+                                     tok_count, _ptr(dx), _stream(stream)))
 
 
 def moe_grouped_swiglu_ffn_fp8(cfg, n_rows, xr_q, x_scale, expert_offsets, w13_q, w13_scale, w2_q,

@@ -21,8 +21,9 @@
  * fixed library array; moe_quantize_fp8_rows, moe_permute_quantize_fp8 and
  * moe_grouped_swiglu_ffn_fp8, the expert FFN on E4M3 codes with UE8M0 row
  * scales (cfg->ffn_fp8);
- * moe_watchdog_selftest, which makes a bounded wait run out on purpose;
- * moe_device_status, the device-side error bits.
+ * moe_combine_backward, moe_route_backward and moe_permute_backward, the
+ * backward's row passes; moe_watchdog_selftest, which makes a bounded wait run
+ * out on purpose; moe_device_status, the device-side error bits.
  *
  * Sources (restated, not copied):
  *   [AX]  axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
@@ -385,6 +386,40 @@ moe_status moe_reduce_finalize(const moe_config *cfg, const float *out_reduce,
 moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32_t tok_count,
                                  const void *x, const void *w13_shared, const void *w2_shared,
                                  void *h_shared, void *y_shared, void *ws, cudaStream_t stream);
+
+/*
+ * Backward steps that are row passes (axolotl ExpertParallelArgs,
+ * expert_parallel_save_dispatch: the layer's backward reuses the saved routing
+ * top-k, keep mask and layout; the expert FFN's backward is not part of this
+ * library yet).  For L = <dout, out>:
+ *
+ * moe_combine_backward, for t in [tok_begin, tok_begin + tok_count):
+ *   dy[pos[t - tok_begin, j]] = topk_w[t, j] * dout[t]     (cfg->dtype, rounded once)
+ *   dw[t, j] = <dout[t], y[pos[t - tok_begin, j]]>         (fp32; 0 for a dropped slot)
+ *   dout [T, H] and y, dy [N_max, H] in cfg->dtype; dw [T, k]; receive rows no slot
+ *   points to are left untouched.  Not for the decode form (y is not stored).
+ *
+ * moe_route_backward, for every token (the softmax over the k selected logits):
+ *   dlogits[t, :] = 0 except dlogits[t, topk_idx[t, j]] = topk_w[t, j] *
+ *                   (dw[t, j] - sum_i topk_w[t, i] dw[t, i])     (fp32 [T, E])
+ *   dbias (optional, fp32 [E]) = sum over t of dlogits[t, :] in a fixed order,
+ *                   or 0 when cfg->bias_select_only.
+ *   ws: moe_workspace_bytes(cfg) (an expert id outside [0, E) sets
+ *   MOE_DEV_BAD_INDEX and is not written).
+ *
+ * moe_permute_backward, for t in [tok_begin, tok_begin + tok_count):
+ *   dx[t] = sum over kept slots j of dxr[pos[t - tok_begin, j]], fp32 in slot
+ *   order, rounded once to cfg->dtype (zeros for a token with every slot
+ *   dropped); dxr [N_max, H], dx [T, H].
+ */
+moe_status moe_combine_backward(const moe_config *cfg, const void *dout, const void *y,
+                                const int32_t *pos, const float *topk_w, int32_t tok_begin,
+                                int32_t tok_count, void *dy, float *dw, cudaStream_t stream);
+moe_status moe_route_backward(const moe_config *cfg, const int32_t *topk_idx, const float *topk_w,
+                              const float *dw, float *dlogits, float *dbias, void *ws,
+                              cudaStream_t stream);
+moe_status moe_permute_backward(const moe_config *cfg, const void *dxr, const int32_t *pos,
+                                int32_t tok_begin, int32_t tok_count, void *dx, cudaStream_t stream);
 
 /*
  * The whole layer, chunked ([AX] expert_parallel_dispatch_chunks; [LL]
