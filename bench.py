@@ -72,6 +72,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    p.add_argument("--backward", action="store_true",
+                   help="also time the backward's row passes (combine, routing, permute) on the "
+                        "last chunk and add a backward_row_passes object to the line")
     p.add_argument("--seed", type=int, default=None)
     p.add_argument("--no-graph", action="store_true",
                    help="time eager launches instead of replaying a captured CUDA graph of the layer")
@@ -336,6 +339,56 @@ def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
         else:
             moe.moe_combine(cfg, B.y, B.pos, B.topk_w, tb, B.tc, B.out, y_shared=B.ys)
         rec(base + 4)
+
+
+def backward_row_passes(moe, wl, cfg, B, n_rows, peaks, flush, args):
+    """Times the backward's row passes on the last chunk's layout (B holds it after
+    the breakdown pass): the combine's backward against the forward's y rows, the
+    permute's backward of synthetic receive-row gradients, and the routing's
+    backward of the resulting dw over all T tokens.  HBM bytes per pass: combine
+    tc·H·b (dout) + 2·N·H·b (y read, dy written) + 4·tc·k (dw); permute N·H·b +
+    tc·H·b; routing 4·T·E written (+ 12·T·k read)."""
+    import torch
+    dev = B.xr.device
+    T, H, k, E, tc = wl.T, wl.H, wl.k, wl.E, B.tc
+    tb = (wl.n_chunks - 1) * tc
+    b = wl.elem_bytes
+    g = torch.Generator(device=dev).manual_seed(17)
+    dout = torch.randn(T, H, generator=g, device=dev).to(wl.torch_dtype)
+    dxr = torch.randn(max(B.nmax, 1), H, generator=g, device=dev).to(wl.torch_dtype)
+    dy = torch.empty(max(B.nmax, 1), H, dtype=wl.torch_dtype, device=dev)
+    dx = torch.empty(T, H, dtype=wl.torch_dtype, device=dev)
+    dw = torch.zeros(T, k, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    db = torch.empty(E, dtype=torch.float32, device=dev)
+    t = {"combine": 0.0, "permute": 0.0, "route": 0.0}
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record()
+        moe.moe_combine_backward(cfg, dout, B.y, B.pos, B.topk_w, tb, tc, dy, dw)
+        ev[1].record()
+        moe.moe_permute_backward(cfg, dxr, B.pos, tb, tc, dx)
+        ev[2].record()
+        moe.moe_route_backward(cfg, B.topk_idx, B.topk_w, dw, dl, db, B.ws)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            for j, name in enumerate(("combine", "permute", "route")):
+                t[name] += ev[j].elapsed_time(ev[j + 1]) / args.steps
+    if moe.moe_device_status(B.ws) != 0:
+        raise RuntimeError("device status bits set during the backward passes")
+    cb = tc * H * b + 2 * n_rows * H * b + 4 * tc * k
+    pb = n_rows * H * b + tc * H * b
+    rb = 4 * T * E + 12 * T * k
+    gbs = lambda by, ms: by / (ms * 1e-3) / 1e9 if ms > 0 else None
+    return {"chunk_tokens": tc, "rows": n_rows,
+            "combine_bwd": {"ms": round(t["combine"], 4), "gbs": gbs(cb, t["combine"]),
+                            "frac": gbs(cb, t["combine"]) / peaks["hbm_gbs"] if t["combine"] > 0 else None},
+            "permute_bwd": {"ms": round(t["permute"], 4), "gbs": gbs(pb, t["permute"]),
+                            "frac": gbs(pb, t["permute"]) / peaks["hbm_gbs"] if t["permute"] > 0 else None},
+            "route_bwd": {"ms": round(t["route"], 4), "gbs": gbs(rb, t["route"])},
+            "timing": "CUDA events around each eager launch, L2 flushed before each pass triple"}
 
 
 def stage_times(wl, ev):
@@ -617,6 +670,8 @@ def run_ours(args):
         n_active.append(int(((B.eoff[1:] - B.eoff[:-1]) > 0).sum().item()))
     tokens_read = int((B.keep.view(wl.T, wl.k) != 0).any(dim=1).sum().item())
     alg = algorithmic(wl, n_kept, n_active, tokens_read)
+    bwd = backward_row_passes(moe, wl, cfg, B, n_kept[-1], peaks, flush, args) \
+        if args.backward and not wl.reduce_dense else None
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -720,6 +775,8 @@ def run_ours(args):
             "gpu_launches": kernels_per_step(wl) * args.steps,
             "clocks": clocks,
         }
+        if bwd is not None:
+            line["backward_row_passes"] = bwd
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
