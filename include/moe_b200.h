@@ -239,7 +239,7 @@ moe_status moe_dispatch_layout(const moe_config *cfg, int32_t tok_begin, int32_t
  * captures the stream into a CUDA graph, code whose device memory belongs to
  * an allocator it cannot grow, and latency-critical loops that must avoid the
  * implicit synchronisation of cudaMalloc / cudaFree.  The pages describe no
- * such variant: the paper has no counterpart of this entry point.
+ * such variant; this entry point has no counterpart on them.
  *   Arguments and outputs are those of moe_dispatch_layout, without ws.
  *   status: device uint32 that receives the MOE_DEV_* bits (OR-ed in), or
  *           NULL to drop them.
