@@ -337,6 +337,27 @@ def ffn_row_backward(x_row, w13_e, w2_e, dy):
     return dx, dW13, dW2, y
 
 
+def ffn_backward(xr, expert_offsets, w13, w2, dy):
+    """The grouped SwiGLU FFN's backward over an expert-contiguous receive buffer:
+    for every row p of expert e, the row backward of orc_ffn_row_bwd with dy[p].
+    Returns float64 (dxr [N, H], dW13 [E, 2I, H], dW2 [E, H, I])."""
+    xr = np.ascontiguousarray(xr)
+    dy = np.ascontiguousarray(dy, np.float64)
+    N, H = xr.shape
+    E = w13.shape[0]
+    I = w13.shape[1] // 2
+    dxr = np.zeros((N, H), np.float64)
+    dW13 = np.zeros((E, 2 * I, H), np.float64)
+    dW2 = np.zeros((E, H, I), np.float64)
+    for e in range(E):
+        for p in range(int(expert_offsets[e]), int(expert_offsets[e + 1])):
+            dx, a, b, _ = ffn_row_backward(xr[p], w13[e], w2[e], dy[p])
+            dxr[p] = dx
+            dW13[e] += a
+            dW2[e] += b
+    return dxr, dW13, dW2
+
+
 def combine_backward(dout, y, pos, topk_w, tok_begin: int = 0):
     """Backward of the combine for the chunk's tokens: (dy [N, H] in y's storage
     type, zero on rows no slot points to; dw [T, k] float64, zero outside the chunk

@@ -180,3 +180,26 @@ def test_backward_steps_compose_to_the_layer_backward():
             dxr[p] = oracle.ffn_row_backward(d["x"][lay["recv_token"][p]], d["w13"][e], d["w2"][e], dy[p])[0]
     dx = oracle.combine(dxr, lay["pos"], np.ones((8, k), np.float32), 8)
     np.testing.assert_allclose(dx, g["dx"], rtol=1e-12, atol=1e-14)
+
+
+def test_grouped_ffn_backward_step_composes_with_the_row_passes():
+    """combine backward -> grouped FFN backward over the receive buffer -> permute
+    backward gives the layer backward's dx, dW13 and dW2 (two chunks)."""
+    d = _inputs(9, T=8, E=4)
+    k, ep = 2, 2
+    g = oracle.moe_layer_backward(d["logits"], None, d["x"], d["w13"], d["w2"], k, ep, d["dout"],
+                                  capacity=3, n_chunks=2)
+    fw = oracle.moe_layer(d["logits"], None, d["x"], d["w13"], d["w2"], k, ep, 3, n_chunks=2)
+    dx = np.zeros_like(d["x"])
+    dW13 = np.zeros_like(g["dW13"])
+    dW2 = np.zeros_like(g["dW2"])
+    for c, ch in enumerate(fw["chunks"]):
+        lay = ch["layout"]
+        dy, _ = oracle.combine_backward(d["dout"], ch["y"], lay["pos"], fw["topk_w"], c * 4)
+        dxr, a, b = oracle.ffn_backward(ch["xr"], lay["expert_offsets"], d["w13"], d["w2"], dy)
+        dW13 += a
+        dW2 += b
+        oracle.combine(dxr, lay["pos"], np.ones((8, k), np.float32), 8, c * 4, dx)
+    np.testing.assert_allclose(dx, g["dx"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dW13, g["dW13"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dW2, g["dW2"], rtol=1e-12, atol=1e-14)
