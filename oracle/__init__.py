@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.orc_ffn_row_bwd.restype = None
         L.orc_layer_bwd.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_layer_bwd.restype = None
+        L.orc_quantize_blocks.argtypes = [ctypes.c_int64, i, i, i, P, P, P]
+        L.orc_quantize_blocks.restype = None
+        L.orc_dot_blocked.argtypes = [i, i, P, P, P, P]
+        L.orc_dot_blocked.restype = ctypes.c_double
         L.orc_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, P]
         L.orc_combine_bwd.restype = None
         L.orc_route_bwd.argtypes = [i, i, i, P, P, P, P]
@@ -288,6 +292,29 @@ def quantize_rows(a: np.ndarray):
     scales = np.zeros(rows, np.uint8)
     lib().orc_quantize_rows(rows, cols, dt, _p(a), _p(codes), _p(scales))
     return codes, scales
+
+
+def quantize_blocks(a: np.ndarray, block: int = 128):
+    """FP8 quantisation with one UE8M0 scale per row and per block of `block`
+    columns.  Returns (codes uint8 [rows, cols], scales uint8 [rows, ceil(cols/block)])."""
+    a = np.ascontiguousarray(a)
+    dt = _dtype_code(a)
+    rows, cols = a.shape
+    nb = (cols + block - 1) // block
+    codes = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros((rows, nb), np.uint8)
+    lib().orc_quantize_blocks(rows, cols, block, dt, _p(a), _p(codes), _p(scales))
+    return codes, scales
+
+
+def dot_blocked(a_codes, a_scales, b_codes, b_scales, block: int = 128) -> float:
+    """<dequant(a), dequant(b)> for two K-blocked FP8 rows, block by block."""
+    a_codes = np.ascontiguousarray(a_codes, np.uint8)
+    b_codes = np.ascontiguousarray(b_codes, np.uint8)
+    a_scales = np.ascontiguousarray(a_scales, np.uint8)
+    b_scales = np.ascontiguousarray(b_scales, np.uint8)
+    return float(lib().orc_dot_blocked(a_codes.shape[0], block, _p(a_codes), _p(a_scales),
+                                       _p(b_codes), _p(b_scales)))
 
 
 def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:

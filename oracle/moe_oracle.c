@@ -731,3 +731,45 @@ void orc_route_bwd(int T, int E, int k, const int32_t *topk_idx, const float *to
                 (double)topk_w[(size_t)t * k + j] * (dw[(size_t)t * k + j] - sw);
     }
 }
+
+/* FP8 with K-blocked scales (the finer granularity of the FP8 grouped GEMM on
+ * the LightLLM PR 1687 page, DeepGEMM's UE8M0 layout): one UE8M0 scale per row
+ * and per block of `block` columns, chosen and applied as orc_quantize_rows does
+ * for a whole row.  scales is [rows, ceil(cols / block)]. */
+void orc_quantize_blocks(int64_t rows, int cols, int block, int dtype, const void *in,
+                         uint8_t *codes, uint8_t *scales)
+{
+    const int nb = (cols + block - 1) / block;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int b = 0; b < nb; ++b) {
+            const int c0 = b * block, c1 = c0 + block < cols ? c0 + block : cols;
+            double amax = 0.0;
+            for (int c = c0; c < c1; ++c) {
+                double a = fabs(orc_load(in, (size_t)r * cols + c, dtype));
+                if (a > amax) amax = a;
+            }
+            uint8_t s = orc_ue8m0_scale(amax);
+            scales[(size_t)r * nb + b] = s;
+            for (int c = c0; c < c1; ++c)
+                codes[(size_t)r * cols + c] =
+                    orc_e4m3_encode(ldexp(orc_load(in, (size_t)r * cols + c, dtype), 127 - (int)s));
+        }
+}
+
+/* Dot product of two K-blocked FP8 rows of length K (same block size): the sum
+ * over blocks of 2^(sa + sb - 254) times the sum of the blocks' decoded code
+ * products, in double (each block's partial sum is exact in double for
+ * E4M3 operands and block <= 2^20). */
+double orc_dot_blocked(int K, int block, const uint8_t *a, const uint8_t *sa, const uint8_t *b,
+                       const uint8_t *sb)
+{
+    const int nb = (K + block - 1) / block;
+    double acc = 0.0;
+    for (int q = 0; q < nb; ++q) {
+        double part = 0.0;
+        for (int c = q * block; c < K && c < (q + 1) * block; ++c)
+            part += orc_e4m3_decode(a[c]) * orc_e4m3_decode(b[c]);
+        acc += ldexp(part, (int)sa[q] + (int)sb[q] - 254);
+    }
+    return acc;
+}

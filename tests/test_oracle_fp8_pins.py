@@ -169,3 +169,41 @@ def test_ffn_row_fp8_weight_row_scale_is_a_power_of_two_per_row():
     _, _, _, _, ye2 = oracle.ffn_row_fp8(x, sx, w13, w13_s, w2, w2_s2)
     assert ye2[5] == 8 * ye[5]
     np.testing.assert_array_equal(np.delete(ye2, 5), np.delete(ye, 5))
+
+
+def test_quantize_blocks_reduces_to_rows_and_is_exact_per_block():
+    rng = np.random.default_rng(9)
+    a = (rng.normal(0, 1, (16, 384)) * np.ldexp(1.0, rng.integers(-20, 20, (16, 1)))).astype(np.float32)
+    a[:, 128:256] *= 1e-3                       # a quiet middle block takes its own scale
+    # one block spanning the row is the row quantisation
+    c_row, s_row = oracle.quantize_rows(a)
+    c1, s1 = oracle.quantize_blocks(a, 384)
+    np.testing.assert_array_equal(c1, c_row)
+    np.testing.assert_array_equal(s1[:, 0], s_row)
+    # each 128-column block is the row quantisation of that block alone
+    c, s = oracle.quantize_blocks(a, 128)
+    for b in range(3):
+        cb, sb = oracle.quantize_rows(np.ascontiguousarray(a[:, 128 * b:128 * (b + 1)]))
+        np.testing.assert_array_equal(c[:, 128 * b:128 * (b + 1)], cb)
+        np.testing.assert_array_equal(s[:, b], sb)
+    assert (s[:, 1] < s[:, 0]).all()            # the quiet block's scale is smaller
+    # a ragged last block
+    c, s = oracle.quantize_blocks(a[:, :300].copy(), 128)
+    assert s.shape == (16, 3)
+    cb, sb = oracle.quantize_rows(np.ascontiguousarray(a[:, 256:300]))
+    np.testing.assert_array_equal(c[:, 256:300], cb)
+    np.testing.assert_array_equal(s[:, 2], sb)
+
+
+def test_dot_blocked_equals_library_dequantised_dot():
+    rng = np.random.default_rng(10)
+    K = 512
+    a = rng.normal(0, 1, (4, K)).astype(np.float32)
+    b = (rng.normal(0, 1, (4, K)) * 50).astype(np.float32)
+    ca, sa = oracle.quantize_blocks(a, 128)
+    cb, sb = oracle.quantize_blocks(b, 128)
+    for r in range(4):
+        deq = lambda c, s: _torch_decode(c) * np.repeat(np.ldexp(1.0, s.astype(np.int32) - 127), 128)
+        ref = float(np.dot(deq(ca[r], sa[r]), deq(cb[r], sb[r])))
+        got = oracle.dot_blocked(ca[r], sa[r], cb[r], sb[r], 128)
+        assert abs(got - ref) <= 1e-12 * max(1.0, abs(ref))
