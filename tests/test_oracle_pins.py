@@ -503,6 +503,127 @@ def test_combine_special_cases():
     np.testing.assert_array_equal(out, y[:T])
 
 
+def _bit_coded_rows(N, H, k):
+    """Receive rows whose every entry is a distinct power of two per (row, slot):
+    y[p, c] = (c + 1) * 2^(-k*p) and slot weights w_j = 2^-(j+1), so the term
+    w_j * y[p] = (c + 1) * 2^-(j + 1 + k*p) lands on its own bit and an exact
+    fp64 sum tells which (slot, row) pairs were added."""
+    y = np.empty((N, H), np.float64)
+    for p in range(N):
+        y[p] = np.arange(1, H + 1) * 2.0 ** (-k * p)
+    return y
+
+
+def _decode_bits(v, k, N):
+    """Inverse of the coding above for column 0 (c + 1 = 1): the set of (slot, row)
+    pairs whose term is present in v (exact fp64)."""
+    pairs = set()
+    for j in range(k):
+        for p in range(N):
+            if math.ldexp(1.0, -(j + 1 + k * p)) <= v and \
+                    int(math.ldexp(v, j + 1 + k * p)) & 1:
+                pairs.add((j, p))
+    return pairs
+
+
+@pytest.mark.parametrize("tok_begin", [0, 4])
+def test_combine_exact_sums_exactly_the_kept_slots(tok_begin):
+    """Decode form of the combine (LightLLM PR 1687: the decode path reduces expert
+    outputs straight into a dense output).  With bit-coded rows and power-of-two
+    weights every (slot, row) term of a token's sum sits on its own bit, so the
+    exact fp64 output names the rows and slots that were added: it must be exactly
+    {(j, pos[i, j]) : pos[i, j] >= 0} for token tok_begin + i, read with the weights
+    of that absolute token row.  A dropped term, a wrong slot weight, pos read
+    against the wrong base or the chunk written to the wrong rows changes the bits."""
+    k, H, tc, T = 2, 3, 4, 8
+    rng = np.random.default_rng(41)
+    N = 7
+    y = _bit_coded_rows(N, H, k)
+    # pos: a permutation of the rows over the chunk's slots, some slots dropped
+    slots = rng.permutation(tc * k)[:N]
+    pos = np.full(tc * k, -1, np.int32)
+    pos[slots] = np.arange(N, dtype=np.int32)
+    pos = pos.reshape(tc, k)
+    w = np.zeros((T, k), np.float32)
+    for j in range(k):
+        w[tok_begin:tok_begin + tc, j] = 2.0 ** -(j + 1)
+    w[:tok_begin] = 7.0               # other chunks' weights must not be read
+    w[tok_begin + tc:] = 7.0
+    out = np.full((T, H), -1.0, np.float64)
+    oracle.combine_exact(y, pos, w, T, np.float64, tok_begin, out)
+    for i in range(tc):
+        want = {(j, int(pos[i, j])) for j in range(k) if pos[i, j] >= 0}
+        got = _decode_bits(out[tok_begin + i, 0], k, N)
+        assert got == want, (i, got, want)
+        for c in range(H):              # column c is column 0 times (c + 1), exactly
+            assert out[tok_begin + i, c] == (c + 1) * out[tok_begin + i, 0]
+    # rows outside the chunk are untouched
+    assert (np.delete(out, range(tok_begin, tok_begin + tc), axis=0) == -1.0).all()
+
+
+def test_combine_exact_adds_the_shared_rows_by_chunk_row():
+    """The shared expert's rows are indexed by chunk-relative row: row i belongs to
+    token tok_begin + i, on bits far below every routed term."""
+    k, H, tc, T, tb = 2, 2, 3, 6, 3
+    y = _bit_coded_rows(4, H, k)
+    pos = np.array([[0, -1], [-1, -1], [1, 2]], np.int32)
+    w = np.zeros((T, k), np.float32)
+    w[tb:, 0], w[tb:, 1] = 0.5, 0.25
+    ys = np.array([[(i + 1) * 2.0 ** -40] * H for i in range(tc)])
+    out = np.zeros((T, H), np.float64)
+    oracle.combine_exact(y, pos, w, T, np.float64, tb, out, y_shared=ys)
+    expect = [0.5 * y[0, 0] + 1 * 2.0 ** -40, 2 * 2.0 ** -40, 0.5 * y[1, 0] + 0.25 * y[2, 0] + 3 * 2.0 ** -40]
+    assert out[tb:, 0].tolist() == expect
+    assert (out[:tb] == 0).all()
+
+
+def test_combine_exact_rounds_once_and_matches_the_stored_form_at_k1():
+    """With one slot of weight 1 the decode form's single rounding of w * y_exact is
+    the rounding of y_exact, which is what the stored form combines: the two give
+    the same bits (fp32 and bf16).  And a token with every slot dropped gets 0."""
+    rng = np.random.default_rng(42)
+    N, H, T = 5, 6, 6
+    ye = rng.standard_normal((N, H)) * 3
+    pos = np.array([[0], [1], [-1], [2], [3], [4]], np.int32)
+    w = np.ones((T, 1), np.float32)
+    for dt, rnd in ((np.float32, lambda a: a.astype(np.float32)),
+                    (np.uint16, lambda a: np.array([[oracle.bf16_bits_from_double(v) for v in r] for r in a],
+                                                   np.uint16))):
+        a = oracle.combine_exact(ye, pos, w, T, dt)
+        b = oracle.combine(rnd(ye), pos, w, T)
+        np.testing.assert_array_equal(a, b)
+        assert (a[2] == 0).all()
+
+
+@pytest.mark.parametrize("capacity,n_chunks", [(-1, 1), (5, 2), (0, 2)])
+def test_decode_layer_equals_dense_sum_of_unrounded_rows(capacity, n_chunks):
+    """The decode-form layer against a per-token dense loop in numpy that keeps y
+    unrounded (h rounded to storage, as the CUDA path stores it): out_t =
+    fp32(sum over kept j of w_j * W2[e_j] h_j), over two chunks with drops."""
+    rng = np.random.default_rng(43)
+    T, H, E, k, I = 24, 16, 6, 2, 12
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w13 = (rng.standard_normal((E, 2 * I, H)) / 4).astype(np.float32)
+    w2 = (rng.standard_normal((E, H, I)) / 4).astype(np.float32)
+    res = oracle.moe_layer(logits, None, x, w13, w2, k, 2, capacity, n_chunks, reduce_dense=True)
+    idx, w, keep = res["topk_idx"], res["topk_w"], res["keep"]
+    ref = np.zeros((T, H))
+    for t in range(T):
+        for j in range(k):
+            if not keep[t, j]:
+                continue
+            e = idx[t, j]
+            xv = x[t].astype(np.float64)
+            g = w13[e, :I].astype(np.float64) @ xv
+            u = w13[e, I:].astype(np.float64) @ xv
+            hh = (g / (1 + np.exp(-g)) * u).astype(np.float32).astype(np.float64)
+            ref[t] += float(w[t, j]) * (w2[e].astype(np.float64) @ hh)
+    np.testing.assert_allclose(res["out"], ref.astype(np.float32), rtol=2e-7, atol=1e-12)
+    if capacity == 0:
+        assert (res["out"] == 0).all()
+
+
 def _dense_reference(logits, bias, x, w13, w2, k, capacity):
     """Per-token dense loop in numpy: out_t = sum_{kept j} w_j * FFN_{e_j}(x_t)."""
     idx, w, _, _ = oracle.route_topk(logits, bias, k)
