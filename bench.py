@@ -6,20 +6,26 @@
 One step = one pass of the whole layer (router top-k, capacity clip, dispatch
 layout, permute, grouped SwiGLU FFN, combine) over one batch of seeded
 synthetic inputs that are resident in HBM.  The default workload is the
-Qwen3-30B-A3B-shaped layer (T=4096, H=2048, E=128, k=8, I=768, bf16, EP=2).
+largest single-GPU configuration, the DeepSeek-V3-shaped prefill layer
+(T=8192, H=7168, E=256, k=8, I=2048, bf16, EP=8 logical ranks, two dispatch
+chunks pipelined on two streams).
 
 Prints one JSON line (rank 0).  Besides the contract keys it reports a
 per-stage breakdown, dispatch+combine HBM GB/s, FFN TFLOP/s, the roofline of
 the dominant kernel (the grouped FFN), an end-to-end number through the
 public API with host buffers, and the CPU oracle timed on a bounded sample.
+For a chunked workload the same line also carries the FFN's roofline with one
+chunk (``roofline_unchunked``: every expert's weights read once per layer pass)
+and ``overlap``: the two-stream step against the same kernels on one stream.
 
 With --gpus N > 1 (launched by torchrun) every rank runs an independent
 replica of the workload (the layer's EP ranks are logical, inside one GPU),
 so there is no data-path collective; the time is the max over ranks and the
 value counts the tokens of all ranks (weak scaling).
 
---impl reference times the CPU oracle (plain C, one core) on a bounded sample
-of the same workload, each step a sample, and prints the same line with
+--impl reference times the CPU oracle (plain C, one core) on the same
+workload, each step the whole layer over a sub-batch of its first tokens (a
+multiple of the logical EP size), and prints the same line with
 "impl": "reference".
 """
 from __future__ import annotations
@@ -56,9 +62,22 @@ FFN_TRAFFIC = {
 
 
 def workload_of(args):
+    """The named workload, with the chunk count, token count or expert count
+    overridden when asked (a smaller case of the same shape, e.g. for a
+    counter capture); an overridden workload carries the changes in its name."""
     from combine_moe_route_12_b200.workload import WORKLOADS
     wl = WORKLOADS[args.config]
-    return wl if args.chunks is None else wl.with_(n_chunks=args.chunks)
+    over = {}
+    if args.chunks is not None:
+        over["n_chunks"] = args.chunks
+    if getattr(args, "tokens", None) is not None:
+        over["T"] = args.tokens
+    if getattr(args, "experts", None) is not None:
+        over["E"] = args.experts
+    if not over:
+        return wl
+    tag = ",".join(f"{k}={v}" for k, v in over.items())
+    return wl.with_(name=f"{wl.name}[{tag}]", **over)
 
 
 def parse_args(argv=None):
@@ -66,12 +85,18 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--config", default="qwen3_30b_a3b")
+    p.add_argument("--config", default="dsv3_prefill")
     p.add_argument("--chunks", type=int, default=None,
                    help="override the workload's dispatch chunk count (e.g. 1 for the unchunked DSV3 prefill FFN)")
+    p.add_argument("--tokens", type=int, default=None, help="override the workload's token count T")
+    p.add_argument("--experts", type=int, default=None, help="override the workload's expert count E")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    p.add_argument("--no-unchunked", action="store_true",
+                   help="skip the one-chunk FFN breakdown of a chunked workload")
+    p.add_argument("--no-overlap", action="store_true",
+                   help="skip the one-stream replay of a chunked workload")
     p.add_argument("--backward", action="store_true",
                    help="also time the backward's row passes (combine, routing, permute) on the "
                         "last chunk and add a backward_row_passes object to the line")
@@ -391,24 +416,138 @@ def backward_row_passes(moe, wl, cfg, B, n_rows, peaks, flush, args):
             "timing": "CUDA events around each eager launch, L2 flushed before each pass triple"}
 
 
-def stage_times(wl, ev):
-    """Per-stage milliseconds of one step recorded by run_steps."""
+def stage_times(wl, ev, per_chunk=False):
+    """Per-stage milliseconds of one step recorded by run_steps (and, with
+    per_chunk, the list of each chunk's dispatch_layout + permute time)."""
     t = {"route_topk": ev[0].elapsed_time(ev[1]), "capacity_clip": ev[1].elapsed_time(ev[2]),
          "dispatch_layout": 0.0, "permute": 0.0, "grouped_ffn": 0.0, "shared_expert": 0.0,
          "combine": 0.0}
+    disp = []
     for c in range(wl.n_chunks):
         b = 3 + 5 * c
         prev = ev[2] if c == 0 else ev[b - 1]
-        t["dispatch_layout"] += prev.elapsed_time(ev[b])
-        t["permute"] += ev[b].elapsed_time(ev[b + 1])
+        lay = prev.elapsed_time(ev[b])
+        per = ev[b].elapsed_time(ev[b + 1])
+        t["dispatch_layout"] += lay
+        t["permute"] += per
         t["grouped_ffn"] += ev[b + 1].elapsed_time(ev[b + 2])
         t["shared_expert"] += ev[b + 2].elapsed_time(ev[b + 3])
         t["combine"] += ev[b + 3].elapsed_time(ev[b + 4])
-    return t
+        disp.append(lay + per)
+    return (t, disp) if per_chunk else t
 
 
 STAGES = ["route_topk", "capacity_clip", "dispatch_layout", "permute", "grouped_ffn",
           "shared_expert", "combine"]
+
+
+def breakdown(moe, wl, cfg, inp, B, fp8, steps, flush, use_graph):
+    """The step ABI on one stream with events between the stages, captured into a
+    CUDA graph with the events (no host launch gaps; eager launches if capture
+    fails), replayed `steps` times with the L2 flushed before each.  Returns
+    (mean stage ms, mean per-chunk dispatch ms, mean step ms, mode)."""
+    import torch
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(n_marks(wl))]
+    for _ in range(2):
+        run_steps(moe, wl, cfg, inp, B, None, fp8)
+    torch.cuda.synchronize()
+    stage_ms = {s: 0.0 for s in STAGES}
+    disp_ms = [0.0] * wl.n_chunks
+    step_sum = 0.0
+    bd_ev = mk()
+    bd_graph = None
+    if use_graph:
+        try:
+            # external events stay timing events inside a captured graph
+            gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks(wl))]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_steps(moe, wl, cfg, inp, B, gev, fp8)
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            stage_times(wl, gev)          # raises if the events cannot be timed
+            bd_graph, bd_ev = g, gev
+        except Exception:
+            bd_graph = None
+            torch.cuda.synchronize()
+    for _ in range(steps):
+        flush.fill_(1)
+        if bd_graph is not None:
+            bd_graph.replay()
+        else:
+            run_steps(moe, wl, cfg, inp, B, bd_ev, fp8)
+        torch.cuda.synchronize()
+        st, dp = stage_times(wl, bd_ev, per_chunk=True)
+        for s_, v in st.items():
+            stage_ms[s_] += v / steps
+        for c, v in enumerate(dp):
+            disp_ms[c] += v / steps
+        step_sum += bd_ev[0].elapsed_time(bd_ev[-1]) / steps
+    if moe.moe_device_status(B.ws) != 0:
+        raise RuntimeError("device status bits set during the breakdown pass")
+    mode = "graph" if bd_graph is not None else "eager"
+    del bd_graph
+    return stage_ms, disp_ms, step_sum, mode
+
+
+def layout_counts(moe, wl, cfg, B):
+    """Kept rows and active experts of each chunk, and the tokens with a kept slot."""
+    n_kept, n_active = [], []
+    for c in range(wl.n_chunks):
+        moe.moe_dispatch_layout(cfg, c * B.tc, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
+                                B.pos, B.spl, None, B.ws)
+        n_kept.append(int(B.eoff[wl.E].item()))
+        n_active.append(int(((B.eoff[1:] - B.eoff[:-1]) > 0).sum().item()))
+    tokens_read = int((B.keep.view(wl.T, wl.k) != 0).any(dim=1).sum().item())
+    return n_kept, n_active, tokens_read
+
+
+def ffn_roofline(wl, alg, ffn_ms, peaks, peak_src, traffic):
+    """The grouped FFN's roofline for one layer pass: its algorithmic bytes and
+    flops over the measured duration, against the binding roof (HBM when the
+    pass's flop per byte is below the ridge).  The tensor fraction is also given
+    against the sustained bf16 figure (a long step runs under the power cap)."""
+    ffn_s = ffn_ms / 1e3
+    f8 = 2.0 if wl.ffn_fp8 else 1.0
+    # the tensor peak of the FFN's operand type: the measured bf16 figure, times
+    # the nominal dense FP8 / bf16 ratio (4.5 / 2.25) for E4M3 operands
+    t_peak = peaks["bf16_tflops"] * f8
+    t_peak_sus = peaks["bf16_tflops_sustained"] * f8
+    t_peak_src = "bf16_tflops (burst) x 2 (nominal e4m3 / bf16)" if wl.ffn_fp8 else "bf16_tflops (burst)"
+    t_flop = alg["ffn_flops"] / (t_peak * 1e12)
+    t_byte = alg["ffn_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    hbm_bound = t_byte > t_flop
+    tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
+    gbs = alg["ffn_bytes"] / ffn_s / 1e9 if ffn_s > 0 else None
+    return {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass"
+                      + (", E4M3 operands, h quantised between them)" if wl.ffn_fp8 else ")"),
+            "bound": "hbm" if hbm_bound else "tensor",
+            "achieved": gbs if hbm_bound else tflops,
+            "peak": peaks["hbm_gbs"] if hbm_bound else t_peak,
+            "unit": "GB/s" if hbm_bound else "TFLOP/s",
+            "frac": (gbs / peaks["hbm_gbs"] if hbm_bound else tflops / t_peak) if ffn_s > 0 else None,
+            "traffic": traffic,
+            "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else t_peak_src),
+            "algorithmic_per_launch": f"{alg['ffn_bytes']:.4g} B and 6*H*I*N = {alg['ffn_flops']:.4g} flop "
+                                      f"over N={alg['N']} kept rows in {wl.n_chunks} chunk(s)",
+            "ms": round(ffn_ms, 4),
+            "tflops": tflops,
+            "gbs": gbs,
+            "tensor_frac": tflops / t_peak if tflops else None,
+            "tensor_frac_sustained": tflops / t_peak_sus if tflops else None,
+            "tensor_peak_sustained": t_peak_sus,
+            "hbm_frac": gbs / peaks["hbm_gbs"] if gbs else None}
+
+
+def dispatch_combine(alg, stage_ms, peaks, peak_src):
+    dc_s = (stage_ms["permute"] + stage_ms["combine"]) / 1e3
+    by = alg["permute_bytes"] + alg["combine_bytes"]
+    gbs = by / dc_s / 1e9 if dc_s > 0 else None
+    return {"achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"] if gbs else None, "bytes_per_step": by,
+            "ms": round(stage_ms["permute"] + stage_ms["combine"], 4),
+            "peak_source": f"{peak_src} hbm_gbs"}
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
@@ -481,54 +620,98 @@ def sample_tokens_for(wl, seconds):
 
 # --------------------------------------------------------------------------- arms
 
+def reference_tokens(wl, seconds):
+    """Tokens of one reference step: about `seconds` of oracle FFN rows, a
+    multiple of the logical EP size (each source rank gets an equal block)."""
+    row_s = (3.0e-3 if wl.ffn_fp8 else 7.7e-3) * (wl.H * wl.I) / (2048 * 768)
+    n = int(seconds / (wl.k * row_s)) // wl.ep * wl.ep
+    return max(wl.ep, min(wl.T, n))
+
+
+def reference_step(wl, Ts, logits, bias, x_np, fetch):
+    """The oracle's whole layer over the first Ts tokens of the workload, one chunk
+    (a capacity scales with the sub-batch: ceil(C * Ts / T)).  Expert weights are
+    fetched (untimed) between the index steps and the FFN.  Returns seconds."""
+    import numpy as np
+    import oracle
+    cap = wl.capacity if wl.capacity < 0 else -(-wl.capacity * Ts // wl.T)
+    t0 = time.perf_counter()
+    idx, w, _, st = oracle.route_topk(logits[:Ts], None if bias is None else bias, wl.k, wl.n_group,
+                                      wl.topk_group, wl.group_score, wl.bias_select_only)
+    keep, _ = oracle.capacity_clip(idx, w, wl.E, cap)
+    lay = oracle.dispatch_layout(idx, keep, wl.E, wl.ep, 0, Ts)
+    if wl.ffn_fp8:
+        xq, xs = oracle.quantize_rows(x_np[:Ts])
+        xr = oracle.permute(xq, lay["recv_token"])
+    else:
+        xr = oracle.permute(x_np[:Ts], lay["recv_token"])
+    t_index = time.perf_counter() - t0
+    eoff = lay["expert_offsets"]
+    weights = {e: fetch(e) for e in range(wl.E) if eoff[e + 1] > eoff[e]}
+    N = lay["N"]
+    y = np.zeros((max(N, 1), wl.H), x_np.dtype)
+    ye = np.zeros((max(N, 1), wl.H), np.float64)
+    t1 = time.perf_counter()
+    for e, wt in weights.items():
+        for p in range(int(eoff[e]), int(eoff[e + 1])):
+            if wl.ffn_fp8:
+                _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xr[p], xs[lay["recv_token"][p]], *wt)
+            else:
+                _, y[p], ye[p] = oracle.ffn_row(xr[p], wt[0], wt[1])
+    if wl.reduce_dense:
+        oracle.combine_exact(ye, lay["pos"], w, Ts, x_np.dtype)
+    else:
+        oracle.combine(y, lay["pos"], w, Ts)
+    return t_index + (time.perf_counter() - t1)
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     import numpy as np
     import torch
-    from combine_moe_route_12_b200.workload import WORKLOADS, make_inputs
+    from combine_moe_route_12_b200.workload import make_inputs
     wl = workload_of(args)
-    # inputs drawn on the CPU generator (no GPU needed for this arm)
+    # inputs drawn on the CPU generator (no GPU needed for this arm); the expert
+    # weights come from their own CPU generator, drawn expert by expert on first
+    # use (same distribution as the GPU arm's, not the same values)
     torch.manual_seed(0)
     inp = make_inputs(wl, "cpu", seed=args.seed, weights=False)
     g = torch.Generator().manual_seed(wl.seed + 1)
     std = 1.0 / math.sqrt(wl.H)
     cache = {}
+    conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
+        else (lambda t: t.numpy().copy())
 
     def fetch(e):
         if e not in cache:
             a = (torch.randn(2 * wl.I, wl.H, generator=g) * std).to(wl.torch_dtype)
             b = (torch.randn(wl.H, wl.I, generator=g) * std).to(wl.torch_dtype)
-            conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
-                else (lambda t: t.numpy().copy())
             cache[e] = fp8_expert(conv(a), conv(b)) if wl.ffn_fp8 else (conv(a), conv(b))
         return cache[e]
 
-    conv = (lambda t: t.view(torch.int16).numpy().view(np.uint16).copy()) if wl.dtype == "bf16" \
-        else (lambda t: t.numpy().copy())
     logits = inp.logits.numpy()
     bias = None if inp.bias is None else inp.bias.numpy()
     x_np = conv(inp.x)
-    shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
-    s_tok = sample_tokens_for(wl, 1.0)
-    vals = []
-    t_all = 0.0
-    desc = ""
+    Ts = reference_tokens(wl, 2.0)
+    secs = []
     for i in range(args.warmup + args.steps):
-        v, secs, desc = oracle_sample(wl, logits, bias, x_np, fetch, s_tok, shared)
+        t = reference_step(wl, Ts, logits, bias, x_np, fetch)
         if i >= args.warmup:
-            vals.append(v)
-            t_all += secs
-    value = statistics.mean(vals)
+            secs.append(t)
+    step_s = statistics.mean(secs)
+    value = Ts / step_s
+    desc = (f"each step: the oracle's whole layer (route, clip, layout, permute, FFN, combine) over the "
+            f"first {Ts} of the {wl.T} tokens in one chunk, {step_s:.2f} s (timed without the untimed "
+            f"draw of the routed experts' weights)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.T / value,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": "each step: " + desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -622,56 +805,79 @@ def run_ours(args):
     if moe.moe_device_status(layer.ws) != 0:
         raise RuntimeError("device status bits set during the timed region")
 
-    # ---------------- per-stage breakdown: the same kernels through the step ABI
-    # on one stream with events between the stages, captured into a CUDA graph
-    # with the events (no host launch gaps); eager launches if capture fails
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(n_marks(wl))]
-    for _ in range(2):
-        run_steps(moe, wl, cfg, inp, B, None, fp8)
-    torch.cuda.synchronize()
-    stage_ms = {s: 0.0 for s in STAGES}
-    step_sum = 0.0
-    bd_ev = mk()
-    bd_graph = None
-    if use_graph:
-        try:
-            # external events stay timing events inside a captured graph
-            gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks(wl))]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                run_steps(moe, wl, cfg, inp, B, gev, fp8)
-            torch.cuda.synchronize()
-            g.replay()
-            torch.cuda.synchronize()
-            stage_times(wl, gev)          # raises if the events cannot be timed
-            bd_graph, bd_ev = g, gev
-        except Exception:
-            bd_graph = None
-            torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.fill_(1)
-        if bd_graph is not None:
-            bd_graph.replay()
-        else:
-            run_steps(moe, wl, cfg, inp, B, bd_ev, fp8)
+    # ---------------- the two-stream overlap: the same layer with both of its
+    # streams the same one (every kernel serialised), replayed from its own graph
+    overlap = None
+    if wl.n_chunks > 1 and not args.no_overlap:
+        s_one = torch.cuda.current_stream()
+
+        def one_stream_pass():
+            moe.moe_forward_chunked(cfg, inp.logits, inp.bias, inp.x, w13_l, w2_l, out_fw,
+                                    layer.topk_idx, layer.topk_w, layer.keep, None, layer.ws,
+                                    s_one, s_one, inp.w13s, inp.w2s, w13_sc, w2_sc)
+
+        one_stream_pass()
         torch.cuda.synchronize()
-        for s_, v in stage_times(wl, bd_ev).items():
-            stage_ms[s_] += v / args.steps
-        step_sum += bd_ev[0].elapsed_time(bd_ev[-1]) / args.steps
-    if moe.moe_device_status(B.ws) != 0:
-        raise RuntimeError("device status bits set during the breakdown pass")
-    eager_step_ms = step_sum
-    breakdown_mode = "graph" if bd_graph is not None else "eager"
-    n_kept, n_active = [], []
-    for c in range(wl.n_chunks):
-        moe.moe_dispatch_layout(cfg, c * B.tc, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
-                                B.pos, B.spl, None, B.ws)
-        n_kept.append(int(B.eoff[wl.E].item()))
-        n_active.append(int(((B.eoff[1:] - B.eoff[:-1]) > 0).sum().item()))
-    tokens_read = int((B.keep.view(wl.T, wl.k) != 0).any(dim=1).sum().item())
+        g1 = None
+        if use_graph:
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1):
+                one_stream_pass()
+            torch.cuda.synchronize()
+        run1 = g1.replay if g1 is not None else one_stream_pass
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            run1()
+        ev1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(1)
+            ev1[i][0].record()
+            run1()
+            ev1[i][1].record()
+        torch.cuda.synchronize()
+        if moe.moe_device_status(layer.ws) != 0:
+            raise RuntimeError("device status bits set during the one-stream pass")
+        one_ms = sum(a.elapsed_time(b) for a, b in ev1) / args.steps
+        del g1
+        overlap = {"one_stream_ms": round(one_ms, 4),
+                   "two_stream_ms": round(sum(step_ms) / args.steps, 4)}
+
+    # ---------------- per-stage breakdown: the same kernels through the step ABI
+    stage_ms, disp_ms, eager_step_ms, breakdown_mode = breakdown(
+        moe, wl, cfg, inp, B, fp8, args.steps, flush, use_graph)
+    n_kept, n_active, tokens_read = layout_counts(moe, wl, cfg, B)
     alg = algorithmic(wl, n_kept, n_active, tokens_read)
     bwd = backward_row_passes(moe, wl, cfg, B, n_kept[-1], peaks, flush, args) \
         if args.backward and not wl.reduce_dense else None
+    if overlap is not None:
+        # what the second stream can hide: the dispatch (layout + permute) of
+        # every chunk after the first, which runs beside the previous chunk's FFN
+        hideable = sum(disp_ms[1:])
+        hidden = overlap["one_stream_ms"] - overlap["two_stream_ms"]
+        overlap.update({"dispatch_ms_per_chunk": [round(v, 4) for v in disp_ms],
+                        "hideable_ms": round(hideable, 4), "hidden_ms": round(hidden, 4),
+                        "hidden_frac": hidden / hideable if hideable > 0 else None,
+                        "note": "one_stream: moe_forward_chunked with s_dispatch = s_compute (same "
+                                "kernels, serialised); hideable: dispatch_layout + permute of chunks "
+                                ">= 1 from the breakdown"})
+
+    # ---------------- the same layer in one chunk: the FFN reads each expert's
+    # weights once per layer pass (the tensor-roof reading of a chunked workload)
+    unchunked = None
+    if wl.n_chunks > 1 and not args.no_unchunked:
+        wl1 = wl.with_(n_chunks=1)
+        cfg1 = moe.config_from_workload(wl1)
+        B1 = StepBuffers(moe, wl1, cfg1, dev)
+        st1, _, step1, _ = breakdown(moe, wl1, cfg1, inp, B1, fp8, args.steps, flush, use_graph)
+        k1, a1, r1 = layout_counts(moe, wl1, cfg1, B1)
+        alg1 = algorithmic(wl1, k1, a1, r1)
+        unchunked = {"roofline": ffn_roofline(wl1, alg1, st1["grouped_ffn"], peaks, peak_src, None),
+                     "dispatch_combine": dispatch_combine(alg1, st1, peaks, peak_src),
+                     "stage_ms": {k: round(v, 4) for k, v in st1.items()},
+                     "breakdown_step_ms": round(step1, 4)}
+        del B1
+        torch.cuda.empty_cache()
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -724,48 +930,21 @@ def run_ours(args):
     if rank == 0:
         ms_per_step = total_ms / args.steps
         value = world * wl.T * args.steps / (total_ms / 1e3)
-        ffn_s = stage_ms["grouped_ffn"] / 1e3
-        dc_s = (stage_ms["permute"] + stage_ms["combine"]) / 1e3
-        ffn_tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
-        ffn_gbs = alg["ffn_bytes"] / ffn_s / 1e9 if ffn_s > 0 else None
-        # the tensor peak of the FFN's operand type: the measured bf16 figure, times
-        # the nominal dense FP8 / bf16 ratio (4.5 / 2.25) for E4M3 operands
-        t_peak = peaks["bf16_tflops"] * (2.0 if wl.ffn_fp8 else 1.0)
-        t_peak_src = "bf16_tflops (burst) x 2 (nominal e4m3 / bf16)" if wl.ffn_fp8 else "bf16_tflops (burst)"
-        # the binding roof: HBM when the pass's flop per byte is below the ridge
-        t_flop = alg["ffn_flops"] / (t_peak * 1e12)
-        t_byte = alg["ffn_bytes"] / (peaks["hbm_gbs"] * 1e9)
-        hbm_bound = t_byte > t_flop
-        dc_gbs = (alg["permute_bytes"] + alg["combine_bytes"]) / dc_s / 1e9 if dc_s > 0 else None
         src = kernel_src_hash(wl.ffn_fp8)
         tr = FFN_TRAFFIC.get(wl.name)
         traffic = tr["bytes"] if tr and tr.get("src") == src and tr.get("chunks", 1) == wl.n_chunks else None
+        roof = ffn_roofline(wl, alg, stage_ms["grouped_ffn"], peaks, peak_src, traffic)
+        dc = dispatch_combine(alg, stage_ms, peaks, peak_src)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 (expert FFN) / bf16" if wl.ffn_fp8 else wl.dtype, "data": "synthetic",
             "config": workload_config(wl, world, use_graph),
-            "roofline": {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass"
-                                   + (", E4M3 operands, h quantised between them)" if wl.ffn_fp8 else ")"),
-                         "bound": "hbm" if hbm_bound else "tensor",
-                         "achieved": ffn_gbs if hbm_bound else ffn_tflops,
-                         "peak": peaks["hbm_gbs"] if hbm_bound else t_peak,
-                         "unit": "GB/s" if hbm_bound else "TFLOP/s",
-                         "frac": (ffn_gbs / peaks["hbm_gbs"] if hbm_bound else ffn_tflops / t_peak)
-                         if ffn_s > 0 else None,
-                         "traffic": traffic,
-                         "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else t_peak_src),
-                         "algorithmic_per_launch": f"{alg['ffn_bytes']:.4g} B and 6*H*I*N = {alg['ffn_flops']:.4g} flop "
-                                                   f"over N={alg['N']} kept rows",
-                         "tensor_frac": ffn_tflops / t_peak if ffn_tflops else None,
-                         "hbm_frac": ffn_gbs / peaks["hbm_gbs"] if ffn_gbs else None},
-            "dispatch_combine": {"achieved_gbs": dc_gbs, "peak_gbs": peaks["hbm_gbs"],
-                                 "frac": dc_gbs / peaks["hbm_gbs"] if dc_gbs else None,
-                                 "bytes_per_step": alg["permute_bytes"] + alg["combine_bytes"],
-                                 "peak_source": f"{peak_src} hbm_gbs"},
-            "ffn_tflops": ffn_tflops,
-            "ffn_gbs": ffn_gbs,
+            "roofline": roof,
+            "dispatch_combine": dc,
+            "ffn_tflops": roof["tflops"],
+            "ffn_gbs": roof["gbs"],
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "breakdown_step_ms": round(eager_step_ms, 4),
             "breakdown_mode": breakdown_mode,
@@ -775,6 +954,10 @@ def run_ours(args):
             "gpu_launches": kernels_per_step(wl) * args.steps,
             "clocks": clocks,
         }
+        if unchunked is not None:
+            line["roofline_unchunked"] = unchunked
+        if overlap is not None:
+            line["overlap"] = overlap
         if bwd is not None:
             line["backward_row_passes"] = bwd
         print(json.dumps(line), flush=True)

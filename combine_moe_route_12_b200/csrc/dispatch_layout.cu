@@ -293,6 +293,10 @@ size_t layout_scatter_smem(const moe_config &c, int tile_tokens) {
                               2 * (size_t)tile_tokens * c.k + split);
 }
 
+// The scatter's dynamic shared memory opt-in, shared by the workspace and the
+// allocation-free entry points.
+SmemOptIn g_scatter_opt_in;
+
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
                                    const int32_t *topk_idx, const uint8_t *keep,
                                    int32_t *expert_offsets, int32_t *rank_offsets,
@@ -321,8 +325,7 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
             tb, tc, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         const size_t smem = layout_scatter_smem(c, tile_tokens);
-        static SmemOptIn opt_in;
-        if ((err = opt_in.ensure(layout_scatter_kernel, smem)) != cudaSuccess) return err;
+        if ((err = g_scatter_opt_in.ensure(layout_scatter_kernel, smem)) != cudaSuccess) return err;
         layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, s>>>(
             tb, tc, c.k, c.E, c.ep, tile_tokens, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
             expert_offsets, rank_offsets, recv_token, recv_slot, pos, send_splits, status);
@@ -360,7 +363,9 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
 // (different streams without ordering, or several host threads) race and
 // corrupt each other's layouts; order them.  The first call on a device looks
 // up the array's device address (cudaGetSymbolAddress) with that device
-// current; make that first call before any stream capture.
+// current; make that first call before any stream capture.  The address is
+// looked up again when the device's context has changed since (after a
+// cudaDeviceReset, which reloads the module and may move the array).
 namespace {
 
 constexpr int kNoAllocMaxTiles = 64;   // 16384 tokens per call
@@ -375,19 +380,25 @@ static __device__ __align__(256) unsigned char g_noalloc_layout_scratch[kNoAlloc
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void *g_noalloc_base[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};
 
-// Device address of the array for the current device (looked up once per device).
+// Device address of the array for the current device: looked up once per
+// device and context (the context id is 0 before the first lookup has created
+// the context, or when the driver cannot report it: then it is looked up on
+// every call).
 cudaError_t noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_base[dev]) {
+    const unsigned long long ctx = moe::current_context_id();
+    if (!g_noalloc_base[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *p = nullptr;
         err = cudaGetSymbolAddress(&p, g_noalloc_layout_scratch);
         if (err != cudaSuccess) return err;
         g_noalloc_base[dev] = p;
+        g_noalloc_ctx[dev] = moe::current_context_id();
     }
     *out = g_noalloc_base[dev];
     return cudaSuccess;
@@ -441,8 +452,7 @@ extern "C" moe_status moe_dispatch_layout_noalloc(
             tok_begin, tok_count, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
         err = cudaGetLastError();
         const size_t smem = layout_scatter_smem(c, tile_tokens);
-        if (err == cudaSuccess && smem > 48 * 1024)
-            err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err == cudaSuccess) err = g_scatter_opt_in.ensure(layout_scatter_kernel, smem);
         if (err == cudaSuccess) {
             layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, stream>>>(
                 tok_begin, tok_count, c.k, c.E, c.ep, tile_tokens, max_recv_rows_of(c, tok_count), topk_idx, keep,

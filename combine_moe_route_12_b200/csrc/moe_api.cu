@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <vector>
 
 #include "moe_common.cuh"
@@ -172,19 +173,25 @@ ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
     return F;
 }
 
-// Per-thread, per-device pool of timing-free events for the chunked forward.
+// Per-thread, per-device pool of timing-free events for the chunked forward,
+// keyed by the device index and refilled when the device's context changed
+// (events of a context that a device reset destroyed are gone with it).
 struct EventPool {
-    int device = -1;
+    unsigned long long ctx = 0;
     std::vector<cudaEvent_t> ev;
 };
-thread_local EventPool g_events[16];
+thread_local std::map<int, EventPool> g_events;
 
 cudaError_t get_events(int n, cudaEvent_t **out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    EventPool &P = g_events[dev & 15];
-    if (P.device != dev) { P.ev.clear(); P.device = dev; }
+    EventPool &P = g_events[dev];
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0 && P.ctx != ctx) {
+        if (P.ctx != 0) P.ev.clear();   // their context is gone: nothing to destroy
+        P.ctx = ctx;
+    }
     while ((int)P.ev.size() < n) {
         cudaEvent_t e;
         if ((err = cudaEventCreateWithFlags(&e, cudaEventDisableTiming)) != cudaSuccess) return err;

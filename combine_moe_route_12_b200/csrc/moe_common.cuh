@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <mutex>
@@ -35,9 +36,41 @@ inline int64_t layout_max_tiles(int64_t tc) {
 }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up after 2 s
 
+// Unique id of the CUDA context current on the calling thread (cuCtxGetId), 0
+// when no context is current yet or the driver does not offer the call.  A
+// device reset (cudaDeviceReset) replaces the context, and with it every
+// module-level state: kernel attributes and the addresses of __device__
+// variables.  Per-device caches of such state compare this id to notice it.
+inline unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    struct Fns {
+        GetCurrent cur = nullptr;
+        GetId id = nullptr;
+        Fns() {
+            void *p = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                cur = reinterpret_cast<GetCurrent>(p);
+            p = nullptr;
+            if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                id = reinterpret_cast<GetId>(p);
+        }
+    };
+    static const Fns fns;   // looked up once per process
+    if (!fns.cur || !fns.id) return 0;
+    CUcontext ctx = nullptr;
+    if (fns.cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long v = 0;
+    return fns.id(ctx, &v) == CUDA_SUCCESS ? v : 0;
+}
+
 // Opens a kernel's dynamic shared memory beyond the default 48 KiB.  The
-// attribute belongs to the current device, so the largest size already set is
-// remembered per device.
+// attribute belongs to the device's current context, so the largest size
+// already set is remembered per device together with the context it was set
+// in; a new context (after a device reset) starts again from the default.
 class SmemOptIn {
   public:
     template <typename Kernel>
@@ -46,9 +79,11 @@ class SmemOptIn {
         int dev = 0;
         cudaError_t err = cudaGetDevice(&dev);
         if (err != cudaSuccess) return err;
-        if (dev < 0 || dev >= kDevices)
+        const unsigned long long ctx = current_context_id();
+        if (dev < 0 || dev >= kDevices || ctx == 0)
             return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         std::lock_guard<std::mutex> lock(m_);
+        if (ctx_[dev] != ctx) { ctx_[dev] = ctx; set_[dev] = 0; }
         if (bytes <= set_[dev]) return cudaSuccess;
         err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (err == cudaSuccess) set_[dev] = bytes;
@@ -60,6 +95,7 @@ class SmemOptIn {
     static constexpr int kDevices = 64;
     std::mutex m_;
     size_t set_[kDevices] = {};
+    unsigned long long ctx_[kDevices] = {};
 };
 
 // ---------------------------------------------------------------- workspace

@@ -29,7 +29,8 @@
  *   [AX]  axolotl docs, "integrations.expert_parallel.args", ExpertParallelArgs:
  *         expert_parallel_backend (torch = all_to_all_single over the EP group),
  *         expert_parallel_dispatch_chunks, expert_parallel_save_dispatch
- *         ("routing topk and host-side split counts are always saved"),
+ *         (the routing choice and the host-side split counts are kept
+ *         either way),
  *         expert_parallel_size, expert_parallel_token_capacity, and
  *         validate_expert_parallel_topology.
  *   [LL]  LightLLM PR 1687 review page: _select_experts / norm_topk_prob,

@@ -45,6 +45,32 @@ def test_kernels_per_step():
 
 def test_default_arguments_finish_within_minutes():
     a = bench.parse_args([])
-    assert a.gpus == 1 and a.config == "qwen3_30b_a3b" and a.impl == "ours"
+    assert a.gpus == 1 and a.config == "dsv3_prefill" and a.impl == "ours"
     assert a.warmup >= 3 and a.steps <= 100
     assert not a.backward
+
+
+def test_reference_steps_are_ep_aligned_sub_batches():
+    for name in ("tiny", "qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode"):
+        wl = WORKLOADS[name]
+        ts = bench.reference_tokens(wl, 2.0)
+        assert ts % wl.ep == 0 and wl.ep <= ts <= wl.T
+
+
+def test_ffn_roofline_picks_the_binding_roof():
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1370.0}
+    wl = WORKLOADS["dsv3_prefill"]
+    # two chunks: every expert's weights twice, HBM-bound
+    a2 = bench.algorithmic(wl, [32768, 32768], [256, 256], tokens_read=8192)
+    r2 = bench.ffn_roofline(wl, a2, 8.0, peaks, "measured", None)
+    assert r2["bound"] == "hbm" and abs(r2["frac"] - r2["hbm_frac"]) < 1e-12
+    # one chunk: one weight read; at 231 flop/B it still sits below this ridge
+    # (254 flop/B), and above a lower one, where the tensor roof binds
+    a1 = bench.algorithmic(wl.with_(n_chunks=1), [65536], [256], tokens_read=8192)
+    assert 230 < a1["ffn_flops"] / a1["ffn_bytes"] < 232
+    r1 = bench.ffn_roofline(wl.with_(n_chunks=1), a1, 6.0, peaks, "measured", None)
+    assert r1["bound"] == "hbm"
+    low = dict(peaks, bf16_tflops=1400.0)
+    r1 = bench.ffn_roofline(wl.with_(n_chunks=1), a1, 6.0, low, "measured", None)
+    assert r1["bound"] == "tensor" and abs(r1["frac"] - r1["tensor_frac"]) < 1e-12
+    assert r1["tensor_frac_sustained"] > r1["tensor_frac"]

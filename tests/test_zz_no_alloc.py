@@ -35,9 +35,21 @@ def _layout(fn, cfg, wl, tb, tc, idx, keep, **kw):
     return {k: (v[:n] if k in ("rt", "rs") else v).cpu().numpy() for k, v in d.items()}, n
 
 
-def test_noalloc_layout_equals_workspace_layout_twice():
-    wl = MoEWorkload("noalloc", T=2048, H=128, E=64, k=6, I=128, dtype="bf16", ep=4,
-                     capacity=150, skew_bias=True)
+# (workload, token ranges): two calls in a row on different ranges (the second
+# reuses the array the first one left behind), then the first range again; the
+# second workload fills the array to its edge - 64 tiles of 256 tokens times
+# 1024 experts of look-back descriptors - and takes the scatter's shared-memory
+# opt-in beyond 48 KiB
+CASES = [
+    (MoEWorkload("noalloc", T=2048, H=128, E=64, k=6, I=128, dtype="bf16", ep=4,
+                 capacity=150, skew_bias=True), ((0, 2048), (512, 1024), (0, 2048))),
+    (MoEWorkload("noalloc_edge", T=16384, H=128, E=1024, k=8, I=128, dtype="bf16", ep=8),
+     ((0, 16384), (8192, 4096), (0, 16384))),
+]
+
+
+@pytest.mark.parametrize("wl,ranges", CASES, ids=[c[0].name for c in CASES])
+def test_noalloc_layout_equals_workspace_layout_twice(wl, ranges):
     cfg = moe.config_from_workload(wl)
     inp = make_inputs(wl, "cuda", seed=5, weights=False)
     ws = moe.alloc_workspace(moe.workspace_bytes(cfg))
@@ -49,9 +61,7 @@ def test_noalloc_layout_equals_workspace_layout_twice():
     moe.moe_route_topk(cfg, inp.logits, inp.bias, idx, w, counts, ws)
     moe.moe_capacity_clip(cfg, idx, w, counts, keep, kept, ws)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    # two calls in a row on different token ranges (the second call reuses the
-    # array the first one left behind), then the first range again
-    for tb, tc in ((0, 2048), (512, 1024), (0, 2048)):
+    for tb, tc in ranges:
         ref, n_ref = _layout(lambda *a: moe.moe_dispatch_layout(*a, ws), cfg, wl, tb, tc, idx, keep)
         got, n_got = _layout(moe.moe_dispatch_layout_noalloc, cfg, wl, tb, tc, idx, keep,
                              status=status)
