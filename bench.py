@@ -58,6 +58,11 @@ FFN_TRAFFIC = {
     "qwen3_30b_a3b": {"bytes": 1560.882432e6, "src": "24bdbd71939c8d30"},
     # both GEMM launches and the quantisation of h between them
     "qwen3_30b_a3b_fp8": {"bytes": 893.983232e6, "src": "ab5f51ea4de56437"},
+    # captured with 32 of the 256 experts and 1024 tokens (the same 128 rows per
+    # expert and chunk), scaled by 8 per chunk, two chunks; see
+    # profiles/ffn_tcgen05_dsv3_prefill.md
+    "dsv3_prefill": {"bytes": 2 * 8 * (1955.491e6 + 18.525e6 + 957.271e6 + 54.639e6),
+                     "src": "24bdbd71939c8d30", "chunks": 2},
 }
 
 
@@ -809,9 +814,9 @@ def run_ours(args):
     # streams the same one (every kernel serialised), replayed from its own graph
     overlap = None
     if wl.n_chunks > 1 and not args.no_overlap:
-        s_one = torch.cuda.current_stream()
-
         def one_stream_pass():
+            # the stream current at the call (inside a capture: the capturing one)
+            s_one = torch.cuda.current_stream()
             moe.moe_forward_chunked(cfg, inp.logits, inp.bias, inp.x, w13_l, w2_l, out_fw,
                                     layer.topk_idx, layer.topk_w, layer.keep, None, layer.ws,
                                     s_one, s_one, inp.w13s, inp.w2s, w13_sc, w2_sc)

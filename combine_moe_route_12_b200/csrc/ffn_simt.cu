@@ -101,4 +101,112 @@ cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ backward (fp32)
+// The same backward as the tcgen05 path (gate / up recomputed, dh, the SwiGLU
+// backward, dxr, the weight gradients), in fp32 FMA.  One CTA per receive row
+// for the data gradients; one CTA per (expert, output row) for the weights.
+
+// g, u of the row (warp per feature, coalesced W13 rows), then per feature
+// (thread per feature, coalesced W2 reads across features) dh = W2[:, i] . dy,
+// h = silu(g) u, dg = dh u s (1 + g (1 - s)), du = dh silu(g).
+__global__ void __launch_bounds__(kSimtThreads) ffn_simt_bwd_rows_kernel(
+    int E, int H, int I, const int32_t *__restrict__ offs, const float *__restrict__ xr,
+    const float *__restrict__ dy, const float *__restrict__ w13, const float *__restrict__ w2,
+    float *__restrict__ h, float *__restrict__ dgu) {
+    extern __shared__ float sm[];   // x [H], dy [H], g [I], u [I]
+    float *s_x = sm, *s_dy = sm + H, *s_g = sm + 2 * H, *s_u = s_g + I;
+    const int p = blockIdx.x;
+    if (p >= offs[E]) return;
+    const int e = expert_of_row(offs, E, p);
+    for (int c = threadIdx.x; c < H; c += blockDim.x) {
+        s_x[c] = xr[(size_t)p * H + c];
+        s_dy[c] = dy[(size_t)p * H + c];
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const float *wg = w13 + (size_t)e * 2 * I * H;
+    for (int i = warp; i < I; i += nw) {
+        const float *rg = wg + (size_t)i * H;
+        const float *ru = wg + (size_t)(I + i) * H;
+        float g = 0.f, u = 0.f;
+        for (int c = lane; c < H; c += 32) {
+            g = __fmaf_rn(__ldg(rg + c), s_x[c], g);
+            u = __fmaf_rn(__ldg(ru + c), s_x[c], u);
+        }
+        g = warp_sum(g);
+        u = warp_sum(u);
+        if (lane == 0) { s_g[i] = g; s_u[i] = u; }
+    }
+    __syncthreads();
+    const float *we = w2 + (size_t)e * H * I;
+    for (int i = threadIdx.x; i < I; i += blockDim.x) {
+        float dh = 0.f;
+        for (int o = 0; o < H; ++o) dh = __fmaf_rn(__ldg(we + (size_t)o * I + i), s_dy[o], dh);
+        const float g = s_g[i], u = s_u[i];
+        const float sg = 1.0f / (1.0f + expf(-g));
+        h[(size_t)p * I + i] = g * sg * u;
+        dgu[(size_t)p * 2 * I + i] = dh * u * sg * (1.0f + g * (1.0f - sg));
+        dgu[(size_t)p * 2 * I + I + i] = dh * g * sg;
+    }
+}
+
+// dxr[p, c] = sum over j < 2I of W13[e][j, c] * dgu[p, j] (thread per c, coalesced)
+__global__ void __launch_bounds__(kSimtThreads) ffn_simt_bwd_dx_kernel(
+    int E, int H, int I, const int32_t *__restrict__ offs, const float *__restrict__ dgu,
+    const float *__restrict__ w13, float *__restrict__ dxr) {
+    extern __shared__ float s_d[];  // [2I]
+    const int p = blockIdx.x;
+    if (p >= offs[E]) return;
+    const int e = expert_of_row(offs, E, p);
+    for (int j = threadIdx.x; j < 2 * I; j += blockDim.x) s_d[j] = dgu[(size_t)p * 2 * I + j];
+    __syncthreads();
+    const float *we = w13 + (size_t)e * 2 * I * H;
+    for (int c = threadIdx.x; c < H; c += blockDim.x) {
+        float acc = 0.f;
+        for (int j = 0; j < 2 * I; ++j) acc = __fmaf_rn(__ldg(we + (size_t)j * H + c), s_d[j], acc);
+        dxr[(size_t)p * H + c] = acc;
+    }
+}
+
+// out[e][m, n] (+)= sum over the expert's rows p of a[p, m] * b[p, n]
+__global__ void __launch_bounds__(kSimtThreads) ffn_simt_wgrad_kernel(
+    int M, int N, const int32_t *__restrict__ offs, const float *__restrict__ a,
+    const float *__restrict__ b, float *__restrict__ out, int accumulate) {
+    const int m = blockIdx.x, e = blockIdx.y;
+    const int p0 = offs[e], p1 = offs[e + 1];
+    float *o = out + ((size_t)e * M + m) * N;
+    for (int n = threadIdx.x; n < N; n += blockDim.x) {
+        float acc = 0.f;
+        for (int p = p0; p < p1; ++p) acc = __fmaf_rn(a[(size_t)p * M + m], b[(size_t)p * N + n], acc);
+        o[n] = accumulate ? o[n] + acc : acc;
+    }
+}
+
+cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                const int32_t *expert_offsets, const void *w13, const void *w2,
+                                void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                int accumulate, cudaStream_t s) {
+    if (n_rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const float *x = static_cast<const float *>(xr), *d = static_cast<const float *>(dy);
+    if (n_rows > 0) {
+        ffn_simt_bwd_rows_kernel<<<(int)n_rows, kSimtThreads, sizeof(float) * (2 * (size_t)c.H + 2 * c.I), s>>>(
+            c.E, c.H, c.I, expert_offsets, x, d, static_cast<const float *>(w13),
+            static_cast<const float *>(w2), static_cast<float *>(h), static_cast<float *>(dgu));
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+        ffn_simt_bwd_dx_kernel<<<(int)n_rows, kSimtThreads, sizeof(float) * 2 * (size_t)c.I, s>>>(
+            c.E, c.H, c.I, expert_offsets, static_cast<const float *>(dgu),
+            static_cast<const float *>(w13), static_cast<float *>(dxr));
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    // the weight gradients run whatever n_rows is: experts without rows get zeros
+    ffn_simt_wgrad_kernel<<<dim3(c.H, c.E), kSimtThreads, 0, s>>>(
+        c.H, c.I, expert_offsets, d, static_cast<const float *>(h), dw2, accumulate);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    ffn_simt_wgrad_kernel<<<dim3(2 * c.I, c.E), kSimtThreads, 0, s>>>(
+        2 * c.I, c.H, expert_offsets, static_cast<const float *>(dgu), x, dw13, accumulate);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -69,7 +69,10 @@ constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 192 KiB
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
 constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (4 warp pairs x 2 ways x 2 KiB)
 
-enum EpiMode : int { kEpiSwiGLU = 0, kEpiStore = 1, kEpiReduce = 2 };
+// Epilogues: the forward's SwiGLU (h), store (y) and decode reduce; the
+// backward's store of the recomputed gate and up values (g | u side by side)
+// and its SwiGLU backward (dh in TMEM, g and u read back: h, dg, du).
+enum EpiMode : int { kEpiSwiGLU = 0, kEpiStore = 1, kEpiReduce = 2, kEpiStoreGU = 3, kEpiSwiGLUBwd = 4 };
 
 struct FfnGemmParams {
     const int32_t *expert_offsets;
@@ -92,6 +95,13 @@ struct FfnGemmParams {
     const uint8_t *w_scale;
     const uint8_t *t_scale;
     int t_scale_by_token;
+    // row stride of `out` in elements (out_cols for the forward's outputs; 2I for
+    // the backward's g | u rows, whose up half starts half_cols further on)
+    int out_ld;
+    int half_cols;
+    // SwiGLU backward: g | u rows [n, 2I] (read) and dg | du rows [n, 2I] (written)
+    const __nv_bfloat16 *gu;
+    __nv_bfloat16 *out2;
 };
 
 constexpr int kQueue = 8;                            // slices published ahead of the slowest consumer
@@ -214,12 +224,18 @@ struct SliceReader {
 
 // F8: E4M3 operands (tcgen05 kind::f8f6f4, 128 columns per k-chunk) with the
 // row scales applied to the fp32 accumulators in the epilogue; else bf16.
-template <int MODE, bool F8>
+// A_MN: the weight operand is read transposed, MN-major (the backward's
+// W2^T and W13^T): a ring stage holds its 128 k rows of the CTA's 128 output
+// features as two 64-feature blocks of 128-byte rows, one 3-D TMA box.
+template <int MODE, bool F8, bool A_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
     const __grid_constant__ CUtensorMap tmap_xs,
     const FfnGemmParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kSwiGLU = MODE == kEpiSwiGLU;
+    // gate and up rows of W13 side by side in a CTA's 128 weight rows
+    constexpr bool kGateUp = MODE == kEpiSwiGLU || MODE == kEpiStoreGU;
+    static_assert(!(A_MN && (F8 || kGateUp)), "the transposed weight operand is bf16 with plain rows");
     // queue consumers per entry: the MMA thread, the follower's producer, and
     // every epilogue warp of both CTAs (GEMM1: the gate warp of each pair only)
     constexpr uint32_t kQueueConsumers = 2 + 2 * (kSwiGLU ? kEpiWarps / 2 : kEpiWarps);
@@ -336,8 +352,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     const int ch = kb * kKS;   // first k-chunk of the stage
                     // full boxes land in both CTAs (rows or chunks past the tensor are zero-filled)
                     if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * stage_bytes);
-                    if (kSwiGLU)
+                    if (kGateUp)
                         tma_load_4d_pair(st, &tmap_w, full_leader, 0, f_row, 2 * se, ch);
+                    else if (A_MN)   // k rows of the expert, the CTA's two 64-feature blocks
+                        tma_load_3d_pair(st, &tmap_w, full_leader, 0, se * P.K + ch * kBK, f_row / kBK);
                     else
                         tma_load_3d_pair(st, &tmap_w, full_leader, 0, w_row, ch);
                     tma_load_3d_pair(st + kKS * kWBytes, small_box ? &tmap_xs : &tmap_x, full_leader, 0, tok_row, ch);
@@ -380,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                   {
                     const TileInfo ti = tile_info(se, sf, t_blk, P);
                     const uint32_t idesc = F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_mma)
-                                              : make_idesc_bf16_f32(2 * kRowsPerCta, ti.n_mma);
+                                              : make_idesc_bf16_f32_major(2 * kRowsPerCta, ti.n_mma, A_MN, false);
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
@@ -394,7 +412,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                         for (int c = 0; c < kKS; ++c) {
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {   // 32-byte k-steps: 16 bf16 or 32 E4M3
-                                const uint64_t wdesc = make_sw128_desc(st + c * kWBytes + kk * 32);
+                                // MN-major: k-chunk c is rows 64c.. of each 64-feature block
+                                // (blocks 16 KiB apart), a k-step 16 rows of 128 bytes
+                                const uint64_t wdesc = A_MN
+                                    ? make_sw128_desc_mn(st + c * (kWBytes / 2) + kk * 2048, kWBytes)
+                                    : make_sw128_desc(st + c * kWBytes + kk * 32);
                                 const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * tchunk + kk * 32);
                                 const uint32_t accum = (kb > 0 || c > 0 || kk > 0) ? 1u : 0u;
                                 if (F8) tc_mma_f8_pair(d, wdesc, tdesc, idesc, accum);
@@ -426,7 +448,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
         const int q = warp & 3, half = warp >> 2;
         // GEMM1: quadrants 0-1 hold gate, quadrants 2-3 the up rows of the same features;
         // GEMM2: quadrant q holds output features 32q .. 32q+31 of this CTA's 128
-        const int feat_lane = kSwiGLU ? (q & 1) * 32 + lane : q * 32 + lane;
+        const int feat_lane = kGateUp ? (q & 1) * 32 + lane : q * 32 + lane;
         const bool is_gate = q < 2;
         const int xpair = half * 2 + (q & 1);                 // gate/up warp pair (GEMM1)
         const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
@@ -467,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
            if (F8) {
                if (f_ok)
                    wsc = ue8m0_value(P.w_scale[(size_t)ti.e * P.w_rows_per_expert +
-                                               (kSwiGLU && !is_gate ? P.out_cols : 0) + f]);
+                                               (kGateUp && !is_gate ? P.out_cols : 0) + f]);
                float t4[4];
 #pragma unroll
                for (int i = 0; i < 4; ++i) {
@@ -551,16 +573,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                             if (tok < nc) *reinterpret_cast<uint4 *>(h + (size_t)tok * P.out_cols) = o[g8];
                         }
                     }
+                } else if (MODE == kEpiStoreGU) {
+                    // the gate value of feature f to column f, the up value to column I + f
+                    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld +
+                                       f + (is_gate ? 0 : P.half_cols);
+                    const int nc = min(32, ti.n_valid - c0);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (f_ok && j < nc) o[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                } else if (MODE == kEpiSwiGLUBwd) {
+                    // r = dh of feature f for 32 tokens; with s = sigmoid(g):
+                    //   h = g s u,  dg = dh u s (1 + g (1 - s)),  du = dh g s
+                    const int nc = min(32, ti.n_valid - c0);
+                    const size_t row0 = (size_t)(ti.p0 + c0);
+                    float g[32], u[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        g[j] = 0.0f;
+                        u[j] = 0.0f;
+                        if (f_ok && j < nc) {
+                            const __nv_bfloat16 *gr = P.gu + (row0 + j) * P.out_ld + f;
+                            g[j] = __bfloat162float(gr[0]);
+                            u[j] = __bfloat162float(gr[P.half_cols]);
+                        }
+                    }
+                    __nv_bfloat16 *ho = static_cast<__nv_bfloat16 *>(P.out) + row0 * P.out_cols + f;
+                    __nv_bfloat16 *dgo = P.out2 + row0 * P.out_ld + f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float dh = __uint_as_float(r[j]);
+                        const float sg = __fdividef(1.0f, 1.0f + __expf(-g[j]));
+                        const float sl = g[j] * sg;
+                        if (f_ok && j < nc) {
+                            ho[(size_t)j * P.out_cols] = __float2bfloat16_rn(sl * u[j]);
+                            dgo[(size_t)j * P.out_ld] =
+                                __float2bfloat16_rn(dh * u[j] * sg * (1.0f + g[j] * (1.0f - sg)));
+                            dgo[(size_t)j * P.out_ld + P.half_cols] = __float2bfloat16_rn(dh * sl);
+                        }
+                    }
                 } else if (MODE == kEpiStore) {
                     // one 64-byte warp store per token row (the shuffle rearrangement
                     // of the SwiGLU epilogue measured slower here)
-                    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_cols + f;
+                    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld + f;
                     const int nc = min(32, ti.n_valid - c0);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         float v = __uint_as_float(r[j]);
                         if (F8) v *= __shfl_sync(0xffffffffu, ts_lane, j) * wsc;
-                        if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(v);
+                        if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(v);
                     }
                 } else {  // kEpiReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
@@ -656,14 +716,14 @@ size_t ffn_tcgen05_smem(int E, bool swiglu) {
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
-template <int MODE, bool F8>
+template <int MODE, bool F8, bool A_MN = false>
 static cudaError_t launch_gemm(const CUtensorMap &tw, const CUtensorMap &tx, const CUtensorMap &txs,
                                const FfnGemmParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_tcgen05_smem(P.E, MODE == kEpiSwiGLU);
     static SmemOptIn opt_in;   // one per kernel instantiation
-    cudaError_t err = opt_in.ensure(ffn_gemm_tcgen05_kernel<MODE, F8>, smem);
+    cudaError_t err = opt_in.ensure(ffn_gemm_tcgen05_kernel<MODE, F8, A_MN>, smem);
     if (err != cudaSuccess) return err;
-    ffn_gemm_tcgen05_kernel<MODE, F8><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
+    ffn_gemm_tcgen05_kernel<MODE, F8, A_MN><<<grid, kFfnThreads, smem, s>>>(tw, tx, txs, P, counter);
     return cudaGetLastError();
 }
 
@@ -679,6 +739,7 @@ static void ffn_params(const moe_config &c, const int32_t *expert_offsets, void 
     P1.n_fblocks = (c.I + 2 * P1.feat_per_cta - 1) / (2 * P1.feat_per_cta);
     P1.w_rows_per_expert = 2 * c.I;
     P1.out_cols = c.I;
+    P1.out_ld = c.I;
     P1.out = h;
     P1.k = c.k;
     P1.status = status;
@@ -689,6 +750,7 @@ static void ffn_params(const moe_config &c, const int32_t *expert_offsets, void 
     P2.n_fblocks = (c.H + 2 * P2.feat_per_cta - 1) / (2 * P2.feat_per_cta);
     P2.w_rows_per_expert = c.H;
     P2.out_cols = c.H;
+    P2.out_ld = c.H;
     P2.out = y;
     P2.out_reduce = out_reduce;
     P2.recv_slot = recv_slot;
@@ -730,6 +792,93 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
     const int grid2 = ffn_grid(c, n_rows, P2, num_sms);
     if (c.reduce_dense) return launch_gemm<kEpiReduce, false>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
     return launch_gemm<kEpiStore, false>(tw2, tx2, tx2s, P2, grid2, counters + 1, s);
+}
+
+// A row-major bf16 [rows, cols] matrix read MN-major: (64, rows, cols / 64),
+// boxes of 128 rows of two 64-element blocks (the smem image: block b's row r at
+// b * 16 KiB + r * 128 bytes, 128-byte swizzle).  Serves the transposed
+// weights of the backward's data-gradient GEMMs (W2^T: rows E*H, cols I; W13^T:
+// rows E*2I, cols H) and the token-row operands of its weight gradients.
+static bool make_tmap_mn(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols) {
+    const cuuint64_t dims[3] = {(cuuint64_t)kBK, rows, cols / kBK};
+    const cuuint64_t strides[2] = {cols * 2, (cuuint64_t)kBK * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kBK, 128u, 2u};
+    return make_tmap_kchunks(m, ptr, false, 3, dims, strides, box);
+}
+
+cudaError_t launch_wgrad_tcgen05(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
+                                 const int32_t *expert_offsets, int E, int M, int N, float *out,
+                                 int accumulate, uint32_t *status, cudaStream_t s, int num_sms);
+
+// Backward of the bf16 grouped SwiGLU FFN over one receive buffer (rows of
+// expert e: [expert_offsets[e], expert_offsets[e+1])), for incoming dy:
+//   1. g | u = W13[e] . xr^T                   (the forward's GEMM1, stored [n, 2I])
+//   2. dh = W2[e]^T . dy^T; h = silu(g) u, dg = dh u s (1 + g (1 - s)),
+//      du = dh silu(g) with s = sigmoid(g)     (h [n, I], dg | du [n, 2I])
+//   3. dxr = W13[e]^T . [dg | du]^T            ([n, H])
+//   4. dW2[e] (+)= dy^T h,  dW13[e] (+)= [dg | du]^T xr   (fp32)
+// counters: three work counters (launches 1-3).
+cudaError_t launch_ffn_tcgen05_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                   const int32_t *expert_offsets, const void *w13, const void *w2,
+                                   void *gu, void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                   int accumulate, uint32_t *status, uint32_t *counters,
+                                   cudaStream_t s, int num_sms) {
+    if (n_rows <= 0) return cudaSuccess;
+    cudaError_t cerr = cudaMemsetAsync(counters, 0, 3 * sizeof(uint32_t), s);
+    if (cerr != cudaSuccess) return cerr;
+    const uint64_t H = c.H, I = c.I, E = c.E, n = (uint64_t)n_rows;
+    CUtensorMap tw13, tx, txs, tw2t, tdy, tdys, tw13t, tdgu, tdgus;
+    CUtensorMap a_dy, b_h, a_dgu, b_xr;
+    if (!make_tmap_w13(&tw13, w13, E, I, H) || !make_tmap_rows(&tx, xr, n, H, kTileTok / 2) ||
+        !make_tmap_rows(&txs, xr, n, H, kSmallBoxRows) || !make_tmap_mn(&tw2t, w2, E * H, I) ||
+        !make_tmap_rows(&tdy, dy, n, H, kTileTok / 2) || !make_tmap_rows(&tdys, dy, n, H, kSmallBoxRows) ||
+        !make_tmap_mn(&tw13t, w13, E * 2 * I, H) || !make_tmap_rows(&tdgu, dgu, n, 2 * I, kTileTok / 2) ||
+        !make_tmap_rows(&tdgus, dgu, n, 2 * I, kSmallBoxRows) || !make_tmap_mn(&a_dy, dy, n, H) ||
+        !make_tmap_mn(&b_h, h, n, I) || !make_tmap_mn(&a_dgu, dgu, n, 2 * I) || !make_tmap_mn(&b_xr, xr, n, H))
+        return cudaErrorNotSupported;
+
+    FfnGemmParams P1, P2;
+    ffn_params(c, expert_offsets, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, status, P1, P2);
+    // 1. the forward's GEMM1, g and u stored side by side
+    FfnGemmParams Pa = P1;
+    Pa.out = gu;
+    Pa.out_ld = 2 * c.I;
+    Pa.half_cols = c.I;
+    cudaError_t err = launch_gemm<kEpiStoreGU, false>(tw13, tx, txs, Pa, ffn_grid(c, n_rows, Pa, num_sms),
+                                                      counters, s);
+    if (err != cudaSuccess) return err;
+    // 2. dh over K = H with W2 read transposed; 128 features of I per CTA
+    FfnGemmParams Pb = P2;
+    Pb.K = c.H;
+    Pb.feat_per_cta = kRowsPerCta;
+    Pb.n_fblocks = (c.I + 2 * kRowsPerCta - 1) / (2 * kRowsPerCta);
+    Pb.w_rows_per_expert = c.H;
+    Pb.out_cols = c.I;
+    Pb.out = h;
+    Pb.out_ld = 2 * c.I;
+    Pb.half_cols = c.I;
+    Pb.gu = static_cast<const __nv_bfloat16 *>(gu);
+    Pb.out2 = static_cast<__nv_bfloat16 *>(dgu);
+    err = launch_gemm<kEpiSwiGLUBwd, false, true>(tw2t, tdy, tdys, Pb, ffn_grid(c, n_rows, Pb, num_sms),
+                                                  counters + 1, s);
+    if (err != cudaSuccess) return err;
+    // 3. dxr over K = 2I with W13 read transposed; 128 features of H per CTA
+    FfnGemmParams Pc = P2;
+    Pc.K = 2 * c.I;
+    Pc.feat_per_cta = kRowsPerCta;
+    Pc.n_fblocks = (c.H + 2 * kRowsPerCta - 1) / (2 * kRowsPerCta);
+    Pc.w_rows_per_expert = 2 * c.I;
+    Pc.out_cols = c.H;
+    Pc.out_ld = c.H;
+    Pc.out = dxr;
+    err = launch_gemm<kEpiStore, false, true>(tw13t, tdgu, tdgus, Pc, ffn_grid(c, n_rows, Pc, num_sms),
+                                              counters + 2, s);
+    if (err != cudaSuccess) return err;
+    // 4. the weight gradients
+    err = launch_wgrad_tcgen05(a_dy, b_h, expert_offsets, c.E, c.H, c.I, dw2, accumulate, status, s, num_sms);
+    if (err != cudaSuccess) return err;
+    return launch_wgrad_tcgen05(a_dgu, b_xr, expert_offsets, c.E, 2 * c.I, c.H, dw13, accumulate, status, s,
+                                num_sms);
 }
 
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,

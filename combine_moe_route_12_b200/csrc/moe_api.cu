@@ -53,6 +53,15 @@ cudaError_t launch_combine_bwd(const moe_config &c, const void *dout, const void
 cudaError_t launch_route_bwd(const moe_config &c, const int32_t *topk_idx, const float *topk_w,
                              const float *dw, float *dlogits, float *dbias, uint32_t *status,
                              cudaStream_t s);
+cudaError_t launch_ffn_tcgen05_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                   const int32_t *expert_offsets, const void *w13, const void *w2,
+                                   void *gu, void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                   int accumulate, uint32_t *status, uint32_t *counters,
+                                   cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                const int32_t *expert_offsets, const void *w13, const void *w2,
+                                void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                int accumulate, cudaStream_t s);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -389,6 +398,55 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
                               recv_slot, topk_w, out_reduce, stream);
     }
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn");
+}
+
+moe_status moe_grouped_swiglu_ffn_backward(const moe_config *cfg, int64_t n_rows, const void *xr,
+                                           const void *dy, const int32_t *expert_offsets,
+                                           const void *w13, const void *w2, void *gu, void *h,
+                                           void *dgu, void *dxr, float *dw13, float *dw2,
+                                           int32_t accumulate, void *ws, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (accumulate != 0 && accumulate != 1) return fail(MOE_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+    if (c.ffn_fp8) return fail(MOE_ERR_UNSUPPORTED, "the FFN backward runs on bf16 or fp32 weights (ffn_fp8 = 0)");
+    if (!expert_offsets || !w13 || !w2 || !dw13 || !dw2) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (n_rows > 0 && (!xr || !dy || !h || !dgu || !dxr || (c.dtype == MOE_BF16 && !gu)))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const void *ptrs[9] = {xr, dy, w13, w2, gu, h, dgu, dxr, dw13};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    if (!aligned(dw2, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err;
+    if (c.dtype == MOE_BF16) {
+        int dev = 0, major = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (major != 10)
+            return fail(MOE_ERR_UNSUPPORTED, "the bf16 FFN backward uses tcgen05 and needs sm_100 (got major %d)", major);
+        if (n_rows == 0) {
+            // no rows: the weight gradients are zero (or unchanged when accumulating)
+            err = cudaSuccess;
+            if (!accumulate) {
+                err = cudaMemsetAsync(dw13, 0, sizeof(float) * (size_t)c.E * 2 * c.I * c.H, stream);
+                if (err == cudaSuccess)
+                    err = cudaMemsetAsync(dw2, 0, sizeof(float) * (size_t)c.E * c.H * c.I, stream);
+            }
+        } else {
+            err = launch_ffn_tcgen05_bwd(c, n_rows, xr, dy, expert_offsets, w13, w2, gu, h, dgu, dxr, dw13,
+                                         dw2, accumulate, ws_at<uint32_t>(ws, L.status),
+                                         ws_at<uint32_t>(ws, L.ffn_ctr), stream, current_num_sms());
+            if (err == cudaErrorNotSupported)
+                return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+        }
+    } else {
+        err = launch_ffn_simt_bwd(c, n_rows, xr, dy, expert_offsets, w13, w2, h, dgu, dxr, dw13, dw2,
+                                  accumulate, stream);
+    }
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn_backward");
 }
 
 moe_status moe_quantize_fp8_rows(int64_t rows, int32_t cols, int32_t in_dtype, const void *in,

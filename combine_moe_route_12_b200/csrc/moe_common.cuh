@@ -377,4 +377,65 @@ __host__ __device__ constexpr uint32_t make_idesc_e4m3_f32(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// kind::f16 with bf16 A and B and an fp32 accumulator, with the major-ness of
+// each operand: bit 15 set = A is MN-major, bit 16 set = B is MN-major.
+__host__ __device__ constexpr uint32_t make_idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+    return make_idesc_bf16_f32(M, N) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
+}
+
+// Shared-memory descriptor of an MN-major operand stored with the 128-byte
+// swizzle: each 128-byte row holds 64 consecutive M (or N) elements of one k,
+// 8 consecutive k rows form a 1024-byte swizzle atom (stride byte offset 1024),
+// and the next 64 M elements start `mn_block_bytes` further on (leading byte
+// offset).  An MMA k-step of 16 k rows starts 2048 bytes after the previous one.
+__device__ __forceinline__ uint64_t make_sw128_desc_mn(uint32_t smem_addr, uint32_t mn_block_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+// ---------------------------------------------------------------- single-CTA tcgen05
+// TMA load into this CTA's shared memory, completion counted on this CTA's mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *mbar,
+                                            int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(mbar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_1(uint32_t *smem_dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(smem_dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_1() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_1(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A * B^T on this CTA alone (M = 64 or 128).
+__device__ __forceinline__ void tc_mma_f16_1(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrives once on this CTA's mbarrier when all tcgen05 ops issued so far by
+// this thread complete.
+__device__ __forceinline__ void tc_commit_1(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (the tensor core's operand fetch, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 }  // namespace moe

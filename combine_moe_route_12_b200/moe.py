@@ -74,6 +74,7 @@ _decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
 _decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
 _decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
 _decl("moe_permute_quantize_fp8", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_grouped_swiglu_ffn_backward", _I32, _CFG, ctypes.c_int64, *([_P] * 12), _I32, _P, _P)
 _decl("moe_combine_backward", _I32, _CFG, _P, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_route_backward", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute_backward", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
@@ -230,6 +231,16 @@ def moe_permute_quantize_fp8(cfg, x, pos, tok_begin, tok_count, xr_q, x_scale, s
     """Kept token rows of x quantised to E4M3 codes and written to their receive rows."""
     _check(_lib.moe_permute_quantize_fp8(ctypes.byref(cfg), _ptr(x), _ptr(pos), tok_begin,
                                          tok_count, _ptr(xr_q), _ptr(x_scale), _stream(stream)))
+
+
+def moe_grouped_swiglu_ffn_backward(cfg, n_rows, xr, dy, expert_offsets, w13, w2, gu, h, dgu, dxr,
+                                    dw13, dw2, accumulate, ws, stream=None):
+    """The expert FFN's backward over one receive buffer: dxr, the recomputed h,
+    [dg | du], and the fp32 weight gradients (written, or added to with accumulate)."""
+    _check(_lib.moe_grouped_swiglu_ffn_backward(
+        ctypes.byref(cfg), n_rows, _ptr(xr), _ptr(dy), _ptr(expert_offsets), _ptr(w13), _ptr(w2),
+        _ptr(gu), _ptr(h), _ptr(dgu), _ptr(dxr), _ptr(dw13), _ptr(dw2), int(accumulate), _ptr(ws),
+        _stream(stream)))
 
 
 def moe_combine_backward(cfg, dout, y, pos, topk_w, tok_begin, tok_count, dy, dw, stream=None):

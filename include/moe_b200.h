@@ -21,8 +21,9 @@
  * fixed library array; moe_quantize_fp8_rows, moe_permute_quantize_fp8 and
  * moe_grouped_swiglu_ffn_fp8, the expert FFN on E4M3 codes with UE8M0 row
  * scales (cfg->ffn_fp8);
- * moe_combine_backward, moe_route_backward and moe_permute_backward, the
- * backward's row passes; moe_watchdog_selftest, which makes a bounded wait run
+ * moe_grouped_swiglu_ffn_backward, the expert FFN's backward (data and
+ * weight gradients); moe_combine_backward, moe_route_backward and
+ * moe_permute_backward, the backward's row passes; moe_watchdog_selftest, which makes a bounded wait run
  * out on purpose; moe_device_status, the device-side error bits.
  *
  * Sources (restated, not copied):
@@ -391,8 +392,7 @@ moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32
 /*
  * Backward steps that are row passes (axolotl ExpertParallelArgs,
  * expert_parallel_save_dispatch: the layer's backward reuses the saved routing
- * top-k, keep mask and layout; the expert FFN's backward is not part of this
- * library yet).  For L = <dout, out>:
+ * top-k, keep mask and layout).  For L = <dout, out>:
  *
  * moe_combine_backward, for t in [tok_begin, tok_begin + tok_count):
  *   dy[pos[t - tok_begin, j]] = topk_w[t, j] * dout[t]     (cfg->dtype, rounded once)
@@ -413,6 +413,35 @@ moe_status moe_shared_expert_ffn(const moe_config *cfg, int32_t tok_begin, int32
  *   order, rounded once to cfg->dtype (zeros for a token with every slot
  *   dropped); dxr [N_max, H], dx [T, H].
  */
+/*
+ * Backward of step 5, the grouped SwiGLU FFN, over one receive buffer (axolotl
+ * ExpertParallelArgs, expert_parallel_save_dispatch: the backward of the
+ * expert GEMMs under activation checkpointing; the pages give no formulas, the
+ * gradient below is that of step 5's function).  For each expert e and row p
+ * in [expert_offsets[e], expert_offsets[e+1]) with incoming gradient dy[p]:
+ *   g, u   = W13[e, 0:I] . xr[p], W13[e, I:2I] . xr[p]   (recomputed)
+ *   dh     = W2[e]^T . dy[p]
+ *   h[p]   = silu(g) * u,  s = sigmoid(g)
+ *   dg     = dh * u * s * (1 + g * (1 - s)),   du = dh * silu(g)
+ *   dxr[p] = W13[e]^T . [dg | du]
+ *   dW2[e]  (+)= sum over the expert's rows of dy[p] (x) h[p]       [H, I]
+ *   dW13[e] (+)= sum over the expert's rows of [dg | du][p] (x) xr[p] [2I, H]
+ *   xr, dy, dxr [n_rows, H]; h [n_rows, I] and dgu [n_rows, 2I] (dg then du)
+ *   are outputs kept for the caller; gu [n_rows, 2I] is scratch (g then u; bf16
+ *   only, may be NULL for MOE_F32); all in cfg->dtype.
+ *   dw13 [E, 2I, H] and dw2 [E, H, I]: fp32, written (accumulate = 0: experts
+ *   without rows get zeros) or added to (accumulate = 1).
+ * MOE_BF16 runs five tcgen05 launches (g | u; dh with the SwiGLU backward;
+ * dxr; the two weight gradients, fp32 accumulation in TMEM, h, dg and du
+ * rounded to bf16 where stored); MOE_F32 runs fp32 FMA on the CUDA cores.
+ * cfg->ffn_fp8 = 1 is MOE_ERR_UNSUPPORTED.  ws: moe_workspace_bytes(cfg).
+ */
+moe_status moe_grouped_swiglu_ffn_backward(const moe_config *cfg, int64_t n_rows, const void *xr,
+                                           const void *dy, const int32_t *expert_offsets,
+                                           const void *w13, const void *w2, void *gu, void *h,
+                                           void *dgu, void *dxr, float *dw13, float *dw2,
+                                           int32_t accumulate, void *ws, cudaStream_t stream);
+
 moe_status moe_combine_backward(const moe_config *cfg, const void *dout, const void *y,
                                 const int32_t *pos, const float *topk_w, int32_t tok_begin,
                                 int32_t tok_count, void *dy, float *dw, cudaStream_t stream);
