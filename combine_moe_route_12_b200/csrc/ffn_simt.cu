@@ -168,24 +168,43 @@ __global__ void __launch_bounds__(kSimtThreads) ffn_simt_bwd_dx_kernel(
     }
 }
 
-// out[e][m, n] (+)= sum over the expert's rows p of a[p, m] * b[p, n]
+// out[e][m, n] (+)= sum over the expert's rows p of a[p, m] * b[p, n], over
+// n_seg segments seg_rows rows apart (segment s: offsets offs + s * (E + 1))
 __global__ void __launch_bounds__(kSimtThreads) ffn_simt_wgrad_kernel(
-    int M, int N, const int32_t *__restrict__ offs, const float *__restrict__ a,
-    const float *__restrict__ b, float *__restrict__ out, int accumulate) {
+    int E, int M, int N, int n_seg, long long seg_rows, const int32_t *__restrict__ offs,
+    const float *__restrict__ a, const float *__restrict__ b, float *__restrict__ out, int accumulate) {
     const int m = blockIdx.x, e = blockIdx.y;
-    const int p0 = offs[e], p1 = offs[e + 1];
     float *o = out + ((size_t)e * M + m) * N;
     for (int n = threadIdx.x; n < N; n += blockDim.x) {
         float acc = 0.f;
-        for (int p = p0; p < p1; ++p) acc = __fmaf_rn(a[(size_t)p * M + m], b[(size_t)p * N + n], acc);
+        for (int sg = 0; sg < n_seg; ++sg) {
+            const int32_t *os = offs + (size_t)sg * (E + 1);
+            const size_t base = (size_t)sg * seg_rows;
+            for (int p = os[e]; p < os[e + 1]; ++p)
+                acc = __fmaf_rn(a[(base + p) * M + m], b[(base + p) * N + n], acc);
+        }
         o[n] = accumulate ? o[n] + acc : acc;
     }
 }
 
-cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
-                                const int32_t *expert_offsets, const void *w13, const void *w2,
-                                void *h, void *dgu, void *dxr, float *dw13, float *dw2,
-                                int accumulate, cudaStream_t s) {
+cudaError_t launch_ffn_simt_wgrad(const moe_config &c, int n_seg, int64_t seg_rows,
+                                  const int32_t *expert_offsets, const void *xr, const void *dy,
+                                  const void *h, const void *dgu, float *dw13, float *dw2,
+                                  int accumulate, cudaStream_t s) {
+    ffn_simt_wgrad_kernel<<<dim3(c.H, c.E), kSimtThreads, 0, s>>>(
+        c.E, c.H, c.I, n_seg, seg_rows, expert_offsets, static_cast<const float *>(dy),
+        static_cast<const float *>(h), dw2, accumulate);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    ffn_simt_wgrad_kernel<<<dim3(2 * c.I, c.E), kSimtThreads, 0, s>>>(
+        c.E, 2 * c.I, c.H, n_seg, seg_rows, expert_offsets, static_cast<const float *>(dgu),
+        static_cast<const float *>(xr), dw13, accumulate);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_simt_dgrad(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                  const int32_t *expert_offsets, const void *w13, const void *w2,
+                                  void *h, void *dgu, void *dxr, cudaStream_t s) {
     if (n_rows > 0x7fffffffLL) return cudaErrorInvalidValue;
     const float *x = static_cast<const float *>(xr), *d = static_cast<const float *>(dy);
     if (n_rows > 0) {
@@ -199,14 +218,17 @@ cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void 
             static_cast<const float *>(w13), static_cast<float *>(dxr));
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
-    // the weight gradients run whatever n_rows is: experts without rows get zeros
-    ffn_simt_wgrad_kernel<<<dim3(c.H, c.E), kSimtThreads, 0, s>>>(
-        c.H, c.I, expert_offsets, d, static_cast<const float *>(h), dw2, accumulate);
-    cudaError_t err = cudaGetLastError();
+    return cudaSuccess;
+}
+
+cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                const int32_t *expert_offsets, const void *w13, const void *w2,
+                                void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                int accumulate, cudaStream_t s) {
+    cudaError_t err = launch_ffn_simt_dgrad(c, n_rows, xr, dy, expert_offsets, w13, w2, h, dgu, dxr, s);
     if (err != cudaSuccess) return err;
-    ffn_simt_wgrad_kernel<<<dim3(2 * c.I, c.E), kSimtThreads, 0, s>>>(
-        2 * c.I, c.H, expert_offsets, static_cast<const float *>(dgu), x, dw13, accumulate);
-    return cudaGetLastError();
+    // the weight gradients run whatever n_rows is: experts without rows get zeros
+    return launch_ffn_simt_wgrad(c, 1, n_rows, expert_offsets, xr, dy, h, dgu, dw13, dw2, accumulate, s);
 }
 
 }  // namespace moe

@@ -807,34 +807,31 @@ static bool make_tmap_mn(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_
 }
 
 cudaError_t launch_wgrad_tcgen05(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
-                                 const int32_t *expert_offsets, int E, int M, int N, float *out,
-                                 int accumulate, uint32_t *status, cudaStream_t s, int num_sms);
+                                 const int32_t *expert_offsets, int n_seg, long long seg_rows, int E,
+                                 int M, int N, float *out, int accumulate, uint32_t *status,
+                                 cudaStream_t s, int num_sms);
 
-// Backward of the bf16 grouped SwiGLU FFN over one receive buffer (rows of
-// expert e: [expert_offsets[e], expert_offsets[e+1])), for incoming dy:
+// Data gradients of the bf16 grouped SwiGLU FFN over one receive buffer (rows
+// of expert e: [expert_offsets[e], expert_offsets[e+1])), for incoming dy:
 //   1. g | u = W13[e] . xr^T                   (the forward's GEMM1, stored [n, 2I])
 //   2. dh = W2[e]^T . dy^T; h = silu(g) u, dg = dh u s (1 + g (1 - s)),
 //      du = dh silu(g) with s = sigmoid(g)     (h [n, I], dg | du [n, 2I])
 //   3. dxr = W13[e]^T . [dg | du]^T            ([n, H])
-//   4. dW2[e] (+)= dy^T h,  dW13[e] (+)= [dg | du]^T xr   (fp32)
-// counters: three work counters (launches 1-3).
-cudaError_t launch_ffn_tcgen05_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
-                                   const int32_t *expert_offsets, const void *w13, const void *w2,
-                                   void *gu, void *h, void *dgu, void *dxr, float *dw13, float *dw2,
-                                   int accumulate, uint32_t *status, uint32_t *counters,
-                                   cudaStream_t s, int num_sms) {
+// counters: three work counters.
+cudaError_t launch_ffn_tcgen05_dgrad(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                     const int32_t *expert_offsets, const void *w13, const void *w2,
+                                     void *gu, void *h, void *dgu, void *dxr, uint32_t *status,
+                                     uint32_t *counters, cudaStream_t s, int num_sms) {
     if (n_rows <= 0) return cudaSuccess;
     cudaError_t cerr = cudaMemsetAsync(counters, 0, 3 * sizeof(uint32_t), s);
     if (cerr != cudaSuccess) return cerr;
     const uint64_t H = c.H, I = c.I, E = c.E, n = (uint64_t)n_rows;
     CUtensorMap tw13, tx, txs, tw2t, tdy, tdys, tw13t, tdgu, tdgus;
-    CUtensorMap a_dy, b_h, a_dgu, b_xr;
     if (!make_tmap_w13(&tw13, w13, E, I, H) || !make_tmap_rows(&tx, xr, n, H, kTileTok / 2) ||
         !make_tmap_rows(&txs, xr, n, H, kSmallBoxRows) || !make_tmap_mn(&tw2t, w2, E * H, I) ||
         !make_tmap_rows(&tdy, dy, n, H, kTileTok / 2) || !make_tmap_rows(&tdys, dy, n, H, kSmallBoxRows) ||
         !make_tmap_mn(&tw13t, w13, E * 2 * I, H) || !make_tmap_rows(&tdgu, dgu, n, 2 * I, kTileTok / 2) ||
-        !make_tmap_rows(&tdgus, dgu, n, 2 * I, kSmallBoxRows) || !make_tmap_mn(&a_dy, dy, n, H) ||
-        !make_tmap_mn(&b_h, h, n, I) || !make_tmap_mn(&a_dgu, dgu, n, 2 * I) || !make_tmap_mn(&b_xr, xr, n, H))
+        !make_tmap_rows(&tdgus, dgu, n, 2 * I, kSmallBoxRows))
         return cudaErrorNotSupported;
 
     FfnGemmParams P1, P2;
@@ -871,14 +868,44 @@ cudaError_t launch_ffn_tcgen05_bwd(const moe_config &c, int64_t n_rows, const vo
     Pc.out_cols = c.H;
     Pc.out_ld = c.H;
     Pc.out = dxr;
-    err = launch_gemm<kEpiStore, false, true>(tw13t, tdgu, tdgus, Pc, ffn_grid(c, n_rows, Pc, num_sms),
-                                              counters + 2, s);
+    return launch_gemm<kEpiStore, false, true>(tw13t, tdgu, tdgus, Pc, ffn_grid(c, n_rows, Pc, num_sms),
+                                               counters + 2, s);
+}
+
+// Weight gradients over n_seg receive buffers laid one after another, seg_rows
+// rows apart (segment s: expert offsets expert_offsets + s * (E + 1)), in one
+// pass: dW2[e] (+)= dy^T h and dW13[e] (+)= [dg | du]^T xr over the expert's
+// rows of every segment (fp32).  xr, dy [n_seg * seg_rows, H], h [.., I],
+// dgu [.., 2I].
+cudaError_t launch_ffn_tcgen05_wgrad(const moe_config &c, int n_seg, int64_t seg_rows,
+                                     const int32_t *expert_offsets, const void *xr, const void *dy,
+                                     const void *h, const void *dgu, float *dw13, float *dw2,
+                                     int accumulate, uint32_t *status, cudaStream_t s, int num_sms) {
+    const uint64_t rows = (uint64_t)n_seg * (uint64_t)seg_rows;
+    if (rows == 0) return cudaErrorInvalidValue;
+    CUtensorMap a_dy, b_h, a_dgu, b_xr;
+    if (!make_tmap_mn(&a_dy, dy, rows, c.H) || !make_tmap_mn(&b_h, h, rows, c.I) ||
+        !make_tmap_mn(&a_dgu, dgu, rows, 2 * (uint64_t)c.I) || !make_tmap_mn(&b_xr, xr, rows, c.H))
+        return cudaErrorNotSupported;
+    cudaError_t err = launch_wgrad_tcgen05(a_dy, b_h, expert_offsets, n_seg, seg_rows, c.E, c.H, c.I, dw2,
+                                           accumulate, status, s, num_sms);
     if (err != cudaSuccess) return err;
-    // 4. the weight gradients
-    err = launch_wgrad_tcgen05(a_dy, b_h, expert_offsets, c.E, c.H, c.I, dw2, accumulate, status, s, num_sms);
+    return launch_wgrad_tcgen05(a_dgu, b_xr, expert_offsets, n_seg, seg_rows, c.E, 2 * c.I, c.H, dw13,
+                                accumulate, status, s, num_sms);
+}
+
+// The whole backward of one receive buffer: data gradients, then weight gradients.
+cudaError_t launch_ffn_tcgen05_bwd(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                   const int32_t *expert_offsets, const void *w13, const void *w2,
+                                   void *gu, void *h, void *dgu, void *dxr, float *dw13, float *dw2,
+                                   int accumulate, uint32_t *status, uint32_t *counters,
+                                   cudaStream_t s, int num_sms) {
+    if (n_rows <= 0) return cudaSuccess;
+    cudaError_t err = launch_ffn_tcgen05_dgrad(c, n_rows, xr, dy, expert_offsets, w13, w2, gu, h, dgu, dxr,
+                                               status, counters, s, num_sms);
     if (err != cudaSuccess) return err;
-    return launch_wgrad_tcgen05(a_dgu, b_xr, expert_offsets, c.E, 2 * c.I, c.H, dw13, accumulate, status, s,
-                                num_sms);
+    return launch_ffn_tcgen05_wgrad(c, 1, n_rows, expert_offsets, xr, dy, h, dgu, dw13, dw2, accumulate,
+                                    status, s, num_sms);
 }
 
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,

@@ -1,22 +1,25 @@
 // Weight gradients of the grouped SwiGLU FFN (the backward of the expert
 // GEMMs; axolotl ExpertParallelArgs, expert_parallel_save_dispatch: the
-// layer's backward under activation checkpointing).  For every expert e with
-// receive rows [off_e, off_e + m_e):
+// layer's backward under activation checkpointing).  For every expert e and
+// its receive rows in each of n_seg segments (the token chunks of a layer
+// pass: segment s holds rows [s * seg_rows + off_s[e], s * seg_rows +
+// off_s[e+1])):
 //   dW2[e]  [H, I]  = sum over its rows p of dy[p] (x) h[p]
 //   dW13[e] [2I, H] = sum over its rows p of [dg | du][p] (x) xr[p]
 // i.e. out[e] = A_e^T B_e with A = the row-major [rows, M] operand and B the
-// row-major [rows, N] operand restricted to the expert's rows.  The reduction
-// runs over token rows, so both operands are read MN-major: a ring stage holds
-// 128 token rows of 128 output rows (A) and of 128 output columns (B), each as
-// two 64-element blocks of 128-byte rows brought by one 3-D TMA box.
+// row-major [rows, N] operand restricted to the expert's rows.  One pass over
+// all segments writes each fp32 gradient once.  The reduction runs over token
+// rows, so both operands are read MN-major: a ring stage holds 128 token rows
+// of 128 output rows (A) and of 128 output columns (B), each as two 64-element
+// blocks of 128-byte rows brought by one 3-D TMA box.
 //
 // One CTA per SM, tiles (expert, 128 output rows, 128 output columns) dealt
 // round-robin (tile = CTA + i * grid), expert by expert, so the tiles that
 // read one expert's rows run side by side and share them through L2.  Warp 8
 // (one lane) streams the ring with TMA; warp 9 waits for each stage and issues
 // the single-CTA tcgen05.mma (bf16 -> fp32, M = N = 128) into one of two TMEM
-// accumulators.  An expert's rows rarely fill the last stage: the MMA stops
-// at the last 16-row k-step that holds a row of the expert, and the warp
+// accumulators.  An expert's rows rarely fill a segment's last stage: the MMA
+// stops at the last 16-row k-step that holds a row of the expert, and the warp
 // first zeroes that step's rows past the expert (they belong to the next
 // expert, or lie past the valid rows) in both operands.  Warps 0-7 drain TMEM
 // (warps q and q + 4 share lane quadrant q and take alternate 64-column
@@ -44,7 +47,9 @@ constexpr uint32_t kWgTmemCols = 2 * kWgTile;             // two 128-column accu
 constexpr int kWgPad = 33;                                // staging row stride in floats
 
 struct WgradParams {
-    const int32_t *expert_offsets;
+    const int32_t *expert_offsets;   // [n_seg][E + 1]
+    int n_seg;
+    long long seg_rows;              // row distance between the segments' buffers
     int E;
     int M, N;              // out[e] is [M, N], row-major
     int m_blocks, n_blocks;
@@ -64,7 +69,7 @@ struct WgSmem {
 };
 
 struct WgTile {
-    int e, mb, nb, p0, rows;
+    int e, mb, nb, rows;   // rows: the expert's rows over all segments
 };
 
 __device__ __forceinline__ WgTile wg_tile(int t, const WgradParams &P) {
@@ -74,9 +79,19 @@ __device__ __forceinline__ WgTile wg_tile(int t, const WgradParams &P) {
     const int r = t - w.e * per_e;
     w.mb = r / P.n_blocks;
     w.nb = r - w.mb * P.n_blocks;
-    w.p0 = P.expert_offsets[w.e];
-    w.rows = P.expert_offsets[w.e + 1] - w.p0;
+    w.rows = 0;
+    for (int sg = 0; sg < P.n_seg; ++sg) {
+        const int32_t *o = P.expert_offsets + (size_t)sg * (P.E + 1) + w.e;
+        w.rows += o[1] - o[0];
+    }
     return w;
+}
+
+// First row and row count of the expert's part of segment sg.
+__device__ __forceinline__ void wg_segment(const WgradParams &P, int e, int sg, int &p0, int &rows) {
+    const int32_t *o = P.expert_offsets + (size_t)sg * (P.E + 1) + e;
+    p0 = (int)(sg * P.seg_rows) + o[0];
+    rows = o[1] - o[0];
 }
 
 __global__ void __launch_bounds__(kWgThreads, 1) wgrad_tcgen05_kernel(
@@ -116,16 +131,20 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_tcgen05_kernel(
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const WgTile w = wg_tile(t, P);
-                const int nk = (w.rows + kWgRows - 1) / kWgRows;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-                    unsigned char *st = ring + stage * kWgStageBytes;
-                    mbar_arrive_expect_tx(&S->full[stage], kWgStageBytes);
-                    const int row = w.p0 + kb * kWgRows;
-                    tma_load_3d(st, &tmap_a, &S->full[stage], 0, row, w.mb * 2);
-                    tma_load_3d(st + kWgOpBytes, &tmap_b, &S->full[stage], 0, row, w.nb * 2);
-                    ++issued;
-                    if (++stage == kWgStages) { stage = 0; phase ^= 1u; }
+                for (int sg = 0; sg < P.n_seg && ok; ++sg) {
+                    int p0, rows;
+                    wg_segment(P, w.e, sg, p0, rows);
+                    const int nk = (rows + kWgRows - 1) / kWgRows;
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                        unsigned char *st = ring + stage * kWgStageBytes;
+                        mbar_arrive_expect_tx(&S->full[stage], kWgStageBytes);
+                        const int row = p0 + kb * kWgRows;
+                        tma_load_3d(st, &tmap_a, &S->full[stage], 0, row, w.mb * 2);
+                        tma_load_3d(st + kWgOpBytes, &tmap_b, &S->full[stage], 0, row, w.nb * 2);
+                        ++issued;
+                        if (++stage == kWgStages) { stage = 0; phase ^= 1u; }
+                    }
                 }
             }
             if (!ok) {
@@ -152,42 +171,48 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_tcgen05_kernel(
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const WgTile w = wg_tile(t, P);
-            const int nk = (w.rows + kWgRows - 1) / kWgRows;
             // lane 0 waits and tells the warp, so that the lanes stay together
             bool got = lane == 0 ? mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag) : true;
             if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d = tmem_base + (uint32_t)(acc * kWgTile);
-            for (int kb = 0; kb < nk; ++kb) {
-                got = lane == 0 ? mbar_wait_bounded(&S->full[stage], phase, abort_flag) : true;
-                if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
-                tc_fence_after();
-                unsigned char *st = ring + stage * kWgStageBytes;
-                const int v = min(kWgRows, w.rows - kb * kWgRows);   // rows of the expert in the stage
-                const int ksteps = (v + 15) >> 4;
-                if (v & 15) {
-                    // zero rows [v, 16 * ksteps) of both operands' two blocks (128 bytes a row)
-                    const int nz = 16 * ksteps - v;
-                    for (int i = lane; i < 4 * nz * 8; i += 32) {
-                        const int region = i / (nz * 8), rem = i - region * nz * 8;
-                        const int row = v + rem / 8, chunk = rem & 7;
-                        uint4 *dst = reinterpret_cast<uint4 *>(st + region * kWgBlockBytes + row * 128) + chunk;
-                        *dst = make_uint4(0u, 0u, 0u, 0u);
+            bool first = true;   // the tile's first MMA overwrites the accumulator
+            for (int sg = 0; sg < P.n_seg && ok; ++sg) {
+                int p0, rows;
+                wg_segment(P, w.e, sg, p0, rows);
+                const int nk = (rows + kWgRows - 1) / kWgRows;
+                for (int kb = 0; kb < nk; ++kb) {
+                    got = lane == 0 ? mbar_wait_bounded(&S->full[stage], phase, abort_flag) : true;
+                    if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
+                    tc_fence_after();
+                    unsigned char *st = ring + stage * kWgStageBytes;
+                    const int v = min(kWgRows, rows - kb * kWgRows);   // rows of the expert in the stage
+                    const int ksteps = (v + 15) >> 4;
+                    if (v & 15) {
+                        // zero rows [v, 16 * ksteps) of both operands' two blocks (128 bytes a row)
+                        const int nz = 16 * ksteps - v;
+                        for (int i = lane; i < 4 * nz * 8; i += 32) {
+                            const int region = i / (nz * 8), rem = i - region * nz * 8;
+                            const int row = v + rem / 8, chunk = rem & 7;
+                            uint4 *dst = reinterpret_cast<uint4 *>(st + region * kWgBlockBytes + row * 128) + chunk;
+                            *dst = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
                     }
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    const uint32_t a0 = smem_u32(st), b0 = smem_u32(st + kWgOpBytes);
-                    for (int ks = 0; ks < ksteps; ++ks) {
-                        const uint64_t ad = make_sw128_desc_mn(a0 + ks * 2048, kWgBlockBytes);
-                        const uint64_t bd = make_sw128_desc_mn(b0 + ks * 2048, kWgBlockBytes);
-                        tc_mma_f16_1(d, ad, bd, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+                    __syncwarp();
+                    if (lane == 0) {
+                        const uint32_t a0 = smem_u32(st), b0 = smem_u32(st + kWgOpBytes);
+                        for (int ks = 0; ks < ksteps; ++ks) {
+                            const uint64_t ad = make_sw128_desc_mn(a0 + ks * 2048, kWgBlockBytes);
+                            const uint64_t bd = make_sw128_desc_mn(b0 + ks * 2048, kWgBlockBytes);
+                            tc_mma_f16_1(d, ad, bd, idesc, (first && ks == 0) ? 0u : 1u);
+                        }
+                        tc_commit_1(&S->empty[stage]);   // frees the stage once these MMAs are done
                     }
-                    tc_commit_1(&S->empty[stage]);   // frees the stage once these MMAs are done
+                    __syncwarp();
+                    first = false;
+                    if (++stage == kWgStages) { stage = 0; phase ^= 1u; }
                 }
-                __syncwarp();
-                if (++stage == kWgStages) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             if (lane == 0) tc_commit_1(&S->tmem_full[acc]);   // accumulator ready (or untouched: no rows)
@@ -267,14 +292,18 @@ size_t wgrad_tcgen05_smem() {
            sizeof(WgSmem) + 64;
 }
 
-// out[e] (+)= A_e^T B_e over the expert segments of expert_offsets; tmap_a and
-// tmap_b view A [rows, M] and B [rows, N] as (64, rows, M/64) with 128-row boxes
-// of two 64-element blocks (make_tmap_mn).
+// out[e] (+)= A_e^T B_e over the expert's rows in n_seg segments (segment s:
+// expert offsets expert_offsets + s * (E + 1), rows seg_rows * s further on);
+// tmap_a and tmap_b view A [rows, M] and B [rows, N] as (64, rows, M/64) with
+// 128-row boxes of two 64-element blocks (make_tmap_mn).
 cudaError_t launch_wgrad_tcgen05(const CUtensorMap &tmap_a, const CUtensorMap &tmap_b,
-                                 const int32_t *expert_offsets, int E, int M, int N, float *out,
-                                 int accumulate, uint32_t *status, cudaStream_t s, int num_sms) {
+                                 const int32_t *expert_offsets, int n_seg, long long seg_rows, int E,
+                                 int M, int N, float *out, int accumulate, uint32_t *status,
+                                 cudaStream_t s, int num_sms) {
     WgradParams P{};
     P.expert_offsets = expert_offsets;
+    P.n_seg = n_seg;
+    P.seg_rows = seg_rows;
     P.E = E;
     P.M = M;
     P.N = N;

@@ -62,6 +62,21 @@ cudaError_t launch_ffn_simt_bwd(const moe_config &c, int64_t n_rows, const void 
                                 const int32_t *expert_offsets, const void *w13, const void *w2,
                                 void *h, void *dgu, void *dxr, float *dw13, float *dw2,
                                 int accumulate, cudaStream_t s);
+cudaError_t launch_ffn_tcgen05_dgrad(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                     const int32_t *expert_offsets, const void *w13, const void *w2,
+                                     void *gu, void *h, void *dgu, void *dxr, uint32_t *status,
+                                     uint32_t *counters, cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_tcgen05_wgrad(const moe_config &c, int n_seg, int64_t seg_rows,
+                                     const int32_t *expert_offsets, const void *xr, const void *dy,
+                                     const void *h, const void *dgu, float *dw13, float *dw2,
+                                     int accumulate, uint32_t *status, cudaStream_t s, int num_sms);
+cudaError_t launch_ffn_simt_dgrad(const moe_config &c, int64_t n_rows, const void *xr, const void *dy,
+                                  const int32_t *expert_offsets, const void *w13, const void *w2,
+                                  void *h, void *dgu, void *dxr, cudaStream_t s);
+cudaError_t launch_ffn_simt_wgrad(const moe_config &c, int n_seg, int64_t seg_rows,
+                                  const int32_t *expert_offsets, const void *xr, const void *dy,
+                                  const void *h, const void *dgu, float *dw13, float *dw2,
+                                  int accumulate, cudaStream_t s);
 cudaError_t launch_ffn_simt(const moe_config &c, int64_t n_rows, const void *xr,
                             const int32_t *expert_offsets, const void *w13, const void *w2,
                             void *h, void *y, const int32_t *recv_token, const int32_t *recv_slot,
@@ -180,6 +195,57 @@ ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
     }
     F.total = off;
     return F;
+}
+
+// Backward workspace: scratch first; the rows the weight gradients read for
+// every chunk (receive rows when recomputed, dy, h, dg | du; chunk c's at rows
+// c * nmax), each chunk's expert offsets, one chunk slot of what is consumed
+// within the chunk, and the fp32 slot gradients of all T tokens.  With a shared
+// expert, its h and dg | du rows for all T tokens and a chunk slot of the rest.
+struct BackwardLayout {
+    size_t eoff;                          // int32 [n_chunks][E + 1]
+    size_t roff, recv_token, recv_slot, pos, splits;
+    size_t xr, h, dy, dgu;                // [n_chunks * nmax, .]
+    size_t y, gu, dxr;                    // [nmax, .]
+    size_t dw;                            // fp32 [T, k]
+    size_t hs, dgus;                      // [T, .]
+    size_t gus, dxs;                      // [tc, .]
+    size_t total;
+    int64_t nmax;
+    int tc;
+};
+
+BackwardLayout backward_layout(const moe_config &c) {
+    BackwardLayout B{};
+    const ScratchLayout L = scratch_layout(c);
+    size_t off = L.total;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + (bytes ? bytes : 1), 256); return o; };
+    B.tc = c.T / c.n_chunks;
+    B.nmax = max_rows(c, B.tc);
+    const size_t eb = c.dtype == MOE_F32 ? 4 : 2;
+    const size_t n = (size_t)(B.nmax > 0 ? B.nmax : 1), nall = n * c.n_chunks;
+    B.eoff = take(sizeof(int32_t) * (size_t)c.n_chunks * (c.E + 1));
+    B.roff = take(sizeof(int32_t) * (c.ep + 1));
+    B.recv_token = take(sizeof(int32_t) * n);
+    B.recv_slot = take(sizeof(int32_t) * n);
+    B.pos = take(sizeof(int32_t) * (size_t)B.tc * c.k);
+    B.splits = take(sizeof(int32_t) * (size_t)c.ep * c.ep);
+    B.xr = take(eb * nall * c.H);
+    B.h = take(eb * nall * c.I);
+    B.dy = take(eb * nall * c.H);
+    B.dgu = take(eb * nall * 2 * c.I);
+    B.y = take(eb * n * c.H);
+    B.gu = take(eb * n * 2 * c.I);
+    B.dxr = take(eb * n * c.H);
+    B.dw = take(sizeof(float) * (size_t)c.T * c.k);
+    if (c.shared_I > 0) {
+        B.hs = take(eb * (size_t)c.T * c.shared_I);
+        B.dgus = take(eb * (size_t)c.T * 2 * c.shared_I);
+        B.gus = take(eb * (size_t)B.tc * 2 * c.shared_I);
+        B.dxs = take(eb * (size_t)B.tc * c.H);
+    }
+    B.total = off;
+    return B;
 }
 
 // Per-thread, per-device pool of timing-free events for the chunked forward,
@@ -672,7 +738,8 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
                               const uint8_t *w13_scale, const uint8_t *w2_scale, void *out,
                               int32_t *topk_idx, float *topk_w, uint8_t *keep,
                               int32_t *splits_host, void *ws, cudaStream_t s_dispatch,
-                              cudaStream_t s_compute, const HostIO *io) {
+                              cudaStream_t s_compute, const HostIO *io, void *xr_save = nullptr,
+                              void *y_save = nullptr) {
     const ScratchLayout L = scratch_layout(c);
     uint32_t *status = ws_at<uint32_t>(ws, L.status);
     int32_t *counts = ws_at<int32_t>(ws, F.counts);
@@ -741,9 +808,13 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
         int32_t *recv_token = ws_at<int32_t>(ws, S.recv_token);
         int32_t *recv_slot = ws_at<int32_t>(ws, S.recv_slot);
         int32_t *pos = ws_at<int32_t>(ws, S.pos);
-        void *xr = ws_at<void>(ws, S.xr);
+        // the saved dispatch outputs ([AX] expert_parallel_save_dispatch): chunk
+        // ch's receive rows and expert outputs in the caller's buffers
+        const size_t save_off = (size_t)ch * F.nmax * c.H * eb;
+        void *xr = xr_save ? static_cast<char *>(xr_save) + save_off : ws_at<void>(ws, S.xr);
         void *h = ws_at<void>(ws, S.h);
-        void *y = c.reduce_dense ? nullptr : ws_at<void>(ws, S.y);
+        void *y = c.reduce_dense ? nullptr
+                  : y_save ? static_cast<char *>(y_save) + save_off : ws_at<void>(ws, S.y);
         MOE_TRY(launch_dispatch_layout(c, tb, tc, topk_idx, keep, eoff, ws_at<int32_t>(ws, S.roff),
                                        recv_token, recv_slot, pos, ws_at<int32_t>(ws, S.splits),
                                        splits_host ? splits_host + (size_t)ch * split_stride : nullptr,
@@ -839,6 +910,183 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
     return forward_run(c, forward_layout(c), logits, bias, x, w13, w2, w13_shared, w2_shared,
                        w13_scale, w2_scale, out, topk_idx, topk_w, keep, splits_host, ws,
                        s_dispatch, s_compute, nullptr);
+}
+
+moe_status moe_forward_chunked_save(const moe_config *cfg, const float *logits, const float *bias,
+                                    const void *x, const void *w13, const void *w2,
+                                    const void *w13_shared, const void *w2_shared, void *out,
+                                    int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                                    int32_t *splits_host, void *xr_save, void *y_save, void *ws,
+                                    cudaStream_t s_dispatch, cudaStream_t s_compute) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.ffn_fp8 || c.reduce_dense)
+        return fail(MOE_ERR_UNSUPPORTED, "saving the dispatch outputs needs ffn_fp8 = 0 and reduce_dense = 0");
+    if (c.T > 0 && (!logits || !x || !w13 || !w2 || !out || !topk_idx || !topk_w || !keep || !xr_save ||
+                    !y_save))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.T > 0 && c.shared_I > 0 && (!w13_shared || !w2_shared))
+        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs w13_shared and w2_shared");
+    if (!aligned(xr_save, 16) || !aligned(y_save, 16))
+        return fail(MOE_ERR_INVALID_ARG, "xr_save / y_save not 16-byte aligned");
+    if (c.T == 0) return MOE_OK;
+    return forward_run(c, forward_layout(c), logits, bias, x, w13, w2, w13_shared, w2_shared, nullptr,
+                       nullptr, out, topk_idx, topk_w, keep, splits_host, ws, s_dispatch, s_compute,
+                       nullptr, xr_save, y_save);
+}
+
+size_t moe_backward_workspace_bytes(const moe_config *cfg) {
+    if (moe_config_check(cfg) != MOE_OK) return 0;
+    return backward_layout(*cfg).total;
+}
+
+moe_status moe_layer_backward(const moe_config *cfg, const void *x, const void *dout,
+                              const void *w13, const void *w2, const void *w13_shared,
+                              const void *w2_shared, const int32_t *topk_idx, const float *topk_w,
+                              const uint8_t *keep, const void *xr_saved, const void *y_saved,
+                              void *dx, float *dlogits, float *dbias, float *dw13, float *dw2,
+                              float *dw13_shared, float *dw2_shared, int32_t accumulate, void *ws,
+                              cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.ffn_fp8 || c.reduce_dense)
+        return fail(MOE_ERR_UNSUPPORTED, "the layer backward needs ffn_fp8 = 0 and reduce_dense = 0");
+    if (accumulate != 0 && accumulate != 1) return fail(MOE_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+    if ((xr_saved == nullptr) != (y_saved == nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "xr_saved and y_saved are both given (saved) or both NULL (recompute)");
+    if (!w13 || !w2 || !dw13 || !dw2 || (c.T > 0 && (!x || !dout || !topk_idx || !topk_w || !keep || !dx ||
+                                                     !dlogits)))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const bool shared = c.shared_I > 0;
+    if (shared && (!w13_shared || !w2_shared || !dw13_shared || !dw2_shared))
+        return fail(MOE_ERR_INVALID_ARG, "shared_I > 0 needs the shared expert's weights and gradients");
+    const void *al[6] = {x, dout, xr_saved, y_saved, dx, w13};
+    for (const void *p : al)
+        if (p && !aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    if (c.dtype == MOE_BF16) {
+        int dev = 0, major = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (major != 10)
+            return fail(MOE_ERR_UNSUPPORTED, "the bf16 backward uses tcgen05 and needs sm_100 (got major %d)", major);
+    }
+    if (c.T == 0) return MOE_OK;
+    const ScratchLayout L = scratch_layout(c);
+    const BackwardLayout B = backward_layout(c);
+    uint32_t *status = ws_at<uint32_t>(ws, L.status);
+    uint32_t *ctr = ws_at<uint32_t>(ws, L.ffn_ctr);
+    const int nsm = current_num_sms();
+    const size_t eb = c.dtype == MOE_F32 ? 4 : 2;
+    const bool bf16 = c.dtype == MOE_BF16;
+    const int tc = B.tc;
+    const int64_t nrow = B.nmax > 0 ? B.nmax : 1;   // the row distance between chunks' rows
+    int32_t *pos = ws_at<int32_t>(ws, B.pos);
+    float *dw = ws_at<float>(ws, B.dw);
+    char *xr_all = xr_saved ? static_cast<char *>(const_cast<void *>(xr_saved)) : ws_at<char>(ws, B.xr);
+    char *h_all = ws_at<char>(ws, B.h), *dy_all = ws_at<char>(ws, B.dy), *dgu_all = ws_at<char>(ws, B.dgu);
+    moe_config cs = c;   // the shared expert: one expert of intermediate size shared_I
+    cs.E = 1;
+    cs.I = c.shared_I;
+    cs.capacity = -1;
+    int32_t *soff = ws_at<int32_t>(ws, L.shared_off);
+#define MOE_TRY(expr, where)                                   \
+    do {                                                       \
+        cudaError_t e_ = (expr);                               \
+        if (e_ == cudaErrorNotSupported)                       \
+            return fail(MOE_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable or rejected a tensor map", where); \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where);    \
+    } while (0)
+    for (int ch = 0; ch < c.n_chunks; ++ch) {
+        const int tb = ch * tc;
+        int32_t *eoff = ws_at<int32_t>(ws, B.eoff) + (size_t)ch * (c.E + 1);
+        // the layout again, from the saved routing and keep mask (index work only)
+        MOE_TRY(launch_dispatch_layout(c, tb, tc, topk_idx, keep, eoff, ws_at<int32_t>(ws, B.roff),
+                                       ws_at<int32_t>(ws, B.recv_token), ws_at<int32_t>(ws, B.recv_slot), pos,
+                                       ws_at<int32_t>(ws, B.splits), nullptr, ws, B.nmax, stream, nsm),
+                "dispatch_layout");
+        const size_t row0 = (size_t)ch * nrow;
+        void *xr = xr_all + row0 * c.H * eb;
+        void *h = h_all + row0 * c.I * eb, *dy = dy_all + row0 * c.H * eb, *dgu = dgu_all + row0 * 2 * c.I * eb;
+        const void *y;
+        if (y_saved) {
+            y = static_cast<const char *>(y_saved) + row0 * c.H * eb;
+        } else {
+            // recompute: dispatch the rows again and run the expert FFN forward
+            void *yw = ws_at<void>(ws, B.y);
+            MOE_TRY(launch_permute(c, x, pos, tb, tc, xr, stream), "permute");
+            if (B.nmax > 0) {
+                if (bf16)
+                    MOE_TRY(launch_ffn_tcgen05(c, B.nmax, xr, eoff, w13, w2, h, yw, nullptr, nullptr, nullptr,
+                                               nullptr, status, ctr, stream, nsm),
+                            "grouped_swiglu_ffn");
+                else
+                    MOE_TRY(launch_ffn_simt(c, B.nmax, xr, eoff, w13, w2, h, yw, nullptr, nullptr, nullptr,
+                                            nullptr, stream),
+                            "grouped_swiglu_ffn");
+            }
+            y = yw;
+        }
+        void *dxr = ws_at<void>(ws, B.dxr);
+        MOE_TRY(launch_combine_bwd(c, dout, y, pos, topk_w, tb, tc, dy, dw, stream), "combine_backward");
+        if (B.nmax > 0) {
+            if (bf16)
+                MOE_TRY(launch_ffn_tcgen05_dgrad(c, B.nmax, xr, dy, eoff, w13, w2, ws_at<void>(ws, B.gu), h, dgu,
+                                                 dxr, status, ctr, stream, nsm),
+                        "grouped_swiglu_ffn_backward");
+            else
+                MOE_TRY(launch_ffn_simt_dgrad(c, B.nmax, xr, dy, eoff, w13, w2, h, dgu, dxr, stream),
+                        "grouped_swiglu_ffn_backward");
+        }
+        void *dxs = nullptr;
+        if (shared) {
+            // the shared expert saw every row of the chunk with weight 1: its dy is dout
+            MOE_TRY(launch_shared_offsets(soff, tc, stream), "shared offsets");
+            const void *xs = static_cast<const char *>(x) + eb * (size_t)tb * c.H;
+            const void *ds = static_cast<const char *>(dout) + eb * (size_t)tb * c.H;
+            void *hs = ws_at<char>(ws, B.hs) + eb * (size_t)tb * c.shared_I;
+            void *dgus = ws_at<char>(ws, B.dgus) + eb * (size_t)tb * 2 * c.shared_I;
+            dxs = ws_at<void>(ws, B.dxs);
+            if (bf16)
+                MOE_TRY(launch_ffn_tcgen05_dgrad(cs, tc, xs, ds, soff, w13_shared, w2_shared, ws_at<void>(ws, B.gus),
+                                                 hs, dgus, dxs, status, ws_at<uint32_t>(ws, L.shared_ctr), stream,
+                                                 nsm),
+                        "shared expert backward");
+            else
+                MOE_TRY(launch_ffn_simt_dgrad(cs, tc, xs, ds, soff, w13_shared, w2_shared, hs, dgus, dxs, stream),
+                        "shared expert backward");
+        }
+        // dx[t] = the sum of the token's kept receive-row gradients (+ its shared-expert row)
+        MOE_TRY(launch_combine(c, dxr, pos, nullptr, tb, tc, dxs, dx, stream), "permute_backward");
+    }
+    // the weight gradients once, over every chunk's rows
+    const int32_t *eoffs = ws_at<int32_t>(ws, B.eoff);
+    if (bf16)
+        MOE_TRY(launch_ffn_tcgen05_wgrad(c, c.n_chunks, nrow, eoffs, xr_all, dy_all, h_all, dgu_all, dw13, dw2,
+                                         accumulate, status, stream, nsm),
+                "weight gradients");
+    else
+        MOE_TRY(launch_ffn_simt_wgrad(c, c.n_chunks, nrow, eoffs, xr_all, dy_all, h_all, dgu_all, dw13, dw2,
+                                      accumulate, stream),
+                "weight gradients");
+    if (shared) {
+        MOE_TRY(launch_shared_offsets(soff, c.T, stream), "shared offsets");
+        if (bf16)
+            MOE_TRY(launch_ffn_tcgen05_wgrad(cs, 1, c.T, soff, x, dout, ws_at<void>(ws, B.hs),
+                                             ws_at<void>(ws, B.dgus), dw13_shared, dw2_shared, accumulate, status,
+                                             stream, nsm),
+                    "shared weight gradients");
+        else
+            MOE_TRY(launch_ffn_simt_wgrad(cs, 1, c.T, soff, x, dout, ws_at<void>(ws, B.hs), ws_at<void>(ws, B.dgus),
+                                          dw13_shared, dw2_shared, accumulate, stream),
+                    "shared weight gradients");
+    }
+    MOE_TRY(launch_route_bwd(c, topk_idx, topk_w, dw, dlogits, dbias, status, stream), "route_backward");
+#undef MOE_TRY
+    return MOE_OK;
 }
 
 size_t moe_forward_host_workspace_bytes(const moe_config *cfg) {

@@ -69,12 +69,15 @@ _decl("moe_combine", _I32, _CFG, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_reduce_finalize", _I32, _CFG, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_shared_expert_ffn", _I32, _CFG, _I32, _I32, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_forward_chunked", _I32, _CFG, *([_P] * 17))
+_decl("moe_forward_chunked_save", _I32, _CFG, *([_P] * 17))
+_decl("moe_backward_workspace_bytes", ctypes.c_size_t, _CFG)
+_decl("moe_layer_backward", _I32, _CFG, *([_P] * 18), _I32, _P, _P)
 _decl("moe_forward_host_workspace_bytes", ctypes.c_size_t, _CFG)
 _decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
 _decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
 _decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
 _decl("moe_permute_quantize_fp8", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
-_decl("moe_grouped_swiglu_ffn_backward", _I32, _CFG, ctypes.c_int64, *([_P] * 12), _I32, _P, _P)
+_decl("moe_grouped_swiglu_ffn_backward", _I32, _CFG, ctypes.c_int64, *([_P] * 11), _I32, _P, _P)
 _decl("moe_combine_backward", _I32, _CFG, _P, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_route_backward", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute_backward", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
@@ -298,6 +301,34 @@ def moe_forward_chunked(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, ke
                                     _ptr(out), _ptr(topk_idx), _ptr(topk_w),
                                     _ptr(keep), _ptr(splits_host), _ptr(ws),
                                     _stream(s_dispatch), _stream(s_compute)))
+
+
+def moe_forward_chunked_save(cfg, logits, bias, x, w13, w2, out, topk_idx, topk_w, keep, splits_host,
+                             xr_save, y_save, ws, s_dispatch=None, s_compute=None, w13_shared=None,
+                             w2_shared=None):
+    """moe_forward_chunked that also writes every chunk's receive rows and expert
+    outputs to xr_save / y_save ([n_chunks, N_max, H])."""
+    _check(_lib.moe_forward_chunked_save(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(x), _ptr(w13),
+                                         _ptr(w2), _ptr(w13_shared), _ptr(w2_shared), _ptr(out),
+                                         _ptr(topk_idx), _ptr(topk_w), _ptr(keep), _ptr(splits_host),
+                                         _ptr(xr_save), _ptr(y_save), _ptr(ws), _stream(s_dispatch),
+                                         _stream(s_compute)))
+
+
+def backward_workspace_bytes(cfg: MoEConfig) -> int:
+    return int(_lib.moe_backward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def moe_layer_backward(cfg, x, dout, w13, w2, topk_idx, topk_w, keep, dx, dlogits, dbias, dw13, dw2,
+                       ws, xr_saved=None, y_saved=None, w13_shared=None, w2_shared=None,
+                       dw13_shared=None, dw2_shared=None, accumulate=False, stream=None):
+    """The layer's backward: with xr_saved / y_saved (from moe_forward_chunked_save)
+    the dispatch outputs are read, without them recomputed."""
+    _check(_lib.moe_layer_backward(ctypes.byref(cfg), _ptr(x), _ptr(dout), _ptr(w13), _ptr(w2),
+                                   _ptr(w13_shared), _ptr(w2_shared), _ptr(topk_idx), _ptr(topk_w),
+                                   _ptr(keep), _ptr(xr_saved), _ptr(y_saved), _ptr(dx), _ptr(dlogits),
+                                   _ptr(dbias), _ptr(dw13), _ptr(dw2), _ptr(dw13_shared),
+                                   _ptr(dw2_shared), int(bool(accumulate)), _ptr(ws), _stream(stream)))
 
 
 def moe_forward_host(cfg, logits_host, bias_host, x_host, w13, w2, out_host, topk_idx, topk_w,

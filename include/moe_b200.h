@@ -13,7 +13,9 @@
  *
  * plus moe_forward_chunked, which runs 1-2 once and pipelines 3-6 over token
  * chunks on two streams (dispatch of chunk c+1 overlaps the FFN of chunk c),
- * and moe_forward_host, the same layer with its activations in host memory.
+ * moe_forward_host, the same layer with its activations in host memory, and
+ * moe_forward_chunked_save / moe_layer_backward, the forward that keeps the
+ * dispatch outputs and the layer's backward that reads them or recomputes them.
  *
  * Also: routing variants through moe_config (grouped top-k, a bias that steers
  * the selection only); moe_shared_expert_ffn, a dense shared expert whose rows
@@ -487,6 +489,59 @@ moe_status moe_forward_chunked(const moe_config *cfg, const float *logits, const
                                int32_t *topk_idx, float *topk_w, uint8_t *keep,
                                int32_t *splits_host, void *ws,
                                cudaStream_t s_dispatch, cudaStream_t s_compute);
+
+/*
+ * moe_forward_chunked that also keeps the dispatch outputs ([AX]
+ * expert_parallel_save_dispatch: under activation checkpointing, hold the
+ * dispatch / combine all-to-all outputs for the backward instead of issuing
+ * the exchanges again): chunk c's receive rows and expert outputs are written
+ * to xr_save + c * N_max * H and y_save + c * N_max * H (both [n_chunks,
+ * N_max, H] in cfg->dtype, N_max = moe_max_recv_rows(cfg, T / n_chunks); rows
+ * past the chunk's N are left untouched).  Otherwise as moe_forward_chunked
+ * (same output bits).  Needs ffn_fp8 = 0 and reduce_dense = 0
+ * (MOE_ERR_UNSUPPORTED).  ws: moe_forward_workspace_bytes(cfg).
+ */
+moe_status moe_forward_chunked_save(const moe_config *cfg, const float *logits, const float *bias,
+                                    const void *x, const void *w13, const void *w2,
+                                    const void *w13_shared, const void *w2_shared, void *out,
+                                    int32_t *topk_idx, float *topk_w, uint8_t *keep,
+                                    int32_t *splits_host, void *xr_save, void *y_save, void *ws,
+                                    cudaStream_t s_dispatch, cudaStream_t s_compute);
+
+/*
+ * The layer's backward for L = <dout, out> ([AX] expert_parallel_save_dispatch:
+ * the routing top-k and the split counts are always kept; the dispatch and
+ * combine outputs are either kept by the forward or produced again).  Chunk by
+ * chunk (cfg->n_chunks contiguous token chunks, as the forward ran), on one
+ * stream:
+ *   1. the chunk's dispatch layout from the saved topk_idx and keep;
+ *   2. save mode (xr_saved and y_saved from moe_forward_chunked_save): the
+ *      chunk's receive rows and expert outputs are read from them; recompute
+ *      mode (both NULL): the rows are permuted again from x and the expert
+ *      FFN's forward runs again (the same bits as the forward's);
+ *   3. moe_combine_backward (dy rows, the slot gradients dw);
+ *   4. moe_grouped_swiglu_ffn_backward (dxr, dW13, dW2);
+ *   5. with a shared expert, its backward over the chunk's rows of x with
+ *      dy = dout (dW13_shared, dW2_shared, its dx rows);
+ *   6. dx[t] = the sum of the token's kept receive-row gradients plus its
+ *      shared-expert row (fp32, one rounding to cfg->dtype);
+ * then moe_route_backward over all T (dlogits fp32 [T, E]; dbias fp32 [E] or
+ * NULL, 0 when cfg->bias_select_only).  The weight gradients (fp32, the
+ * layouts of w13 / w2 / w13_shared / w2_shared) are written by the first chunk
+ * (added to when accumulate = 1) and added to by the later ones.  Save and
+ * recompute give the same bits.  Needs ffn_fp8 = 0 and reduce_dense = 0.
+ *   x, dout [T, H] cfg->dtype; topk_idx, topk_w, keep: the forward's (saved).
+ *   ws: moe_backward_workspace_bytes(cfg) bytes (one chunk slot of receive-row
+ *   buffers and the fp32 slot gradients), zero-filled once before first use.
+ */
+size_t moe_backward_workspace_bytes(const moe_config *cfg);
+moe_status moe_layer_backward(const moe_config *cfg, const void *x, const void *dout,
+                              const void *w13, const void *w2, const void *w13_shared,
+                              const void *w2_shared, const int32_t *topk_idx, const float *topk_w,
+                              const uint8_t *keep, const void *xr_saved, const void *y_saved,
+                              void *dx, float *dlogits, float *dbias, float *dw13, float *dw2,
+                              float *dw13_shared, float *dw2_shared, int32_t accumulate, void *ws,
+                              cudaStream_t stream);
 
 /*
  * moe_forward_chunked with the activations in HOST memory: what a caller whose

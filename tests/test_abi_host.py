@@ -130,3 +130,46 @@ def test_forward_workspace_sizes():
     extra = moe.forward_host_workspace_bytes(bf) - moe.forward_workspace_bytes(bf)
     assert extra >= 4 * 4096 * 128 + 4 * 128 + 2 * 2 * 4096 * 2048
     assert extra < 4 * 4096 * 128 + 4 * 128 + 2 * 2 * 4096 * 2048 + 4 * 256
+
+
+def test_backward_entry_points_reject_bad_arguments_before_any_launch():
+    ws = ctypes.c_void_p(256)            # aligned, never dereferenced on these paths
+    p = ctypes.c_void_p(512)
+    bf = moe.make_config(64, 128, 8, 2, 128, 2)
+    f8 = moe.make_config(64, 128, 8, 2, 128, 2, ffn_fp8=True)
+    dec = moe.make_config(64, 128, 8, 2, 128, 2, reduce_dense=True)
+    ffn_bwd = moe._lib.moe_grouped_swiglu_ffn_backward
+    st = ffn_bwd(ctypes.byref(bf), 16, *([p] * 11), 2, ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "accumulate" in moe.last_error_detail()
+    st = ffn_bwd(ctypes.byref(f8), 16, *([p] * 11), 0, ws, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    st = ffn_bwd(ctypes.byref(bf), 16, None, *([p] * 10), 0, ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+    st = ffn_bwd(ctypes.byref(bf), -1, *([p] * 11), 0, ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    bwd = moe._lib.moe_layer_backward
+    # save mode needs both saved buffers: one alone is an error
+    args = [p] * 9 + [p, None] + [p] * 7
+    st = bwd(ctypes.byref(bf), *args, 0, ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "saved" in moe.last_error_detail()
+    args = [p] * 9 + [None, None] + [p] * 7
+    for cfg in (f8, dec):
+        st = bwd(ctypes.byref(cfg), *args, 0, ws, None)
+        assert st == moe.MOE_ERR_UNSUPPORTED
+    st = bwd(ctypes.byref(bf), *([None] * 18), 0, ws, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+    sv = moe._lib.moe_forward_chunked_save
+    st = sv(ctypes.byref(dec), *([p] * 14), ws, None, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    st = sv(ctypes.byref(bf), *([p] * 12), None, p, ws, None, None)
+    assert st == moe.MOE_ERR_INVALID_ARG and "NULL" in moe.last_error_detail()
+
+
+def test_backward_workspace_holds_every_chunks_rows():
+    one = moe.make_config(8192, 7168, 256, 8, 2048, 8, n_chunks=1)
+    two = moe.make_config(8192, 7168, 256, 8, 2048, 8, n_chunks=2)
+    # the rows the weight gradients read (receive rows, dy, h, dg | du) for all
+    # chunks, plus one chunk's slot of the rest: the two-chunk layer needs less
+    b1, b2 = moe.backward_workspace_bytes(one), moe.backward_workspace_bytes(two)
+    rows_all = 65536 * (7168 + 7168 + 2048 + 2 * 2048) * 2
+    assert rows_all < b1 and rows_all < b2 < b1
