@@ -103,8 +103,9 @@ def parse_args(argv=None):
     p.add_argument("--no-overlap", action="store_true",
                    help="skip the one-stream replay of a chunked workload")
     p.add_argument("--backward", action="store_true",
-                   help="also time the backward's row passes (combine, routing, permute) on the "
-                        "last chunk and add a backward_row_passes object to the line")
+                   help="also time the backward: the layer's backward with the dispatch outputs saved "
+                        "and recomputed, the expert FFN's backward step (with its roofline), and the "
+                        "row passes on the last chunk (backward and backward_row_passes objects)")
     p.add_argument("--seed", type=int, default=None)
     p.add_argument("--no-graph", action="store_true",
                    help="time eager launches instead of replaying a captured CUDA graph of the layer")
@@ -419,6 +420,146 @@ def backward_row_passes(moe, wl, cfg, B, n_rows, peaks, flush, args):
                             "frac": gbs(pb, t["permute"]) / peaks["hbm_gbs"] if t["permute"] > 0 else None},
             "route_bwd": {"ms": round(t["route"], 4), "gbs": gbs(rb, t["route"])},
             "timing": "CUDA events around each eager launch, L2 flushed before each pass triple"}
+
+
+def ffn_backward_algorithmic(wl, N, active):
+    """Bytes and flops of the expert FFN's backward over N receive rows with
+    `active` experts holding rows: W13 read twice (g | u recomputed; dxr) and W2
+    once (dh); xr and dy read twice (data and weight gradients); g | u written
+    and read; h written and read; dg | du written and read twice; dxr written;
+    the fp32 weight gradients of all E experts written once.  Flops:
+    2 * N * (2IH + HI + 2IH + HI + 2IH) = 16 * H * I * N."""
+    b = wl.elem_bytes
+    H, I = wl.H, wl.I
+    w = 5 * active * H * I * b
+    act = N * (2 * H + 2 * H + 2 * 2 * I + 2 * I + 3 * 2 * I + H) * b
+    dw = wl.E * 3 * H * I * 4
+    return {"bytes": w + act + dw, "flops": 16.0 * H * I * N, "weight_bytes": w, "act_bytes": act,
+            "dw_bytes": dw}
+
+
+def layer_backward(moe, wl, cfg, inp, layer, flush, args, peaks, peak_src):
+    """Times the layer's backward (moe_layer_backward) with the dispatch outputs
+    saved by the forward and with them recomputed, alternating step by step,
+    and the expert FFN's backward step alone over the whole batch's receive rows
+    (one-chunk layout), with its roofline."""
+    import torch
+    dev = inp.x.device
+    T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
+    dt = wl.torch_dtype
+    nmax = moe.max_recv_rows(cfg, T // wl.n_chunks)
+    xr_s = torch.empty(wl.n_chunks, max(nmax, 1), H, dtype=dt, device=dev)
+    y_s = torch.empty(wl.n_chunks, max(nmax, 1), H, dtype=dt, device=dev)
+    out = torch.empty(T, H, dtype=dt, device=dev)
+    s = torch.cuda.current_stream()
+    moe.moe_forward_chunked_save(cfg, inp.logits, inp.bias, inp.x, inp.w13, inp.w2, out, layer.topk_idx,
+                                 layer.topk_w, layer.keep, None, xr_s, y_s, layer.ws, s, s, inp.w13s, inp.w2s)
+    g = torch.Generator(device=dev).manual_seed(17)
+    dout = torch.randn(T, H, generator=g, device=dev).to(dt)
+    bws = moe.alloc_workspace(moe.backward_workspace_bytes(cfg), dev)
+    dx = torch.empty(T, H, dtype=dt, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    db = torch.empty(E, dtype=torch.float32, device=dev)
+    dw13 = torch.empty(E, 2 * I, H, dtype=torch.float32, device=dev)
+    dw2 = torch.empty(E, H, I, dtype=torch.float32, device=dev)
+    sh = {}
+    if wl.shared_I > 0:
+        sh = dict(w13_shared=inp.w13s, w2_shared=inp.w2s,
+                  dw13_shared=torch.empty(2 * wl.shared_I, H, device=dev),
+                  dw2_shared=torch.empty(H, wl.shared_I, device=dev))
+
+    def bwd(saved):
+        moe.moe_layer_backward(cfg, inp.x, dout, inp.w13, inp.w2, layer.topk_idx, layer.topk_w, layer.keep,
+                               dx, dl, db, dw13, dw2, bws, xr_saved=xr_s if saved else None,
+                               y_saved=y_s if saved else None, **sh)
+
+    for _ in range(max(1, args.warmup)):
+        bwd(True)
+        bwd(False)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(1)
+        ev[i][0].record()
+        bwd(True)
+        ev[i][1].record()
+        flush.fill_(1)
+        ev[i][2].record()
+        bwd(False)
+        ev[i][3].record()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(bws) != 0:
+        raise RuntimeError("device status bits set during the layer backward")
+    save_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    rec_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    del bws, xr_s, y_s
+
+    # the expert FFN's backward step over the whole batch in one receive buffer
+    w1 = wl.with_(n_chunks=1)
+    c1 = moe.config_from_workload(w1)
+    ws1 = moe.alloc_workspace(moe.workspace_bytes(c1), dev)
+    n1 = moe.max_recv_rows(c1, T)
+    eoff = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    roff = torch.empty(w1.ep + 1, dtype=torch.int32, device=dev)
+    rt = torch.empty(max(n1, 1), dtype=torch.int32, device=dev)
+    rs = torch.empty(max(n1, 1), dtype=torch.int32, device=dev)
+    pos = torch.empty(T, k, dtype=torch.int32, device=dev)
+    spl = torch.empty(w1.ep, w1.ep, dtype=torch.int32, device=dev)
+    moe.moe_dispatch_layout(c1, 0, T, layer.topk_idx, layer.keep, eoff, roff, rt, rs, pos, spl, None, ws1)
+    xr = torch.empty(max(n1, 1), H, dtype=dt, device=dev)
+    moe.moe_permute(c1, inp.x, pos, 0, T, xr)
+    dyr = torch.randn(max(n1, 1), H, generator=g, device=dev).to(dt)
+    gu = torch.empty(max(n1, 1), 2 * I, dtype=dt, device=dev)
+    hh = torch.empty(max(n1, 1), I, dtype=dt, device=dev)
+    dgu = torch.empty(max(n1, 1), 2 * I, dtype=dt, device=dev)
+    dxr = torch.empty(max(n1, 1), H, dtype=dt, device=dev)
+    torch.cuda.synchronize()
+    N = int(eoff[E].item())
+    active = int(((eoff[1:] - eoff[:-1]) > 0).sum().item())
+
+    def step():
+        moe.moe_grouped_swiglu_ffn_backward(c1, n1, xr, dyr, eoff, inp.w13, inp.w2, gu, hh, dgu, dxr,
+                                            dw13, dw2, 0, ws1)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(1)
+        evs[i][0].record()
+        step()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    if moe.moe_device_status(ws1) != 0:
+        raise RuntimeError("device status bits set during the FFN backward")
+    ffn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    alg = ffn_backward_algorithmic(wl, N, active)
+    t = ffn_ms / 1e3
+    tflops = alg["flops"] / t / 1e12
+    gbs = alg["bytes"] / t / 1e9
+    t_flop = alg["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_byte = alg["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    hbm = t_byte > t_flop
+    return {
+        "layer_backward_ms": {"save_dispatch": round(save_ms, 4), "recompute": round(rec_ms, 4),
+                              "recompute_minus_save": round(rec_ms - save_ms, 4),
+                              "tokens_per_s_save": T / (save_ms / 1e3),
+                              "timing": "moe_layer_backward, the two modes alternated step by step, "
+                                        "L2 flushed before each"},
+        "ffn_backward": {"kernel": "moe_grouped_swiglu_ffn_backward: g|u, dh + SwiGLU backward, dxr "
+                                   "(ffn_gemm_tcgen05_kernel), dW2 and dW13 (wgrad_tcgen05_kernel)",
+                         "rows": N, "active_experts": active, "ms": round(ffn_ms, 4),
+                         "bound": "hbm" if hbm else "tensor",
+                         "achieved": gbs if hbm else tflops,
+                         "peak": peaks["hbm_gbs"] if hbm else peaks["bf16_tflops"],
+                         "unit": "GB/s" if hbm else "TFLOP/s",
+                         "frac": gbs / peaks["hbm_gbs"] if hbm else tflops / peaks["bf16_tflops"],
+                         "tflops": tflops, "gbs": gbs,
+                         "tensor_frac": tflops / peaks["bf16_tflops"],
+                         "tensor_frac_sustained": tflops / peaks["bf16_tflops_sustained"],
+                         "hbm_frac": gbs / peaks["hbm_gbs"],
+                         "algorithmic": alg, "peak_source": peak_src},
+    }
 
 
 def stage_times(wl, ev, per_chunk=False):
@@ -861,6 +1002,8 @@ def run_ours(args):
     alg = algorithmic(wl, n_kept, n_active, tokens_read)
     bwd = backward_row_passes(moe, wl, cfg, B, n_kept[-1], peaks, flush, args) \
         if args.backward and not wl.reduce_dense else None
+    lbwd = layer_backward(moe, wl, cfg, inp, layer, flush, args, peaks, peak_src) \
+        if args.backward and not wl.reduce_dense and not wl.ffn_fp8 else None
     if overlap is not None:
         # what the second stream can hide: the dispatch (layout + permute) of
         # every chunk after the first, which runs beside the previous chunk's FFN
@@ -971,6 +1114,8 @@ def run_ours(args):
             line["overlap"] = overlap
         if bwd is not None:
             line["backward_row_passes"] = bwd
+        if lbwd is not None:
+            line["backward"] = lbwd
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

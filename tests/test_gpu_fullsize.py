@@ -3,12 +3,17 @@ benchmark times.
 
 Routing, drop sets, layouts and split counts are compared whole against the
 oracle (bit-exact).  Permuted rows are checked whole by the defining property
-xr[p] = x[recv_token[p]] (bitwise).  The FFN and the combined output are
-compared on sampled rows and tokens that the oracle computes one by one:
-experts at both ends of the expert range, the most loaded expert and a random
-one, each with its first, last and random rows; and tokens spread over the
-batch.
+xr[p] = x[recv_token[p]] (bitwise).  The FFN is compared on every tile the
+grouped GEMM deals: the first and the last row of every (expert, 256-token
+block) of every chunk, and two more rows of each expert's short last block
+(the 32-row token box of tiles with at most 64 rows).  The combined output is
+compared on 128 sampled tokens, whose expert rows the oracle also computes.
+The oracle's rows run in threads (its C calls release the interpreter lock),
+expert by expert, each with its own host copy of that expert's weights.
 """
+import concurrent.futures as cf
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -25,10 +30,42 @@ pytestmark = pytest.mark.gpu
 FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode", "dsv3_grouped"]
 
 
-def _host_expert(inp, e, cache):
-    if e not in cache:
-        cache[e] = (storage_np(inp.w13[e]), storage_np(inp.w2[e]))
-    return cache[e]
+TILE = 256          # token rows per FFN tile
+SHORT = 64          # tiles of at most this many rows take the short token box
+N_TOKENS = 128      # sampled tokens of the combined output
+
+
+def select_rows(lay, rng):
+    """Receive rows that cover every FFN tile of a chunk: per (expert, 256-row
+    block) its first and last row; a short last block (<= 64 rows) two more."""
+    eoff = lay["expert_offsets"]
+    rows = set()
+    for e in range(len(eoff) - 1):
+        lo, hi = int(eoff[e]), int(eoff[e + 1])
+        for b0 in range(lo, hi, TILE):
+            b1 = min(b0 + TILE, hi) - 1
+            rows.update((b0, b1))
+            if b1 - b0 + 1 <= SHORT:
+                rows.update(int(v) for v in rng.integers(b0, b1 + 1, 2))
+    return rows
+
+
+def expert_of(eoff, p):
+    return int(np.searchsorted(eoff, p, side="right") - 1)
+
+
+def oracle_rows(row_fn, fetch, wanted):
+    """wanted: {expert: [(key, x_row), ...]} -> {key: row_fn(x_row, weights)}, run
+    expert by expert in threads."""
+    def work(e, items):
+        w = fetch(e)
+        return [(key, row_fn(xv, w)) for key, xv in items]
+    out = {}
+    n = max(1, min(32, os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(n) as ex:
+        for res in ex.map(lambda kv: work(*kv), wanted.items()):
+            out.update(res)
+    return out
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -47,58 +84,63 @@ def test_fullsize_against_oracle(name):
 
     x_np = storage_np(inp.x)
     rng = np.random.default_rng(0)
-    cache = {}
-    for c, (gc, lay) in enumerate(zip(g["chunks"], orc["layouts"])):
+    tc = wl.T // wl.n_chunks
+    tokens = sorted({0, wl.T - 1, *rng.choice(wl.T, N_TOKENS - 2, replace=False).tolist()})
+    # every tile's rows, and the rows of the sampled tokens' kept slots
+    wanted = {}
+    for c, lay in enumerate(orc["layouts"]):
         n = lay["N"]
         rt = torch.from_numpy(lay["recv_token"]).long().cuda()
-        assert torch.equal(gc["xr_dev"][:n], inp.x[rt]), "permute must copy rows bitwise"
-        eoff = lay["expert_offsets"]
-        sizes = np.diff(eoff)
-        nonempty = np.nonzero(sizes)[0]
-        experts = {int(nonempty[0]), int(nonempty[-1]), int(np.argmax(sizes)),
-                   int(rng.choice(nonempty))}
-        for e in sorted(experts):
-            lo, hi = int(eoff[e]), int(eoff[e + 1])
-            rows = sorted({lo, hi - 1, *rng.integers(lo, hi, 2).tolist()})
-            w13e, w2e = _host_expert(inp, e, cache)
-            for p in rows:
-                h_ref, y_ref, ye_ref = oracle.ffn_row(x_np[lay["recv_token"][p]], w13e, w2e)
-                assert_float_close(storage_np(gc["h_dev"][p]), h_ref, wl.dtype, f"h[{p}] expert {e}")
-                if gc["y_dev"] is not None:
-                    assert_float_close(storage_np(gc["y_dev"][p]), y_ref, wl.dtype, f"y[{p}] expert {e}")
+        assert torch.equal(g["chunks"][c]["xr_dev"][:n], inp.x[rt]), "permute must copy rows bitwise"
+        rows = select_rows(lay, rng)
+        for t in tokens:
+            if c * tc <= t < (c + 1) * tc:
+                rows.update(int(p) for p in lay["pos"][t - c * tc] if p >= 0)
+        for p in rows:
+            e = expert_of(lay["expert_offsets"], p)
+            wanted.setdefault(e, []).append(((c, p), x_np[lay["recv_token"][p]]))
+    fetch = lambda e: (storage_np(inp.w13[e]), storage_np(inp.w2[e]))
+    ref = oracle_rows(lambda xv, w: oracle.ffn_row(xv, w[0], w[1]), fetch, wanted)
+
+    assert len(ref) == sum(len(v) for v in wanted.values())
+    for (c, p), (h_ref, y_ref, _) in sorted(ref.items()):
+        gc = g["chunks"][c]
+        assert_float_close(storage_np(gc["h_dev"][p]), h_ref, wl.dtype, f"h[{p}] chunk {c}")
+        if gc["y_dev"] is not None:
+            assert_float_close(storage_np(gc["y_dev"][p]), y_ref, wl.dtype, f"y[{p}] chunk {c}")
 
     out = storage_np(g["out"])
-    tokens = sorted({0, wl.T - 1, *rng.integers(0, wl.T, 2).tolist()})
     shared = None
     if wl.shared_I > 0:
         shared = (storage_np(inp.w13s), storage_np(inp.w2s))
-    tc = wl.T // wl.n_chunks
     for t in tokens:
+        c = t // tc
+        lay = orc["layouts"][c]
         ysh = None
         if shared is not None:
             # the shared expert's row of token t, checked against the GPU's and used below
             _, ysh, _ = oracle.shared_expert(x_np[t:t + 1], *shared)
-            gys = storage_np(g["chunks"][t // tc]["ys_dev"][t % tc:t % tc + 1])
+            gys = storage_np(g["chunks"][c]["ys_dev"][t % tc:t % tc + 1])
             assert_float_close(gys, ysh, wl.dtype, f"y_shared[{t}]")
         ys, yes, pos = [], [], []
         for j in range(wl.k):
-            if not orc["keep"][t, j]:
+            p = int(lay["pos"][t - c * tc, j])
+            if p < 0:
                 pos.append(-1)
                 continue
-            w13e, w2e = _host_expert(inp, int(orc["topk_idx"][t, j]), cache)
-            _, y_ref, ye_ref = oracle.ffn_row(x_np[t], w13e, w2e)
+            _, y_ref, ye_ref = ref[(c, p)]
             pos.append(len(ys))
             ys.append(y_ref)
             yes.append(ye_ref)
         posa = np.array([pos], np.int32)
         w_t = orc["topk_w"][t:t + 1]
         if not ys:
-            ref = np.zeros((1, wl.H), x_np.dtype) if ysh is None else ysh
+            want = np.zeros((1, wl.H), x_np.dtype) if ysh is None else ysh
         elif wl.reduce_dense:
-            ref = oracle.combine_exact(np.stack(yes), posa, w_t, 1, x_np.dtype, y_shared=ysh)
+            want = oracle.combine_exact(np.stack(yes), posa, w_t, 1, x_np.dtype, y_shared=ysh)
         else:
-            ref = oracle.combine(np.stack(ys), posa, w_t, 1, y_shared=ysh)
-        assert_float_close(out[t:t + 1], ref, wl.dtype, f"out[{t}]")
+            want = oracle.combine(np.stack(ys), posa, w_t, 1, y_shared=ysh)
+        assert_float_close(out[t:t + 1], want, wl.dtype, f"out[{t}]")
     del g, inp
     torch.cuda.empty_cache()
 
@@ -129,9 +171,9 @@ def test_dsv3_prefill_chunked_forward_equals_steps():
 @pytest.mark.parametrize("name", ["qwen3_30b_a3b_fp8", "dsv3_prefill_fp8"])
 def test_fp8_fullsize_against_oracle(name):
     """The FP8 layer at full size: x's codes and scales whole and bit-exact,
-    the weight codes of the sampled experts bit-exact, permuted codes by the
-    defining property, sampled FFN rows and tokens against the oracle's FP8
-    rows (its own quantisation of the bf16 weights)."""
+    the weight codes of every checked expert bit-exact, permuted codes by the
+    defining property, the rows of every FFN tile and 128 sampled tokens
+    against the oracle's FP8 rows (its own quantisation of the bf16 weights)."""
     wl = WORKLOADS[name]
     torch.cuda.empty_cache()
     inp = make_inputs(wl, "cuda")
@@ -148,49 +190,53 @@ def test_fp8_fullsize_against_oracle(name):
     np.testing.assert_array_equal(g["xs"], xs)
     xq_dev = torch.from_numpy(xq).cuda()
     rng = np.random.default_rng(0)
-    cache = {}
 
-    def expert(e):
-        if e not in cache:
-            cache[e] = oracle_fp8_weights(inp, [e])[e]
-            ref = cache[e]
-            np.testing.assert_array_equal(w13q[e].cpu().numpy(), ref["w13q"])
-            np.testing.assert_array_equal(w13s[e].cpu().numpy(), ref["w13s"])
-            np.testing.assert_array_equal(w2q[e].cpu().numpy(), ref["w2q"])
-            np.testing.assert_array_equal(w2s[e].cpu().numpy(), ref["w2s"])
-        return cache[e]
+    def fetch(e):
+        # the oracle's codes of expert e's weights, checked against the GPU's
+        ref = oracle_fp8_weights(inp, [e])[e]
+        np.testing.assert_array_equal(w13q[e].cpu().numpy(), ref["w13q"])
+        np.testing.assert_array_equal(w13s[e].cpu().numpy(), ref["w13s"])
+        np.testing.assert_array_equal(w2q[e].cpu().numpy(), ref["w2q"])
+        np.testing.assert_array_equal(w2s[e].cpu().numpy(), ref["w2s"])
+        return ref
 
-    def row(p_token, e):
-        w = expert(e)
-        return oracle.ffn_row_fp8(xq[p_token], xs[p_token], w["w13q"], w["w13s"], w["w2q"], w["w2s"])
-
+    tc = wl.T // wl.n_chunks
+    tokens = sorted({0, wl.T - 1, *rng.choice(wl.T, N_TOKENS - 2, replace=False).tolist()})
+    wanted = {}
     for c, (gc, lay) in enumerate(zip(g["chunks"], orc["layouts"])):
         n = lay["N"]
         rt = torch.from_numpy(lay["recv_token"]).long().cuda()
         assert torch.equal(gc["xr_dev"][:n], xq_dev[rt]), "permute must copy the code rows bitwise"
-        eoff = lay["expert_offsets"]
-        sizes = np.diff(eoff)
-        nonempty = np.nonzero(sizes)[0]
-        experts = {int(nonempty[0]), int(nonempty[-1]), int(np.argmax(sizes)), int(rng.choice(nonempty))}
-        for e in sorted(experts):
-            lo, hi = int(eoff[e]), int(eoff[e + 1])
-            for p in sorted({lo, hi - 1, *rng.integers(lo, hi, 2).tolist()}):
-                h, hq, hs, y, ye = row(int(lay["recv_token"][p]), e)
-                assert_float_close(storage_np(gc["h_dev"][p]), h, "bf16", f"h[{p}] expert {e}")
-                assert_codes_close(gc["hq_dev"][p:p + 1].cpu().numpy(), gc["hs_dev"][p:p + 1].cpu().numpy(),
-                                   hq[None], np.array([hs], np.uint8), f"h codes[{p}]", min_equal=0.98)
-                assert_float_close(storage_np(gc["y_dev"][p]), y, "bf16", f"y[{p}] expert {e}")
+        rows = select_rows(lay, rng)
+        for t in tokens:
+            if c * tc <= t < (c + 1) * tc:
+                rows.update(int(p) for p in lay["pos"][t - c * tc] if p >= 0)
+        for p in rows:
+            e = expert_of(lay["expert_offsets"], p)
+            wanted.setdefault(e, []).append(((c, p), int(lay["recv_token"][p])))
+    ref = oracle_rows(lambda tok, w: oracle.ffn_row_fp8(xq[tok], xs[tok], w["w13q"], w["w13s"], w["w2q"],
+                                                        w["w2s"]), fetch, wanted)
+    assert len(ref) == sum(len(v) for v in wanted.values())
+    for (c, p), (h, hq, hs, y, ye) in sorted(ref.items()):
+        gc = g["chunks"][c]
+        assert_float_close(storage_np(gc["h_dev"][p]), h, "bf16", f"h[{p}] chunk {c}")
+        assert_codes_close(gc["hq_dev"][p:p + 1].cpu().numpy(), gc["hs_dev"][p:p + 1].cpu().numpy(),
+                           hq[None], np.array([hs], np.uint8), f"h codes[{p}]", min_equal=0.98)
+        assert_float_close(storage_np(gc["y_dev"][p]), y, "bf16", f"y[{p}] chunk {c}")
 
     out = storage_np(g["out"])
-    for t in sorted({0, wl.T - 1, *rng.integers(0, wl.T, 2).tolist()}):
+    for t in tokens:
+        c = t // tc
+        lay = orc["layouts"][c]
         ys, pos = [], []
         for j in range(wl.k):
-            if not orc["keep"][t, j]:
+            p = int(lay["pos"][t - c * tc, j])
+            if p < 0:
                 pos.append(-1)
                 continue
             pos.append(len(ys))
-            ys.append(row(t, int(orc["topk_idx"][t, j]))[3])
-        ref = oracle.combine(np.stack(ys), np.array([pos], np.int32), orc["topk_w"][t:t + 1], 1)
-        assert_float_close(out[t:t + 1], ref, "bf16", f"out[{t}]")
+            ys.append(ref[(c, p)][3])
+        want = oracle.combine(np.stack(ys), np.array([pos], np.int32), orc["topk_w"][t:t + 1], 1)
+        assert_float_close(out[t:t + 1], want, "bf16", f"out[{t}]")
     del g, inp
     torch.cuda.empty_cache()
