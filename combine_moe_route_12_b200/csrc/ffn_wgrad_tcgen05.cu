@@ -34,7 +34,7 @@
 
 namespace moe {
 
-constexpr int kWgStages = 2;
+constexpr int kWgStages = 3;                             // 3 x 64 KiB + 33 KiB staging fits the 227 KiB limit
 constexpr int kWgTile = 128;                              // output rows / columns per tile
 constexpr int kWgRows = 128;                              // token rows per ring stage
 constexpr uint32_t kWgBlockBytes = kWgRows * 128;         // 64 elements x 128 rows (16 KiB)

@@ -4,7 +4,8 @@ on one set of inputs, run the CPU oracle on the same inputs, and compare.
 Tolerances (from the layer's stated contract): indices, drop sets, layouts,
 split counts, routing weights and permuted rows bit-exact; floating outputs
 within max-abs 1e-4 (fp32) or max|a-b| / max|ref| <= 2e-2 (bf16, fp32
-accumulate).
+accumulate), with for bf16 also ||a-b||_2 / ||ref||_2 <= 2e-2 and at most 0.5 %
+of the elements with |ref| > rms(ref) past 2e-2 of their own value.
 """
 from __future__ import annotations
 
@@ -17,6 +18,7 @@ from combine_moe_route_12_b200.workload import MoEInputs, MoEWorkload
 
 F32_ABS_TOL = 1e-4
 BF16_REL_TOL = 2e-2
+SIGNIFICANT_FRAC = 5e-3   # bf16: share of |ref| > rms(ref) elements allowed past 2e-2 relative
 
 
 def storage_np(t: torch.Tensor) -> np.ndarray:
@@ -47,6 +49,17 @@ def assert_float_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str) 
     scale = float(np.max(np.abs(r)))
     rel = err / scale if scale > 0 else err
     assert rel <= BF16_REL_TOL, f"{what}: max err {err:.3e} / max|ref| {scale:.3e} = {rel:.3e}"
+    # the max-normalised bar alone would let an error confined to small values pass:
+    # also the L2-relative error, and among the significant elements (|ref| above
+    # the tensor's rms) the share whose own relative error exceeds the bar
+    nr = float(np.linalg.norm(r))
+    if nr > 0:
+        l2 = float(np.linalg.norm(g - r)) / nr
+        assert l2 <= BF16_REL_TOL, f"{what}: L2-relative error {l2:.3e}"
+        big = np.abs(r) > np.sqrt(np.mean(r * r))
+        if big.any():
+            frac = float(np.mean(np.abs(g[big] - r[big]) > BF16_REL_TOL * np.abs(r[big])))
+            assert frac <= SIGNIFICANT_FRAC, f"{what}: {frac:.2%} of the significant elements beyond the bar"
     return rel
 
 
@@ -219,12 +232,30 @@ def oracle_fp8_ffn_and_out(wl: MoEWorkload, inp: MoEInputs, orc: dict, wq: dict)
     return dict(xq=xq, xs=xs, chunks=res, out=out)
 
 
+def _signed_code(c):
+    """E4M3 codes as signed integers ordered like their values (magnitude field
+    with the sign), so that neighbouring representable values differ by one."""
+    c = np.asarray(c, np.int32)
+    return np.where(c & 0x80, -(c & 0x7F), c & 0x7F)
+
+
 def assert_codes_close(got_codes, got_scales, ref_codes, ref_scales, what, min_equal=0.99):
-    """Quantised rows whose inputs differ by float rounding: almost every code
-    and scale equal, and the dequantised values within the bf16 tolerance."""
+    """Quantised rows whose inputs differ by float rounding (h summed in fp32 on the
+    GPU, in fp64 by the oracle, then rounded to bf16): a value that sits on a
+    rounding boundary can land one code away.  So: almost every code and scale
+    equal; where the scales agree, every differing code is a neighbour of the
+    oracle's (one E4M3 step); the dequantised rows of the other rows within the
+    bf16 bar."""
     if ref_codes.size == 0:
         return
     assert (got_codes == ref_codes).mean() >= min_equal, f"{what}: codes differ too often"
+    got_scales, ref_scales = np.asarray(got_scales), np.asarray(ref_scales)
     assert (got_scales == ref_scales).mean() >= min_equal, f"{what}: scales differ too often"
-    assert_float_close(oracle.dequantize_rows(got_codes, got_scales),
-                       oracle.dequantize_rows(ref_codes, ref_scales), "bf16", what)
+    same = (got_scales == ref_scales).reshape(-1)
+    g2 = np.asarray(got_codes).reshape(len(same), -1)
+    r2 = np.asarray(ref_codes).reshape(len(same), -1)
+    step = np.abs(_signed_code(g2[same]) - _signed_code(r2[same]))
+    assert step.size == 0 or step.max() <= 1, f"{what}: a code differs by {step.max()} steps"
+    if (~same).any():
+        assert_float_close(oracle.dequantize_rows(g2[~same], got_scales.reshape(-1)[~same]),
+                           oracle.dequantize_rows(r2[~same], ref_scales.reshape(-1)[~same]), "bf16", what)
