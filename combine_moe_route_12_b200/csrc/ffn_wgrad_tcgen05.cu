@@ -23,8 +23,10 @@
 // first zeroes that step's rows past the expert (they belong to the next
 // expert, or lie past the valid rows) in both operands.  Warps 0-7 drain TMEM
 // (warps q and q + 4 share lane quadrant q and take alternate 64-column
-// halves), turn each 32 x 32 block around through shared memory and write
-// whole 128-byte row pieces of the fp32 output (or add to it).
+// halves), turn each 32 x 32 block around through shared memory with 16-byte
+// accesses (chunk c of row r stored at chunk c ^ (r % 8): no bank conflicts) and
+// write it as 16-byte stores, eight lanes per 128-byte row piece of the fp32
+// output (or add to it).
 //
 // Every wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT, stops the
 // other roles, lets in-flight copies and MMAs land, frees TMEM and returns.
@@ -44,7 +46,7 @@ constexpr int kWgEpiWarps = 8;
 constexpr int kWgProdWarp = kWgEpiWarps, kWgMmaWarp = kWgEpiWarps + 1;
 constexpr int kWgThreads = 32 * (kWgEpiWarps + 2);
 constexpr uint32_t kWgTmemCols = 2 * kWgTile;             // two 128-column accumulators
-constexpr int kWgPad = 33;                                // staging row stride in floats
+constexpr int kWgPad = 32;                                // staging row stride in floats (16-byte chunks XOR-swizzled by row)
 
 struct WgradParams {
     const int32_t *expert_offsets;   // [n_seg][E + 1]
@@ -256,18 +258,32 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_tcgen05_kernel(
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = 0u;
                 }
-                // row (row0 + lane), columns c0.. : turned around so that each store
-                // below writes 32 consecutive columns of one row
+                // row (row0 + lane), columns c0..c0+31, as eight 16-byte stores into
+                // its staging row (chunk j/4 at chunk (j/4) ^ (lane % 8): the eight
+                // lanes of a store phase hit all 32 banks once)
 #pragma unroll
-                for (int j = 0; j < 32; ++j) my[lane * kWgPad + j] = __uint_as_float(r[j]);
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(my + lane * kWgPad + 4 * ((j >> 2) ^ (lane & 7))) =
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                    __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
                 __syncwarp();
-                const int col = w.nb * kWgTile + c0 + lane;
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int row = row0 + rr;
-                    if (row < P.M && col < P.N) {
-                        float *o = P.out + ((size_t)w.e * P.M + row) * P.N + col;
-                        const float v = my[rr * kWgPad + lane];
-                        *o = P.accumulate ? *o + v : v;
+                // read back four rows per pass: lane -> row rr0 + lane / 8, columns
+                // 4 (lane % 8) .. +3; each row's 32 columns leave as one 128-byte piece
+                const int sub = lane >> 3, cq = (lane & 7) * 4;
+                const int col = w.nb * kWgTile + c0 + cq;
+                const bool full = row0 + 32 <= P.M && w.nb * kWgTile + c0 + 32 <= P.N;
+                float *obase = P.out + ((size_t)w.e * P.M + row0) * P.N + col;
+#pragma unroll
+                for (int rr0 = 0; rr0 < 32; rr0 += 4) {
+                    const int rr = rr0 + sub;
+                    if (full || (row0 + rr < P.M && col < P.N)) {
+                        float4 v = *reinterpret_cast<const float4 *>(my + rr * kWgPad + 4 * ((cq >> 2) ^ (rr & 7)));
+                        float4 *o = reinterpret_cast<float4 *>(obase + (size_t)rr * P.N);
+                        if (P.accumulate) {
+                            const float4 a = *o;
+                            v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
+                        }
+                        *o = v;
                     }
                 }
                 __syncwarp();
