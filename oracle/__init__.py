@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.orc_quantize_blocks.restype = None
         L.orc_dot_blocked.argtypes = [i, i, P, P, P, P]
         L.orc_dot_blocked.restype = ctypes.c_double
+        L.orc_ffn_row_fp8_blocked.argtypes = [i, i, i, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_ffn_row_fp8_blocked.restype = None
         L.orc_combine_bwd.argtypes = [i, i, i, i, i, P, P, P, P, P, P]
         L.orc_combine_bwd.restype = None
         L.orc_route_bwd.argtypes = [i, i, i, P, P, P, P]
@@ -341,6 +343,31 @@ def ffn_row_fp8(x_codes, x_scale, w13_codes, w13_scales, w2_codes, w2_scales):
     lib().orc_ffn_row_fp8(H, I, _p(x_codes), int(x_scale), _p(w13_codes), _p(w13_scales),
                           _p(w2_codes), _p(w2_scales), _p(h), _p(hq), ctypes.byref(sh), _p(y), _p(ye))
     return h, hq, int(sh.value), y, ye
+
+
+def ffn_row_fp8_blocked(x_codes, x_scales, w13_codes, w13_scales, w2_codes, w2_scales, block=32):
+    """One expert's FP8 SwiGLU FFN on one row with K-blocked scales (one UE8M0
+    scale per row and per `block` K values; h quantised by blocks of I).  Returns
+    (h bf16 bits [I], hq codes [I], h scales [I/block], y bf16 bits [H], y_exact [H])."""
+    x_codes = np.ascontiguousarray(x_codes, np.uint8)
+    x_scales = np.ascontiguousarray(x_scales, np.uint8)
+    w13_codes = np.ascontiguousarray(w13_codes, np.uint8)
+    w13_scales = np.ascontiguousarray(w13_scales, np.uint8)
+    w2_codes = np.ascontiguousarray(w2_codes, np.uint8)
+    w2_scales = np.ascontiguousarray(w2_scales, np.uint8)
+    H = x_codes.shape[0]
+    I = w13_codes.shape[0] // 2
+    nbh, nbi = -(-H // block), -(-I // block)
+    assert w13_codes.shape == (2 * I, H) and w2_codes.shape == (H, I)
+    assert x_scales.shape == (nbh,) and w13_scales.shape == (2 * I, nbh) and w2_scales.shape == (H, nbi)
+    h = np.zeros(I, np.uint16)
+    hq = np.zeros(I, np.uint8)
+    hs = np.zeros(nbi, np.uint8)
+    y = np.zeros(H, np.uint16)
+    ye = np.zeros(H, np.float64)
+    lib().orc_ffn_row_fp8_blocked(H, I, block, _p(x_codes), _p(x_scales), _p(w13_codes), _p(w13_scales),
+                                  _p(w2_codes), _p(w2_scales), _p(h), _p(hq), _p(hs), _p(y), _p(ye))
+    return h, hq, hs, y, ye
 
 
 # --------------------------------------------------------------------------- backward

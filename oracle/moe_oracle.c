@@ -773,3 +773,44 @@ double orc_dot_blocked(int K, int block, const uint8_t *a, const uint8_t *sa, co
     }
     return acc;
 }
+
+/* One expert's SwiGLU FFN on one receive row in FP8 with K-blocked scales (the
+ * finer granularity of the LightLLM PR 1687 page's FP8 grouped GEMM: UE8M0
+ * scales along K, four of them packed in an int32).  Reading: one UE8M0 scale
+ * per row and per `block` consecutive K values, chosen as orc_quantize_rows does
+ * for a whole row, for x, W13 and W2 alike, and h quantised by blocks of its I
+ * values.  The steps of orc_ffn_row_fp8 with the blocked dot products:
+ *   x [H] codes, xs [H/block]; w13 [2I, H] codes, w13_s [2I, H/block];
+ *   w2 [H, I] codes, w2_s [H, I/block];
+ *   g_i = orc_dot_blocked(w13 row i, x), u_i = the same with row I + i;
+ *   h_i = silu(g_i) u_i rounded to bf16 (h_store, bf16 bits, optional);
+ *   (hq_store [I], hs_store [I/block]) = orc_quantize_blocks of that bf16 row;
+ *   y_o = orc_dot_blocked(w2 row o, hq) (y_exact optional; y_store bf16). */
+void orc_ffn_row_fp8_blocked(int H, int I, int block, const uint8_t *x, const uint8_t *xs,
+                             const uint8_t *w13, const uint8_t *w13_s, const uint8_t *w2,
+                             const uint8_t *w2_s, uint16_t *h_store, uint8_t *hq_store,
+                             uint8_t *hs_store, uint16_t *y_store, double *y_exact)
+{
+    const int nbh = (H + block - 1) / block, nbi = (I + block - 1) / block;
+    uint16_t *h = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
+    uint8_t *hq = (uint8_t *)malloc((size_t)I);
+    uint8_t *hs = (uint8_t *)malloc((size_t)nbi);
+    for (int i = 0; i < I; ++i) {
+        const double g = orc_dot_blocked(H, block, w13 + (size_t)i * H, w13_s + (size_t)i * nbh, x, xs);
+        const double u = orc_dot_blocked(H, block, w13 + (size_t)(I + i) * H, w13_s + (size_t)(I + i) * nbh,
+                                         x, xs);
+        h[i] = orc_bf16_from_double(g / (1.0 + exp(-g)) * u);
+    }
+    orc_quantize_blocks(1, I, block, 1, h, hq, hs);
+    for (int o = 0; o < H; ++o) {
+        const double acc = orc_dot_blocked(I, block, w2 + (size_t)o * I, w2_s + (size_t)o * nbi, hq, hs);
+        if (y_exact) y_exact[o] = acc;
+        if (y_store) y_store[o] = orc_bf16_from_double(acc);
+    }
+    if (h_store) memcpy(h_store, h, sizeof(uint16_t) * (size_t)I);
+    if (hq_store) memcpy(hq_store, hq, (size_t)I);
+    if (hs_store) memcpy(hs_store, hs, (size_t)nbi);
+    free(h);
+    free(hq);
+    free(hs);
+}

@@ -207,3 +207,82 @@ def test_dot_blocked_equals_library_dequantised_dot():
         ref = float(np.dot(deq(ca[r], sa[r]), deq(cb[r], sb[r])))
         got = oracle.dot_blocked(ca[r], sa[r], cb[r], sb[r], 128)
         assert abs(got - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+# ----------------------------------------------------------------- K-blocked FP8 expert row
+
+def _blocked_operands(rng, H, I, block, uniform_rows=False):
+    """x [H], W13 [2I, H], W2 [H, I] as bf16-representable floats quantised by
+    rows and `block`-column blocks.  uniform_rows: every block of a row holds the
+    row's largest magnitude (its first element), so each block's scale is the row's."""
+    def mat(rows, cols, scale):
+        a = (rng.normal(0, 1, (rows, cols)) * scale).astype(np.float32)
+        a *= np.ldexp(1.0, rng.integers(-3, 4, (rows, 1)))
+        if uniform_rows:
+            m = np.abs(a).max(axis=1, keepdims=True) * 1.5
+            a[:, ::block] = m * np.sign(a[:, ::block] + 0.5)
+        return a
+    x = mat(1, H, 1.0)
+    w13 = mat(2 * I, H, 1.0 / np.sqrt(H))
+    w2 = mat(H, I, 1.0 / np.sqrt(H))
+    q = lambda a: oracle.quantize_blocks(a, block)
+    return q(x), q(w13), q(w2), (x, w13, w2)
+
+
+def test_ffn_row_fp8_blocked_equals_row_form_when_every_block_holds_the_row_max():
+    """When each block's largest magnitude is its row's, every block scale equals
+    the row scale and the codes are those of the row quantisation: g, u and so h
+    must be the row form's bit for bit (block partial sums and the whole sum are
+    both exact in double for E4M3 products)."""
+    rng = np.random.default_rng(21)
+    H, I, block = 128, 64, 32
+    (xq, xs), (wq, ws), (w2q, w2s), raw = _blocked_operands(rng, H, I, block, uniform_rows=True)
+    for a, (c, s) in zip(raw, ((xq, xs), (wq, ws), (w2q, w2s))):
+        cr, sr = oracle.quantize_rows(a)
+        np.testing.assert_array_equal(c, cr)
+        assert (s == sr[:, None]).all()
+    h_b, _, _, _, _ = oracle.ffn_row_fp8_blocked(xq[0], xs[0], wq, ws, w2q, w2s, block)
+    h_r, _, _, _, _ = oracle.ffn_row_fp8(xq[0], xs[0, 0], wq, ws[:, 0], w2q, w2s[:, 0])
+    np.testing.assert_array_equal(h_b, h_r)
+    assert (h_b != 0).sum() > I // 2
+
+
+@pytest.mark.parametrize("block", [32, 128])
+def test_ffn_row_fp8_blocked_against_library_dequantised_matmuls(block):
+    """Every step of the blocked row against library-decoded operands (torch's
+    float8_e4m3fn, each block times its power of two) and numpy matmuls in fp64:
+    g and u, h rounded to bf16 once, h's block quantisation, and y."""
+    rng = np.random.default_rng(22 + block)
+    H, I = 256, 128
+    (xq, xs), (wq, ws), (w2q, w2s), _ = _blocked_operands(rng, H, I, block)
+    h, hq, hs, y, ye = oracle.ffn_row_fp8_blocked(xq[0], xs[0], wq, ws, w2q, w2s, block)
+    deq = lambda c, s: _torch_decode(c) * np.repeat(np.ldexp(1.0, s.astype(np.int32) - 127), block, axis=-1)
+    x = deq(xq[0], xs[0])
+    g = deq(wq[:I], ws[:I]) @ x
+    u = deq(wq[I:], ws[I:]) @ x
+    hv = g / (1.0 + np.exp(-g)) * u
+    h_ref = np.array([oracle.bf16_bits_from_double(v) for v in hv], np.uint16)
+    # the fp64 sums run in another order: h may differ where a value sits on a bf16 boundary
+    assert (h == h_ref).mean() >= 0.99
+    hq_ref, hs_ref = oracle.quantize_blocks(h[None], block)
+    np.testing.assert_array_equal(hq, hq_ref[0])
+    np.testing.assert_array_equal(hs, hs_ref[0])
+    ref = deq(w2q, w2s) @ deq(hq, hs)
+    np.testing.assert_allclose(ye, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    np.testing.assert_array_equal(y, [oracle.bf16_bits_from_double(v) for v in ye])
+    assert len(set(hs.tolist())) > 1 or I == block     # blocks take their own scales
+
+
+def test_ffn_row_fp8_blocked_block_scale_multiplies_its_block_only():
+    """Raising one W2 block scale by 3 multiplies that block's contribution to its
+    output by 8 and changes nothing else."""
+    rng = np.random.default_rng(25)
+    H, I, block = 64, 64, 32
+    (xq, xs), (wq, ws), (w2q, w2s), _ = _blocked_operands(rng, H, I, block)
+    h, hq, hs, _, ye = oracle.ffn_row_fp8_blocked(xq[0], xs[0], wq, ws, w2q, w2s, block)
+    w2s2 = w2s.copy()
+    w2s2[7, 1] += 3
+    _, _, _, _, ye2 = oracle.ffn_row_fp8_blocked(xq[0], xs[0], wq, ws, w2q, w2s2, block)
+    part = lambda s: oracle.dot_blocked(w2q[7, 32:], s[7, 1:], hq[32:], hs[1:], block)
+    assert abs((ye2[7] - ye[7]) - 7 * part(w2s)) <= 1e-12 * max(1.0, abs(ye[7]))
+    np.testing.assert_array_equal(np.delete(ye2, 7), np.delete(ye, 7))
