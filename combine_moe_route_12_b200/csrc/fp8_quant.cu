@@ -191,6 +191,115 @@ cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ K-blocked scales
+// One UE8M0 scale per 32 consecutive values of a row (the MX block of the
+// block-scaled tensor-core MMA): a row-major [rows, cols] array with cols % 32 ==
+// 0 is a flat run of 32-value blocks.  LPB consecutive lanes take one block (4
+// bf16 or 8 fp32 vectors of 16 bytes), its maximum by shuffles among them; the
+// codes as in the row form; scales[b] for block b (row-major [rows, cols / 32]).
+template <bool BF16>
+__global__ void __launch_bounds__(256) quant_blocks_kernel(int64_t n_blocks, const uint4 *__restrict__ src,
+                                                           uint8_t *__restrict__ codes,
+                                                           uint8_t *__restrict__ scales) {
+    constexpr int LPB = BF16 ? 4 : 8;      // lanes per block
+    const int64_t n_vec = n_blocks * LPB;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    // every lane of a warp runs the same trips (the shuffles need them all)
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); v0 < n_vec; v0 += step) {
+        const int64_t v = v0 + (threadIdx.x & 31);
+        const bool live = v < n_vec;
+        const uint4 q = live ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+        float amax = vec_amax<BF16>(q);
+#pragma unroll
+        for (int off = 1; off < LPB; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (!live) continue;
+        const int e = ue8m0_exponent(amax);
+        const float inv = pow2_neg(e);
+        if (BF16) {
+            reinterpret_cast<uint2 *>(codes)[v] = bf16_vec_codes(q, inv);
+        } else {
+            reinterpret_cast<uint32_t *>(codes)[v] =
+                e4m3x2(__uint_as_float(q.x) * inv, __uint_as_float(q.y) * inv) |
+                e4m3x2(__uint_as_float(q.z) * inv, __uint_as_float(q.w) * inv) << 16;
+        }
+        if ((v & (LPB - 1)) == 0) scales[v / LPB] = (uint8_t)(e + 127);
+    }
+}
+
+cudaError_t launch_quant_blocks(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
+                                uint8_t *scales, cudaStream_t s, int num_sms) {
+    const int64_t n_blocks = rows * (int64_t)(cols / 32);
+    if (n_blocks <= 0) return cudaSuccess;
+    const int64_t n_vec = n_blocks * (bf16 ? 4 : 8);
+    long long grid = (n_vec + 255) / 256;
+    const long long cap = (long long)num_sms * 8;
+    if (grid > cap) grid = cap;
+    if (bf16)
+        quant_blocks_kernel<true><<<(unsigned)grid, 256, 0, s>>>(n_blocks, static_cast<const uint4 *>(in),
+                                                                codes, scales);
+    else
+        quant_blocks_kernel<false><<<(unsigned)grid, 256, 0, s>>>(n_blocks, static_cast<const uint4 *>(in),
+                                                                 codes, scales);
+    return cudaGetLastError();
+}
+
+// Quantise-and-permute with K-blocked scales: one CTA per token of the chunk;
+// thread t holds vectors t, t + 128, ... of the bf16 row (a 32-value block is
+// four consecutive vectors, so four consecutive lanes), the block maximum by two
+// shuffles; each kept receive row p gets the codes and the row's block scales
+// (xr_sf [N_max, H / 32]).  A token with every slot dropped is not read.
+template <int VPT>
+__global__ void __launch_bounds__(kPqThreads) permute_quant_blocks_kernel(
+    int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
+    uint8_t *__restrict__ xr_q, uint8_t *__restrict__ xr_sf) {
+    __shared__ int32_t s_pos[kMaxTopK];
+    __shared__ int s_any;
+    const int i = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        const int p = lane < k ? pos[(size_t)i * k + lane] : -1;
+        if (lane < k) s_pos[lane] = p;
+        const uint32_t any = __ballot_sync(0xffffffffu, p >= 0);
+        if (lane == 0) s_any = any != 0u;
+    }
+    __syncthreads();
+    if (!s_any) return;
+    const uint4 *src = x + (size_t)(tb + i) * row_vecs;
+    const size_t row_bytes = (size_t)row_vecs * 8, sf_bytes = (size_t)row_vecs / 4;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+        const int v = threadIdx.x + kPqThreads * j;
+        const uint4 q = v < row_vecs ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+        float amax = vec_amax<true>(q);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        if (v >= row_vecs) continue;
+        const int e = ue8m0_exponent(amax);
+        const uint2 c = bf16_vec_codes(q, pow2_neg(e));
+        for (int jj = 0; jj < k; ++jj) {
+            const int p = s_pos[jj];
+            if (p < 0) continue;
+            reinterpret_cast<uint2 *>(xr_q + (size_t)p * row_bytes)[v] = c;
+            if ((v & 3) == 0) xr_sf[(size_t)p * sf_bytes + v / 4] = (uint8_t)(e + 127);
+        }
+    }
+}
+
+// Returns cudaErrorNotSupported for rows longer than 1024 vectors (8192 values).
+cudaError_t launch_permute_quant_blocks(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                                        int tc, uint8_t *xr_q, uint8_t *xr_sf, cudaStream_t s) {
+    if (tc == 0) return cudaSuccess;
+    const int row_vecs = c.H / 8;
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    if (row_vecs <= 2 * kPqThreads)
+        permute_quant_blocks_kernel<2><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
+    else if (row_vecs <= 8 * kPqThreads)
+        permute_quant_blocks_kernel<8><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
+    else
+        return cudaErrorNotSupported;
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
                               uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms) {
     if (rows <= 0) return cudaSuccess;

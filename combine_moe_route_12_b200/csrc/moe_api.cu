@@ -47,6 +47,15 @@ cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in,
                               uint8_t *scales, const int32_t *n_dev, cudaStream_t s, int num_sms);
 cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32_t *pos, int tb,
                                  int tc, uint8_t *xr_q, uint8_t *x_scale, cudaStream_t s);
+cudaError_t launch_quant_blocks(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,
+                                uint8_t *scales, cudaStream_t s, int num_sms);
+cudaError_t launch_permute_quant_blocks(const moe_config &c, const void *x, const int32_t *pos, int tb,
+                                        int tc, uint8_t *xr_q, uint8_t *xr_sf, cudaStream_t s);
+cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr_q, const uint8_t *xr_sf,
+                          const int32_t *expert_offsets, const uint8_t *w13_q, const uint8_t *w13_sf,
+                          const uint8_t *w2_q, const uint8_t *w2_sf, uint8_t *h_q, uint8_t *h_sf, void *y,
+                          const int32_t *recv_token, const int32_t *recv_slot, const float *topk_w,
+                          float *out_reduce, uint32_t *status, cudaStream_t s, int num_sms);
 cudaError_t launch_combine_bwd(const moe_config &c, const void *dout, const void *y,
                                const int32_t *pos, const float *topk_w, int tb, int tc, void *dy,
                                float *dw, cudaStream_t s);
@@ -142,7 +151,8 @@ bool fused_permute_quant(const moe_config &c) { return c.H <= 8192; }
 struct Slot {
     size_t eoff, roff, recv_token, recv_slot, pos, splits, xr, h, y;
     size_t hs, ys;   // the shared expert's h and y for the chunk's rows (shared_I > 0)
-    size_t hq, hsc;  // ffn_fp8: h's E4M3 codes and row scales
+    size_t hq, hsc;  // ffn_fp8: h's E4M3 codes and scales (one per row, or per 32 values: [nmax, I/32])
+    size_t xsf;      // ffn_fp8 = 2: the receive rows' scales [nmax, H/32]
 };
 struct ForwardLayout {
     size_t counts, kept_counts;
@@ -182,10 +192,11 @@ ForwardLayout forward_layout(const moe_config &c, bool host_io = false) {
         S.hs = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.shared_I) : 0;
         S.ys = c.shared_I > 0 ? take(eb * (size_t)F.tc * c.H) : 0;
         S.hq = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1) * c.I) : 0;
-        S.hsc = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1)) : 0;
+        S.hsc = c.ffn_fp8 ? take((size_t)(F.nmax > 0 ? F.nmax : 1) * (c.ffn_fp8 == 2 ? c.I / 32 : 1)) : 0;
+        S.xsf = c.ffn_fp8 == 2 ? take((size_t)(F.nmax > 0 ? F.nmax : 1) * (c.H / 32)) : 0;
     }
-    F.xq = c.ffn_fp8 && !fused_permute_quant(c) ? take((size_t)c.T * c.H) : 0;
-    F.xsc = c.ffn_fp8 ? take((size_t)c.T) : 0;
+    F.xq = c.ffn_fp8 == 1 && !fused_permute_quant(c) ? take((size_t)c.T * c.H) : 0;
+    F.xsc = c.ffn_fp8 == 1 ? take((size_t)c.T) : 0;
     F.out_reduce = c.reduce_dense ? take(sizeof(float) * (size_t)c.T * c.H) : 0;
     if (host_io) {
         F.stage_logits = take(sizeof(float) * (size_t)c.T * c.E);
@@ -300,12 +311,15 @@ moe_status moe_config_check(const moe_config *cfg) {
     if (c.bias_select_only != 0 && c.bias_select_only != 1)
         return fail(MOE_ERR_INVALID_ARG, "bias_select_only must be 0 or 1");
     if (c.shared_I < 0) return fail(MOE_ERR_INVALID_ARG, "shared_I=%d < 0", c.shared_I);
-    if (c.ffn_fp8 != 0 && c.ffn_fp8 != 1) return fail(MOE_ERR_INVALID_ARG, "ffn_fp8 must be 0 or 1");
+    if (c.ffn_fp8 < 0 || c.ffn_fp8 > 2) return fail(MOE_ERR_INVALID_ARG, "ffn_fp8 must be 0, 1 or 2");
     if (c.ffn_fp8) {
         if (c.dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 needs dtype MOE_BF16");
         if (c.H % 128 != 0 || c.I % 128 != 0)
             return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 needs H and I multiples of 128 (H=%d, I=%d)", c.H, c.I);
         if (c.shared_I != 0) return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 with a shared expert");
+        if (c.ffn_fp8 == 2 && (c.E > 512 || c.H > 8192))
+            return fail(MOE_ERR_UNSUPPORTED, "ffn_fp8 = 2 (K-blocked scales) needs E <= 512 and H <= 8192 "
+                        "(E=%d, H=%d)", c.E, c.H);
     }
     if (c.shared_I > 0 && c.dtype == MOE_BF16 && c.shared_I % 64 != 0)
         return fail(MOE_ERR_UNSUPPORTED, "bf16 needs shared_I a multiple of 64 (got %d)", c.shared_I);
@@ -432,7 +446,8 @@ moe_status moe_grouped_swiglu_ffn(const moe_config *cfg, int64_t n_rows, const v
     if ((st = check_ws(ws)) != MOE_OK) return st;
     const moe_config &c = *cfg;
     if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
-    if (c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 1: use moe_grouped_swiglu_ffn_fp8");
+    if (c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = %d: use moe_grouped_swiglu_ffn_%s",
+                               c.ffn_fp8, c.ffn_fp8 == 2 ? "mxfp8" : "fp8");
     if (n_rows == 0) return MOE_OK;
     if (!xr || !expert_offsets || !w13 || !w2 || !h)
         return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
@@ -538,7 +553,8 @@ moe_status moe_permute_quantize_fp8(const moe_config *cfg, const void *x, const 
     moe_status st = moe_config_check(cfg);
     if (st != MOE_OK) return st;
     const moe_config &c = *cfg;
-    if (!c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 0: use moe_permute");
+    if (c.ffn_fp8 != 1) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = %d: use moe_permute%s", c.ffn_fp8,
+                                    c.ffn_fp8 == 2 ? "_quantize_fp8_blocks" : "");
     if (!fused_permute_quant(c)) return fail(MOE_ERR_UNSUPPORTED, "H=%d > 8192", c.H);
     if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
     if (tok_count > 0 && (!x || !pos || !xr_q || !x_scale))
@@ -560,7 +576,8 @@ moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, con
     if (st != MOE_OK) return st;
     if ((st = check_ws(ws)) != MOE_OK) return st;
     const moe_config &c = *cfg;
-    if (!c.ffn_fp8) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = 0: use moe_grouped_swiglu_ffn");
+    if (c.ffn_fp8 != 1) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 = %d: use moe_grouped_swiglu_ffn%s",
+                                    c.ffn_fp8, c.ffn_fp8 == 2 ? "_mxfp8" : "");
     if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
     if (n_rows == 0) return MOE_OK;
     if (!xr_q || !x_scale || !expert_offsets || !w13_q || !w13_scale || !w2_q || !w2_scale || !h ||
@@ -590,6 +607,79 @@ moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, con
     if (err == cudaErrorNotSupported)
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn_fp8");
+}
+
+moe_status moe_quantize_fp8_blocks(int64_t rows, int32_t cols, int32_t in_dtype, const void *in,
+                                   uint8_t *codes, uint8_t *scales, cudaStream_t stream) {
+    if (rows < 0 || cols < 1) return fail(MOE_ERR_INVALID_ARG, "rows < 0 or cols < 1");
+    if (in_dtype != MOE_BF16 && in_dtype != MOE_F32)
+        return fail(MOE_ERR_INVALID_ARG, "in_dtype must be MOE_BF16 or MOE_F32");
+    if (cols % 32 != 0) return fail(MOE_ERR_UNSUPPORTED, "cols %% 32 != 0 (cols=%d)", cols);
+    if (rows == 0) return MOE_OK;
+    if (!in || !codes || !scales) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    const bool bf16 = in_dtype == MOE_BF16;
+    if (!aligned(in, 16) || !aligned(codes, bf16 ? 8 : 4))
+        return fail(MOE_ERR_INVALID_ARG, "in not 16-byte or codes not %d-byte aligned", bf16 ? 8 : 4);
+    cudaError_t err = launch_quant_blocks(rows, cols, bf16, in, codes, scales, stream, current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_quantize_fp8_blocks");
+}
+
+moe_status moe_permute_quantize_fp8_blocks(const moe_config *cfg, const void *x, const int32_t *pos,
+                                           int32_t tok_begin, int32_t tok_count, uint8_t *xr_q,
+                                           uint8_t *xr_sf, cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.ffn_fp8 != 2) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 must be 2 (K-blocked scales)");
+    if (!fused_permute_quant(c)) return fail(MOE_ERR_UNSUPPORTED, "H=%d > 8192", c.H);
+    if ((st = check_range(c, tok_begin, tok_count, false)) != MOE_OK) return st;
+    if (tok_count > 0 && (!x || !pos || !xr_q || !xr_sf))
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned(x, 16) || !aligned(xr_q, 16)) return fail(MOE_ERR_INVALID_ARG, "x / xr_q not 16-byte aligned");
+    cudaError_t err = launch_permute_quant_blocks(c, x, pos, tok_begin, tok_count, xr_q, xr_sf, stream);
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute_quantize_fp8_blocks");
+}
+
+moe_status moe_grouped_swiglu_ffn_mxfp8(const moe_config *cfg, int64_t n_rows, const uint8_t *xr_q,
+                                        const uint8_t *xr_sf, const int32_t *expert_offsets,
+                                        const uint8_t *w13_q, const uint8_t *w13_sf, const uint8_t *w2_q,
+                                        const uint8_t *w2_sf, uint8_t *h_q, uint8_t *h_sf, void *y,
+                                        const int32_t *recv_token, const int32_t *recv_slot,
+                                        const float *topk_w, float *out_reduce, void *ws,
+                                        cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.ffn_fp8 != 2) return fail(MOE_ERR_INVALID_ARG, "cfg->ffn_fp8 must be 2 (K-blocked scales)");
+    if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows < 0");
+    if (n_rows == 0) return MOE_OK;
+    if (!xr_q || !xr_sf || !expert_offsets || !w13_q || !w13_sf || !w2_q || !w2_sf || !h_q || !h_sf)
+        return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (c.reduce_dense) {
+        if (!recv_token || !recv_slot || !topk_w || !out_reduce)
+            return fail(MOE_ERR_INVALID_ARG, "decode form needs recv_token, recv_slot, topk_w, out_reduce");
+    } else if (!y) {
+        return fail(MOE_ERR_INVALID_ARG, "y is NULL");
+    }
+    const void *a16[5] = {xr_q, w13_q, w2_q, h_q, y};
+    for (const void *p : a16)
+        if (p && !aligned(p, 16)) return fail(MOE_ERR_INVALID_ARG, "operand not 16-byte aligned");
+    const void *a4[4] = {xr_sf, w13_sf, w2_sf, h_sf};
+    for (const void *p : a4)
+        if (!aligned(p, 4)) return fail(MOE_ERR_INVALID_ARG, "scale array not 4-byte aligned");
+    int dev = 0, major = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10)
+        return fail(MOE_ERR_UNSUPPORTED, "the MX FP8 FFN uses tcgen05 and needs sm_100 (got major %d)", major);
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_ffn_mx(c, n_rows, xr_q, xr_sf, expert_offsets, w13_q, w13_sf, w2_q, w2_sf, h_q,
+                                    h_sf, y, recv_token, recv_slot, topk_w, out_reduce,
+                                    ws_at<uint32_t>(ws, L.status), stream, current_num_sms());
+    if (err == cudaErrorNotSupported)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn_mxfp8");
 }
 
 // The shared expert over rows [tb, tb + tc) of x: the step-5 kernel as one
@@ -821,7 +911,11 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
                                        ws, F.nmax, s_dispatch, nsm),
                 "dispatch_layout");
         if (io) MOE_TRY(cudaStreamWaitEvent(s_dispatch, ev_x[ch], 0), "wait x");
-        if (c.ffn_fp8 && fused_permute_quant(c)) {
+        if (c.ffn_fp8 == 2) {
+            // codes of the kept rows and their 32-value block scales, per receive row
+            MOE_TRY(launch_permute_quant_blocks(c, x, pos, tb, tc, static_cast<uint8_t *>(xr),
+                                                ws_at<uint8_t>(ws, S.xsf), s_dispatch), "permute + quantize x");
+        } else if (c.ffn_fp8 && fused_permute_quant(c)) {
             // each kept token row quantised once and its codes written to its receive rows
             MOE_TRY(launch_permute_quant(c, x, pos, tb, tc, static_cast<uint8_t *>(xr),
                                          ws_at<uint8_t>(ws, F.xsc), s_dispatch), "permute + quantize x");
@@ -849,7 +943,14 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
         if (io && ch >= 1) MOE_TRY(copy_out(ch - 1), "copy out");
         MOE_TRY(cudaStreamWaitEvent(s_compute, ev_disp[ch], 0), "wait dispatch");
         if (F.nmax > 0) {
-            if (c.ffn_fp8) {
+            if (c.ffn_fp8 == 2) {
+                err = launch_ffn_mx(c, F.nmax, static_cast<const uint8_t *>(xr), ws_at<uint8_t>(ws, S.xsf), eoff,
+                                    static_cast<const uint8_t *>(w13), w13_scale, static_cast<const uint8_t *>(w2),
+                                    w2_scale, ws_at<uint8_t>(ws, S.hq), ws_at<uint8_t>(ws, S.hsc), y, recv_token,
+                                    recv_slot, topk_w, out_reduce, status, s_compute, nsm);
+                if (err == cudaErrorNotSupported)
+                    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
+            } else if (c.ffn_fp8) {
                 err = launch_ffn_tcgen05_fp8(c, F.nmax, static_cast<const uint8_t *>(xr),
                                              ws_at<uint8_t>(ws, F.xsc), eoff,
                                              static_cast<const uint8_t *>(w13), w13_scale,

@@ -408,6 +408,14 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
         ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(mbar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(void *smem_dst, const void *tmap, uint64_t *mbar,
+                                            int32_t x, int32_t y, int32_t z, int32_t w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(mbar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_1(uint32_t *smem_dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(smem_dst)), "r"(ncols) : "memory");
@@ -432,6 +440,42 @@ __device__ __forceinline__ void tc_commit_1(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
 }
+// ---------------------------------------------------------------- block-scaled FP8 (MX) tcgen05
+// Shared-memory descriptor of a 512-byte scale-factor atom for tcgen05.cp: 32
+// rows of 16 bytes, no swizzle (K-major, 8-row core groups 128 bytes apart).
+__device__ __forceinline__ uint64_t make_sf_atom_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;                 // leading byte offset 16 (one 16-byte column)
+    d |= (uint64_t)(128u >> 4) << 32;        // stride byte offset 128
+    d |= (uint64_t)1u << 46;                 // version 1; layout 0 = no swizzle
+    return d;
+}
+// 32 TMEM lanes x 128 bits from the atom, the same into each of the four lane
+// quadrants (tmem_col .. tmem_col + 3).
+__device__ __forceinline__ void tc_cp_sf_atom(uint32_t tmem_col, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col), "l"(sdesc) : "memory");
+}
+// Instruction descriptor of kind::mxf8f6f4 with E4M3 A and B, UE8M0 scale
+// factors (scale format bit 23), K-major operands, the scale byte sf_id of the
+// TMEM scale words for both A (bits 29-30) and B (bits 4-5).
+__host__ __device__ constexpr uint32_t make_idesc_mx_e4m3(int M, int N, uint32_t sf_id) {
+    return ((sf_id & 3u) << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+           ((sf_id & 3u) << 29);
+}
+// D (+)= (A * 2^sfa) * (B * 2^sfb)^T with one UE8M0 scale per row (column) and
+// 32 K values, the scales read from TMEM at tsfa / tsfb (top two address bits:
+// the scale byte).  Single CTA, M = 128.
+__device__ __forceinline__ void tc_mma_mx_1(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                            uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                 : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads of them (the tensor core's operand fetch, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -77,6 +77,9 @@ _decl("moe_forward_host", _I32, _CFG, *([_P] * 17))
 _decl("moe_quantize_fp8_rows", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
 _decl("moe_grouped_swiglu_ffn_fp8", _I32, _CFG, ctypes.c_int64, *([_P] * 17))
 _decl("moe_permute_quantize_fp8", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_quantize_fp8_blocks", _I32, ctypes.c_int64, _I32, _I32, _P, _P, _P, _P)
+_decl("moe_permute_quantize_fp8_blocks", _I32, _CFG, _P, _P, _I32, _I32, _P, _P, _P)
+_decl("moe_grouped_swiglu_ffn_mxfp8", _I32, _CFG, ctypes.c_int64, *([_P] * 14), _P, _P)
 _decl("moe_grouped_swiglu_ffn_backward", _I32, _CFG, ctypes.c_int64, *([_P] * 11), _I32, _P, _P)
 _decl("moe_combine_backward", _I32, _CFG, _P, _P, _P, _P, _I32, _I32, _P, _P, _P)
 _decl("moe_route_backward", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
@@ -128,7 +131,7 @@ def make_config(T, H, E, k, I, ep, capacity=-1, dtype=MOE_BF16, n_chunks=1,
         dtype = MOE_F32 if dtype == "f32" else MOE_BF16
     return MoEConfig(T, H, E, k, I, ep, -1 if capacity is None else capacity, dtype, n_chunks,
                      int(bool(reduce_dense)), n_group, topk_group, group_score,
-                     int(bool(bias_select_only)), shared_I, int(bool(ffn_fp8)))
+                     int(bool(bias_select_only)), shared_I, int(ffn_fp8))
 
 
 def config_from_workload(wl) -> MoEConfig:
@@ -228,6 +231,40 @@ def quantize_fp8(inp, stream=None):
     scales = torch.empty(flat.shape[0], dtype=torch.uint8, device=inp.device)
     moe_quantize_fp8_rows(flat, codes, scales, stream)
     return codes.view(inp.shape), scales.view(inp.shape[:-1])
+
+
+def moe_quantize_fp8_blocks(inp, codes, scales, stream=None):
+    """E4M3 codes and one UE8M0 scale byte per 32 values of each row of a bf16 or
+    fp32 [rows, cols] tensor (scales [rows, cols / 32])."""
+    rows, cols = inp.shape
+    in_dtype = MOE_BF16 if inp.dtype == torch.bfloat16 else MOE_F32
+    assert codes.dtype == torch.uint8 and scales.dtype == torch.uint8
+    assert tuple(codes.shape) == (rows, cols) and scales.numel() >= rows * (cols // 32)
+    _check(_lib.moe_quantize_fp8_blocks(rows, cols, in_dtype, _ptr(inp), _ptr(codes), _ptr(scales),
+                                        _stream(stream)))
+
+
+def quantize_fp8_blocks(inp, stream=None):
+    """(codes, scales [..., cols / 32]) of moe_quantize_fp8_blocks over the last dimension."""
+    flat = inp.reshape(-1, inp.shape[-1])
+    codes = torch.empty(flat.shape, dtype=torch.uint8, device=inp.device)
+    scales = torch.empty(flat.shape[0], flat.shape[1] // 32, dtype=torch.uint8, device=inp.device)
+    moe_quantize_fp8_blocks(flat, codes, scales, stream)
+    return codes.view(inp.shape), scales.view(*inp.shape[:-1], inp.shape[-1] // 32)
+
+
+def moe_permute_quantize_fp8_blocks(cfg, x, pos, tok_begin, tok_count, xr_q, xr_sf, stream=None):
+    """Kept token rows of x quantised by 32-value blocks; codes and scales to their receive rows."""
+    _check(_lib.moe_permute_quantize_fp8_blocks(ctypes.byref(cfg), _ptr(x), _ptr(pos), tok_begin,
+                                                tok_count, _ptr(xr_q), _ptr(xr_sf), _stream(stream)))
+
+
+def moe_grouped_swiglu_ffn_mxfp8(cfg, n_rows, xr_q, xr_sf, expert_offsets, w13_q, w13_sf, w2_q, w2_sf,
+                                 h_q, h_sf, y, recv_token, recv_slot, topk_w, out_reduce, ws, stream=None):
+    _check(_lib.moe_grouped_swiglu_ffn_mxfp8(
+        ctypes.byref(cfg), n_rows, _ptr(xr_q), _ptr(xr_sf), _ptr(expert_offsets), _ptr(w13_q),
+        _ptr(w13_sf), _ptr(w2_q), _ptr(w2_sf), _ptr(h_q), _ptr(h_sf), _ptr(y), _ptr(recv_token),
+        _ptr(recv_slot), _ptr(topk_w), _ptr(out_reduce), _ptr(ws), _stream(stream)))
 
 
 def moe_permute_quantize_fp8(cfg, x, pos, tok_begin, tok_count, xr_q, x_scale, stream=None):

@@ -43,7 +43,7 @@ Input recipe (the pages fix none of it; every choice is a stated reading):
   bias[e] ~ N(0, 0.5^2) (seeded) that steers the selection only.
 * ``qwen3_30b_a3b_fp8`` and ``dsv3_prefill_fp8``: the Qwen3 and DSV3 prefill
   shapes with the expert FFN in FP8 (LightLLM PR 1687: FP8 grouped GEMM with
-  UE8M0 scales).  Inputs are drawn exactly as for the bf16 workloads; the
+  UE8M0 scales); ``*_mxfp8``: the same with one scale per 32 K values.  Inputs are drawn exactly as for the bf16 workloads; the
   weights are quantised row by row to E4M3 codes with UE8M0 scales once, before
   the layer runs, and x per call inside it.
 """
@@ -77,7 +77,8 @@ class MoEWorkload:
     bias_select_only: bool = False
     balance_bias: bool = False    # a small per-expert bias ~ N(0, 0.5^2), the load-balancing kind
     shared_I: int = 0             # a shared expert of this intermediate size (0: none)
-    ffn_fp8: bool = False         # the expert FFN on E4M3 codes with UE8M0 row scales
+    ffn_fp8: int = 0              # the expert FFN on E4M3 codes: 1 with UE8M0 row scales,
+                                  # 2 with one UE8M0 scale per 32 K values
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -112,6 +113,12 @@ WORKLOADS = {
                                      dtype="bf16", ep=2, ffn_fp8=True),
     "dsv3_prefill_fp8": MoEWorkload("dsv3_prefill_fp8", T=8192, H=7168, E=256, k=8, I=2048,
                                     dtype="bf16", ep=8, n_chunks=2, ffn_fp8=True),
+    # the expert FFN in FP8 with K-blocked scales (one per 32 values), h quantised
+    # inside the SwiGLU epilogue
+    "qwen3_30b_a3b_mxfp8": MoEWorkload("qwen3_30b_a3b_mxfp8", T=4096, H=2048, E=128, k=8, I=768,
+                                       dtype="bf16", ep=2, ffn_fp8=2),
+    "dsv3_prefill_mxfp8": MoEWorkload("dsv3_prefill_mxfp8", T=8192, H=7168, E=256, k=8, I=2048,
+                                      dtype="bf16", ep=8, n_chunks=2, ffn_fp8=2),
 }
 
 

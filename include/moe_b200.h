@@ -22,7 +22,10 @@
  * the combine adds; moe_dispatch_layout_noalloc, step 3 with its scratch in a
  * fixed library array; moe_quantize_fp8_rows, moe_permute_quantize_fp8 and
  * moe_grouped_swiglu_ffn_fp8, the expert FFN on E4M3 codes with UE8M0 row
- * scales (cfg->ffn_fp8);
+ * scales (cfg->ffn_fp8 = 1); moe_quantize_fp8_blocks,
+ * moe_permute_quantize_fp8_blocks and moe_grouped_swiglu_ffn_mxfp8, the same
+ * with one UE8M0 scale per 32 K values and h quantised inside the SwiGLU
+ * epilogue (cfg->ffn_fp8 = 2);
  * moe_grouped_swiglu_ffn_backward, the expert FFN's backward (data and
  * weight gradients); moe_combine_backward, moe_route_backward and
  * moe_permute_backward, the backward's row passes; moe_watchdog_selftest, which makes a bounded wait run
@@ -110,8 +113,8 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * bias_select_only in {0, 1}, shared_I >= 0 (a multiple of 64 for MOE_BF16, of
  * 4 for MOE_F32).
  * Limits (MOE_ERR_UNSUPPORTED): k <= 32, E <= 1024, ep <= E, T*k < 2^30,
- * n_group <= 32; ffn_fp8 = 1 only with MOE_BF16, H % 128 == I % 128 == 0 and
- * shared_I = 0;
+ * n_group <= 32; ffn_fp8 = 1 or 2 only with MOE_BF16, H % 128 == I % 128 == 0
+ * and shared_I = 0 (2: also E <= 512 and H <= 8192);
  * MOE_BF16 needs H % 64 == 0 and I % 64 == 0 (tensor-core tiles);
  * MOE_F32 needs H % 4 == 0 and I % 4 == 0.
  */
@@ -148,8 +151,10 @@ typedef struct {
     /* FP8 expert FFN ([LL]: the FP8 grouped GEMM with UE8M0 scales over the
      * psum layout, silu_and_mul followed by quantisation): 1 runs step 5 on
      * E4M3 codes with one UE8M0 (power-of-two) scale per row, see
-     * moe_quantize_fp8_rows; the permuted rows are then E4M3 codes.  Needs
-     * dtype MOE_BF16, H and I multiples of 128 and shared_I = 0. */
+     * moe_quantize_fp8_rows; the permuted rows are then E4M3 codes.  2 runs
+     * it with one UE8M0 scale per row and 32 K values (moe_quantize_fp8_blocks,
+     * moe_grouped_swiglu_ffn_mxfp8).  Needs dtype MOE_BF16, H and I multiples
+     * of 128 and shared_I = 0. */
     int32_t ffn_fp8;
 } moe_config;
 
@@ -355,6 +360,63 @@ moe_status moe_grouped_swiglu_ffn_fp8(const moe_config *cfg, int64_t n_rows, con
                                       cudaStream_t stream);
 
 /*
+ * FP8 quantisation with K-blocked scales (LightLLM PR 1687: UE8M0 scales along
+ * K, packed four to an int32; the pages give no block length).  Reading: one
+ * UE8M0 scale per row and per 32 consecutive values - the block the
+ * block-scaled tcgen05 MMA (kind::mxf8f6f4) applies - chosen and applied as
+ * moe_quantize_fp8_rows does for a whole row:
+ *   scales[r, b] = e + 127 with e the smallest integer such that the largest
+ *       |in[r, 32b .. 32b+31]| <= 448 * 2^e (clamped to [-126, 127], 0 for a
+ *       zero block);  codes[r, c] = E4M3(in[r, c] / 2^e), nearest even,
+ *       saturating.
+ *   in [rows, cols] (MOE_BF16 or MOE_F32), cols % 32 == 0; codes [rows, cols];
+ *   scales [rows, cols / 32] bytes - four consecutive ones read as an int32
+ *   (block 4i in the low byte) are the packed form.
+ * Use it once on W13 ([E*2I, H] rows) and W2 ([E*H, I] rows) for
+ * moe_grouped_swiglu_ffn_mxfp8.
+ */
+moe_status moe_quantize_fp8_blocks(int64_t rows, int32_t cols, int32_t in_dtype, const void *in,
+                                   uint8_t *codes, uint8_t *scales, cudaStream_t stream);
+
+/*
+ * Steps 4 and the K-blocked quantisation of x fused (cfg->ffn_fp8 = 2): for t in
+ * [tok_begin, tok_begin + tok_count) with a kept slot, x[t] (bf16) is quantised
+ * as moe_quantize_fp8_blocks does and each kept receive row p gets its codes in
+ * xr_q [N_max, H] and its block scales in xr_sf [N_max, H/32] (the scales are
+ * stored per receive row, beside the codes).  Rows of tokens without a kept slot
+ * are left untouched.  Needs H <= 8192.
+ */
+moe_status moe_permute_quantize_fp8_blocks(const moe_config *cfg, const void *x, const int32_t *pos,
+                                           int32_t tok_begin, int32_t tok_count, uint8_t *xr_q,
+                                           uint8_t *xr_sf, cudaStream_t stream);
+
+/*
+ * Step 5 in FP8 with K-blocked UE8M0 scales (cfg->ffn_fp8 = 2; [LL] the FP8
+ * grouped GEMM over the psum layout with UE8M0 scales, and silu_and_mul with the
+ * quantisation of its output): value = E4M3(code) * 2^(scale - 127), one scale
+ * per row and 32 K values, on every operand:
+ *   xr_q [n_rows, H], xr_sf [n_rows, H/32]: the receive rows
+ *        (moe_permute_quantize_fp8_blocks);
+ *   w13_q [E, 2I, H] with w13_sf [E*2I, H/32], w2_q [E, H, I] with
+ *        w2_sf [E*H, I/32] (moe_quantize_fp8_blocks);
+ *   g, u = the dequantised dot products (tcgen05 kind::mxf8f6f4 with the block
+ *        scales read from TMEM, fp32 accumulation);
+ *   h = silu(g) * u rounded to bf16 and quantised by 32-value blocks inside the
+ *        same kernel: h_q [n_rows, I] codes, h_sf [n_rows, I/32] (no bf16 h);
+ *   y [n_rows, H] bf16 = the dequantised W2[e] . h, or in decode form the fp32
+ *        reduce into out_reduce as in moe_grouped_swiglu_ffn.
+ * Scale arrays 4-byte aligned.  recv_token, recv_slot, topk_w: decode form only.
+ * ws: moe_workspace_bytes(cfg).
+ */
+moe_status moe_grouped_swiglu_ffn_mxfp8(const moe_config *cfg, int64_t n_rows, const uint8_t *xr_q,
+                                        const uint8_t *xr_sf, const int32_t *expert_offsets,
+                                        const uint8_t *w13_q, const uint8_t *w13_sf, const uint8_t *w2_q,
+                                        const uint8_t *w2_sf, uint8_t *h_q, uint8_t *h_sf, void *y,
+                                        const int32_t *recv_token, const int32_t *recv_slot,
+                                        const float *topk_w, float *out_reduce, void *ws,
+                                        cudaStream_t stream);
+
+/*
  * Step 6 - combine back to token order ([AX] combine all-to-all then the
  * weighted sum): for t in [tok_begin, tok_begin + tok_count)
  *   out[t, :] = sum over j = 0..k-1 with pos[t - tok_begin, j] >= 0 of
@@ -471,7 +533,9 @@ moe_status moe_permute_backward(const moe_config *cfg, const void *dxr, const in
  *            these their row scales (moe_grouped_swiglu_ffn_fp8); x stays
  *            bf16 and each chunk's kept rows are quantised inside the permute
  *            (moe_permute_quantize_fp8; for H > 8192 by moe_quantize_fp8_rows
- *            then moe_permute).  Else ignored, may be NULL.
+ *            then moe_permute).  With cfg->ffn_fp8 = 2, the block scales of
+ *            moe_quantize_fp8_blocks (moe_permute_quantize_fp8_blocks,
+ *            moe_grouped_swiglu_ffn_mxfp8).  Else ignored, may be NULL.
  *   topk_idx [T,k], topk_w [T,k], keep [T,k]: caller-owned saved state
  *            ([AX] the routing top-k is always saved).
  *   splits_host: pinned host int32 [n_chunks * (E+1 + ep*ep)] or NULL; chunk c
