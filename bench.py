@@ -141,12 +141,13 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_src_hash(fp8: bool = False):
+def kernel_src_hash(fp8: bool = False, mx: bool = False):
     """Hash of the FFN's sources: the grouped GEMM kernel, and for the FP8 FFN also
-    the row quantisation between its launches.  Recorded traffic holds only for
-    these bytes."""
+    the row quantisation between its launches (the block-scaled FP8 FFN: its own
+    kernel).  Recorded traffic holds only for these bytes."""
     h = hashlib.sha256()
-    for name in ("ffn_tcgen05.cu", "fp8_quant.cu") if fp8 else ("ffn_tcgen05.cu",):
+    names = ("ffn_mx_tcgen05.cu",) if mx else ("ffn_tcgen05.cu", "fp8_quant.cu") if fp8 else ("ffn_tcgen05.cu",)
+    for name in names:
         with open(os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -232,14 +233,21 @@ def kernels_per_step(wl) -> int:
     # with a shared expert, per chunk 3 more (its offsets and two GEMM launches);
     # with the FP8 FFN, per chunk 1 more (h's row quantisation), 2 when x's
     # quantisation is not fused into the permute (H > 8192)
+    # with the block-scaled FP8 FFN (ffn_fp8 = 2) nothing more: x is quantised inside
+    # the permute and h inside GEMM1
     clip = 4 if wl.capacity > 0 else 2
-    fp8 = (1 if fused_permute_quant(wl) else 2) if wl.ffn_fp8 else 0
+    fp8 = 0 if is_mx(wl) else (1 if fused_permute_quant(wl) else 2) if wl.ffn_fp8 else 0
     return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + fp8)
 
 
 def fused_permute_quant(wl) -> bool:
     """The FP8 path quantises x inside the permute for rows of up to 8192 values."""
-    return wl.ffn_fp8 and wl.H <= 8192
+    return bool(wl.ffn_fp8) and wl.H <= 8192
+
+
+def is_mx(wl) -> bool:
+    """The FP8 FFN with one UE8M0 scale per 32 K values (ffn_fp8 = 2)."""
+    return wl.ffn_fp8 == 2
 
 
 def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
@@ -256,14 +264,22 @@ def algorithmic(wl, n_kept_chunks, active_chunks, tokens_read=None):
     per weight row); h is written in bf16, read by its quantisation, whose
     codes are written and read by GEMM2; the permute stage reads the kept
     tokens' bf16 rows and writes their codes (H <= 8192: one fused pass), or
-    quantises all of x, writes its codes and permutes them (longer rows)."""
+    quantises all of x, writes its codes and permutes them (longer rows).
+    Block-scaled FP8 (ffn_fp8 = 2): one scale byte per 32 values beside every
+    code row (weights, receive rows, h); h is quantised inside GEMM1, so only
+    its codes and scales are written and read."""
     b = wl.elem_bytes
     N = sum(n_kept_chunks)
     tok_bytes = wl.T * wl.H * b
     read_bytes = (wl.T if tokens_read is None else tokens_read) * wl.H
     y_bytes = N * wl.H * b
     out_bytes = 2 * wl.T * wl.H * 4 if wl.reduce_dense else y_bytes
-    if wl.ffn_fp8:
+    if is_mx(wl):
+        row_bytes = N * wl.H * 33 // 32
+        w_bytes = sum(active_chunks) * 3 * wl.H * wl.I * 33 // 32
+        permute_bytes = read_bytes * b + row_bytes
+        h_bytes = 2 * N * wl.I * 33 // 32
+    elif wl.ffn_fp8:
         row_bytes = N * wl.H
         w_bytes = sum(active_chunks) * (3 * wl.H * wl.I + 2 * wl.I + wl.H)
         if fused_permute_quant(wl):
@@ -308,7 +324,11 @@ class StepBuffers:
         self.pos = torch.empty(tc, k, dtype=torch.int32, device=dev)
         self.spl = torch.empty(ep, ep, dtype=torch.int32, device=dev)
         self.xr = torch.empty(n, H, dtype=torch.uint8 if wl.ffn_fp8 else wl.torch_dtype, device=dev)
-        if wl.ffn_fp8:
+        if is_mx(wl):
+            self.xsf = torch.empty(n, H // 32, dtype=torch.uint8, device=dev)
+            self.hq = torch.empty(n, I, dtype=torch.uint8, device=dev)
+            self.hsf = torch.empty(n, I // 32, dtype=torch.uint8, device=dev)
+        elif wl.ffn_fp8:
             self.xq = torch.empty(T, H, dtype=torch.uint8, device=dev)
             self.xsc = torch.empty(T, dtype=torch.uint8, device=dev)
             self.hq = torch.empty(n, I, dtype=torch.uint8, device=dev)
@@ -346,7 +366,9 @@ def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
         moe.moe_dispatch_layout(cfg, tb, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs,
                                 B.pos, B.spl, None, B.ws)
         rec(base)
-        if fused_permute_quant(wl):
+        if is_mx(wl):
+            moe.moe_permute_quantize_fp8_blocks(cfg, inp.x, B.pos, tb, B.tc, B.xr, B.xsf)
+        elif fused_permute_quant(wl):
             moe.moe_permute_quantize_fp8(cfg, inp.x, B.pos, tb, B.tc, B.xr, B.xsc)
         elif wl.ffn_fp8:
             moe.moe_quantize_fp8_rows(inp.x[tb:tb + B.tc], B.xq[tb:tb + B.tc], B.xsc[tb:tb + B.tc])
@@ -354,7 +376,11 @@ def run_steps(moe, wl, cfg, inp, B, ev=None, fp8=None):
         else:
             moe.moe_permute(cfg, inp.x, B.pos, tb, B.tc, B.xr)
         rec(base + 1)
-        if wl.ffn_fp8:
+        if is_mx(wl):
+            w13q, w13s, w2q, w2s = fp8
+            moe.moe_grouped_swiglu_ffn_mxfp8(cfg, B.nmax, B.xr, B.xsf, B.eoff, w13q, w13s, w2q, w2s, B.hq,
+                                             B.hsf, B.y, B.rt, B.rs, B.topk_w, B.red, B.ws)
+        elif wl.ffn_fp8:
             w13q, w13s, w2q, w2s = fp8
             moe.moe_grouped_swiglu_ffn_fp8(cfg, B.nmax, B.xr, B.xsc, B.eoff, w13q, w13s, w2q, w2s,
                                            B.h, B.hq, B.hsc, B.y, B.rt, B.rs, B.topk_w, B.red, B.ws)
@@ -666,8 +692,11 @@ def ffn_roofline(wl, alg, ffn_ms, peaks, peak_src, traffic):
     hbm_bound = t_byte > t_flop
     tflops = alg["ffn_flops"] / ffn_s / 1e12 if ffn_s > 0 else None
     gbs = alg["ffn_bytes"] / ffn_s / 1e9 if ffn_s > 0 else None
-    return {"kernel": "grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass"
-                      + (", E4M3 operands, h quantised between them)" if wl.ffn_fp8 else ")"),
+    kname = ("grouped SwiGLU FFN (ffn_mx_tcgen05_kernel, GEMM1 with h quantised in its epilogue + GEMM2, "
+             "E4M3 operands with one UE8M0 scale per 32 K values)") if is_mx(wl) else \
+        ("grouped SwiGLU FFN (ffn_gemm_tcgen05_kernel, GEMM1 + GEMM2 per layer pass"
+         + (", E4M3 operands, h quantised between them)" if wl.ffn_fp8 else ")"))
+    return {"kernel": kname,
             "bound": "hbm" if hbm_bound else "tensor",
             "achieved": gbs if hbm_bound else tflops,
             "peak": peaks["hbm_gbs"] if hbm_bound else t_peak,
@@ -712,7 +741,10 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     keep, _ = oracle.capacity_clip(idx, w, wl.E, wl.capacity)
     tc = wl.T // wl.n_chunks
     lays = [oracle.dispatch_layout(idx, keep, wl.E, wl.ep, c * tc, tc) for c in range(wl.n_chunks)]
-    if wl.ffn_fp8:
+    if is_mx(wl):
+        xq, xs = oracle.quantize_blocks(x_np, 32)
+        xrs = [oracle.permute(xq, lay["recv_token"]) for lay in lays]
+    elif wl.ffn_fp8:
         xq, xs = oracle.quantize_rows(x_np)
         xrs = [oracle.permute(xq, lay["recv_token"]) for lay in lays]
     else:
@@ -728,7 +760,9 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     ye = np.zeros((max(N, 1), wl.H), np.float64)
     t1 = time.perf_counter()
     for p, e in rows:
-        if wl.ffn_fp8:
+        if is_mx(wl):
+            _, _, _, y[p], ye[p] = oracle.ffn_row_fp8_blocked(xrs[0][p], xs[lay["recv_token"][p]], *weights[e], 32)
+        elif wl.ffn_fp8:
             _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xrs[0][p], xs[lay["recv_token"][p]], *weights[e])
         else:
             _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
@@ -748,18 +782,27 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     return wl.T / layer_s, t_index + t_ffn, desc
 
 
-def fp8_expert(w13_e, w2_e):
-    """The oracle's codes and row scales of one expert's bf16 weights (host
-    uint16 bits): (w13 codes, w13 scales, w2 codes, w2 scales)."""
+def fp8_expert(w13_e, w2_e, blocks=False):
+    """The oracle's codes and scales of one expert's bf16 weights (host uint16
+    bits): (w13 codes, w13 scales, w2 codes, w2 scales); one scale per row, or
+    with blocks one per row and 32 values."""
     import oracle
-    a, sa = oracle.quantize_rows(w13_e)
-    b, sb = oracle.quantize_rows(w2_e)
+    q = (lambda a: oracle.quantize_blocks(a, 32)) if blocks else oracle.quantize_rows
+    a, sa = q(w13_e)
+    b, sb = q(w2_e)
     return a, sa, b, sb
+
+
+def oracle_row_seconds(wl):
+    """Measured oracle cost of one FFN row, scaled from H = 2048, I = 768: bf16
+    7.7 ms, FP8 with row scales 3 ms, FP8 with block scales 4.6 ms."""
+    base = 4.6e-3 if is_mx(wl) else 3.0e-3 if wl.ffn_fp8 else 7.7e-3
+    return base * (wl.H * wl.I) / (2048 * 768)
 
 
 def sample_tokens_for(wl, seconds):
     # measured oracle cost of one FFN row at H = 2048, I = 768 (bf16 / FP8)
-    row_s = (3.0e-3 if wl.ffn_fp8 else 7.7e-3) * (wl.H * wl.I) / (2048 * 768)
+    row_s = oracle_row_seconds(wl)
     s = int(seconds / (wl.k * row_s))
     return max(1, min(wl.T // wl.n_chunks, s))
 
@@ -769,7 +812,7 @@ def sample_tokens_for(wl, seconds):
 def reference_tokens(wl, seconds):
     """Tokens of one reference step: about `seconds` of oracle FFN rows, a
     multiple of the logical EP size (each source rank gets an equal block)."""
-    row_s = (3.0e-3 if wl.ffn_fp8 else 7.7e-3) * (wl.H * wl.I) / (2048 * 768)
+    row_s = oracle_row_seconds(wl)
     n = int(seconds / (wl.k * row_s)) // wl.ep * wl.ep
     return max(wl.ep, min(wl.T, n))
 
@@ -786,7 +829,10 @@ def reference_step(wl, Ts, logits, bias, x_np, fetch):
                                       wl.topk_group, wl.group_score, wl.bias_select_only)
     keep, _ = oracle.capacity_clip(idx, w, wl.E, cap)
     lay = oracle.dispatch_layout(idx, keep, wl.E, wl.ep, 0, Ts)
-    if wl.ffn_fp8:
+    if is_mx(wl):
+        xq, xs = oracle.quantize_blocks(x_np[:Ts], 32)
+        xr = oracle.permute(xq, lay["recv_token"])
+    elif wl.ffn_fp8:
         xq, xs = oracle.quantize_rows(x_np[:Ts])
         xr = oracle.permute(xq, lay["recv_token"])
     else:
@@ -800,7 +846,9 @@ def reference_step(wl, Ts, logits, bias, x_np, fetch):
     t1 = time.perf_counter()
     for e, wt in weights.items():
         for p in range(int(eoff[e]), int(eoff[e + 1])):
-            if wl.ffn_fp8:
+            if is_mx(wl):
+                _, _, _, y[p], ye[p] = oracle.ffn_row_fp8_blocked(xr[p], xs[lay["recv_token"][p]], *wt, 32)
+            elif wl.ffn_fp8:
                 _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xr[p], xs[lay["recv_token"][p]], *wt)
             else:
                 _, y[p], ye[p] = oracle.ffn_row(xr[p], wt[0], wt[1])
@@ -834,7 +882,7 @@ def run_reference(args):
         if e not in cache:
             a = (torch.randn(2 * wl.I, wl.H, generator=g) * std).to(wl.torch_dtype)
             b = (torch.randn(wl.H, wl.I, generator=g) * std).to(wl.torch_dtype)
-            cache[e] = fp8_expert(conv(a), conv(b)) if wl.ffn_fp8 else (conv(a), conv(b))
+            cache[e] = fp8_expert(conv(a), conv(b), is_mx(wl)) if wl.ffn_fp8 else (conv(a), conv(b))
         return cache[e]
 
     logits = inp.logits.numpy()
@@ -909,8 +957,9 @@ def run_ours(args):
     fp8 = None
     w13_l, w2_l, w13_sc, w2_sc = inp.w13, inp.w2, None, None
     if wl.ffn_fp8:
-        w13_l, w13_sc = moe.quantize_fp8(inp.w13)
-        w2_l, w2_sc = moe.quantize_fp8(inp.w2)
+        q = moe.quantize_fp8_blocks if is_mx(wl) else moe.quantize_fp8
+        w13_l, w13_sc = q(inp.w13)
+        w2_l, w2_sc = q(inp.w2)
         fp8 = (w13_l, w13_sc, w2_l, w2_sc)
         torch.cuda.synchronize()
 
@@ -1071,7 +1120,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         conv = (lambda t: t.detach().cpu().view(torch.int16).numpy().view(np.uint16).copy()) \
             if wl.dtype == "bf16" else (lambda t: t.detach().cpu().numpy().copy())
-        fetch = (lambda e: fp8_expert(conv(inp.w13[e]), conv(inp.w2[e]))) if wl.ffn_fp8 else \
+        fetch = (lambda e: fp8_expert(conv(inp.w13[e]), conv(inp.w2[e]), is_mx(wl))) if wl.ffn_fp8 else \
             (lambda e: (conv(inp.w13[e]), conv(inp.w2[e])))
         s_tok = sample_tokens_for(wl, 15.0)
         shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
@@ -1084,7 +1133,7 @@ def run_ours(args):
     if rank == 0:
         ms_per_step = total_ms / args.steps
         value = world * wl.T * args.steps / (total_ms / 1e3)
-        src = kernel_src_hash(wl.ffn_fp8)
+        src = kernel_src_hash(wl.ffn_fp8, is_mx(wl))
         tr = FFN_TRAFFIC.get(wl.name)
         traffic = tr["bytes"] if tr and tr.get("src") == src and tr.get("chunks", 1) == wl.n_chunks else None
         roof = ffn_roofline(wl, alg, stage_ms["grouped_ffn"], peaks, peak_src, traffic)

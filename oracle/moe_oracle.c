@@ -759,19 +759,27 @@ void orc_quantize_blocks(int64_t rows, int cols, int block, int dtype, const voi
 /* Dot product of two K-blocked FP8 rows of length K (same block size): the sum
  * over blocks of 2^(sa + sb - 254) times the sum of the blocks' decoded code
  * products, in double (each block's partial sum is exact in double for
- * E4M3 operands and block <= 2^20). */
-double orc_dot_blocked(int K, int block, const uint8_t *a, const uint8_t *sa, const uint8_t *b,
-                       const uint8_t *sb)
+ * E4M3 operands and block <= 2^20).  dec: the decoded value of every code. */
+static double orc_dot_blocked_dec(int K, int block, const uint8_t *a, const uint8_t *sa,
+                                  const uint8_t *b, const uint8_t *sb, const double *dec)
 {
     const int nb = (K + block - 1) / block;
     double acc = 0.0;
     for (int q = 0; q < nb; ++q) {
         double part = 0.0;
         for (int c = q * block; c < K && c < (q + 1) * block; ++c)
-            part += orc_e4m3_decode(a[c]) * orc_e4m3_decode(b[c]);
+            part += dec[a[c]] * dec[b[c]];
         acc += ldexp(part, (int)sa[q] + (int)sb[q] - 254);
     }
     return acc;
+}
+
+double orc_dot_blocked(int K, int block, const uint8_t *a, const uint8_t *sa, const uint8_t *b,
+                       const uint8_t *sb)
+{
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = orc_e4m3_decode((uint8_t)c);
+    return orc_dot_blocked_dec(K, block, a, sa, b, sb, dec);
 }
 
 /* One expert's SwiGLU FFN on one receive row in FP8 with K-blocked scales (the
@@ -792,18 +800,20 @@ void orc_ffn_row_fp8_blocked(int H, int I, int block, const uint8_t *x, const ui
                              uint8_t *hs_store, uint16_t *y_store, double *y_exact)
 {
     const int nbh = (H + block - 1) / block, nbi = (I + block - 1) / block;
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = orc_e4m3_decode((uint8_t)c);
     uint16_t *h = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
     uint8_t *hq = (uint8_t *)malloc((size_t)I);
     uint8_t *hs = (uint8_t *)malloc((size_t)nbi);
     for (int i = 0; i < I; ++i) {
-        const double g = orc_dot_blocked(H, block, w13 + (size_t)i * H, w13_s + (size_t)i * nbh, x, xs);
-        const double u = orc_dot_blocked(H, block, w13 + (size_t)(I + i) * H, w13_s + (size_t)(I + i) * nbh,
-                                         x, xs);
+        const double g = orc_dot_blocked_dec(H, block, w13 + (size_t)i * H, w13_s + (size_t)i * nbh, x, xs, dec);
+        const double u = orc_dot_blocked_dec(H, block, w13 + (size_t)(I + i) * H,
+                                             w13_s + (size_t)(I + i) * nbh, x, xs, dec);
         h[i] = orc_bf16_from_double(g / (1.0 + exp(-g)) * u);
     }
     orc_quantize_blocks(1, I, block, 1, h, hq, hs);
     for (int o = 0; o < H; ++o) {
-        const double acc = orc_dot_blocked(I, block, w2 + (size_t)o * I, w2_s + (size_t)o * nbi, hq, hs);
+        const double acc = orc_dot_blocked_dec(I, block, w2 + (size_t)o * I, w2_s + (size_t)o * nbi, hq, hs, dec);
         if (y_exact) y_exact[o] = acc;
         if (y_store) y_store[o] = orc_bf16_from_double(acc);
     }

@@ -74,3 +74,15 @@ def test_ffn_roofline_picks_the_binding_roof():
     r1 = bench.ffn_roofline(wl.with_(n_chunks=1), a1, 6.0, low, "measured", None)
     assert r1["bound"] == "tensor" and abs(r1["frac"] - r1["tensor_frac"]) < 1e-12
     assert r1["tensor_frac_sustained"] > r1["tensor_frac"]
+
+
+def test_block_scaled_fp8_counts():
+    mx = WORKLOADS["dsv3_prefill_mxfp8"]
+    bf = WORKLOADS["dsv3_prefill"]
+    # x quantised inside the permute, h inside GEMM1: the bf16 layer's launches
+    assert bench.kernels_per_step(mx) == bench.kernels_per_step(bf)
+    a = bench.algorithmic(mx, [32768, 32768], [256, 256], tokens_read=8192)
+    H, I, N = 7168, 2048, 65536
+    # one byte per weight plus a scale byte per 32; h's codes and scales written and read
+    assert a["ffn_bytes"] == 2 * 256 * 3 * H * I * 33 // 32 + N * H * 33 // 32 + 2 * N * I * 33 // 32 + N * H * 2
+    assert a["permute_bytes"] == 8192 * H * 2 + N * H * 33 // 32
