@@ -5,51 +5,81 @@
 // row of W13 and W2; four consecutive block scales of a row read as an int32
 // (block 4i in the low byte) are one 128-value k-chunk's scales.
 //
-// Two launches of one persistent, warp-specialised single-CTA kernel with the
-// block-scaled tensor-core MMA (tcgen05.mma kind::mxf8f6f4.block_scale, M = 128
-// weight rows, N <= 128 tokens, K = 32 per instruction, fp32 in TMEM):
+// Two launches of one persistent, warp-specialised kernel on CTA pairs
+// (clusters of 2) with the block-scaled tensor-core MMA across the pair
+// (tcgen05.mma cta_group::2 kind::mxf8f6f4.block_scale, M = 256 weight rows,
+// N <= 224 tokens, K = 32 per instruction, fp32 in TMEM):
 //   GEMM1  gate|up = W13[e] . xr^T; epilogue h = silu(gate) * up rounded to
 //          bf16, then quantised by 32-feature blocks: E4M3 codes h_q [n, I]
 //          and scales h_sf [n, I/32] (no bf16 h is stored);
 //   GEMM2  y = W2[e] . h_q^T (bf16), or in decode form out_reduce += w * y.
 //
-// A tile is (expert, 128 weight rows, 128 tokens): in GEMM1 the gate rows of
-// 64 features followed by their 64 up rows (TMEM lanes i and 64 + i), in GEMM2
-// 128 output features.  Warp 8 streams each ring stage (two 128-value
-// k-chunks: 32 KiB of weight rows and 32 KiB of token rows, one TMA box each)
-// and, with all its lanes, gathers the stage's scale words - 128 weight rows
-// and 128 token rows, two words each - into four 512-byte scale atoms in shared
-// memory (row r's word at byte 16 (r % 32) + 4 (r / 32), the layout tcgen05.cp
-// spreads over the four TMEM lane quadrants).  Warp 9 (one lane) copies the
-// atoms to TMEM with tcgen05.cp and issues the stage's eight MMAs, each reading
-// its block's scale byte.  Warps 0-7 drain TMEM (warps q and q + 4 share lane
-// quadrant q and take alternate 32-token chunks): GEMM1's gate and up warps
-// swap half their tokens through shared memory as in the bf16 kernel; each
-// warp then holds 32 features (one 32-value block of h) of 16 tokens and
-// quantises them with a warp max per token.
+// Why pairs: with one CTA per 128 x 128 tile every SM streams 256 operand bytes
+// per 128-value k-step for 128 x 128 products, and FP8's doubled MMA rate made
+// that stream (through L2, where each token block is re-read for every weight
+// block and each weight block for every token block) the bound.  A pair tile
+// (256 weight rows, up to 224 tokens) keeps 128 weight rows and half the
+// tokens in each CTA, so each SM streams half the bytes per product.
+//
+// A pair tile is (expert, 256 weight rows, <= 224 tokens); 224, not 256,
+// because TMEM holds two accumulators (epilogue of tile i beside the main loop
+// of tile i+1) and the scales: accumulators at columns 0 and 256, the scales
+// of alternate ring stages at columns 224 and 480 (weight-row scales of the
+// stage's two k-chunks in 8 columns, then token scales in 16).  In GEMM1 a
+// CTA's 128 weight rows are the gate rows of 64 features and their 64 up rows
+// (TMEM lanes i and 64 + i); in GEMM2 128 output features.
+//
+// Roles (10 warps per CTA).  Warp 8 of each CTA streams its ring stages (two
+// k-chunks: 32 KiB of weight rows and 28 KiB of token rows by TMA, counted on
+// the leader's barrier) and, with all its lanes, gathers the stage's scale
+// words with 4-byte cp.async into 512-byte scale atoms (row r's word at byte
+// 16 (r % 32) + 4 (r / 32), the layout tcgen05.cp spreads over the four TMEM
+// lane quadrants): its own 128 weight rows, and all the tile's tokens, which
+// both CTAs hold in TMEM.  The leader's lanes signal their copies on the
+// leader's full barrier; the follower's on a local barrier that the follower's
+// warp 9 (otherwise idle) forwards to the leader's.  The leader's warp 9 (one
+// lane) copies both CTAs' atoms to TMEM (tcgen05.cp cta_group::2), issues the
+// stage's eight block-scaled MMAs and commits to both CTAs' barriers.  Warps
+// 0-7 of each CTA drain TMEM (warps q and q + 4 share lane quadrant q and take
+// alternate 32-token chunks); in GEMM1 the gate and up warps swap half their
+// tokens through shared memory, and each warp then quantises its 32 features
+// (one 32-value block of h) for 16 tokens with a warp max per token.  Tiles are
+// dealt from a global counter and published through the pair's slice queue.
 //
 // Every wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT, stops the
-// other roles, lets in-flight copies and MMAs land, frees TMEM and returns.
-#include <cfloat>
+// other roles, lets in-flight copies and MMAs land, frees TMEM and returns.  No
+// TMA load uses cluster multicast.
 #include <cudaTypedefs.h>
 #include <cuda_fp8.h>
 
-#include "moe_common.cuh"
+#include "ffn_pair.cuh"
 
 namespace moe {
 
-constexpr int kMxTile = 128;                                 // weight rows and tokens per tile
+constexpr int kMxRows = 128;                                  // weight rows per CTA (MMA M / 2)
+constexpr int kMxTileTok = 224;                               // tokens per tile (MMA N <= 224)
+constexpr int kMxBoxTok = kMxTileTok / 2;                     // token rows per CTA box
+constexpr int kMxSmallBox = 32;                               // token box of tiles with N <= 64
+constexpr int kMxKS = 2;                                      // 128-value k-chunks per ring stage
+constexpr uint32_t kMxWChunk = kMxRows * 128;                 // 16 KiB of weight rows per k-chunk
+constexpr uint32_t kMxTChunk = kMxBoxTok * 128;               // 14 KiB of token rows per k-chunk
+constexpr uint32_t kMxAtom = 512;                             // 128 rows x 4 block scales
+// stage: [W c0 | W c1 | T c0 | T c1 | SFA c0 | SFA c1 | SFB c0 a0 | c0 a1 | c1 a0 | c1 a1]
+constexpr uint32_t kMxTOff = kMxKS * kMxWChunk;
+constexpr uint32_t kMxSfOff = kMxTOff + kMxKS * kMxTChunk;
+constexpr uint32_t kMxStageBytes = kMxSfOff + 6 * kMxAtom;    // 63 KiB
 constexpr int kMxStages = 3;
-constexpr uint32_t kMxChunkBytes = 128 * 128;                 // 128 rows x one 128-value k-chunk
-constexpr uint32_t kMxOpBytes = 2 * kMxChunkBytes;            // one operand of a stage (32 KiB)
-constexpr uint32_t kMxAtomBytes = 512;                       // 128 rows x 4 block scales
-constexpr uint32_t kMxStageBytes = 2 * kMxOpBytes + 4 * kMxAtomBytes;   // 66 KiB
+constexpr uint32_t kMxRingBytes = kMxStages * kMxStageBytes;
+static_assert(kMxStageBytes % 1024 == 0 && kMxTOff % 1024 == 0 && kMxTChunk % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
 constexpr int kMxEpiWarps = 8;
 constexpr int kMxProdWarp = kMxEpiWarps, kMxMmaWarp = kMxEpiWarps + 1;
 constexpr int kMxThreads = 32 * (kMxEpiWarps + 2);
-constexpr uint32_t kMxTmemCols = 512;                        // accumulators 0-255, scales from 256
-constexpr uint32_t kMxSfaCol = 256, kMxSfbCol = 264;         // 8 columns each (two atoms)
-constexpr uint32_t kMxXchgBytes = 16 * 1024;                 // GEMM1 gate / up exchange
+constexpr uint32_t kMxTmemCols = 512;
+constexpr uint32_t kMxAccStride = 256;                        // accumulator a at column 256 a
+constexpr uint32_t kMxSfCol = kMxTileTok;                    // scale slot a at kMxSfCol + 256 a (24 columns)
+static_assert(kMxAccStride + kMxTileTok + 24 <= kMxTmemCols, "scale columns exceed TMEM");
+constexpr uint32_t kMxXchgBytes = 16 * 1024;                  // GEMM1 gate / up exchange
 constexpr int kMxMaxExperts = 512;
 
 enum MxMode : int { kMxSwiGLUQuant = 0, kMxStore = 1, kMxReduce = 2 };
@@ -58,16 +88,15 @@ struct MxParams {
     const int32_t *expert_offsets;
     int E;
     int K;                  // H (GEMM1) or I (GEMM2)
-    int n_fblocks;          // weight-row tiles per expert: I/64 (GEMM1) or H/128 (GEMM2)
+    int n_fblocks;          // pair feature blocks per expert: I/128 (GEMM1) or ceil(H/256) (GEMM2)
+    int feat_per_cta;       // output features per CTA of a pair tile: 64 (GEMM1) or 128 (GEMM2)
     int w_rows_per_expert;  // 2I or H
-    int half_rows;          // GEMM1: I (the up rows start there)
     int out_cols;           // I (h) or H (y)
     const uint32_t *w_sf;   // [E * w_rows_per_expert, K/128] scale words
     const uint32_t *t_sf;   // [n_rows, K/128] scale words of the token rows
-    int64_t n_rows;
     uint8_t *h_q;           // GEMM1: [n_rows, I] codes
     uint8_t *h_sf;          // GEMM1: [n_rows, I/32] scale bytes
-    void *y;                // GEMM2: [n_rows, H] bf16
+    __nv_bfloat16 *y;       // GEMM2: [n_rows, H]
     float *out_reduce;      // GEMM2 decode form: [T, H]
     const int32_t *recv_token;
     const int32_t *recv_slot;
@@ -77,80 +106,83 @@ struct MxParams {
 };
 
 struct MxSmem {
-    uint64_t full[kMxStages];
+    uint64_t full[kMxStages];      // leader: TMA bytes of both CTAs, its 32 gather lanes, the follower's forward
     uint64_t empty[kMxStages];
+    uint64_t sf_full[kMxStages];   // follower: its 32 gather lanes
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
+    uint64_t q_full[kQueue];
+    uint64_t q_empty[kQueue];
+    int q_slice[kQueue];
     uint32_t tmem_base;
+    int pair_slice[4];
+    int go_flag[4];
     int abort_flag;
-    int total;
-    int pair_go[4];        // GEMM1: did the gate warp of each warp pair get its accumulator
+    int total_slices;
 };
 
 struct MxTile {
-    int e, fb, p0, n_valid, n_mma;
+    int e, f_blk, p0, n_valid, n_mma;   // n_valid <= 224 tokens; n_mma: the MMA's N (rounded to 16)
 };
 
-__device__ __forceinline__ MxTile mx_tile(int t, const int32_t *s_tpre, const int32_t *s_tb,
-                                          const MxParams &P) {
-    int lo = 0, hi = P.E - 1;   // last e with s_tpre[e] <= t
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_tpre[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    MxTile w;
-    w.e = lo;
-    const int local = t - s_tpre[lo];
-    w.fb = local / s_tb[lo];
-    const int tb = local - w.fb * s_tb[lo];
-    const int off = P.expert_offsets[lo];
-    w.p0 = off + tb * kMxTile;
-    w.n_valid = min(kMxTile, P.expert_offsets[lo + 1] - w.p0);
-    w.n_mma = (w.n_valid + 15) & ~15;
-    return w;
+__device__ __forceinline__ MxTile mx_tile_info(int e, int f_blk, int t_blk, const MxParams &P) {
+    MxTile t;
+    t.e = e;
+    t.f_blk = f_blk;
+    const int off = P.expert_offsets[e];
+    t.p0 = off + t_blk * kMxTileTok;
+    t.n_valid = min(kMxTileTok, P.expert_offsets[e + 1] - t.p0);
+    t.n_mma = (t.n_valid + 15) & ~15;
+    return t;
 }
 
-__device__ __forceinline__ int mx_exponent(float amax) {
-    // the smallest e with amax <= 448 * 2^e (amax = m 2^x, m in [0.5, 1), 448 = 0.875 2^9)
-    if (!(amax > 0.0f)) return 0;
-    if (amax > FLT_MAX) return 127;
-    int x;
-    const float m = frexpf(amax, &x);
-    const int e = m <= 0.875f ? x - 9 : x - 8;
+// The block exponent of a 32-value block whose largest magnitude has the float
+// bits b (b >= 0 as a float): the smallest e in [-126, 127] with
+// amax <= 448 * 2^e; 0 for a zero (or NaN) block, 127 for an infinite one.
+// With amax = 1.m * 2^(x - 127) (x the biased exponent) and 448 = 1.75 * 2^8:
+// e = x - 135 when 1.m <= 1.75 (m <= 0x600000), else x - 134.
+__device__ __forceinline__ int mx_exponent_bits(uint32_t b) {
+    if (b == 0u || b > 0x7F800000u) return 0;
+    if (b == 0x7F800000u) return 127;
+    const int x = (int)(b >> 23);
+    const int e = x == 0 ? -126 : x - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
     return min(127, max(-126, e));
 }
 
+// 2^-e as a float for e in [-126, 127] (e = 127: the subnormal 2^-127).
 __device__ __forceinline__ float mx_pow2_neg(int e) {
     return e == 127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(127 - e) << 23);
 }
 
-__device__ __forceinline__ void mx_named_barrier(uint32_t id, uint32_t nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 template <int MODE>
-__global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_t,
-    const MxParams P) {
+    const __grid_constant__ CUtensorMap tmap_ts, const MxParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kG1 = MODE == kMxSwiGLUQuant;
+    // queue consumers per entry: the leader's MMA thread, the follower's producer
+    // and forwarder, and every epilogue warp of both CTAs (GEMM1: the gate warps)
+    constexpr uint32_t kQueueConsumers = 3 + 2 * (kG1 ? kMxEpiWarps / 2 : kMxEpiWarps);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled tiles (same offsets in both CTAs of the pair)
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *ring = base;                                       // [stages][A | B | SFA | SFB]
-    float *xchg = reinterpret_cast<float *>(base + kMxStages * kMxStageBytes);   // GEMM1
-    MxSmem *S = reinterpret_cast<MxSmem *>(base + kMxStages * kMxStageBytes + (kG1 ? kMxXchgBytes : 0));
-    int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);           // [E + 1] tile prefix
-    int32_t *s_tb = s_tpre + (P.E + 1);                              // [E] token blocks per expert
+    unsigned char *ring = base;                                       // [stages][W | T | scale atoms]
+    float *xchg = reinterpret_cast<float *>(base + kMxRingBytes);     // GEMM1 only
+    MxSmem *S = reinterpret_cast<MxSmem *>(base + kMxRingBytes + (kG1 ? kMxXchgBytes : 0));
+    int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);            // [E + 1] tile prefix
+    int32_t *s_tb = s_tpre + (P.E + 1);                               // [E] token blocks per expert
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();                          // 0: leader (issues the MMA)
+
     if (warp == 0) {
         int run = 0;
         for (int e0 = 0; e0 < P.E; e0 += 32) {
             const int e = e0 + lane;
             int tb = 0;
             if (e < P.E) {
-                tb = (P.expert_offsets[e + 1] - P.expert_offsets[e] + kMxTile - 1) / kMxTile;
+                tb = (P.expert_offsets[e + 1] - P.expert_offsets[e] + kMxTileTok - 1) / kMxTileTok;
                 s_tb[e] = tb;
             }
             const int t = tb * P.n_fblocks;
@@ -163,84 +195,135 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
             if (e < P.E) s_tpre[e] = run + incl - t;
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) { s_tpre[P.E] = run; S->total = run; }
+        if (lane == 0) { s_tpre[P.E] = run; S->total_slices = run; }
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kMxStages; ++s) {
-            mbar_init(&S->full[s], 2);       // the TMA bytes' arrival and the scale atoms' arrival
+            mbar_init(&S->full[s], 1 + 32 + 1);
             mbar_init(&S->empty[s], 1);
+            mbar_init(&S->sf_full[s], 32);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&S->tmem_full[a], 1);
-            mbar_init(&S->tmem_empty[a], kMxEpiWarps);
+            mbar_init(&S->tmem_empty[a], 2 * kMxEpiWarps);   // every epilogue warp of both CTAs
         }
+        for (int i = 0; i < kQueue; ++i) { mbar_init(&S->q_full[i], 1); mbar_init(&S->q_empty[i], kQueueConsumers); }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kMxProdWarp && lane == 0) { tma_prefetch_desc(&tmap_w); tma_prefetch_desc(&tmap_t); }
-    if (warp == kMxMmaWarp) { tmem_alloc_1(&S->tmem_base, kMxTmemCols); tmem_relinquish_1(); }
+    if (warp == kMxProdWarp && lane == 0) {
+        tma_prefetch_desc(&tmap_w);
+        tma_prefetch_desc(&tmap_t);
+        tma_prefetch_desc(&tmap_ts);
+    }
+    if (warp == kMxMmaWarp) { tmem_alloc_pair(&S->tmem_base, kMxTmemCols); tmem_relinquish_pair(); }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();      // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
 
-    const int total = S->total;
+    const int total = S->total_slices;
     const uint32_t tmem_base = S->tmem_base;
+    const int kwords = P.K / 128;                             // scale words per row
+    const int num_k = (P.K + 128 * kMxKS - 1) / (128 * kMxKS);   // ring stages per tile (a last
+                                                              // chunk past K loads zeros, scale words 0)
     volatile int *abort_flag = &S->abort_flag;
-    const int kwords = P.K / 128;          // scale words per row
-    const int num_k = (P.K + 255) / 256;   // ring stages per tile (two k-chunks each; a last
-                                           // stage past K loads zeros and scale words 0)
 
     if (warp == kMxProdWarp) {
-        // ------------------------------------------------ TMA + scale gather (whole warp)
+        // ------------------------------------------------ TMA + scale gather (whole warp, both CTAs)
         int stage = 0;
         uint32_t phase = 0;
         long long issued = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const MxTile w = mx_tile(t, s_tpre, s_tb, P);
-            // this lane's four weight rows and four token rows (r = lane + 32 i)
-            int64_t wrow[4], trow[4];
+        int qi = 0;
+        uint32_t qph = 0;
+        SliceReader reader;
+        // the leader holds one ticket ahead: the counter's round trip for the
+        // next tile overlaps the loads of the current one
+        int ticket = (rank == 0 && lane == 0) ? (int)atomicAdd(work_counter, 1u) : 0;
+        uint64_t *my_full = rank == 0 ? S->full : S->sf_full;
+        while (ok) {
+            int slice = 0;
+            bool got = true;
+            if (lane == 0) {
+                if (rank != 0) {
+                    got = reader.next(S, abort_flag, true, slice);
+                } else if ((got = mbar_wait_bounded(&S->q_empty[qi], qph ^ 1u, abort_flag))) {
+                    slice = ticket < total ? ticket : -1;
+                    S->q_slice[qi] = slice;
+                    st_cluster_u32(mapa_shared(smem_u32(&S->q_slice[qi]), 1), (uint32_t)slice);
+                    mbar_arrive(&S->q_full[qi]);
+                    mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->q_full[qi]), 1));
+                    if (++qi == kQueue) { qi = 0; qph ^= 1u; }
+                    if (slice >= 0) ticket = (int)atomicAdd(work_counter, 1u);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
+            slice = __shfl_sync(0xffffffffu, slice, 0);
+            if (slice < 0) break;
+            int se, sfb, t_blk;
+            decode_tile(slice, s_tpre, s_tb, P.E, se, sfb, t_blk);
+            const MxTile ti = mx_tile_info(se, sfb, t_blk, P);
+            // this CTA's first output feature, weight rows and token rows
+            const int f0 = (sfb * 2 + (int)rank) * P.feat_per_cta;
+            const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
+            const bool small_box = ti.n_mma / 2 <= kMxSmallBox;
+            const uint32_t stage_tx = kMxKS * (kMxWChunk + (small_box ? kMxSmallBox : kMxBoxTok) * 128);
+            // the scale rows this lane gathers: weight rows r = lane + 32 i (-1: past
+            // the expert's features) and the tile's tokens n = lane + 32 i (-1: past n_valid)
+            int64_t wrow[4], trow[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = lane + 32 * i;
-                if (kG1)   // gate rows of 64 features, then their up rows
-                    wrow[i] = (int64_t)w.e * P.w_rows_per_expert + (r < 64 ? 0 : P.half_rows) + w.fb * 64 + (r & 63);
-                else
-                    wrow[i] = (int64_t)w.e * P.w_rows_per_expert + w.fb * 128 + r;
-                trow[i] = r < w.n_valid ? (int64_t)w.p0 + r : -1;
+                const int64_t eb = (int64_t)se * P.w_rows_per_expert;
+                if (kG1) {   // gate rows of 64 features, then their up rows
+                    const int f = f0 + (r & 63);
+                    wrow[i] = f < P.out_cols ? eb + (r < 64 ? 0 : P.out_cols) + f : -1;
+                } else {
+                    const int f = f0 + r;
+                    wrow[i] = f < P.out_cols ? eb + f : -1;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int n = lane + 32 * i;
+                trow[i] = n < ti.n_valid ? (int64_t)ti.p0 + n : -1;
             }
             for (int kb = 0; kb < num_k; ++kb) {
-                bool got = lane == 0 ? mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag) : true;
-                if (!__shfl_sync(0xffffffffu, got ? 1 : 0, 0)) { ok = false; break; }
+                const bool w_ok = lane == 0 ? mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag) : true;
+                if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
                 unsigned char *st = ring + stage * kMxStageBytes;
-                const int ch = 2 * kb;
+                const int ch = kb * kMxKS;   // first k-chunk of the stage
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&S->full[stage], 2 * kMxOpBytes);
+                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * stage_tx);
                     if (kG1)
-                        tma_load_4d(st, &tmap_w, &S->full[stage], 0, w.fb * 64, 2 * w.e, ch);
+                        tma_load_4d_pair(st, &tmap_w, full_leader, 0, f0, 2 * se, ch);
                     else
-                        tma_load_3d(st, &tmap_w, &S->full[stage], 0, w.e * P.w_rows_per_expert + w.fb * 128, ch);
-                    tma_load_3d(st + kMxOpBytes, &tmap_t, &S->full[stage], 0, w.p0, ch);
+                        tma_load_3d_pair(st, &tmap_w, full_leader, 0, se * P.w_rows_per_expert + f0, ch);
+                    tma_load_3d_pair(st + kMxTOff, small_box ? &tmap_ts : &tmap_t, full_leader, 0, tok_row, ch);
                 }
-                // scale atoms: atom a (a = 0, 1) holds word ch + a of each row; row r's
-                // word at byte 16 (r % 32) + 4 (r / 32), so lane's four rows are one uint4
+                // scale atoms (row r's word at byte 16 (r % 32) + 4 (r / 32)): weight rows
+                // of chunk c at atom c, tokens 128 a .. 128 a + 127 of chunk c at atom 2 + 2c + a;
+                // words past K or of rows past the tile are zeros
+                const uint32_t sfs = smem_u32(st + kMxSfOff) + 16 * lane;
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    uint4 wa, ta;
-                    uint32_t *pw = &wa.x, *pt = &ta.x;
+                for (int c = 0; c < kMxKS; ++c) {
+                    const bool in_k = ch + c < kwords;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const bool in_k = ch + a < kwords;
-                        pw[i] = in_k ? __ldg(P.w_sf + wrow[i] * kwords + ch + a) : 0u;
-                        pt[i] = in_k && trow[i] >= 0 ? __ldg(P.t_sf + trow[i] * kwords + ch + a) : 0u;
+                        const bool ok_w = in_k && wrow[i] >= 0;
+                        cp_async_4(sfs + c * kMxAtom + 4 * i, ok_w ? P.w_sf + wrow[i] * kwords + ch + c : P.w_sf,
+                                   ok_w ? 4u : 0u);
                     }
-                    *reinterpret_cast<uint4 *>(st + 2 * kMxOpBytes + a * kMxAtomBytes + 16 * lane) = wa;
-                    *reinterpret_cast<uint4 *>(st + 2 * kMxOpBytes + (2 + a) * kMxAtomBytes + 16 * lane) = ta;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const bool ok_t = in_k && trow[i] >= 0;
+                        cp_async_4(sfs + (2 + 2 * c + (i >> 2)) * kMxAtom + 4 * (i & 3),
+                                   ok_t ? P.t_sf + trow[i] * kwords + ch + c : P.t_sf, ok_t ? 4u : 0u);
+                    }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S->full[stage]);
+                cp_async_mbar_arrive_noinc(&my_full[stage]);
                 ++issued;
                 if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
             }
@@ -249,8 +332,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
             raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
         }
-        if (lane == 0) {
-            // let the last copies land before the CTA can leave
+        cp_async_wait_all();   // this lane's scale copies have landed
+        // the leader's full barriers count both CTAs' bytes: let the last copies land
+        if (rank == 0 && lane == 0) {
             volatile int never = 0;
             const long long last = issued < kMxStages ? issued : kMxStages;
             int st = stage;
@@ -262,88 +346,149 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
         }
         __syncwarp();
     } else if (warp == kMxMmaWarp) {
-        // ------------------------------------------------ scale copies + MMA issuer (one lane)
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const MxTile w = mx_tile(t, s_tpre, s_tb, P);
-                if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d = tmem_base + (uint32_t)(acc * kMxTile);
-                for (int kb = 0; kb < num_k; ++kb) {
-                    if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+            if (rank == 0) {
+                // ------------------------------------------------ scale copies + MMA issuer (leader)
+                int stage = 0;
+                uint32_t phase = 0;
+                int acc = 0;
+                uint32_t acc_phase = 0;
+                uint32_t slot = 0;     // scale columns alternate between two slots, stage by stage
+                bool ok = true;
+                SliceReader reader;
+                int slice;
+                while (ok) {
+                    if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
+                    if (slice < 0) break;
+                    int se, sfb, t_blk;
+                    decode_tile(slice, s_tpre, s_tb, P.E, se, sfb, t_blk);
+                    const MxTile ti = mx_tile_info(se, sfb, t_blk, P);
+                    if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t st = smem_u32(ring + stage * kMxStageBytes);
-                    const uint32_t sf = st + 2 * kMxOpBytes;
+                    const uint32_t d = tmem_base + (uint32_t)acc * kMxAccStride;
+                    // k-chunk stride inside the stage's token box (32 or 112 rows)
+                    const uint32_t tchunk = ti.n_mma / 2 <= kMxSmallBox ? kMxSmallBox * 128 : kMxTChunk;
+                    for (int kb = 0; kb < num_k; ++kb) {
+                        if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        fence_proxy_async_smem();   // the leader's cp.async scale words, before tcgen05.cp
+                        const uint32_t st = smem_u32(ring + stage * kMxStageBytes);
+                        const uint32_t sf = st + kMxSfOff;
+                        const uint32_t tsf = tmem_base + kMxSfCol + kMxAccStride * slot;
+                        // weight-row scales of chunk c at tsf + 4c, token scales at tsf + 8 + 8c
 #pragma unroll
-                    for (int a = 0; a < 2; ++a) {
-                        tc_cp_sf_atom(tmem_base + kMxSfaCol + 4 * a, make_sf_atom_desc(sf + a * kMxAtomBytes));
-                        tc_cp_sf_atom(tmem_base + kMxSfbCol + 4 * a, make_sf_atom_desc(sf + (2 + a) * kMxAtomBytes));
-                    }
+                        for (int a = 0; a < 6; ++a)
+                            tc_cp_sf_atom_pair(tsf + 4 * a, make_sf_atom_desc(sf + a * kMxAtom));
 #pragma unroll
-                    for (int blk = 0; blk < 8; ++blk) {   // 32-value K blocks of the stage
-                        const int c = blk >> 2, kk = blk & 3;
-                        const uint64_t ad = make_sw128_desc(st + c * kMxChunkBytes + kk * 32);
-                        const uint64_t bd = make_sw128_desc(st + kMxOpBytes + c * kMxChunkBytes + kk * 32);
-                        const uint32_t sel = (uint32_t)kk << 30;
-                        tc_mma_mx_1(d, ad, bd, make_idesc_mx_e4m3(kMxTile, w.n_mma, kk),
-                                    (tmem_base + kMxSfaCol + 4 * c) | sel, (tmem_base + kMxSfbCol + 4 * c) | sel,
-                                    (kb > 0 || blk > 0) ? 1u : 0u);
+                        for (int c = 0; c < kMxKS; ++c) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {   // 32-value K blocks of the chunk
+                                const uint64_t wd = make_sw128_desc(st + c * kMxWChunk + kk * 32);
+                                const uint64_t td = make_sw128_desc(st + kMxTOff + c * tchunk + kk * 32);
+                                const uint32_t sel = (uint32_t)kk << 30;
+                                tc_mma_mx_pair(d, wd, td, make_idesc_mx_e4m3(2 * kMxRows, ti.n_mma, kk),
+                                               (tsf + 4 * c) | sel, (tsf + 8 + 8 * c) | sel,
+                                               (kb > 0 || c > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
+                        slot ^= 1u;
+                        if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
                     }
-                    tc_commit_1(&S->empty[stage]);    // frees the stage (and its scale atoms)
-                    if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
+                    if (!ok) break;
+                    tc_commit_pair_mc(&S->tmem_full[acc], 0x3);    // accumulator ready in both CTAs
+                    if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
                 }
-                if (!ok) break;
-                tc_commit_1(&S->tmem_full[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+                if (!ok) {
+                    raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                tc_commit_pair_mc(&S->mma_done, 0x3);
+            } else {
+                // ------------------------------------------------ forwarder (follower)
+                // each stage's scale copies of this CTA, once landed, counted on the
+                // leader's full barrier
+                int stage = 0;
+                uint32_t phase = 0;
+                bool ok = true;
+                SliceReader reader;
+                int slice;
+                while (ok) {
+                    if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
+                    if (slice < 0) break;
+                    for (int kb = 0; kb < num_k; ++kb) {
+                        if (!mbar_wait_bounded(&S->sf_full[stage], phase, abort_flag)) { ok = false; break; }
+                        fence_proxy_async_smem();   // before the leader's tcgen05.cp reads them
+                        mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->full[stage]), 0));
+                        if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
+                    }
+                }
+                if (!ok) {
+                    raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
+                    *abort_flag = 1;
+                }
             }
-            if (!ok) {
-                raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
-                *abort_flag = 1;
-            }
-            tc_commit_1(&S->mma_done);
+            // every MMA issued so far must finish before TMEM is released
             volatile int never = 0;
             mbar_wait_bounded(&S->mma_done, 0, &never);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue (warps 0-7)
+        // ------------------------------------------------ epilogue (warps 0-7 of both CTAs)
+        // warp w drains TMEM lanes 32q .. 32q+31 (q = w % 4) for the 32-token
+        // chunks of parity w / 4.  GEMM1: quadrants 0-1 hold gate, 2-3 the up rows
+        // of the same features; GEMM2: quadrant q holds features 32q .. 32q+31.
         const int q = warp & 3, half = warp >> 2;
+        const int feat_lane = kG1 ? (q & 1) * 32 + lane : q * 32 + lane;
         const bool is_gate = q < 2;
-        const int xpair = half * 2 + (q & 1);
+        const int xpair = half * 2 + (q & 1);                 // gate/up warp pair (GEMM1)
+        const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
+                                          mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const MxTile w = mx_tile(t, s_tpre, s_tb, P);
-            // GEMM1: features fb*64 + (q & 1)*32 + lane; GEMM2: fb*128 + q*32 + lane
-            const int f = kG1 ? w.fb * 64 + (q & 1) * 32 + lane : w.fb * 128 + q * 32 + lane;
+        SliceReader reader;
+        while (true) {
+            int slice = -1;
+            if (kG1) {
+                // the gate warp reads the queue and hands the slice to its up partner;
+                // both then pass the same exchange barriers or both leave
+                if (is_gate) {
+                    if (!reader.next(S, abort_flag, lane == 0, slice)) slice = -2;
+                    if (lane == 0) S->pair_slice[xpair] = slice;
+                }
+                named_barrier_sync(1 + xpair, 64);
+                if (!is_gate) slice = *reinterpret_cast<volatile int *>(&S->pair_slice[xpair]);
+            } else {
+                if (!reader.next(S, abort_flag, lane == 0, slice)) slice = -2;
+            }
+            if (slice == -2) {
+                if (lane == 0) { raise_status(P.status, MOE_DEV_WAIT_TIMEOUT); *abort_flag = 1; }
+                break;
+            }
+            if (slice < 0) break;
+            int se, sfb, t_blk;
+            decode_tile(slice, s_tpre, s_tb, P.E, se, sfb, t_blk);
+            const MxTile ti = mx_tile_info(se, sfb, t_blk, P);
+            const int f = (sfb * 2 + (int)rank) * P.feat_per_cta + feat_lane;   // output feature
             const bool f_ok = f < P.out_cols;
             bool go;
             if (kG1) {
-                // the gate warp waits and tells its up partner, so that both pass the
-                // same exchange barriers or both leave
                 if (is_gate) {
-                    const bool g = lane == 0 ? mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag) : true;
-                    go = __shfl_sync(0xffffffffu, g ? 1 : 0, 0) != 0;
-                    if (lane == 0) S->pair_go[xpair] = go ? 1 : 0;
+                    go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
+                    if (lane == 0) S->go_flag[xpair] = go ? 1 : 0;
                 }
-                mx_named_barrier(1 + xpair, 64);
-                if (!is_gate) go = *reinterpret_cast<volatile int *>(&S->pair_go[xpair]) != 0;
+                named_barrier_sync(1 + xpair, 64);
+                if (!is_gate) go = *reinterpret_cast<volatile int *>(&S->go_flag[xpair]) != 0;
             } else {
-                const bool g = lane == 0 ? mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag) : true;
-                go = __shfl_sync(0xffffffffu, g ? 1 : 0, 0) != 0;
+                go = mbar_wait_bounded(&S->tmem_full[acc], acc_phase, abort_flag);
             }
             if (!go) {
                 if (lane == 0) { raise_status(P.status, MOE_DEV_WAIT_TIMEOUT); *abort_flag = 1; }
                 break;
             }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (uint32_t)(acc * kMxTile) + ((uint32_t)(q * 32) << 16);
-            for (int c0 = half * 32; c0 < w.n_mma; c0 += 64) {
+            const uint32_t tbase = tmem_base + (uint32_t)acc * kMxAccStride + ((uint32_t)(q * 32) << 16);
+            for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c0, r);
                 tc_wait_ld_regs(r);
@@ -353,68 +498,76 @@ __global__ void __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
                     float *theirs = xchg + (xpair * 2 + (is_gate ? 1 : 0)) * 512;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]);
-                    mx_named_barrier(1 + xpair, 64);
+                    named_barrier_sync(1 + xpair, 64);
                     float other[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) other[j] = theirs[j * 32 + lane];
-                    mx_named_barrier(1 + xpair, 64);
+                    named_barrier_sync(1 + xpair, 64);   // both read before the next chunk's writes
                     const int cbase = c0 + (is_gate ? 0 : 16);
-                    const int nc = min(16, w.n_valid - cbase);
-                    // h of 16 tokens for this lane's feature; the warp's 32 features are
-                    // one 32-value block of h: scale per token by the warp's maximum
-                    const size_t row0 = (size_t)(w.p0 + cbase);
+                    const int nc = min(16, ti.n_valid - cbase);
+                    // h of 16 tokens for this lane's feature, rounded to bf16; the warp's
+                    // 32 features are one 32-value block of h: per token, the block's
+                    // exponent from the warp's largest magnitude, then the E4M3 codes
+                    float hv[16];
+                    uint32_t amax[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float own = __uint_as_float(r[is_gate ? j : 16 + j]);
                         const float g = is_gate ? own : other[j], u = is_gate ? other[j] : own;
-                        const float hv = __bfloat162float(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u));
-                        const float a = f_ok ? fabsf(hv) : 0.0f;
-                        const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
-                        const int e = mx_exponent(__uint_as_float(amax_bits));
-                        const float sc = hv * mx_pow2_neg(e);
-                        const uint8_t code = (uint8_t)(__nv_cvt_float_to_fp8(sc, __NV_SATFINITE, __NV_E4M3));
+                        hv[j] = __bfloat162float(__float2bfloat16_rn(silu_f(g) * u));
+                        amax[j] = __reduce_max_sync(0xffffffffu, f_ok ? __float_as_uint(fabsf(hv[j])) : 0u);
+                    }
+                    const size_t row0 = (size_t)(ti.p0 + cbase);
+                    uint8_t *hq = P.h_q + row0 * P.out_cols + f;
+                    uint8_t *hs = P.h_sf + row0 * (P.out_cols / 32) + (f - lane) / 32;
+                    const bool blk_ok = f - lane < P.out_cols;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int e = mx_exponent_bits(amax[j]);
+                        const uint8_t code =
+                            (uint8_t)__nv_cvt_float_to_fp8(hv[j] * mx_pow2_neg(e), __NV_SATFINITE, __NV_E4M3);
                         if (j < nc) {
-                            if (f_ok) P.h_q[(row0 + j) * P.out_cols + f] = code;
-                            if (lane == 0 && f - lane < P.out_cols)
-                                P.h_sf[(row0 + j) * (P.out_cols / 32) + f / 32] = (uint8_t)(e + 127);
+                            if (f_ok) hq[(size_t)j * P.out_cols] = code;
+                            if (lane == 0 && blk_ok) hs[(size_t)j * (P.out_cols / 32)] = (uint8_t)(e + 127);
                         }
                     }
                 } else if (MODE == kMxStore) {
-                    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.y) + (size_t)w.p0 * P.out_cols + f;
-                    const int nc = min(32, w.n_valid - c0);
+                    // one 64-byte warp store per token row
+                    __nv_bfloat16 *y = P.y + (size_t)(ti.p0 + c0) * P.out_cols + f;
+                    const int nc = min(32, ti.n_valid - c0);
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_cols] = __float2bfloat16_rn(__uint_as_float(r[j]));
-                } else {
+                        if (f_ok && j < nc) y[(size_t)j * P.out_cols] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                } else {   // kMxReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
                     float my_w = 0.0f;
-                    const int nc = min(32, w.n_valid - c0);
+                    const int nc = min(32, ti.n_valid - c0);
                     if (lane < nc) {
-                        const int p = w.p0 + c0 + lane;
+                        const int p = ti.p0 + c0 + lane;
                         my_t = P.recv_token[p];
                         my_w = P.topk_w[(size_t)my_t * P.k + P.recv_slot[p]];
                     }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int tt = __shfl_sync(0xffffffffu, my_t, j);
-                        const float ww = __shfl_sync(0xffffffffu, my_w, j);
+                        const int t = __shfl_sync(0xffffffffu, my_t, j);
+                        const float w = __shfl_sync(0xffffffffu, my_w, j);
                         if (j < nc && f_ok)
-                            atomicAdd(P.out_reduce + (size_t)tt * P.out_cols + f, ww * __uint_as_float(r[j]));
+                            atomicAdd(P.out_reduce + (size_t)t * P.out_cols + f, w * __uint_as_float(r[j]));
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S->tmem_empty[acc]);
+            if (lane == 0) mbar_arrive_cluster(empty_leader[acc]);   // release the pair's accumulator
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();      // both CTAs done: no MMA, copy or remote arrive in flight
     if (warp == kMxMmaWarp) {
         tc_fence_after();
-        tmem_dealloc_1(tmem_base, kMxTmemCols);
+        tmem_dealloc_pair(tmem_base, kMxTmemCols);
     }
 }
 
@@ -432,13 +585,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 mx_encode_fn() {
     return fn;
 }
 
-// E4M3 rows [rows][K] as (128, rows, K / 128): 128-row boxes of two k-chunks.
-static bool mx_tmap_rows(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t K) {
+// E4M3 rows [rows][K] as (128, rows, K / 128): boxes of box_rows rows and two k-chunks.
+static bool mx_tmap_rows(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t K, uint32_t box_rows) {
     auto enc = mx_encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {128, rows, K / 128};
     const cuuint64_t strides[2] = {K, 128};
-    const cuuint32_t box[3] = {128, 128, 2};
+    const cuuint32_t box[3] = {128, box_rows, (cuuint32_t)kMxKS};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -452,7 +605,7 @@ static bool mx_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I,
     if (!enc) return false;
     const cuuint64_t dims[4] = {128, I, 2 * E, H / 128};
     const cuuint64_t strides[3] = {H, I * H, 128};
-    const cuuint32_t box[4] = {128, 64, 2, 2};
+    const cuuint32_t box[4] = {128, (cuuint32_t)kMxRows / 2, 2, (cuuint32_t)kMxKS};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -460,73 +613,83 @@ static bool mx_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I,
 }
 
 size_t ffn_mx_smem(int E, bool g1) {
-    return 1024 + (size_t)kMxStages * kMxStageBytes + (g1 ? kMxXchgBytes : 0) + sizeof(MxSmem) +
+    return 1024 + (size_t)kMxRingBytes + (g1 ? kMxXchgBytes : 0) + sizeof(MxSmem) +
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
 template <int MODE>
-static cudaError_t launch_mx(const CUtensorMap &tw, const CUtensorMap &tt, const MxParams &P, int grid,
-                             cudaStream_t s) {
+static cudaError_t launch_mx(const CUtensorMap &tw, const CUtensorMap &tt, const CUtensorMap &tts,
+                             const MxParams &P, int grid, uint32_t *counter, cudaStream_t s) {
     const size_t smem = ffn_mx_smem(P.E, MODE == kMxSwiGLUQuant);
-    static SmemOptIn opt_in;
+    static SmemOptIn opt_in;   // one per kernel instantiation
     cudaError_t err = opt_in.ensure(ffn_mx_tcgen05_kernel<MODE>, smem);
     if (err != cudaSuccess) return err;
-    ffn_mx_tcgen05_kernel<MODE><<<grid, kMxThreads, smem, s>>>(tw, tt, P);
+    ffn_mx_tcgen05_kernel<MODE><<<grid, kMxThreads, smem, s>>>(tw, tt, tts, P, counter);
     return cudaGetLastError();
+}
+
+// CTA pairs: an upper bound on the pair tiles is (n_rows / 224 + E) * n_fblocks
+static int mx_grid(const moe_config &c, int64_t n_rows, const MxParams &P, int num_sms) {
+    const long long max_pairs = num_sms / 2;
+    const long long g = (n_rows / kMxTileTok + c.E) * (long long)P.n_fblocks;
+    return 2 * (int)(g < max_pairs ? g : max_pairs);
 }
 
 // The block-scaled FP8 FFN: GEMM1 (SwiGLU, h quantised by 32-value blocks) then
 // GEMM2.  Scale arrays are bytes, one per row and 32 K values (read as words of
-// four).  Returns cudaErrorNotSupported when the tensor-map encoder is
-// unavailable or E exceeds the tile table's room.
+// four).  counters: two work counters.  Returns cudaErrorNotSupported when the
+// tensor-map encoder is unavailable or E exceeds the tile table's room.
 cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr_q, const uint8_t *xr_sf,
                           const int32_t *expert_offsets, const uint8_t *w13_q, const uint8_t *w13_sf,
                           const uint8_t *w2_q, const uint8_t *w2_sf, uint8_t *h_q, uint8_t *h_sf, void *y,
                           const int32_t *recv_token, const int32_t *recv_slot, const float *topk_w,
-                          float *out_reduce, uint32_t *status, cudaStream_t s, int num_sms) {
+                          float *out_reduce, uint32_t *status, uint32_t *counters, cudaStream_t s,
+                          int num_sms) {
     if (n_rows <= 0) return cudaSuccess;
     if (c.E > kMxMaxExperts) return cudaErrorNotSupported;
-    CUtensorMap tw1, tx, tw2, th;
-    if (!mx_tmap_w13(&tw1, w13_q, c.E, c.I, c.H) || !mx_tmap_rows(&tx, xr_q, n_rows, c.H) ||
-        !mx_tmap_rows(&tw2, w2_q, (uint64_t)c.E * c.H, c.I) || !mx_tmap_rows(&th, h_q, n_rows, c.I))
+    cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
+    if (cerr != cudaSuccess) return cerr;
+    const uint64_t n = (uint64_t)n_rows;
+    CUtensorMap tw1, tx, txs, tw2, th, ths;
+    if (!mx_tmap_w13(&tw1, w13_q, c.E, c.I, c.H) || !mx_tmap_rows(&tx, xr_q, n, c.H, kMxBoxTok) ||
+        !mx_tmap_rows(&txs, xr_q, n, c.H, kMxSmallBox) ||
+        !mx_tmap_rows(&tw2, w2_q, (uint64_t)c.E * c.H, c.I, kMxRows) ||
+        !mx_tmap_rows(&th, h_q, n, c.I, kMxBoxTok) || !mx_tmap_rows(&ths, h_q, n, c.I, kMxSmallBox))
         return cudaErrorNotSupported;
     MxParams P{};
     P.expert_offsets = expert_offsets;
     P.E = c.E;
-    P.n_rows = n_rows;
     P.k = c.k;
     P.status = status;
     P.recv_token = recv_token;
     P.recv_slot = recv_slot;
     P.topk_w = topk_w;
-    // GEMM1: 128 rows = the gate and up rows of 64 features
+    // GEMM1: each CTA's 128 rows are the gate and up rows of 64 features
     MxParams P1 = P;
     P1.K = c.H;
-    P1.n_fblocks = c.I / 64;
+    P1.feat_per_cta = kMxRows / 2;
+    P1.n_fblocks = c.I / (2 * P1.feat_per_cta);   // I is a multiple of 128
     P1.w_rows_per_expert = 2 * c.I;
-    P1.half_rows = c.I;
     P1.out_cols = c.I;
     P1.w_sf = reinterpret_cast<const uint32_t *>(w13_sf);
     P1.t_sf = reinterpret_cast<const uint32_t *>(xr_sf);
     P1.h_q = h_q;
     P1.h_sf = h_sf;
-    const long long cap = num_sms;
-    long long g1 = (n_rows / kMxTile + c.E) * (long long)P1.n_fblocks;
-    cudaError_t err = launch_mx<kMxSwiGLUQuant>(tw1, tx, P1, (int)(g1 < cap ? g1 : cap), s);
+    cudaError_t err = launch_mx<kMxSwiGLUQuant>(tw1, tx, txs, P1, mx_grid(c, n_rows, P1, num_sms), counters, s);
     if (err != cudaSuccess) return err;
     MxParams P2 = P;
     P2.K = c.I;
-    P2.n_fblocks = c.H / 128;
+    P2.feat_per_cta = kMxRows;
+    P2.n_fblocks = (c.H + 2 * kMxRows - 1) / (2 * kMxRows);
     P2.w_rows_per_expert = c.H;
     P2.out_cols = c.H;
     P2.w_sf = reinterpret_cast<const uint32_t *>(w2_sf);
     P2.t_sf = reinterpret_cast<const uint32_t *>(h_sf);
-    P2.y = y;
+    P2.y = static_cast<__nv_bfloat16 *>(y);
     P2.out_reduce = out_reduce;
-    long long g2 = (n_rows / kMxTile + c.E) * (long long)P2.n_fblocks;
-    const int grid2 = (int)(g2 < cap ? g2 : cap);
-    if (c.reduce_dense) return launch_mx<kMxReduce>(tw2, th, P2, grid2, s);
-    return launch_mx<kMxStore>(tw2, th, P2, grid2, s);
+    const int grid2 = mx_grid(c, n_rows, P2, num_sms);
+    if (c.reduce_dense) return launch_mx<kMxReduce>(tw2, th, ths, P2, grid2, counters + 1, s);
+    return launch_mx<kMxStore>(tw2, th, ths, P2, grid2, counters + 1, s);
 }
 
 }  // namespace moe

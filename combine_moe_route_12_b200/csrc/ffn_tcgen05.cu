@@ -48,7 +48,7 @@
 // returns.  No TMA load uses cluster multicast.
 #include <cudaTypedefs.h>
 
-#include "moe_common.cuh"
+#include "ffn_pair.cuh"
 
 namespace moe {
 
@@ -104,8 +104,6 @@ struct FfnGemmParams {
     __nv_bfloat16 *out2;
 };
 
-constexpr int kQueue = 8;                            // slices published ahead of the slowest consumer
-
 struct FfnSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
@@ -126,23 +124,6 @@ struct TileInfo {
     int e, f_blk, p0, n_valid, n_mma;   // n_valid <= 256 tokens; n_mma: the MMA's N (rounded to 16)
 };
 
-// Work is dealt out tile by tile from a global counter, so a pair that finishes
-// early takes more.  Tiles are numbered expert by expert, weight slice (expert,
-// pair feature block) by weight slice, token block innermost: the tiles of one
-// slice are taken back to back and stream the same weights at the same time.
-__device__ __forceinline__ void decode_tile(int tile, const int32_t *s_tpre, const int32_t *s_tb,
-                                            int E, int &e, int &f_blk, int &t_blk) {
-    int lo = 0, hi = E - 1;  // last e with s_tpre[e] <= tile (it owns >= 1 tile)
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_tpre[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    e = lo;
-    const int local = tile - s_tpre[lo];
-    f_blk = local / s_tb[lo];
-    t_blk = local - f_blk * s_tb[lo];
-}
-
 __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const FfnGemmParams &P) {
     TileInfo t;
     t.e = e;
@@ -154,11 +135,6 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
     t.n_mma = (t.n_valid + 15) & ~15;
     return t;
 }
-
-// silu in the bf16 epilogue: the fast exponential and reciprocal-based divide
-// (a few ulp in fp32) are far inside the bf16 rounding of h, and the IEEE divide
-// made the epilogue instruction-bound.  For g -> -inf the quotient is -0.
-__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // A UE8M0 scale byte as a float: 2^(b - 127) (b = 0 gives the subnormal 2^-127).
 __device__ __forceinline__ float ue8m0_value(uint32_t b) {
@@ -201,26 +177,6 @@ __device__ __forceinline__ void warp_tokens_to_rows(const float (&v)[T], uint4 (
         out[g].w = b2 ? q[2 * g + 1][1] : r1;
     }
 }
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// One consumer's position in the slice queue.  next() waits (bounded) for the
-// next published slice, reads it and releases the entry on the leader's
-// q_empty; it returns false on a timeout.  A slice of -1 ends the work.
-struct SliceReader {
-    int qi = 0;
-    uint32_t qph = 0;
-    __device__ __forceinline__ bool next(FfnSmem *S, volatile int *abort_flag, bool release,
-                                         int &slice) {
-        if (!mbar_wait_cluster_bounded(&S->q_full[qi], qph, abort_flag)) return false;
-        slice = *reinterpret_cast<volatile int *>(&S->q_slice[qi]);
-        if (release) mbar_arrive_cluster(mapa_shared(smem_u32(&S->q_empty[qi]), 0));
-        if (++qi == kQueue) { qi = 0; qph ^= 1u; }
-        return true;
-    }
-};
 
 // F8: E4M3 operands (tcgen05 kind::f8f6f4, 128 columns per k-chunk) with the
 // row scales applied to the fp32 accumulators in the epilogue; else bf16.

@@ -55,7 +55,8 @@ cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr
                           const int32_t *expert_offsets, const uint8_t *w13_q, const uint8_t *w13_sf,
                           const uint8_t *w2_q, const uint8_t *w2_sf, uint8_t *h_q, uint8_t *h_sf, void *y,
                           const int32_t *recv_token, const int32_t *recv_slot, const float *topk_w,
-                          float *out_reduce, uint32_t *status, cudaStream_t s, int num_sms);
+                          float *out_reduce, uint32_t *status, uint32_t *counters, cudaStream_t s,
+                          int num_sms);
 cudaError_t launch_combine_bwd(const moe_config &c, const void *dout, const void *y,
                                const int32_t *pos, const float *topk_w, int tb, int tc, void *dy,
                                float *dw, cudaStream_t s);
@@ -676,7 +677,8 @@ moe_status moe_grouped_swiglu_ffn_mxfp8(const moe_config *cfg, int64_t n_rows, c
     const ScratchLayout L = scratch_layout(c);
     cudaError_t err = launch_ffn_mx(c, n_rows, xr_q, xr_sf, expert_offsets, w13_q, w13_sf, w2_q, w2_sf, h_q,
                                     h_sf, y, recv_token, recv_slot, topk_w, out_reduce,
-                                    ws_at<uint32_t>(ws, L.status), stream, current_num_sms());
+                                    ws_at<uint32_t>(ws, L.status), ws_at<uint32_t>(ws, L.ffn_ctr), stream,
+                                    current_num_sms());
     if (err == cudaErrorNotSupported)
         return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_swiglu_ffn_mxfp8");
@@ -947,7 +949,8 @@ static moe_status forward_run(const moe_config &c, const ForwardLayout &F, const
                 err = launch_ffn_mx(c, F.nmax, static_cast<const uint8_t *>(xr), ws_at<uint8_t>(ws, S.xsf), eoff,
                                     static_cast<const uint8_t *>(w13), w13_scale, static_cast<const uint8_t *>(w2),
                                     w2_scale, ws_at<uint8_t>(ws, S.hq), ws_at<uint8_t>(ws, S.hsc), y, recv_token,
-                                    recv_slot, topk_w, out_reduce, status, s_compute, nsm);
+                                    recv_slot, topk_w, out_reduce, status, ws_at<uint32_t>(ws, L.ffn_ctr),
+                                    s_compute, nsm);
                 if (err == cudaErrorNotSupported)
                     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or rejected a tensor map");
             } else if (c.ffn_fp8) {

@@ -476,10 +476,44 @@ __device__ __forceinline__ void tc_mma_mx_1(uint32_t d_tmem, uint64_t a_desc, ui
                  : "memory");
 }
 
+// The same across a CTA pair (issued by the leader): each CTA's atom, at the
+// same shared-memory offset, into its own TMEM at tmem_col.
+__device__ __forceinline__ void tc_cp_sf_atom_pair(uint32_t tmem_col, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col), "l"(sdesc) : "memory");
+}
+// Block-scaled MMA across the CTA pair (M = 256, issued by the leader): each
+// CTA's TMEM holds the scales of its own 128 A rows at tsfa and the scales of
+// all N B rows at tsfb.
+__device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                               uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                 : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads of them (the tensor core's operand fetch, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+
+// 4-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros and reads
+// nothing (src must still be a 4-byte aligned address).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// One arrival on `bar` once every cp.async this thread issued before it has
+// landed; the arrival is counted in the barrier's initial count (.noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Waits until every cp.async this thread issued has landed.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 }  // namespace moe

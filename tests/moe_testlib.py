@@ -77,8 +77,10 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
     """Runs the six ABI steps chunk by chunk on the current CUDA stream.
 
     fp8: for a workload with ffn_fp8, the device (w13 codes, w13 scales, w2
-    codes, w2 scales); x is then quantised once, its codes are permuted and
-    step 5 is moe_grouped_swiglu_ffn_fp8."""
+    codes, w2 scales).  ffn_fp8 = 1: x is quantised once by rows, its codes are
+    permuted and step 5 is moe_grouped_swiglu_ffn_fp8.  ffn_fp8 = 2: the
+    permute quantises by 32-value blocks (moe_permute_quantize_fp8_blocks) and
+    step 5 is moe_grouped_swiglu_ffn_mxfp8 (no bf16 h)."""
     cfg = moe.config_from_workload(wl)
     dev = inp.logits.device
     T, E, k, H, I, ep = wl.T, wl.E, wl.k, wl.H, wl.I, wl.ep
@@ -96,7 +98,8 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
     nmax = moe.max_recv_rows(cfg, tc)
     chunks = []
     xq = xs = None
-    if wl.ffn_fp8:
+    mx = wl.ffn_fp8 == 2
+    if wl.ffn_fp8 and not mx:
         xq, xs = moe.quantize_fp8(inp.x)
     for c in range(wl.n_chunks):
         tb = c * tc
@@ -110,11 +113,22 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
         moe.moe_dispatch_layout(cfg, tb, tc, topk_idx, keep, eoff, roff, rt, rs, pos, spl, host, ws)
         xr = torch.empty((max(nmax, 1), H), dtype=torch.uint8 if wl.ffn_fp8 else wl.torch_dtype,
                          device=dev)
-        moe.moe_permute(cfg, xq if wl.ffn_fp8 else inp.x, pos, tb, tc, xr)
-        h = torch.empty((max(nmax, 1), I), dtype=wl.torch_dtype, device=dev)
+        xsf = hsf = None
+        if mx:
+            xsf = torch.full((max(nmax, 1), H // 32), 7, dtype=torch.uint8, device=dev)
+            moe.moe_permute_quantize_fp8_blocks(cfg, inp.x, pos, tb, tc, xr, xsf)
+        else:
+            moe.moe_permute(cfg, xq if wl.ffn_fp8 else inp.x, pos, tb, tc, xr)
+        h = None if mx else torch.empty((max(nmax, 1), I), dtype=wl.torch_dtype, device=dev)
         y = None if wl.reduce_dense else torch.empty((max(nmax, 1), H), dtype=wl.torch_dtype, device=dev)
         hq = hsc = None
-        if wl.ffn_fp8:
+        if mx:
+            hq = torch.empty((max(nmax, 1), I), dtype=torch.uint8, device=dev)
+            hsf = torch.full((max(nmax, 1), I // 32), 7, dtype=torch.uint8, device=dev)
+            w13q, w13s, w2q, w2s = fp8
+            moe.moe_grouped_swiglu_ffn_mxfp8(cfg, nmax, xr, xsf, eoff, w13q, w13s, w2q, w2s, hq, hsf, y,
+                                             rt, rs, topk_w, red, ws)
+        elif wl.ffn_fp8:
             hq = torch.empty((max(nmax, 1), I), dtype=torch.uint8, device=dev)
             hsc = torch.empty((max(nmax, 1),), dtype=torch.uint8, device=dev)
             w13q, w13s, w2q, w2s = fp8
@@ -138,13 +152,16 @@ def run_gpu_steps(wl: MoEWorkload, inp: MoEInputs, keep_rows: bool = True, fp8=N
                   recv_token=rt[:n].cpu().numpy(), recv_slot=rs[:n].cpu().numpy(),
                   pos=pos.cpu().numpy(), send_splits=spl.cpu().numpy(), host=host.numpy().copy())
         if keep_rows:
-            ch.update(xr=storage_np(xr[:n]), h=storage_np(h[:n]),
+            ch.update(xr=storage_np(xr[:n]), h=None if h is None else storage_np(h[:n]),
+                      xsf=None if xsf is None else xsf[:n].cpu().numpy(),
+                      hsf=None if hsf is None else hsf[:n].cpu().numpy(),
                       y=None if y is None else storage_np(y[:n]),
                       ys=None if ys is None else storage_np(ys),
                       hq=None if hq is None else hq[:n].cpu().numpy(),
                       hs=None if hsc is None else hsc[:n].cpu().numpy())
         else:
-            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys, hq_dev=hq, hs_dev=hsc)
+            ch.update(xr_dev=xr, h_dev=h, y_dev=y, ys_dev=ys, hq_dev=hq, hs_dev=hsc, xsf_dev=xsf,
+                      hsf_dev=hsf)
         chunks.append(ch)
     status = moe.moe_device_status(ws)
     torch.cuda.synchronize()

@@ -35,17 +35,17 @@ SHORT = 64          # tiles of at most this many rows take the short token box
 N_TOKENS = 128      # sampled tokens of the combined output
 
 
-def select_rows(lay, rng):
-    """Receive rows that cover every FFN tile of a chunk: per (expert, 256-row
-    block) its first and last row; a short last block (<= 64 rows) two more."""
+def select_rows(lay, rng, tile=TILE, short=SHORT):
+    """Receive rows that cover every FFN tile of a chunk: per (expert, tile-row
+    block) its first and last row; a short last block (<= short rows) two more."""
     eoff = lay["expert_offsets"]
     rows = set()
     for e in range(len(eoff) - 1):
         lo, hi = int(eoff[e]), int(eoff[e + 1])
-        for b0 in range(lo, hi, TILE):
-            b1 = min(b0 + TILE, hi) - 1
+        for b0 in range(lo, hi, tile):
+            b1 = min(b0 + tile, hi) - 1
             rows.update((b0, b1))
-            if b1 - b0 + 1 <= SHORT:
+            if b1 - b0 + 1 <= short:
                 rows.update(int(v) for v in rng.integers(b0, b1 + 1, 2))
     return rows
 
@@ -223,6 +223,98 @@ def test_fp8_fullsize_against_oracle(name):
         assert_codes_close(gc["hq_dev"][p:p + 1].cpu().numpy(), gc["hs_dev"][p:p + 1].cpu().numpy(),
                            hq[None], np.array([hs], np.uint8), f"h codes[{p}]", min_equal=0.98)
         assert_float_close(storage_np(gc["y_dev"][p]), y, "bf16", f"y[{p}] chunk {c}", per_element=False)
+
+    out = storage_np(g["out"])
+    for t in tokens:
+        c = t // tc
+        lay = orc["layouts"][c]
+        ys, pos = [], []
+        for j in range(wl.k):
+            p = int(lay["pos"][t - c * tc, j])
+            if p < 0:
+                pos.append(-1)
+                continue
+            pos.append(len(ys))
+            ys.append(ref[(c, p)][3])
+        want = oracle.combine(np.stack(ys), np.array([pos], np.int32), orc["topk_w"][t:t + 1], 1)
+        assert_float_close(out[t:t + 1], want, "bf16", f"out[{t}]", per_element=False)
+    del g, inp
+    torch.cuda.empty_cache()
+
+
+MX_TILE = 128       # token rows per tile of the block-scaled FP8 FFN
+
+
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b_mxfp8", "dsv3_prefill_mxfp8"])
+def test_mxfp8_fullsize_against_oracle(name):
+    """The FP8 layer with K-blocked scales at full size: x's block quantisation
+    whole and bit-exact (the standalone kernel), the fused permute's codes and
+    scales whole by the defining property (xr[p] = q(x)[recv_token[p]]), every
+    checked expert's weight codes and scales bit-exact, the rows of every
+    128-row FFN tile and of 128 sampled tokens against the oracle's blocked FP8
+    rows (h's codes by the adjacency bar, y by the bf16 bar), and the combined
+    output of those tokens."""
+    wl = WORKLOADS[name]
+    torch.cuda.empty_cache()
+    inp = make_inputs(wl, "cuda")
+    w13q, w13s = moe.quantize_fp8_blocks(inp.w13)
+    w2q, w2s = moe.quantize_fp8_blocks(inp.w2)
+    g = run_gpu_steps(wl, inp, keep_rows=False, fp8=(w13q, w13s, w2q, w2s))
+    assert g["status"] == 0
+    cpu_inp = MoEInputs(logits=inp.logits.cpu(), bias=None if inp.bias is None else inp.bias.cpu(),
+                        x=inp.x.cpu(), w13=inp.w13, w2=inp.w2)
+    orc = oracle_routing(wl, cpu_inp)
+    assert_routing_equal(g, orc, wl)
+    xq, xs = oracle.quantize_blocks(storage_np(inp.x), 32)
+    gxq, gxs = moe.quantize_fp8_blocks(inp.x)
+    np.testing.assert_array_equal(gxq.cpu().numpy(), xq)
+    np.testing.assert_array_equal(gxs.cpu().numpy(), xs)
+    xq_dev, xs_dev = torch.from_numpy(xq).cuda(), torch.from_numpy(xs).cuda()
+    del gxq, gxs
+    rng = np.random.default_rng(0)
+    H, I = wl.H, wl.I
+
+    def fetch(e):
+        # the oracle's block codes of expert e's weights, checked against the GPU's
+        a13, s13 = oracle.quantize_blocks(storage_np(inp.w13[e]), 32)
+        a2, s2 = oracle.quantize_blocks(storage_np(inp.w2[e]), 32)
+        np.testing.assert_array_equal(w13q[e].cpu().numpy().reshape(a13.shape), a13)
+        np.testing.assert_array_equal(w13s[e].cpu().numpy().reshape(s13.shape), s13)
+        np.testing.assert_array_equal(w2q[e].cpu().numpy().reshape(a2.shape), a2)
+        np.testing.assert_array_equal(w2s[e].cpu().numpy().reshape(s2.shape), s2)
+        return a13, s13, a2, s2
+
+    tc = wl.T // wl.n_chunks
+    tokens = sorted({0, wl.T - 1, *rng.choice(wl.T, N_TOKENS - 2, replace=False).tolist()})
+    wanted = {}
+    for c, (gc, lay) in enumerate(zip(g["chunks"], orc["layouts"])):
+        n = lay["N"]
+        rt = torch.from_numpy(lay["recv_token"]).long().cuda()
+        assert torch.equal(gc["xr_dev"][:n], xq_dev[rt]), "fused permute: codes"
+        assert torch.equal(gc["xsf_dev"][:n], xs_dev[rt]), "fused permute: block scales"
+        rows = select_rows(lay, rng, tile=MX_TILE, short=0)
+        for t in tokens:
+            if c * tc <= t < (c + 1) * tc:
+                rows.update(int(p) for p in lay["pos"][t - c * tc] if p >= 0)
+        for p in rows:
+            e = expert_of(lay["expert_offsets"], p)
+            wanted.setdefault(e, []).append(((c, p), int(lay["recv_token"][p])))
+    ref = oracle_rows(lambda tok, w: oracle.ffn_row_fp8_blocked(xq[tok], xs[tok], *w, 32), fetch, wanted)
+    assert len(ref) == sum(len(v) for v in wanted.values())
+    keys = sorted(ref)
+    for c in range(wl.n_chunks):
+        ps = [p for cc, p in keys if cc == c]
+        if not ps:
+            continue
+        gc = g["chunks"][c]
+        sel = torch.tensor(ps, dtype=torch.long, device="cuda")
+        ghq, ghs = gc["hq_dev"][sel].cpu().numpy(), gc["hsf_dev"][sel].cpu().numpy()
+        rhq = np.stack([ref[(c, p)][1] for p in ps])
+        rhs = np.stack([ref[(c, p)][2] for p in ps])
+        assert_codes_close(ghq, ghs.reshape(-1), rhq, rhs.reshape(-1), f"h codes chunk {c}")
+        gy = storage_np(gc["y_dev"][sel])
+        for j, p in enumerate(ps):
+            assert_float_close(gy[j], ref[(c, p)][3], "bf16", f"y[{p}] chunk {c}", per_element=False)
 
     out = storage_np(g["out"])
     for t in tokens:

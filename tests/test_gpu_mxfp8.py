@@ -19,7 +19,7 @@ from combine_moe_route_12_b200 import moe
 from combine_moe_route_12_b200.workload import MoEWorkload, make_inputs
 
 from moe_testlib import (assert_codes_close, assert_float_close, assert_routing_equal,
-                         oracle_routing, storage_np)
+                         oracle_routing, run_gpu_steps, storage_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -41,59 +41,6 @@ CASES = {
     "mx_decode": W("mx_decode", T=128, H=256, E=16, k=4, I=256, dtype="bf16", ep=4, capacity=64,
                    reduce_dense=True, ffn_fp8=2),
 }
-
-
-def _run_steps(wl, inp, w13q, w13s, w2q, w2s):
-    cfg = moe.config_from_workload(wl)
-    dev = "cuda"
-    T, E, k, H, I, ep = wl.T, wl.E, wl.k, wl.H, wl.I, wl.ep
-    ws = moe.alloc_workspace(moe.workspace_bytes(cfg), dev)
-    idx = torch.empty(T, k, dtype=torch.int32, device=dev)
-    w = torch.empty(T, k, dtype=torch.float32, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    keep = torch.empty(T, k, dtype=torch.uint8, device=dev)
-    kept = torch.empty(E, dtype=torch.int32, device=dev)
-    moe.moe_route_topk(cfg, inp.logits, inp.bias, idx, w, counts, ws)
-    moe.moe_capacity_clip(cfg, idx, w, counts, keep, kept, ws)
-    out = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device=dev)
-    red = torch.zeros(T, H, dtype=torch.float32, device=dev) if wl.reduce_dense else None
-    tc = T // wl.n_chunks
-    nmax = moe.max_recv_rows(cfg, tc)
-    n = max(nmax, 1)
-    chunks = []
-    for c in range(wl.n_chunks):
-        tb = c * tc
-        eoff = torch.empty(E + 1, dtype=torch.int32, device=dev)
-        roff = torch.empty(ep + 1, dtype=torch.int32, device=dev)
-        rt = torch.empty(n, dtype=torch.int32, device=dev)
-        rs = torch.empty(n, dtype=torch.int32, device=dev)
-        pos = torch.empty(tc, k, dtype=torch.int32, device=dev)
-        spl = torch.empty(ep, ep, dtype=torch.int32, device=dev)
-        host = torch.empty(E + 1 + ep * ep, dtype=torch.int32).pin_memory()
-        moe.moe_dispatch_layout(cfg, tb, tc, idx, keep, eoff, roff, rt, rs, pos, spl, host, ws)
-        xr = torch.empty(n, H, dtype=torch.uint8, device=dev)
-        xsf = torch.empty(n, H // 32, dtype=torch.uint8, device=dev)
-        moe.moe_permute_quantize_fp8_blocks(cfg, inp.x, pos, tb, tc, xr, xsf)
-        hq = torch.empty(n, I, dtype=torch.uint8, device=dev)
-        hsf = torch.empty(n, I // 32, dtype=torch.uint8, device=dev)
-        y = None if wl.reduce_dense else torch.empty(n, H, dtype=torch.bfloat16, device=dev)
-        moe.moe_grouped_swiglu_ffn_mxfp8(cfg, nmax, xr, xsf, eoff, w13q, w13s, w2q, w2s, hq, hsf, y, rt, rs,
-                                         w, red, ws)
-        if wl.reduce_dense:
-            moe.moe_reduce_finalize(cfg, red, tb, tc, out)
-        else:
-            moe.moe_combine(cfg, y, pos, w, tb, tc, out)
-        torch.cuda.synchronize()
-        N = int(eoff[E].item())
-        chunks.append(dict(N=N, expert_offsets=eoff.cpu().numpy(), rank_offsets=roff.cpu().numpy(),
-                           recv_token=rt[:N].cpu().numpy(), recv_slot=rs[:N].cpu().numpy(),
-                           pos=pos.cpu().numpy(), send_splits=spl.cpu().numpy(), host=host.numpy().copy(),
-                           xr=xr[:N].cpu().numpy(), xsf=xsf[:N].cpu().numpy(), hq=hq[:N].cpu().numpy(),
-                           hsf=hsf[:N].cpu().numpy(), y=None if y is None else storage_np(y[:N])))
-    status = moe.moe_device_status(ws)
-    return dict(topk_idx=idx.cpu().numpy(), topk_w=w.cpu().numpy(), counts=counts.cpu().numpy(),
-                keep=keep.cpu().numpy(), kept_counts=kept.cpu().numpy(), chunks=chunks, out=out,
-                status=status)
 
 
 def _quantized_weights(inp):
@@ -120,7 +67,7 @@ def test_mxfp8_layer_steps_match_oracle(name):
     wl = CASES[name]
     inp = make_inputs(wl, "cuda", seed=2)
     w13q, w13s, w2q, w2s = _quantized_weights(inp)
-    g = _run_steps(wl, inp, w13q, w13s, w2q, w2s)
+    g = run_gpu_steps(wl, inp, fp8=(w13q, w13s, w2q, w2s))
     assert g["status"] == 0
     orc = oracle_routing(wl, inp)
     assert_routing_equal(g, orc, wl)
@@ -172,7 +119,7 @@ def test_mxfp8_forward_equals_steps(name):
     wl = CASES[name]
     inp = make_inputs(wl, "cuda", seed=4)
     w13q, w13s, w2q, w2s = _quantized_weights(inp)
-    g = _run_steps(wl, inp, w13q, w13s, w2q, w2s)
+    g = run_gpu_steps(wl, inp, fp8=(w13q, w13s, w2q, w2s))
     cfg = moe.config_from_workload(wl)
     layer = moe.MoELayer(cfg, host_io=True)
     out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device="cuda")
