@@ -146,7 +146,8 @@ def kernel_src_hash(fp8: bool = False, mx: bool = False):
     the row quantisation between its launches (the block-scaled FP8 FFN: its own
     kernel).  Recorded traffic holds only for these bytes."""
     h = hashlib.sha256()
-    names = ("ffn_mx_tcgen05.cu",) if mx else ("ffn_tcgen05.cu", "fp8_quant.cu") if fp8 else ("ffn_tcgen05.cu",)
+    names = (("ffn_mx_tcgen05.cu", "ffn_pair.cuh") if mx else
+             ("ffn_tcgen05.cu", "ffn_pair.cuh", "fp8_quant.cu") if fp8 else ("ffn_tcgen05.cu", "ffn_pair.cuh"))
     for name in names:
         with open(os.path.join(ROOT, "combine_moe_route_12_b200", "csrc", name), "rb") as f:
             h.update(f.read())

@@ -270,10 +270,37 @@ __global__ void clip_mark_kernel(int T, int E, int k, const int32_t *__restrict_
     if (bad) raise_status(status, MOE_DEV_BAD_INDEX);
 }
 
+// No capacity (C < 0): every valid assignment is kept and the kept counts are
+// the routed counts; one pass, the same index check as the marking pass.
+__global__ void clip_all_kernel(int T, int E, int k, const int32_t *__restrict__ topk_idx,
+                                const int32_t *__restrict__ counts, uint8_t *__restrict__ keep,
+                                int32_t *__restrict__ kept_counts, uint32_t *__restrict__ status) {
+    if (blockIdx.x == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) kept_counts[e] = counts[e];
+    const size_t total = (size_t)T * k;
+    bool bad = false;
+    for (size_t a = (size_t)blockIdx.x * blockDim.x + threadIdx.x; a < total;
+         a += (size_t)gridDim.x * blockDim.x) {
+        const int e = topk_idx[a];
+        const bool ok = e >= 0 && e < E;
+        bad |= !ok;
+        keep[a] = ok ? 1 : 0;
+    }
+    if (bad) raise_status(status, MOE_DEV_BAD_INDEX);
+}
+
 cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
                                  const float *topk_w, const int32_t *counts, uint8_t *keep,
                                  int32_t *kept_counts, uint64_t *thr, int32_t *seg, uint64_t *keys,
                                  uint32_t *status, cudaStream_t s, int num_sms) {
+    if (c.capacity < 0) {
+        const size_t total = (size_t)c.T * c.k;
+        int blocks = (int)((total + 255) / 256);
+        if (blocks > num_sms * 16) blocks = num_sms * 16;
+        if (blocks < 1) blocks = 1;
+        clip_all_kernel<<<blocks, 256, 0, s>>>(c.T, c.E, c.k, topk_idx, counts, keep, kept_counts, status);
+        return cudaGetLastError();
+    }
     clip_prep_kernel<<<1, 1024, 0, s>>>(c.E, c.capacity, counts, seg, kept_counts, thr);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -29,22 +29,27 @@
 // CTA's 128 weight rows are the gate rows of 64 features and their 64 up rows
 // (TMEM lanes i and 64 + i); in GEMM2 128 output features.
 //
-// Roles (10 warps per CTA).  Warp 8 of each CTA streams its ring stages (two
-// k-chunks: 32 KiB of weight rows and 28 KiB of token rows by TMA, counted on
-// the leader's barrier) and, with all its lanes, gathers the stage's scale
-// words with 4-byte cp.async into 512-byte scale atoms (row r's word at byte
+// Roles (11 warps per CTA).  Warp 8 (one lane) of each CTA streams its ring
+// stages (two k-chunks: 32 KiB of weight rows and 28 KiB of token rows by TMA,
+// counted on the leader's barrier).  Warp 10 gathers, with all its lanes, the
+// scale words of the same stages into a separate, deeper ring of 3 KiB slots:
+// 4-byte cp.async copies into 512-byte scale atoms (row r's word at byte
 // 16 (r % 32) + 4 (r / 32), the layout tcgen05.cp spreads over the four TMEM
-// lane quadrants): its own 128 weight rows, and all the tile's tokens, which
-// both CTAs hold in TMEM.  The leader's lanes signal their copies on the
-// leader's full barrier; the follower's on a local barrier that the follower's
-// warp 9 (otherwise idle) forwards to the leader's.  The leader's warp 9 (one
-// lane) copies both CTAs' atoms to TMEM (tcgen05.cp cta_group::2), issues the
-// stage's eight block-scaled MMAs and commits to both CTAs' barriers.  Warps
-// 0-7 of each CTA drain TMEM (warps q and q + 4 share lane quadrant q and take
-// alternate 32-token chunks); in GEMM1 the gate and up warps swap half their
-// tokens through shared memory, and each warp then quantises its 32 features
-// (one 32-value block of h) for 16 tokens with a warp max per token.  Tiles are
-// dealt from a global counter and published through the pair's slice queue.
+// lane quadrants) - its CTA's own 128 weight rows, and all the tile's tokens,
+// which both CTAs hold in TMEM.  A scale slot is free again as soon as its atoms
+// are in TMEM, so the gather runs several stages ahead of the operands and its
+// latency (scattered words, and the hop below) stays off the stage's refill
+// chain.  The leader's gather lanes signal the leader's scale barrier; the
+// follower's signal a local one that the follower's warp 9 (otherwise idle)
+// forwards to the leader's.  The leader's warp 10 also deals the tiles (a global
+// counter, one ticket ahead) and publishes them to every role of both CTAs
+// through the pair's slice queue.  The leader's warp 9 (one lane) copies both
+// CTAs' atoms to TMEM (tcgen05.cp cta_group::2), frees the scale slot, issues
+// the stage's eight block-scaled MMAs and commits to both CTAs' barriers.
+// Warps 0-7 of each CTA drain TMEM (warps q and q + 4 share lane quadrant q and
+// take alternate 32-token chunks); in GEMM1 the gate and up warps swap half
+// their tokens through shared memory, and each warp then quantises its 32
+// features (one 32-value block of h) for 16 tokens with a warp max per token.
 //
 // Every wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT, stops the
 // other roles, lets in-flight copies and MMAs land, frees TMEM and returns.  No
@@ -64,17 +69,20 @@ constexpr int kMxKS = 2;                                      // 128-value k-chu
 constexpr uint32_t kMxWChunk = kMxRows * 128;                 // 16 KiB of weight rows per k-chunk
 constexpr uint32_t kMxTChunk = kMxBoxTok * 128;               // 14 KiB of token rows per k-chunk
 constexpr uint32_t kMxAtom = 512;                             // 128 rows x 4 block scales
-// stage: [W c0 | W c1 | T c0 | T c1 | SFA c0 | SFA c1 | SFB c0 a0 | c0 a1 | c1 a0 | c1 a1]
+// operand stage: [W c0 | W c1 | T c0 | T c1]
 constexpr uint32_t kMxTOff = kMxKS * kMxWChunk;
-constexpr uint32_t kMxSfOff = kMxTOff + kMxKS * kMxTChunk;
-constexpr uint32_t kMxStageBytes = kMxSfOff + 6 * kMxAtom;    // 63 KiB
+constexpr uint32_t kMxStageBytes = kMxTOff + kMxKS * kMxTChunk;   // 60 KiB
 constexpr int kMxStages = 3;
 constexpr uint32_t kMxRingBytes = kMxStages * kMxStageBytes;
 static_assert(kMxStageBytes % 1024 == 0 && kMxTOff % 1024 == 0 && kMxTChunk % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
+// scale slot of one stage: [SFA c0 | SFA c1 | SFB c0 a0 | c0 a1 | c1 a0 | c1 a1]
+constexpr uint32_t kMxSfSlotBytes = 6 * kMxAtom;
+constexpr int kMxSfStages = 6;
+constexpr uint32_t kMxSfRingBytes = kMxSfStages * kMxSfSlotBytes;
 constexpr int kMxEpiWarps = 8;
-constexpr int kMxProdWarp = kMxEpiWarps, kMxMmaWarp = kMxEpiWarps + 1;
-constexpr int kMxThreads = 32 * (kMxEpiWarps + 2);
+constexpr int kMxProdWarp = kMxEpiWarps, kMxMmaWarp = kMxEpiWarps + 1, kMxSfWarp = kMxEpiWarps + 2;
+constexpr int kMxThreads = 32 * (kMxEpiWarps + 3);
 constexpr uint32_t kMxTmemCols = 512;
 constexpr uint32_t kMxAccStride = 256;                        // accumulator a at column 256 a
 constexpr uint32_t kMxSfCol = kMxTileTok;                    // scale slot a at kMxSfCol + 256 a (24 columns)
@@ -106,9 +114,11 @@ struct MxParams {
 };
 
 struct MxSmem {
-    uint64_t full[kMxStages];      // leader: TMA bytes of both CTAs, its 32 gather lanes, the follower's forward
-    uint64_t empty[kMxStages];
-    uint64_t sf_full[kMxStages];   // follower: its 32 gather lanes
+    uint64_t full[kMxStages];        // leader: the TMA bytes of both CTAs
+    uint64_t empty[kMxStages];       // the stage's MMAs are done (both CTAs)
+    uint64_t sf_full[kMxSfStages];   // leader: its 32 gather lanes and the follower's forward;
+                                     // follower: its 32 gather lanes
+    uint64_t sf_empty[kMxSfStages];  // the slot's atoms are in TMEM (both CTAs)
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t mma_done;
@@ -160,16 +170,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_t,
     const __grid_constant__ CUtensorMap tmap_ts, const MxParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kG1 = MODE == kMxSwiGLUQuant;
-    // queue consumers per entry: the leader's MMA thread, the follower's producer
-    // and forwarder, and every epilogue warp of both CTAs (GEMM1: the gate warps)
-    constexpr uint32_t kQueueConsumers = 3 + 2 * (kG1 ? kMxEpiWarps / 2 : kMxEpiWarps);
+    // queue consumers per entry: the leader's MMA thread and operand producer, the
+    // follower's operand producer, scale gatherer and forwarder, and every epilogue
+    // warp of both CTAs (GEMM1: the gate warps); the leader's scale warp publishes
+    constexpr uint32_t kQueueConsumers = 5 + 2 * (kG1 ? kMxEpiWarps / 2 : kMxEpiWarps);
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled tiles (same offsets in both CTAs of the pair)
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *ring = base;                                       // [stages][W | T | scale atoms]
-    float *xchg = reinterpret_cast<float *>(base + kMxRingBytes);     // GEMM1 only
-    MxSmem *S = reinterpret_cast<MxSmem *>(base + kMxRingBytes + (kG1 ? kMxXchgBytes : 0));
+    unsigned char *ring = base;                                       // [stages][W | T]
+    unsigned char *sf_ring = base + kMxRingBytes;                     // [scale stages][6 atoms]
+    float *xchg = reinterpret_cast<float *>(sf_ring + kMxSfRingBytes);   // GEMM1 only
+    MxSmem *S = reinterpret_cast<MxSmem *>(sf_ring + kMxSfRingBytes + (kG1 ? kMxXchgBytes : 0));
     int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);            // [E + 1] tile prefix
     int32_t *s_tb = s_tpre + (P.E + 1);                               // [E] token blocks per expert
 
@@ -199,9 +211,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kMxStages; ++s) {
-            mbar_init(&S->full[s], 1 + 32 + 1);
+            mbar_init(&S->full[s], 1);
             mbar_init(&S->empty[s], 1);
-            mbar_init(&S->sf_full[s], 32);
+        }
+        for (int s = 0; s < kMxSfStages; ++s) {
+            mbar_init(&S->sf_full[s], rank == 0 ? 32 + 1 : 32);
+            mbar_init(&S->sf_empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&S->tmem_full[a], 1);
@@ -230,18 +245,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
     volatile int *abort_flag = &S->abort_flag;
 
     if (warp == kMxProdWarp) {
-        // ------------------------------------------------ TMA + scale gather (whole warp, both CTAs)
-        int stage = 0;
-        uint32_t phase = 0;
-        long long issued = 0;
+        // ------------------------------------------------ TMA producer (one lane, both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            SliceReader reader;
+            int slice;
+            while (ok) {
+                if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
+                if (slice < 0) break;
+                int se, sfb, t_blk;
+                decode_tile(slice, s_tpre, s_tb, P.E, se, sfb, t_blk);
+                const MxTile ti = mx_tile_info(se, sfb, t_blk, P);
+                // this CTA's weight rows and its half of the tile's tokens
+                const int f0 = (sfb * 2 + (int)rank) * P.feat_per_cta;
+                const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
+                const bool small_box = ti.n_mma / 2 <= kMxSmallBox;
+                const uint32_t stage_tx = kMxKS * (kMxWChunk + (small_box ? kMxSmallBox : kMxBoxTok) * 128);
+                for (int kb = 0; kb < num_k; ++kb) {
+                    if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+                    unsigned char *st = ring + stage * kMxStageBytes;
+                    const int ch = kb * kMxKS;   // first k-chunk of the stage
+                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * stage_tx);
+                    if (kG1)
+                        tma_load_4d_pair(st, &tmap_w, full_leader, 0, f0, 2 * se, ch);
+                    else
+                        tma_load_3d_pair(st, &tmap_w, full_leader, 0, se * P.w_rows_per_expert + f0, ch);
+                    tma_load_3d_pair(st + kMxTOff, small_box ? &tmap_ts : &tmap_t, full_leader, 0, tok_row, ch);
+                    ++issued;
+                    if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {
+                raise_status(P.status, MOE_DEV_WAIT_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // the leader's full barriers count both CTAs' bytes: let the last copies land
+            if (rank == 0) {
+                volatile int never = 0;
+                const long long last = issued < kMxStages ? issued : kMxStages;
+                int st = stage;
+                uint32_t ph = phase;
+                for (long long i = 0; i < last; ++i) {
+                    if (--st < 0) { st = kMxStages - 1; ph ^= 1u; }
+                    mbar_wait_bounded(&S->full[st], ph, &never);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMxSfWarp) {
+        // ------------------------------------------------ scale gather (whole warp, both CTAs);
+        // the leader's also deals the tiles
+        int sstage = 0;
+        uint32_t sphase = 0;
         bool ok = true;
         int qi = 0;
         uint32_t qph = 0;
         SliceReader reader;
         // the leader holds one ticket ahead: the counter's round trip for the
-        // next tile overlaps the loads of the current one
+        // next tile overlaps the gathers of the current one
         int ticket = (rank == 0 && lane == 0) ? (int)atomicAdd(work_counter, 1u) : 0;
-        uint64_t *my_full = rank == 0 ? S->full : S->sf_full;
         while (ok) {
             int slice = 0;
             bool got = true;
@@ -264,11 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
             int se, sfb, t_blk;
             decode_tile(slice, s_tpre, s_tb, P.E, se, sfb, t_blk);
             const MxTile ti = mx_tile_info(se, sfb, t_blk, P);
-            // this CTA's first output feature, weight rows and token rows
             const int f0 = (sfb * 2 + (int)rank) * P.feat_per_cta;
-            const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
-            const bool small_box = ti.n_mma / 2 <= kMxSmallBox;
-            const uint32_t stage_tx = kMxKS * (kMxWChunk + (small_box ? kMxSmallBox : kMxBoxTok) * 128);
             // the scale rows this lane gathers: weight rows r = lane + 32 i (-1: past
             // the expert's features) and the tile's tokens n = lane + 32 i (-1: past n_valid)
             int64_t wrow[4], trow[8];
@@ -290,23 +352,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                 trow[i] = n < ti.n_valid ? (int64_t)ti.p0 + n : -1;
             }
             for (int kb = 0; kb < num_k; ++kb) {
-                const bool w_ok = lane == 0 ? mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag) : true;
+                const bool w_ok = lane == 0 ? mbar_wait_bounded(&S->sf_empty[sstage], sphase ^ 1u, abort_flag) : true;
                 if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
-                unsigned char *st = ring + stage * kMxStageBytes;
-                const int ch = kb * kMxKS;   // first k-chunk of the stage
-                if (lane == 0) {
-                    const uint32_t full_leader = mapa_shared(smem_u32(&S->full[stage]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&S->full[stage], 2 * stage_tx);
-                    if (kG1)
-                        tma_load_4d_pair(st, &tmap_w, full_leader, 0, f0, 2 * se, ch);
-                    else
-                        tma_load_3d_pair(st, &tmap_w, full_leader, 0, se * P.w_rows_per_expert + f0, ch);
-                    tma_load_3d_pair(st + kMxTOff, small_box ? &tmap_ts : &tmap_t, full_leader, 0, tok_row, ch);
-                }
-                // scale atoms (row r's word at byte 16 (r % 32) + 4 (r / 32)): weight rows
-                // of chunk c at atom c, tokens 128 a .. 128 a + 127 of chunk c at atom 2 + 2c + a;
-                // words past K or of rows past the tile are zeros
-                const uint32_t sfs = smem_u32(st + kMxSfOff) + 16 * lane;
+                const int ch = kb * kMxKS;
+                // weight rows of chunk c at atom c, tokens 128 a .. 128 a + 127 of chunk c
+                // at atom 2 + 2c + a; words past K or of rows past the tile are zeros
+                const uint32_t sfs = smem_u32(sf_ring + sstage * kMxSfSlotBytes) + 16 * lane;
 #pragma unroll
                 for (int c = 0; c < kMxKS; ++c) {
                     const bool in_k = ch + c < kwords;
@@ -323,9 +374,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                                    ok_t ? P.t_sf + trow[i] * kwords + ch + c : P.t_sf, ok_t ? 4u : 0u);
                     }
                 }
-                cp_async_mbar_arrive_noinc(&my_full[stage]);
-                ++issued;
-                if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
+                cp_async_mbar_arrive_noinc(&S->sf_full[sstage]);
+                if (++sstage == kMxSfStages) { sstage = 0; sphase ^= 1u; }
             }
         }
         if (!ok && lane == 0) {
@@ -333,27 +383,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
             *abort_flag = 1;
         }
         cp_async_wait_all();   // this lane's scale copies have landed
-        // the leader's full barriers count both CTAs' bytes: let the last copies land
-        if (rank == 0 && lane == 0) {
-            volatile int never = 0;
-            const long long last = issued < kMxStages ? issued : kMxStages;
-            int st = stage;
-            uint32_t ph = phase;
-            for (long long i = 0; i < last; ++i) {
-                if (--st < 0) { st = kMxStages - 1; ph ^= 1u; }
-                mbar_wait_bounded(&S->full[st], ph, &never);
-            }
-        }
         __syncwarp();
     } else if (warp == kMxMmaWarp) {
         if (lane == 0) {
             if (rank == 0) {
                 // ------------------------------------------------ scale copies + MMA issuer (leader)
-                int stage = 0;
-                uint32_t phase = 0;
+                int stage = 0, sstage = 0;
+                uint32_t phase = 0, sphase = 0;
                 int acc = 0;
                 uint32_t acc_phase = 0;
-                uint32_t slot = 0;     // scale columns alternate between two slots, stage by stage
+                uint32_t slot = 0;     // TMEM scale columns alternate between two slots, stage by stage
                 bool ok = true;
                 SliceReader reader;
                 int slice;
@@ -369,16 +408,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                     // k-chunk stride inside the stage's token box (32 or 112 rows)
                     const uint32_t tchunk = ti.n_mma / 2 <= kMxSmallBox ? kMxSmallBox * 128 : kMxTChunk;
                     for (int kb = 0; kb < num_k; ++kb) {
-                        if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+                        // the stage's scales: both CTAs' atoms into TMEM, then the slot is free
+                        if (!mbar_wait_bounded(&S->sf_full[sstage], sphase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         fence_proxy_async_smem();   // the leader's cp.async scale words, before tcgen05.cp
-                        const uint32_t st = smem_u32(ring + stage * kMxStageBytes);
-                        const uint32_t sf = st + kMxSfOff;
+                        const uint32_t sf = smem_u32(sf_ring + sstage * kMxSfSlotBytes);
                         const uint32_t tsf = tmem_base + kMxSfCol + kMxAccStride * slot;
                         // weight-row scales of chunk c at tsf + 4c, token scales at tsf + 8 + 8c
 #pragma unroll
                         for (int a = 0; a < 6; ++a)
                             tc_cp_sf_atom_pair(tsf + 4 * a, make_sf_atom_desc(sf + a * kMxAtom));
+                        tc_commit_pair_mc(&S->sf_empty[sstage], 0x3);
+                        if (++sstage == kMxSfStages) { sstage = 0; sphase ^= 1u; }
+                        // the stage's operands
+                        if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t st = smem_u32(ring + stage * kMxStageBytes);
 #pragma unroll
                         for (int c = 0; c < kMxKS; ++c) {
 #pragma unroll
@@ -406,10 +451,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                 tc_commit_pair_mc(&S->mma_done, 0x3);
             } else {
                 // ------------------------------------------------ forwarder (follower)
-                // each stage's scale copies of this CTA, once landed, counted on the
-                // leader's full barrier
-                int stage = 0;
-                uint32_t phase = 0;
+                // each scale slot of this CTA, once its copies have landed, counted on
+                // the leader's scale barrier
+                int sstage = 0;
+                uint32_t sphase = 0;
                 bool ok = true;
                 SliceReader reader;
                 int slice;
@@ -417,10 +462,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                     if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
                     if (slice < 0) break;
                     for (int kb = 0; kb < num_k; ++kb) {
-                        if (!mbar_wait_bounded(&S->sf_full[stage], phase, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait_bounded(&S->sf_full[sstage], sphase, abort_flag)) { ok = false; break; }
                         fence_proxy_async_smem();   // before the leader's tcgen05.cp reads them
-                        mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->full[stage]), 0));
-                        if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
+                        mbar_arrive_cluster_release(mapa_shared(smem_u32(&S->sf_full[sstage]), 0));
+                        if (++sstage == kMxSfStages) { sstage = 0; sphase ^= 1u; }
                     }
                 }
                 if (!ok) {
@@ -613,7 +658,7 @@ static bool mx_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t I,
 }
 
 size_t ffn_mx_smem(int E, bool g1) {
-    return 1024 + (size_t)kMxRingBytes + (g1 ? kMxXchgBytes : 0) + sizeof(MxSmem) +
+    return 1024 + (size_t)kMxRingBytes + kMxSfRingBytes + (g1 ? kMxXchgBytes : 0) + sizeof(MxSmem) +
            sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
 }
 
