@@ -570,13 +570,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 } else if (MODE == kEpiStore) {
                     // one 64-byte warp store per token row (the shuffle rearrangement
                     // of the SwiGLU epilogue measured slower here)
-                    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld + f;
-                    const int nc = min(32, ti.n_valid - c0);
+                    if (F8) {
+                        // each token's scale from the lane that loaded it, times this
+                        // lane's weight-row scale, all taken before the stores
+                        float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float v = __uint_as_float(r[j]);
-                        if (F8) v *= __shfl_sync(0xffffffffu, ts_lane, j) * wsc;
-                        if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(v);
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = __uint_as_float(r[j]) * (__shfl_sync(0xffffffffu, ts_lane, j) * wsc);
+                        const int nc = f_ok ? min(32, ti.n_valid - c0) : 0;
+                        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)(ti.p0 + c0) * P.out_ld + f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            if (j < nc) *y = __float2bfloat16_rn(v[j]);
+                            y += P.out_ld;
+                        }
+                    } else {
+                        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld + f;
+                        const int nc = min(32, ti.n_valid - c0);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(__uint_as_float(r[j]));
                     }
                 } else {  // kEpiReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
