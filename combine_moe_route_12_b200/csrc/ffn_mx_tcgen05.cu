@@ -577,12 +577,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                         }
                     }
                 } else if (MODE == kMxStore) {
-                    // one 64-byte warp store per token row
+                    // one 64-byte warp store per token row, down a running row pointer
                     __nv_bfloat16 *y = P.y + (size_t)(ti.p0 + c0) * P.out_cols + f;
-                    const int nc = min(32, ti.n_valid - c0);
+                    const int nc = f_ok ? min(32, ti.n_valid - c0) : 0;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (f_ok && j < nc) y[(size_t)j * P.out_cols] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                    for (int j = 0; j < 32; ++j) {
+                        if (j < nc) *y = __float2bfloat16_rn(__uint_as_float(r[j]));
+                        y += P.out_cols;
+                    }
                 } else {   // kMxReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
                     float my_w = 0.0f;
