@@ -55,14 +55,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": 1560.882432e6, "src": "24bdbd71939c8d30"},
+    "qwen3_30b_a3b": {"bytes": (941.411328 + 48.232192 + 453.837312 + 115.365120) * 1e6,
+                      "src": "a15a55f4109395c7"},
     # both GEMM launches and the quantisation of h between them
-    "qwen3_30b_a3b_fp8": {"bytes": 893.983232e6, "src": "ab5f51ea4de56437"},
+    "qwen3_30b_a3b_fp8": {"bytes": (470.987520 + 44.082688 + 50.341376 + 1.413888 + 227.298304 +
+                                    102.075648) * 1e6, "src": "67604f868e3e8b13"},
+    "qwen3_30b_a3b_mxfp8": {"bytes": (484.921344 + 24.599296 + 233.696768 + 106.839296) * 1e6,
+                            "src": "32d5db20d0508550"},
     # captured with 32 of the 256 experts and 1024 tokens (the same 128 rows per
     # expert and chunk), scaled by 8 per chunk, two chunks; see
-    # profiles/ffn_tcgen05_dsv3_prefill.md
-    "dsv3_prefill": {"bytes": 2 * 8 * (1955.491e6 + 18.525e6 + 957.271e6 + 54.639e6),
-                     "src": "24bdbd71939c8d30", "chunks": 2},
+    # profiles/ffn_tcgen05_dsv3_prefill.md and profiles/ffn_mx_tcgen05_dsv3_prefill_mxfp8.md
+    "dsv3_prefill": {"bytes": 2 * 8 * (1955.436e6 + 18.376e6 + 957.506e6 + 54.893e6),
+                     "src": "a15a55f4109395c7", "chunks": 2},
+    "dsv3_prefill_mxfp8": {"bytes": 2 * 8 * (1008.788e6 + 11.774e6 + 494.242e6 + 50.586e6),
+                           "src": "32d5db20d0508550", "chunks": 2},
 }
 
 
