@@ -734,12 +734,39 @@ def dispatch_combine(alg, stage_ms, peaks, peak_src):
 
 # --------------------------------------------------------------------------- CPU oracle sample
 
-def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=None):
+def host_threads():
+    """The host cores this process may run on (its affinity set)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def oracle_rows(row_fn, rows_by_expert, threads):
+    """Runs the oracle's FFN row `row_fn(p, e)` for every (expert, rows) item, the
+    experts spread over `threads` host threads (the oracle's C calls release the
+    interpreter lock; each row writes only its own outputs)."""
+    import concurrent.futures as cf
+
+    def work(item):
+        e, ps = item
+        for p in ps:
+            row_fn(p, e)
+    items = [(e, ps) for e, ps in rows_by_expert.items() if ps]
+    if threads <= 1:
+        for it in items:
+            work(it)
+        return
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, items))
+
+
+def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=None, threads=1):
     """Times the oracle, as it stands, on a bounded sample: route + clip +
     layout + permute over all T tokens, then FFN + combine (+ the shared expert,
     `shared` = its host weights) for the rows of the first `sample_tokens`
-    tokens.  Returns (tokens/s extrapolated to the whole layer, seconds of CPU
-    work, description)."""
+    tokens, the FFN rows spread over `threads` host threads.  Returns (tokens/s
+    extrapolated to the whole layer, seconds of wall time, description)."""
     import numpy as np
     import oracle
     t0 = time.perf_counter()
@@ -765,14 +792,18 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
     N = lay["N"]
     y = np.zeros((max(N, 1), wl.H), x_np.dtype)
     ye = np.zeros((max(N, 1), wl.H), np.float64)
-    t1 = time.perf_counter()
-    for p, e in rows:
+    def row(p, e):
         if is_mx(wl):
             _, _, _, y[p], ye[p] = oracle.ffn_row_fp8_blocked(xrs[0][p], xs[lay["recv_token"][p]], *weights[e], 32)
         elif wl.ffn_fp8:
             _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xrs[0][p], xs[lay["recv_token"][p]], *weights[e])
         else:
             _, y[p], ye[p] = oracle.ffn_row(xrs[0][p], weights[e][0], weights[e][1])
+    by_expert = {}
+    for p, e in rows:
+        by_expert.setdefault(e, []).append(p)
+    t1 = time.perf_counter()
+    oracle_rows(row, by_expert, threads)
     sub_pos = lay["pos"][:sample_tokens]
     ys = None
     if shared is not None:
@@ -783,9 +814,9 @@ def oracle_sample(wl, logits, bias, x_np, fetch_expert, sample_tokens, shared=No
         oracle.combine(y, sub_pos, w, wl.T, y_shared=ys)
     t_ffn = time.perf_counter() - t1
     layer_s = t_index + t_ffn * (wl.T / sample_tokens)
-    desc = (f"oracle route+clip+layout+permute over all {wl.T} tokens ({t_index:.2f} s), FFN+combine "
-            f"for the {len(rows)} rows of the first {sample_tokens} tokens ({t_ffn:.2f} s), "
-            f"extrapolated linearly to {wl.T} tokens")
+    desc = (f"oracle route+clip+layout+permute over all {wl.T} tokens ({t_index:.2f} s, one thread), "
+            f"FFN+combine for the {len(rows)} rows of the first {sample_tokens} tokens ({t_ffn:.2f} s, "
+            f"rows in {threads} threads), extrapolated linearly to {wl.T} tokens")
     return wl.T / layer_s, t_index + t_ffn, desc
 
 
@@ -824,10 +855,11 @@ def reference_tokens(wl, seconds):
     return max(wl.ep, min(wl.T, n))
 
 
-def reference_step(wl, Ts, logits, bias, x_np, fetch):
+def reference_step(wl, Ts, logits, bias, x_np, fetch, threads=1):
     """The oracle's whole layer over the first Ts tokens of the workload, one chunk
-    (a capacity scales with the sub-batch: ceil(C * Ts / T)).  Expert weights are
-    fetched (untimed) between the index steps and the FFN.  Returns seconds."""
+    (a capacity scales with the sub-batch: ceil(C * Ts / T)), the FFN rows spread
+    over `threads` host threads.  Expert weights are fetched (untimed) between the
+    index steps and the FFN.  Returns seconds."""
     import numpy as np
     import oracle
     cap = wl.capacity if wl.capacity < 0 else -(-wl.capacity * Ts // wl.T)
@@ -850,15 +882,16 @@ def reference_step(wl, Ts, logits, bias, x_np, fetch):
     N = lay["N"]
     y = np.zeros((max(N, 1), wl.H), x_np.dtype)
     ye = np.zeros((max(N, 1), wl.H), np.float64)
+    def row(p, e):
+        wt = weights[e]
+        if is_mx(wl):
+            _, _, _, y[p], ye[p] = oracle.ffn_row_fp8_blocked(xr[p], xs[lay["recv_token"][p]], *wt, 32)
+        elif wl.ffn_fp8:
+            _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xr[p], xs[lay["recv_token"][p]], *wt)
+        else:
+            _, y[p], ye[p] = oracle.ffn_row(xr[p], wt[0], wt[1])
     t1 = time.perf_counter()
-    for e, wt in weights.items():
-        for p in range(int(eoff[e]), int(eoff[e + 1])):
-            if is_mx(wl):
-                _, _, _, y[p], ye[p] = oracle.ffn_row_fp8_blocked(xr[p], xs[lay["recv_token"][p]], *wt, 32)
-            elif wl.ffn_fp8:
-                _, _, _, y[p], ye[p] = oracle.ffn_row_fp8(xr[p], xs[lay["recv_token"][p]], *wt)
-            else:
-                _, y[p], ye[p] = oracle.ffn_row(xr[p], wt[0], wt[1])
+    oracle_rows(row, {e: range(int(eoff[e]), int(eoff[e + 1])) for e in weights}, threads)
     if wl.reduce_dense:
         oracle.combine_exact(ye, lay["pos"], w, Ts, x_np.dtype)
     else:
@@ -895,24 +928,25 @@ def run_reference(args):
     logits = inp.logits.numpy()
     bias = None if inp.bias is None else inp.bias.numpy()
     x_np = conv(inp.x)
-    Ts = reference_tokens(wl, 2.0)
+    threads = host_threads()
+    Ts = reference_tokens(wl, 2.0 * threads)
     secs = []
     for i in range(args.warmup + args.steps):
-        t = reference_step(wl, Ts, logits, bias, x_np, fetch)
+        t = reference_step(wl, Ts, logits, bias, x_np, fetch, threads)
         if i >= args.warmup:
             secs.append(t)
     step_s = statistics.mean(secs)
     value = Ts / step_s
     desc = (f"each step: the oracle's whole layer (route, clip, layout, permute, FFN, combine) over the "
-            f"first {Ts} of the {wl.T} tokens in one chunk, {step_s:.2f} s (timed without the untimed "
-            f"draw of the routed experts' weights)")
+            f"first {Ts} of the {wl.T} tokens in one chunk, the FFN rows in {threads} threads, "
+            f"{step_s:.2f} s (timed without the untimed draw of the routed experts' weights)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -1129,12 +1163,13 @@ def run_ours(args):
             if wl.dtype == "bf16" else (lambda t: t.detach().cpu().numpy().copy())
         fetch = (lambda e: fp8_expert(conv(inp.w13[e]), conv(inp.w2[e]), is_mx(wl))) if wl.ffn_fp8 else \
             (lambda e: (conv(inp.w13[e]), conv(inp.w2[e])))
-        s_tok = sample_tokens_for(wl, 15.0)
+        threads = host_threads()
+        s_tok = sample_tokens_for(wl, 15.0 * threads)
         shared = None if inp.w13s is None else (conv(inp.w13s), conv(inp.w2s))
         v, secs, desc = oracle_sample(wl, inp.logits.cpu().numpy(),
                                       None if inp.bias is None else inp.bias.cpu().numpy(),
-                                      conv(inp.x), fetch, s_tok, shared)
-        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                                      conv(inp.x), fetch, s_tok, shared, threads)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "cpu_seconds": round(secs, 2)}
 
     if rank == 0:

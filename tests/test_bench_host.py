@@ -86,3 +86,21 @@ def test_block_scaled_fp8_counts():
     # one byte per weight plus a scale byte per 32; h's codes and scales written and read
     assert a["ffn_bytes"] == 2 * 256 * 3 * H * I * 33 // 32 + N * H * 33 // 32 + 2 * N * I * 33 // 32 + N * H * 2
     assert a["permute_bytes"] == 8192 * H * 2 + N * H * 33 // 32
+
+
+def test_oracle_rows_visits_every_row_once_in_threads():
+    """The CPU baseline's threaded runner calls the row function once per row,
+    whatever the thread count, and only with the row's own expert."""
+    import threading
+    rows_by_expert = {e: list(range(10 * e, 10 * e + e % 4)) for e in range(32)}
+    for threads in (1, 3, 8):
+        seen = []
+        lock = threading.Lock()
+
+        def row(p, e):
+            with lock:
+                seen.append((p, e))
+        bench.oracle_rows(row, rows_by_expert, threads)
+        want = sorted((p, e) for e, ps in rows_by_expert.items() for p in ps)
+        assert sorted(seen) == want
+    assert bench.host_threads() >= 1
