@@ -65,6 +65,7 @@ constexpr int kMxRows = 128;                                  // weight rows per
 constexpr int kMxTileTok = 224;                               // tokens per tile (MMA N <= 224)
 constexpr int kMxBoxTok = kMxTileTok / 2;                     // token rows per CTA box
 constexpr int kMxSmallBox = 32;                               // token box of tiles with N <= 64
+constexpr int kMxMidBox = 64;                                 // token box of tiles with N <= 128
 constexpr int kMxKS = 2;                                      // 128-value k-chunks per ring stage
 constexpr uint32_t kMxWChunk = kMxRows * 128;                 // 16 KiB of weight rows per k-chunk
 constexpr uint32_t kMxTChunk = kMxBoxTok * 128;               // 14 KiB of token rows per k-chunk
@@ -77,7 +78,9 @@ constexpr uint32_t kMxRingBytes = kMxStages * kMxStageBytes;
 static_assert(kMxStageBytes % 1024 == 0 && kMxTOff % 1024 == 0 && kMxTChunk % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 // scale slot of one stage: [SFA c0 | SFA c1 | SFB c0 a0 | c0 a1 | c1 a0 | c1 a1]
-constexpr uint32_t kMxSfSlotBytes = 6 * kMxAtom;
+constexpr int kMxSfAtoms = 3 * kMxKS;                         // per stage: one weight atom and two token atoms per k-chunk
+constexpr uint32_t kMxSfSlotBytes = kMxSfAtoms * kMxAtom;
+constexpr uint32_t kMxSfCols = 4 * kMxSfAtoms;                 // TMEM columns of one scale slot
 constexpr int kMxSfStages = 6;
 constexpr uint32_t kMxSfRingBytes = kMxSfStages * kMxSfSlotBytes;
 constexpr int kMxEpiWarps = 8;
@@ -85,8 +88,8 @@ constexpr int kMxProdWarp = kMxEpiWarps, kMxMmaWarp = kMxEpiWarps + 1, kMxSfWarp
 constexpr int kMxThreads = 32 * (kMxEpiWarps + 3);
 constexpr uint32_t kMxTmemCols = 512;
 constexpr uint32_t kMxAccStride = 256;                        // accumulator a at column 256 a
-constexpr uint32_t kMxSfCol = kMxTileTok;                    // scale slot a at kMxSfCol + 256 a (24 columns)
-static_assert(kMxAccStride + kMxTileTok + 24 <= kMxTmemCols, "scale columns exceed TMEM");
+constexpr uint32_t kMxSfCol = kMxTileTok;                    // scale slot a at kMxSfCol + 256 a
+static_assert(kMxAccStride + kMxTileTok + kMxSfCols <= kMxTmemCols, "scale columns exceed TMEM");
 constexpr uint32_t kMxXchgBytes = 16 * 1024;                  // GEMM1 gate / up exchange
 constexpr int kMxMaxExperts = 512;
 
@@ -136,6 +139,11 @@ struct MxTile {
     int e, f_blk, p0, n_valid, n_mma;   // n_valid <= 224 tokens; n_mma: the MMA's N (rounded to 16)
 };
 
+// Rows of the token box a CTA loads for a tile of n_mma tokens (it reads n_mma / 2).
+__device__ __forceinline__ int mx_token_box(int n_mma) {
+    return n_mma / 2 <= kMxSmallBox ? kMxSmallBox : n_mma / 2 <= kMxMidBox ? kMxMidBox : kMxBoxTok;
+}
+
 __device__ __forceinline__ MxTile mx_tile_info(int e, int f_blk, int t_blk, const MxParams &P) {
     MxTile t;
     t.e = e;
@@ -168,7 +176,8 @@ __device__ __forceinline__ float mx_pow2_neg(int e) {
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_mx_tcgen05_kernel(
     const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_t,
-    const __grid_constant__ CUtensorMap tmap_ts, const MxParams P, uint32_t *__restrict__ work_counter) {
+    const __grid_constant__ CUtensorMap tmap_tm, const __grid_constant__ CUtensorMap tmap_ts,
+    const MxParams P, uint32_t *__restrict__ work_counter) {
     constexpr bool kG1 = MODE == kMxSwiGLUQuant;
     // queue consumers per entry: the leader's MMA thread and operand producer, the
     // follower's operand producer, scale gatherer and forwarder, and every epilogue
@@ -230,6 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
     if (warp == kMxProdWarp && lane == 0) {
         tma_prefetch_desc(&tmap_w);
         tma_prefetch_desc(&tmap_t);
+        tma_prefetch_desc(&tmap_tm);
         tma_prefetch_desc(&tmap_ts);
     }
     if (warp == kMxMmaWarp) { tmem_alloc_pair(&S->tmem_base, kMxTmemCols); tmem_relinquish_pair(); }
@@ -262,8 +272,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                 // this CTA's weight rows and its half of the tile's tokens
                 const int f0 = (sfb * 2 + (int)rank) * P.feat_per_cta;
                 const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
-                const bool small_box = ti.n_mma / 2 <= kMxSmallBox;
-                const uint32_t stage_tx = kMxKS * (kMxWChunk + (small_box ? kMxSmallBox : kMxBoxTok) * 128);
+                // the smallest token box that holds this CTA's n_mma / 2 rows: fewer bytes
+                // through L2 for the same stage slot
+                const int box = mx_token_box(ti.n_mma);
+                const CUtensorMap *tmap_tok = box == kMxSmallBox ? &tmap_ts : box == kMxMidBox ? &tmap_tm : &tmap_t;
+                const uint32_t stage_tx = kMxKS * (kMxWChunk + (uint32_t)box * 128);
                 for (int kb = 0; kb < num_k; ++kb) {
                     if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
                     unsigned char *st = ring + stage * kMxStageBytes;
@@ -274,7 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                         tma_load_4d_pair(st, &tmap_w, full_leader, 0, f0, 2 * se, ch);
                     else
                         tma_load_3d_pair(st, &tmap_w, full_leader, 0, se * P.w_rows_per_expert + f0, ch);
-                    tma_load_3d_pair(st + kMxTOff, small_box ? &tmap_ts : &tmap_t, full_leader, 0, tok_row, ch);
+                    tma_load_3d_pair(st + kMxTOff, tmap_tok, full_leader, 0, tok_row, ch);
                     ++issued;
                     if (++stage == kMxStages) { stage = 0; phase ^= 1u; }
                 }
@@ -370,7 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const bool ok_t = in_k && trow[i] >= 0;
-                        cp_async_4(sfs + (2 + 2 * c + (i >> 2)) * kMxAtom + 4 * (i & 3),
+                        cp_async_4(sfs + (kMxKS + 2 * c + (i >> 2)) * kMxAtom + 4 * (i & 3),
                                    ok_t ? P.t_sf + trow[i] * kwords + ch + c : P.t_sf, ok_t ? 4u : 0u);
                     }
                 }
@@ -405,8 +418,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d = tmem_base + (uint32_t)acc * kMxAccStride;
-                    // k-chunk stride inside the stage's token box (32 or 112 rows)
-                    const uint32_t tchunk = ti.n_mma / 2 <= kMxSmallBox ? kMxSmallBox * 128 : kMxTChunk;
+                    // k-chunk stride inside the stage's token box (32, 64 or 112 rows)
+                    const uint32_t tchunk = (uint32_t)mx_token_box(ti.n_mma) * 128;
                     for (int kb = 0; kb < num_k; ++kb) {
                         // the stage's scales: both CTAs' atoms into TMEM, then the slot is free
                         if (!mbar_wait_bounded(&S->sf_full[sstage], sphase, abort_flag)) { ok = false; break; }
@@ -416,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                         const uint32_t tsf = tmem_base + kMxSfCol + kMxAccStride * slot;
                         // weight-row scales of chunk c at tsf + 4c, token scales at tsf + 8 + 8c
 #pragma unroll
-                        for (int a = 0; a < 6; ++a)
+                        for (int a = 0; a < kMxSfAtoms; ++a)
                             tc_cp_sf_atom_pair(tsf + 4 * a, make_sf_atom_desc(sf + a * kMxAtom));
                         tc_commit_pair_mc(&S->sf_empty[sstage], 0x3);
                         if (++sstage == kMxSfStages) { sstage = 0; sphase ^= 1u; }
@@ -432,7 +445,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxThreads, 1) ffn_m
                                 const uint64_t td = make_sw128_desc(st + kMxTOff + c * tchunk + kk * 32);
                                 const uint32_t sel = (uint32_t)kk << 30;
                                 tc_mma_mx_pair(d, wd, td, make_idesc_mx_e4m3(2 * kMxRows, ti.n_mma, kk),
-                                               (tsf + 4 * c) | sel, (tsf + 8 + 8 * c) | sel,
+                                               (tsf + 4 * c) | sel, (tsf + 4 * kMxKS + 8 * c) | sel,
                                                (kb > 0 || c > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
@@ -665,13 +678,14 @@ size_t ffn_mx_smem(int E, bool g1) {
 }
 
 template <int MODE>
-static cudaError_t launch_mx(const CUtensorMap &tw, const CUtensorMap &tt, const CUtensorMap &tts,
-                             const MxParams &P, int grid, uint32_t *counter, cudaStream_t s) {
+static cudaError_t launch_mx(const CUtensorMap &tw, const CUtensorMap &tt, const CUtensorMap &ttm,
+                             const CUtensorMap &tts, const MxParams &P, int grid, uint32_t *counter,
+                             cudaStream_t s) {
     const size_t smem = ffn_mx_smem(P.E, MODE == kMxSwiGLUQuant);
     static SmemOptIn opt_in;   // one per kernel instantiation
     cudaError_t err = opt_in.ensure(ffn_mx_tcgen05_kernel<MODE>, smem);
     if (err != cudaSuccess) return err;
-    ffn_mx_tcgen05_kernel<MODE><<<grid, kMxThreads, smem, s>>>(tw, tt, tts, P, counter);
+    ffn_mx_tcgen05_kernel<MODE><<<grid, kMxThreads, smem, s>>>(tw, tt, ttm, tts, P, counter);
     return cudaGetLastError();
 }
 
@@ -697,9 +711,10 @@ cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr
     cudaError_t cerr = cudaMemsetAsync(counters, 0, 2 * sizeof(uint32_t), s);
     if (cerr != cudaSuccess) return cerr;
     const uint64_t n = (uint64_t)n_rows;
-    CUtensorMap tw1, tx, txs, tw2, th, ths;
+    CUtensorMap tw1, tx, txm, txs, tw2, th, thm, ths;
     if (!mx_tmap_w13(&tw1, w13_q, c.E, c.I, c.H) || !mx_tmap_rows(&tx, xr_q, n, c.H, kMxBoxTok) ||
-        !mx_tmap_rows(&txs, xr_q, n, c.H, kMxSmallBox) ||
+        !mx_tmap_rows(&txs, xr_q, n, c.H, kMxSmallBox) || !mx_tmap_rows(&txm, xr_q, n, c.H, kMxMidBox) ||
+        !mx_tmap_rows(&thm, h_q, n, c.I, kMxMidBox) ||
         !mx_tmap_rows(&tw2, w2_q, (uint64_t)c.E * c.H, c.I, kMxRows) ||
         !mx_tmap_rows(&th, h_q, n, c.I, kMxBoxTok) || !mx_tmap_rows(&ths, h_q, n, c.I, kMxSmallBox))
         return cudaErrorNotSupported;
@@ -722,7 +737,7 @@ cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr
     P1.t_sf = reinterpret_cast<const uint32_t *>(xr_sf);
     P1.h_q = h_q;
     P1.h_sf = h_sf;
-    cudaError_t err = launch_mx<kMxSwiGLUQuant>(tw1, tx, txs, P1, mx_grid(c, n_rows, P1, num_sms), counters, s);
+    cudaError_t err = launch_mx<kMxSwiGLUQuant>(tw1, tx, txm, txs, P1, mx_grid(c, n_rows, P1, num_sms), counters, s);
     if (err != cudaSuccess) return err;
     MxParams P2 = P;
     P2.K = c.I;
@@ -735,8 +750,8 @@ cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr
     P2.y = static_cast<__nv_bfloat16 *>(y);
     P2.out_reduce = out_reduce;
     const int grid2 = mx_grid(c, n_rows, P2, num_sms);
-    if (c.reduce_dense) return launch_mx<kMxReduce>(tw2, th, ths, P2, grid2, counters + 1, s);
-    return launch_mx<kMxStore>(tw2, th, ths, P2, grid2, counters + 1, s);
+    if (c.reduce_dense) return launch_mx<kMxReduce>(tw2, th, thm, ths, P2, grid2, counters + 1, s);
+    return launch_mx<kMxStore>(tw2, th, thm, ths, P2, grid2, counters + 1, s);
 }
 
 }  // namespace moe
