@@ -57,6 +57,9 @@ cudaError_t launch_ffn_mx(const moe_config &c, int64_t n_rows, const uint8_t *xr
                           const int32_t *recv_token, const int32_t *recv_slot, const float *topk_w,
                           float *out_reduce, uint32_t *status, uint32_t *counters, cudaStream_t s,
                           int num_sms);
+cudaError_t launch_ep_regroup(int n_src, int n_exp, const int32_t *counts, const void *in, void *out,
+                              int64_t rows, int row_bytes, int inverse, int32_t *expert_offsets, uint32_t *status,
+                              cudaStream_t s, int num_sms);
 cudaError_t launch_combine_bwd(const moe_config &c, const void *dout, const void *y,
                                const int32_t *pos, const float *topk_w, int tb, int tc, void *dy,
                                float *dw, cudaStream_t s);
@@ -1258,6 +1261,35 @@ moe_status moe_watchdog_selftest(const moe_config *cfg, int32_t which, int32_t l
                                                    ws_at<uint32_t>(ws, L.status));
     cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_watchdog_selftest");
+}
+
+moe_status moe_ep_regroup(const moe_config *cfg, const int32_t *counts, const void *in, void *out,
+                          int64_t rows, int32_t inverse, int32_t *expert_offsets, void *ws,
+                          cudaStream_t stream) {
+    moe_status st = moe_config_check(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ws(ws)) != MOE_OK) return st;
+    const moe_config &c = *cfg;
+    if (c.ffn_fp8) return fail(MOE_ERR_UNSUPPORTED, "the EP regroup moves bf16 / fp32 rows (ffn_fp8 = 0)");
+    if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows < 0");
+    if (inverse != 0 && inverse != 1) return fail(MOE_ERR_INVALID_ARG, "inverse must be 0 or 1");
+    if (rows == 0) {
+        if (expert_offsets) {
+            cudaError_t err = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (size_t)(c.E / c.ep + 1), stream);
+            if (err != cudaSuccess) return cuda_fail(err, "moe_ep_regroup");
+        }
+        return MOE_OK;
+    }
+    if (!counts || !in || !out) return fail(MOE_ERR_INVALID_ARG, "NULL pointer argument");
+    if (in == out) return fail(MOE_ERR_INVALID_ARG, "in and out must not be the same buffer");
+    const int row_bytes = c.H * (c.dtype == MOE_F32 ? 4 : 2);
+    if (row_bytes % 16 != 0) return fail(MOE_ERR_UNSUPPORTED, "rows of %d bytes: a multiple of 16 is needed", row_bytes);
+    if (!aligned(in, 16) || !aligned(out, 16)) return fail(MOE_ERR_INVALID_ARG, "in / out not 16-byte aligned");
+    if (!aligned(counts, 4)) return fail(MOE_ERR_INVALID_ARG, "counts not 4-byte aligned");
+    const ScratchLayout L = scratch_layout(c);
+    cudaError_t err = launch_ep_regroup(c.ep, c.E / c.ep, counts, in, out, rows, row_bytes, inverse,
+                                        expert_offsets, ws_at<uint32_t>(ws, L.status), stream, current_num_sms());
+    return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ep_regroup");
 }
 
 moe_status moe_device_status(void *ws, uint32_t *flags, cudaStream_t stream) {

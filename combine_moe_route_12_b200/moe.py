@@ -85,6 +85,7 @@ _decl("moe_combine_backward", _I32, _CFG, _P, _P, _P, _P, _I32, _I32, _P, _P, _P
 _decl("moe_route_backward", _I32, _CFG, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute_backward", _I32, _CFG, _P, _P, _I32, _I32, _P, _P)
 _decl("moe_watchdog_selftest", _I32, _CFG, _I32, _I32, _P, _P)
+_decl("moe_ep_regroup", _I32, _CFG, _P, _P, _P, ctypes.c_int64, ctypes.c_int32, _P, _P, _P)
 _decl("moe_device_status", _I32, _P, ctypes.POINTER(ctypes.c_uint32), _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_last_error_detail", ctypes.c_char_p)
@@ -386,6 +387,14 @@ def moe_watchdog_selftest(cfg, which: int, limit_us: int, ws, stream=None):
     """Runs one of the library's bounded waits on something that never completes
     (0: the look-back spin, 1: an mbarrier wait); it sets MOE_DEV_WAIT_TIMEOUT."""
     _check(_lib.moe_watchdog_selftest(ctypes.byref(cfg), which, limit_us, _ptr(ws), _stream(stream)))
+
+
+def moe_ep_regroup(cfg, counts, inp, out, rows, inverse, ws, expert_offsets=None, stream=None):
+    """Source-major receive rows -> expert-major (inverse = 0), or back (1); see
+    include/moe_b200.h.  counts: device int32 [ep, E // ep]; expert_offsets: the
+    expert-major buffer's local expert offsets [E // ep + 1] (written when given)."""
+    _check(_lib.moe_ep_regroup(ctypes.byref(cfg), _ptr(counts), _ptr(inp), _ptr(out), ctypes.c_int64(rows),
+                               ctypes.c_int32(int(inverse)), _ptr(expert_offsets), _ptr(ws), _stream(stream)))
 
 
 def moe_device_status(ws, stream=None) -> int:

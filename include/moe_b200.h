@@ -654,6 +654,35 @@ moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
 moe_status moe_watchdog_selftest(const moe_config *cfg, int32_t which, int32_t limit_us,
                                  void *ws, cudaStream_t stream);
 
+/* Expert-parallel exchange, receive side: regroup the rows one rank received from
+ * the other ranks of its EP group (axolotl docs, integrations.expert_parallel.args:
+ * expert_parallel_backend = torch, all_to_all_single over the EP group).
+ *
+ * With experts owned by contiguous blocks of E / ep per rank and tokens by
+ * contiguous blocks per source rank, a rank that sent each destination the rows of
+ * that destination's experts in its own (expert, token) order (rows
+ * [rank_offsets[d], rank_offsets[d+1]) of moe_dispatch_layout, permuted by
+ * moe_permute) receives, after a variable all-to-all, cells (s, e) - the rows
+ * source rank s sent for this rank's local expert e - source after source, each
+ * source's cells in expert order.  The grouped FFN wants them expert after expert;
+ * (expert, source, token) is then the (expert, token) order of the whole group.
+ *
+ *   inverse = 0: in  source-major (rows [src_off(s, e), +counts[s][e]) per cell),
+ *                out expert-major (expert e's rows from sources 0, 1, ... in turn);
+ *   inverse = 1: in  expert-major (the FFN's outputs), out source-major (for the
+ *                reverse all-to-all).
+ * counts: device int32 [ep][E / ep], counts[s][e] = rows of cell (s, e); their sum
+ * must be `rows` (else MOE_DEV_BAD_INDEX is set in ws's status word and nothing is
+ * read or written past `rows`).  in, out: [rows, H] in the layer dtype (bf16 or
+ * fp32; cfg->ffn_fp8 = 0), 16-byte aligned, distinct.  expert_offsets (device
+ * int32 [E / ep + 1], or NULL): written with the expert-major buffer's offsets of
+ * each local expert (the grouped FFN's expert_offsets for these rows; all zero when
+ * rows = 0).  cfg: ep = the EP group's size, E its experts.
+ * ws: moe_workspace_bytes(cfg). */
+moe_status moe_ep_regroup(const moe_config *cfg, const int32_t *counts, const void *in, void *out,
+                          int64_t rows, int32_t inverse, int32_t *expert_offsets, void *ws,
+                          cudaStream_t stream);
+
 /* Synchronises `stream`, copies the device status word of ws to *flags and
  * clears it.  Returns MOE_ERR_DEVICE if any bit was set. */
 moe_status moe_device_status(void *ws, uint32_t *flags, cudaStream_t stream);
