@@ -30,8 +30,9 @@
 // (TMEM lanes i and 64 + i); in GEMM2 128 output features.
 //
 // Roles (11 warps per CTA).  Warp 8 (one lane) of each CTA streams its ring
-// stages (two k-chunks: 32 KiB of weight rows and 28 KiB of token rows by TMA,
-// counted on the leader's barrier).  Warp 10 gathers, with all its lanes, the
+// stages (two k-chunks: 32 KiB of weight rows and up to 28 KiB of token rows by
+// TMA - a 112-row token box, or 64 or 32 rows for tiles of at most 128 or 64
+// tokens - counted on the leader's barrier).  Warp 10 gathers, with all its lanes, the
 // scale words of the same stages into a separate, deeper ring of 3 KiB slots:
 // 4-byte cp.async copies into 512-byte scale atoms (row r's word at byte
 // 16 (r % 32) + 4 (r / 32), the layout tcgen05.cp spreads over the four TMEM
