@@ -234,7 +234,8 @@ class ClockSampler:
 # --------------------------------------------------------------------------- workload
 
 def kernels_per_step(wl) -> int:
-    # route 1; clip 2 (prep, mark) or 4 with a binding capacity (+ gather, select);
+    # route 1; clip 1 without a capacity (one pass), 2 with capacity 0 (prep, mark),
+    # 4 with a positive capacity (+ gather, select);
     # per chunk: layout 2 (hist, scatter), permute 1, FFN 2 (two GEMM launches),
     # combine or finalize 1
     # with a shared expert, per chunk 3 more (its offsets and two GEMM launches);
@@ -242,7 +243,7 @@ def kernels_per_step(wl) -> int:
     # quantisation is not fused into the permute (H > 8192)
     # with the block-scaled FP8 FFN (ffn_fp8 = 2) nothing more: x is quantised inside
     # the permute and h inside GEMM1
-    clip = 4 if wl.capacity > 0 else 2
+    clip = 4 if wl.capacity > 0 else 2 if wl.capacity == 0 else 1
     fp8 = 0 if is_mx(wl) else (1 if fused_permute_quant(wl) else 2) if wl.ffn_fp8 else 0
     return 1 + clip + wl.n_chunks * (6 + (3 if wl.shared_I > 0 else 0) + fp8)
 
@@ -670,6 +671,47 @@ def breakdown(moe, wl, cfg, inp, B, fp8, steps, flush, use_graph):
     return stage_ms, disp_ms, step_sum, mode
 
 
+def index_path_ms(moe, wl, cfg, inp, B, steps, flush):
+    """The index path (route, clip and the first chunk's dispatch layout) as one
+    CUDA graph with no events inside, replayed `steps` times with the L2 flushed
+    before each: milliseconds per replay, or None if capture fails.  The
+    per-stage breakdown's events sit between graph nodes and add their own
+    cost to every stage."""
+    import torch
+
+    def path():
+        moe.moe_route_topk(cfg, inp.logits, inp.bias, B.topk_idx, B.topk_w, B.counts, B.ws)
+        moe.moe_capacity_clip(cfg, B.topk_idx, B.topk_w, B.counts, B.keep, B.kept, B.ws)
+        moe.moe_dispatch_layout(cfg, 0, B.tc, B.topk_idx, B.keep, B.eoff, B.roff, B.rt, B.rs, B.pos, B.spl,
+                                None, B.ws)
+
+    path()
+    torch.cuda.synchronize()
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            path()
+        torch.cuda.synchronize()
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+    for _ in range(3):
+        g.replay()
+    total = 0.0
+    for _ in range(steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    del g
+    if moe.moe_device_status(B.ws) != 0:
+        raise RuntimeError("device status bits set during the index path timing")
+    return total / steps
+
+
 def layout_counts(moe, wl, cfg, B):
     """Kept rows and active experts of each chunk, and the tokens with a kept slot."""
     n_kept, n_active = [], []
@@ -1088,6 +1130,7 @@ def run_ours(args):
     # ---------------- per-stage breakdown: the same kernels through the step ABI
     stage_ms, disp_ms, eager_step_ms, breakdown_mode = breakdown(
         moe, wl, cfg, inp, B, fp8, args.steps, flush, use_graph)
+    idx_ms = index_path_ms(moe, wl, cfg, inp, B, args.steps, flush) if use_graph else None
     n_kept, n_active, tokens_read = layout_counts(moe, wl, cfg, B)
     alg = algorithmic(wl, n_kept, n_active, tokens_read)
     bwd = backward_row_passes(moe, wl, cfg, B, n_kept[-1], peaks, flush, args) \
@@ -1193,6 +1236,10 @@ def run_ours(args):
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "breakdown_step_ms": round(eager_step_ms, 4),
             "breakdown_mode": breakdown_mode,
+            "index_path": None if idx_ms is None else {
+                "ms": round(idx_ms, 4),
+                "what": "route + clip + the first chunk's dispatch layout as one CUDA graph (no events "
+                        "inside), L2 flushed before each replay"},
             "kept_rows": alg["N"],
             "e2e": e2e,
             "cpu_baseline": cpu,

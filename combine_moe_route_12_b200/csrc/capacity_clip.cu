@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(1024) clip_prep_kernel(int E, int C, const int
                                                          int32_t *__restrict__ seg,  // [2][E+1]: offsets, cursors
                                                          int32_t *__restrict__ kept_counts,
                                                          uint64_t *__restrict__ thr) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_v[1025];
     __shared__ int32_t s_w[33];
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -150,6 +152,8 @@ __global__ void __launch_bounds__(kGatherThreads) clip_gather_kernel(
     int T, int E, int k, int C, const int32_t *__restrict__ topk_idx,
     const float *__restrict__ topk_w, const int32_t *__restrict__ counts,
     int32_t *__restrict__ seg, uint64_t *__restrict__ keys) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ int32_t s_cnt[];   // [E] this CTA's keys per expert, then its base
     const size_t total = (size_t)T * k;
     const size_t a0 = (size_t)blockIdx.x * kGatherThreads * kGatherPerThread;
@@ -211,6 +215,8 @@ __global__ void __launch_bounds__(kGatherThreads) clip_gather_kernel(
 __global__ void __launch_bounds__(kClipThreads) clip_select_kernel(
     int E, int C, int smem_keys, long long total_keys, const int32_t *__restrict__ counts,
     const int32_t *__restrict__ seg, const uint64_t *__restrict__ keys, uint64_t *__restrict__ thr) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ __align__(16) unsigned char s_raw[];
     __shared__ uint32_t s_hist[256];
     __shared__ uint32_t s_sel[3];
@@ -257,6 +263,8 @@ __global__ void clip_mark_kernel(int T, int E, int k, const int32_t *__restrict_
                                  const float *__restrict__ topk_w,
                                  const uint64_t *__restrict__ thr, uint8_t *__restrict__ keep,
                                  uint32_t *__restrict__ status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const size_t total = (size_t)T * k;
     bool bad = false;
     for (size_t a = (size_t)blockIdx.x * blockDim.x + threadIdx.x; a < total;
@@ -275,6 +283,8 @@ __global__ void clip_mark_kernel(int T, int E, int k, const int32_t *__restrict_
 __global__ void clip_all_kernel(int T, int E, int k, const int32_t *__restrict__ topk_idx,
                                 const int32_t *__restrict__ counts, uint8_t *__restrict__ keep,
                                 int32_t *__restrict__ kept_counts, uint32_t *__restrict__ status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     if (blockIdx.x == 0)
         for (int e = threadIdx.x; e < E; e += blockDim.x) kept_counts[e] = counts[e];
     const size_t total = (size_t)T * k;
@@ -298,33 +308,31 @@ cudaError_t launch_capacity_clip(const moe_config &c, const int32_t *topk_idx,
         int blocks = (int)((total + 255) / 256);
         if (blocks > num_sms * 16) blocks = num_sms * 16;
         if (blocks < 1) blocks = 1;
-        clip_all_kernel<<<blocks, 256, 0, s>>>(c.T, c.E, c.k, topk_idx, counts, keep, kept_counts, status);
-        return cudaGetLastError();
+        return launch_dependent(clip_all_kernel, blocks, 256, 0, s, c.T, c.E, c.k, topk_idx, counts, keep,
+                                kept_counts, status);
     }
-    clip_prep_kernel<<<1, 1024, 0, s>>>(c.E, c.capacity, counts, seg, kept_counts, thr);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_dependent(clip_prep_kernel, 1, 1024, 0, s, c.E, c.capacity, counts, seg, kept_counts, thr);
     if (err != cudaSuccess) return err;
     const size_t total = (size_t)c.T * c.k;
     if (total == 0) return cudaSuccess;
     if (c.capacity > 0) {
         const int per_block = kGatherThreads * kGatherPerThread;
         const int gblocks = (int)((total + per_block - 1) / per_block);
-        clip_gather_kernel<<<gblocks, kGatherThreads, sizeof(int32_t) * c.E, s>>>(
-            c.T, c.E, c.k, c.capacity, topk_idx, topk_w, counts, seg, keys);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        err = launch_dependent(clip_gather_kernel, gblocks, kGatherThreads, sizeof(int32_t) * c.E, s,
+                               c.T, c.E, c.k, c.capacity, topk_idx, topk_w, counts, seg, keys);
+        if (err != cudaSuccess) return err;
         int smem_keys = c.T < kClipMaxSmemKeys ? c.T : kClipMaxSmemKeys;
         if (smem_keys < 1) smem_keys = 1;
         const size_t smem = sizeof(uint64_t) * (size_t)smem_keys;
         static SmemOptIn opt_in;
         if ((err = opt_in.ensure(clip_select_kernel, smem)) != cudaSuccess) return err;
-        clip_select_kernel<<<c.E, kClipThreads, smem, s>>>(c.E, c.capacity, smem_keys, (long long)total,
-                                                           counts, seg, keys, thr);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        err = launch_dependent(clip_select_kernel, c.E, kClipThreads, smem, s, c.E, c.capacity, smem_keys,
+                               (long long)total, counts, seg, keys, thr);
+        if (err != cudaSuccess) return err;
     }
     int blocks = (int)((total + 255) / 256);
     if (blocks > num_sms * 16) blocks = num_sms * 16;
-    clip_mark_kernel<<<blocks, 256, 0, s>>>(c.T, c.E, c.k, topk_idx, topk_w, thr, keep, status);
-    return cudaGetLastError();
+    return launch_dependent(clip_mark_kernel, blocks, 256, 0, s, c.T, c.E, c.k, topk_idx, topk_w, thr, keep, status);
 }
 
 }  // namespace moe

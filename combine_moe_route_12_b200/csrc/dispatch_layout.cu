@@ -6,26 +6,27 @@
 // stable order by (expert, token).  With experts owned by contiguous rank
 // blocks this is also the (destination rank, expert, token) order, i.e. the
 // all_to_all_single arrival order regrouped by expert.  The order is built by
-// a stable counting sort:
+// a stable counting sort over tiles of 64, 128 or 256 tokens (the smallest
+// that keeps the launch within max(64, tokens / 256) tiles):
 //
-//   layout_hist     per-expert kept counts of the chunk (shared-memory
-//                   histogram, one global atomic per CTA and expert);
-//   layout_scatter  one CTA per tile of 64, 128 or 256 tokens (the smallest that
-//                   keeps the launch within max(64, tokens / 256) tiles), taken in launch order
-//                   from an atomic ticket.  Each tile ranks its assignments
-//                   per expert in token order (warps walk their tokens with
-//                   __match_any_sync), publishes its per-expert counts, and
-//                   finds its prefix over earlier tiles by a decoupled
-//                   look-back (Merrill & Garland 2016), one expert per thread.
-//                   The row of (t, j) is expert_offsets[e] + (rows of e in
-//                   earlier tiles) + (rank of t among this tile's rows of e).
-//                   While scattering, each tile also counts its rows by
-//                   (source rank, destination rank): the EP x EP
-//                   all_to_all_single split matrix.
+//   layout_hist     one CTA per tile: the tile's kept assignments per expert
+//                   (shared-memory histogram), written column by column to
+//                   tile_counts[expert][tile], zeros included;
+//   layout_scatter  one CTA per tile.  Each warp sums one expert's column of
+//                   tile_counts at a time (lanes over tiles, two warp
+//                   reductions): the expert's rows in the tiles before this one
+//                   and in the whole chunk; a block scan of the totals gives the
+//                   expert offsets.  The tile ranks its assignments per expert in
+//                   token order (warps walk their tokens with __match_any_sync);
+//                   the row of (t, j) is expert_offsets[e] + (rows of e in earlier
+//                   tiles) + (rank of t among this tile's rows of e).  While
+//                   scattering, each tile also counts its rows by (source rank,
+//                   destination rank): the EP x EP all_to_all_single split matrix.
 //
-// The look-back waits are bounded: on a timeout the tile raises
-// MOE_DEV_WAIT_TIMEOUT, publishes what it has so that later tiles finish,
-// and skips every write that would leave the receive buffers.
+// No CTA waits for another: the first kernel's histograms are complete when the
+// second starts, and every scatter CTA reads them all (n_tiles x E counts, from
+// L2).  Rows outside the receive buffer, and expert ids outside [0, E) of kept
+// assignments, raise MOE_DEV_BAD_INDEX and are not written.
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -35,28 +36,25 @@ namespace moe {
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kLoadBatch = 8;              // warp steps whose loads are issued together
-constexpr uint32_t kFlagAggregate = 1u << 30;
-constexpr uint32_t kFlagInclusive = 2u << 30;
-constexpr uint32_t kValueMask = (1u << 30) - 1;
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_hist_kernel(
-    int tb, int tc, int k, int E, int ep, const int32_t *__restrict__ topk_idx,
-    const uint8_t *__restrict__ keep, int32_t *__restrict__ chunk_counts,
-    int32_t *__restrict__ send_splits) {
+    int tb, int tc, int k, int E, int ep, int tile_tokens, int n_tiles, const int32_t *__restrict__ topk_idx,
+    const uint8_t *__restrict__ keep, int32_t *__restrict__ tile_counts, int32_t *__restrict__ send_splits) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ int32_t s_hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
     if (blockIdx.x == 0)   // the scatter kernel accumulates the split matrix into zeros
         for (int i = threadIdx.x; i < ep * ep; i += blockDim.x) send_splits[i] = 0;
     __syncthreads();
-    const size_t a0 = (size_t)tb * k, a1 = (size_t)(tb + tc) * k;
-    for (size_t a = a0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; a < a1;
-         a += (size_t)gridDim.x * blockDim.x) {
+    const int t0 = tb + blockIdx.x * tile_tokens;
+    const int t1 = min(tb + tc, t0 + tile_tokens);
+    for (size_t a = (size_t)t0 * k + threadIdx.x; a < (size_t)t1 * k; a += blockDim.x) {
         const int e = keep[a] ? topk_idx[a] : -1;
         if (e >= 0 && e < E) atomicAdd(&s_hist[e], 1);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        if (s_hist[e]) atomicAdd(&chunk_counts[e], s_hist[e]);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) tile_counts[(size_t)e * n_tiles + blockIdx.x] = s_hist[e];
 }
 
 // Exclusive scan of s[0..n) in place (n <= 4 * blockDim.x); returns the total.
@@ -101,52 +99,17 @@ __device__ int block_exclusive_scan(int32_t *s, int n, int32_t *s_warp_tot) {
 
 // The split matrix is accumulated in shared memory when it fits.
 constexpr int kSplitSmemMax = 4096;
-constexpr int kLookbackWindow = 8;
-
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Exclusive prefix of expert e over the tiles before `tile`, by decoupled
-// look-back: descriptors pack a 2-bit flag (aggregate / inclusive prefix) and a
-// 30-bit count in one word, so relaxed loads of the word are enough.  Loads run
-// kLookbackWindow predecessors at a time.  Returns false if a predecessor never
-// published within the wait limit.
-__device__ __forceinline__ bool lookback_prefix(const uint32_t *tile_state, int tile, int E, int e,
-                                                uint32_t &excl) {
-    excl = 0;
-    int p = tile - 1;
-    while (p >= 0) {
-        const int n = min(kLookbackWindow, p + 1);
-        uint32_t v[kLookbackWindow];
-#pragma unroll
-        for (int i = 0; i < kLookbackWindow; ++i)
-            if (i < n) v[i] = ld_relaxed_u32(tile_state + (size_t)(p - i) * E + e);
-#pragma unroll
-        for (int i = 0; i < kLookbackWindow; ++i) {
-            if (i >= n) break;
-            uint32_t w = v[i];
-            if ((w >> 30) == 0 &&
-                !wait_flag_word_bounded(tile_state + (size_t)(p - i) * E + e, w))
-                return false;
-            excl += w & kValueMask;
-            if ((w & ~kValueMask) == kFlagInclusive) return true;
-        }
-        p -= n;
-    }
-    return true;
-}
+constexpr int kColBatch = 8;   // expert columns a warp sums together (loads in flight)
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
-    int tb, int tc, int k, int E, int ep, int tile_tokens, int64_t n_rows_max,
+    int tb, int tc, int k, int E, int ep, int tile_tokens, int n_tiles, int64_t n_rows_max,
     const int32_t *__restrict__ topk_idx, const uint8_t *__restrict__ keep,
-    const int32_t *__restrict__ chunk_counts, uint32_t *__restrict__ ticket,
-    uint32_t *__restrict__ tile_state, int32_t *__restrict__ expert_offsets,
+    const int32_t *__restrict__ tile_counts, int32_t *__restrict__ expert_offsets,
     int32_t *__restrict__ rank_offsets, int32_t *__restrict__ recv_token,
     int32_t *__restrict__ recv_slot, int32_t *__restrict__ pos, int32_t *__restrict__ send_splits,
     uint32_t *__restrict__ status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ int32_t s_dyn[];
     int32_t *s_eoff = s_dyn;                                 // [E + 1]
     int32_t *s_base = s_eoff + (E + 1);                      // [E]
@@ -155,16 +118,42 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     int32_t *s_exp = s_rank + tile_tokens * k;               // [tile_tokens * k] expert or -1
     int32_t *s_split = s_exp + tile_tokens * k;              // [ep * ep] when it fits
     __shared__ int32_t s_warp_tot[33];
-    __shared__ uint32_t s_tile;
     const bool split_in_smem = ep * ep <= kSplitSmemMax;
+    const int tile = blockIdx.x;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 
-    if (threadIdx.x == 0) s_tile = atomicAdd(ticket, 1u);
-    for (int e = threadIdx.x; e < E; e += blockDim.x) s_eoff[e] = chunk_counts[e];
     for (int i = threadIdx.x; i < kLayoutWarps * E; i += blockDim.x) s_cnt[i] = 0;
     if (split_in_smem)
         for (int i = threadIdx.x; i < ep * ep; i += blockDim.x) s_split[i] = 0;
+    // 0) each expert's rows in the tiles before this one (s_base) and in the chunk
+    // (s_eoff): warp w sums the columns of experts w, w + 8, ..., kColBatch at a
+    // time, lane j the tiles j, j + 32, ...
+    for (int e0 = wid; e0 < E; e0 += kLayoutWarps * kColBatch) {
+        int pre[kColBatch], tot[kColBatch];
+#pragma unroll
+        for (int u = 0; u < kColBatch; ++u) pre[u] = tot[u] = 0;
+        for (int j = lane; j < n_tiles; j += 32) {
+            int v[kColBatch];
+#pragma unroll
+            for (int u = 0; u < kColBatch; ++u) {
+                const int e = e0 + u * kLayoutWarps;
+                v[u] = e < E ? __ldg(tile_counts + (size_t)e * n_tiles + j) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < kColBatch; ++u) {
+                tot[u] += v[u];
+                if (j < tile) pre[u] += v[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kColBatch; ++u) {
+            const int e = e0 + u * kLayoutWarps;
+            const int p = __reduce_add_sync(0xffffffffu, pre[u]);
+            const int q = __reduce_add_sync(0xffffffffu, tot[u]);
+            if (lane == 0 && e < E) { s_base[e] = p; s_eoff[e] = q; }
+        }
+    }
     __syncthreads();
-    const int tile = (int)s_tile;
     const int total = block_exclusive_scan(s_eoff, E, s_warp_tot);
     if (threadIdx.x == 0) s_eoff[E] = total;
     __syncthreads();
@@ -180,7 +169,6 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     // b + lane / k, slot lane % k).  The experts of up to kLoadBatch steps are
     // loaded before the first is ranked, so a walk costs a memory round trip per
     // batch instead of per step; step 3 reads them back from shared memory.
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int t_tile0 = tb + tile * tile_tokens;
     const int tokens_per_warp = tile_tokens / kLayoutWarps;   // 8, 16 or 32
     const int G = 32 / k;                      // tokens per warp step
@@ -225,7 +213,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
     }
     __syncthreads();
 
-    // 2) per-expert warp offsets and tile aggregate; publish, look back, publish inclusive
+    // 2) per-expert warp offsets inside the tile; the tile's first row of each expert
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int w = 0; w < kLayoutWarps; ++w) {
@@ -233,20 +221,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scatter_kernel(
             s_cnt[w * E + e] = run;
             run += c;
         }
-        const uint32_t agg = (uint32_t)run;
-        uint32_t *my = tile_state + (size_t)tile * E + e;
-        uint32_t excl = 0;
-        if (tile == 0) {
-            st_release_u32(my, kFlagInclusive | agg);
-        } else {
-            st_release_u32(my, kFlagAggregate | agg);
-            if (!lookback_prefix(tile_state, tile, E, e, excl)) {
-                raise_status(status, MOE_DEV_WAIT_TIMEOUT);
-                excl = 0x3FFFFFFFu;  // forces every write of this expert out of range
-            }
-            st_release_u32(my, kFlagInclusive | ((excl + agg) & kValueMask));
-        }
-        s_base[e] = s_eoff[e] + (int)excl;
+        s_base[e] += s_eoff[e];
     }
     __syncthreads();
 
@@ -297,6 +272,24 @@ size_t layout_scatter_smem(const moe_config &c, int tile_tokens) {
 // allocation-free entry points.
 SmemOptIn g_scatter_opt_in;
 
+// Both layout kernels over tc > 0 tokens; tile_counts holds n_tiles * E int32.
+cudaError_t launch_layout_kernels(const moe_config &c, int tb, int tc, const int32_t *topk_idx,
+                                  const uint8_t *keep, int32_t *tile_counts, int32_t *expert_offsets,
+                                  int32_t *rank_offsets, int32_t *recv_token, int32_t *recv_slot, int32_t *pos,
+                                  int32_t *send_splits, uint32_t *status, int64_t n_rows_max, cudaStream_t s) {
+    const int tile_tokens = layout_tile_tokens(tc);
+    const int n_tiles = (tc + tile_tokens - 1) / tile_tokens;
+    cudaError_t err = launch_dependent(layout_hist_kernel, n_tiles, kLayoutThreads, sizeof(int32_t) * c.E, s,
+                                       tb, tc, c.k, c.E, c.ep, tile_tokens, n_tiles, topk_idx, keep, tile_counts,
+                                       send_splits);
+    if (err != cudaSuccess) return err;
+    const size_t smem = layout_scatter_smem(c, tile_tokens);
+    if ((err = g_scatter_opt_in.ensure(layout_scatter_kernel, smem)) != cudaSuccess) return err;
+    return launch_dependent(layout_scatter_kernel, n_tiles, kLayoutThreads, smem, s, tb, tc, c.k, c.E, c.ep,
+                            tile_tokens, n_tiles, n_rows_max, topk_idx, keep, tile_counts, expert_offsets,
+                            rank_offsets, recv_token, recv_slot, pos, send_splits, status);
+}
+
 cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
                                    const int32_t *topk_idx, const uint8_t *keep,
                                    int32_t *expert_offsets, int32_t *rank_offsets,
@@ -305,31 +298,15 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
                                    int64_t n_rows_max, cudaStream_t s, int num_sms) {
     const ScratchLayout L = scratch_layout(c);
     uint32_t *status = ws_at<uint32_t>(ws, L.status);
-    uint32_t *ticket = ws_at<uint32_t>(ws, L.ticket);
-    int32_t *chunk_counts = ws_at<int32_t>(ws, L.chunk_counts);
-    uint32_t *tile_state = ws_at<uint32_t>(ws, L.tile_state);
-    const int tile_tokens = layout_tile_tokens(tc);
-    const int n_tiles = (tc + tile_tokens - 1) / tile_tokens;
-    // ticket, chunk counts and the tiles' look-back descriptors start at zero
-    const size_t clear_bytes = L.tile_state - L.ticket + sizeof(uint32_t) * (size_t)n_tiles * c.E;
-    cudaError_t err = cudaMemsetAsync(ws_at<char>(ws, L.ticket), 0, clear_bytes, s);
-    if (err != cudaSuccess) return err;
+    int32_t *tile_counts = ws_at<int32_t>(ws, L.tile_counts);
+    cudaError_t err = cudaSuccess;
     if (tc == 0) {
         err = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (size_t)(c.E + 1), s);
         if (err == cudaSuccess) err = cudaMemsetAsync(rank_offsets, 0, sizeof(int32_t) * (size_t)(c.ep + 1), s);
         if (err == cudaSuccess) err = cudaMemsetAsync(send_splits, 0, sizeof(int32_t) * (size_t)c.ep * c.ep, s);
     } else {
-        int hb = (int)(((size_t)tc * c.k + kLayoutThreads - 1) / kLayoutThreads);
-        if (hb > num_sms * 2) hb = num_sms * 2;
-        layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, s>>>(
-            tb, tc, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
-        const size_t smem = layout_scatter_smem(c, tile_tokens);
-        if ((err = g_scatter_opt_in.ensure(layout_scatter_kernel, smem)) != cudaSuccess) return err;
-        layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, s>>>(
-            tb, tc, c.k, c.E, c.ep, tile_tokens, n_rows_max, topk_idx, keep, chunk_counts, ticket, tile_state,
-            expert_offsets, rank_offsets, recv_token, recv_slot, pos, send_splits, status);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        err = launch_layout_kernels(c, tb, tc, topk_idx, keep, tile_counts, expert_offsets, rank_offsets,
+                                    recv_token, recv_slot, pos, send_splits, status, n_rows_max, s);
     }
     if (err != cudaSuccess) return err;
     if (splits_host) {
@@ -353,12 +330,12 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
 // device memory all belongs to an allocator it does not control (a
 // pre-reserved pool it may not grow), and latency-critical loops that must not
 // hit the implicit device synchronisation of cudaMalloc / cudaFree.  For them
-// this entry point keeps the dispatch layout's scratch (the tile ticket, the
-// chunk's per-expert counts and the look-back descriptors) in one fixed
-// device array inside the library instead of a caller workspace.
+// this entry point keeps the dispatch layout's scratch (a status word and the
+// tiles' per-expert counts) in one fixed device array inside the library
+// instead of a caller workspace.
 //
 // Limits: at most kNoAllocMaxTiles * 256 tokens per call and E <= 1024.  The
-// array (about 261 KiB) exists on every device that loads the library, until
+// array (about 256 KiB) exists on every device that loads the library, until
 // the process exits.  Every call shares it: calls that may overlap on the GPU
 // (different streams without ordering, or several host threads) race and
 // corrupt each other's layouts; order them.  The first call on a device looks
@@ -369,11 +346,9 @@ cudaError_t launch_dispatch_layout(const moe_config &c, int tb, int tc,
 namespace {
 
 constexpr int kNoAllocMaxTiles = 64;   // 16384 tokens per call
-constexpr size_t kNoAllocTicket = 0;
-constexpr size_t kNoAllocStatus = 256;
-constexpr size_t kNoAllocCounts = 512;
-constexpr size_t kNoAllocTiles = kNoAllocCounts + sizeof(int32_t) * moe::kMaxExperts;
-constexpr size_t kNoAllocBytes = kNoAllocTiles + sizeof(uint32_t) * (size_t)kNoAllocMaxTiles * moe::kMaxExperts;
+constexpr size_t kNoAllocStatus = 0;
+constexpr size_t kNoAllocTiles = 256;
+constexpr size_t kNoAllocBytes = kNoAllocTiles + sizeof(int32_t) * (size_t)kNoAllocMaxTiles * moe::kMaxExperts;
 
 static __device__ __align__(256) unsigned char g_noalloc_layout_scratch[kNoAllocBytes];
 
@@ -434,32 +409,16 @@ extern "C" moe_status moe_dispatch_layout_noalloc(
     cudaError_t err = noalloc_scratch(&base);
     if (err != cudaSuccess) return report_error(MOE_ERR_CUDA, cudaGetErrorString(err));
     unsigned char *b = static_cast<unsigned char *>(base);
-    uint32_t *ticket = reinterpret_cast<uint32_t *>(b + kNoAllocTicket);
     uint32_t *st_word = status ? status : reinterpret_cast<uint32_t *>(b + kNoAllocStatus);
-    int32_t *chunk_counts = reinterpret_cast<int32_t *>(b + kNoAllocCounts);
-    uint32_t *tile_state = reinterpret_cast<uint32_t *>(b + kNoAllocTiles);
-    const int num_sms = [] { int d = 0, n = 148; cudaGetDevice(&d); cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d); return n; }();
-    // the previous call's ticket, counts and look-back descriptors start again at zero
-    err = cudaMemsetAsync(b, 0, kNoAllocTiles + sizeof(uint32_t) * (size_t)n_tiles * c.E, stream);
-    if (err == cudaSuccess && tok_count == 0) {
+    int32_t *tile_counts = reinterpret_cast<int32_t *>(b + kNoAllocTiles);
+    if (tok_count == 0) {
         err = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (size_t)(c.E + 1), stream);
         if (err == cudaSuccess) err = cudaMemsetAsync(rank_offsets, 0, sizeof(int32_t) * (size_t)(c.ep + 1), stream);
         if (err == cudaSuccess) err = cudaMemsetAsync(send_splits, 0, sizeof(int32_t) * (size_t)c.ep * c.ep, stream);
-    } else if (err == cudaSuccess) {
-        int hb = (int)(((size_t)tok_count * c.k + kLayoutThreads - 1) / kLayoutThreads);
-        if (hb > num_sms * 2) hb = num_sms * 2;
-        layout_hist_kernel<<<hb, kLayoutThreads, sizeof(int32_t) * c.E, stream>>>(
-            tok_begin, tok_count, c.k, c.E, c.ep, topk_idx, keep, chunk_counts, send_splits);
-        err = cudaGetLastError();
-        const size_t smem = layout_scatter_smem(c, tile_tokens);
-        if (err == cudaSuccess) err = g_scatter_opt_in.ensure(layout_scatter_kernel, smem);
-        if (err == cudaSuccess) {
-            layout_scatter_kernel<<<n_tiles, kLayoutThreads, smem, stream>>>(
-                tok_begin, tok_count, c.k, c.E, c.ep, tile_tokens, max_recv_rows_of(c, tok_count), topk_idx, keep,
-                chunk_counts, ticket, tile_state, expert_offsets, rank_offsets, recv_token, recv_slot,
-                pos, send_splits, st_word);
-            err = cudaGetLastError();
-        }
+    } else {
+        err = launch_layout_kernels(c, tok_begin, tok_count, topk_idx, keep, tile_counts, expert_offsets,
+                                    rank_offsets, recv_token, recv_slot, pos, send_splits, st_word,
+                                    max_recv_rows_of(c, tok_count), stream);
     }
     if (err == cudaSuccess && splits_host) {
         err = cudaMemcpyAsync(splits_host, expert_offsets, sizeof(int32_t) * (size_t)(c.E + 1),

@@ -132,6 +132,8 @@ template <int VPT>
 __global__ void __launch_bounds__(kPqThreads) permute_quant_kernel(
     int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint8_t *__restrict__ xr_q, uint8_t *__restrict__ x_scale) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_pos[kMaxTopK];
     __shared__ float s_red[kPqThreads / 32];
     __shared__ int s_any;
@@ -183,12 +185,10 @@ cudaError_t launch_permute_quant(const moe_config &c, const void *x, const int32
     const int row_vecs = c.H / 8;
     const uint4 *xv = static_cast<const uint4 *>(x);
     if (row_vecs <= 2 * kPqThreads)
-        permute_quant_kernel<2><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
-    else if (row_vecs <= 8 * kPqThreads)
-        permute_quant_kernel<8><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
-    else
-        return cudaErrorNotSupported;
-    return cudaGetLastError();
+        return launch_dependent(permute_quant_kernel<2>, tc, kPqThreads, 0, s, tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
+    if (row_vecs <= 8 * kPqThreads)
+        return launch_dependent(permute_quant_kernel<8>, tc, kPqThreads, 0, s, tb, c.k, row_vecs, xv, pos, xr_q, x_scale);
+    return cudaErrorNotSupported;
 }
 
 // ------------------------------------------------------------------ K-blocked scales
@@ -252,6 +252,8 @@ template <int VPT>
 __global__ void __launch_bounds__(kPqThreads) permute_quant_blocks_kernel(
     int tb, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint8_t *__restrict__ xr_q, uint8_t *__restrict__ xr_sf) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_pos[kMaxTopK];
     __shared__ int s_any;
     const int i = blockIdx.x;
@@ -292,12 +294,10 @@ cudaError_t launch_permute_quant_blocks(const moe_config &c, const void *x, cons
     const int row_vecs = c.H / 8;
     const uint4 *xv = static_cast<const uint4 *>(x);
     if (row_vecs <= 2 * kPqThreads)
-        permute_quant_blocks_kernel<2><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
-    else if (row_vecs <= 8 * kPqThreads)
-        permute_quant_blocks_kernel<8><<<tc, kPqThreads, 0, s>>>(tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
-    else
-        return cudaErrorNotSupported;
-    return cudaGetLastError();
+        return launch_dependent(permute_quant_blocks_kernel<2>, tc, kPqThreads, 0, s, tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
+    if (row_vecs <= 8 * kPqThreads)
+        return launch_dependent(permute_quant_blocks_kernel<8>, tc, kPqThreads, 0, s, tb, c.k, row_vecs, xv, pos, xr_q, xr_sf);
+    return cudaErrorNotSupported;
 }
 
 cudaError_t launch_quant_rows(int64_t rows, int cols, bool bf16, const void *in, uint8_t *codes,

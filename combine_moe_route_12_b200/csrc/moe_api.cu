@@ -1231,20 +1231,15 @@ moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
 
 // One thread waits on something that never completes, through the same bounded
 // helpers the kernels use, and reports the timeout like they do.
-__global__ void watchdog_selftest_kernel(int which, uint64_t limit_ns, const uint32_t *never_set,
-                                         uint32_t *status) {
+__global__ void watchdog_selftest_kernel(int which, uint64_t limit_ns, uint32_t *status) {
     __shared__ uint64_t bar;
     if (threadIdx.x != 0) return;
-    bool ok;
-    if (which == 0) {
-        uint32_t w = 0;
-        ok = wait_flag_word_bounded(never_set, w, limit_ns);
-    } else {
-        mbar_init(&bar, 1);
-        fence_mbar_init();
-        volatile int never = 0;
-        ok = mbar_wait_bounded(&bar, 0, &never, limit_ns);   // phase 0 never completes
-    }
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    volatile int never = 0;
+    // phase 0 never completes
+    const bool ok = which == 0 ? mbar_wait_cluster_bounded(&bar, 0, &never, limit_ns)
+                               : mbar_wait_bounded(&bar, 0, &never, limit_ns);
     if (!ok) raise_status(status, MOE_DEV_WAIT_TIMEOUT);
 }
 
@@ -1257,7 +1252,6 @@ moe_status moe_watchdog_selftest(const moe_config *cfg, int32_t which, int32_t l
     if (limit_us < 1 || limit_us > 2000000) return fail(MOE_ERR_INVALID_ARG, "limit_us outside [1, 2e6]");
     const ScratchLayout L = scratch_layout(*cfg);
     watchdog_selftest_kernel<<<1, 32, 0, stream>>>(which, (uint64_t)limit_us * 1000ull,
-                                                   ws_at<uint32_t>(ws, L.watchdog),
                                                    ws_at<uint32_t>(ws, L.status));
     cudaError_t err = cudaGetLastError();
     return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_watchdog_selftest");

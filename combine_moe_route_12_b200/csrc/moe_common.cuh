@@ -101,15 +101,14 @@ class SmemOptIn {
 // ---------------------------------------------------------------- workspace
 // Scratch layout (all offsets 256-byte aligned):
 //   [0, 256)        status word (uint32 at offset 0)
-//   layout ticket   uint32, then chunk_counts int32[E]
-//   tile_state      uint32[max_tiles * E] (decoupled-lookback descriptors)
+//   tile_counts     int32[E * max_tiles] (dispatch layout: rows per expert and tile)
 //   clip threshold  uint64[E]
 //   ffn counters    uint32[2] (dynamic work distribution of the FFN GEMMs)
 //   shared expert   uint32[2] counters, int32[2] expert offsets
 //   clip segments   int32[2 * (E + 1)] offsets / cursors, keys uint64[T * k]
 struct ScratchLayout {
-    size_t status, ticket, chunk_counts, tile_state, clip_thr, ffn_ctr;
-    size_t shared_ctr, shared_off, watchdog;
+    size_t status, tile_counts, clip_thr, ffn_ctr;
+    size_t shared_ctr, shared_off;
     size_t clip_seg, clip_keys, total;
     int max_tiles;
 };
@@ -120,15 +119,12 @@ inline ScratchLayout scratch_layout(const moe_config &c) {
     ScratchLayout L{};
     size_t off = 0;
     L.status = off;               off += 256;
-    L.ticket = off;               off += 256;
-    L.chunk_counts = off;         off = align_up(off + sizeof(int32_t) * (size_t)c.E, 256);
     L.max_tiles = (int)layout_max_tiles(c.T);
-    L.tile_state = off;           off = align_up(off + sizeof(uint32_t) * (size_t)L.max_tiles * c.E, 256);
+    L.tile_counts = off;          off = align_up(off + sizeof(int32_t) * (size_t)L.max_tiles * c.E, 256);
     L.clip_thr = off;             off = align_up(off + sizeof(uint64_t) * (size_t)c.E, 256);
     L.ffn_ctr = off;              off += 256;   // work counters of the two FFN launches
     L.shared_ctr = off;           off += 256;   // the shared expert's own two counters
     L.shared_off = off;           off += 256;   // its expert offsets {0, rows}
-    L.watchdog = off;             off += 256;   // a word nothing ever sets (watchdog self-test)
     L.clip_seg = off;             off = align_up(off + sizeof(int32_t) * 2 * ((size_t)c.E + 1), 256);
     L.clip_keys = off;            off = align_up(off + sizeof(uint64_t) * (size_t)c.T * c.k, 256);
     L.total = off;
@@ -197,17 +193,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// Spins (relaxed loads) until the 2-bit flag field (bits 30-31) of *q is set,
-// as the dispatch layout's look-back waits for a predecessor's descriptor.
-// Returns false after limit_ns; w receives the last value read.
-__device__ __forceinline__ bool wait_flag_word_bounded(const uint32_t *q, uint32_t &w,
-                                                       uint64_t limit_ns = kWaitLimitNs) {
-    const uint64_t t0 = global_timer_ns();
-    for (;;) {
-        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w) : "l"(q) : "memory");
-        if ((w >> 30) != 0) return true;
-        if (global_timer_ns() - t0 > limit_ns) return false;
-    }
+// ---------------------------------------------------------------- dependent launch
+// The index-path, permute and combine kernels are launched with programmatic
+// stream serialisation: the GPU may start one while the kernel before it in the
+// stream is still finishing, which hides the launch gap between two dependent
+// kernels.  Each such kernel calls grid_dependency_wait() before its first
+// global-memory access, in every thread: the wait returns once the earlier
+// kernels of the stream have completed and their writes are visible (at once
+// when the kernel was launched without the attribute).  grid_dependents_launch()
+// lets the next kernel be scheduled early; it still waits for this one to
+// complete before it touches memory.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                                    cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // ---------------------------------------------------------------- TMA
@@ -281,14 +295,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity,
-                                                          volatile int *abort_flag) {
+                                                          volatile int *abort_flag,
+                                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((i & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
         }
     }
 }

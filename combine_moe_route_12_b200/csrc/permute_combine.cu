@@ -46,6 +46,8 @@ __device__ __forceinline__ void load_slots(int tb, int i0, int n, int k, const i
 __global__ void __launch_bounds__(kRowThreads) permute_rows_kernel(
     int tb, int tc, int tpc, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint4 *__restrict__ xr) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_pos[kTokPerCta][kMaxTopK];
     const int i0 = blockIdx.x * tpc;
     const int n = min(tpc, tc - i0);
@@ -86,6 +88,8 @@ constexpr int kCombineBatch = 4;   // expert rows of a token loaded together
 __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
     int tb, int tc, int tpc, int k, int row_vecs, const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const uint4 *__restrict__ y_shared, uint4 *__restrict__ out) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
     __shared__ float s_w_all[kTokPerCta][kMaxTopK];
     const int i0 = blockIdx.x * tpc;
@@ -152,6 +156,8 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_bf16_kernel(
 __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
     int tb, int tc, int tpc, int k, int row_vecs, const float4 *__restrict__ y, const int32_t *__restrict__ pos,
     const float *__restrict__ topk_w, const float4 *__restrict__ y_shared, float4 *__restrict__ out) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     __shared__ int32_t s_pos_all[kTokPerCta][kMaxTopK];
     __shared__ float s_w_all[kTokPerCta][kMaxTopK];
     const int i0 = blockIdx.x * tpc;
@@ -184,6 +190,8 @@ __global__ void __launch_bounds__(kRowThreads) combine_rows_f32_kernel(
 __global__ void reduce_finalize_kernel(int tb, int tc, int H, int dtype,
                                        const float4 *__restrict__ red, const void *__restrict__ y_shared,
                                        void *__restrict__ out) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const size_t n4 = (size_t)tc * H / 4;
     const size_t base4 = (size_t)tb * H / 4;
     for (size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
@@ -224,6 +232,8 @@ constexpr int kWarpVecs = 8;
 __global__ void __launch_bounds__(kRowThreads) permute_rows_warp_kernel(
     int tb, int tc, int k, int row_vecs, const uint4 *__restrict__ x, const int32_t *__restrict__ pos,
     uint4 *__restrict__ xr) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int lane = threadIdx.x & 31;
     const int i = blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     if (i >= tc) return;
@@ -257,13 +267,11 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *po
     const int row_vecs = (int)((size_t)c.H * (c.ffn_fp8 ? 1 : c.dtype == MOE_F32 ? 4 : 2) / 16);
     const int tpc = tok_per_cta(tc);
     if (tpc > 1 && row_vecs <= 32 * kWarpVecs) {
-        permute_rows_warp_kernel<<<(tc + 3) / 4, kRowThreads, 0, s>>>(
-            tb, tc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
-        return cudaGetLastError();
+        return launch_dependent(permute_rows_warp_kernel, (tc + 3) / 4, kRowThreads, 0, s,
+                                tb, tc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
     }
-    permute_rows_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
-        tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
-    return cudaGetLastError();
+    return launch_dependent(permute_rows_kernel, (tc + tpc - 1) / tpc, kRowThreads, 0, s,
+                            tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(x), pos, static_cast<uint4 *>(xr));
 }
 
 cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *pos,
@@ -273,16 +281,15 @@ cudaError_t launch_combine(const moe_config &c, const void *y, const int32_t *po
     const int tpc = tok_per_cta(tc);
     if (c.dtype == MOE_F32) {
         const int row_vecs = c.H / 4;
-        combine_rows_f32_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
-            tb, tc, tpc, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
-            static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
+        return launch_dependent(combine_rows_f32_kernel, (tc + tpc - 1) / tpc, kRowThreads, 0, s,
+                                tb, tc, tpc, c.k, row_vecs, static_cast<const float4 *>(y), pos, topk_w,
+                                static_cast<const float4 *>(y_shared), static_cast<float4 *>(out));
     } else {
         const int row_vecs = c.H / 8;
-        combine_rows_bf16_kernel<<<(tc + tpc - 1) / tpc, kRowThreads, 0, s>>>(
-            tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
-            static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
+        return launch_dependent(combine_rows_bf16_kernel, (tc + tpc - 1) / tpc, kRowThreads, 0, s,
+                                tb, tc, tpc, c.k, row_vecs, static_cast<const uint4 *>(y), pos, topk_w,
+                                static_cast<const uint4 *>(y_shared), static_cast<uint4 *>(out));
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb, int tc,
@@ -291,9 +298,8 @@ cudaError_t launch_reduce_finalize(const moe_config &c, const float *red, int tb
     const size_t n4 = (size_t)tc * c.H / 4;
     int blocks = (int)((n4 + 255) / 256);
     if (blocks > num_sms * 8) blocks = num_sms * 8;
-    reduce_finalize_kernel<<<blocks, 256, 0, s>>>(tb, tc, c.H, c.dtype,
-                                                  reinterpret_cast<const float4 *>(red), y_shared, out);
-    return cudaGetLastError();
+    return launch_dependent(reduce_finalize_kernel, blocks, 256, 0, s, tb, tc, c.H, c.dtype,
+                            reinterpret_cast<const float4 *>(red), y_shared, out);
 }
 
 // Expert offsets {0, rows} of the shared expert's one-expert FFN launch.

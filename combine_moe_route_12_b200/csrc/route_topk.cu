@@ -3,13 +3,19 @@
 // top-k is saved state), and its variants: grouped top-k (the experts() path of
 // the same page) and a bias that steers the selection only.
 //
-// A group of LPT lanes (8, 16 or 32) per token, 32/LPT tokens per warp at a
-// time.  Lane l of a group holds the biased logits of experts l, l+LPT, ... as
-// 64-bit rank keys (value descending, lower expert index first among equal
+// Plain top-k: one warp per token.  Lane l holds the biased logits of experts
+// l, l+32, ... as 32-bit order keys (the fp32 bits mapped so that unsigned order
+// is value order) and tracks its best remaining one (the lowest expert among
+// equal values).  A round is two warp reductions in hardware (redux.sync): the
+// largest key over the lanes, then the lowest expert among the lanes holding it;
+// lane j keeps slot j, and only the winning lane rescans its few values.  The
+// next token's logits are loaded while the current token's rounds run.
+// Grouped top-k: a group of LPT lanes (8, 16 or 32) per token, 32/LPT tokens per
+// warp at a time.  Lane l of a group holds the biased logits of experts l, l+LPT,
+// ... as 64-bit rank keys (value descending, lower expert index first among equal
 // values).  k rounds of a butterfly max over the lanes' best remaining keys pick
 // the experts in rank order; lane j of the group keeps slot j, and only the lane
-// whose key won rescans its values.  Narrow groups keep each round's shuffle
-// chain short and several tokens in flight per warp.
+// whose key won rescans its values.
 // The weights w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0) use a fixed fp32
 // exponential (Cody & Waite reduction, degree-7 Taylor polynomial, every step
 // one IEEE-rounded operation) and a slot-ordered sum, so they are bit-exact
@@ -84,12 +90,115 @@ __device__ __forceinline__ void merge_top2(uint64_t &a1, uint64_t &a2, uint64_t 
     }
 }
 
-template <int LPT, int VPL, bool kGrouped>
-__global__ void __launch_bounds__(256) route_topk_kernel(
+// Unsigned order key of a (finite or infinite) fp32 value: larger value, larger
+// key; every real key is > 0, which marks a taken or missing expert.
+__device__ __forceinline__ uint32_t order_key(float l) {
+    const uint32_t u = __float_as_uint(l);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_value(uint32_t ord) {
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+}
+
+// The lane's best remaining key and its index (the first among equal keys: the
+// lowest expert, since the lane's experts ascend with i).
+template <int VPL>
+__device__ __forceinline__ void lane_best(const uint32_t (&ord)[VPL], uint32_t &best, int &bi) {
+    best = ord[0];
+    bi = 0;
+#pragma unroll
+    for (int i = 1; i < VPL; ++i)
+        if (ord[i] > best) { best = ord[i]; bi = i; }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_topk_warp_kernel(
+    int T, int E, int k, const float *__restrict__ logits, const float *__restrict__ bias,
+    int bias_select_only, int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+    int32_t *__restrict__ counts, uint32_t *__restrict__ status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    extern __shared__ int32_t s_hist[];  // [E]
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const long long warps_total = (long long)gridDim.x * (blockDim.x >> 5);
+    long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    float bv[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        bv[i] = (bias && e < E) ? __ldg(bias + e) : 0.0f;
+    }
+    float nxt[VPL];
+    auto load_row = [&](long long tt) {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            nxt[i] = (tt < T && e < E) ? __ldg(logits + (size_t)tt * E + e) : 0.0f;
+        }
+    };
+    load_row(t);
+    bool nonfinite = false;
+    for (; t < T; t += warps_total) {
+        uint32_t ord[VPL];
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            // the add also turns -0 into +0, so the key order matches IEEE ==
+            float l = __fadd_rn(nxt[i], bv[i]);
+            if (!isfinite(l)) {
+                if (lane + 32 * i < E) nonfinite = true;
+                if (isnan(l)) l = -INFINITY;  // keep the ranking a total order
+            }
+            ord[i] = lane + 32 * i < E ? order_key(l) : 0u;
+        }
+        load_row(t + warps_total);   // the next token's logits, in flight during the rounds
+        uint32_t best;
+        int bi;
+        lane_best(ord, best, bi);
+        uint32_t my_ord = 0;
+        int my_e = -1;
+        for (int j = 0; j < k; ++j) {
+            const uint32_t top = __reduce_max_sync(0xffffffffu, best);
+            const uint32_t cand = (best == top) ? (uint32_t)(lane + 32 * bi) : 0xFFFFFFFFu;
+            const uint32_t e_top = __reduce_min_sync(0xffffffffu, cand);
+            if (lane == j) { my_ord = top; my_e = (int)e_top; }
+            if (cand == e_top) {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i)
+                    if (i == bi) ord[i] = 0u;
+                lane_best(ord, best, bi);
+            }
+        }
+        // the weights' logit: biased, or the unbiased logit when the bias only selects
+        float my_v = order_value(my_ord);
+        if (bias_select_only && lane < k) my_v = __fadd_rn(__ldg(logits + (size_t)t * E + my_e), 0.0f);
+        float m = lane < k ? my_v : -INFINITY;   // the largest of the k
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float ex = (lane < k) ? det_exp_nonpos(__fsub_rn(my_v, m)) : 0.0f;
+        float S = 0.0f;
+        for (int j = 0; j < k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, ex, j));
+        if (lane < k) {
+            topk_idx[(size_t)t * k + lane] = my_e;
+            topk_w[(size_t)t * k + lane] = __fdiv_rn(ex, S);
+            if (my_e >= 0 && my_e < E) atomicAdd(&s_hist[my_e], 1);   // always, as k <= E
+        }
+    }
+    if (nonfinite) raise_status(status, MOE_DEV_NONFINITE_LOGIT);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        if (s_hist[e]) atomicAdd(&counts[e], s_hist[e]);
+}
+
+template <int LPT, int VPL>
+__global__ void __launch_bounds__(256) route_topk_grouped_kernel(
     int T, int E, int k, const float *__restrict__ logits, const float *__restrict__ bias,
     RouteVariant rv,
     int32_t *__restrict__ topk_idx, float *__restrict__ topk_w, int32_t *__restrict__ counts,
     uint32_t *__restrict__ status) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     extern __shared__ int32_t s_hist[];  // [E]
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
     __syncthreads();
@@ -121,7 +230,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
                 key[i] = rank_key(l, e);
             }
         }
-        if (kGrouped) {
+        {
             // grouped top-k: the score of every expert group (in-group butterfly per
             // group), kept as rank keys (score, group) spread over the lanes like the
             // experts (lane l holds groups l, l + LPT, ...); the topk_group best groups
@@ -235,7 +344,23 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     if (blocks > cap) blocks = cap;
     const size_t smem = sizeof(int32_t) * (size_t)c.E;
     const RouteVariant rv{c.n_group, c.topk_group, c.group_score, c.bias_select_only};
-    // lanes per token: at least k (slot j lives in group lane j), at most 32,
+    if (rv.n_group <= 1) {
+        // one warp per token, up to 8 CTAs of 8 warps per SM
+        int wb = (c.T + warps_per_block - 1) / warps_per_block;
+        if (wb > num_sms * 8) wb = num_sms * 8;
+        const int v = (c.E + 31) / 32;
+#define MOE_ROUTE_WARP(V)                                                                                 \
+    return launch_dependent(route_topk_warp_kernel<V>, wb, 256, smem, s, c.T, c.E, c.k, logits, bias,     \
+                            c.bias_select_only, topk_idx, topk_w, counts, status)
+        if (v <= 1) MOE_ROUTE_WARP(1);
+        if (v <= 2) MOE_ROUTE_WARP(2);
+        if (v <= 4) MOE_ROUTE_WARP(4);
+        if (v <= 8) MOE_ROUTE_WARP(8);
+        if (v <= 16) MOE_ROUTE_WARP(16);
+        MOE_ROUTE_WARP(32);
+#undef MOE_ROUTE_WARP
+    }
+    // grouped: lanes per token: at least k (slot j lives in group lane j), at most 32,
     // aiming at 16 values per lane
     int lpt = 8;
     while (lpt < 32 && (lpt < c.k || (c.E + lpt - 1) / lpt > 16)) lpt *= 2;
@@ -243,14 +368,9 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
     blocks = (int)(((long long)c.T * lpt / 32 + warps_per_block - 1) / warps_per_block);
     if (blocks < 1) blocks = 1;
     if (blocks > cap) blocks = cap;
-#define MOE_ROUTE_LAUNCH(L, V, G)                                                               \
-    route_topk_kernel<L, V, G><<<blocks, 256, smem, s>>>(c.T, c.E, c.k, logits, bias, rv, topk_idx, \
-                                                         topk_w, counts, status)
-#define MOE_ROUTE_CASE(L, V)                      \
-    do {                                          \
-        if (rv.n_group > 1) MOE_ROUTE_LAUNCH(L, V, true); \
-        else MOE_ROUTE_LAUNCH(L, V, false);       \
-    } while (0)
+#define MOE_ROUTE_CASE(L, V)                                                                                 \
+    return launch_dependent(route_topk_grouped_kernel<L, V>, blocks, 256, smem, s, c.T, c.E, c.k, logits, bias, \
+                            rv, topk_idx, topk_w, counts, status)
     if (lpt == 8) {
         if (vpl <= 1) MOE_ROUTE_CASE(8, 1);
         else if (vpl <= 2) MOE_ROUTE_CASE(8, 2);
@@ -271,9 +391,7 @@ cudaError_t launch_route_topk(const moe_config &c, const float *logits, const fl
         else if (vpl <= 16) MOE_ROUTE_CASE(32, 16);
         else MOE_ROUTE_CASE(32, 32);
     }
-#undef MOE_ROUTE_LAUNCH
 #undef MOE_ROUTE_CASE
-    return cudaGetLastError();
 }
 
 }  // namespace moe

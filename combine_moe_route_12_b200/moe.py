@@ -385,7 +385,8 @@ def moe_forward_host(cfg, logits_host, bias_host, x_host, w13, w2, out_host, top
 
 def moe_watchdog_selftest(cfg, which: int, limit_us: int, ws, stream=None):
     """Runs one of the library's bounded waits on something that never completes
-    (0: the look-back spin, 1: an mbarrier wait); it sets MOE_DEV_WAIT_TIMEOUT."""
+    (0: a cluster-scope mbarrier wait, 1: a CTA-scope mbarrier wait); it sets
+    MOE_DEV_WAIT_TIMEOUT."""
     _check(_lib.moe_watchdog_selftest(ctypes.byref(cfg), which, limit_us, _ptr(ws), _stream(stream)))
 
 

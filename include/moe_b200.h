@@ -91,7 +91,7 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
 /* Device status bits (moe_device_status). */
 #define MOE_DEV_NONFINITE_LOGIT 0x1u  /* a logit (+bias) was NaN or +-Inf          */
-#define MOE_DEV_WAIT_TIMEOUT    0x2u  /* a bounded spin (lookback scan, mbarrier)  */
+#define MOE_DEV_WAIT_TIMEOUT    0x2u  /* a bounded wait ran out (mbarrier)         */
                                       /* gave up; outputs of that call are invalid */
 #define MOE_DEV_BAD_INDEX       0x4u  /* an expert id outside [0, E) was read      */
 
@@ -253,7 +253,7 @@ moe_status moe_dispatch_layout(const moe_config *cfg, int32_t tok_begin, int32_t
  *   status: device uint32 that receives the MOE_DEV_* bits (OR-ed in), or
  *           NULL to drop them.
  * The layout's scratch lives in one fixed device array inside the library
- * (about 261 KiB per device, held until the process exits).  Limits:
+ * (about 256 KiB per device, held until the process exits).  Limits:
  * tok_count <= 16384 (MOE_ERR_UNSUPPORTED beyond).  All calls share the
  * array: calls that may overlap on the GPU race and must be ordered.  The
  * first call on a device looks up the array's address with that device
@@ -644,9 +644,10 @@ moe_status moe_forward_host(const moe_config *cfg, const float *logits_host,
  * library's own bounded-wait code on something that never completes, with a
  * short limit, so a caller can check that a wait that runs out is reported and
  * that the context stays usable.
- *   which 0: the dispatch layout's look-back spin on a descriptor word nothing
- *            publishes (a zero word of ws);
- *   which 1: the FFN's mbarrier wait on a barrier nothing arrives at.
+ *   which 0: the FFN's cluster-scope mbarrier wait (slice queue, scale ring) on a
+ *            barrier nothing arrives at;
+ *   which 1: the FFN's CTA-scope mbarrier wait (operand ring, accumulators) on a
+ *            barrier nothing arrives at.
  *   limit_us in [1, 2000000].
  * One thread waits about limit_us, sets MOE_DEV_WAIT_TIMEOUT in ws's status word
  * and returns; read it with moe_device_status.  ws: moe_workspace_bytes(cfg).

@@ -35,12 +35,14 @@ def test_algorithmic_counts_only_needed_x_rows_and_fp8_bytes():
 
 
 def test_kernels_per_step():
-    assert bench.kernels_per_step(WORKLOADS["qwen3_30b_a3b"]) == 1 + 2 + 6
+    # no capacity: the clip is one pass
+    assert bench.kernels_per_step(WORKLOADS["qwen3_30b_a3b"]) == 1 + 1 + 6
     assert bench.kernels_per_step(WORKLOADS["skew_capacity"]) == 1 + 4 + 6
-    assert bench.kernels_per_step(WORKLOADS["dsv3_prefill"]) == 1 + 2 + 2 * 6
-    assert bench.kernels_per_step(WORKLOADS["dsv3_grouped"]) == 1 + 2 + 6 + 3
-    assert bench.kernels_per_step(WORKLOADS["qwen3_30b_a3b_fp8"]) == 1 + 2 + 6 + 1
-    assert bench.kernels_per_step(WORKLOADS["dsv3_prefill_fp8"]) == 1 + 2 + 2 * (6 + 1)
+    assert bench.kernels_per_step(WORKLOADS["dsv3_prefill"]) == 1 + 1 + 2 * 6
+    assert bench.kernels_per_step(WORKLOADS["dsv3_grouped"]) == 1 + 1 + 6 + 3
+    assert bench.kernels_per_step(WORKLOADS["qwen3_30b_a3b_fp8"]) == 1 + 1 + 6 + 1
+    assert bench.kernels_per_step(WORKLOADS["dsv3_prefill_fp8"]) == 1 + 1 + 2 * (6 + 1)
+    assert bench.kernels_per_step(WORKLOADS["qwen3_30b_a3b"].with_(capacity=0)) == 1 + 2 + 6
 
 
 def test_default_arguments_finish_within_minutes():

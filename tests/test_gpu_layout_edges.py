@@ -3,7 +3,7 @@ its tiling: a chunk smaller than one warp step per tile, k = 1 and k = 32
 (thirty-two slots per token: one token per warp step), a chunk of 16384 tokens
 (64 tiles of 256), a binding capacity (dropped slots, pos = -1), E = 1024
 experts with 64 ranks (a 4096-entry split matrix in shared memory), and chunks
-beyond 64 tiles (the look-back walks more than one window of predecessors).
+beyond 64 tiles (each tile's column sums run over more than one 32-tile lane stride).
 Routing is taken from the GPU's own route + clip, compared here with the
 oracle's, so the layout inputs are the oracle's.
 """

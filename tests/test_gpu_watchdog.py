@@ -1,9 +1,9 @@
 """Failure detection on the GPU without a fault: every device-side wait of the
 library is bounded; a wait that runs out sets MOE_DEV_WAIT_TIMEOUT in the
 status word and the kernel returns, leaving the context usable.  The watchdog
-self-test entry point runs the library's own bounded waits (the dispatch
-layout's look-back spin, the FFN's mbarrier wait) on something that never
-completes, with a 20 ms limit."""
+self-test entry point runs the library's own bounded waits (the FFN's
+cluster-scope and CTA-scope mbarrier waits) on a barrier that nothing arrives
+at, with a 20 ms limit."""
 import time
 
 import pytest

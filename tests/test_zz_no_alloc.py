@@ -38,7 +38,7 @@ def _layout(fn, cfg, wl, tb, tc, idx, keep, **kw):
 # (workload, token ranges): two calls in a row on different ranges (the second
 # reuses the array the first one left behind), then the first range again; the
 # second workload fills the array to its edge - 64 tiles of 256 tokens times
-# 1024 experts of look-back descriptors - and takes the scatter's shared-memory
+# 1024 experts of per-tile counts - and takes the scatter's shared-memory
 # opt-in beyond 48 KiB
 CASES = [
     (MoEWorkload("noalloc", T=2048, H=128, E=64, k=6, I=128, dtype="bf16", ep=4,
