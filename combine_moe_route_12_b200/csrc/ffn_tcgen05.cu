@@ -10,10 +10,10 @@
 //
 // Operands are swapped relative to the row-major product: the weights are the
 // M operand and the expert's tokens are the N operand, so a pair tile is
-// (expert, 256 weight rows, up to 256 tokens) and the token count is only
+// (expert, 256 weight rows, up to 288 tokens) and the token count is only
 // rounded up to the MMA's N granularity of 16: a ragged expert segment wastes
-// < 16 rows instead of up to 127, and each weight tile meets all (up to 256)
-// tokens of its expert while it sits in shared memory.  The pair's MMA keeps
+// < 16 rows instead of up to 127, and each weight tile meets all of its tile's
+// tokens while it sits in shared memory.  The pair's MMA keeps
 // 128 weight rows and half the tokens in each CTA's shared memory, which
 // halves the operand bytes each SM's shared memory must deliver per MMA;
 // with one CTA per MMA the shared memory (tile fills plus operand reads), not
@@ -25,22 +25,28 @@
 // through shared memory and each finishes h for half the tokens.
 //
 // CTA = 10 warps.  Warp 8 (one lane) of each CTA streams its weight and token
-// tiles with TMA into a ring of three 64 KiB stages of 128B-swizzled buffers,
+// tiles with TMA into a ring of three 68 KiB stages of 128B-swizzled buffers,
 // counting the bytes on the leader CTA's mbarrier.  A stage holds two 64-column
 // k-chunks and takes two TMA boxes: the weights (GEMM1: one 4-D box of 64 gate
-// rows and the 64 matching up rows) and 128 token rows.  Each TMA issue costs
+// rows and the 64 matching up rows) and 144 token rows.  Each TMA issue costs
 // the producer on the order of a hundred cycles whatever its size, so few large
 // boxes keep it ahead of the tensor pipe (token rows of a box past the tile's N
 // are loaded but never read by the MMA).  Warp 9 (one lane) of the leader
-// issues the pair's tcgen05.mma (bf16 -> fp32) into one of two 256-column TMEM
+// issues the pair's tcgen05.mma (bf16 -> fp32) into one of two 224-column TMEM
 // accumulator buffers and commits to both CTAs' barriers, so the epilogue of
-// tile i overlaps the main loop of tile i+1.  An expert with more than 256 rows
-// takes one tile per 256-token block; the tiles of one weight slice are dealt
-// back to back, so the later ones read the slice from L2.  The leader's
+// tile i overlaps the main loop of tile i+1.  Tiles cover an expert's rows 224
+// at a time, and its last tile takes up to 288: such a merged tile issues a
+// second MMA per k-step (N = 32 or 64, the same weights) into a 64-column extra
+// part of TMEM, so an expert of 225..288 rows streams its weights once instead
+// of twice.  The extra part is one buffer: the epilogue drains it first and
+// releases it on its own barrier, and the next merged tile's MMAs wait for
+// that.  An expert of more rows takes several tiles; the tiles of one weight
+// slice are dealt back to back, so the later ones read the slice from L2.  The leader's
 // producer takes tiles from a global counter, one ticket ahead, and publishes
 // them to both CTAs through a small mbarrier queue; warps 0-7 of each CTA
 // drain its TMEM (warps q and q+4 own lanes 32q..32q+31 and take alternate
-// 32-token chunks) and write h / y one token row at a time.  Tiles run expert
+// 32-column chunks, each two runs of 16 consecutive receive rows) and write
+// h / y one token row at a time.  Tiles run expert
 // by expert, weight block by weight block, token block innermost.
 //
 // Every mbarrier wait is bounded (2 s); a timeout raises MOE_DEV_WAIT_TIMEOUT,
@@ -56,17 +62,21 @@ constexpr int kBK = 64;                              // bf16 columns of one 128-
 constexpr int kBK8 = 128;                            // E4M3 columns of one 128-byte k-chunk
 constexpr int kKS = 2;                               // k-chunks per ring stage (one TMA box each)
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
-constexpr int kTileTok = 256;                        // tokens per tile (MMA N <= 256)
+constexpr int kTileTok = 224;                        // tokens of a tile's main part (MMA N <= 224)
+constexpr int kXTok = 64;                            // tokens of a merged tile's extra part (N = 32 or 64)
+constexpr int kTileMax = kTileTok + kXTok;           // an expert's last tile takes up to 288 tokens
+constexpr int kBoxRows = kTileTok / 2 + kXTok / 2;   // 144 token rows per CTA: main half, then extra half
 constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
 constexpr int kProdWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
 constexpr uint32_t kWBytes = kRowsPerCta * kBK * 2;         // 16 KiB: a CTA's weight rows of one k-chunk
-constexpr uint32_t kTokBytes = (kTileTok / 2) * kBK * 2;    // 16 KiB: a CTA's 128 token rows of one k-chunk
-constexpr uint32_t kStageBytes = kKS * (kWBytes + kTokBytes);  // 64 KiB
+constexpr uint32_t kTokBytes = kBoxRows * kBK * 2;           // 18 KiB: a CTA's 144 token rows of one k-chunk
+constexpr uint32_t kStageBytes = kKS * (kWBytes + kTokBytes);  // 68 KiB
 constexpr int kSmallBoxRows = 32;                            // token box of tiles with N <= 64
 constexpr int kStages = 3;
-constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 192 KiB
-constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulator buffers
+constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 204 KiB
+constexpr uint32_t kTmemCols = 512;                  // two 224-column accumulators + the 64-column extra part
+constexpr uint32_t kXCol = 2 * kTileTok;             // TMEM column of the extra part
 constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (4 warp pairs x 2 ways x 2 KiB)
 
 // Epilogues: the forward's SwiGLU (h), store (y) and decode reduce; the
@@ -109,6 +119,7 @@ struct FfnSmem {
     uint64_t empty[kStages];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
+    uint64_t x_empty;          // the extra part's columns drained (leader CTA)
     uint64_t mma_done;
     uint64_t q_full[kQueue];   // slice queue: published (count 1), per CTA
     uint64_t q_empty[kQueue];  // slice queue: read by every consumer (leader CTA only)
@@ -120,8 +131,21 @@ struct FfnSmem {
     int total_slices;      // tiles (the name is kept for the queue's work units)
 };
 
+// Token blocks of an expert with m rows: 224-token tiles, the last one taking up
+// to 288, so an expert of 225..288 rows streams its weights once.
+__device__ __forceinline__ int expert_tiles(int m) {
+    return m <= 0 ? 0 : m <= kTileMax ? 1 : (m - kXTok + kTileTok - 1) / kTileTok;
+}
+
+// A tile: n_valid <= 288 tokens from receive row p0.  n_main: the main MMA's N
+// (rounded to 16, <= 224); n_x: the extra MMA's N (0, 32 or 64), for a tile of
+// more than 224 tokens.  The pair's token rows: CTA 0 holds main columns
+// [0, n_main / 2) then extra columns [0, n_x / 2), CTA 1 the rest of both, each
+// in one box of consecutive receive rows: so main column j is receive row
+// p0 + j (+ n_x / 2 past CTA 0's half) and extra column j is p0 + 112 + j
+// (+ 112 past CTA 0's half).
 struct TileInfo {
-    int e, f_blk, p0, n_valid, n_mma;   // n_valid <= 256 tokens; n_mma: the MMA's N (rounded to 16)
+    int e, f_blk, p0, n_valid, n_main, n_x;
 };
 
 __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const FfnGemmParams &P) {
@@ -131,9 +155,57 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
     const int off = P.expert_offsets[e];
     const int m_e = P.expert_offsets[e + 1] - off;
     t.p0 = off + t_blk * kTileTok;
-    t.n_valid = min(kTileTok, m_e - t_blk * kTileTok);
-    t.n_mma = (t.n_valid + 15) & ~15;
+    t.n_valid = t_blk == expert_tiles(m_e) - 1 ? m_e - t_blk * kTileTok : kTileTok;
+    if (t.n_valid > kTileTok) {
+        t.n_main = kTileTok;
+        t.n_x = t.n_valid - kTileTok <= kXTok / 2 ? kXTok / 2 : kXTok;
+    } else {
+        t.n_main = (t.n_valid + 15) & ~15;
+        t.n_x = 0;
+    }
     return t;
+}
+
+// Epilogue chunk ch of a tile (32 TMEM columns; the extra part's chunks first):
+// its first TMEM column in the accumulator `acc`, and the receive rows (from
+// p0) of its two 16-column halves, each a run of consecutive rows.
+struct ChunkMap {
+    uint32_t tcol;
+    int rel_lo, rel_hi;
+};
+__device__ __forceinline__ int chunk_count(const TileInfo &ti) { return ti.n_x / 32 + (ti.n_main + 31) / 32; }
+__device__ __forceinline__ ChunkMap chunk_map(const TileInfo &ti, int ch, int acc) {
+    ChunkMap m;
+    const int nxc = ti.n_x / 32;
+    if (ch < nxc) {
+        const int j = 32 * ch;
+        m.tcol = kXCol + (uint32_t)j;
+        m.rel_lo = j < ti.n_x / 2 ? kTileTok / 2 + j : kTileTok + j;
+        m.rel_hi = j + 16 < ti.n_x / 2 ? kTileTok / 2 + j + 16 : kTileTok + j + 16;
+    } else {
+        const int j = 32 * (ch - nxc);
+        m.tcol = (uint32_t)(acc * kTileTok + j);
+        m.rel_lo = j < ti.n_main / 2 ? j : j + ti.n_x / 2;
+        m.rel_hi = j + 16 < ti.n_main / 2 ? j + 16 : j + 16 + ti.n_x / 2;
+    }
+    return m;
+}
+__device__ __forceinline__ int chunk_rel(const ChunkMap &m, int j) { return j < 16 ? m.rel_lo + j : m.rel_hi + j - 16; }
+
+// Tile number -> (expert, feature block, token block); s_tpre[e] is the first
+// tile of expert e, which owns tb(e) * n_fblocks tiles.
+__device__ __forceinline__ void decode_tile_pre(int tile, const int32_t *s_tpre, int E, int n_fblocks,
+                                                int &e, int &f_blk, int &t_blk) {
+    int lo = 0, hi = E - 1;  // last e with s_tpre[e] <= tile (it owns >= 1 tile)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_tpre[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    const int local = tile - s_tpre[lo];
+    const int tb = (s_tpre[lo + 1] - s_tpre[lo]) / n_fblocks;
+    f_blk = local / tb;
+    t_blk = local - f_blk * tb;
 }
 
 // A UE8M0 scale byte as a float: 2^(b - 127) (b = 0 gives the subnormal 2^-127).
@@ -203,7 +275,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
     float *xchg = reinterpret_cast<float *>(base + kRingBytes);   // GEMM1 only
     FfnSmem *S = reinterpret_cast<FfnSmem *>(base + kRingBytes + (kSwiGLU ? kXchgBytes : 0));
     int32_t *s_tpre = reinterpret_cast<int32_t *>(S + 1);   // [E + 1] tile prefix
-    int32_t *s_tb = s_tpre + (P.E + 1);                       // [E] token blocks per expert
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();                  // 0: leader (issues the MMA)
@@ -214,11 +285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
         for (int e0 = 0; e0 < P.E; e0 += 32) {
             const int e = e0 + lane;
             int tb = 0;
-            if (e < P.E) {
-                const int m = P.expert_offsets[e + 1] - P.expert_offsets[e];
-                tb = (m + kTileTok - 1) / kTileTok;
-                s_tb[e] = tb;
-            }
+            if (e < P.E) tb = expert_tiles(P.expert_offsets[e + 1] - P.expert_offsets[e]);
             const int t = tb * P.n_fblocks;
             int incl = t;
 #pragma unroll
@@ -237,6 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             mbar_init(&S->tmem_full[a], 1);
             mbar_init(&S->tmem_empty[a], 2 * kEpiWarps);   // every epilogue warp of both CTAs
         }
+        mbar_init(&S->x_empty, 2 * kEpiWarps);
         for (int i = 0; i < kQueue; ++i) { mbar_init(&S->q_full[i], 1); mbar_init(&S->q_empty[i], kQueueConsumers); }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
@@ -290,16 +358,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 if (!next_slice(slice)) { ok = false; break; }
                 if (slice < 0) break;
                 int se, sf, t_blk;
-                decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
+                decode_tile_pre(slice, s_tpre, P.E, P.n_fblocks, se, sf, t_blk);
                 // this CTA's weight rows: GEMM1 64 gate rows + the matching 64 up rows
                 // (one 4-D box), GEMM2 128 rows; its token rows: half of the tile's N
                 const int f_row = (sf * 2 + (int)rank) * P.feat_per_cta;
                 const int w_row = se * P.w_rows_per_expert + f_row;
                 const TileInfo ti = tile_info(se, sf, t_blk, P);
-                const int tok_row = ti.p0 + (int)rank * (ti.n_mma / 2);
+                const int tok_row = ti.p0 + (int)rank * (ti.n_main / 2 + ti.n_x / 2);
                 // a tile of an expert's short last token block takes a 32-row token box:
                 // fewer bytes through L2 for the same stage slot
-                const bool small_box = ti.n_mma / 2 <= kSmallBoxRows;
+                const bool small_box = ti.n_x == 0 && ti.n_main / 2 <= kSmallBoxRows;
                 const uint32_t stage_bytes = small_box ? kKS * (kWBytes + kSmallBoxRows * kBK * 2) : kStageBytes;
                 for (int kb = 0; kb < num_k; ++kb) {
                     if (!mbar_wait_bounded(&S->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -343,6 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 uint32_t phase = 0;
                 int acc = 0;
                 uint32_t acc_phase = 0;
+                uint32_t x_phase = 0;
                 bool ok = true;
                 SliceReader reader;
                 int slice;
@@ -350,33 +419,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                   if (!reader.next(S, abort_flag, true, slice)) { ok = false; break; }
                   if (slice < 0) break;
                   int se, sf, t_blk;
-                  decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
+                  decode_tile_pre(slice, s_tpre, P.E, P.n_fblocks, se, sf, t_blk);
                   {
                     const TileInfo ti = tile_info(se, sf, t_blk, P);
-                    const uint32_t idesc = F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_mma)
-                                              : make_idesc_bf16_f32_major(2 * kRowsPerCta, ti.n_mma, A_MN, false);
+                    const uint32_t idesc = F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_main)
+                                              : make_idesc_bf16_f32_major(2 * kRowsPerCta, ti.n_main, A_MN, false);
+                    const bool merged = ti.n_x > 0;
+                    const uint32_t idesc_x = !merged ? 0u
+                                             : F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_x)
+                                                  : make_idesc_bf16_f32_major(2 * kRowsPerCta, ti.n_x, A_MN, false);
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+                    // the extra part's columns: drained by the previous merged tile's epilogue
+                    if (merged) {
+                        if (!mbar_wait_bounded(&S->x_empty, x_phase ^ 1u, abort_flag)) { ok = false; break; }
+                        x_phase ^= 1u;
+                    }
                     tc_fence_after();
                     const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
-                    // k-chunk stride inside the stage's token box (32 or 128 rows)
-                    const uint32_t tchunk = ti.n_mma / 2 <= kSmallBoxRows ? kSmallBoxRows * kBK * 2 : kTokBytes;
+                    const uint32_t dx = tmem_base + kXCol;
+                    // k-chunk stride inside the stage's token box (32 or 144 rows); the
+                    // extra part's rows follow the main half's in both CTAs
+                    const bool small_box = ti.n_x == 0 && ti.n_main / 2 <= kSmallBoxRows;
+                    const uint32_t tchunk = small_box ? kSmallBoxRows * kBK * 2 : kTokBytes;
+                    constexpr uint32_t kXRowOff = (kTileTok / 2) * 128;   // 112 rows of 128 bytes
                     for (int kb = 0; kb < num_k; ++kb) {
                         if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t st = smem_u32(tiles + stage * kStageBytes);
+                        // the stage's main MMAs, then its extra-part MMAs: consecutive MMAs
+                        // into the same accumulator
 #pragma unroll
-                        for (int c = 0; c < kKS; ++c) {
+                        for (int part = 0; part < 2; ++part) {
+                            if (part == 1 && !merged) break;
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {   // 32-byte k-steps: 16 bf16 or 32 E4M3
-                                // MN-major: k-chunk c is rows 64c.. of each 64-feature block
-                                // (blocks 16 KiB apart), a k-step 16 rows of 128 bytes
-                                const uint64_t wdesc = A_MN
-                                    ? make_sw128_desc_mn(st + c * (kWBytes / 2) + kk * 2048, kWBytes)
-                                    : make_sw128_desc(st + c * kWBytes + kk * 32);
-                                const uint64_t tdesc = make_sw128_desc(st + kKS * kWBytes + c * tchunk + kk * 32);
-                                const uint32_t accum = (kb > 0 || c > 0 || kk > 0) ? 1u : 0u;
-                                if (F8) tc_mma_f8_pair(d, wdesc, tdesc, idesc, accum);
-                                else tc_mma_f16_pair(d, wdesc, tdesc, idesc, accum);
+                            for (int c = 0; c < kKS; ++c) {
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk) {   // 32-byte k-steps: 16 bf16 or 32 E4M3
+                                    // MN-major: k-chunk c is rows 64c.. of each 64-feature block
+                                    // (blocks 16 KiB apart), a k-step 16 rows of 128 bytes
+                                    const uint64_t wdesc = A_MN
+                                        ? make_sw128_desc_mn(st + c * (kWBytes / 2) + kk * 2048, kWBytes)
+                                        : make_sw128_desc(st + c * kWBytes + kk * 32);
+                                    const uint32_t taddr = st + kKS * kWBytes + c * tchunk + kk * 32 +
+                                                           (part ? kXRowOff : 0u);
+                                    const uint64_t tdesc = make_sw128_desc(taddr);
+                                    const uint32_t accum = (kb > 0 || c > 0 || kk > 0) ? 1u : 0u;
+                                    if (F8) tc_mma_f8_pair(part ? dx : d, wdesc, tdesc, part ? idesc_x : idesc, accum);
+                                    else tc_mma_f16_pair(part ? dx : d, wdesc, tdesc, part ? idesc_x : idesc, accum);
+                                }
                             }
                         }
                         tc_commit_pair_mc(&S->empty[stage], 0x3);   // frees the stage in both CTAs
@@ -409,6 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
         const int xpair = half * 2 + (q & 1);                 // gate/up warp pair (GEMM1)
         const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
                                           mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
+        const uint32_t x_empty_leader = mapa_shared(smem_u32(&S->x_empty), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
         SliceReader reader;
@@ -433,30 +524,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
           }
           if (slice < 0) break;
           int se, sf, t_blk;
-          decode_tile(slice, s_tpre, s_tb, P.E, se, sf, t_blk);
+          decode_tile_pre(slice, s_tpre, P.E, P.n_fblocks, se, sf, t_blk);
           {
            const TileInfo ti = tile_info(se, sf, t_blk, P);
            const int f = (ti.f_blk * 2 + (int)rank) * P.feat_per_cta + feat_lane;  // output feature
            const bool f_ok = f < P.out_cols;
-           // FP8: this lane's weight-row scale, and the token scales of the warp's
-           // 32-token chunks (token half*32 + 64i + lane in chunk i), loaded before
+           // FP8: this lane's weight-row scale, and the token scale of column `lane`
+           // of each of the warp's chunks (chunks half, half + 2, ...), loaded before
            // the accumulator wait so that their latency hides behind it
-           float wsc = 1.0f, tsc0 = 1.0f, tsc1 = 1.0f, tsc2 = 1.0f, tsc3 = 1.0f;
+           const int nch = chunk_count(ti);
+           const int nxc = ti.n_x / 32;
+           float wsc = 1.0f;
+           float tsc[5] = {1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
            if (F8) {
                if (f_ok)
                    wsc = ue8m0_value(P.w_scale[(size_t)ti.e * P.w_rows_per_expert +
                                                (kGateUp && !is_gate ? P.out_cols : 0) + f]);
-               float t4[4];
 #pragma unroll
-               for (int i = 0; i < 4; ++i) {
-                   const int c = half * 32 + 64 * i + lane;
-                   t4[i] = 1.0f;
-                   if (c < ti.n_valid) {
-                       const int p = ti.p0 + c;
-                       t4[i] = ue8m0_value(P.t_scale[P.t_scale_by_token ? P.recv_token[p] : p]);
+               for (int i = 0; i < 5; ++i) {
+                   const int ch = half + 2 * i;
+                   if (ch < nch) {
+                       const int rel = chunk_rel(chunk_map(ti, ch, 0), lane);
+                       if (rel < ti.n_valid) {
+                           const int p = ti.p0 + rel;
+                           tsc[i] = ue8m0_value(P.t_scale[P.t_scale_by_token ? P.recv_token[p] : p]);
+                       }
                    }
                }
-               tsc0 = t4[0]; tsc1 = t4[1]; tsc2 = t4[2]; tsc3 = t4[3];
            }
            do {   // one pass; `break` leaves it on a failed wait
             bool go;
@@ -477,25 +571,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 break;
             }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (uint32_t)(acc * kTileTok) + ((uint32_t)(q * 32) << 16);
+            const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
+            // a warp with no chunk of the extra part releases it at once
+            if (nxc > 0 && half >= nxc) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(x_empty_leader);
+            }
 
             int ci = 0;
-            for (int c0 = half * 32; c0 < ti.n_mma; c0 += 64, ++ci) {
+            for (int ch = half; ch < nch; ch += 2, ++ci) {
+                const ChunkMap cm = chunk_map(ti, ch, acc);
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tbase + c0, r);
+                tmem_ld_32x32b_x32(tlane + cm.tcol, r);
                 tc_wait_ld_regs(r);
-                // FP8: the scale of token c0 + lane
-                const float ts_lane = ci == 0 ? tsc0 : ci == 1 ? tsc1 : ci == 2 ? tsc2 : tsc3;
+                if (ch < nxc) {   // the extra part's columns are in registers: release them
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(x_empty_leader);
+                }
+                // FP8: the scale of the token in column `lane`
+                const float ts_lane = ci == 0 ? tsc[0] : ci == 1 ? tsc[1] : ci == 2 ? tsc[2] : ci == 3 ? tsc[3] : tsc[4];
+                // rows of the two 16-column halves, and how many of each are tokens
+                const int nc_lo = min(16, ti.n_valid - cm.rel_lo), nc_hi = min(16, ti.n_valid - cm.rel_hi);
                 if (kSwiGLU) {
-                    // exchange: gate warps hand over tokens 16..31, up warps tokens 0..15
+                    // exchange: gate warps hand over columns 16..31, up warps columns 0..15
                     float *mine = xchg + (xpair * 2 + (is_gate ? 0 : 1)) * 512;
                     float *theirs = xchg + (xpair * 2 + (is_gate ? 1 : 0)) * 512;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         mine[j * 32 + lane] = __uint_as_float(r[is_gate ? 16 + j : j]) * (F8 ? wsc : 1.0f);
                     named_barrier_sync(1 + xpair, 64);
-                    const int cbase = c0 + (is_gate ? 0 : 16);
-                    const int nc = min(16, ti.n_valid - cbase);
+                    const int cbase = is_gate ? cm.rel_lo : cm.rel_hi;
+                    const int nc = is_gate ? nc_lo : nc_hi;
                     // all 16 partner values into registers before the first store:
                     // h and the exchange buffer are both generic pointers, so a load
                     // after a store could not be moved ahead of it and every token
@@ -533,43 +640,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     // the gate value of feature f to column f, the up value to column I + f
                     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld +
                                        f + (is_gate ? 0 : P.half_cols);
-                    const int nc = min(32, ti.n_valid - c0);
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (f_ok && j < nc) o[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                        if (f_ok && (j < 16 ? j < nc_lo : j - 16 < nc_hi))
+                            o[(size_t)chunk_rel(cm, j) * P.out_ld] = __float2bfloat16_rn(__uint_as_float(r[j]));
                 } else if (MODE == kEpiSwiGLUBwd) {
                     // r = dh of feature f for 32 tokens; with s = sigmoid(g):
                     //   h = g s u,  dg = dh u s (1 + g (1 - s)),  du = dh g s
-                    const int nc = min(32, ti.n_valid - c0);
-                    const size_t row0 = (size_t)(ti.p0 + c0);
                     float g[32], u[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         g[j] = 0.0f;
                         u[j] = 0.0f;
-                        if (f_ok && j < nc) {
-                            const __nv_bfloat16 *gr = P.gu + (row0 + j) * P.out_ld + f;
+                        if (f_ok && (j < 16 ? j < nc_lo : j - 16 < nc_hi)) {
+                            const __nv_bfloat16 *gr = P.gu + (size_t)(ti.p0 + chunk_rel(cm, j)) * P.out_ld + f;
                             g[j] = __bfloat162float(gr[0]);
                             u[j] = __bfloat162float(gr[P.half_cols]);
                         }
                     }
-                    __nv_bfloat16 *ho = static_cast<__nv_bfloat16 *>(P.out) + row0 * P.out_cols + f;
-                    __nv_bfloat16 *dgo = P.out2 + row0 * P.out_ld + f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float dh = __uint_as_float(r[j]);
                         const float sg = __fdividef(1.0f, 1.0f + __expf(-g[j]));
                         const float sl = g[j] * sg;
-                        if (f_ok && j < nc) {
-                            ho[(size_t)j * P.out_cols] = __float2bfloat16_rn(sl * u[j]);
-                            dgo[(size_t)j * P.out_ld] =
-                                __float2bfloat16_rn(dh * u[j] * sg * (1.0f + g[j] * (1.0f - sg)));
-                            dgo[(size_t)j * P.out_ld + P.half_cols] = __float2bfloat16_rn(dh * sl);
+                        if (f_ok && (j < 16 ? j < nc_lo : j - 16 < nc_hi)) {
+                            const size_t row = (size_t)(ti.p0 + chunk_rel(cm, j));
+                            static_cast<__nv_bfloat16 *>(P.out)[row * P.out_cols + f] = __float2bfloat16_rn(sl * u[j]);
+                            __nv_bfloat16 *dgo = P.out2 + row * P.out_ld + f;
+                            dgo[0] = __float2bfloat16_rn(dh * u[j] * sg * (1.0f + g[j] * (1.0f - sg)));
+                            dgo[P.half_cols] = __float2bfloat16_rn(dh * sl);
                         }
                     }
                 } else if (MODE == kEpiStore) {
                     // one 64-byte warp store per token row (the shuffle rearrangement
-                    // of the SwiGLU epilogue measured slower here)
+                    // of the SwiGLU epilogue measured slower here), down a running row
+                    // pointer that restarts at the second half's first row
+                    __nv_bfloat16 *const out = static_cast<__nv_bfloat16 *>(P.out);
                     if (F8) {
                         // each token's scale from the lane that loaded it, times this
                         // lane's weight-row scale, all taken before the stores
@@ -577,26 +683,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             v[j] = __uint_as_float(r[j]) * (__shfl_sync(0xffffffffu, ts_lane, j) * wsc);
-                        const int nc = f_ok ? min(32, ti.n_valid - c0) : 0;
-                        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)(ti.p0 + c0) * P.out_ld + f;
+                        const int lo = f_ok ? nc_lo : 0, hi = f_ok ? nc_hi : 0;
+                        __nv_bfloat16 *y = out + (size_t)(ti.p0 + cm.rel_lo) * P.out_ld + f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            if (j < nc) *y = __float2bfloat16_rn(v[j]);
+                            if (j == 16) y = out + (size_t)(ti.p0 + cm.rel_hi) * P.out_ld + f;
+                            if (j < 16 ? j < lo : j - 16 < hi) *y = __float2bfloat16_rn(v[j]);
                             y += P.out_ld;
                         }
                     } else {
-                        __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(P.out) + (size_t)ti.p0 * P.out_ld + f;
-                        const int nc = min(32, ti.n_valid - c0);
+                        __nv_bfloat16 *y = out + (size_t)(ti.p0 + cm.rel_lo) * P.out_ld + f;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (f_ok && j < nc) y[(size_t)(c0 + j) * P.out_ld] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                        for (int j = 0; j < 32; ++j) {
+                            if (j == 16) y = out + (size_t)(ti.p0 + cm.rel_hi) * P.out_ld + f;
+                            if (f_ok && (j < 16 ? j < nc_lo : j - 16 < nc_hi))
+                                *y = __float2bfloat16_rn(__uint_as_float(r[j]));
+                            y += P.out_ld;
+                        }
                     }
                 } else {  // kEpiReduce: out_reduce[t] += w * y, one token column at a time
                     int my_t = 0;
                     float my_w = 0.0f;
-                    const int nc = min(32, ti.n_valid - c0);
-                    if (lane < nc) {
-                        const int p = ti.p0 + c0 + lane;
+                    const bool tok_ok = lane < 16 ? lane < nc_lo : lane - 16 < nc_hi;
+                    if (tok_ok) {
+                        const int p = ti.p0 + chunk_rel(cm, lane);
                         my_t = P.recv_token[p];
                         my_w = P.topk_w[(size_t)my_t * P.k + P.recv_slot[p]];
                         if (F8) my_w *= ts_lane;
@@ -605,7 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                     for (int j = 0; j < 32; ++j) {
                         const int t = __shfl_sync(0xffffffffu, my_t, j);
                         const float w = __shfl_sync(0xffffffffu, my_w, j);
-                        if (j < nc && f_ok)
+                        if ((j < 16 ? j < nc_lo : j - 16 < nc_hi) && f_ok)
                             atomicAdd(P.out_reduce + (size_t)t * P.out_cols + f,
                                       w * (__uint_as_float(r[j]) * (F8 ? wsc : 1.0f)));
                     }
@@ -682,7 +792,7 @@ static bool make_tmap_w13(CUtensorMap *m, const void *ptr, uint64_t E, uint64_t 
 
 size_t ffn_tcgen05_smem(int E, bool swiglu) {
     return 1024 + (size_t)kRingBytes + (swiglu ? kXchgBytes : 0) + sizeof(FfnSmem) +
-           sizeof(int32_t) * (2 * (size_t)E + 1) + 64;
+           sizeof(int32_t) * ((size_t)E + 1) + 64;
 }
 
 template <int MODE, bool F8, bool A_MN = false>
@@ -726,7 +836,7 @@ static void ffn_params(const moe_config &c, const int32_t *expert_offsets, void 
     P2.topk_w = topk_w;
 }
 
-// CTA pairs: an upper bound on the pair tiles is (n_rows / 256 + E) * n_fblocks
+// CTA pairs: an upper bound on the pair tiles is (n_rows / 224 + E) * n_fblocks
 static int ffn_grid(const moe_config &c, int64_t n_rows, const FfnGemmParams &P, int num_sms) {
     const long long max_pairs = num_sms / 2;
     const long long g = (n_rows / kTileTok + c.E) * (long long)P.n_fblocks;
@@ -748,9 +858,9 @@ cudaError_t launch_ffn_tcgen05(const moe_config &c, int64_t n_rows, const void *
         !make_tmap_rows(&tx2s, h, (uint64_t)n_rows, (uint64_t)c.I, kSmallBoxRows))
         return cudaErrorNotSupported;
     if (!make_tmap_w13(&tw1, w13, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H) ||
-        !make_tmap_rows(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kTileTok / 2) ||
+        !make_tmap_rows(&tx1, xr, (uint64_t)n_rows, (uint64_t)c.H, kBoxRows) ||
         !make_tmap_rows(&tw2, w2, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta) ||
-        !make_tmap_rows(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kTileTok / 2))
+        !make_tmap_rows(&tx2, h, (uint64_t)n_rows, (uint64_t)c.I, kBoxRows))
         return cudaErrorNotSupported;
 
     FfnGemmParams P1, P2;
@@ -796,10 +906,10 @@ cudaError_t launch_ffn_tcgen05_dgrad(const moe_config &c, int64_t n_rows, const 
     if (cerr != cudaSuccess) return cerr;
     const uint64_t H = c.H, I = c.I, E = c.E, n = (uint64_t)n_rows;
     CUtensorMap tw13, tx, txs, tw2t, tdy, tdys, tw13t, tdgu, tdgus;
-    if (!make_tmap_w13(&tw13, w13, E, I, H) || !make_tmap_rows(&tx, xr, n, H, kTileTok / 2) ||
+    if (!make_tmap_w13(&tw13, w13, E, I, H) || !make_tmap_rows(&tx, xr, n, H, kBoxRows) ||
         !make_tmap_rows(&txs, xr, n, H, kSmallBoxRows) || !make_tmap_mn(&tw2t, w2, E * H, I) ||
-        !make_tmap_rows(&tdy, dy, n, H, kTileTok / 2) || !make_tmap_rows(&tdys, dy, n, H, kSmallBoxRows) ||
-        !make_tmap_mn(&tw13t, w13, E * 2 * I, H) || !make_tmap_rows(&tdgu, dgu, n, 2 * I, kTileTok / 2) ||
+        !make_tmap_rows(&tdy, dy, n, H, kBoxRows) || !make_tmap_rows(&tdys, dy, n, H, kSmallBoxRows) ||
+        !make_tmap_mn(&tw13t, w13, E * 2 * I, H) || !make_tmap_rows(&tdgu, dgu, n, 2 * I, kBoxRows) ||
         !make_tmap_rows(&tdgus, dgu, n, 2 * I, kSmallBoxRows))
         return cudaErrorNotSupported;
 
@@ -899,9 +1009,9 @@ cudaError_t launch_ffn_tcgen05_fp8(const moe_config &c, int64_t n_rows, const ui
     if (!make_tmap_rows(&tx1s, xr_q, (uint64_t)n_rows, (uint64_t)c.H, kSmallBoxRows, true) ||
         !make_tmap_rows(&tx2s, h_q, (uint64_t)n_rows, (uint64_t)c.I, kSmallBoxRows, true) ||
         !make_tmap_w13(&tw1, w13_q, (uint64_t)c.E, (uint64_t)c.I, (uint64_t)c.H, true) ||
-        !make_tmap_rows(&tx1, xr_q, (uint64_t)n_rows, (uint64_t)c.H, kTileTok / 2, true) ||
+        !make_tmap_rows(&tx1, xr_q, (uint64_t)n_rows, (uint64_t)c.H, kBoxRows, true) ||
         !make_tmap_rows(&tw2, w2_q, (uint64_t)c.E * c.H, (uint64_t)c.I, kRowsPerCta, true) ||
-        !make_tmap_rows(&tx2, h_q, (uint64_t)n_rows, (uint64_t)c.I, kTileTok / 2, true))
+        !make_tmap_rows(&tx2, h_q, (uint64_t)n_rows, (uint64_t)c.I, kBoxRows, true))
         return cudaErrorNotSupported;
     FfnGemmParams P1, P2;
     ffn_params(c, expert_offsets, h, y, recv_token, recv_slot, topk_w, out_reduce, status, P1, P2);
