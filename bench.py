@@ -55,20 +55,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": (941.411328 + 48.232192 + 453.837312 + 115.365120) * 1e6,
-                      "src": "a15a55f4109395c7"},
+    "qwen3_30b_a3b": {"bytes": (943.448832 + 46.416640 + 453.957120 + 113.494784) * 1e6,
+                      "src": "ae304e0a3accf960"},
     # both GEMM launches and the quantisation of h between them
-    "qwen3_30b_a3b_fp8": {"bytes": (470.987520 + 44.082688 + 50.341376 + 1.413888 + 227.298304 +
-                                    102.075648) * 1e6, "src": "67604f868e3e8b13"},
-    "qwen3_30b_a3b_mxfp8": {"bytes": (484.921344 + 24.599296 + 233.696768 + 106.839296) * 1e6,
-                            "src": "32d5db20d0508550"},
+    "qwen3_30b_a3b_fp8": {"bytes": (471.292416 + 41.976832 + 50.341376 + 1.413888 + 226.893056 +
+                                    97.778688) * 1e6, "src": "f7a63551cfc9ed2a"},
+    "qwen3_30b_a3b_mxfp8": {"bytes": (484.897024 + 24.313600 + 233.751296 + 105.241344) * 1e6,
+                            "src": "f91c44b09b122286"},
     # captured with 32 of the 256 experts and 1024 tokens (the same 128 rows per
     # expert and chunk), scaled by 8 per chunk, two chunks; see
     # profiles/ffn_tcgen05_dsv3_prefill.md and profiles/ffn_mx_tcgen05_dsv3_prefill_mxfp8.md
-    "dsv3_prefill": {"bytes": 2 * 8 * (1955.436e6 + 18.376e6 + 957.506e6 + 54.893e6),
-                     "src": "a15a55f4109395c7", "chunks": 2},
-    "dsv3_prefill_mxfp8": {"bytes": 2 * 8 * (1008.788e6 + 11.774e6 + 494.242e6 + 50.586e6),
-                           "src": "32d5db20d0508550", "chunks": 2},
+    "dsv3_prefill": {"bytes": 2 * 8 * (1956.813568e6 + 18.363648e6 + 958.455040e6 + 55.145984e6),
+                     "src": "ae304e0a3accf960", "chunks": 2},
+    "dsv3_prefill_mxfp8": {"bytes": 2 * 8 * (1008.328192e6 + 11.598080e6 + 494.208000e6 + 49.762304e6),
+                           "src": "f91c44b09b122286", "chunks": 2},
 }
 
 
