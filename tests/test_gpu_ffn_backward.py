@@ -6,9 +6,9 @@ The backward of the grouped SwiGLU FFN is the gradient of step 5's function
 expert GEMMs under activation checkpointing); the oracle's form of it is pinned
 by central finite differences of the forward oracle.  Cases span ragged expert
 segments (empty, one row, fewer than one 16-row MMA step, more than one
-256-token tile, an exact ring stage), feature and hidden sizes that are not
-multiples of a 128-row tile, and the fp32 path.  Tolerances: fp32 max-abs 1e-4,
-bf16 max|a-b| / max|ref| <= 2e-2 per tensor.
+token tile, an exact ring stage, every edge of the tiling's merged last tile),
+feature and hidden sizes that are not multiples of a 128-row tile, and the fp32
+path.  Tolerances: fp32 max-abs 1e-4, bf16 max|a-b| / max|ref| <= 2e-2 per tensor.
 """
 import numpy as np
 import pytest
@@ -27,6 +27,9 @@ CASES = [
     ("bf16_ragged", "bf16", 256, 256, [0, 1, 15, 17, 128, 129, 300, 40]),
     ("bf16_partial_tiles", "bf16", 192, 192, [5, 300, 0, 77]),
     ("bf16_wide", "bf16", 512, 128, [250, 3, 0, 511, 16, 33, 260, 127, 64, 1, 0, 190, 129, 255, 18, 70]),
+    # the token tiling's edges: 224-token tiles, the last one of up to 288 tokens
+    # through a second MMA (N = 32 / 64), merged tiles back to back
+    ("bf16_tile_edges", "bf16", 256, 128, [224, 225, 240, 241, 256, 257, 288, 289, 0, 449, 513, 288, 288, 257]),
 ]
 
 
