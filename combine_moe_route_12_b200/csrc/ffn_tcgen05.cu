@@ -32,17 +32,18 @@
 // the producer on the order of a hundred cycles whatever its size, so few large
 // boxes keep it ahead of the tensor pipe (token rows of a box past the tile's N
 // are loaded but never read by the MMA).  Warp 9 (one lane) of the leader
-// issues the pair's tcgen05.mma (bf16 -> fp32) into one of two 224-column TMEM
-// accumulator buffers and commits to both CTAs' barriers, so the epilogue of
-// tile i overlaps the main loop of tile i+1.  Tiles cover an expert's rows 224
-// at a time, and its last tile takes up to 288: such a merged tile issues a
-// second MMA per k-step (N = 32 or 64, the same weights) into a 64-column extra
-// part of TMEM, so an expert of 225..288 rows streams its weights once instead
-// of twice.  The extra part is one buffer: the epilogue drains it first and
-// releases it on its own barrier, and the next merged tile's MMAs wait for
-// that.  An expert of more rows takes several tiles; the tiles of one weight
-// slice are dealt back to back, so the later ones read the slice from L2.  The leader's
-// producer takes tiles from a global counter, one ticket ahead, and publishes
+// issues the pair's tcgen05.mma (bf16 -> fp32) into one of two TMEM accumulators
+// and commits to both CTAs' barriers, so the epilogue of tile i overlaps the main
+// loop of tile i+1.  Tiles cover an expert's rows 256 at a time, and its last tile
+// takes up to 288.  Each accumulator owns 224 TMEM columns, and the 64 between them
+// are two halves of a shared part: a main MMA of more than 224 tokens extends into
+// its accumulator's adjacent half, and a tile of more than 256 tokens issues a
+// second MMA per k-step (N = 32, the same weights) into the other half, so an
+// expert of up to 288 rows streams its weights once.  Each half has its own
+// barrier: the epilogue drains the chunks that hold a half first and releases it,
+// and the next tile that writes it waits for that.  An expert of more rows takes
+// several tiles; the tiles of one weight slice are dealt back to back, so the
+// later ones read the slice from L2.  The leader's producer takes tiles from a global counter, one ticket ahead, and publishes
 // them to both CTAs through a small mbarrier queue; warps 0-7 of each CTA
 // drain its TMEM (warps q and q+4 own lanes 32q..32q+31 and take alternate
 // 32-column chunks, each two runs of 16 consecutive receive rows) and write
@@ -62,10 +63,11 @@ constexpr int kBK = 64;                              // bf16 columns of one 128-
 constexpr int kBK8 = 128;                            // E4M3 columns of one 128-byte k-chunk
 constexpr int kKS = 2;                               // k-chunks per ring stage (one TMA box each)
 constexpr int kRowsPerCta = 128;                     // weight rows (MMA M / 2) per CTA
-constexpr int kTileTok = 224;                        // tokens of a tile's main part (MMA N <= 224)
-constexpr int kXTok = 64;                            // tokens of a merged tile's extra part (N = 32 or 64)
-constexpr int kTileMax = kTileTok + kXTok;           // an expert's last tile takes up to 288 tokens
-constexpr int kBoxRows = kTileTok / 2 + kXTok / 2;   // 144 token rows per CTA: main half, then extra half
+constexpr int kSlotCols = 224;                       // TMEM columns each accumulator owns outright
+constexpr int kXHalf = 32;                           // TMEM columns of each half of the shared part
+constexpr int kTileTok = kSlotCols + kXHalf;         // 256: tokens of a tile's main MMA (N <= 256)
+constexpr int kTileMax = kTileTok + kXHalf;          // an expert's last tile takes up to 288 tokens
+constexpr int kBoxRows = kTileTok / 2 + kXHalf / 2;  // 144 token rows per CTA: main half, then extra half
 constexpr int kEpiWarps = 8;                         // two per TMEM lane quadrant
 constexpr int kProdWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kFfnThreads = 32 * (kEpiWarps + 2);
@@ -75,8 +77,12 @@ constexpr uint32_t kStageBytes = kKS * (kWBytes + kTokBytes);  // 68 KiB
 constexpr int kSmallBoxRows = 32;                            // token box of tiles with N <= 64
 constexpr int kStages = 3;
 constexpr uint32_t kRingBytes = kStages * kStageBytes;       // 204 KiB
-constexpr uint32_t kTmemCols = 512;                  // two 224-column accumulators + the 64-column extra part
-constexpr uint32_t kXCol = 2 * kTileTok;             // TMEM column of the extra part
+// TMEM: accumulator 0 owns [0, 224), half a of the shared part is [224, 256), half b
+// [256, 288), accumulator 1 owns [288, 512).  A main MMA of more than 224 tokens
+// takes its accumulator's adjacent half (0: [0, 256), 1: [256, 512)); a tile of
+// more than 256 tokens puts its extra 32 columns in the other half.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kXCol = kSlotCols;                // half a; half b follows
 constexpr uint32_t kXchgBytes = 16 * 1024;           // GEMM1 gate/up exchange (4 warp pairs x 2 ways x 2 KiB)
 
 // Epilogues: the forward's SwiGLU (h), store (y) and decode reduce; the
@@ -119,7 +125,7 @@ struct FfnSmem {
     uint64_t empty[kStages];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
-    uint64_t x_empty;          // the extra part's columns drained (leader CTA)
+    uint64_t x_empty[2];       // a half of the shared part drained (leader CTA): a, b
     uint64_t mma_done;
     uint64_t q_full[kQueue];   // slice queue: published (count 1), per CTA
     uint64_t q_empty[kQueue];  // slice queue: read by every consumer (leader CTA only)
@@ -131,19 +137,19 @@ struct FfnSmem {
     int total_slices;      // tiles (the name is kept for the queue's work units)
 };
 
-// Token blocks of an expert with m rows: 224-token tiles, the last one taking up
-// to 288, so an expert of 225..288 rows streams its weights once.
+// Token blocks of an expert with m rows: 256-token tiles, the last one taking up to
+// 288, so an expert of up to 288 rows streams its weights once.
 __device__ __forceinline__ int expert_tiles(int m) {
-    return m <= 0 ? 0 : m <= kTileMax ? 1 : (m - kXTok + kTileTok - 1) / kTileTok;
+    return m <= 0 ? 0 : m <= kTileMax ? 1 : (m - kXHalf + kTileTok - 1) / kTileTok;
 }
 
-// A tile: n_valid <= 288 tokens from receive row p0.  n_main: the main MMA's N
-// (rounded to 16, <= 224); n_x: the extra MMA's N (0, 32 or 64), for a tile of
-// more than 224 tokens.  The pair's token rows: CTA 0 holds main columns
-// [0, n_main / 2) then extra columns [0, n_x / 2), CTA 1 the rest of both, each
-// in one box of consecutive receive rows: so main column j is receive row
-// p0 + j (+ n_x / 2 past CTA 0's half) and extra column j is p0 + 112 + j
-// (+ 112 past CTA 0's half).
+// A tile: n_valid <= 288 tokens from receive row p0.  n_main: the main MMA's N (the
+// token count rounded to 16, or 256 past 224 tokens); n_x: the extra MMA's N, 32 for
+// a tile of more than 256 tokens, else 0.  The pair's token rows: CTA 0 holds main
+// columns [0, n_main / 2) then extra columns [0, n_x / 2), CTA 1 the rest of both,
+// each in one box of consecutive receive rows: main column j is receive row p0 + j
+// (+ n_x / 2 past CTA 0's half), extra column j is p0 + n_main / 2 + j (+ n_main / 2
+// past CTA 0's half).
 struct TileInfo {
     int e, f_blk, p0, n_valid, n_main, n_x;
 };
@@ -156,38 +162,47 @@ __device__ __forceinline__ TileInfo tile_info(int e, int f_blk, int t_blk, const
     const int m_e = P.expert_offsets[e + 1] - off;
     t.p0 = off + t_blk * kTileTok;
     t.n_valid = t_blk == expert_tiles(m_e) - 1 ? m_e - t_blk * kTileTok : kTileTok;
-    if (t.n_valid > kTileTok) {
-        t.n_main = kTileTok;
-        t.n_x = t.n_valid - kTileTok <= kXTok / 2 ? kXTok / 2 : kXTok;
-    } else {
-        t.n_main = (t.n_valid + 15) & ~15;
-        t.n_x = 0;
-    }
+    t.n_main = t.n_valid > kSlotCols ? kTileTok : (t.n_valid + 15) & ~15;
+    t.n_x = t.n_valid > kTileTok ? kXHalf : 0;
     return t;
 }
 
-// Epilogue chunk ch of a tile (32 TMEM columns; the extra part's chunks first):
-// its first TMEM column in the accumulator `acc`, and the receive rows (from
-// p0) of its two 16-column halves, each a run of consecutive rows.
+// TMEM columns of a tile in accumulator acc: its main MMA's first column and its
+// extra MMA's; the half a main MMA of more than 224 columns takes is the
+// accumulator's own (a for 0, b for 1), the extra MMA's the other one.
+__device__ __forceinline__ uint32_t main_col(const TileInfo &ti, int acc) {
+    return acc == 0 ? 0u : ti.n_main > kSlotCols ? (uint32_t)kSlotCols + kXHalf : (uint32_t)kSlotCols + 2 * kXHalf;
+}
+__device__ __forceinline__ uint32_t extra_col(int acc) { return acc == 0 ? kXCol + kXHalf : kXCol; }
+
+// Epilogue chunk ch of a tile (32 TMEM columns): its first TMEM column, the receive
+// rows (from p0) of its two 16-column halves, each a run of consecutive rows, and
+// the half of the shared part it holds (-1: none).  Chunks that hold a half of the
+// shared part come first (the extra MMA's, then the main MMA's own half), so that
+// the epilogue can release them before the rest.
 struct ChunkMap {
     uint32_t tcol;
-    int rel_lo, rel_hi;
+    int rel_lo, rel_hi, xh;
 };
 __device__ __forceinline__ int chunk_count(const TileInfo &ti) { return ti.n_x / 32 + (ti.n_main + 31) / 32; }
 __device__ __forceinline__ ChunkMap chunk_map(const TileInfo &ti, int ch, int acc) {
     ChunkMap m;
     const int nxc = ti.n_x / 32;
-    if (ch < nxc) {
-        const int j = 32 * ch;
-        m.tcol = kXCol + (uint32_t)j;
-        m.rel_lo = j < ti.n_x / 2 ? kTileTok / 2 + j : kTileTok + j;
-        m.rel_hi = j + 16 < ti.n_x / 2 ? kTileTok / 2 + j + 16 : kTileTok + j + 16;
-    } else {
-        const int j = 32 * (ch - nxc);
-        m.tcol = (uint32_t)(acc * kTileTok + j);
-        m.rel_lo = j < ti.n_main / 2 ? j : j + ti.n_x / 2;
-        m.rel_hi = j + 16 < ti.n_main / 2 ? j + 16 : j + 16 + ti.n_x / 2;
+    if (ch < nxc) {   // the extra MMA: columns [0, 16) from CTA 0, [16, 32) from CTA 1
+        m.tcol = extra_col(acc);
+        m.rel_lo = ti.n_main / 2;
+        m.rel_hi = ti.n_main + 16;
+        m.xh = acc ^ 1;
+        return m;
     }
+    int c = ch - nxc;   // main MMA chunk; accumulator 0's own half is its last chunk (7)
+    const bool own = ti.n_main > kSlotCols;
+    if (own && acc == 0) c = c == 0 ? kSlotCols / 32 : c - 1;
+    const int j = 32 * c;
+    m.tcol = main_col(ti, acc) + (uint32_t)j;
+    m.rel_lo = j < ti.n_main / 2 ? j : j + ti.n_x / 2;
+    m.rel_hi = j + 16 < ti.n_main / 2 ? j + 16 : j + 16 + ti.n_x / 2;
+    m.xh = own && ch == nxc ? acc : -1;
     return m;
 }
 __device__ __forceinline__ int chunk_rel(const ChunkMap &m, int j) { return j < 16 ? m.rel_lo + j : m.rel_hi + j - 16; }
@@ -304,7 +319,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             mbar_init(&S->tmem_full[a], 1);
             mbar_init(&S->tmem_empty[a], 2 * kEpiWarps);   // every epilogue warp of both CTAs
         }
-        mbar_init(&S->x_empty, 2 * kEpiWarps);
+        mbar_init(&S->x_empty[0], 2 * kEpiWarps);
+        mbar_init(&S->x_empty[1], 2 * kEpiWarps);
         for (int i = 0; i < kQueue; ++i) { mbar_init(&S->q_full[i], 1); mbar_init(&S->q_empty[i], kQueueConsumers); }
         mbar_init(&S->mma_done, 1);
         S->abort_flag = 0;
@@ -411,7 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 uint32_t phase = 0;
                 int acc = 0;
                 uint32_t acc_phase = 0;
-                uint32_t x_phase = 0;
+                uint32_t x_phase = 0;   // bit h: the phase of half h's barrier
                 bool ok = true;
                 SliceReader reader;
                 int slice;
@@ -429,19 +445,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                                              : F8 ? make_idesc_e4m3_f32(2 * kRowsPerCta, ti.n_x)
                                                   : make_idesc_bf16_f32_major(2 * kRowsPerCta, ti.n_x, A_MN, false);
                     if (!mbar_wait_bounded(&S->tmem_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-                    // the extra part's columns: drained by the previous merged tile's epilogue
-                    if (merged) {
-                        if (!mbar_wait_bounded(&S->x_empty, x_phase ^ 1u, abort_flag)) { ok = false; break; }
-                        x_phase ^= 1u;
+                    // the halves of the shared part this tile writes (its own past 224 main
+                    // columns, the other one for the extra MMA): drained by the epilogue of
+                    // the last tile that wrote them
+                    {
+                        bool x_ok = true;
+                        for (int hx = 0; hx < 2 && x_ok; ++hx) {
+                            const bool uses = hx == acc ? ti.n_main > kSlotCols : merged;
+                            if (!uses) continue;
+                            x_ok = mbar_wait_bounded(&S->x_empty[hx], ((x_phase >> hx) & 1u) ^ 1u, abort_flag);
+                            x_phase ^= 1u << hx;
+                        }
+                        if (!x_ok) { ok = false; break; }
                     }
                     tc_fence_after();
-                    const uint32_t d = tmem_base + (uint32_t)(acc * kTileTok);
-                    const uint32_t dx = tmem_base + kXCol;
+                    const uint32_t d = tmem_base + main_col(ti, acc);
+                    const uint32_t dx = tmem_base + extra_col(acc);
                     // k-chunk stride inside the stage's token box (32 or 144 rows); the
                     // extra part's rows follow the main half's in both CTAs
                     const bool small_box = ti.n_x == 0 && ti.n_main / 2 <= kSmallBoxRows;
                     const uint32_t tchunk = small_box ? kSmallBoxRows * kBK * 2 : kTokBytes;
-                    constexpr uint32_t kXRowOff = (kTileTok / 2) * 128;   // 112 rows of 128 bytes
+                    const uint32_t x_row_off = (uint32_t)(ti.n_main / 2) * 128;   // 128 rows of 128 bytes
                     for (int kb = 0; kb < num_k; ++kb) {
                         if (!mbar_wait_bounded(&S->full[stage], phase, abort_flag)) { ok = false; break; }
                         tc_fence_after();
@@ -461,7 +485,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                                         ? make_sw128_desc_mn(st + c * (kWBytes / 2) + kk * 2048, kWBytes)
                                         : make_sw128_desc(st + c * kWBytes + kk * 32);
                                     const uint32_t taddr = st + kKS * kWBytes + c * tchunk + kk * 32 +
-                                                           (part ? kXRowOff : 0u);
+                                                           (part ? x_row_off : 0u);
                                     const uint64_t tdesc = make_sw128_desc(taddr);
                                     const uint32_t accum = (kb > 0 || c > 0 || kk > 0) ? 1u : 0u;
                                     if (F8) tc_mma_f8_pair(part ? dx : d, wdesc, tdesc, part ? idesc_x : idesc, accum);
@@ -499,7 +523,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
         const int xpair = half * 2 + (q & 1);                 // gate/up warp pair (GEMM1)
         const uint32_t empty_leader[2] = {mapa_shared(smem_u32(&S->tmem_empty[0]), 0),
                                           mapa_shared(smem_u32(&S->tmem_empty[1]), 0)};
-        const uint32_t x_empty_leader = mapa_shared(smem_u32(&S->x_empty), 0);
+        // the leader's barrier of half h of the shared part (the two are adjacent)
+        const uint32_t x_empty_leader0 = mapa_shared(smem_u32(&S->x_empty[0]), 0);
+        auto x_empty_leader = [&](int h) { return x_empty_leader0 + 8u * (uint32_t)h; };
         int acc = 0;
         uint32_t acc_phase = 0;
         SliceReader reader;
@@ -533,7 +559,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
            // of each of the warp's chunks (chunks half, half + 2, ...), loaded before
            // the accumulator wait so that their latency hides behind it
            const int nch = chunk_count(ti);
-           const int nxc = ti.n_x / 32;
            float wsc = 1.0f;
            float tsc[5] = {1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
            if (F8) {
@@ -544,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                for (int i = 0; i < 5; ++i) {
                    const int ch = half + 2 * i;
                    if (ch < nch) {
-                       const int rel = chunk_rel(chunk_map(ti, ch, 0), lane);
+                       const int rel = chunk_rel(chunk_map(ti, ch, acc), lane);
                        if (rel < ti.n_valid) {
                            const int p = ti.p0 + rel;
                            tsc[i] = ue8m0_value(P.t_scale[P.t_scale_by_token ? P.recv_token[p] : p]);
@@ -572,10 +597,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
             }
             tc_fence_after();
             const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
-            // a warp with no chunk of the extra part releases it at once
-            if (nxc > 0 && half >= nxc) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(x_empty_leader);
+            // a half of the shared part held by a chunk of the other warp parity is
+            // released at once (such chunks are the first one or two of the tile)
+            for (int ch = 0; ch < 2 && ch < nch; ++ch) {
+                const int xh = chunk_map(ti, ch, acc).xh;
+                if (xh >= 0 && (ch & 1) != half) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(x_empty_leader(xh));
+                }
             }
 
             int ci = 0;
@@ -584,10 +613,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFfnThreads, 1) ffn_
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tlane + cm.tcol, r);
                 tc_wait_ld_regs(r);
-                if (ch < nxc) {   // the extra part's columns are in registers: release them
+                if (cm.xh >= 0) {   // a half of the shared part is in registers: release it
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(x_empty_leader);
+                    if (lane == 0) mbar_arrive_cluster(x_empty_leader(cm.xh));
                 }
                 // FP8: the scale of the token in column `lane`
                 const float ts_lane = ci == 0 ? tsc[0] : ci == 1 ? tsc[1] : ci == 2 ? tsc[2] : ci == 3 ? tsc[3] : tsc[4];

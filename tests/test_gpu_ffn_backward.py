@@ -27,9 +27,9 @@ CASES = [
     ("bf16_ragged", "bf16", 256, 256, [0, 1, 15, 17, 128, 129, 300, 40]),
     ("bf16_partial_tiles", "bf16", 192, 192, [5, 300, 0, 77]),
     ("bf16_wide", "bf16", 512, 128, [250, 3, 0, 511, 16, 33, 260, 127, 64, 1, 0, 190, 129, 255, 18, 70]),
-    # the token tiling's edges: 224-token tiles, the last one of up to 288 tokens
-    # through a second MMA (N = 32 / 64), merged tiles back to back
-    ("bf16_tile_edges", "bf16", 256, 128, [224, 225, 240, 241, 256, 257, 288, 289, 0, 449, 513, 288, 288, 257]),
+    # the token tiling's edges: 256-token tiles, the last one of up to 288 tokens,
+    # the shared TMEM part past 224, a second MMA past 256, such tiles back to back
+    ("bf16_tile_edges", "bf16", 256, 128, [224, 225, 240, 241, 256, 257, 288, 289, 0, 449, 513, 545, 288, 288, 257]),
 ]
 
 

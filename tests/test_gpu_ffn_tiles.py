@@ -1,18 +1,20 @@
 """The grouped FFN at the edges of its token tiling, element by element against
 the oracle.
 
-The kernel covers an expert's rows 224 at a time and lets the last tile take up
-to 288: a tile of 225..288 tokens issues a second MMA (N = 32 for up to 256
-tokens, N = 64 above) into a separate part of TMEM, and each 32-column chunk of
-its accumulators maps to two runs of 16 receive rows.  The segment sizes here sit
-on every boundary of that rule: one row, under one 16-row MMA step, 224 / 225
-(the first merged tile), 240 / 241 and 256 / 257 (the extra MMA's N = 32 / 64
-switch and its halves), 288 / 289 (the largest merged tile, then two tiles),
-448 / 449, 512 / 513, 736 and an empty expert, several of them back to back so
-that merged tiles follow one another on the same CTA pair.  Every row of h and y
-is compared with the oracle, for the bf16 store epilogue, the decode form's
-reduce epilogue and the FP8 path (row scales on codes).  The backward's modes on
-the same sizes are in tests/test_gpu_ffn_backward.py.
+The kernel covers an expert's rows 256 at a time and lets the last tile take up
+to 288.  Each TMEM accumulator owns 224 columns; a main MMA of more than 224
+tokens extends into a 32-column half of a shared part beside it, and a tile of
+more than 256 tokens issues a second MMA (N = 32) into the other half; each
+32-column chunk of the accumulators maps to two runs of 16 receive rows.  The
+segment sizes here sit on every boundary of that rule: one row, under one 16-row
+MMA step, 224 / 225 (into the shared part), 240 / 241, 256 / 257 (the extra MMA),
+288 / 289 (the largest single tile, then two), 448 / 449, 512 / 513, 544 / 545
+(256 + 288, then three tiles), 736 and an empty expert, several of them back to
+back so that tiles writing the shared part follow one another on the same CTA
+pair, in both accumulators.  Every row of h and y is compared with the oracle,
+for the bf16 store epilogue, the decode form's reduce epilogue and the FP8 path
+(row scales on codes).  The backward's modes on the same sizes are in
+tests/test_gpu_ffn_backward.py.
 """
 import numpy as np
 import pytest
@@ -25,8 +27,8 @@ from moe_testlib import assert_float_close, storage_np
 
 pytestmark = pytest.mark.gpu
 
-SIZES = [224, 225, 240, 241, 256, 257, 272, 273, 288, 289, 304, 0, 1, 15, 33, 448, 449, 512, 513, 736, 65,
-         288, 288, 257]
+SIZES = [224, 225, 240, 241, 256, 257, 272, 273, 288, 289, 304, 0, 1, 15, 33, 448, 449, 512, 513, 544, 545,
+         736, 65, 288, 288, 257, 256, 256, 225]
 H, I = 256, 256
 
 
