@@ -55,18 +55,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sha256 prefix of the kernel source the counters were taken on - a changed
 # kernel reports null until it is captured again.
 FFN_TRAFFIC = {
-    "qwen3_30b_a3b": {"bytes": (943.448832 + 46.416640 + 453.957120 + 113.494784) * 1e6,
-                      "src": "ae304e0a3accf960"},
+    "qwen3_30b_a3b": {"bytes": (942.794240 + 45.979648 + 453.990656 + 113.344512) * 1e6,
+                      "src": "52e786192f9b24d0"},
     # both GEMM launches and the quantisation of h between them
-    "qwen3_30b_a3b_fp8": {"bytes": (471.292416 + 41.976832 + 50.341376 + 1.413888 + 226.893056 +
-                                    97.778688) * 1e6, "src": "f7a63551cfc9ed2a"},
+    "qwen3_30b_a3b_fp8": {"bytes": (471.297792 + 42.182400 + 50.341376 + 1.413888 + 226.896384 +
+                                    96.848640) * 1e6, "src": "18a4e475b021b023"},
     "qwen3_30b_a3b_mxfp8": {"bytes": (484.897024 + 24.313600 + 233.751296 + 105.241344) * 1e6,
                             "src": "f91c44b09b122286"},
     # captured with 32 of the 256 experts and 1024 tokens (the same 128 rows per
     # expert and chunk), scaled by 8 per chunk, two chunks; see
     # profiles/ffn_tcgen05_dsv3_prefill.md and profiles/ffn_mx_tcgen05_dsv3_prefill_mxfp8.md
-    "dsv3_prefill": {"bytes": 2 * 8 * (1956.813568e6 + 18.363648e6 + 958.455040e6 + 55.145984e6),
-                     "src": "ae304e0a3accf960", "chunks": 2},
+    "dsv3_prefill": {"bytes": 2 * 8 * (1956.903168e6 + 18.358016e6 + 958.769664e6 + 54.941440e6),
+                     "src": "52e786192f9b24d0", "chunks": 2},
     "dsv3_prefill_mxfp8": {"bytes": 2 * 8 * (1008.328192e6 + 11.598080e6 + 494.208000e6 + 49.762304e6),
                            "src": "f91c44b09b122286", "chunks": 2},
 }
