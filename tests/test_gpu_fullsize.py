@@ -4,9 +4,12 @@ benchmark times.
 Routing, drop sets, layouts and split counts are compared whole against the
 oracle (bit-exact).  Permuted rows are checked whole by the defining property
 xr[p] = x[recv_token[p]] (bitwise).  The FFN is compared on every tile the
-grouped GEMM deals: the first and the last row of every (expert, 256-token
-block) of every chunk, and two more rows of each expert's short last block
-(the 32-row token box of tiles with at most 64 rows).  The combined output is
+grouped GEMM deals, at both sides of every boundary inside it: an expert's rows
+in 256-token tiles, the last one of up to 288 (its main MMA of N <= 256 split
+between the two CTAs of the pair, the rows past 256 in a second MMA split the
+same way), so per tile its first and last row and the rows on either side of
+each CTA half; two more rows of each short tile (the 32-row token box of tiles
+with at most 64 rows).  The combined output is
 compared on 128 sampled tokens, whose expert rows the oracle also computes.
 The oracle's rows run in threads (its C calls release the interpreter lock),
 expert by expert, each with its own host copy of that expert's weights.
@@ -30,23 +33,49 @@ pytestmark = pytest.mark.gpu
 FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode", "dsv3_grouped"]
 
 
-TILE = 256          # token rows per FFN tile
+TILE = 256          # token rows per FFN tile (an expert's last takes up to TILE_MAX)
+TILE_MAX = 288
 SHORT = 64          # tiles of at most this many rows take the short token box
 N_TOKENS = 128      # sampled tokens of the combined output
 
 
+def ffn_tiles(m):
+    """(first row, rows, main MMA N, extra MMA N) of the FFN's tiles over an expert
+    of m rows: 256-row tiles, the last one of up to 288."""
+    if m <= 0:
+        return []
+    n = 1 if m <= TILE_MAX else (m - (TILE_MAX - TILE) + TILE - 1) // TILE
+    out = []
+    for t in range(n):
+        nv = m - t * TILE if t == n - 1 else TILE
+        n_main = TILE if nv > 224 else (nv + 15) // 16 * 16
+        out.append((t * TILE, nv, n_main, 32 if nv > TILE else 0))
+    return out
+
+
 def select_rows(lay, rng, tile=TILE, short=SHORT):
-    """Receive rows that cover every FFN tile of a chunk: per (expert, tile-row
-    block) its first and last row; a short last block (<= short rows) two more."""
+    """Receive rows that cover every FFN tile of a chunk.  With the bf16 / FP8
+    kernel's tiling (tile = TILE): per tile its first and last row and the rows on
+    either side of each CTA half of its main and extra MMA; a short tile (<= short
+    rows) two more.  Otherwise: per (expert, tile-row block) its first and last
+    row."""
     eoff = lay["expert_offsets"]
     rows = set()
     for e in range(len(eoff) - 1):
         lo, hi = int(eoff[e]), int(eoff[e + 1])
-        for b0 in range(lo, hi, tile):
-            b1 = min(b0 + tile, hi) - 1
-            rows.update((b0, b1))
-            if b1 - b0 + 1 <= short:
-                rows.update(int(v) for v in rng.integers(b0, b1 + 1, 2))
+        if tile != TILE:
+            for b0 in range(lo, hi, tile):
+                b1 = min(b0 + tile, hi) - 1
+                rows.update((b0, b1))
+                if b1 - b0 + 1 <= short:
+                    rows.update(int(v) for v in rng.integers(b0, b1 + 1, 2))
+            continue
+        for r0, nv, n_main, n_x in ffn_tiles(hi - lo):
+            a, b = n_main // 2, n_x // 2
+            edges = {0, a - 1, a, a + b - 1, a + b, 2 * a + b - 1, 2 * a + b, nv - 1}
+            rows.update(lo + r0 + r for r in edges if 0 <= r < nv)
+            if nv <= short:
+                rows.update(int(v) for v in rng.integers(lo + r0, lo + r0 + nv, 2))
     return rows
 
 
