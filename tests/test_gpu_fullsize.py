@@ -35,6 +35,7 @@ FULL = ["qwen3_30b_a3b", "skew_capacity", "dsv3_prefill", "dsv3_decode", "dsv3_g
 
 TILE = 256          # token rows per FFN tile (an expert's last takes up to TILE_MAX)
 TILE_MAX = 288
+MX_TILE = 224       # token rows per tile of the block-scaled FP8 FFN
 SHORT = 64          # tiles of at most this many rows take the short token box
 N_TOKENS = 128      # sampled tokens of the combined output
 
@@ -53,24 +54,25 @@ def ffn_tiles(m):
     return out
 
 
-def select_rows(lay, rng, tile=TILE, short=SHORT):
-    """Receive rows that cover every FFN tile of a chunk.  With the bf16 / FP8
-    kernel's tiling (tile = TILE): per tile its first and last row and the rows on
-    either side of each CTA half of its main and extra MMA; a short tile (<= short
-    rows) two more.  Otherwise: per (expert, tile-row block) its first and last
-    row."""
+def mx_tiles(m):
+    """The block-scaled FFN's tiles over an expert of m rows: 224 rows each (its MMA
+    N rounded to 16, split between the two CTAs)."""
+    return [(r0, min(MX_TILE, m - r0), (min(MX_TILE, m - r0) + 15) // 16 * 16, 0)
+            for r0 in range(0, m, MX_TILE)]
+
+
+def select_rows(lay, rng, tiles=None, short=SHORT):
+    """Receive rows that cover every FFN tile of a chunk, following the kernel's
+    tiling (tiles: rows -> [(first row, rows, main N, extra N)], the bf16 / FP8
+    kernel's by default): per tile its first and last row and the rows on either
+    side of each CTA half of its main and extra MMA; a short tile (<= short rows)
+    two more."""
+    tiles = tiles or ffn_tiles
     eoff = lay["expert_offsets"]
     rows = set()
     for e in range(len(eoff) - 1):
         lo, hi = int(eoff[e]), int(eoff[e + 1])
-        if tile != TILE:
-            for b0 in range(lo, hi, tile):
-                b1 = min(b0 + tile, hi) - 1
-                rows.update((b0, b1))
-                if b1 - b0 + 1 <= short:
-                    rows.update(int(v) for v in rng.integers(b0, b1 + 1, 2))
-            continue
-        for r0, nv, n_main, n_x in ffn_tiles(hi - lo):
+        for r0, nv, n_main, n_x in tiles(hi - lo):
             a, b = n_main // 2, n_x // 2
             edges = {0, a - 1, a, a + b - 1, a + b, 2 * a + b - 1, 2 * a + b, nv - 1}
             rows.update(lo + r0 + r for r in edges if 0 <= r < nv)
@@ -271,16 +273,13 @@ def test_fp8_fullsize_against_oracle(name):
     torch.cuda.empty_cache()
 
 
-MX_TILE = 128       # token rows per tile of the block-scaled FP8 FFN
-
-
 @pytest.mark.parametrize("name", ["qwen3_30b_a3b_mxfp8", "dsv3_prefill_mxfp8"])
 def test_mxfp8_fullsize_against_oracle(name):
     """The FP8 layer with K-blocked scales at full size: x's block quantisation
     whole and bit-exact (the standalone kernel), the fused permute's codes and
     scales whole by the defining property (xr[p] = q(x)[recv_token[p]]), every
-    checked expert's weight codes and scales bit-exact, the rows of every
-    128-row FFN tile and of 128 sampled tokens against the oracle's blocked FP8
+    checked expert's weight codes and scales bit-exact, the rows at every boundary
+    of every 224-row FFN tile and of 128 sampled tokens against the oracle's blocked FP8
     rows (h's codes by the adjacency bar, y by the bf16 bar), and the combined
     output of those tokens."""
     wl = WORKLOADS[name]
@@ -321,7 +320,7 @@ def test_mxfp8_fullsize_against_oracle(name):
         rt = torch.from_numpy(lay["recv_token"]).long().cuda()
         assert torch.equal(gc["xr_dev"][:n], xq_dev[rt]), "fused permute: codes"
         assert torch.equal(gc["xsf_dev"][:n], xs_dev[rt]), "fused permute: block scales"
-        rows = select_rows(lay, rng, tile=MX_TILE, short=0)
+        rows = select_rows(lay, rng, tiles=mx_tiles, short=0)
         for t in tokens:
             if c * tc <= t < (c + 1) * tc:
                 rows.update(int(p) for p in lay["pos"][t - c * tc] if p >= 0)
