@@ -145,11 +145,7 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-// ---------------------------------------------------------------- memory ordering
-__device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
+// ---------------------------------------------------------------- shared memory
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
